@@ -1,0 +1,317 @@
+#!/usr/bin/env python
+"""Throughput of the routed-MoE FFN step on B200, one JSON line on rank 0.
+
+Default workload: decode, one layer, one token per step (hidden 2048, 512
+routed experts + 1 shared, intermediate 768, top-10, int4 group-32 experts,
+Zipf(1.1) router prior, 200 fresh seeded tokens). A step is one full pass of
+the step (route -> dispatch -> experts -> combine) over that step's token.
+
+Timing: W untimed warm-up steps, then K timed steps. Every step is bracketed
+by its own pair of CUDA events on the launching stream; between steps a
+2 x L2-sized buffer is overwritten (outside the event pairs) so every step
+streams its expert weights from HBM rather than L2. Multi-GPU (torchrun):
+every rank runs an independent replica on its own token stream (weak
+scaling, no collective in the data path); the reported time is the max over
+ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode1]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_moe_gemv_b200 import workload as wlm  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (decode b=1..4, 8K prefill); % of HBM / tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode1", choices=["decode1"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the CPU-baseline sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.path = None
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(gpu_index)], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r for r in csv.reader(io.StringIO(open(self.path).read())) if len(r) >= 9]
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU side
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle(wl, lay, bias, n_steps_max, seconds, step_offset=0):
+    """Run the fp64 oracle layer step by step until `seconds` or n_steps_max.
+    Returns (tokens, elapsed seconds, steps)."""
+    import oracle
+    tokens, steps, t0 = 0, 0, time.perf_counter()
+    while steps < n_steps_max:
+        xb = wlm.gen_x(wl, step=step_offset + steps)
+        oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared)
+        tokens += wl.T
+        steps += 1
+        if time.perf_counter() - t0 >= seconds and steps >= 2:
+            break
+    return tokens, time.perf_counter() - t0, steps
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, rank, world, peaks, peak_kind):
+    import torch
+
+    from bit_quantized_moe_gemv_b200 import _lib as L
+    from bit_quantized_moe_gemv_b200.device import DeviceExperts, bf16_tensor
+
+    wl = wlm.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lay = wlm.gen_layer(wl)
+    bias, stride = wlm.gen_bias(wl)
+    experts, shared = DeviceExperts(lay.experts), DeviceExperts([lay.shared])
+    w_r = torch.from_numpy(lay.w_router).to(dev)
+    b = torch.from_numpy(np.ascontiguousarray(bias)).to(dev)
+    n_steps = args.warmup + args.steps
+    # each rank gets its own stream of fresh tokens (replicas)
+    xs_host = np.stack([wlm.gen_x(wl, step=rank * n_steps + s) for s in range(n_steps)])
+    xs = bf16_tensor(xs_host)
+    idx = torch.empty((n_steps, wl.T, wl.k), dtype=torch.int32, device=dev)
+    gw = torch.empty((n_steps, wl.T, wl.k), dtype=torch.float32, device=dev)
+    out = torch.empty((n_steps, wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * max(l2, 126 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        L.layer(xs[s], wl.I, wl.E, wl.k, w_r, b, stride, experts.table, shared.table, idx[s], gw[s], out[s], ws,
+                stream=stream)
+
+    def timed_loop(first, count, flush_between=True, host_io=None):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(count)]
+        for i in range(count):
+            s = first + i
+            evs[i][0].record(stream)
+            if host_io is None:
+                step(s)
+            else:
+                xin, xout = host_io
+                xs[s].copy_(xin[s], non_blocking=True)
+                step(s)
+                xout[s].copy_(out[s], non_blocking=True)
+            evs[i][1].record(stream)
+            if flush_between:
+                flush.fill_(i & 0xff)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(z) for a, z in evs]
+
+    # warm-up (untimed), same protocol
+    timed_loop(0, args.warmup)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    launches0 = L.launch_count()
+    t_wall = time.perf_counter()
+    times = timed_loop(args.warmup, args.steps)
+    t_wall = time.perf_counter() - t_wall
+    launches = L.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
+
+    total_ms = float(np.sum(times))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    tokens_all = world * wl.T * args.steps
+    value = tokens_all / (total_ms / 1e3)
+
+    # warm-L2 figure (context only): same steps without the flush
+    warm = timed_loop(args.warmup, min(args.steps, 50), flush_between=False)
+
+    # e2e: pinned host tokens in, pinned host output back, every step
+    xin = xs_host.copy()
+    xin_t = torch.from_numpy(xin.view(np.int16)).view(torch.bfloat16).pin_memory()
+    xout_t = torch.empty((n_steps, wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    e2e_times = timed_loop(args.warmup, args.steps, host_io=(xin_t, xout_t))
+    e2e_ms = float(np.sum(e2e_times))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # algorithmic bytes per step: distinct routed experts + shared + router
+    idx_h = idx[args.warmup:].cpu().numpy()
+    uniq = np.array([len(np.unique(s)) for s in idx_h.reshape(args.steps, -1)])
+    bytes_per_step = np.array([wlm.per_token_layer_bytes(wl, u) for u in uniq])
+    achieved_gbs = float(np.sum(bytes_per_step) / (np.sum(times) / 1e3) / 1e9)
+    peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; random weights of the stated architecture)",
+        "config": {
+            "workload": f"decode one layer: T={wl.T}, H={wl.H}, I={wl.I}, E={wl.E}+1 shared, k={wl.k}, "
+                        f"int4 sym g32 experts, Zipf({wl.zipf_s}) prior, fresh token per step",
+            "global_batch": wl.T * world,
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (2 x L2 write, outside the timed events)",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "moe_layer step (all launches of one step)",
+            "achieved": achieved_gbs,
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": achieved_gbs / peak,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_step": float(np.mean(bytes_per_step)),
+            "traffic": None,
+        },
+        "warm_l2": {"ms_per_step": float(np.mean(warm)), "note": "context only, weights partly L2-resident"},
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(wl.T * wl.H * 2), "d2h_bytes_per_step": int(wl.T * wl.H * 2)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "wall_s_timed_region": t_wall,
+    }
+    return line, wl, lay, bias
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks, peak_kind = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        wl = wlm.WORKLOADS[args.workload]
+        lay = wlm.gen_layer(wl)
+        bias, _ = wlm.gen_bias(wl)
+        budget = 150.0
+        _, s_warm, _ = time_oracle(wl, lay, bias, args.warmup, budget / 4)
+        tokens, secs, steps = time_oracle(wl, lay, bias, args.steps, budget, step_offset=args.warmup)
+        value = tokens / secs
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": f"decode one layer: T={wl.T}, H={wl.H}, I={wl.I}, E={wl.E}+1 shared, k={wl.k}",
+                       "global_batch": wl.T},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": f"{steps} of {args.steps} requested steps (1 token each), bounded to "
+                                       f"{budget:.0f} s"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    line, wl, lay, bias = run_ours(args, rank, world, peaks, peak_kind)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tokens, secs, steps = time_oracle(wl, lay, bias, 10 ** 6, args.cpu_seconds, step_offset=10 ** 5)
+        line["cpu_baseline"] = {"value": tokens / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"{steps} decode steps of 1 token through the fp64 oracle "
+                                          f"({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

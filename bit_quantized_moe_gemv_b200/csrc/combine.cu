@@ -1,0 +1,63 @@
+// Combine: out[t] = sum_{j=0..k-1} w[t,j] * y_perm[inv_perm[t*k+j]] + shared(x_t),
+// summed in j order in fp32 and rounded once to bf16 (nearest even).
+//
+// Each token uses its k routed experts plus the one shared expert: the telli.sh
+// page "Strata 与 Qwen3.8-Flash-Next：如何在个人电脑上运行 180B 级模型", section
+// "稀疏架构创造了机会". The gate-weighted sum with an ungated shared expert is
+// this library's reading of that sentence.
+//
+// Gather form (no atomics): one thread owns 8 consecutive outputs of a token
+// and reads the k expert rows with 16-byte loads, so the result does not depend
+// on scheduling.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256)
+combine_kernel(const uint16_t* __restrict__ y_perm, const int* __restrict__ inv_perm, const float* __restrict__ topk_w,
+               int T, int H, int k, const float* __restrict__ shared_y, uint16_t* __restrict__ out) {
+  const int per_tok = H / 8;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= (long long)T * per_tok) return;
+  const int t = int(tid / per_tok), c = int(tid % per_tok);
+  float acc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+  const long long nrows = (long long)T * k;
+  for (int j = 0; j < k; ++j) {
+    const int r = inv_perm[(long long)t * k + j];
+    if (r < 0 || r >= nrows) continue;  // invalid expert id upstream (flagged there)
+    const float w = topk_w[(long long)t * k + j];
+    const uint4 v = *reinterpret_cast<const uint4*>(y_perm + (size_t)r * H + 8 * c);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[2 * q] = fmaf(w, __uint_as_float(u[q] << 16), acc[2 * q]);
+      acc[2 * q + 1] = fmaf(w, __uint_as_float(u[q] & 0xffff0000u), acc[2 * q + 1]);
+    }
+  }
+  if (shared_y) {
+    const float4* s = reinterpret_cast<const float4*>(shared_y + (size_t)t * H + 8 * c);
+    const float4 a = s[0], b = s[1];
+    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+  }
+  uint4 o;
+  o.x = uint32_t(f32_to_bf16_rn(acc[0])) | (uint32_t(f32_to_bf16_rn(acc[1])) << 16);
+  o.y = uint32_t(f32_to_bf16_rn(acc[2])) | (uint32_t(f32_to_bf16_rn(acc[3])) << 16);
+  o.z = uint32_t(f32_to_bf16_rn(acc[4])) | (uint32_t(f32_to_bf16_rn(acc[5])) << 16);
+  o.w = uint32_t(f32_to_bf16_rn(acc[6])) | (uint32_t(f32_to_bf16_rn(acc[7])) << 16);
+  *reinterpret_cast<uint4*>(out + (size_t)t * H + 8 * c) = o;
+}
+
+cudaError_t launch_combine(const uint16_t* y_perm, const int* inv_perm, const float* topk_w, int T, int H, int k,
+                           const float* shared_y, uint16_t* out, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const long long n = (long long)T * (H / 8);
+  combine_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(y_perm, inv_perm, topk_w, T, H, k, shared_y, out);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

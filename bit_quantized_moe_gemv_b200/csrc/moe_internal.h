@@ -1,0 +1,37 @@
+// Internal launcher declarations shared by the ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+// Host-side count of kernel launches (diagnostic).
+void count_launches(int n);
+
+enum TicketSlot { kTicketRoute = 0, kTicketDecodeRoute = 1, kTicketDecodeGateUp = 2 };
+
+cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
+                         long long bstride, int k, int* topk_idx, float* topk_w, float* logits, WsHeader* hdr,
+                         cudaStream_t st);
+
+// Blocks the multi-block dispatch uses for n = T*k pairs (1 = single-CTA path).
+int dispatch_blocks(long long n);
+
+cudaError_t launch_dispatch(const int* topk_idx, int T, int k, int E, int* counts, int* offsets, int* perm_src,
+                            int* inv_perm, int* hist, WsHeader* hdr, cudaStream_t st);
+
+// Routed experts over dispatched rows (identity = false) or one expert over
+// the T tokens in order (identity = true; used for the shared expert).
+// Writes y as bf16 rows (y_bf16 != nullptr) or fp32 rows (y_f32 != nullptr).
+cudaError_t launch_expert_ffn(const uint16_t* x, int T, int H, int I, int k, int E, const int* perm_src,
+                              const int* offsets, const int* counts, const moe_expert* experts, bool identity,
+                              float* h_ws, int* active_ws, uint16_t* y_bf16, float* y_f32, WsHeader* hdr,
+                              cudaStream_t st);
+
+cudaError_t launch_combine(const uint16_t* y_perm, const int* inv_perm, const float* topk_w, int T, int H, int k,
+                           const float* shared_y, uint16_t* out, cudaStream_t st);
+
+}  // namespace moe

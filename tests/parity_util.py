@@ -1,0 +1,96 @@
+"""Helpers shared by the GPU parity tests: tolerance checks, routing agreement
+with near-tie handling, and device upload of seeded workloads."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+
+# Float tolerance for bf16 activations with fp32 accumulation.
+REL_L2 = 5e-3
+MAX_ABS_RMS = 2e-2
+
+
+def assert_close(got, ref, what="output"):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    rms = np.sqrt(np.mean(ref ** 2))
+    err = got - ref
+    rel = np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300)
+    mx = np.abs(err).max() if err.size else 0.0
+    assert rel <= REL_L2, f"{what}: rel L2 {rel:.3e} > {REL_L2}"
+    assert mx <= MAX_ABS_RMS * rms, f"{what}: max abs {mx:.3e} > {MAX_ABS_RMS} x rms {rms:.3e}"
+    return rel, mx / max(rms, 1e-300)
+
+
+def bf16_to_f64(bits):
+    return oracle.bf16_bits_to_f64(bits)
+
+
+def near_tie_tau(x_bits, w_router, bias):
+    """Per-token tie tolerance: 64 ulp(fp32) of the largest sum |W x| + |b|."""
+    x = np.abs(bf16_to_f64(x_bits))
+    a = x @ np.abs(np.asarray(w_router, np.float64)).T + np.abs(np.asarray(bias, np.float64))
+    return 64.0 * 2.0 ** -24 * a.max(axis=1)
+
+
+def oracle_gates_for(logits64, idx):
+    """Renormalised softmax gates of the given picks, from fp64 logits."""
+    p = oracle.softmax(logits64)
+    sel = np.take_along_axis(p, np.asarray(idx, np.int64), axis=1)
+    return sel / sel.sum(axis=1, keepdims=True)
+
+
+def check_routing(gpu_idx, gpu_w, gpu_logits, x_bits, w_router, bias, k):
+    """Routing parity.
+
+    1. The selection logic, exactly: the oracle's top-k and gates evaluated on
+       the device's own fp32 logits give the device's indices bit for bit and
+       its gates within a few fp32 ulps.
+    2. Against the fp64 oracle logits: identical indices on every token whose
+       top-(k+1) logits are separated by more than the fp32 rounding bound tau;
+       on near-tied tokens, the device's picks are a valid top-k within tau.
+    Returns (number of near-tied tokens, oracle fp64 logits).
+    """
+    gpu_idx = np.asarray(gpu_idx)
+    T = gpu_idx.shape[0]
+    gl = np.asarray(gpu_logits, dtype=np.float64)
+    ref_idx_on_gpu_logits = oracle.topk_order(gl, k)
+    np.testing.assert_array_equal(gpu_idx, ref_idx_on_gpu_logits)
+    np.testing.assert_allclose(gpu_w, oracle_gates_for(gl, gpu_idx), rtol=2e-6, atol=1e-7)
+    logits64 = oracle.router_logits(x_bits, w_router, bias)
+    ref_idx = oracle.topk_order(logits64, k)
+    tau = near_tie_tau(x_bits, w_router, bias)
+    srt = -np.sort(-logits64, axis=1)[:, :k + 1]
+    gaps = srt[:, :-1] - srt[:, 1:] if srt.shape[1] > k else srt[:, :-1] - srt[:, 1:]
+    tied = (gaps < tau[:, None]).any(axis=1)
+    for t in range(T):
+        if not tied[t]:
+            assert gpu_idx[t].tolist() == ref_idx[t].tolist(), f"token {t}: {gpu_idx[t]} vs {ref_idx[t]}"
+        else:
+            sel = gpu_idx[t]
+            assert len(set(sel.tolist())) == k
+            kth = srt[t, k - 1]
+            assert np.all(logits64[t, sel] >= kth - tau[t])
+            assert np.all(np.diff(logits64[t, sel]) <= tau[t])
+    return int(tied.sum()), logits64
+
+
+def upload_layer(lay, device="cuda"):
+    """Device copies of a workload.LayerInputs (router, routed + shared experts)."""
+    import torch
+
+    from bit_quantized_moe_gemv_b200.device import DeviceExperts
+    d = dict(
+        w_router=torch.from_numpy(lay.w_router).to(device),
+        experts=DeviceExperts(lay.experts, device),
+        shared=DeviceExperts([lay.shared], device) if lay.shared is not None else None,
+    )
+    return d
+
+
+def bias_tensor(bias, device="cuda"):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bias, dtype=np.float32)).to(device)

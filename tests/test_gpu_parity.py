@@ -1,0 +1,270 @@
+"""GPU parity of every step against the fp64 oracle, through the C ABI.
+
+Integer outputs (top-k indices, counts, offsets, permutations) must be
+bit-exact; floating outputs must be within rel L2 <= 5e-3 and max abs <=
+2e-2 x rms of the oracle. Small cases are compared element by element over
+all outputs; the full-size workloads on sampled tokens/rows.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from bit_quantized_moe_gemv_b200 import workload as wlm
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from bit_quantized_moe_gemv_b200 import build
+    build.build()
+    from bit_quantized_moe_gemv_b200 import _lib
+    return _lib
+
+
+def _t(a, dtype=None):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.cuda() if dtype is None else t.to(dtype).cuda()
+
+
+def _small_mixed():
+    return wlm.Workload("small_mixed", T=19, H=128, I=64, E=12, k=3, zipf_s=0.5, uniform_frac=0.3,
+                        routed_qtypes=((0, 4, wlm.Q_INT4_SYM_G32), (4, 8, wlm.Q_INT2_ASYM_G16),
+                                       (8, None, wlm.Q_INT8_PER_CHANNEL)),
+                        shared_qtype=wlm.Q_INT8_PER_CHANNEL, seed=3)
+
+
+SMALL = {
+    "tiny": wlm.WORKLOADS["tiny"],
+    "small_mixed": _small_mixed(),
+    "k_equals_E": wlm.Workload("k_equals_E", T=5, H=128, I=64, E=16, k=16, seed=4),
+    "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
+                              shared_qtype=wlm.Q_INT2_ASYM_G16),
+}
+
+
+def _run_steps(L, wl, lay, dev, xb, bias, stride, ws):
+    """Run route/dispatch/expert_ffn/combine separately; return host results."""
+    import torch
+    T, k, E, H, I = wl.T, wl.k, wl.E, wl.H, wl.I
+    from bit_quantized_moe_gemv_b200.device import bf16_bits, bf16_tensor
+    x = bf16_tensor(xb)
+    b = pu.bias_tensor(bias)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    L.route(x, dev["w_router"], b, stride, k, idx, w, ws, logits=logits)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    L.dispatch(idx, E, counts, offsets, perm, inv, ws)
+    y_perm = torch.empty((T * k, H), dtype=torch.bfloat16, device="cuda")
+    L.expert_ffn(x, I, k, E, perm, offsets, counts, dev["experts"].table, y_perm, ws)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    L.combine(y_perm, inv, w, I, x, dev["shared"].table if dev["shared"] else None, out, ws)
+    torch.cuda.synchronize()
+    assert L.get_status(ws) == 0
+    return dict(idx=idx.cpu().numpy(), w=w.cpu().numpy(), logits=logits.cpu().numpy(), counts=counts.cpu().numpy(),
+                offsets=offsets.cpu().numpy(), perm=perm.cpu().numpy(), inv=inv.cpu().numpy(),
+                y_perm=bf16_bits(y_perm), out=bf16_bits(out))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_steps_small_all_outputs(L, name):
+    wl = SMALL[name]
+    lay = wlm.gen_layer(wl)
+    dev = pu.upload_layer(lay)
+    xb = wlm.gen_x(wl)
+    bias, stride = wlm.gen_bias(wl)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+    g = _run_steps(L, wl, lay, dev, xb, bias, stride, ws)
+    ntied, logits64 = pu.check_routing(g["idx"], g["w"], g["logits"], xb, lay.w_router, bias, wl.k)
+    assert ntied == 0
+    counts, offsets, perm, inv = oracle.dispatch(g["idx"], wl.E)
+    np.testing.assert_array_equal(g["counts"], counts)
+    np.testing.assert_array_equal(g["offsets"], offsets)
+    np.testing.assert_array_equal(g["perm"], perm)
+    np.testing.assert_array_equal(g["inv"], inv)
+    y_ref = oracle.expert_rows(xb, perm, offsets, wl.k, lay.experts)
+    pu.assert_close(pu.bf16_to_f64(g["y_perm"]), y_ref, "y_perm")
+    ref = oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared)
+    pu.assert_close(pu.bf16_to_f64(g["out"]), ref["out"], "out")
+    # combine alone: oracle combine on the device's own y_perm and gates
+    sy = oracle.shared_rows(xb, lay.shared)
+    comb = oracle.combine(pu.bf16_to_f64(g["y_perm"]), g["inv"], g["w"].astype(np.float64), wl.k, sy)
+    pu.assert_close(pu.bf16_to_f64(g["out"]), comb, "combine")
+
+
+def _layer_call(L, wl, dev, xb, bias, stride, ws):
+    import torch
+
+    from bit_quantized_moe_gemv_b200.device import bf16_bits, bf16_tensor
+    x = bf16_tensor(xb)
+    idx = torch.empty((x.shape[0], wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((x.shape[0], wl.k), dtype=torch.float32, device="cuda")
+    out = torch.empty((x.shape[0], wl.H), dtype=torch.bfloat16, device="cuda")
+    L.layer(x, wl.I, wl.E, wl.k, dev["w_router"], pu.bias_tensor(bias), stride, dev["experts"].table,
+            dev["shared"].table if dev["shared"] else None, idx, w, out, ws)
+    torch.cuda.synchronize()
+    assert L.get_status(ws) == 0
+    return idx.cpu().numpy(), w.cpu().numpy(), bf16_bits(out)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small(L, name):
+    wl = SMALL[name]
+    lay = wlm.gen_layer(wl)
+    dev = pu.upload_layer(lay)
+    xb = wlm.gen_x(wl)
+    bias, stride = wlm.gen_bias(wl)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+    idx, w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+    ref = oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    np.testing.assert_allclose(w, ref["w"], rtol=1e-5, atol=1e-6)
+    pu.assert_close(pu.bf16_to_f64(out), ref["out"])
+    # determinism: a second call gives identical bits
+    idx2, w2, out2 = _layer_call(L, wl, dev, xb, bias, stride, ws)
+    np.testing.assert_array_equal(out2, out)
+    np.testing.assert_array_equal(w2, w)
+
+
+def _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, tokens):
+    cache = oracle.DequantCache(lay.experts, capacity=256)
+    sh = tuple(oracle.dequant_qm(m) for m in (lay.shared.gate, lay.shared.up, lay.shared.down))
+    logits64 = oracle.router_logits(xb[tokens], lay.w_router, bias[tokens] if stride else bias)
+    for n, t in enumerate(tokens):
+        brow = bias[t] if stride else bias
+        # same expert set as the device (identical except on flagged near-ties)
+        gates = pu.oracle_gates_for(logits64[n:n + 1], idx[t:t + 1])[0]
+        _, _, ref = oracle.moe_token(xb[t], lay.w_router, brow, wl.k, cache, sh, routing=(idx[t], gates))
+        pu.assert_close(pu.bf16_to_f64(out[t]), ref, f"token {t}")
+        np.testing.assert_allclose(w[t], gates, rtol=1e-5, atol=1e-6)
+
+
+def test_layer_decode1_steps(L):
+    wl = wlm.WORKLOADS["decode1"]
+    lay = wlm.gen_layer(wl)
+    dev = pu.upload_layer(lay)
+    bias, stride = wlm.gen_bias(wl)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+    for step in range(6):
+        xb = wlm.gen_x(wl, step=step)
+        idx, w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+        logits64 = oracle.router_logits(xb, lay.w_router, bias)
+        ref_idx = oracle.topk_order(logits64, wl.k)
+        tau = pu.near_tie_tau(xb, lay.w_router, bias)
+        srt = -np.sort(-logits64, axis=1)[:, :wl.k + 1]
+        if not (np.diff(-srt, axis=1) < tau[:, None]).any():
+            np.testing.assert_array_equal(idx, ref_idx)
+        _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, [0])
+
+
+@pytest.mark.parametrize("name", ["prefill8k", "prefill32k"])
+def test_prefill_full_routing_dispatch_sampled_outputs(L, name):
+    import torch
+
+    from bit_quantized_moe_gemv_b200.device import bf16_tensor
+    wl = wlm.WORKLOADS[name]
+    lay = wlm.gen_layer(wl)
+    dev = pu.upload_layer(lay)
+    xb = wlm.gen_x(wl)
+    bias, stride = wlm.gen_bias(wl)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+    x = bf16_tensor(xb)
+    T, k, E = wl.T, wl.k, wl.E
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    logits = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    L.route(x, dev["w_router"], pu.bias_tensor(bias), stride, k, idx, w, ws, logits=logits)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    L.dispatch(idx, E, counts, offsets, perm, inv, ws)
+    torch.cuda.synchronize()
+    gi = idx.cpu().numpy()
+    ntied, _ = pu.check_routing(gi, w.cpu().numpy(), logits.cpu().numpy(), xb, lay.w_router, bias, k)
+    assert ntied <= max(3, T // 200)
+    c, o, p, v = oracle.dispatch(gi, E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), c)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), o)
+    np.testing.assert_array_equal(perm.cpu().numpy(), p)
+    np.testing.assert_array_equal(inv.cpu().numpy(), v)
+    # whole layer through moe_layer, sampled tokens against the oracle
+    out_idx, out_w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+    np.testing.assert_array_equal(out_idx, gi)
+    rng = np.random.default_rng(0)
+    tokens = sorted(set([0, T - 1] + rng.choice(T, 14, replace=False).tolist()))
+    _check_sampled_tokens(wl, lay, xb, bias, stride, out_idx, out_w, out, tokens)
+
+
+def test_decode48_two_layers(L):
+    wl = wlm.WORKLOADS["decode48"]
+    for layer in (0, 47):
+        lay = wlm.gen_layer(wl, layer)
+        dev = pu.upload_layer(lay)
+        bias, stride = wlm.gen_bias(wl)
+        ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+        for step in (0, 199):
+            xb = wlm.gen_x(wl, step=step, layer=layer)
+            idx, w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+            _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, list(range(wl.T)))
+
+
+def test_dispatch_invalid_id_flags_device_fault(L):
+    import torch
+    E, T, k = 8, 3, 2
+    ids = torch.tensor([[0, 1], [8, 2], [3, 1]], dtype=torch.int32, device="cuda")
+    ws = L.new_workspace(T, 64, 64, E, k)
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    L.dispatch(ids, E, counts, offsets, perm, inv, ws)
+    assert L.get_status(ws) == 5
+    assert inv.cpu().numpy()[2] == -1
+    assert counts.cpu().numpy().sum() == 5 and offsets.cpu().numpy()[-1] == 5
+    L.reset_status(ws)
+    assert L.get_status(ws) == 0
+
+
+def test_bad_descriptor_flags_device_fault(L):
+    import torch
+    wl = SMALL["tiny"]
+    lay = wlm.gen_layer(wl)
+    dev = pu.upload_layer(lay)
+    # corrupt every routed expert's gate qtype (first int32 of each descriptor)
+    tab = dev["experts"].table.view(torch.int32).view(wl.E, -1)
+    tab[:, 0] = 9
+    xb = wlm.gen_x(wl)
+    bias, stride = wlm.gen_bias(wl)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+    from bit_quantized_moe_gemv_b200.device import bf16_tensor
+    x = bf16_tensor(xb)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    L.layer(x, wl.I, wl.E, wl.k, dev["w_router"], pu.bias_tensor(bias), stride, dev["experts"].table,
+            dev["shared"].table, idx, w, out, ws)
+    assert L.get_status(ws) == 5
+
+
+def test_zero_tokens_is_noop(L):
+    import torch
+    ws = L.new_workspace(0, 128, 64, 8, 2)
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    counts = torch.full((8,), 3, dtype=torch.int32, device="cuda")
+    offsets = torch.full((9,), 3, dtype=torch.int32, device="cuda")
+    idx = torch.empty((0, 2), dtype=torch.int32, device="cuda")
+    L.dispatch(idx, 8, counts, offsets, torch.empty(0, dtype=torch.int32, device="cuda"),
+               torch.empty(0, dtype=torch.int32, device="cuda"), ws)
+    torch.cuda.synchronize()
+    assert counts.cpu().numpy().tolist() == [0] * 8 and offsets.cpu().numpy().tolist() == [0] * 9
+    assert L.get_status(ws) == 0
+    del x
