@@ -104,7 +104,7 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
                                       ws_at<float>(ws, L.h), nullptr, nullptr, shared_y, ws_at<WsHeader>(ws, 0), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
-  return cuda_status(launch_combine(y_perm, inv_perm, topk_w, T, H, k, shared_y, out, st));
+  return cuda_status(launch_combine(y_perm, nullptr, inv_perm, topk_w, T, H, k, shared_y, out, st));
 }
 
 moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k, const float* w_router,
@@ -122,24 +122,28 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   const WsLayout L = ws_layout(T, H, I, E, k);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WsHeader* hdr = ws_at<WsHeader>(ws, 0);
+  if (decode_fused_eligible(T, H, I, E, k))
+    return cuda_status(launch_decode_fused(x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev,
+                                           topk_idx, topk_w, out, ws_at<float>(ws, L.partial), ws_at<float>(ws, L.h),
+                                           hdr, st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
   int* perm = ws_at<int>(ws, L.perm);
   int* inv = ws_at<int>(ws, L.inv);
-  uint16_t* y_perm = ws_at<uint16_t>(ws, L.y_perm);
+  float* y_perm = ws_at<float>(ws, L.y_perm);  // fp32: out is rounded only once
   cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w,
                                ws_at<float>(ws, L.logits), hdr, st);
   if (e == cudaSuccess) e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, inv, ws_at<int>(ws, L.hist), hdr, st);
   if (e == cudaSuccess)
     e = launch_expert_ffn(x, T, H, I, k, E, perm, offsets, counts, experts_dev, false, ws_at<float>(ws, L.h),
-                          ws_at<int>(ws, L.active), y_perm, nullptr, hdr, st);
+                          ws_at<int>(ws, L.active), nullptr, y_perm, hdr, st);
   float* shared_y = nullptr;
   if (e == cudaSuccess && shared_dev) {
     shared_y = ws_at<float>(ws, L.shared_y);
     e = launch_expert_ffn(x, T, H, I, k, 1, nullptr, nullptr, nullptr, shared_dev, true,
                           ws_at<float>(ws, L.h) + size_t(T) * k * I, nullptr, nullptr, shared_y, hdr, st);
   }
-  if (e == cudaSuccess) e = launch_combine(y_perm, inv, topk_w, T, H, k, shared_y, out, st);
+  if (e == cudaSuccess) e = launch_combine(nullptr, y_perm, inv, topk_w, T, H, k, shared_y, out, st);
   return cuda_status(e);
 }
 

@@ -14,8 +14,24 @@
 
 namespace moe {
 
+// Eight consecutive values of row r of y (bf16 or fp32 rows) as fp32.
+__device__ __forceinline__ void load8(const uint16_t* y, size_t off, float* v) {
+  const uint4 q = *reinterpret_cast<const uint4*>(y + off);
+  const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(u[i] << 16);
+    v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void load8(const float* y, size_t off, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(y + off), b = *reinterpret_cast<const float4*>(y + off + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <typename YT>
 __global__ void __launch_bounds__(256)
-combine_kernel(const uint16_t* __restrict__ y_perm, const int* __restrict__ inv_perm, const float* __restrict__ topk_w,
+combine_kernel(const YT* __restrict__ y_perm, const int* __restrict__ inv_perm, const float* __restrict__ topk_w,
                int T, int H, int k, const float* __restrict__ shared_y, uint16_t* __restrict__ out) {
   const int per_tok = H / 8;
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -29,13 +45,10 @@ combine_kernel(const uint16_t* __restrict__ y_perm, const int* __restrict__ inv_
     const int r = inv_perm[(long long)t * k + j];
     if (r < 0 || r >= nrows) continue;  // invalid expert id upstream (flagged there)
     const float w = topk_w[(long long)t * k + j];
-    const uint4 v = *reinterpret_cast<const uint4*>(y_perm + (size_t)r * H + 8 * c);
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    float v[8];
+    load8(y_perm, (size_t)r * H + 8 * c, v);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      acc[2 * q] = fmaf(w, __uint_as_float(u[q] << 16), acc[2 * q]);
-      acc[2 * q + 1] = fmaf(w, __uint_as_float(u[q] & 0xffff0000u), acc[2 * q + 1]);
-    }
+    for (int q = 0; q < 8; ++q) acc[q] = fmaf(w, v[q], acc[q]);
   }
   if (shared_y) {
     const float4* s = reinterpret_cast<const float4*>(shared_y + (size_t)t * H + 8 * c);
@@ -51,11 +64,15 @@ combine_kernel(const uint16_t* __restrict__ y_perm, const int* __restrict__ inv_
   *reinterpret_cast<uint4*>(out + (size_t)t * H + 8 * c) = o;
 }
 
-cudaError_t launch_combine(const uint16_t* y_perm, const int* inv_perm, const float* topk_w, int T, int H, int k,
-                           const float* shared_y, uint16_t* out, cudaStream_t st) {
+cudaError_t launch_combine(const uint16_t* y_bf16, const float* y_f32, const int* inv_perm, const float* topk_w,
+                           int T, int H, int k, const float* shared_y, uint16_t* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const long long n = (long long)T * (H / 8);
-  combine_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(y_perm, inv_perm, topk_w, T, H, k, shared_y, out);
+  const unsigned grid = unsigned((n + 255) / 256);
+  if (y_f32)
+    combine_kernel<float><<<grid, 256, 0, st>>>(y_f32, inv_perm, topk_w, T, H, k, shared_y, out);
+  else
+    combine_kernel<uint16_t><<<grid, 256, 0, st>>>(y_bf16, inv_perm, topk_w, T, H, k, shared_y, out);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -18,14 +18,17 @@ constexpr int kTicketSlots = 16;
 struct WsHeader {
   int32_t status;        // first device-side error code (MOE_OK = none)
   int32_t detail;        // code-specific detail (e.g. the bad expert id)
-  int32_t pad[14];
+  int32_t abort;         // set when a bounded grid barrier gave up
+  uint32_t bar_count;    // grid-barrier arrivals of the running fused launch
+  uint32_t exit_count;   // CTAs that left the running fused launch
+  int32_t pad[11];
   uint32_t tickets[kTicketSlots];  // last-CTA tickets, always left at 0
 };
 static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 
 // Offsets (bytes from the workspace base) of every workspace segment.
 struct WsLayout {
-  size_t counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, h, shared_y, y_perm;
+  size_t counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, partial, h, shared_y, y_perm;
   size_t total;
 };
 
@@ -45,9 +48,10 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   L.topk_idx = take(4 * n);
   L.topk_w = take(4 * n);
   L.logits = take(4 * T * E);
+  L.partial = take(16 * T * E);  // router partial sums of the fused decode path
   L.h = take(4 * (n + T) * I);
   L.shared_y = take(4 * T * H);
-  L.y_perm = take(2 * n * H);
+  L.y_perm = take(4 * n * H);  // fp32 routed rows inside moe_layer
   L.total = o;
   return L;
 }
@@ -85,11 +89,11 @@ __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)
 // Validate one packed matrix descriptor against the expected shape.
 __device__ inline bool qmatrix_ok(const moe_qmatrix& m, int rows, int cols) {
   if (m.rows != rows || m.cols != cols || m.codes == nullptr || m.scales == nullptr) return false;
-  if ((reinterpret_cast<uintptr_t>(m.codes) & 15) || (reinterpret_cast<uintptr_t>(m.scales) & 1)) return false;
+  if ((reinterpret_cast<uintptr_t>(m.codes) & 15) || (reinterpret_cast<uintptr_t>(m.scales) & 15)) return false;
   switch (m.qtype) {
     case MOE_Q_INT4_SYM_G32: return m.group == 32 && (cols % 64) == 0;
     case MOE_Q_INT2_ASYM_G16:
-      return m.group == 16 && (cols % 64) == 0 && m.mins != nullptr && !(reinterpret_cast<uintptr_t>(m.mins) & 1);
+      return m.group == 16 && (cols % 64) == 0 && m.mins != nullptr && !(reinterpret_cast<uintptr_t>(m.mins) & 15);
     case MOE_Q_INT8_PER_CHANNEL: return m.group == 0 && (cols % 64) == 0;
     default: return false;
   }

@@ -31,7 +31,15 @@ cudaError_t launch_expert_ffn(const uint16_t* x, int T, int H, int I, int k, int
                               float* h_ws, int* active_ws, uint16_t* y_bf16, float* y_f32, WsHeader* hdr,
                               cudaStream_t st);
 
-cudaError_t launch_combine(const uint16_t* y_perm, const int* inv_perm, const float* topk_w, int T, int H, int k,
-                           const float* shared_y, uint16_t* out, cudaStream_t st);
+// Fused single-launch decode step (T <= 4); see decode_fused.cu.
+bool decode_fused_eligible(int T, int H, int I, int E, int k);
+cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
+                                const float* bias, long long bstride, const moe_expert* experts,
+                                const moe_expert* shared, int* topk_idx, float* topk_w, uint16_t* out,
+                                float* partial, float* h, WsHeader* hdr, cudaStream_t st);
+
+// Combine routed rows given as bf16 (y_bf16) or fp32 (y_f32; the other NULL).
+cudaError_t launch_combine(const uint16_t* y_bf16, const float* y_f32, const int* inv_perm, const float* topk_w,
+                           int T, int H, int k, const float* shared_y, uint16_t* out, cudaStream_t st);
 
 }  // namespace moe

@@ -70,9 +70,9 @@ typedef int32_t moe_status;
 #define MOE_Q_INT2_ASYM_G16 2
 #define MOE_Q_INT8_PER_CHANNEL 3
 
-/* One packed matrix. `codes` must be 16-byte aligned, `scales`/`mins`
- * 2-byte aligned; `mins` is NULL except for MOE_Q_INT2_ASYM_G16. `group` is
- * 32, 16 or 0 (per channel) and must agree with `qtype`. */
+/* One packed matrix. `codes`, `scales` and `mins` must be 16-byte aligned;
+ * `mins` is NULL except for MOE_Q_INT2_ASYM_G16. `group` is 32, 16 or 0
+ * (per channel) and must agree with `qtype`. */
 typedef struct moe_qmatrix {
   int32_t qtype;
   int32_t rows;
@@ -92,7 +92,8 @@ typedef struct moe_expert {
 } moe_expert;
 
 /* Bytes of workspace the calls below need for a problem of this size (the
- * same value serves every call). Returns 0 for shapes outside the limits. */
+ * same value serves every call). Returns 0 for shapes outside the limits.
+ * Call moe_reset_status once on a new workspace before its first use. */
 size_t moe_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k);
 
 /*
@@ -172,9 +173,11 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
 /*
  * moe_layer - the whole step (route, dispatch, experts, combine) in one call.
  * Same arguments and layouts as the four calls above; dispatch arrays and
- * intermediate rows live in the workspace. Small batches (T*k <= 64) take a
- * fused decode path that never materialises y_perm and keeps the expert
- * outputs in fp32 until the final rounding.
+ * intermediate rows live in the workspace and stay fp32, so `out` is rounded
+ * once. Decode batches (1 <= T <= 4, H and I <= 2048) run as ONE cooperative
+ * persistent kernel whose grid barriers are bounded: if one expires the call
+ * leaves MOE_ERR_TIMEOUT in the status word, and the workspace must be reset
+ * with moe_reset_status before it is used again.
  */
 moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k,
                      const float* w_router, const float* bias, int64_t bias_row_stride,

@@ -25,6 +25,14 @@ def assert_close(got, ref, what="output"):
     return rel, mx / max(rms, 1e-300)
 
 
+def round_bf16(a):
+    """Round float64 values to bf16 (nearest even), returned as float64."""
+    f = np.asarray(a, dtype=np.float64).astype(np.float32)  # exact enough: bf16 keeps 8 of fp32's 24 bits
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint32) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def bf16_to_f64(bits):
     return oracle.bf16_bits_to_f64(bits)
 

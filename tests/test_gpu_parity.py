@@ -40,6 +40,14 @@ def _small_mixed():
 
 SMALL = {
     "tiny": wlm.WORKLOADS["tiny"],
+    # decode-sized batches that take the fused single-launch path (T <= 4)
+    "fused_mixed_T3": wlm.Workload("fused_mixed_T3", T=3, H=512, I=256, E=32, k=4, zipf_s=0.8, seed=7,
+                                   routed_qtypes=((0, 10, wlm.Q_INT4_SYM_G32), (10, 20, wlm.Q_INT2_ASYM_G16),
+                                                  (20, None, wlm.Q_INT8_PER_CHANNEL)),
+                                   shared_qtype=wlm.Q_INT8_PER_CHANNEL),
+    "fused_int4_T1": wlm.Workload("fused_int4_T1", T=1, H=1024, I=512, E=64, k=6, zipf_s=1.1, seed=8),
+    "fused_int2_T4": wlm.Workload("fused_int2_T4", T=4, H=768, I=512, E=24, k=5, seed=9,
+                                  routed_qtypes=((0, None, wlm.Q_INT2_ASYM_G16),), shared_qtype=wlm.Q_INT4_SYM_G32),
     "small_mixed": _small_mixed(),
     "k_equals_E": wlm.Workload("k_equals_E", T=5, H=128, I=64, E=16, k=16, seed=4),
     "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
@@ -92,12 +100,19 @@ def test_steps_small_all_outputs(L, name):
     np.testing.assert_array_equal(g["inv"], inv)
     y_ref = oracle.expert_rows(xb, perm, offsets, wl.k, lay.experts)
     pu.assert_close(pu.bf16_to_f64(g["y_perm"]), y_ref, "y_perm")
-    ref = oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared)
-    pu.assert_close(pu.bf16_to_f64(g["out"]), ref["out"], "out")
+    # The four-call path defines y_perm as bf16: compare with the oracle's rows
+    # rounded the same way (moe_layer keeps them in fp32; see test_layer_small).
+    sy = oracle.shared_rows(xb, lay.shared)
+    ref_out = oracle.combine(pu.round_bf16(y_ref), inv, oracle_gates(xb, lay, bias, g["idx"]), wl.k, sy)
+    pu.assert_close(pu.bf16_to_f64(g["out"]), ref_out, "out")
     # combine alone: oracle combine on the device's own y_perm and gates
     sy = oracle.shared_rows(xb, lay.shared)
     comb = oracle.combine(pu.bf16_to_f64(g["y_perm"]), g["inv"], g["w"].astype(np.float64), wl.k, sy)
     pu.assert_close(pu.bf16_to_f64(g["out"]), comb, "combine")
+
+
+def oracle_gates(xb, lay, bias, idx):
+    return pu.oracle_gates_for(oracle.router_logits(xb, lay.w_router, bias), idx)
 
 
 def _layer_call(L, wl, dev, xb, bias, stride, ws):
@@ -190,7 +205,8 @@ def test_prefill_full_routing_dispatch_sampled_outputs(L, name):
     torch.cuda.synchronize()
     gi = idx.cpu().numpy()
     ntied, _ = pu.check_routing(gi, w.cpu().numpy(), logits.cpu().numpy(), xb, lay.w_router, bias, k)
-    assert ntied <= max(3, T // 200)
+    print(f"{name}: {ntied} of {T} tokens have a near-tie within tau among their top-{k + 1} logits")
+    assert ntied <= T // 50
     c, o, p, v = oracle.dispatch(gi, E)
     np.testing.assert_array_equal(counts.cpu().numpy(), c)
     np.testing.assert_array_equal(offsets.cpu().numpy(), o)
