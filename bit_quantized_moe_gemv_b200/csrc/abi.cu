@@ -17,6 +17,8 @@ void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order
 
 namespace {
 
+constexpr int kDecodeMaxT = 4;  // larger batches take the tensor-core prefill path
+
 bool shape_ok(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
   if (T < 0 || H <= 0 || I <= 0 || E < 1 || E > kMaxE || k < 1 || k > E || k > kMaxK) return false;
   if (H % 64 || I % 64) return false;
@@ -81,6 +83,10 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, in
   moe_status s = ws_check(ws, ws_bytes, T, H, I, E, k);
   if (s != MOE_OK) return s;
   const WsLayout L = ws_layout(T, H, I, E, k);
+  if (T > kDecodeMaxT && grouped_eligible(H, I, E, false))
+    return cuda_status(launch_grouped_ffn(x, T, H, I, k, E, perm_src, offsets, counts, experts_dev, nullptr, nullptr,
+                                          y_perm, nullptr, ws_at<void>(ws, L.gemm), ws_at<WsHeader>(ws, 0),
+                                          static_cast<cudaStream_t>(stream)));
   return cuda_status(launch_expert_ffn(x, T, H, I, k, E, perm_src, offsets, counts, experts_dev, false,
                                        ws_at<float>(ws, L.h), ws_at<int>(ws, L.active), y_perm, nullptr,
                                        ws_at<WsHeader>(ws, 0), static_cast<cudaStream_t>(stream)));
@@ -100,8 +106,13 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
   float* shared_y = nullptr;
   if (shared_dev) {
     shared_y = ws_at<float>(ws, L.shared_y);
-    cudaError_t e = launch_expert_ffn(x, T, H, I, k, 1, nullptr, nullptr, nullptr, shared_dev, true,
-                                      ws_at<float>(ws, L.h), nullptr, nullptr, shared_y, ws_at<WsHeader>(ws, 0), st);
+    cudaError_t e;
+    if (T > kDecodeMaxT && grouped_eligible(H, I, 0, true))
+      e = launch_grouped_ffn(x, T, H, I, k, 0, nullptr, nullptr, nullptr, nullptr, shared_dev, nullptr, nullptr,
+                             shared_y, ws_at<void>(ws, L.gemm), ws_at<WsHeader>(ws, 0), st);
+    else
+      e = launch_expert_ffn(x, T, H, I, k, 1, nullptr, nullptr, nullptr, shared_dev, true, ws_at<float>(ws, L.h),
+                            nullptr, nullptr, shared_y, ws_at<WsHeader>(ws, 0), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   return cuda_status(launch_combine(y_perm, nullptr, inv_perm, topk_w, T, H, k, shared_y, out, st));
@@ -134,10 +145,18 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w,
                                ws_at<float>(ws, L.logits), hdr, st);
   if (e == cudaSuccess) e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, inv, ws_at<int>(ws, L.hist), hdr, st);
+  float* shared_y = nullptr;
+  if (T > kDecodeMaxT && grouped_eligible(H, I, E, shared_dev != nullptr)) {
+    if (shared_dev) shared_y = ws_at<float>(ws, L.shared_y);
+    if (e == cudaSuccess)
+      e = launch_grouped_ffn(x, T, H, I, k, E, perm, offsets, counts, experts_dev, shared_dev, y_perm, nullptr,
+                             shared_y, ws_at<void>(ws, L.gemm), hdr, st);
+    if (e == cudaSuccess) e = launch_combine(nullptr, y_perm, inv, topk_w, T, H, k, shared_y, out, st);
+    return cuda_status(e);
+  }
   if (e == cudaSuccess)
     e = launch_expert_ffn(x, T, H, I, k, E, perm, offsets, counts, experts_dev, false, ws_at<float>(ws, L.h),
                           ws_at<int>(ws, L.active), nullptr, y_perm, hdr, st);
-  float* shared_y = nullptr;
   if (e == cudaSuccess && shared_dev) {
     shared_y = ws_at<float>(ws, L.shared_y);
     e = launch_expert_ffn(x, T, H, I, k, 1, nullptr, nullptr, nullptr, shared_dev, true,

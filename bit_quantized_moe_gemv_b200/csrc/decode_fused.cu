@@ -88,52 +88,6 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   return v;
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* base, size_t lo, size_t hi) {
-  // L2 prefetch of [lo, hi) bytes from base; only whole 16-byte blocks inside
-  // the range are touched.
-  const uintptr_t a = (reinterpret_cast<uintptr_t>(base) + lo + 15) & ~uintptr_t(15);
-  const uintptr_t b = (reinterpret_cast<uintptr_t>(base) + hi) & ~uintptr_t(15);
-  if (b <= a) return;
-  uint32_t left = uint32_t(b - a);
-  uintptr_t p = a;
-  while (left) {
-    const uint32_t n = left > (1u << 20) ? (1u << 20) : left;
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(n) : "memory");
-    p += n;
-    left -= n;
-  }
-}
-
-// Bounded grid barrier. Returns false (on every thread of the CTA) if the
-// wait expired or another CTA gave up; the status word then reads TIMEOUT.
-__device__ bool grid_sync(WsHeader* hdr, uint32_t target) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    __threadfence();
-    atomicAdd(&hdr->bar_count, 1u);
-    const long long t0 = clock64();
-    while (ld_acquire(&hdr->bar_count) < target) {
-      if (*reinterpret_cast<volatile int*>(&hdr->abort)) {
-        ok = 0;
-        break;
-      }
-      if (clock64() - t0 > kSpinCycles) {
-        flag_error(hdr, MOE_ERR_TIMEOUT, int(target));
-        atomicExch(&hdr->abort, 1);
-        ok = 0;
-        break;
-      }
-      __nanosleep(64);
-    }
-    __threadfence();
-    s_ok = ok;
-  }
-  __syncthreads();
-  return s_ok != 0;
-}
-
 // ---------------------------------------------------------------- dot engine
 // One warp computes dot products of whole rows of a packed matrix with one
 // activation vector kept in registers. Lane l owns chunks c = l + 32 j
@@ -224,74 +178,48 @@ struct XRegs {
   }
 };
 
-// Partial dot product of this lane's chunks of one row with x. `codes` is
-// the row's packed codes (shared memory), `sc`/`mn` its fp16 group scales and
-// mins (shared memory; int8 rows take their scale from the caller instead).
-template <int QT, int CPL>
-__device__ __forceinline__ float row_dot(const uint8_t* codes, const uint16_t* sc, const uint16_t* mn, int CPR,
-                                         const XRegs<QT, CPL>& x) {
-  const int lane = threadIdx.x & 31;
-  float acc = 0.f;
-#pragma unroll
-  for (int j = 0; j < CPL; ++j) {
-    const int c = lane + 32 * j;
-    if (c >= CPR) continue;
-    const uint4 raw = *reinterpret_cast<const uint4*>(codes + 16 * c);
-    const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
-    if (QT == MOE_Q_INT4_SYM_G32) {
-      float2 s2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t lo = wd[w] & 0x0F0F0F0Fu, hi = (wd[w] >> 4) & 0x0F0F0F0Fu;
-        const float* xv = x.v[j] + 8 * w;
-        s2 = ffma2(make_float2(code_f<0>(lo), code_f<1>(lo)), make_float2(xv[0], xv[1]), s2);
-        s2 = ffma2(make_float2(code_f<2>(lo), code_f<3>(lo)), make_float2(xv[2], xv[3]), s2);
-        s2 = ffma2(make_float2(code_f<0>(hi), code_f<1>(hi)), make_float2(xv[4], xv[5]), s2);
-        s2 = ffma2(make_float2(code_f<2>(hi), code_f<3>(hi)), make_float2(xv[6], xv[7]), s2);
-      }
-      const float s = f16_to_f32(sc[c]);
-      // sum (c - 8) x = 256 S - 136 X
-      acc = fmaf(s, fmaf(256.f, s2.x + s2.y, -136.f * x.gsum[j][0]), acc);
-    } else if (QT == MOE_Q_INT2_ASYM_G16) {
-      const uint2 scw = *reinterpret_cast<const uint2*>(sc + 4 * c);
-      const uint2 mnw = *reinterpret_cast<const uint2*>(mn + 4 * c);
-      const uint32_t sv[4] = {scw.x & 0xffffu, scw.x >> 16, scw.y & 0xffffu, scw.y >> 16};
-      const uint32_t mv[4] = {mnw.x & 0xffffu, mnw.x >> 16, mnw.y & 0xffffu, mnw.y >> 16};
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t b0 = wd[w] & 0x03030303u, b1 = (wd[w] >> 2) & 0x03030303u;
-        const uint32_t b2 = (wd[w] >> 4) & 0x03030303u, b3 = (wd[w] >> 6) & 0x03030303u;
-        const float* xv = x.v[j] + 16 * w;
-        float2 s2 = make_float2(0.f, 0.f);
-        s2 = ffma2(make_float2(code_f<0>(b0), code_f<1>(b0)), make_float2(xv[0], xv[1]), s2);
-        s2 = ffma2(make_float2(code_f<2>(b0), code_f<3>(b0)), make_float2(xv[2], xv[3]), s2);
-        s2 = ffma2(make_float2(code_f<0>(b1), code_f<1>(b1)), make_float2(xv[4], xv[5]), s2);
-        s2 = ffma2(make_float2(code_f<2>(b1), code_f<3>(b1)), make_float2(xv[6], xv[7]), s2);
-        s2 = ffma2(make_float2(code_f<0>(b2), code_f<1>(b2)), make_float2(xv[8], xv[9]), s2);
-        s2 = ffma2(make_float2(code_f<2>(b2), code_f<3>(b2)), make_float2(xv[10], xv[11]), s2);
-        s2 = ffma2(make_float2(code_f<0>(b3), code_f<1>(b3)), make_float2(xv[12], xv[13]), s2);
-        s2 = ffma2(make_float2(code_f<2>(b3), code_f<3>(b3)), make_float2(xv[14], xv[15]), s2);
-        const float s = f16_to_f32(uint16_t(sv[w])), m = f16_to_f32(uint16_t(mv[w]));
-        // sum (c s + m) x = 256 s S + (m - 128 s) X
-        acc = fmaf(256.f * s, s2.x + s2.y, fmaf(m - 128.f * s, x.gsum[j][w], acc));
-      }
-    } else {
-      float2 s2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const uint32_t u = wd[w] ^ 0x80808080u;  // q + 128 in each byte
-        const float* xv = x.v[j] + 4 * w;
-        float q[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          q[b] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | b)) - 8388736.0f;  // - (2^23 + 128)
-        s2 = ffma2(make_float2(q[0], q[1]), make_float2(xv[0], xv[1]), s2);
-        s2 = ffma2(make_float2(q[2], q[3]), make_float2(xv[2], xv[3]), s2);
-      }
-      acc += s2.x + s2.y;  // the row scale is applied by the caller
-    }
+__device__ __forceinline__ void prefetch_l2(const void* base, size_t lo, size_t hi) {
+  // L2 prefetch of [lo, hi) bytes from base; only whole 16-byte blocks inside
+  // the range are touched.
+  const uintptr_t a = (reinterpret_cast<uintptr_t>(base) + lo + 15) & ~uintptr_t(15);
+  const uintptr_t b = (reinterpret_cast<uintptr_t>(base) + hi) & ~uintptr_t(15);
+  if (b <= a) return;
+  uint32_t left = uint32_t(b - a);
+  uintptr_t p = a;
+  while (left) {
+    const uint32_t n = left > (1u << 20) ? (1u << 20) : left;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(n) : "memory");
+    p += n;
+    left -= n;
   }
-  return acc;
+}
+
+// Bounded grid barrier. Returns false (on every thread of the CTA) if the
+// wait expired or another CTA gave up; the status word then reads TIMEOUT.
+__device__ bool grid_sync(WsHeader* hdr, uint32_t target) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    atomicAdd(&hdr->bar_count, 1u);
+    const long long t0 = clock64();
+    while (ld_acquire(&hdr->bar_count) < target) {
+      if (*reinterpret_cast<volatile int*>(&hdr->abort)) {
+        ok = 0;
+        break;
+      }
+      if (clock64() - t0 > kSpinCycles) {
+        flag_error(hdr, MOE_ERR_TIMEOUT, int(target));
+        atomicExch(&hdr->abort, 1);
+        ok = 0;
+        break;
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
 }
 
 __host__ __device__ __forceinline__ int bits_of(int qt) {
@@ -299,523 +227,740 @@ __host__ __device__ __forceinline__ int bits_of(int qt) {
 }
 // Chunks (16 bytes of codes) per row of K inputs.
 __host__ __device__ __forceinline__ int chunks_per_row(int qt, int K) { return K * bits_of(qt) / 128; }
-// Bytes of group scales (and of mins) per row; 0 for int8 (scale per row,
-// read from global memory at use).
 __host__ __device__ __forceinline__ int scale_row_bytes(int qt, int K) {
-  return qt == MOE_Q_INT4_SYM_G32 ? K / 16 : qt == MOE_Q_INT2_ASYM_G16 ? K / 8 : 0;
+  return qt == MOE_Q_INT4_SYM_G32 ? K / 16 : qt == MOE_Q_INT2_ASYM_G16 ? K / 8 : 2;
 }
 
-// ---------------------------------------------------------------- staging ring
-// Every warp owns kSlots shared-memory slots filled by 1-D bulk (TMA) copies
-// that complete on one mbarrier per slot. Lane 0 issues, all lanes wait.
-constexpr int kSlots = 4;
-constexpr int kSlotBytes = 4608;
+// ---------------------------------------------------------------- lane-private staging ring
+// Each lane copies (cp.async, 16/8/4 bytes) exactly the chunks of the rows it
+// will itself consume into its own slots of shared memory, so no cross-lane
+// synchronisation is needed: cp.async.wait_group is the only wait. A warp
+// keeps kSlots batches in flight; one batch is at most 8 chunks of codes per
+// lane (4 KiB per warp) plus their scales and mins.
+constexpr int kSlots = 3;
+constexpr int kSlotCodeBytes = 4096;  // 8 items x 32 lanes x 16 B
+constexpr int kSlotAuxBytes = 2048;   // 8 aux words x 32 lanes x 8 B
+constexpr int kSlotBytes = kSlotCodeBytes + kSlotAuxBytes;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
+__device__ __forceinline__ void cp_async16(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
                : "memory");
 }
-
-// Bounded wait for the phase with the given parity. false = gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if (clock64() - t0 > kSpinCycles) return false;
-  }
+__device__ __forceinline__ void cp_async8(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-struct Ring {
-  uint8_t* slots;       // kSlots x kSlotBytes, this warp's
-  uint32_t bar0;        // shared address of this warp's first mbarrier
-  uint32_t parity;      // bit s: parity of the next completion of slot s
-  uint32_t pending;     // bit s: a copy into slot s is in flight
-  __device__ uint32_t bar(int s) const { return bar0 + 8u * s; }
-  __device__ uint8_t* slot(int s) const { return slots + size_t(s) * kSlotBytes; }
+__device__ __forceinline__ uint8_t* code_item(uint8_t* slot, int item, int lane) {
+  return slot + (item * 32 + lane) * 16;
+}
+__device__ __forceinline__ uint8_t* aux_word(uint8_t* slot, int a, int lane) {
+  return slot + kSlotCodeBytes + (a * 32 + lane) * 8;
+}
+
+// Rows per batch for a qtype, chunks per lane and matrices per row (gate+up
+// = 2, down = 1): at most 8 code items per lane, int2 at most 4 (its aux
+// holds 8 scales and 8 mins per item).
+__host__ __device__ constexpr int batch_rows(int qt, int cpl, int m) {
+  return qt == MOE_Q_INT2_ASYM_G16 ? (4 / (m * cpl) > 0 ? 4 / (m * cpl) : 1) : (8 / (m * cpl) > 0 ? 8 / (m * cpl) : 1);
+}
+
+// A batch: rows [row0, row0 + nrow) of M matrices (W0, W1) sharing a qtype.
+struct Batch {
+  const moe_qmatrix* W0;
+  const moe_qmatrix* W1;
+  int qt;
+  int row0, nrow;
+  int dest;  // phase-specific destination (pair index)
 };
 
-// Copy up to 6 (src, bytes) segments into consecutive 16-byte aligned places
-// of slot s. Lane 0 only. Segments with bytes == 0 are skipped.
-struct Seg {
-  const void* src;
-  uint32_t bytes;
-};
-
-__device__ __forceinline__ void ring_issue(Ring& r, int s, const Seg* segs, int nseg) {
-  uint32_t total = 0;
-  for (int i = 0; i < nseg; ++i) total += segs[i].bytes;
-  if ((threadIdx.x & 31) == 0) {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // earlier generic reads of the slot
-    mbar_expect_tx(r.bar(s), total);
-    uint32_t off = 0;
-    for (int i = 0; i < nseg; ++i) {
-      if (segs[i].bytes) bulk_g2s(smem_u32(r.slot(s)) + off, segs[i].src, segs[i].bytes, r.bar(s));
-      off += segs[i].bytes;
+template <int QT, int CPL, int M>
+__device__ __forceinline__ void issue_batch_t(uint8_t* slot, const Batch& b, int K) {
+  constexpr int R = batch_rows(QT, CPL, M);
+  const int lane = threadIdx.x & 31;
+  const int CPR = chunks_per_row(QT, K);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (r >= b.nrow) continue;
+    const int row = b.row0 + r;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const moe_qmatrix& W = m == 0 ? *b.W0 : *b.W1;
+      const uint8_t* sc = reinterpret_cast<const uint8_t*>(W.scales);
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int c = lane + 32 * j;
+        if (c >= CPR) continue;
+        const int item = (r * M + m) * CPL + j;
+        cp_async16(code_item(slot, item, lane), W.codes + (size_t(row) * CPR + c) * 16);
+        if (QT == MOE_Q_INT4_SYM_G32) {
+          cp_async4(aux_word(slot, item, lane), sc + size_t(row) * (K / 16) + 4 * (c >> 1));
+        } else if (QT == MOE_Q_INT2_ASYM_G16) {
+          cp_async8(aux_word(slot, 2 * item, lane), sc + (size_t(row) * (K / 16) + 4 * c) * 2);
+          cp_async8(aux_word(slot, 2 * item + 1, lane),
+                    reinterpret_cast<const uint8_t*>(W.mins) + (size_t(row) * (K / 16) + 4 * c) * 2);
+        }
+      }
+      if (QT == MOE_Q_INT8_PER_CHANNEL) cp_async4(aux_word(slot, r * M + m, lane), sc + 4 * size_t(row >> 1));
     }
   }
-  r.pending |= 1u << s;
 }
 
-// Wait for slot s (all lanes). false = the bounded wait expired.
-__device__ __forceinline__ bool ring_wait(Ring& r, int s) {
-  const bool ok = mbar_wait(r.bar(s), (r.parity >> s) & 1u);
-  if (ok) {
-    r.parity ^= 1u << s;
-    r.pending &= ~(1u << s);
+// int8 activations in natural order read straight from shared memory (used
+// where keeping them in registers would exhaust the register file).
+template <int CPL>
+struct XPtr {
+  const float* v[CPL];
+  float gsum[CPL][1];
+  __device__ __forceinline__ void load(const float* xs, int CPR) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+      const int c = lane + 32 * j;
+      v[j] = xs + size_t(c < CPR ? c : 0) * 16;
+      gsum[j][0] = 0.f;
+    }
   }
-  return ok;
+};
+
+// Partial dot products (this lane's chunks) of the batch's R x M rows with x.
+template <int QT, int CPL, int M, class X>
+__device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, int K, const X& x, float* v) {
+  constexpr int R = batch_rows(QT, CPL, M);
+  const int lane = threadIdx.x & 31;
+  const int CPR = chunks_per_row(QT, K);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      float acc = 0.f;
+      if (r < b.nrow) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+          const int c = lane + 32 * j;
+          if (c >= CPR) continue;
+          const int item = (r * M + m) * CPL + j;
+          const uint4 raw = *reinterpret_cast<const uint4*>(code_item(slot, item, lane));
+          const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+          if (QT == MOE_Q_INT4_SYM_G32) {
+            float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t lo = wd[w] & 0x0F0F0F0Fu, hi = (wd[w] >> 4) & 0x0F0F0F0Fu;
+              const float* xv = x.v[j] + 8 * w;
+              s2 = ffma2(make_float2(code_f<0>(lo), code_f<1>(lo)), make_float2(xv[0], xv[1]), s2);
+              s2 = ffma2(make_float2(code_f<2>(lo), code_f<3>(lo)), make_float2(xv[2], xv[3]), s2);
+              s2 = ffma2(make_float2(code_f<0>(hi), code_f<1>(hi)), make_float2(xv[4], xv[5]), s2);
+              s2 = ffma2(make_float2(code_f<2>(hi), code_f<3>(hi)), make_float2(xv[6], xv[7]), s2);
+            }
+            const uint32_t sw = *reinterpret_cast<const uint32_t*>(aux_word(slot, item, lane));
+            const float s = f16_to_f32(uint16_t((c & 1) ? (sw >> 16) : (sw & 0xffffu)));
+            // sum (c - 8) x = 256 S - 136 X
+            acc = fmaf(s, fmaf(256.f, s2.x + s2.y, -136.f * x.gsum[j][0]), acc);
+          } else if (QT == MOE_Q_INT2_ASYM_G16) {
+            const uint2 scw = *reinterpret_cast<const uint2*>(aux_word(slot, 2 * item, lane));
+            const uint2 mnw = *reinterpret_cast<const uint2*>(aux_word(slot, 2 * item + 1, lane));
+            const uint32_t sv[4] = {scw.x & 0xffffu, scw.x >> 16, scw.y & 0xffffu, scw.y >> 16};
+            const uint32_t mv[4] = {mnw.x & 0xffffu, mnw.x >> 16, mnw.y & 0xffffu, mnw.y >> 16};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t b0 = wd[w] & 0x03030303u, b1 = (wd[w] >> 2) & 0x03030303u;
+              const uint32_t b2 = (wd[w] >> 4) & 0x03030303u, b3 = (wd[w] >> 6) & 0x03030303u;
+              const float* xv = x.v[j] + 16 * w;
+              float2 s2 = make_float2(0.f, 0.f);
+              s2 = ffma2(make_float2(code_f<0>(b0), code_f<1>(b0)), make_float2(xv[0], xv[1]), s2);
+              s2 = ffma2(make_float2(code_f<2>(b0), code_f<3>(b0)), make_float2(xv[2], xv[3]), s2);
+              s2 = ffma2(make_float2(code_f<0>(b1), code_f<1>(b1)), make_float2(xv[4], xv[5]), s2);
+              s2 = ffma2(make_float2(code_f<2>(b1), code_f<3>(b1)), make_float2(xv[6], xv[7]), s2);
+              s2 = ffma2(make_float2(code_f<0>(b2), code_f<1>(b2)), make_float2(xv[8], xv[9]), s2);
+              s2 = ffma2(make_float2(code_f<2>(b2), code_f<3>(b2)), make_float2(xv[10], xv[11]), s2);
+              s2 = ffma2(make_float2(code_f<0>(b3), code_f<1>(b3)), make_float2(xv[12], xv[13]), s2);
+              s2 = ffma2(make_float2(code_f<2>(b3), code_f<3>(b3)), make_float2(xv[14], xv[15]), s2);
+              const float s = f16_to_f32(uint16_t(sv[w])), mn = f16_to_f32(uint16_t(mv[w]));
+              // sum (c s + m) x = 256 s S + (m - 128 s) X
+              acc = fmaf(256.f * s, s2.x + s2.y, fmaf(mn - 128.f * s, x.gsum[j][w], acc));
+            }
+          } else {
+            float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t u = wd[w] ^ 0x80808080u;  // q + 128 in each byte
+              const float* xv = x.v[j] + 4 * w;
+              float q[4];
+#pragma unroll
+              for (int bb = 0; bb < 4; ++bb)
+                q[bb] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | bb)) - 8388736.0f;  // - (2^23+128)
+              s2 = ffma2(make_float2(q[0], q[1]), make_float2(xv[0], xv[1]), s2);
+              s2 = ffma2(make_float2(q[2], q[3]), make_float2(xv[2], xv[3]), s2);
+            }
+            acc += s2.x + s2.y;
+          }
+        }
+        if (QT == MOE_Q_INT8_PER_CHANNEL) {
+          const uint32_t sw = *reinterpret_cast<const uint32_t*>(aux_word(slot, r * M + m, lane));
+          acc *= f16_to_f32(uint16_t(((b.row0 + r) & 1) ? (sw >> 16) : (sw & 0xffffu)));
+        }
+      }
+      v[r * M + m] = acc;
+    }
+  }
 }
 
-// Segments of one gate/up unit: row `row` of gate and of up (codes, then
-// scales, then mins). Returns the number of segments (0 = unit skipped).
-__device__ __forceinline__ int gate_up_segs(const moe_expert& ex, int H, int row, Seg* segs) {
-  const int qt = ex.gate.qtype;
-  const uint32_t cb = uint32_t(chunks_per_row(qt, H)) * 16u, sb = uint32_t(scale_row_bytes(qt, H));
-  segs[0] = {ex.gate.codes + size_t(row) * cb, cb};
-  segs[1] = {ex.up.codes + size_t(row) * cb, cb};
-  segs[2] = {reinterpret_cast<const uint8_t*>(ex.gate.scales) + size_t(row) * sb, sb};
-  segs[3] = {reinterpret_cast<const uint8_t*>(ex.up.scales) + size_t(row) * sb, sb};
-  const bool mins = qt == MOE_Q_INT2_ASYM_G16;
-  segs[4] = {mins ? reinterpret_cast<const uint8_t*>(ex.gate.mins) + size_t(row) * sb : nullptr, mins ? sb : 0u};
-  segs[5] = {mins ? reinterpret_cast<const uint8_t*>(ex.up.mins) + size_t(row) * sb : nullptr, mins ? sb : 0u};
-  return 6;
+// Butterfly reduce-scatter of V (power of two) per-lane partials: lane l ends
+// with the warp-wide sum of value (l >> (5 - log2 V)). V-1 + log2(32/V)
+// shuffles instead of 5 V.
+template <int V>
+__device__ __forceinline__ float reduce_scatter(float* v) {
+  const int lane = threadIdx.x & 31;
+  int w = 16;
+#pragma unroll
+  for (int cnt = V; cnt > 1; cnt >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < cnt / 2; ++i) {
+      const float send = upper ? v[i] : v[i + cnt / 2];
+      const float keep = upper ? v[i + cnt / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+    w >>= 1;
+  }
+  float r = v[0];
+#pragma unroll
+  for (; w >= 1; w >>= 1) r += __shfl_xor_sync(0xffffffffu, r, w);
+  return r;
 }
 
-// Segments of one down unit: rows [n0, n0 + nr) of matrix m (K = I).
-__device__ __forceinline__ int down_segs(const moe_qmatrix& m, int I, int n0, int nr, Seg* segs) {
-  const int qt = m.qtype;
-  const uint32_t cb = uint32_t(chunks_per_row(qt, I)) * 16u, sb = uint32_t(scale_row_bytes(qt, I));
-  segs[0] = {m.codes + size_t(n0) * cb, cb * nr};
-  segs[1] = {reinterpret_cast<const uint8_t*>(m.scales) + size_t(n0) * sb, sb * nr};
-  const bool mins = qt == MOE_Q_INT2_ASYM_G16;
-  segs[2] = {mins ? reinterpret_cast<const uint8_t*>(m.mins) + size_t(n0) * sb : nullptr, mins ? sb * nr : 0u};
-  return 3;
+template <int V>
+struct Log2;
+template <>
+struct Log2<1> { static constexpr int v = 0; };
+template <>
+struct Log2<2> { static constexpr int v = 1; };
+template <>
+struct Log2<4> { static constexpr int v = 2; };
+template <>
+struct Log2<8> { static constexpr int v = 3; };
+
+// ---------------------------------------------------------------- job lists
+// Gate/up batches of one warp: pairs j in [0, npair) (expert table + ids, or
+// the shared expert), rows [r0, r0 + nr) of each, cut into batches of the
+// expert's batch_rows; this warp owns batches [b0, b1) of that sequence.
+struct GateUpJobs {
+  const moe_expert* experts;
+  const int* ids;  // expert id per pair, or nullptr for the shared expert
+  int npair, r0, nr, H;
+  int dest0;       // destination pair index of pair 0 (h row block)
+  __device__ const moe_expert& ex(int j) const { return ids ? experts[ids[j]] : experts[0]; }
+  __device__ int rows_per_batch(int j) const {
+    const int qt = ex(j).gate.qtype;
+    const int cpl = (chunks_per_row(qt, H) + 31) / 32;
+    return batch_rows(qt, cpl, 2);
+  }
+  __device__ int total() const {
+    int t = 0;
+    for (int j = 0; j < npair; ++j) t += (nr + rows_per_batch(j) - 1) / rows_per_batch(j);
+    return t;
+  }
+  __device__ Batch get(int b) const {
+    for (int j = 0; j < npair; ++j) {
+      const int R = rows_per_batch(j), nb = (nr + R - 1) / R;
+      if (b < nb) {
+        const moe_expert& e = ex(j);
+        return Batch{&e.gate, &e.up, e.gate.qtype, r0 + b * R, min(R, nr - b * R), dest0 + j};
+      }
+      b -= nb;
+    }
+    return Batch{nullptr, nullptr, 0, 0, 0, 0};
+  }
+};
+
+// Down batches: pairs p in [0, npair) (routed pairs then shared rows), rows
+// [n0, n0 + nn) of each pair's down matrix.
+struct DownJobs {
+  const moe_expert* experts;
+  const moe_expert* shared;
+  const int* ids;
+  int nrouted, npair, n0, nn, I;
+  __device__ const moe_qmatrix& mat(int p) const { return p < nrouted ? experts[ids[p]].down : shared->down; }
+  __device__ int rows_per_batch(int p) const {
+    const int qt = mat(p).qtype;
+    const int cpl = (chunks_per_row(qt, I) + 31) / 32;
+    return batch_rows(qt, cpl, 1);
+  }
+  __device__ int total() const {
+    int t = 0;
+    for (int p = 0; p < npair; ++p) t += (nn + rows_per_batch(p) - 1) / rows_per_batch(p);
+    return t;
+  }
+  __device__ Batch get(int b) const {
+    for (int p = 0; p < npair; ++p) {
+      const int R = rows_per_batch(p), nb = (nn + R - 1) / R;
+      if (b < nb) {
+        const moe_qmatrix& m = mat(p);
+        return Batch{&m, nullptr, m.qtype, n0 + b * R, min(R, nn - b * R), p};
+      }
+      b -= nb;
+    }
+    return Batch{nullptr, nullptr, 0, 0, 0, 0};
+  }
+};
+
+// Runtime qtype / chunks-per-lane dispatch of a batch issue. Unsupported
+// combinations issue nothing (the caller checks support up front).
+template <int M>
+__device__ __forceinline__ void issue_any(uint8_t* slot, const Batch& b, int K) {
+  if (b.nrow > 0) {
+    const int cpl = (chunks_per_row(b.qt, K) + 31) / 32;
+    if (b.qt == MOE_Q_INT4_SYM_G32) {
+      if (cpl == 1) issue_batch_t<MOE_Q_INT4_SYM_G32, 1, M>(slot, b, K);
+      else if (cpl == 2) issue_batch_t<MOE_Q_INT4_SYM_G32, 2, M>(slot, b, K);
+    } else if (b.qt == MOE_Q_INT2_ASYM_G16) {
+      if (cpl == 1) issue_batch_t<MOE_Q_INT2_ASYM_G16, 1, M>(slot, b, K);
+    } else if (b.qt == MOE_Q_INT8_PER_CHANNEL) {
+      if (cpl == 1) issue_batch_t<MOE_Q_INT8_PER_CHANNEL, 1, M>(slot, b, K);
+      else if (cpl == 2) issue_batch_t<MOE_Q_INT8_PER_CHANNEL, 2, M>(slot, b, K);
+      else if (cpl <= 4) issue_batch_t<MOE_Q_INT8_PER_CHANNEL, 4, M>(slot, b, K);
+    }
+  }
+  cp_commit();  // one group per batch, empty or not
 }
 
-// Rows of a down matrix that fit one slot.
-__host__ __device__ __forceinline__ int down_rows_per_slot(int qt, int I) {
-  const int per = chunks_per_row(qt, I) * 16 + scale_row_bytes(qt, I) * (qt == MOE_Q_INT2_ASYM_G16 ? 2 : 1);
-  return kSlotBytes / per;
+__device__ __forceinline__ bool qt_supported(int qt, int K) {
+  const int cpl = (chunks_per_row(qt, K) + 31) / 32;
+  if (qt == MOE_Q_INT4_SYM_G32) return cpl <= 2;
+  if (qt == MOE_Q_INT2_ASYM_G16) return cpl <= 1;
+  if (qt == MOE_Q_INT8_PER_CHANNEL) return cpl <= 4;
+  return false;
 }
+// Down matrices (K = I) keep activations in registers: int8 up to 2 chunks per lane.
+__device__ __forceinline__ bool qt_supported_down(int qt, int K) {
+  const int cpl = (chunks_per_row(qt, K) + 31) / 32;
+  return qt == MOE_Q_INT8_PER_CHANNEL ? cpl <= 2 : qt_supported(qt, K);
+}
+
+// Stream this warp's gate/up batches [b, b1) of one qtype through its ring:
+// h[dest * I + row] = silu(W_g x) * (W_u x). xs: the token's activations
+// (shared memory, fp32). Returns the first batch of a different qtype.
+template <int QT, int CPL, class X = XRegs<QT, CPL>>
+__device__ int gate_up_run(uint8_t* ring, const GateUpJobs& J, int b, int b0, int b1, const float* xs, float* h,
+                           int I) {
+  constexpr int R = batch_rows(QT, CPL, 2), V = 2 * R, SH = 5 - Log2<V>::v;
+  const int lane = threadIdx.x & 31;
+  X x;
+  x.load(xs, chunks_per_row(QT, J.H));
+  for (; b < b1; ++b) {
+    const Batch bt = J.get(b);
+    if (bt.qt != QT) break;
+    uint8_t* slot = ring + ((b - b0) % kSlots) * kSlotBytes;
+    cp_wait<kSlots - 1>();
+    float v[V];
+    compute_batch_t<QT, CPL, 2, X>(slot, bt, J.H, x, v);
+    const float sum = reduce_scatter<V>(v);
+    const float u = __shfl_down_sync(0xffffffffu, sum, 32 / V);
+    const int idx = lane >> SH;  // = 2 r + m
+    if ((lane & ((32 / V) - 1)) == 0 && (idx & 1) == 0 && (idx >> 1) < bt.nrow)
+      h[size_t(bt.dest) * I + bt.row0 + (idx >> 1)] = silu_f32(sum) * u;
+    const int nb = b + kSlots;
+    issue_any<2>(slot, nb < b1 ? J.get(nb) : Batch{nullptr, nullptr, 0, 0, 0, 0}, J.H);
+  }
+  return b;
+}
+
+__device__ void gate_up_stream(uint8_t* ring, const GateUpJobs& J, int b0, int b1, const float* xs, float* h, int I,
+                               bool primed) {
+  if (!primed)
+    for (int i = 0; i < kSlots; ++i)
+      issue_any<2>(ring + i * kSlotBytes, b0 + i < b1 ? J.get(b0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, J.H);
+  int b = b0;
+  while (b < b1) {
+    const int qt = J.get(b).qt;
+    const int cpl = (chunks_per_row(qt, J.H) + 31) / 32;
+    int nb = b1;
+    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) nb = gate_up_run<MOE_Q_INT4_SYM_G32, 1>(ring, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) nb = gate_up_run<MOE_Q_INT4_SYM_G32, 2>(ring, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) nb = gate_up_run<MOE_Q_INT2_ASYM_G16, 1>(ring, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 1>(ring, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 2>(ring, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl <= 4)
+      nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 4, XPtr<4>>(ring, J, b, b0, b1, xs, h, I);
+    if (nb == b) {  // unsupported batch: consume its (empty) group and move on
+      cp_wait<kSlots - 1>();
+      const int nx = b + kSlots;
+      issue_any<2>(ring + ((b - b0) % kSlots) * kSlotBytes, nx < b1 ? J.get(nx) : Batch{nullptr, nullptr, 0, 0, 0, 0},
+                   J.H);
+      nb = b + 1;
+    }
+    b = nb;
+  }
+  cp_wait<0>();
+}
+
+// Down batches [b, b1) of one qtype: ys[dest * nn + row - n0] = W_d h_dest.
+template <int QT, int CPL>
+__device__ int down_run(uint8_t* ring, const DownJobs& J, int b, int b0, int b1, const float* h, float* ys) {
+  constexpr int R = batch_rows(QT, CPL, 1), V = R, SH = 5 - Log2<V>::v;
+  const int lane = threadIdx.x & 31;
+  XRegs<QT, CPL> x;
+  int xp = -1;
+  for (; b < b1; ++b) {
+    const Batch bt = J.get(b);
+    if (bt.qt != QT) break;
+    if (bt.dest != xp) {
+      x.template load<true>(h + size_t(bt.dest) * J.I, chunks_per_row(QT, J.I));
+      xp = bt.dest;
+    }
+    uint8_t* slot = ring + ((b - b0) % kSlots) * kSlotBytes;
+    cp_wait<kSlots - 1>();
+    float v[V];
+    compute_batch_t<QT, CPL, 1, XRegs<QT, CPL>>(slot, bt, J.I, x, v);
+    const float sum = reduce_scatter<V>(v);
+    const int r = lane >> SH;
+    if ((lane & ((32 / V) - 1)) == 0 && r < bt.nrow) ys[size_t(bt.dest) * J.nn + (bt.row0 - J.n0) + r] = sum;
+    const int nb = b + kSlots;
+    issue_any<1>(slot, nb < b1 ? J.get(nb) : Batch{nullptr, nullptr, 0, 0, 0, 0}, J.I);
+  }
+  return b;
+}
+
+__device__ void down_stream(uint8_t* ring, const DownJobs& J, int b0, int b1, const float* h, float* ys) {
+  for (int i = 0; i < kSlots; ++i)
+    issue_any<1>(ring + i * kSlotBytes, b0 + i < b1 ? J.get(b0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, J.I);
+  int b = b0;
+  while (b < b1) {
+    const int qt = J.get(b).qt;
+    const int cpl = (chunks_per_row(qt, J.I) + 31) / 32;
+    int nb = b1;
+    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) nb = down_run<MOE_Q_INT4_SYM_G32, 1>(ring, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) nb = down_run<MOE_Q_INT4_SYM_G32, 2>(ring, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) nb = down_run<MOE_Q_INT2_ASYM_G16, 1>(ring, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) nb = down_run<MOE_Q_INT8_PER_CHANNEL, 1>(ring, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) nb = down_run<MOE_Q_INT8_PER_CHANNEL, 2>(ring, J, b, b0, b1, h, ys);
+    if (nb == b) {
+      cp_wait<kSlots - 1>();
+      const int nx = b + kSlots;
+      issue_any<1>(ring + ((b - b0) % kSlots) * kSlotBytes, nx < b1 ? J.get(nx) : Batch{nullptr, nullptr, 0, 0, 0, 0},
+                   J.I);
+      nb = b + 1;
+    }
+    b = nb;
+  }
+  cp_wait<0>();
+}
+
 // ---------------------------------------------------------------- top-k
 __device__ __forceinline__ uint32_t f2key(float f) {
+  if (f != f) f = -CUDART_INF_F;  // NaN loses to every number
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+__device__ __forceinline__ float key2f(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
-// Warp top-k over logits lg[0..E) (smem, E <= 1024): repeated warp-wide
-// argmax (larger value, then lower index) with redux.sync.
-__device__ void warp_topk(const float* lg, int E, int k, int* sidx, float* sw) {
+// Warp selection of the best `k` of n (key, id) candidates, NPL per lane
+// (candidate i at lane i % 32, slot i / 32): larger key first, ties to the
+// lower id. Writes keys and ids of the picks in order.
+template <int NPL>
+__device__ void warp_select(const uint32_t* keys, const int* ids, int n, int k, uint32_t* out_key, int* out_id) {
   const int lane = threadIdx.x & 31;
-  const int nper = (E + 31) / 32;
-  uint32_t key[32];
-  uint32_t avail = 0;
+  uint32_t kk[NPL];
+  int id[NPL];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = 0;
-    if (i < nper && e < E) {
-      float v = lg[e];
-      if (v != v) v = -CUDART_INF_F;
-      key[i] = f2key(v);
-      avail |= 1u << i;
-    }
+  for (int i = 0; i < NPL; ++i) {
+    const int c = lane + 32 * i;
+    kk[i] = c < n ? keys[c] : 0u;
+    id[i] = c < n ? ids[c] : 0x7fffffff;
   }
-  float sel0 = 0.f, denom = 0.f;
   for (int j = 0; j < k; ++j) {
-    uint32_t best = 0;
-    int bi = -1;
+    uint32_t bk = 0u;
+    int bi = 0x7fffffff, bs = -1;
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (((avail >> i) & 1u) && (bi < 0 || key[i] > best)) {
-        best = key[i];
-        bi = i;
+    for (int i = 0; i < NPL; ++i)
+      if (id[i] != 0x7fffffff && (bs < 0 || kk[i] > bk || (kk[i] == bk && id[i] < bi))) {
+        bk = kk[i];
+        bi = id[i];
+        bs = i;
       }
-    const uint32_t wmax = __reduce_max_sync(0xffffffffu, bi >= 0 ? best : 0u);
-    const uint32_t cand = (bi >= 0 && best == wmax) ? uint32_t(lane + 32 * bi) : 0xffffffffu;
-    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
-    if (int(win & 31) == lane) avail &= ~(1u << (win >> 5));
-    // recover the float value of the winning key
-    const uint32_t u = (wmax & 0x80000000u) ? (wmax & 0x7fffffffu) : ~wmax;
-    const float v = __uint_as_float(u);
-    if (j == 0) sel0 = v;
-    const float ev = expf(v - sel0);
-    denom += ev;
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bs >= 0 ? bk : 0u);
+    const uint32_t wi = __reduce_min_sync(0xffffffffu, (bs >= 0 && bk == wk) ? uint32_t(bi) : 0xffffffffu);
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (i == bs && uint32_t(bi) == wi) id[i] = 0x7fffffff;
     if (lane == 0) {
-      sidx[j] = int(win);
-      sw[j] = ev;
+      out_key[j] = wk;
+      out_id[j] = int(wi);
     }
   }
   __syncwarp();
-  for (int j = lane; j < k; j += 32) sw[j] = sw[j] / denom;
-  __syncwarp();
-}
-
-// ---------------------------------------------------------------- unit runners
-// Issue the copy of gate/up unit (expert ex, row) into slot s.
-__device__ __forceinline__ void issue_gate_up(Ring& R, int s, const moe_expert& ex, int H, int row) {
-  Seg segs[6];
-  gate_up_segs(ex, H, row, segs);
-  ring_issue(R, s, segs, 6);
-}
-
-// A warp's list of gate/up units: unit i (0 <= i < n) is row
-// r0 + (q0 + i) % nr of the expert of pair pidx[(q0 + i) / nr]; results go to
-// h[(pair_base + (q0 + i) / nr) * I + row]. expert_of(i) gives the descriptor.
-struct GateUpList {
-  const moe_expert* experts;  // routed table, or the shared descriptor
-  const int* pidx;            // expert id per local pair (nullptr: always experts[0])
-  int q0, n, nr, r0, pair_base;
-  float* h;
-  int H, I;
-  __device__ int pair(int i) const { return (q0 + i) / nr; }
-  __device__ int row(int i) const { return r0 + (q0 + i) % nr; }
-  __device__ const moe_expert& ex(int i) const { return experts[pidx ? pidx[pair(i)] : 0]; }
-};
-
-__device__ __forceinline__ bool unit_ok(const GateUpList& L, int i) { return expert_ok(L.ex(i), L.H, L.I); }
-
-template <int QT, int CPL>
-__device__ int gate_up_run(Ring& R, const GateUpList& L, int i, const float* xs, WsHeader* hdr, bool& failed) {
-  const int CPR = chunks_per_row(QT, L.H);
-  const uint32_t cb = uint32_t(CPR) * 16u, sb = uint32_t(scale_row_bytes(QT, L.H));
-  XRegs<QT, CPL> x;
-  x.load(xs, CPR);
-  for (; i < L.n; ++i) {
-    const moe_expert& ex = L.ex(i);
-    if (ex.gate.qtype != QT) break;
-    const int s = i % kSlots;
-    if (unit_ok(L, i)) {
-      if (!ring_wait(R, s)) {
-        if ((threadIdx.x & 31) == 0) {
-          flag_error(hdr, MOE_ERR_TIMEOUT, 4000000);
-          atomicExch(&hdr->abort, 1);
-        }
-        failed = true;
-        return L.n;
-      }
-      const uint8_t* base = R.slot(s);
-      const int row = L.row(i);
-      const uint16_t* gs = reinterpret_cast<const uint16_t*>(base + 2 * cb);
-      const uint16_t* us = reinterpret_cast<const uint16_t*>(base + 2 * cb + sb);
-      const uint16_t* gm = reinterpret_cast<const uint16_t*>(base + 2 * cb + 2 * sb);
-      const uint16_t* um = reinterpret_cast<const uint16_t*>(base + 2 * cb + 3 * sb);
-      float g = warp_sum(row_dot<QT, CPL>(base, gs, gm, CPR, x));
-      float u = warp_sum(row_dot<QT, CPL>(base + cb, us, um, CPR, x));
-      if (QT == MOE_Q_INT8_PER_CHANNEL) {
-        g *= f16_to_f32(ex.gate.scales[row]);
-        u *= f16_to_f32(ex.up.scales[row]);
-      }
-      if ((threadIdx.x & 31) == 0) L.h[size_t(L.pair_base + L.pair(i)) * L.I + row] = silu_f32(g) * u;
-      __syncwarp();
-    } else if ((threadIdx.x & 31) == 0) {
-      flag_error(hdr, MOE_ERR_DEVICE_FAULT, 1000000 + L.pair(i));
-    }
-    const int nx = i + kSlots;
-    if (nx < L.n && unit_ok(L, nx)) issue_gate_up(R, s, L.ex(nx), L.H, L.row(nx));
-  }
-  return i;
-}
-
-__device__ void gate_up_prime(Ring& R, const GateUpList& L) {
-  for (int i = 0; i < L.n && i < kSlots; ++i)
-    if (unit_ok(L, i)) issue_gate_up(R, i % kSlots, L.ex(i), L.H, L.row(i));
-}
-
-// Consume a primed list (units stream through the ring, kSlots ahead).
-__device__ void gate_up_consume(Ring& R, const GateUpList& L, const float* xs, WsHeader* hdr, bool& failed) {
-  int i = 0;
-  while (i < L.n && !failed) {
-    const int qt = L.ex(i).gate.qtype;
-    const int cpl = (chunks_per_row(qt, L.H) + 31) / 32;
-    int j = L.n;
-    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) j = gate_up_run<MOE_Q_INT4_SYM_G32, 1>(R, L, i, xs, hdr, failed);
-    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) j = gate_up_run<MOE_Q_INT4_SYM_G32, 2>(R, L, i, xs, hdr, failed);
-    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) j = gate_up_run<MOE_Q_INT2_ASYM_G16, 1>(R, L, i, xs, hdr, failed);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) j = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 1>(R, L, i, xs, hdr, failed);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) j = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 2>(R, L, i, xs, hdr, failed);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl <= 4) j = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 4>(R, L, i, xs, hdr, failed);
-    else {
-      // Malformed or unsupported: the descriptor check flags it; drain the unit.
-      if ((threadIdx.x & 31) == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 5000000 + qt);
-      const int s = i % kSlots;
-      if ((R.pending >> s) & 1u) ring_wait(R, s);
-      const int nx = i + kSlots;
-      if (nx < L.n && unit_ok(L, nx)) issue_gate_up(R, s, L.ex(nx), L.H, L.row(nx));
-      j = i + 1;
-    }
-    i = j;
-  }
-}
-
-// Down units of one warp: unit i covers pair p = (u0 + i) / nsub, rows
-// n0 + sub*rpu .. (clipped to n1), sub = (u0 + i) % nsub.
-struct DownList {
-  const moe_expert* experts;
-  const moe_expert* shared;
-  const int* pidx;  // expert ids of the routed pairs
-  int nrouted;      // pairs < nrouted are routed, the rest shared (token p - nrouted)
-  int u0, n, nsub, rpu, n0, n1, nn;
-  const float* h;   // [npairs][I] (global, written by other CTAs)
-  float* ys;        // [npairs][nn] (shared)
-  int H, I;
-  __device__ int pair(int i) const { return (u0 + i) / nsub; }
-  __device__ int rlo(int i) const { return n0 + ((u0 + i) % nsub) * rpu; }
-  __device__ int rhi(int i) const { return min(n1, rlo(i) + rpu); }
-  __device__ const moe_qmatrix& mat(int i) const {
-    const int p = pair(i);
-    return p < nrouted ? experts[pidx[p]].down : shared->down;
-  }
-};
-
-__device__ __forceinline__ void issue_down(Ring& R, int s, const DownList& L, int i) {
-  Seg segs[3];
-  down_segs(L.mat(i), L.I, L.rlo(i), L.rhi(i) - L.rlo(i), segs);
-  ring_issue(R, s, segs, 3);
-}
-
-template <int QT, int CPL>
-__device__ int down_run(Ring& R, const DownList& L, int i, WsHeader* hdr, bool& failed) {
-  const int CPR = chunks_per_row(QT, L.I);
-  const uint32_t cb = uint32_t(CPR) * 16u, sb = uint32_t(scale_row_bytes(QT, L.I));
-  XRegs<QT, CPL> x;
-  int xp = -1;
-  for (; i < L.n; ++i) {
-    const moe_qmatrix& m = L.mat(i);
-    if (m.qtype != QT) break;
-    const int s = i % kSlots;
-    const int p = L.pair(i);
-    if (qmatrix_ok(m, L.H, L.I)) {
-      if (p != xp) {
-        x.template load<true>(L.h + size_t(p) * L.I, CPR);
-        xp = p;
-      }
-      if (!ring_wait(R, s)) {
-        if ((threadIdx.x & 31) == 0) {
-          flag_error(hdr, MOE_ERR_TIMEOUT, 4000001);
-          atomicExch(&hdr->abort, 1);
-        }
-        failed = true;
-        return L.n;
-      }
-      const uint8_t* base = R.slot(s);
-      const int lo = L.rlo(i), hi = L.rhi(i), nr = hi - lo;
-      const uint16_t* sc = reinterpret_cast<const uint16_t*>(base + nr * cb);
-      const uint16_t* mn = reinterpret_cast<const uint16_t*>(base + nr * cb + nr * sb);
-      for (int r = 0; r < nr; ++r) {
-        float y = warp_sum(row_dot<QT, CPL>(base + r * cb, sc + r * (sb / 2), mn + r * (sb / 2), CPR, x));
-        if (QT == MOE_Q_INT8_PER_CHANNEL) y *= f16_to_f32(m.scales[lo + r]);
-        if ((threadIdx.x & 31) == 0) L.ys[size_t(p) * L.nn + (lo - L.n0) + r] = y;
-      }
-      __syncwarp();
-    }
-    const int nx = i + kSlots;
-    if (nx < L.n && qmatrix_ok(L.mat(nx), L.H, L.I)) issue_down(R, s, L, nx);
-  }
-  return i;
-}
-
-__device__ void down_list(Ring& R, const DownList& L, WsHeader* hdr, bool& failed) {
-  if (L.n <= 0) return;
-  for (int i = 0; i < L.n && i < kSlots; ++i)
-    if (qmatrix_ok(L.mat(i), L.H, L.I)) issue_down(R, i % kSlots, L, i);
-  int i = 0;
-  while (i < L.n && !failed) {
-    const int qt = L.mat(i).qtype;
-    const int cpl = (chunks_per_row(qt, L.I) + 31) / 32;
-    int j;
-    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) j = down_run<MOE_Q_INT4_SYM_G32, 1>(R, L, i, hdr, failed);
-    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) j = down_run<MOE_Q_INT4_SYM_G32, 2>(R, L, i, hdr, failed);
-    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) j = down_run<MOE_Q_INT2_ASYM_G16, 1>(R, L, i, hdr, failed);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) j = down_run<MOE_Q_INT8_PER_CHANNEL, 1>(R, L, i, hdr, failed);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) j = down_run<MOE_Q_INT8_PER_CHANNEL, 2>(R, L, i, hdr, failed);
-    else {
-      const int s = i % kSlots;
-      if ((R.pending >> s) & 1u) ring_wait(R, s);
-      const int nx = i + kSlots;
-      if (nx < L.n && qmatrix_ok(L.mat(nx), L.H, L.I)) issue_down(R, s, L, nx);
-      j = i + 1;
-    }
-    i = j;
-  }
 }
 
 // ---------------------------------------------------------------- kernel
+
+struct Smem {
+  // carved from dynamic shared memory
+  uint8_t* ring;  // kWarps x kSlots x kSlotBytes
+  float* xs;      // [T][H]
+  float* lg;      // [T][E]
+  uint32_t* ck;   // [T][kWarps][k] candidate keys
+  int* ci;        // [T][kWarps][k] candidate ids
+  float* ys;      // [npairs][nn_max]
+};
+
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(8) uint64_t bars[kWarps * kSlots];
   __shared__ int s_idx[kMaxT * kMaxK];
   __shared__ float s_w[kMaxT * kMaxK];
+  __shared__ uint32_t s_key[kMaxT * kMaxK];
   const int T = P.T, H = P.H, I = P.I, E = P.E, k = P.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, b = blockIdx.x;
   const bool has_shared = P.shared != nullptr;
   WsHeader* hdr = P.hdr;
-  bool failed = false;
 
-  uint8_t* ring_base = smem;                                      // kWarps x kSlots x kSlotBytes
-  float* xs = reinterpret_cast<float*>(smem + kWarps * kSlots * kSlotBytes);  // [T][H]
-  float* lg = xs + T * H;                                         // [T][E] (phase B), ys (phase C)
+  int n0, n1;
+  split_range(H, G, b, n0, n1);
+  const int nn = n1 - n0;
+  const int nn_max = (H + G - 1) / G;
+  Smem S;
+  S.ring = smem;
+  S.xs = reinterpret_cast<float*>(smem + size_t(kWarps) * kSlots * kSlotBytes);
+  S.lg = S.xs + size_t(T) * H;
+  S.ck = reinterpret_cast<uint32_t*>(S.lg + size_t(T) * E);
+  S.ci = reinterpret_cast<int*>(S.ck + size_t(T) * kWarps * k);
+  S.ys = reinterpret_cast<float*>(S.ci + size_t(T) * kWarps * k);
+  uint8_t* ring = S.ring + size_t(warp) * kSlots * kSlotBytes;
 
-  Ring R;
-  R.slots = ring_base + size_t(warp) * kSlots * kSlotBytes;
-  R.bar0 = smem_u32(&bars[warp * kSlots]);
-  R.parity = 0;
-  R.pending = 0;
-  if (lane == 0)
-    for (int s = 0; s < kSlots; ++s) mbar_init(R.bar(s));
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  for (int i = threadIdx.x; i < T * H; i += kThreads) xs[i] = bf16_to_f32(P.x[i]);
-  bool shared_ok = false;
-  if (has_shared) {
-    shared_ok = expert_ok(*P.shared, H, I);
-    if (!shared_ok && b == 0 && threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
-  }
-  __syncthreads();
-
-  // Warps are pinned to tokens (warp w serves token w % T): the activation
-  // registers are loaded once per phase.
+  // Warps are pinned to tokens (warp w serves token w % T) for gate/up, so the
+  // activation registers are loaded once per phase.
   const int my_t = warp % T;
   const int grp = warp / T, ngrp = (kWarps - my_t + T - 1) / T;
 
   // ------------------------------------------------ phase A
-  {
-    // Shared expert gate/up of this CTA's intermediate rows (through the ring).
-    GateUpList L{};
-    if (shared_ok) {
-      int r0, r1;
-      split_range(I, G, b, r0, r1);
-      const int nr = r1 - r0;
-      int q0, q1;
-      split_range(nr, ngrp, grp, q0, q1);
-      L = GateUpList{P.shared, nullptr, q0, q1 - q0, nr > 0 ? nr : 1, r0, T * k + my_t, P.h, H, I};
-      gate_up_prime(R, L);  // the copies overlap the router below
+  // 1) issue this warp's router loads (registers) and shared gate/up copies
+  //    before waiting for anything.
+  int u0, u1;
+  split_range(E * kRQ, G, b, u0, u1);
+  const int qlen = H / kRQ;          // floats per router quarter-row
+  const int q4 = qlen / 128;         // float4 per lane per quarter-row (qlen multiple of 128)
+  bool shared_ok = false;
+  GateUpJobs SJ{};
+  int sb0 = 0, sb1 = 0;
+  if (has_shared) {
+    shared_ok = expert_ok(*P.shared, H, I) && qt_supported(P.shared->gate.qtype, H) &&
+                qt_supported_down(P.shared->down.qtype, I);
+    if (!shared_ok && b == 0 && threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
+  }
+  if (shared_ok) {
+    int r0, r1;
+    split_range(I, G, b, r0, r1);
+    SJ = GateUpJobs{P.shared, nullptr, 1, r0, r1 - r0, H, T * k + my_t};
+    const int nb = SJ.total();
+    split_range(nb, ngrp, grp, sb0, sb1);
+    for (int i = 0; i < kSlots; ++i)
+      issue_any<2>(ring + i * kSlotBytes, sb0 + i < sb1 ? SJ.get(sb0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, H);
+  }
+  for (int i = threadIdx.x; i < T * H; i += kThreads) S.xs[i] = bf16_to_f32(P.x[i]);
+  // Router: this CTA's quarter-rows, two at a time per warp, loads first.
+  float4 wv[2][4];
+  int ucur = u0 + warp;
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const int u = ucur + s * kWarps;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (u < u1 && c < q4) {
+        const float4* wr = reinterpret_cast<const float4*>(P.w_router + size_t(u / kRQ) * H + (u % kRQ) * qlen);
+        wv[s][c] = __ldg(wr + lane + 32 * c);
+      }
     }
-    // Router quarter-rows of this CTA, loaded straight into registers.
-    int u0, u1;
-    split_range(E * kRQ, G, b, u0, u1);
-    const int qlen = H / kRQ;
-    for (int u = u0 + warp; u < u1; u += kWarps) {
+  }
+  __syncthreads();
+  for (; ucur < u1; ucur += 2 * kWarps) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int u = ucur + s * kWarps;
+      if (u >= u1) continue;
       const int e = u / kRQ, q = u % kRQ;
-      const float4* wr = reinterpret_cast<const float4*>(P.w_router + size_t(e) * H + q * qlen);
       float acc[kMaxT] = {0.f, 0.f, 0.f, 0.f};
-      for (int c = lane; c < qlen / 4; c += 32) {
-        const float4 w4 = __ldg(wr + c);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c >= q4) continue;
+        const float4 w4 = wv[s][c];
 #pragma unroll
         for (int t = 0; t < kMaxT; ++t)
           if (t < T) {
-            const float4 x4 = *reinterpret_cast<const float4*>(xs + t * H + q * qlen + 4 * c);
+            const float4 x4 = *reinterpret_cast<const float4*>(S.xs + t * H + q * qlen + 4 * (lane + 32 * c));
             acc[t] = fmaf(w4.x, x4.x, fmaf(w4.y, x4.y, fmaf(w4.z, x4.z, fmaf(w4.w, x4.w, acc[t]))));
           }
       }
 #pragma unroll
       for (int t = 0; t < kMaxT; ++t)
         if (t < T) {
-          const float s = warp_sum(acc[t]);
-          if (lane == 0) P.partial[(size_t(t) * E + e) * kRQ + q] = s;
+          const float sum = warp_sum(acc[t]);
+          if (lane == 0) P.partial[(size_t(t) * E + e) * kRQ + q] = sum;
         }
     }
-    if (shared_ok) gate_up_consume(R, L, xs + my_t * H, hdr, failed);
-    // L2 prefetch of the shared down rows this CTA will use in phase C.
-    if (shared_ok && threadIdx.x == 0) {
-      int n0, n1;
-      split_range(H, G, b, n0, n1);
-      const moe_qmatrix& d = P.shared->down;
-      const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
-      prefetch_l2(d.codes, n0 * rb, n1 * rb);
-      if (sb) prefetch_l2(d.scales, n0 * sb, n1 * sb);
-      if (d.mins) prefetch_l2(d.mins, n0 * sb, n1 * sb);
+    // loads of the next pair of units (rare: more than 16 units per CTA)
+    const int un = ucur + 2 * kWarps;
+    if (un < u1) {
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const int u = un + s * kWarps;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (u < u1 && c < q4) {
+            const float4* wr = reinterpret_cast<const float4*>(P.w_router + size_t(u / kRQ) * H + (u % kRQ) * qlen);
+            wv[s][c] = __ldg(wr + lane + 32 * c);
+          }
+      }
     }
   }
-  if (__syncthreads_or(failed) || !grid_sync(hdr, uint32_t(G))) goto done;
+  // 2) shared expert gate/up, already in flight
+  if (shared_ok) gate_up_stream(ring, SJ, sb0, sb1, S.xs + my_t * H, P.h, I, true);
+  // 3) L2 prefetch of the shared down rows this CTA uses in phase C
+  if (shared_ok && threadIdx.x == 0) {
+    const moe_qmatrix& d = P.shared->down;
+    const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
+    prefetch_l2(d.codes, n0 * rb, n1 * rb);
+    if (d.qtype != MOE_Q_INT8_PER_CHANNEL) prefetch_l2(d.scales, n0 * sb, n1 * sb);
+    if (d.mins) prefetch_l2(d.mins, n0 * sb, n1 * sb);
+  }
+  if (!grid_sync(hdr, uint32_t(G))) goto done;
 
   // ------------------------------------------------ phase B
   {
     for (int i = threadIdx.x; i < T * E; i += kThreads) {
       const int t = i / E, e = i % E;
       const float4 p4 = __ldcg(reinterpret_cast<const float4*>(P.partial + size_t(i) * kRQ));
-      lg[i] = ((p4.x + p4.y) + (p4.z + p4.w)) + (P.bias ? P.bias[t * P.bstride + e] : 0.f);
+      S.lg[i] = ((p4.x + p4.y) + (p4.z + p4.w)) + (P.bias ? P.bias[t * P.bstride + e] : 0.f);
     }
     __syncthreads();
-    if (warp < T) warp_topk(lg + warp * E, E, k, s_idx + warp * k, s_w + warp * k);
+    // Top-k, stage 1: warp w selects the best k of its slice of the experts.
+    const int chunk = (E + kWarps - 1) / kWarps;  // <= 128
+    for (int t = 0; t < T; ++t) {
+      const int e0 = min(E, warp * chunk), e1 = min(E, e0 + chunk);
+      const int n = e1 - e0, kk = min(k, n);
+      uint32_t* ck = S.ck + (size_t(t) * kWarps + warp) * k;
+      int* ci = S.ci + (size_t(t) * kWarps + warp) * k;
+      // candidates straight from the logits row
+      uint32_t keys[4];
+      int ids[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        keys[i] = c < n ? f2key(S.lg[size_t(t) * E + e0 + c]) : 0u;
+        ids[i] = c < n ? e0 + c : 0x7fffffff;
+      }
+      // reuse warp_select through a per-lane view: stage the 128 keys in ck/ci
+      // scratch is too small, so select directly here
+      for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u;
+        int bi = 0x7fffffff, bs = -1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (ids[i] != 0x7fffffff && (bs < 0 || keys[i] > bk || (keys[i] == bk && ids[i] < bi))) {
+            bk = keys[i];
+            bi = ids[i];
+            bs = i;
+          }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bs >= 0 ? bk : 0u);
+        const uint32_t wi = __reduce_min_sync(0xffffffffu, (bs >= 0 && bk == wk) ? uint32_t(bi) : 0xffffffffu);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i == bs && uint32_t(bi) == wi) ids[i] = 0x7fffffff;
+        if (lane == 0) {
+          ck[j] = j < kk ? wk : 0u;
+          ci[j] = j < kk ? int(wi) : 0x7fffffff;
+        }
+      }
+    }
+    __syncthreads();
+    // Stage 2: warp t picks the best k of the kWarps * k candidates.
+    if (warp < T) {
+      const int t = warp;
+      const int nc = kWarps * k;
+      if (nc <= 256) warp_select<8>(S.ck + size_t(t) * nc, S.ci + size_t(t) * nc, nc, k, s_key + t * k, s_idx + t * k);
+      else warp_select<16>(S.ck + size_t(t) * nc, S.ci + size_t(t) * nc, nc, k, s_key + t * k, s_idx + t * k);
+      // renormalised softmax over the picks
+      const float v0 = key2f(s_key[t * k]);
+      float part = 0.f;
+      for (int j = lane; j < k; j += 32) part += expf(key2f(s_key[t * k + j]) - v0);
+      const float denom = warp_sum(part);
+      for (int j = lane; j < k; j += 32) s_w[t * k + j] = expf(key2f(s_key[t * k + j]) - v0) / denom;
+    }
     __syncthreads();
     if (b == 0)
       for (int i = threadIdx.x; i < T * k; i += kThreads) {
         P.topk_idx[i] = s_idx[i];
         P.topk_w[i] = s_w[i];
       }
-    // Routed gate/up: this CTA's intermediate rows, this warp's token.
-    int r0, r1;
-    split_range(I, G, b, r0, r1);
-    const int nr = r1 - r0;
-    int q0, q1;
-    split_range(k * nr, ngrp, grp, q0, q1);
-    GateUpList L{P.experts, s_idx + my_t * k, q0, q1 - q0, nr > 0 ? nr : 1, r0, my_t * k, P.h, H, I};
-    gate_up_prime(R, L);
-    gate_up_consume(R, L, xs + my_t * H, hdr, failed);
+    // Routed gate/up of this CTA's intermediate rows, this warp's token.
+    bool bad = false;
+    for (int j = 0; j < k; ++j) {
+      const moe_expert& ex = P.experts[s_idx[my_t * k + j]];
+      if (!expert_ok(ex, H, I) || !qt_supported(ex.gate.qtype, H) || !qt_supported_down(ex.down.qtype, I)) bad = true;
+    }
+    if (bad) {
+      if (lane == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 1000000);
+    } else {
+      int r0, r1;
+      split_range(I, G, b, r0, r1);
+      GateUpJobs RJ{P.experts, s_idx + my_t * k, k, r0, r1 - r0, H, my_t * k};
+      int b0, b1;
+      split_range(RJ.total(), ngrp, grp, b0, b1);
+      gate_up_stream(ring, RJ, b0, b1, S.xs + my_t * H, P.h, I, false);
+    }
     // L2 prefetch of the routed down rows this CTA owns in phase C.
-    int n0, n1;
-    split_range(H, G, b, n0, n1);
     for (int p = threadIdx.x; p < T * k; p += kThreads) {
       const moe_qmatrix& d = P.experts[s_idx[p]].down;
       if (!qmatrix_ok(d, H, I)) continue;
       const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
       prefetch_l2(d.codes, n0 * rb, n1 * rb);
-      if (sb) prefetch_l2(d.scales, n0 * sb, n1 * sb);
+      if (d.qtype != MOE_Q_INT8_PER_CHANNEL) prefetch_l2(d.scales, n0 * sb, n1 * sb);
       if (d.mins) prefetch_l2(d.mins, n0 * sb, n1 * sb);
     }
   }
-  if (__syncthreads_or(failed) || !grid_sync(hdr, uint32_t(2 * G))) goto done;
+  if (__syncthreads_or(0) || !grid_sync(hdr, uint32_t(2 * G))) goto done;
 
   // ------------------------------------------------ phase C
   {
-    int n0, n1;
-    split_range(H, G, b, n0, n1);
-    const int nn = n1 - n0;
     const int nrouted = T * k;
     const int npairs = nrouted + (shared_ok ? T : 0);
-    float* ys = lg;  // [npairs][nn]
-    const int rpu = down_rows_per_slot(MOE_Q_INT8_PER_CHANNEL, I);  // fits every qtype
-    const int nsub = (nn + rpu - 1) / rpu;
-    int u0, u1;
-    split_range(npairs * nsub, kWarps, warp, u0, u1);
-    DownList D{P.experts, P.shared, s_idx, nrouted, u0, u1 - u0, nsub, rpu, n0, n1, nn, P.h, ys, H, I};
-    down_list(R, D, hdr, failed);
+    bool bad = false;
+    for (int p = 0; p < nrouted; ++p)
+      if (!qmatrix_ok(P.experts[s_idx[p]].down, H, I) || !qt_supported_down(P.experts[s_idx[p]].down.qtype, I)) bad = true;
+    if (!bad) {
+      DownJobs D{P.experts, P.shared, s_idx, nrouted, npairs, n0, nn, I};
+      int b0, b1;
+      split_range(D.total(), kWarps, warp, b0, b1);
+      down_stream(ring, D, b0, b1, P.h, S.ys);
+    }
     __syncthreads();
     // Gate-weighted sum in slot order plus the shared expert; one rounding.
-    for (int i = threadIdx.x; i < T * nn; i += kThreads) {
-      const int t = i / nn, n = i % nn;
-      float acc = 0.f;
-      for (int j = 0; j < k; ++j) acc = fmaf(s_w[t * k + j], ys[size_t(t * k + j) * nn + n], acc);
-      if (shared_ok) acc += ys[size_t(nrouted + t) * nn + n];
-      P.out[size_t(t) * H + n0 + n] = f32_to_bf16_rn(acc);
-    }
+    if (!bad)
+      for (int i = threadIdx.x; i < T * nn; i += kThreads) {
+        const int t = i / nn, n = i % nn;
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j) acc = fmaf(s_w[t * k + j], S.ys[size_t(t * k + j) * nn + n], acc);
+        if (shared_ok) acc += S.ys[size_t(nrouted + t) * nn + n];
+        P.out[size_t(t) * H + n0 + n] = f32_to_bf16_rn(acc);
+      }
+    (void)nn_max;
   }
 
 done:
-  // Copies still in flight (only after a failure) are waited for, bounded.
-  for (int s = 0; s < kSlots; ++s)
-    if ((R.pending >> s) & 1u) mbar_wait(R.bar(s), (R.parity >> s) & 1u);
   // The last CTA out resets the barrier words for the next launch.
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -836,14 +981,15 @@ done:
 static size_t decode_fused_smem(int T, int H, int I, int E, int k, int grid) {
   const size_t ring = size_t(dec::kWarps) * dec::kSlots * dec::kSlotBytes;
   const int nn = (H + grid - 1) / grid;
-  const size_t lgc = std::max(size_t(T) * E, size_t(T * k + T) * nn);
-  return ring + 4 * (size_t(T) * H + lgc);
+  const size_t floats = size_t(T) * H + size_t(T) * E + size_t(T * k + T) * nn;
+  const size_t cand = 2 * 4 * size_t(T) * dec::kWarps * k;
+  return ring + 4 * floats + cand;
 }
 
 bool decode_fused_eligible(int T, int H, int I, int E, int k) {
   if (T < 1 || T > dec::kMaxT || E > kMaxE || k > kMaxK) return false;
-  if (H > 2048 || I > 2048 || (H % 256) || (I % 256)) return false;
-  if (dec::down_rows_per_slot(MOE_Q_INT8_PER_CHANNEL, I) < 1) return false;
+  if (H > 2048 || I > 1024 || (H % 512) || (I % 256)) return false;
+  if (E > dec::kWarps * 128) return false;
   return decode_fused_smem(T, H, I, E, k, 148) <= 220 * 1024;
 }
 

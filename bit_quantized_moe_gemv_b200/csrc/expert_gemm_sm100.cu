@@ -1,0 +1,636 @@
+// Prefill experts: grouped GEMM on the 5th-generation tensor cores (tcgen05,
+// accumulators in TMEM), dequantising the packed weights to bf16 in shared
+// memory.
+//
+// Prefill pushes many tokens through each expert at once (the telli.sh page
+// "Strata 与 Qwen3.8-Flash-Next：如何在个人电脑上运行 180B 级模型", section
+// "GPU、RAM 和 SSD 各司其职": larger batches, kernels separate from decode), so
+// the expert FFN is a dense contraction per expert:
+//   gate/up:  H_e = silu(X_e Wg_e^T) * (X_e Wu_e^T)     [n_e x I]
+//   down:     Y_e = H_e Wd_e^T                          [n_e x H]
+// over the rows X_e the dispatch grouped for expert e (the shared expert is
+// one more group holding every token).
+//
+// Layout ("swap AB"): the weight rows are the MMA's M side (128 per tile),
+// tokens its N side (up to 128 per tile), so a small expert wastes no M.
+// Activations are stored once, by `gather_rows_kernel`, as 16 KiB tiles of
+// 128 rows x 64 bf16 already in the 128-byte-swizzled K-major shared-memory
+// image, so one 1-D bulk copy loads a B tile. Inside every 8-element group
+// the K order is (0,4,1,5,2,6,3,7): the order in which a byte-free lop3
+// unpacks eight int4 codes of one 32-bit word. Weights (A) are produced by
+// 8 dequant warps straight into the swizzled image in the same K order, so
+// the MMA's sum over K is unchanged. The gate/up epilogue writes H in the
+// same tiled form, which is the down GEMM's B operand.
+//
+// Warp roles (448 threads, one CTA per SM, persistent over the tile list):
+//   warp 0      bulk-copy producer of B tiles, TMEM allocation
+//   warp 1      MMA issuer (one thread)
+//   warps 2-5   epilogue (TMEM -> registers -> global)
+//   warps 6-13  dequant producers of A tiles
+// Every wait is bounded; an expired wait flags MOE_ERR_TIMEOUT, stops the
+// CTA's loops, drains what it issued and frees TMEM.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace gemm {
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int kTileBytes = BN * BK * 2;  // 16 KiB: one A or B tile
+constexpr int kThreads = 14 * 32;
+constexpr int kDqWarps = 8, kDqThreads = kDqWarps * 32;
+constexpr int kPD = 4;  // dequant global-load prefetch depth (k-blocks)
+
+// ---------------------------------------------------------------- plan
+// Row tiles: every group (routed expert e < E, or the shared expert = E) is
+// cut into tiles of at most BN rows. For each tile: group, first row (a
+// dispatched row, or a token for the shared group) and row count.
+struct Plan {
+  int* count;   // [1] number of row tiles
+  int* group;   // [max]
+  int* row0;    // [max]
+  int* nrows;   // [max]
+};
+
+__global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
+                                                    int E, int shared_rows, int max_tiles, Plan plan) {
+  __shared__ int base[kMaxE + 2];
+  __shared__ int wsum[32];
+  const int ngroups = E + (shared_rows > 0 ? 1 : 0);
+  const int g = threadIdx.x;
+  int nt = 0;
+  if (g < ngroups) {
+    const int n = g < E ? counts[g] : shared_rows;
+    nt = (n + BN - 1) / BN;
+  }
+  // block-wide exclusive scan of nt (1024 threads)
+  int incl = nt;
+  const int lane = g & 31, w = g >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  int wb = 0, total = 0;
+  for (int i = 0; i < 32; ++i) {
+    if (i < w) wb += wsum[i];
+    total += wsum[i];
+  }
+  const int excl = wb + incl - nt;
+  if (g < ngroups) base[g] = excl;
+  __syncthreads();
+  if (g < ngroups) {
+    const int n = g < E ? counts[g] : shared_rows;
+    const int r0 = g < E ? offsets[g] : 0;
+    for (int t = 0; t < nt && excl + t < max_tiles; ++t) {
+      plan.group[excl + t] = g;
+      plan.row0[excl + t] = r0 + t * BN;
+      plan.nrows[excl + t] = min(BN, n - t * BN);
+    }
+  }
+  if (g == 0) plan.count[0] = min(total, max_tiles);
+}
+
+// Byte offset of element (row, k) inside a swizzled 128-row x 64-col bf16 tile,
+// with the (0,4,1,5,2,6,3,7) order inside each 8-element group.
+__device__ __forceinline__ uint32_t tile_off(int row, int k) {
+  const int chunk = k >> 3, e = k & 7;
+  const int pos = e < 4 ? 2 * e : 2 * (e - 4) + 1;
+  return uint32_t(row) * 128u + (uint32_t((chunk ^ (row & 7))) << 4) + uint32_t(pos) * 2u;
+}
+
+// ---------------------------------------------------------------- gather
+// One warp per tile row: token row -> 16 KiB swizzled tiles of X (K = H).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x, int H, int k,
+                                                          const int* __restrict__ perm_src, int E, Plan plan,
+                                                          uint8_t* __restrict__ xt) {
+  const int ntiles = plan.count[0];
+  const int KB = H / BK;
+  const int lane = threadIdx.x & 31;
+  for (long long wr = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); wr < (long long)ntiles * BN;
+       wr += (long long)gridDim.x * 8) {
+    const int rt = int(wr / BN), row = int(wr % BN);
+    if (row >= plan.nrows[rt]) continue;
+    const int g = plan.group[rt];
+    const int r = plan.row0[rt] + row;
+    const int tok = g < E ? perm_src[r] / k : r;
+    const uint4* src = reinterpret_cast<const uint4*>(x + size_t(tok) * H);
+    for (int c = lane; c < H / 8; c += 32) {
+      const uint4 v = __ldg(src + c);
+      uint4 o;
+      o.x = __byte_perm(v.x, v.z, 0x5410);
+      o.y = __byte_perm(v.x, v.z, 0x7632);
+      o.z = __byte_perm(v.y, v.w, 0x5410);
+      o.w = __byte_perm(v.y, v.w, 0x7632);
+      const int kb = c >> 3, chunk = c & 7;
+      uint8_t* dst = xt + (size_t(rt) * KB + kb) * kTileBytes + size_t(row) * 128 + ((chunk ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- dequant
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b),
+                             *reinterpret_cast<__nv_bfloat162*>(&c));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf2_splat_from_f16(uint16_t h) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(__half2float(__ushort_as_half(h)));
+  const uint32_t u = *reinterpret_cast<const uint16_t*>(&b);
+  return u | (u << 16);
+}
+
+// Raw data one dequant thread needs for one k-block of one matrix: 32
+// consecutive K elements of one weight row.
+struct RawK {
+  uint4 c0, c1;      // codes (int4: c0; int2: c0.x,c0.y; int8: c0,c1)
+  uint32_t s, m;     // scale(s) / min(s) as fp16 bit patterns
+};
+
+__device__ __forceinline__ void load_raw(const moe_qmatrix& W, int row, int k0, RawK& r) {
+  const int K = W.cols;
+  if (W.qtype == MOE_Q_INT4_SYM_G32) {
+    r.c0 = __ldg(reinterpret_cast<const uint4*>(W.codes + size_t(row) * (K / 2) + k0 / 2));
+    r.s = W.scales[size_t(row) * (K / 32) + k0 / 32];
+  } else if (W.qtype == MOE_Q_INT2_ASYM_G16) {
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(W.codes + size_t(row) * (K / 4) + k0 / 4));
+    r.c0 = make_uint4(c.x, c.y, 0, 0);
+    const size_t gi = size_t(row) * (K / 16) + k0 / 16;
+    r.s = __ldg(reinterpret_cast<const unsigned int*>(W.scales + gi));
+    r.m = __ldg(reinterpret_cast<const unsigned int*>(W.mins + gi));
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(W.codes + size_t(row) * K + k0);
+    r.c0 = __ldg(p);
+    r.c1 = __ldg(p + 1);
+    r.s = W.scales[row];
+  }
+}
+
+// 32 weights -> 4 x 16-byte chunks (bf16, K order 0,4,1,5,2,6,3,7 per 8).
+__device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4]) {
+  if (qtype == MOE_Q_INT4_SYM_G32) {
+    const uint32_t s2 = bf2_splat_from_f16(uint16_t(r.s));
+    const uint32_t w[4] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w};
+    const uint32_t k136 = 0x43084308u;  // bf16x2 (136, 136)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = bf2_mul(bf2_sub(((w[c] >> (4 * j)) & 0x000F000Fu) | 0x43004300u, k136), s2);
+      o[c] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+  } else if (qtype == MOE_Q_INT2_ASYM_G16) {
+    const uint32_t sA = bf2_splat_from_f16(uint16_t(r.s & 0xffffu)), sB = bf2_splat_from_f16(uint16_t(r.s >> 16));
+    const uint32_t mA = bf2_splat_from_f16(uint16_t(r.m & 0xffffu)), mB = bf2_splat_from_f16(uint16_t(r.m >> 16));
+    const uint32_t k128 = 0x43004300u;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t word = c < 2 ? r.c0.x : r.c0.y;
+      const uint32_t t = __byte_perm(word, 0u, (c & 1) ? 0x4342u : 0x4140u);
+      const uint32_t s2 = c < 2 ? sA : sB, m2 = c < 2 ? mA : mB;
+      uint32_t v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] = bf2_fma(bf2_sub(((t >> (2 * j)) & 0x00030003u) | 0x43004300u, k128), s2, m2);
+      o[c] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+  } else {
+    const float s = __half2float(__ushort_as_half(uint16_t(r.s)));
+    const uint32_t w[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t a = w[2 * c] ^ 0x80808080u, b = w[2 * c + 1] ^ 0x80808080u;  // elements 0-3, 4-7
+      float q[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        q[j] = __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7540u | j)) - 8388736.0f;
+        q[4 + j] = __uint_as_float(__byte_perm(b, 0x4B000000u, 0x7540u | j)) - 8388736.0f;
+      }
+      uint32_t v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(q[j] * s, q[4 + j] * s);
+        v[j] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+      o[c] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- GEMM kernel
+struct Args {
+  Plan plan;
+  const moe_expert* experts;  // routed table
+  const moe_expert* shared;   // shared descriptor or nullptr
+  int E;
+  int K;              // reduction length (H for gate/up, I for down)
+  int M;              // weight rows (I for gate/up, H for down)
+  int I, H;
+  const uint8_t* bt;  // B tiles [tiles][K/64][16 KiB]
+  uint8_t* ht;        // gate/up: H tiles out [tiles][I/64][16 KiB]
+  float* y_f32;       // down: fp32 rows out (routed rows), or nullptr
+  uint16_t* y_bf16;   // down: bf16 rows out, or nullptr
+  float* ys_f32;      // down: shared expert rows out (fp32 [T][H])
+  WsHeader* hdr;
+};
+
+template <bool kGateUp>
+struct Cfg {
+  static constexpr int kStages = kGateUp ? 4 : 6;
+  static constexpr int kATiles = kGateUp ? 2 : 1;
+  static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
+  static constexpr int kAccCols = kGateUp ? 256 : 128;  // one accumulator buffer
+  static constexpr int kTmemCols = 2 * kAccCols;
+};
+
+template <bool kGateUp>
+__device__ __forceinline__ const moe_qmatrix& pick(const moe_expert& e, int which) {
+  if (kGateUp) return which == 0 ? e.gate : e.up;
+  return e.down;
+}
+
+// One job = one k-block of one tile: 128 weight rows x 64 K of each A matrix.
+// Thread (row, half) of the 256 dequant threads handles 32 K elements of one
+// row. Global loads run kPD jobs ahead of the dequant.
+template <bool kGateUp>
+struct DqJob {
+  const moe_qmatrix* W[2];
+  int row, k0;
+  bool valid;
+};
+
+template <bool kGateUp>
+__device__ __forceinline__ DqJob<kGateUp> make_job(const Args& a, long long j, int MT, int KB, long long ntiles,
+                                                    int dt) {
+  DqJob<kGateUp> J;
+  const long long t = blockIdx.x + (j / KB) * gridDim.x;
+  J.valid = t < ntiles;
+  J.W[0] = J.W[1] = nullptr;
+  J.row = 0;
+  J.k0 = 0;
+  if (!J.valid) return J;
+  const int rt = int(t / MT), mt = int(t % MT), kb = int(j % KB);
+  const int g = a.plan.group[rt];
+  const moe_expert* ex = g < a.E ? a.experts + g : a.shared;
+  J.W[0] = kGateUp ? &ex->gate : &ex->down;
+  J.W[1] = kGateUp ? &ex->up : nullptr;
+  J.row = mt * BM + ((threadIdx.x - 6 * 32) >> 1);
+  J.k0 = kb * BK + (dt & 1) * 32;
+  return J;
+}
+
+template <bool kGateUp>
+__device__ __forceinline__ void job_load(const Args& a, const DqJob<kGateUp>& J, RawK (&r)[2], int& qt) {
+  qt = 0;
+  if (!J.valid) return;
+#pragma unroll
+  for (int w = 0; w < (kGateUp ? 2 : 1); ++w) {
+    const moe_qmatrix& W = *J.W[w];
+    if (!qmatrix_ok(W, a.M, a.K)) {
+      r[w].c0 = r[w].c1 = make_uint4(0, 0, 0, 0);
+      r[w].s = r[w].m = 0;
+      if ((threadIdx.x & 31) == 0) flag_error(a.hdr, MOE_ERR_DEVICE_FAULT, 7000000);
+      continue;
+    }
+    qt = W.qtype;
+    load_raw(W, J.row, J.k0, r[w]);
+  }
+}
+
+template <bool kGateUp>
+__device__ void dequant_role(const Args& a, uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
+                             volatile int* abort_p, int MT, int KB, long long ntiles) {
+  using C = Cfg<kGateUp>;
+  const int dt = threadIdx.x - 6 * 32;  // 0 .. 255
+  const int row = dt >> 1, half = dt & 1;
+  const long long per_cta = ntiles > blockIdx.x ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const long long njobs = per_cta * KB;
+  RawK raw[kPD][2];
+  int qts[kPD];
+#pragma unroll
+  for (int p = 0; p < kPD; ++p) {
+    qts[p] = 0;
+    if (p < njobs) job_load<kGateUp>(a, make_job<kGateUp>(a, p, MT, KB, ntiles, dt), raw[p], qts[p]);
+  }
+  int s = 0;
+  uint32_t ph = 0;
+  for (long long j0 = 0; j0 < njobs; j0 += kPD) {
+#pragma unroll
+    for (int p = 0; p < kPD; ++p) {
+      const long long j = j0 + p;
+      if (j < njobs && !*abort_p) {
+        if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
+          flag_error(a.hdr, MOE_ERR_TIMEOUT, 6000005);
+          *abort_p = 1;
+        } else {
+#pragma unroll
+          for (int w = 0; w < C::kATiles; ++w) {
+            uint4 o[4];
+            dequant32(qts[p], raw[p][w], o);
+            uint8_t* tile = smem + size_t(s) * C::kStageBytes + size_t(w) * kTileBytes;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int chunk = 4 * half + c;
+              *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = o[c];
+            }
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(ptx::smem_addr(&full_bar[s]));
+        }
+        if (++s == C::kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+        const long long jn = j + kPD;
+        if (jn < njobs) job_load<kGateUp>(a, make_job<kGateUp>(a, jn, MT, KB, ntiles, dt), raw[p], qts[p]);
+      }
+    }
+  }
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
+  using C = Cfg<kGateUp>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages], accf_bar[2], acce_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles_rows = a.plan.count[0];
+  const int MT = a.M / BM, KB = a.K / BK;
+  const long long ntiles = (long long)ntiles_rows * MT;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&full_bar[s]), 1 + kDqWarps);
+      ptx::mbar_init(ptx::smem_addr(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_addr(&accf_bar[b]), 1);
+      ptx::mbar_init(ptx::smem_addr(&acce_bar[b]), 4);
+    }
+    ptx::mbar_init(ptx::smem_addr(&drain_bar), 1);
+    abort_sh = 0;
+    ptx::mbar_init_fence();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_p = &abort_sh;
+
+  auto fail = [&](int where) {
+    flag_error(a.hdr, MOE_ERR_TIMEOUT, where);
+    *abort_p = 1;
+  };
+  auto stage_a = [&](int s, int which) { return smem + size_t(s) * C::kStageBytes + size_t(which) * kTileBytes; };
+  auto stage_b = [&](int s) { return smem + size_t(s) * C::kStageBytes + size_t(C::kATiles) * kTileBytes; };
+
+  if (warp == 0) {
+    // ------------------------------------------------ B producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
+        const int rt = int(t / MT);
+        const int nrows = a.plan.nrows[rt];
+        const uint32_t bytes = uint32_t((nrows + 15) & ~15) * 128u;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
+            fail(6000001);
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(ptx::smem_addr(&full_bar[s]), bytes);
+          ptx::bulk_g2s(ptx::smem_addr(stage_b(s)), a.bt + (size_t(rt) * KB + kb) * kTileBytes, bytes,
+                        ptx::smem_addr(&full_bar[s]));
+          if (++s == C::kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
+        const int rt = int(t / MT);
+        const int nrows = a.plan.nrows[rt];
+        const int N = (nrows + 15) & ~15;
+        const uint32_t idesc = ptx::idesc_bf16(BM, N);
+        const int buf = it & 1;
+        const uint32_t use = uint32_t(it >> 1) & 1u;
+        if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar[buf]), use ^ 1u, abort_p)) {
+          fail(6000002);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d0 = tmem + uint32_t(buf * C::kAccCols);
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!ptx::mbar_wait(ptx::smem_addr(&full_bar[s]), ph, abort_p)) {
+            fail(6000003);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa0 = ptx::smem_addr(stage_a(s, 0));
+          const uint32_t sb = ptx::smem_addr(stage_b(s));
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks) {
+            const uint64_t bdesc = ptx::smem_desc_k128(sb + 32 * ks);
+            const uint32_t acc = (kb | ks) != 0;
+            ptx::mma_bf16(d0, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
+            if (kGateUp) {
+              const uint32_t sa1 = ptx::smem_addr(stage_a(s, 1));
+              ptx::mma_bf16(d0 + 128, ptx::smem_desc_k128(sa1 + 32 * ks), bdesc, idesc, acc);
+            }
+          }
+          ptx::mma_commit(ptx::smem_addr(&empty_bar[s]));
+          if (++s == C::kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_addr(&accf_bar[buf]));
+      }
+      // Drain: wait (bounded) for every MMA this thread issued.
+      ptx::mma_commit(ptx::smem_addr(&drain_bar));
+      ptx::mbar_wait(ptx::smem_addr(&drain_bar), 0, nullptr);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    int it = 0;
+    for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
+      const int rt = int(t / MT), mt = int(t % MT);
+      const int nrows = a.plan.nrows[rt];
+      const int g = a.plan.group[rt];
+      const int row0 = a.plan.row0[rt];
+      const int buf = it & 1;
+      const uint32_t use = uint32_t(it >> 1) & 1u;
+      if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar[buf]), use, abort_p)) {
+        fail(6000004);
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * C::kAccCols);
+      const int m = mt * BM + 32 * q + lane;  // weight row of this thread
+      for (int c0 = 0; c0 < nrows; c0 += 32) {
+        uint32_t v0[32];
+        ptx::tmem_ld32(taddr + uint32_t(c0), v0);
+        if (kGateUp) {
+          uint32_t v1[32];
+          ptx::tmem_ld32(taddr + 128u + uint32_t(c0), v1);
+          ptx::tmem_ld_wait();
+          // h = silu(g) * u -> bf16 into the H tiles (K index m of the down GEMM)
+          uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = c0 + j;
+            if (n < nrows) {
+              const float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]);
+              const __nv_bfloat16 hb = __float2bfloat16_rn(silu_f32(gv) * uv);
+              *reinterpret_cast<__nv_bfloat16*>(base + tile_off(n, m & 63)) = hb;
+            }
+          }
+        } else {
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = c0 + j;
+            if (n < nrows) {
+              const float yv = __uint_as_float(v0[j]);
+              if (g < a.E) {
+                const size_t o = size_t(row0 + n) * a.H + m;
+                if (a.y_f32) a.y_f32[o] = yv;
+                else a.y_bf16[o] = f32_to_bf16_rn(yv);
+              } else {
+                a.ys_f32[size_t(row0 + n) * a.H + m] = yv;
+              }
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&acce_bar[buf]));
+    }
+  } else {
+    // ------------------------------------------------ dequant producers
+    dequant_role<kGateUp>(a, smem, full_bar, empty_bar, abort_p, MT, KB, ntiles);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace gemm
+}  // namespace moe
+
+namespace moe {
+
+// Upper bound on row tiles: every group adds at most one partial tile.
+long long grouped_max_tiles(long long T, int k, int E, bool with_shared) {
+  // at most one partial tile per non-empty group, and at most T k non-empty groups
+  const long long routed = (T * k + gemm::BN - 1) / gemm::BN + (E < T * k ? E : T * k);
+  return routed + (with_shared ? (T + gemm::BN - 1) / gemm::BN + 1 : 0) + 1;
+}
+
+bool grouped_eligible(int H, int I, int E, bool with_shared) {
+  return (H % 128) == 0 && (I % 128) == 0 && H <= 16384 && I <= 16384 && E + (with_shared ? 1 : 0) <= 1024;
+}
+
+size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
+  const long long mt = grouped_max_tiles(T, k, E, with_shared);
+  return align256(16 * size_t(mt) + 16) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
+         align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes);
+}
+
+cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, int E, const int* perm_src,
+                               const int* offsets, const int* counts, const moe_expert* experts,
+                               const moe_expert* shared, float* y_f32, uint16_t* y_bf16, float* ys_f32,
+                               void* scratch, WsHeader* hdr, cudaStream_t st) {
+  using namespace gemm;
+  if (T == 0) return cudaSuccess;
+  const bool with_shared = shared != nullptr;
+  const long long mt = grouped_max_tiles(T, k, E, with_shared);
+  uint8_t* p = static_cast<uint8_t*>(scratch);
+  Plan plan;
+  plan.count = reinterpret_cast<int*>(p);
+  plan.group = plan.count + 4;
+  plan.row0 = plan.group + mt;
+  plan.nrows = plan.row0 + mt;
+  p += align256(16 * size_t(mt) + 16);
+  uint8_t* xt = p;
+  p += align256(size_t(mt) * (H / BK) * kTileBytes);
+  uint8_t* ht = p;
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), plan);
+  gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt);
+  const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + 1024;
+  const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem_gu));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_dn));
+  if (e != cudaSuccess) return e;
+  Args a{};
+  a.plan = plan;
+  a.experts = experts;
+  a.shared = shared;
+  a.E = E;
+  a.I = I;
+  a.H = H;
+  a.hdr = hdr;
+  // gate/up: K = H, M = I; B = gathered X tiles; out = H tiles
+  a.K = H;
+  a.M = I;
+  a.bt = xt;
+  a.ht = ht;
+  grouped_gemm_kernel<true><<<sms, kThreads, smem_gu, st>>>(a);
+  // down: K = I, M = H; B = H tiles; out = rows
+  a.K = I;
+  a.M = H;
+  a.bt = ht;
+  a.ht = nullptr;
+  a.y_f32 = y_f32;
+  a.y_bf16 = y_bf16;
+  a.ys_f32 = ys_f32;
+  grouped_gemm_kernel<false><<<sms, kThreads, smem_dn, st>>>(a);
+  count_launches(4);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -38,6 +38,16 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
                                 const moe_expert* shared, int* topk_idx, float* topk_w, uint16_t* out,
                                 float* partial, float* h, WsHeader* hdr, cudaStream_t st);
 
+// Prefill experts on tcgen05 (expert_gemm_sm100.cu): plan, gather, gate/up
+// GEMM with SwiGLU epilogue, down GEMM. Routed rows go to y_f32 or y_bf16
+// (dispatched order), the shared expert's rows (if any) to ys_f32 [T][H].
+bool grouped_eligible(int H, int I, int E, bool with_shared);
+size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared);
+cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, int E, const int* perm_src,
+                               const int* offsets, const int* counts, const moe_expert* experts,
+                               const moe_expert* shared, float* y_f32, uint16_t* y_bf16, float* ys_f32,
+                               void* scratch, WsHeader* hdr, cudaStream_t st);
+
 // Combine routed rows given as bf16 (y_bf16) or fp32 (y_f32; the other NULL).
 cudaError_t launch_combine(const uint16_t* y_bf16, const float* y_f32, const int* inv_perm, const float* topk_w,
                            int T, int H, int k, const float* shared_y, uint16_t* out, cudaStream_t st);

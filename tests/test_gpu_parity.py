@@ -46,10 +46,17 @@ SMALL = {
                                                   (20, None, wlm.Q_INT8_PER_CHANNEL)),
                                    shared_qtype=wlm.Q_INT8_PER_CHANNEL),
     "fused_int4_T1": wlm.Workload("fused_int4_T1", T=1, H=1024, I=512, E=64, k=6, zipf_s=1.1, seed=8),
-    "fused_int2_T4": wlm.Workload("fused_int2_T4", T=4, H=768, I=512, E=24, k=5, seed=9,
+    "fused_int2_T4": wlm.Workload("fused_int2_T4", T=4, H=1536, I=512, E=24, k=5, seed=9,
                                   routed_qtypes=((0, None, wlm.Q_INT2_ASYM_G16),), shared_qtype=wlm.Q_INT4_SYM_G32),
     "small_mixed": _small_mixed(),
     "k_equals_E": wlm.Workload("k_equals_E", T=5, H=128, I=64, E=16, k=16, seed=4),
+    # batches > 4 tokens with H, I multiples of 128 take the tcgen05 grouped GEMM
+    "tc_int4": wlm.Workload("tc_int4", T=200, H=256, I=256, E=8, k=2, zipf_s=0.5, seed=12),
+    "tc_mixed": wlm.Workload("tc_mixed", T=300, H=512, I=384, E=16, k=4, zipf_s=1.0, uniform_frac=0.1, seed=13,
+                             routed_qtypes=((0, 6, wlm.Q_INT4_SYM_G32), (6, 11, wlm.Q_INT2_ASYM_G16),
+                                            (11, None, wlm.Q_INT8_PER_CHANNEL)),
+                             shared_qtype=wlm.Q_INT8_PER_CHANNEL),
+    "tc_skew": wlm.Workload("tc_skew", T=1000, H=256, I=128, E=64, k=3, zipf_s=2.0, seed=14),
     "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
                               shared_qtype=wlm.Q_INT2_ASYM_G16),
 }
