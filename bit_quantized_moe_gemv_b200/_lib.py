@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 
 # Every symbol include/moe.h declares (checked by the CPU test suite).
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer",
-           "moe_reset_status", "moe_get_status", "moe_launch_count", "moe_status_string")
+           "moe_layer_decode_noalloc", "moe_reset_status", "moe_get_status", "moe_launch_count",
+           "moe_status_string")
 
 
 class QMatrixC(ctypes.Structure):
@@ -54,6 +55,8 @@ def _load():
         "moe_combine": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
         "moe_layer": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
                               c_vp, c_vp, c_sz, c_vp]),
+        "moe_layer_decode_noalloc": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp,
+                                             c_vp, c_vp, c_vp, c_vp, c_vp]),
         "moe_reset_status": (c_i32, [c_vp, c_vp]),
         "moe_get_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32)]),
         "moe_launch_count": (ctypes.c_uint64, []),
@@ -143,6 +146,16 @@ def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_tab
     _check("moe_layer", LIB.moe_layer(_p(x), T, H, I, E, k, _p(w_router), _p(bias), bias_row_stride,
                                       _p(experts_table), _p(shared_table), _p(topk_idx), _p(topk_w), _p(out), _p(ws),
                                       ws.numel(), _stream(stream)))
+
+
+def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx,
+                         topk_w, out, stream=None):
+    """moe_layer_decode_noalloc: the fused decode step without a workspace."""
+    T, H = x.shape
+    _check("moe_layer_decode_noalloc",
+           LIB.moe_layer_decode_noalloc(_p(x), T, H, I, E, k, _p(w_router), _p(bias), bias_row_stride,
+                                        _p(experts_table), _p(shared_table), _p(topk_idx), _p(topk_w), _p(out),
+                                        _stream(stream)))
 
 
 def reset_status(ws, stream=None):

@@ -1,0 +1,85 @@
+// moe_layer_decode_noalloc: the fused decode step with its scratch memory in
+// a file-scope device array, for callers that cannot allocate device memory.
+//
+// Some hosts hand a kernel library only its inputs and outputs and own every
+// allocation themselves (a plugin slot in another runtime, a process under a
+// fixed device-memory budget): such a caller has no way to provide the
+// workspace that moe_layer needs. This entry point needs none. It runs the
+// same kernel as moe_layer's decode path; only the scratch pointers differ.
+//
+// The scratch is kNoAllocBytes of device memory held by every GPU that loads
+// this library until the process exits. Every call shares it, so calls that
+// may overlap on the GPU (different streams, different host threads) race
+// and must be serialised by the caller.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "moe.h"
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace {
+
+// Header (256 B) + router partials (4 T E floats) + intermediate rows
+// ((T k + T) I floats) at the limits T <= 4, E <= 1024, k <= 16, I <= 2048.
+constexpr size_t kNoAllocBytes = 640u * 1024u;
+constexpr int kNoAllocMaxT = 4, kNoAllocMaxE = 1024, kNoAllocMaxK = 16, kNoAllocMaxHI = 2048;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. Host code may
+// not use the symbol itself as a device pointer: cudaGetSymbolAddress gives
+// the address, once per device, with that device current.
+cudaError_t scratch_for_current_device(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E,
+                                               int32_t k, const float* w_router, const float* bias,
+                                               int64_t bias_row_stride, const moe_expert* experts_dev,
+                                               const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w,
+                                               uint16_t* out, void* stream) {
+  if (T < 1 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T > kNoAllocMaxT || E > kNoAllocMaxE || k > kNoAllocMaxK || H > kNoAllocMaxHI || I > kNoAllocMaxHI)
+    return MOE_ERR_UNSUPPORTED;
+  if (!moe::decode_fused_eligible(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
+  if (!x || !w_router || !experts_dev || !topk_idx || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  const uintptr_t misalign = (reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router) |
+                              reinterpret_cast<uintptr_t>(out)) & 15u;
+  if (misalign || (reinterpret_cast<uintptr_t>(experts_dev) & 7u)) return MOE_ERR_INVALID_ARG;
+
+  const size_t off_partial = 256;
+  const size_t off_h = moe::align256(off_partial + 16u * size_t(T) * E);
+  const size_t total = off_h + 4u * size_t(T * k + T) * I;
+  if (total > kNoAllocBytes) return MOE_ERR_UNSUPPORTED;
+
+  void* base = nullptr;
+  if (scratch_for_current_device(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The previous call's status and barrier words stay in the array: clear them.
+  if (cudaMemsetAsync(base, 0, sizeof(moe::WsHeader), st) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = moe::launch_decode_fused(
+      x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, out,
+      moe::ws_at<float>(base, off_partial), moe::ws_at<float>(base, off_h), moe::ws_at<moe::WsHeader>(base, 0), st);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

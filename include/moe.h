@@ -184,6 +184,34 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
                      const moe_expert* experts_dev, const moe_expert* shared_dev, int32_t* topk_idx,
                      float* topk_w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * moe_layer_decode_noalloc - moe_layer's fused decode step for callers that
+ * cannot allocate device memory.
+ * No counterpart on the pages: this is an interface variant, not a step of
+ * the method. Some hosts give a kernel library only its inputs and outputs
+ * and own every device allocation themselves (for example a plugin slot in
+ * another runtime, or a process held to a fixed device-memory budget); they
+ * cannot provide the workspace moe_layer needs. This call takes the same
+ * arguments as moe_layer without `ws`/`ws_bytes`, allocates nothing (no
+ * cudaMalloc, no allocating library routine) and keeps its scratch in a
+ * 640 KiB device array inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   Limits: 1 <= T <= 4, E <= 1024, k <= 16, H <= 2048 (a multiple of 512),
+ *   I <= 1024 (a multiple of 256); anything else returns MOE_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ *   All calls share the array: calls that may overlap on the GPU (other
+ *   streams, other host threads) race and must be serialised by the caller.
+ *   Device-side checks still skip bad experts, but their status word lives
+ *   in the shared array and is cleared by the next call; use moe_layer when
+ *   that status is needed.
+ */
+moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k,
+                                    const float* w_router, const float* bias, int64_t bias_row_stride,
+                                    const moe_expert* experts_dev, const moe_expert* shared_dev,
+                                    int32_t* topk_idx, float* topk_w, uint16_t* out, void* stream);
+
 /* Clear the device status word of a workspace (asynchronous on `stream`).
  * Call once on a fresh workspace before its first use. */
 moe_status moe_reset_status(void* ws, void* stream);
