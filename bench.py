@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode1", choices=["decode1"])
+    ap.add_argument("--workload", default="decode1", choices=["decode1", "prefill8k", "prefill32k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the CPU-baseline sample")
     return ap.parse_args()
@@ -262,6 +262,105 @@ def run_ours(args, rank, world, peaks, peak_kind):
     return line, wl, lay, bias
 
 
+def run_prefill(args, rank, world, peaks, peak_kind):
+    """Prefill workload: one step = moe_layer over all T tokens of one layer.
+
+    Weights (1.36 GB) and activations exceed L2, so no flush is needed. The
+    tensor-core roofline is taken on the expert FFN alone (moe_expert_ffn:
+    gather + gate/up GEMM + down GEMM), timed with its own events.
+    """
+    import torch
+
+    from bit_quantized_moe_gemv_b200 import _lib as L
+    from bit_quantized_moe_gemv_b200.device import DeviceExperts, bf16_tensor
+
+    wl = wlm.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lay = wlm.gen_layer(wl)
+    bias, stride = wlm.gen_bias(wl)
+    experts, shared = DeviceExperts(lay.experts), DeviceExperts([lay.shared])
+    w_r = torch.from_numpy(lay.w_router).to(dev)
+    b = torch.from_numpy(np.ascontiguousarray(bias)).to(dev)
+    xh = wlm.gen_x(wl, step=rank)
+    x = bf16_tensor(xh)
+    T, k, E, H, I = wl.T, wl.k, wl.E, wl.H, wl.I
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    gw = torch.empty((T, k), dtype=torch.float32, device=dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    ws = L.new_workspace(T, H, I, E, k, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        L.layer(x, I, E, k, w_r, b, stride, experts.table, shared.table, idx, gw, out, ws, stream=stream)
+
+    def timed(fn, n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, z in evs:
+            a.record(stream)
+            fn()
+            z.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(z) for a, z in evs]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    launches0 = L.launch_count()
+    times = timed(step, args.steps)
+    launches = L.launch_count() - launches0
+    clk = clocks.stop() if clocks else None
+    assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
+    total_ms = float(np.sum(times))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * T * args.steps / (total_ms / 1e3)
+
+    # expert FFN alone (routed experts), on the routing of the last step
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    L.dispatch(idx, E, counts, offsets, perm, inv, ws, stream=stream)
+    y = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    ffn = lambda: L.expert_ffn(x, I, k, E, perm, offsets, counts, experts.table, y, ws, stream=stream)  # noqa: E731
+    ffn()
+    ffn_ms = float(np.mean(timed(ffn, max(3, min(args.steps, 10)))))
+    flops = 2.0 * 3 * H * I * T * k
+    achieved = flops / (ffn_ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+
+    # e2e: host tokens in, host output back
+    xin = torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).pin_memory()
+    xout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        x.copy_(xin, non_blocking=True)
+        step()
+        xout.copy_(out, non_blocking=True)
+
+    e2e_ms = float(np.sum(timed(e2e_step, args.steps)))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random weights of the stated architecture)",
+        "config": {"workload": f"{wl.name}: T={T}, H={H}, I={I}, E={E}+1 shared, k={k}, Zipf({wl.zipf_s})",
+                   "global_batch": T * world, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (1.36 GB of expert weights)"},
+        "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (gather + tcgen05 gate/up + down)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops, "ms_per_launch": ffn_ms,
+                     "traffic": None},
+        "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(T * H * 2), "d2h_bytes_per_step": int(T * H * 2)},
+        "gpu_launches": int(launches), "clocks": clk,
+    }
+    return line, wl, lay, bias
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -300,8 +399,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     else:
         torch.cuda.set_device(0)
-    line, wl, lay, bias = run_ours(args, rank, world, peaks, peak_kind)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.workload.startswith("prefill"):
+        line, wl, lay, bias = run_prefill(args, rank, world, peaks, peak_kind)
+    else:
+        line, wl, lay, bias = run_ours(args, rank, world, peaks, peak_kind)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.workload.startswith("prefill"):
         tokens, secs, steps = time_oracle(wl, lay, bias, 10 ** 6, args.cpu_seconds, step_offset=10 ** 5)
         line["cpu_baseline"] = {"value": tokens / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": f"{steps} decode steps of 1 token through the fp64 oracle "

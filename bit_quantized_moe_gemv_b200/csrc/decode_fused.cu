@@ -291,11 +291,11 @@ __device__ __forceinline__ void issue_batch_t(uint8_t* slot, const Batch& b, int
   constexpr int R = batch_rows(QT, CPL, M);
   const int lane = threadIdx.x & 31;
   const int CPR = chunks_per_row(QT, K);
-#pragma unroll
+#pragma unroll 1
   for (int r = 0; r < R; ++r) {
     if (r >= b.nrow) continue;
     const int row = b.row0 + r;
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < M; ++m) {
       const moe_qmatrix& W = m == 0 ? *b.W0 : *b.W1;
       const uint8_t* sc = reinterpret_cast<const uint8_t*>(W.scales);
@@ -336,14 +336,17 @@ struct XPtr {
 };
 
 // Partial dot products (this lane's chunks) of the batch's R x M rows with x.
+// The partial of item (r, m) goes to red[(r M + m) * 32 + lane] (this warp's
+// shared scratch); the item loop is kept rolled so the executed code stays
+// small (this kernel is latency-bound and runs each code path once per step).
 template <int QT, int CPL, int M, class X>
-__device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, int K, const X& x, float* v) {
+__device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, int K, const X& x, float* red) {
   constexpr int R = batch_rows(QT, CPL, M);
   const int lane = threadIdx.x & 31;
   const int CPR = chunks_per_row(QT, K);
-#pragma unroll
+#pragma unroll 1
   for (int r = 0; r < R; ++r) {
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < M; ++m) {
       float acc = 0.f;
       if (r < b.nrow) {
@@ -355,16 +358,19 @@ __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, i
           const uint4 raw = *reinterpret_cast<const uint4*>(code_item(slot, item, lane));
           const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
           if (QT == MOE_Q_INT4_SYM_G32) {
-            float2 s2 = make_float2(0.f, 0.f);
+            // one accumulator per 32-bit word: four independent FMA chains
+            float2 a4[4];
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               const uint32_t lo = wd[w] & 0x0F0F0F0Fu, hi = (wd[w] >> 4) & 0x0F0F0F0Fu;
               const float* xv = x.v[j] + 8 * w;
-              s2 = ffma2(make_float2(code_f<0>(lo), code_f<1>(lo)), make_float2(xv[0], xv[1]), s2);
-              s2 = ffma2(make_float2(code_f<2>(lo), code_f<3>(lo)), make_float2(xv[2], xv[3]), s2);
-              s2 = ffma2(make_float2(code_f<0>(hi), code_f<1>(hi)), make_float2(xv[4], xv[5]), s2);
-              s2 = ffma2(make_float2(code_f<2>(hi), code_f<3>(hi)), make_float2(xv[6], xv[7]), s2);
+              float2 t2 = make_float2(code_f<0>(lo) * xv[0], code_f<1>(lo) * xv[1]);
+              t2 = ffma2(make_float2(code_f<2>(lo), code_f<3>(lo)), make_float2(xv[2], xv[3]), t2);
+              t2 = ffma2(make_float2(code_f<0>(hi), code_f<1>(hi)), make_float2(xv[4], xv[5]), t2);
+              a4[w] = ffma2(make_float2(code_f<2>(hi), code_f<3>(hi)), make_float2(xv[6], xv[7]), t2);
             }
+            const float2 s2 = make_float2((a4[0].x + a4[1].x) + (a4[2].x + a4[3].x),
+                                          (a4[0].y + a4[1].y) + (a4[2].y + a4[3].y));
             const uint32_t sw = *reinterpret_cast<const uint32_t*>(aux_word(slot, item, lane));
             const float s = f16_to_f32(uint16_t((c & 1) ? (sw >> 16) : (sw & 0xffffu)));
             // sum (c - 8) x = 256 S - 136 X
@@ -393,7 +399,7 @@ __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, i
               acc = fmaf(256.f * s, s2.x + s2.y, fmaf(mn - 128.f * s, x.gsum[j][w], acc));
             }
           } else {
-            float2 s2 = make_float2(0.f, 0.f);
+            float2 a4[4];
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               const uint32_t u = wd[w] ^ 0x80808080u;  // q + 128 in each byte
@@ -402,10 +408,10 @@ __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, i
 #pragma unroll
               for (int bb = 0; bb < 4; ++bb)
                 q[bb] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | bb)) - 8388736.0f;  // - (2^23+128)
-              s2 = ffma2(make_float2(q[0], q[1]), make_float2(xv[0], xv[1]), s2);
-              s2 = ffma2(make_float2(q[2], q[3]), make_float2(xv[2], xv[3]), s2);
+              a4[w] = ffma2(make_float2(q[2], q[3]), make_float2(xv[2], xv[3]),
+                            make_float2(q[0] * xv[0], q[1] * xv[1]));
             }
-            acc += s2.x + s2.y;
+            acc += ((a4[0].x + a4[1].x) + (a4[2].x + a4[3].x)) + ((a4[0].y + a4[1].y) + (a4[2].y + a4[3].y));
           }
         }
         if (QT == MOE_Q_INT8_PER_CHANNEL) {
@@ -413,9 +419,10 @@ __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, i
           acc *= f16_to_f32(uint16_t(((b.row0 + r) & 1) ? (sw >> 16) : (sw & 0xffffu)));
         }
       }
-      v[r * M + m] = acc;
+      red[(r * M + m) * 32 + lane] = acc;
     }
   }
+  __syncwarp();
 }
 
 // Butterfly reduce-scatter of V (power of two) per-lane partials: lane l ends
@@ -442,6 +449,22 @@ __device__ __forceinline__ float reduce_scatter(float* v) {
   return r;
 }
 
+// Sum the 32 lane partials of each of V outputs held in red[V][32]: lane l
+// ends with the total of output l >> (5 - log2 V). Fixed summation order.
+template <int V>
+__device__ __forceinline__ float reduce_smem(const float* red) {
+  constexpr int G = 32 / V;  // lanes per output
+  const int lane = threadIdx.x & 31;
+  const int o = lane / G, sidx = lane % G;
+  float acc = 0.f;
+#pragma unroll 1
+  for (int i = 0; i < V; ++i) acc += red[o * 32 + sidx * V + i];
+#pragma unroll
+  for (int w = G / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+  __syncwarp();
+  return acc;
+}
+
 template <int V>
 struct Log2;
 template <>
@@ -454,68 +477,53 @@ template <>
 struct Log2<8> { static constexpr int v = 3; };
 
 // ---------------------------------------------------------------- job lists
-// Gate/up batches of one warp: pairs j in [0, npair) (expert table + ids, or
-// the shared expert), rows [r0, r0 + nr) of each, cut into batches of the
-// expert's batch_rows; this warp owns batches [b0, b1) of that sequence.
+// The descriptors a step uses are copied into shared memory once, with a
+// per-pair table of rows per batch and a prefix over the pairs' batch counts,
+// so mapping a batch index to its rows never touches global memory.
+//
+// Gate/up batches: pairs j in [0, npair) with descriptors desc[j], rows
+// [r0, r0 + nr) of each, cut into batches of rpb[j] rows; pre[j] = first
+// batch of pair j (pre[npair] = total).
 struct GateUpJobs {
-  const moe_expert* experts;
-  const int* ids;  // expert id per pair, or nullptr for the shared expert
+  const moe_expert* desc;
+  const int* pre;
+  const int* rpb;
   int npair, r0, nr, H;
-  int dest0;       // destination pair index of pair 0 (h row block)
-  __device__ const moe_expert& ex(int j) const { return ids ? experts[ids[j]] : experts[0]; }
-  __device__ int rows_per_batch(int j) const {
-    const int qt = ex(j).gate.qtype;
-    const int cpl = (chunks_per_row(qt, H) + 31) / 32;
-    return batch_rows(qt, cpl, 2);
-  }
-  __device__ int total() const {
-    int t = 0;
-    for (int j = 0; j < npair; ++j) t += (nr + rows_per_batch(j) - 1) / rows_per_batch(j);
-    return t;
-  }
+  int dest0;  // h row block of pair 0
+  __device__ int total() const { return pre[npair]; }
   __device__ Batch get(int b) const {
-    for (int j = 0; j < npair; ++j) {
-      const int R = rows_per_batch(j), nb = (nr + R - 1) / R;
-      if (b < nb) {
-        const moe_expert& e = ex(j);
-        return Batch{&e.gate, &e.up, e.gate.qtype, r0 + b * R, min(R, nr - b * R), dest0 + j};
-      }
-      b -= nb;
-    }
-    return Batch{nullptr, nullptr, 0, 0, 0, 0};
+    int j = 0;
+    while (j + 1 < npair && pre[j + 1] <= b) ++j;
+    const int R = rpb[j], lb = b - pre[j];
+    const moe_expert& e = desc[j];
+    return Batch{&e.gate, &e.up, e.gate.qtype, r0 + lb * R, min(R, nr - lb * R), dest0 + j};
   }
 };
 
-// Down batches: pairs p in [0, npair) (routed pairs then shared rows), rows
-// [n0, n0 + nn) of each pair's down matrix.
+// Down batches: pairs p in [0, npair) (routed picks, then the shared expert's
+// T rows: desc index min(p, nrouted)), rows [n0, n0 + nn).
 struct DownJobs {
-  const moe_expert* experts;
-  const moe_expert* shared;
-  const int* ids;
+  const moe_expert* desc;
+  const int* pre;
+  const int* rpb;
   int nrouted, npair, n0, nn, I;
-  __device__ const moe_qmatrix& mat(int p) const { return p < nrouted ? experts[ids[p]].down : shared->down; }
-  __device__ int rows_per_batch(int p) const {
-    const int qt = mat(p).qtype;
-    const int cpl = (chunks_per_row(qt, I) + 31) / 32;
-    return batch_rows(qt, cpl, 1);
-  }
-  __device__ int total() const {
-    int t = 0;
-    for (int p = 0; p < npair; ++p) t += (nn + rows_per_batch(p) - 1) / rows_per_batch(p);
-    return t;
-  }
+  __device__ int total() const { return pre[npair]; }
   __device__ Batch get(int b) const {
-    for (int p = 0; p < npair; ++p) {
-      const int R = rows_per_batch(p), nb = (nn + R - 1) / R;
-      if (b < nb) {
-        const moe_qmatrix& m = mat(p);
-        return Batch{&m, nullptr, m.qtype, n0 + b * R, min(R, nn - b * R), p};
-      }
-      b -= nb;
-    }
-    return Batch{nullptr, nullptr, 0, 0, 0, 0};
+    int p = 0;
+    while (p + 1 < npair && pre[p + 1] <= b) ++p;
+    const int R = rpb[p], lb = b - pre[p];
+    const moe_qmatrix& m = desc[p < nrouted ? p : nrouted].down;
+    return Batch{&m, nullptr, m.qtype, n0 + lb * R, min(R, nn - lb * R), p};
   }
 };
+
+__device__ __forceinline__ int gu_rows_per_batch(const moe_expert& e, int H) {
+  const int qt = e.gate.qtype;
+  return batch_rows(qt, (chunks_per_row(qt, H) + 31) / 32, 2);
+}
+__device__ __forceinline__ int dn_rows_per_batch(const moe_qmatrix& m, int I) {
+  return batch_rows(m.qtype, (chunks_per_row(m.qtype, I) + 31) / 32, 1);
+}
 
 // Runtime qtype / chunks-per-lane dispatch of a batch issue. Unsupported
 // combinations issue nothing (the caller checks support up front).
@@ -554,8 +562,8 @@ __device__ __forceinline__ bool qt_supported_down(int qt, int K) {
 // h[dest * I + row] = silu(W_g x) * (W_u x). xs: the token's activations
 // (shared memory, fp32). Returns the first batch of a different qtype.
 template <int QT, int CPL, class X = XRegs<QT, CPL>>
-__device__ int gate_up_run(uint8_t* ring, const GateUpJobs& J, int b, int b0, int b1, const float* xs, float* h,
-                           int I) {
+__device__ __noinline__ int gate_up_run(uint8_t* ring, float* red, const GateUpJobs& J, int b, int b0, int b1,
+                                        const float* xs, float* h, int I) {
   constexpr int R = batch_rows(QT, CPL, 2), V = 2 * R, SH = 5 - Log2<V>::v;
   const int lane = threadIdx.x & 31;
   X x;
@@ -565,9 +573,8 @@ __device__ int gate_up_run(uint8_t* ring, const GateUpJobs& J, int b, int b0, in
     if (bt.qt != QT) break;
     uint8_t* slot = ring + ((b - b0) % kSlots) * kSlotBytes;
     cp_wait<kSlots - 1>();
-    float v[V];
-    compute_batch_t<QT, CPL, 2, X>(slot, bt, J.H, x, v);
-    const float sum = reduce_scatter<V>(v);
+    compute_batch_t<QT, CPL, 2, X>(slot, bt, J.H, x, red);
+    const float sum = reduce_smem<V>(red);
     const float u = __shfl_down_sync(0xffffffffu, sum, 32 / V);
     const int idx = lane >> SH;  // = 2 r + m
     if ((lane & ((32 / V) - 1)) == 0 && (idx & 1) == 0 && (idx >> 1) < bt.nrow)
@@ -578,8 +585,8 @@ __device__ int gate_up_run(uint8_t* ring, const GateUpJobs& J, int b, int b0, in
   return b;
 }
 
-__device__ void gate_up_stream(uint8_t* ring, const GateUpJobs& J, int b0, int b1, const float* xs, float* h, int I,
-                               bool primed) {
+__device__ __noinline__ void gate_up_stream(uint8_t* ring, float* red, const GateUpJobs& J, int b0, int b1,
+                                            const float* xs, float* h, int I, bool primed) {
   if (!primed)
     for (int i = 0; i < kSlots; ++i)
       issue_any<2>(ring + i * kSlotBytes, b0 + i < b1 ? J.get(b0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, J.H);
@@ -588,13 +595,13 @@ __device__ void gate_up_stream(uint8_t* ring, const GateUpJobs& J, int b0, int b
     const int qt = J.get(b).qt;
     const int cpl = (chunks_per_row(qt, J.H) + 31) / 32;
     int nb = b1;
-    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) nb = gate_up_run<MOE_Q_INT4_SYM_G32, 1>(ring, J, b, b0, b1, xs, h, I);
-    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) nb = gate_up_run<MOE_Q_INT4_SYM_G32, 2>(ring, J, b, b0, b1, xs, h, I);
-    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) nb = gate_up_run<MOE_Q_INT2_ASYM_G16, 1>(ring, J, b, b0, b1, xs, h, I);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 1>(ring, J, b, b0, b1, xs, h, I);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 2>(ring, J, b, b0, b1, xs, h, I);
+    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) nb = gate_up_run<MOE_Q_INT4_SYM_G32, 1>(ring, red, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) nb = gate_up_run<MOE_Q_INT4_SYM_G32, 2>(ring, red, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) nb = gate_up_run<MOE_Q_INT2_ASYM_G16, 1>(ring, red, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 1>(ring, red, J, b, b0, b1, xs, h, I);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 2>(ring, red, J, b, b0, b1, xs, h, I);
     else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl <= 4)
-      nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 4, XPtr<4>>(ring, J, b, b0, b1, xs, h, I);
+      nb = gate_up_run<MOE_Q_INT8_PER_CHANNEL, 4, XPtr<4>>(ring, red, J, b, b0, b1, xs, h, I);
     if (nb == b) {  // unsupported batch: consume its (empty) group and move on
       cp_wait<kSlots - 1>();
       const int nx = b + kSlots;
@@ -609,7 +616,8 @@ __device__ void gate_up_stream(uint8_t* ring, const GateUpJobs& J, int b0, int b
 
 // Down batches [b, b1) of one qtype: ys[dest * nn + row - n0] = W_d h_dest.
 template <int QT, int CPL>
-__device__ int down_run(uint8_t* ring, const DownJobs& J, int b, int b0, int b1, const float* h, float* ys) {
+__device__ __noinline__ int down_run(uint8_t* ring, float* red, const DownJobs& J, int b, int b0, int b1,
+                                     const float* h, float* ys) {
   constexpr int R = batch_rows(QT, CPL, 1), V = R, SH = 5 - Log2<V>::v;
   const int lane = threadIdx.x & 31;
   XRegs<QT, CPL> x;
@@ -623,9 +631,8 @@ __device__ int down_run(uint8_t* ring, const DownJobs& J, int b, int b0, int b1,
     }
     uint8_t* slot = ring + ((b - b0) % kSlots) * kSlotBytes;
     cp_wait<kSlots - 1>();
-    float v[V];
-    compute_batch_t<QT, CPL, 1, XRegs<QT, CPL>>(slot, bt, J.I, x, v);
-    const float sum = reduce_scatter<V>(v);
+    compute_batch_t<QT, CPL, 1, XRegs<QT, CPL>>(slot, bt, J.I, x, red);
+    const float sum = reduce_smem<V>(red);
     const int r = lane >> SH;
     if ((lane & ((32 / V) - 1)) == 0 && r < bt.nrow) ys[size_t(bt.dest) * J.nn + (bt.row0 - J.n0) + r] = sum;
     const int nb = b + kSlots;
@@ -634,7 +641,8 @@ __device__ int down_run(uint8_t* ring, const DownJobs& J, int b, int b0, int b1,
   return b;
 }
 
-__device__ void down_stream(uint8_t* ring, const DownJobs& J, int b0, int b1, const float* h, float* ys) {
+__device__ __noinline__ void down_stream(uint8_t* ring, float* red, const DownJobs& J, int b0, int b1, const float* h,
+                                         float* ys) {
   for (int i = 0; i < kSlots; ++i)
     issue_any<1>(ring + i * kSlotBytes, b0 + i < b1 ? J.get(b0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, J.I);
   int b = b0;
@@ -642,11 +650,11 @@ __device__ void down_stream(uint8_t* ring, const DownJobs& J, int b0, int b1, co
     const int qt = J.get(b).qt;
     const int cpl = (chunks_per_row(qt, J.I) + 31) / 32;
     int nb = b1;
-    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) nb = down_run<MOE_Q_INT4_SYM_G32, 1>(ring, J, b, b0, b1, h, ys);
-    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) nb = down_run<MOE_Q_INT4_SYM_G32, 2>(ring, J, b, b0, b1, h, ys);
-    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) nb = down_run<MOE_Q_INT2_ASYM_G16, 1>(ring, J, b, b0, b1, h, ys);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) nb = down_run<MOE_Q_INT8_PER_CHANNEL, 1>(ring, J, b, b0, b1, h, ys);
-    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) nb = down_run<MOE_Q_INT8_PER_CHANNEL, 2>(ring, J, b, b0, b1, h, ys);
+    if (qt == MOE_Q_INT4_SYM_G32 && cpl == 1) nb = down_run<MOE_Q_INT4_SYM_G32, 1>(ring, red, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT4_SYM_G32 && cpl == 2) nb = down_run<MOE_Q_INT4_SYM_G32, 2>(ring, red, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT2_ASYM_G16 && cpl == 1) nb = down_run<MOE_Q_INT2_ASYM_G16, 1>(ring, red, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 1) nb = down_run<MOE_Q_INT8_PER_CHANNEL, 1>(ring, red, J, b, b0, b1, h, ys);
+    else if (qt == MOE_Q_INT8_PER_CHANNEL && cpl == 2) nb = down_run<MOE_Q_INT8_PER_CHANNEL, 2>(ring, red, J, b, b0, b1, h, ys);
     if (nb == b) {
       cp_wait<kSlots - 1>();
       const int nx = b + kSlots;
@@ -716,6 +724,13 @@ struct Smem {
   uint32_t* ck;   // [T][kWarps][k] candidate keys
   int* ci;        // [T][kWarps][k] candidate ids
   float* ys;      // [npairs][nn_max]
+  moe_expert* desc;  // [T k + 1]: the picks' descriptors, then the shared expert's
+  int* gpre;      // [T][k + 1] gate/up batch prefix per token
+  int* grpb;      // [T][k]     gate/up rows per batch
+  int* dpre;      // [T k + T + 1] down batch prefix
+  int* drpb;      // [T k + T]     down rows per batch
+  int* spre;      // [2] shared gate/up prefix
+  int* srpb;      // [1]
 };
 
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
@@ -723,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
   __shared__ int s_idx[kMaxT * kMaxK];
   __shared__ float s_w[kMaxT * kMaxK];
   __shared__ uint32_t s_key[kMaxT * kMaxK];
+  __shared__ float s_red[kWarps][8 * 32];  // per-warp partials of one batch
   const int T = P.T, H = P.H, I = P.I, E = P.E, k = P.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, b = blockIdx.x;
@@ -740,7 +756,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
   S.ck = reinterpret_cast<uint32_t*>(S.lg + size_t(T) * E);
   S.ci = reinterpret_cast<int*>(S.ck + size_t(T) * kWarps * k);
   S.ys = reinterpret_cast<float*>(S.ci + size_t(T) * kWarps * k);
+  {
+    uintptr_t q = reinterpret_cast<uintptr_t>(S.ys + size_t(T * k + T) * nn_max);
+    q = (q + 15) & ~uintptr_t(15);
+    S.desc = reinterpret_cast<moe_expert*>(q);
+    S.gpre = reinterpret_cast<int*>(S.desc + T * k + 1);
+    S.grpb = S.gpre + T * (k + 1);
+    S.dpre = S.grpb + T * k;
+    S.drpb = S.dpre + T * k + T + 1;
+    S.spre = S.drpb + T * k + T;
+    S.srpb = S.spre + 2;
+  }
+  __shared__ int s_bad;
   uint8_t* ring = S.ring + size_t(warp) * kSlots * kSlotBytes;
+  float* red = s_red[warp];
 
   // Warps are pinned to tokens (warp w serves token w % T) for gate/up, so the
   // activation registers are loaded once per phase.
@@ -757,21 +786,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
   bool shared_ok = false;
   GateUpJobs SJ{};
   int sb0 = 0, sb1 = 0;
-  if (has_shared) {
-    shared_ok = expert_ok(*P.shared, H, I) && qt_supported(P.shared->gate.qtype, H) &&
-                qt_supported_down(P.shared->down.qtype, I);
-    if (!shared_ok && b == 0 && threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
+  // The shared expert's descriptor into shared memory; the routed table into
+  // L2 (its rows are read right after the top-k).
+  if (has_shared && threadIdx.x < int(sizeof(moe_expert) / 4))
+    reinterpret_cast<uint32_t*>(S.desc + T * k)[threadIdx.x] = reinterpret_cast<const uint32_t*>(P.shared)[threadIdx.x];
+  if (threadIdx.x == 32) {
+    int e0, e1;
+    split_range(E, G, b, e0, e1);
+    prefetch_l2(P.experts, size_t(e0) * sizeof(moe_expert), size_t(e1) * sizeof(moe_expert));
   }
-  if (shared_ok) {
-    int r0, r1;
-    split_range(I, G, b, r0, r1);
-    SJ = GateUpJobs{P.shared, nullptr, 1, r0, r1 - r0, H, T * k + my_t};
-    const int nb = SJ.total();
-    split_range(nb, ngrp, grp, sb0, sb1);
-    for (int i = 0; i < kSlots; ++i)
-      issue_any<2>(ring + i * kSlotBytes, sb0 + i < sb1 ? SJ.get(sb0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, H);
-  }
-  for (int i = threadIdx.x; i < T * H; i += kThreads) S.xs[i] = bf16_to_f32(P.x[i]);
   // Router: this CTA's quarter-rows, two at a time per warp, loads first.
   float4 wv[2][4];
   int ucur = u0 + warp;
@@ -786,7 +809,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
       }
     }
   }
+  for (int i = threadIdx.x; i < T * H; i += kThreads) S.xs[i] = bf16_to_f32(P.x[i]);
   __syncthreads();
+  if (has_shared) {
+    const moe_expert& sd = S.desc[T * k];
+    shared_ok = expert_ok(sd, H, I) && qt_supported(sd.gate.qtype, H) && qt_supported_down(sd.down.qtype, I);
+    if (!shared_ok && b == 0 && threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
+  }
+  if (shared_ok) {
+    int r0, r1;
+    split_range(I, G, b, r0, r1);
+    const int R = gu_rows_per_batch(S.desc[T * k], H);
+    if (threadIdx.x == 0) {
+      S.spre[0] = 0;
+      S.spre[1] = (r1 - r0 + R - 1) / R;
+      S.srpb[0] = R;
+    }
+    __syncthreads();
+    SJ = GateUpJobs{S.desc + T * k, S.spre, S.srpb, 1, r0, r1 - r0, H, T * k + my_t};
+    split_range(SJ.total(), ngrp, grp, sb0, sb1);
+    for (int i = 0; i < kSlots; ++i)
+      issue_any<2>(ring + i * kSlotBytes, sb0 + i < sb1 ? SJ.get(sb0 + i) : Batch{nullptr, nullptr, 0, 0, 0, 0}, H);
+  }
   for (; ucur < u1; ucur += 2 * kWarps) {
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
@@ -828,10 +872,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
     }
   }
   // 2) shared expert gate/up, already in flight
-  if (shared_ok) gate_up_stream(ring, SJ, sb0, sb1, S.xs + my_t * H, P.h, I, true);
+  if (shared_ok) gate_up_stream(ring, red, SJ, sb0, sb1, S.xs + my_t * H, P.h, I, true);
   // 3) L2 prefetch of the shared down rows this CTA uses in phase C
   if (shared_ok && threadIdx.x == 0) {
-    const moe_qmatrix& d = P.shared->down;
+    const moe_qmatrix& d = S.desc[T * k].down;
     const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
     prefetch_l2(d.codes, n0 * rb, n1 * rb);
     if (d.qtype != MOE_Q_INT8_PER_CHANNEL) prefetch_l2(d.scales, n0 * sb, n1 * sb);
@@ -906,26 +950,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
         P.topk_idx[i] = s_idx[i];
         P.topk_w[i] = s_w[i];
       }
-    // Routed gate/up of this CTA's intermediate rows, this warp's token.
-    bool bad = false;
-    for (int j = 0; j < k; ++j) {
-      const moe_expert& ex = P.experts[s_idx[my_t * k + j]];
-      if (!expert_ok(ex, H, I) || !qt_supported(ex.gate.qtype, H) || !qt_supported_down(ex.down.qtype, I)) bad = true;
+    // The picks' descriptors into shared memory, then the batch tables.
+    {
+      constexpr int W = int(sizeof(moe_expert) / 4);
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
+      uint32_t* dst = reinterpret_cast<uint32_t*>(S.desc);
+      for (int i = threadIdx.x; i < T * k * W; i += kThreads) dst[i] = src[size_t(s_idx[i / W]) * W + (i % W)];
     }
-    if (bad) {
-      if (lane == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 1000000);
+    if (threadIdx.x == 0) s_bad = 0;
+    __syncthreads();
+    int r0, r1;
+    split_range(I, G, b, r0, r1);
+    const int nr = r1 - r0;
+    const int nrouted = T * k, npairs = nrouted + (shared_ok ? T : 0);
+    for (int p = threadIdx.x; p < npairs; p += kThreads) {
+      const moe_expert& e = S.desc[p < nrouted ? p : nrouted];
+      if (p < nrouted) {
+        if (!expert_ok(e, H, I) || !qt_supported(e.gate.qtype, H) || !qt_supported_down(e.down.qtype, I)) {
+          s_bad = 1;
+          continue;
+        }
+        S.grpb[p] = gu_rows_per_batch(e, H);
+      }
+      S.drpb[p] = dn_rows_per_batch(e.down, I);
+    }
+    __syncthreads();
+    if (s_bad) {
+      if (threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 1000000);
     } else {
-      int r0, r1;
-      split_range(I, G, b, r0, r1);
-      GateUpJobs RJ{P.experts, s_idx + my_t * k, k, r0, r1 - r0, H, my_t * k};
+      if (threadIdx.x < T) {  // gate/up prefix per token
+        const int t = threadIdx.x;
+        int acc = 0;
+        for (int j = 0; j < k; ++j) {
+          S.gpre[t * (k + 1) + j] = acc;
+          const int R = S.grpb[t * k + j];
+          acc += (nr + R - 1) / R;
+        }
+        S.gpre[t * (k + 1) + k] = acc;
+      }
+      if (threadIdx.x == 32) {  // down prefix over all pairs
+        int acc = 0;
+        for (int p = 0; p < npairs; ++p) {
+          S.dpre[p] = acc;
+          const int R = S.drpb[p];
+          acc += (nn + R - 1) / R;
+        }
+        S.dpre[npairs] = acc;
+      }
+      __syncthreads();
+      GateUpJobs RJ{S.desc + my_t * k, S.gpre + my_t * (k + 1), S.grpb + my_t * k, k, r0, nr, H, my_t * k};
       int b0, b1;
       split_range(RJ.total(), ngrp, grp, b0, b1);
-      gate_up_stream(ring, RJ, b0, b1, S.xs + my_t * H, P.h, I, false);
+      gate_up_stream(ring, red, RJ, b0, b1, S.xs + my_t * H, P.h, I, false);
     }
     // L2 prefetch of the routed down rows this CTA owns in phase C.
-    for (int p = threadIdx.x; p < T * k; p += kThreads) {
-      const moe_qmatrix& d = P.experts[s_idx[p]].down;
-      if (!qmatrix_ok(d, H, I)) continue;
+    for (int p = threadIdx.x; p < T * k && !s_bad; p += kThreads) {
+      const moe_qmatrix& d = S.desc[p].down;
       const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
       prefetch_l2(d.codes, n0 * rb, n1 * rb);
       if (d.qtype != MOE_Q_INT8_PER_CHANNEL) prefetch_l2(d.scales, n0 * sb, n1 * sb);
@@ -938,14 +1018,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
   {
     const int nrouted = T * k;
     const int npairs = nrouted + (shared_ok ? T : 0);
-    bool bad = false;
-    for (int p = 0; p < nrouted; ++p)
-      if (!qmatrix_ok(P.experts[s_idx[p]].down, H, I) || !qt_supported_down(P.experts[s_idx[p]].down.qtype, I)) bad = true;
+    const bool bad = s_bad != 0;
     if (!bad) {
-      DownJobs D{P.experts, P.shared, s_idx, nrouted, npairs, n0, nn, I};
+      DownJobs D{S.desc, S.dpre, S.drpb, nrouted, npairs, n0, nn, I};
       int b0, b1;
       split_range(D.total(), kWarps, warp, b0, b1);
-      down_stream(ring, D, b0, b1, P.h, S.ys);
+      down_stream(ring, red, D, b0, b1, P.h, S.ys);
     }
     __syncthreads();
     // Gate-weighted sum in slot order plus the shared expert; one rounding.
@@ -983,7 +1061,8 @@ static size_t decode_fused_smem(int T, int H, int I, int E, int k, int grid) {
   const int nn = (H + grid - 1) / grid;
   const size_t floats = size_t(T) * H + size_t(T) * E + size_t(T * k + T) * nn;
   const size_t cand = 2 * 4 * size_t(T) * dec::kWarps * k;
-  return ring + 4 * floats + cand;
+  const size_t tables = 16 + sizeof(moe_expert) * size_t(T * k + 1) + 4 * size_t(T * (k + 1) + T * k + 2 * (T * k + T) + 4);
+  return ring + 4 * floats + cand + tables;
 }
 
 bool decode_fused_eligible(int T, int H, int I, int E, int k) {

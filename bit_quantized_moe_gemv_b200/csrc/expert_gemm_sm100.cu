@@ -1,6 +1,13 @@
 // Prefill experts: grouped GEMM on the 5th-generation tensor cores (tcgen05,
-// accumulators in TMEM), dequantising the packed weights to bf16 in shared
-// memory.
+// accumulators in TMEM), dequantising the packed weights to 16-bit floats in
+// shared memory.
+//
+// Operand type: fp16 for both A and B (kind::f16 needs them equal). An int4
+// or int2 code maps exactly to an fp16 integer and the fp16 group scale is
+// used as stored, so each weight rounds once, at 2^-11; bf16 would round the
+// scale and then the product at 2^-8 each, which breaks the 2e-2 x rms
+// max-error bound on long dot products. The bf16 activations convert to fp16
+// exactly in the normal range (values beyond +-65504 saturate).
 //
 // Prefill pushes many tokens through each expert at once (the telli.sh page
 // "Strata 与 Qwen3.8-Flash-Next：如何在个人电脑上运行 180B 级模型", section
@@ -14,7 +21,7 @@
 // Layout ("swap AB"): the weight rows are the MMA's M side (128 per tile),
 // tokens its N side (up to 128 per tile), so a small expert wastes no M.
 // Activations are stored once, by `gather_rows_kernel`, as 16 KiB tiles of
-// 128 rows x 64 bf16 already in the 128-byte-swizzled K-major shared-memory
+// 128 rows x 64 fp16 already in the 128-byte-swizzled K-major shared-memory
 // image, so one 1-D bulk copy loads a B tile. Inside every 8-element group
 // the K order is (0,4,1,5,2,6,3,7): the order in which a byte-free lop3
 // unpacks eight int4 codes of one 32-bit word. Weights (A) are produced by
@@ -97,12 +104,19 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   if (g == 0) plan.count[0] = min(total, max_tiles);
 }
 
-// Byte offset of element (row, k) inside a swizzled 128-row x 64-col bf16 tile,
+// Byte offset of element (row, k) inside a swizzled 128-row x 64-col 16-bit tile,
 // with the (0,4,1,5,2,6,3,7) order inside each 8-element group.
 __device__ __forceinline__ uint32_t tile_off(int row, int k) {
   const int chunk = k >> 3, e = k & 7;
   const int pos = e < 4 ? 2 * e : 2 * (e - 4) + 1;
   return uint32_t(row) * 128u + (uint32_t((chunk ^ (row & 7))) << 4) + uint32_t(pos) * 2u;
+}
+
+// ---------------------------------------------------------------- fp16 helpers
+__device__ __forceinline__ float sat_f16(float v) { return fminf(fmaxf(v, -65504.f), 65504.f); }
+__device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // ---------------------------------------------------------------- gather
@@ -123,11 +137,19 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     const uint4* src = reinterpret_cast<const uint4*>(x + size_t(tok) * H);
     for (int c = lane; c < H / 8; c += 32) {
       const uint4 v = __ldg(src + c);
+      // bf16 -> fp16 (saturating at +-65504), K order (0,4,1,5,2,6,3,7)
+      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = sat_f16(__uint_as_float(in[i] << 16));
+        f[2 * i + 1] = sat_f16(__uint_as_float(in[i] & 0xffff0000u));
+      }
       uint4 o;
-      o.x = __byte_perm(v.x, v.z, 0x5410);
-      o.y = __byte_perm(v.x, v.z, 0x7632);
-      o.z = __byte_perm(v.y, v.w, 0x5410);
-      o.w = __byte_perm(v.y, v.w, 0x7632);
+      o.x = h2_bits(f[0], f[4]);
+      o.y = h2_bits(f[1], f[5]);
+      o.z = h2_bits(f[2], f[6]);
+      o.w = h2_bits(f[3], f[7]);
       const int kb = c >> 3, chunk = c & 7;
       uint8_t* dst = xt + (size_t(rt) * KB + kb) * kTileBytes + size_t(row) * 128 + ((chunk ^ (row & 7)) << 4);
       *reinterpret_cast<uint4*>(dst) = o;
@@ -136,24 +158,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 }
 
 // ---------------------------------------------------------------- dequant
-__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
 }
-__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
 }
-__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
-  __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b),
-                             *reinterpret_cast<__nv_bfloat162*>(&c));
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b),
+                      *reinterpret_cast<__half2*>(&c));
   return *reinterpret_cast<uint32_t*>(&r);
 }
-__device__ __forceinline__ uint32_t bf2_splat_from_f16(uint16_t h) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(__half2float(__ushort_as_half(h)));
-  const uint32_t u = *reinterpret_cast<const uint16_t*>(&b);
-  return u | (u << 16);
-}
+__device__ __forceinline__ uint32_t h2_splat(uint16_t h) { return uint32_t(h) | (uint32_t(h) << 16); }
 
 // Raw data one dequant thread needs for one k-block of one matrix: 32
 // consecutive K elements of one weight row.
@@ -181,23 +199,25 @@ __device__ __forceinline__ void load_raw(const moe_qmatrix& W, int row, int k0, 
   }
 }
 
-// 32 weights -> 4 x 16-byte chunks (bf16, K order 0,4,1,5,2,6,3,7 per 8).
+// 32 weights -> 4 x 16-byte chunks of fp16, K order (0,4,1,5,2,6,3,7) per 8.
+// A code c sits in the mantissa of the fp16 1024 + c (0x6400 | c), so the
+// code-to-integer step is exact and the scale product rounds once.
 __device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4]) {
   if (qtype == MOE_Q_INT4_SYM_G32) {
-    const uint32_t s2 = bf2_splat_from_f16(uint16_t(r.s));
+    const uint32_t s2 = h2_splat(uint16_t(r.s));
     const uint32_t w[4] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w};
-    const uint32_t k136 = 0x43084308u;  // bf16x2 (136, 136)
+    const uint32_t k1032 = 0x64086408u;  // fp16x2 (1032, 1032): 1024 + 8
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = bf2_mul(bf2_sub(((w[c] >> (4 * j)) & 0x000F000Fu) | 0x43004300u, k136), s2);
+      for (int j = 0; j < 4; ++j) v[j] = h2_mul(h2_sub(((w[c] >> (4 * j)) & 0x000F000Fu) | 0x64006400u, k1032), s2);
       o[c] = make_uint4(v[0], v[1], v[2], v[3]);
     }
   } else if (qtype == MOE_Q_INT2_ASYM_G16) {
-    const uint32_t sA = bf2_splat_from_f16(uint16_t(r.s & 0xffffu)), sB = bf2_splat_from_f16(uint16_t(r.s >> 16));
-    const uint32_t mA = bf2_splat_from_f16(uint16_t(r.m & 0xffffu)), mB = bf2_splat_from_f16(uint16_t(r.m >> 16));
-    const uint32_t k128 = 0x43004300u;
+    const uint32_t sA = h2_splat(uint16_t(r.s & 0xffffu)), sB = h2_splat(uint16_t(r.s >> 16));
+    const uint32_t mA = h2_splat(uint16_t(r.m & 0xffffu)), mB = h2_splat(uint16_t(r.m >> 16));
+    const uint32_t k1024 = 0x64006400u;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const uint32_t word = c < 2 ? r.c0.x : r.c0.y;
@@ -205,7 +225,7 @@ __device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4
       const uint32_t s2 = c < 2 ? sA : sB, m2 = c < 2 ? mA : mB;
       uint32_t v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = bf2_fma(bf2_sub(((t >> (2 * j)) & 0x00030003u) | 0x43004300u, k128), s2, m2);
+      for (int j = 0; j < 4; ++j) v[j] = h2_fma(h2_sub(((t >> (2 * j)) & 0x00030003u) | 0x64006400u, k1024), s2, m2);
       o[c] = make_uint4(v[0], v[1], v[2], v[3]);
     }
   } else {
@@ -222,10 +242,7 @@ __device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4
       }
       uint32_t v[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 p = __floats2bfloat162_rn(q[j] * s, q[4 + j] * s);
-        v[j] = *reinterpret_cast<const uint32_t*>(&p);
-      }
+      for (int j = 0; j < 4; ++j) v[j] = h2_bits(q[j] * s, q[4 + j] * s);
       o[c] = make_uint4(v[0], v[1], v[2], v[3]);
     }
   }
@@ -441,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
         const int rt = int(t / MT);
         const int nrows = a.plan.nrows[rt];
         const int N = (nrows + 15) & ~15;
-        const uint32_t idesc = ptx::idesc_bf16(BM, N);
+        const uint32_t idesc = ptx::idesc_f16(BM, N);
         const int buf = it & 1;
         const uint32_t use = uint32_t(it >> 1) & 1u;
         if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar[buf]), use ^ 1u, abort_p)) {
@@ -464,10 +481,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t bdesc = ptx::smem_desc_k128(sb + 32 * ks);
             const uint32_t acc = (kb | ks) != 0;
-            ptx::mma_bf16(d0, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
+            ptx::mma_f16(d0, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
             if (kGateUp) {
               const uint32_t sa1 = ptx::smem_addr(stage_a(s, 1));
-              ptx::mma_bf16(d0 + 128, ptx::smem_desc_k128(sa1 + 32 * ks), bdesc, idesc, acc);
+              ptx::mma_f16(d0 + 128, ptx::smem_desc_k128(sa1 + 32 * ks), bdesc, idesc, acc);
             }
           }
           ptx::mma_commit(ptx::smem_addr(&empty_bar[s]));
@@ -508,15 +525,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           uint32_t v1[32];
           ptx::tmem_ld32(taddr + 128u + uint32_t(c0), v1);
           ptx::tmem_ld_wait();
-          // h = silu(g) * u -> bf16 into the H tiles (K index m of the down GEMM)
+          // h = silu(g) * u -> fp16 into the H tiles (K index m of the down GEMM)
           uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int n = c0 + j;
             if (n < nrows) {
               const float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]);
-              const __nv_bfloat16 hb = __float2bfloat16_rn(silu_f32(gv) * uv);
-              *reinterpret_cast<__nv_bfloat16*>(base + tile_off(n, m & 63)) = hb;
+              *reinterpret_cast<__half*>(base + tile_off(n, m & 63)) = __float2half_rn(sat_f16(silu_f32(gv) * uv));
             }
           }
         } else {

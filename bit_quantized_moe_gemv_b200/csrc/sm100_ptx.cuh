@@ -77,8 +77,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 in, fp32 acc).
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (16-bit inputs as the
+// instruction descriptor says, fp32 accumulation).
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -118,6 +119,15 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
   d |= uint64_t(1) << 46;                          // descriptor version (sm_100)
   d |= uint64_t(2) << 61;                          // layout: 128-byte swizzle
   return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 D, M x N.
+__host__ __device__ __forceinline__ uint32_t idesc_f16(int M, int N) {
+  return (1u << 4)                      // D format fp32
+         | (0u << 7)                    // A format fp16
+         | (0u << 10)                   // B format fp16
+         | (uint32_t(N >> 3) << 17)     // N / 8
+         | (uint32_t(M >> 4) << 24);    // M / 16
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, M x N.
