@@ -52,6 +52,18 @@ def parse():
     return ap.parse_args()
 
 
+def workload_config(wl, world=1):
+    """The `config` object of the JSON line (identical for both arms)."""
+    q = {wlm.Q_INT4_SYM_G32: "int4 sym g32", wlm.Q_INT2_ASYM_G16: "int2 asym g16",
+         wlm.Q_INT8_PER_CHANNEL: "int8 per-channel"}
+    routed = ", ".join(f"experts {lo}-{(hi or wl.E) - 1} {q[t]}" for lo, hi, t in wl.routed_qtypes)
+    desc = (f"{wl.name}: T={wl.T} tokens/step, H={wl.H}, I={wl.I}, E={wl.E} routed + 1 shared "
+            f"({q[wl.shared_qtype]}), top-{wl.k}, {routed}, Zipf({wl.zipf_s}) router prior"
+            + (f", {wl.uniform_frac:.0%} uniform rows" if wl.uniform_frac else "")
+            + (", fresh token per step" if wl.T <= 4 else ""))
+    return {"workload": desc, "global_batch": wl.T * world, "parallelism": f"replicas x{world}"}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -234,13 +246,8 @@ def run_ours(args, rank, world, peaks, peak_kind):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded; random weights of the stated architecture)",
-        "config": {
-            "workload": f"decode one layer: T={wl.T}, H={wl.H}, I={wl.I}, E={wl.E}+1 shared, k={wl.k}, "
-                        f"int4 sym g32 experts, Zipf({wl.zipf_s}) prior, fresh token per step",
-            "global_batch": wl.T * world,
-            "parallelism": f"replicas x{world}",
-            "l2": "flushed between steps (2 x L2 write, outside the timed events)",
-        },
+        "config": dict(workload_config(wl, world),
+                       l2="flushed between steps (2 x L2 write, outside the timed events)"),
         "roofline": {
             "bound": "hbm",
             "kernel": "moe_layer step (all launches of one step)",
@@ -347,9 +354,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; random weights of the stated architecture)",
-        "config": {"workload": f"{wl.name}: T={T}, H={H}, I={I}, E={E}+1 shared, k={k}, Zipf({wl.zipf_s})",
-                   "global_batch": T * world, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (1.36 GB of expert weights)"},
+        "config": dict(workload_config(wl, world), l2="inputs larger than L2 (1.36 GB of expert weights)"),
         "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (gather + tcgen05 gate/up + down)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops, "ms_per_launch": ffn_ms,
@@ -382,8 +387,9 @@ def main():
             "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": f"decode one layer: T={wl.T}, H={wl.H}, I={wl.I}, E={wl.E}+1 shared, k={wl.k}",
-                       "global_batch": wl.T},
+            "config": dict(workload_config(wl, 1),
+                           l2="flushed between steps (2 x L2 write, outside the timed events)"
+                           if wl.T <= 4 else "inputs larger than L2 (1.36 GB of expert weights)"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                              "sample": f"{steps} of {args.steps} requested steps (1 token each), bounded to "
                                        f"{budget:.0f} s"},

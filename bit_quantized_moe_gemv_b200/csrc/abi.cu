@@ -58,7 +58,8 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_rou
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   float* logits = logits_out ? logits_out : ws_at<float>(ws, L.logits);
   return cuda_status(launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w, logits,
-                                  ws_at<WsHeader>(ws, 0), static_cast<cudaStream_t>(stream)));
+                                  ws_at<void>(ws, L.router), ws_at<WsHeader>(ws, 0),
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_dispatch(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E, int32_t* counts, int32_t* offsets,
@@ -143,7 +144,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   int* inv = ws_at<int>(ws, L.inv);
   float* y_perm = ws_at<float>(ws, L.y_perm);  // fp32: out is rounded only once
   cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w,
-                               ws_at<float>(ws, L.logits), hdr, st);
+                               ws_at<float>(ws, L.logits), ws_at<void>(ws, L.router), hdr, st);
   if (e == cudaSuccess) e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, inv, ws_at<int>(ws, L.hist), hdr, st);
   float* shared_y = nullptr;
   if (T > kDecodeMaxT && grouped_eligible(H, I, E, shared_dev != nullptr)) {

@@ -60,15 +60,8 @@ struct Params {
 };
 
 // ---------------------------------------------------------------- helpers
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
+// Packed fp32x2 FMA (sm_100): two lanes of work per instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // Code byte b of `w` (a nibble or crumb already isolated in the low bits of
 // each byte) -> 0.5 + c/256.
@@ -201,11 +194,12 @@ __device__ bool grid_sync(WsHeader* hdr, uint32_t target) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
-    __threadfence();
-    atomicAdd(&hdr->bar_count, 1u);
+    // release: the CTA's writes (ordered before this thread by the CTA
+    // barrier above) become visible before the arrival is counted
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&hdr->bar_count) : "memory");
     const long long t0 = clock64();
-    while (ld_acquire(&hdr->bar_count) < target) {
-      if (*reinterpret_cast<volatile int*>(&hdr->abort)) {
+    for (uint32_t it = 1; ld_acquire(&hdr->bar_count) < target; ++it) {
+      if ((it & 31) == 0 && *reinterpret_cast<volatile int*>(&hdr->abort)) {
         ok = 0;
         break;
       }
@@ -342,12 +336,16 @@ struct XPtr {
 template <int QT, int CPL, int M, class X>
 __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, int K, const X& x, float* red) {
   constexpr int R = batch_rows(QT, CPL, M);
+  // two independent items per iteration: the gate and up rows of one row
+  // index (M = 2), or two consecutive rows (M = 1)
+  constexpr int U = (M == 2 || R == 1) ? 1 : 2;
   const int lane = threadIdx.x & 31;
   const int CPR = chunks_per_row(QT, K);
 #pragma unroll 1
-  for (int r = 0; r < R; ++r) {
-#pragma unroll 1
-    for (int m = 0; m < M; ++m) {
+  for (int r0i = 0; r0i < R; r0i += U) {
+#pragma unroll
+    for (int it = 0; it < U * M; ++it) {
+      const int r = r0i + it / M, m = it % M;
       float acc = 0.f;
       if (r < b.nrow) {
 #pragma unroll
@@ -364,7 +362,7 @@ __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, i
             for (int w = 0; w < 4; ++w) {
               const uint32_t lo = wd[w] & 0x0F0F0F0Fu, hi = (wd[w] >> 4) & 0x0F0F0F0Fu;
               const float* xv = x.v[j] + 8 * w;
-              float2 t2 = make_float2(code_f<0>(lo) * xv[0], code_f<1>(lo) * xv[1]);
+              float2 t2 = __fmul2_rn(make_float2(code_f<0>(lo), code_f<1>(lo)), make_float2(xv[0], xv[1]));
               t2 = ffma2(make_float2(code_f<2>(lo), code_f<3>(lo)), make_float2(xv[2], xv[3]), t2);
               t2 = ffma2(make_float2(code_f<0>(hi), code_f<1>(hi)), make_float2(xv[4], xv[5]), t2);
               a4[w] = ffma2(make_float2(code_f<2>(hi), code_f<3>(hi)), make_float2(xv[6], xv[7]), t2);
@@ -409,7 +407,7 @@ __device__ __forceinline__ void compute_batch_t(uint8_t* slot, const Batch& b, i
               for (int bb = 0; bb < 4; ++bb)
                 q[bb] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | bb)) - 8388736.0f;  // - (2^23+128)
               a4[w] = ffma2(make_float2(q[2], q[3]), make_float2(xv[2], xv[3]),
-                            make_float2(q[0] * xv[0], q[1] * xv[1]));
+                            __fmul2_rn(make_float2(q[0], q[1]), make_float2(xv[0], xv[1])));
             }
             acc += ((a4[0].x + a4[1].x) + (a4[2].x + a4[3].x)) + ((a4[0].y + a4[1].y) + (a4[2].y + a4[3].y));
           }
@@ -874,7 +872,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
   // 2) shared expert gate/up, already in flight
   if (shared_ok) gate_up_stream(ring, red, SJ, sb0, sb1, S.xs + my_t * H, P.h, I, true);
   // 3) L2 prefetch of the shared down rows this CTA uses in phase C
-  if (shared_ok && threadIdx.x == 0) {
+  if (shared_ok && threadIdx.x == kThreads - 32) {  // not the barrier thread
     const moe_qmatrix& d = S.desc[T * k].down;
     const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
     prefetch_l2(d.codes, n0 * rb, n1 * rb);
@@ -891,14 +889,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
       S.lg[i] = ((p4.x + p4.y) + (p4.z + p4.w)) + (P.bias ? P.bias[t * P.bstride + e] : 0.f);
     }
     __syncthreads();
-    // Top-k, stage 1: warp w selects the best k of its slice of the experts.
+    // Top-k, stage 1: warp w selects the best k of its slice of the experts
+    // (loop-based, so the code stays small: it runs once per launch, cold).
     const int chunk = (E + kWarps - 1) / kWarps;  // <= 128
     for (int t = 0; t < T; ++t) {
       const int e0 = min(E, warp * chunk), e1 = min(E, e0 + chunk);
       const int n = e1 - e0, kk = min(k, n);
       uint32_t* ck = S.ck + (size_t(t) * kWarps + warp) * k;
       int* ci = S.ci + (size_t(t) * kWarps + warp) * k;
-      // candidates straight from the logits row
       uint32_t keys[4];
       int ids[4];
 #pragma unroll
@@ -907,8 +905,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
         keys[i] = c < n ? f2key(S.lg[size_t(t) * E + e0 + c]) : 0u;
         ids[i] = c < n ? e0 + c : 0x7fffffff;
       }
-      // reuse warp_select through a per-lane view: stage the 128 keys in ck/ci
-      // scratch is too small, so select directly here
       for (int j = 0; j < k; ++j) {
         uint32_t bk = 0u;
         int bi = 0x7fffffff, bs = -1;
@@ -1004,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(Params P) {
       gate_up_stream(ring, red, RJ, b0, b1, S.xs + my_t * H, P.h, I, false);
     }
     // L2 prefetch of the routed down rows this CTA owns in phase C.
-    for (int p = threadIdx.x; p < T * k && !s_bad; p += kThreads) {
+    for (int p = threadIdx.x - (kThreads - 64); p >= 0 && p < T * k && !s_bad; p += 64) {  // last two warps
       const moe_qmatrix& d = S.desc[p].down;
       const size_t rb = size_t(chunks_per_row(d.qtype, I)) * 16, sb = size_t(scale_row_bytes(d.qtype, I));
       prefetch_l2(d.codes, n0 * rb, n1 * rb);

@@ -50,7 +50,7 @@ constexpr int BM = 128, BN = 128, BK = 64;
 constexpr int kTileBytes = BN * BK * 2;  // 16 KiB: one A or B tile
 constexpr int kThreads = 14 * 32;
 constexpr int kDqWarps = 8, kDqThreads = kDqWarps * 32;
-constexpr int kPD = 4;  // dequant global-load prefetch depth (k-blocks)
+constexpr int kPD = 3;  // dequant global-load prefetch depth (k-blocks)
 
 // ---------------------------------------------------------------- plan
 // Row tiles: every group (routed expert e < E, or the shared expert = E) is
@@ -265,9 +265,16 @@ struct Args {
   WsHeader* hdr;
 };
 
+// Raw-code staging: each dequant thread copies (cp.async) its own codes and
+// scales kRawDepth k-blocks ahead into a private area of shared memory.
+constexpr int kRawDepth = 4;
+constexpr int kRawCodeBytes = 2 * 2 * 256 * 16;  // [matrix][16-B unit][thread] (int8 needs two units)
+constexpr int kRawAuxBytes = 2 * 256 * 8;        // [matrix][thread] 8 B (scale / scales + mins)
+constexpr int kRawSlotBytes = kRawCodeBytes + kRawAuxBytes;
+
 template <bool kGateUp>
 struct Cfg {
-  static constexpr int kStages = kGateUp ? 4 : 6;
+  static constexpr int kStages = kGateUp ? 3 : 4;
   static constexpr int kATiles = kGateUp ? 2 : 1;
   static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
   static constexpr int kAccCols = kGateUp ? 256 : 128;  // one accumulator buffer
@@ -282,82 +289,159 @@ __device__ __forceinline__ const moe_qmatrix& pick(const moe_expert& e, int whic
 
 // One job = one k-block of one tile: 128 weight rows x 64 K of each A matrix.
 // Thread (row, half) of the 256 dequant threads handles 32 K elements of one
-// row. Global loads run kPD jobs ahead of the dequant.
-template <bool kGateUp>
-struct DqJob {
-  const moe_qmatrix* W[2];
-  int row, k0;
-  bool valid;
+// row. The tile's matrix pointers are resolved once per tile into registers;
+// global loads of the codes run kPD jobs ahead of the dequant.
+struct DqMat {
+  const uint8_t* codes;   // start of this thread's row
+  const uint16_t* scales; // start of this thread's row of scales (int8: &scale[row])
+  const uint16_t* mins;
+  int qtype;
 };
 
-template <bool kGateUp>
-__device__ __forceinline__ DqJob<kGateUp> make_job(const Args& a, long long j, int MT, int KB, long long ntiles,
-                                                    int dt) {
-  DqJob<kGateUp> J;
-  const long long t = blockIdx.x + (j / KB) * gridDim.x;
-  J.valid = t < ntiles;
-  J.W[0] = J.W[1] = nullptr;
-  J.row = 0;
-  J.k0 = 0;
-  if (!J.valid) return J;
-  const int rt = int(t / MT), mt = int(t % MT), kb = int(j % KB);
-  const int g = a.plan.group[rt];
-  const moe_expert* ex = g < a.E ? a.experts + g : a.shared;
-  J.W[0] = kGateUp ? &ex->gate : &ex->down;
-  J.W[1] = kGateUp ? &ex->up : nullptr;
-  J.row = mt * BM + ((threadIdx.x - 6 * 32) >> 1);
-  J.k0 = kb * BK + (dt & 1) * 32;
-  return J;
+__device__ __forceinline__ DqMat dq_mat(const moe_qmatrix& W, int row, int M, int K, WsHeader* hdr) {
+  DqMat d{nullptr, nullptr, nullptr, 0};
+  if (!qmatrix_ok(W, M, K)) {
+    if ((threadIdx.x & 31) == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 7000000);
+    return d;
+  }
+  d.qtype = W.qtype;
+  d.codes = W.codes + size_t(row) * row_code_bytes(W.qtype, K);
+  if (W.qtype == MOE_Q_INT8_PER_CHANNEL) {
+    d.scales = W.scales + row;
+  } else {
+    const int g = W.qtype == MOE_Q_INT4_SYM_G32 ? 32 : 16;
+    d.scales = W.scales + size_t(row) * (K / g);
+    d.mins = W.mins ? W.mins + size_t(row) * (K / g) : nullptr;
+  }
+  return d;
 }
 
-template <bool kGateUp>
-__device__ __forceinline__ void job_load(const Args& a, const DqJob<kGateUp>& J, RawK (&r)[2], int& qt) {
-  qt = 0;
-  if (!J.valid) return;
-#pragma unroll
-  for (int w = 0; w < (kGateUp ? 2 : 1); ++w) {
-    const moe_qmatrix& W = *J.W[w];
-    if (!qmatrix_ok(W, a.M, a.K)) {
-      r[w].c0 = r[w].c1 = make_uint4(0, 0, 0, 0);
-      r[w].s = r[w].m = 0;
-      if ((threadIdx.x & 31) == 0) flag_error(a.hdr, MOE_ERR_DEVICE_FAULT, 7000000);
-      continue;
-    }
-    qt = W.qtype;
-    load_raw(W, J.row, J.k0, r[w]);
+__device__ __forceinline__ void dq_load(const DqMat& d, int k0, RawK& r) {
+  if (d.qtype == MOE_Q_INT4_SYM_G32) {
+    r.c0 = __ldg(reinterpret_cast<const uint4*>(d.codes + k0 / 2));
+    r.s = __ldg(d.scales + k0 / 32);
+  } else if (d.qtype == MOE_Q_INT2_ASYM_G16) {
+    const uint2 c = __ldg(reinterpret_cast<const uint2*>(d.codes + k0 / 4));
+    r.c0 = make_uint4(c.x, c.y, 0, 0);
+    r.s = __ldg(reinterpret_cast<const unsigned int*>(d.scales + k0 / 16));
+    r.m = __ldg(reinterpret_cast<const unsigned int*>(d.mins + k0 / 16));
+  } else if (d.qtype == MOE_Q_INT8_PER_CHANNEL) {
+    const uint4* p = reinterpret_cast<const uint4*>(d.codes + k0);
+    r.c0 = __ldg(p);
+    r.c1 = __ldg(p + 1);
+    r.s = __ldg(d.scales);
+  } else {
+    r.c0 = r.c1 = make_uint4(0, 0, 0, 0);
+    r.s = r.m = 0;
+  }
+}
+
+__device__ __forceinline__ void cp16(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp8(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(ptx::smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp4(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(ptx::smem_addr(dst)), "l"(src) : "memory");
+}
+
+// Copy this thread's raw data of one k-block of matrix d into its slot.
+__device__ __forceinline__ void raw_issue(const DqMat& d, int k0, uint8_t* slot, int w, int dt) {
+  uint8_t* code0 = slot + ((w * 2 + 0) * 256 + dt) * 16;
+  uint8_t* code1 = slot + ((w * 2 + 1) * 256 + dt) * 16;
+  uint8_t* aux = slot + kRawCodeBytes + (w * 256 + dt) * 8;
+  if (d.qtype == MOE_Q_INT4_SYM_G32) {
+    cp16(code0, d.codes + k0 / 2);
+    cp4(aux, d.scales + ((k0 / 32) & ~1));
+  } else if (d.qtype == MOE_Q_INT2_ASYM_G16) {
+    cp8(code0, d.codes + k0 / 4);
+    cp4(aux, d.scales + k0 / 16);
+    cp4(aux + 4, d.mins + k0 / 16);
+  } else if (d.qtype == MOE_Q_INT8_PER_CHANNEL) {
+    cp16(code0, d.codes + k0);
+    cp16(code1, d.codes + k0 + 16);
+    cp4(aux, reinterpret_cast<const uint16_t*>(reinterpret_cast<uintptr_t>(d.scales) & ~uintptr_t(3)));
+  }
+}
+
+__device__ __forceinline__ void raw_read(const uint8_t* slot, int w, int dt, int qtype, int k0, bool odd_row_scale,
+                                         RawK& r) {
+  r.c0 = *reinterpret_cast<const uint4*>(slot + ((w * 2 + 0) * 256 + dt) * 16);
+  r.c1 = *reinterpret_cast<const uint4*>(slot + ((w * 2 + 1) * 256 + dt) * 16);
+  const uint2 aux = *reinterpret_cast<const uint2*>(slot + kRawCodeBytes + (w * 256 + dt) * 8);
+  if (qtype == MOE_Q_INT4_SYM_G32) {
+    r.s = ((k0 / 32) & 1) ? (aux.x >> 16) : (aux.x & 0xffffu);
+  } else if (qtype == MOE_Q_INT2_ASYM_G16) {
+    r.s = aux.x;
+    r.m = aux.y;
+  } else {
+    r.s = odd_row_scale ? (aux.x >> 16) : (aux.x & 0xffffu);
   }
 }
 
 template <bool kGateUp>
-__device__ void dequant_role(const Args& a, uint8_t* smem, uint64_t* full_bar, uint64_t* empty_bar,
-                             volatile int* abort_p, int MT, int KB, long long ntiles) {
+__device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, uint64_t* full_bar,
+                             uint64_t* empty_bar, volatile int* abort_p, int MT, int KB, long long ntiles) {
   using C = Cfg<kGateUp>;
+  constexpr int NW = kGateUp ? 2 : 1;
   const int dt = threadIdx.x - 6 * 32;  // 0 .. 255
   const int row = dt >> 1, half = dt & 1;
   const long long per_cta = ntiles > blockIdx.x ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
   const long long njobs = per_cta * KB;
-  RawK raw[kPD][2];
-  int qts[kPD];
+  DqMat ld[NW];
+  long long ld_tile = -1;
+  int ld_wrow = 0;
+  auto resolve = [&](long long j) {
+    const long long t = blockIdx.x + (j / KB) * gridDim.x;
+    const int rt = int(t / MT), mt = int(t % MT);
+    const int g = a.plan.group[rt];
+    const moe_expert* ex = g < a.E ? a.experts + g : a.shared;
+    ld_wrow = mt * BM + row;
+    ld[0] = dq_mat(kGateUp ? ex->gate : ex->down, ld_wrow, a.M, a.K, a.hdr);
+    if (kGateUp) ld[NW - 1] = dq_mat(ex->up, ld_wrow, a.M, a.K, a.hdr);
+  };
+  int qts[kRawDepth][NW];
+  int odd[kRawDepth];
+  auto issue = [&](long long j, int p) {
+    if (j < njobs) {
+      if (j / KB != ld_tile) {
+        resolve(j);
+        ld_tile = j / KB;
+      }
+      uint8_t* slot = raw_smem + size_t(p) * kRawSlotBytes;
 #pragma unroll
-  for (int p = 0; p < kPD; ++p) {
-    qts[p] = 0;
-    if (p < njobs) job_load<kGateUp>(a, make_job<kGateUp>(a, p, MT, KB, ntiles, dt), raw[p], qts[p]);
-  }
+      for (int w = 0; w < NW; ++w) {
+        raw_issue(ld[w], int(j % KB) * BK + half * 32, slot, w, dt);
+        qts[p][w] = ld[w].qtype;
+      }
+      odd[p] = ld_wrow & 1;
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+#pragma unroll
+  for (int p = 0; p < kRawDepth; ++p) issue(p, p);
   int s = 0;
   uint32_t ph = 0;
-  for (long long j0 = 0; j0 < njobs; j0 += kPD) {
+  for (long long j0 = 0; j0 < njobs; j0 += kRawDepth) {
 #pragma unroll
-    for (int p = 0; p < kPD; ++p) {
+    for (int p = 0; p < kRawDepth; ++p) {
       const long long j = j0 + p;
       if (j < njobs && !*abort_p) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(kRawDepth - 1) : "memory");
+        RawK raw[NW];
+        const uint8_t* slot = raw_smem + size_t(p) * kRawSlotBytes;
+        const int k0 = int(j % KB) * BK + half * 32;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) raw_read(slot, w, dt, qts[p][w], k0, odd[p] != 0, raw[w]);
         if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
           flag_error(a.hdr, MOE_ERR_TIMEOUT, 6000005);
           *abort_p = 1;
         } else {
 #pragma unroll
-          for (int w = 0; w < C::kATiles; ++w) {
+          for (int w = 0; w < NW; ++w) {
             uint4 o[4];
-            dequant32(qts[p], raw[p][w], o);
+            dequant32(qts[p][w], raw[w], o);
             uint8_t* tile = smem + size_t(s) * C::kStageBytes + size_t(w) * kTileBytes;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -369,15 +453,16 @@ __device__ void dequant_role(const Args& a, uint8_t* smem, uint64_t* full_bar, u
           __syncwarp();
           if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(ptx::smem_addr(&full_bar[s]));
         }
+        // refill this raw slot (its data is consumed: the dequant used the registers)
+        issue(j + kRawDepth, p);
         if (++s == C::kStages) {
           s = 0;
           ph ^= 1u;
         }
-        const long long jn = j + kPD;
-        if (jn < njobs) job_load<kGateUp>(a, make_job<kGateUp>(a, jn, MT, KB, ntiles, dt), raw[p], qts[p]);
       }
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 template <bool kGateUp>
@@ -518,27 +603,28 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * C::kAccCols);
       const int m = mt * BM + 32 * q + lane;  // weight row of this thread
-      for (int c0 = 0; c0 < nrows; c0 += 32) {
-        uint32_t v0[32];
-        ptx::tmem_ld32(taddr + uint32_t(c0), v0);
+      for (int c0 = 0; c0 < nrows; c0 += 16) {
+        uint32_t v0[16];
+        ptx::tmem_ld16(taddr + uint32_t(c0), v0);
         if (kGateUp) {
-          uint32_t v1[32];
-          ptx::tmem_ld32(taddr + 128u + uint32_t(c0), v1);
+          uint32_t v1[16];
+          ptx::tmem_ld16(taddr + 128u + uint32_t(c0), v1);
           ptx::tmem_ld_wait();
           // h = silu(g) * u -> fp16 into the H tiles (K index m of the down GEMM)
           uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
             if (n < nrows) {
               const float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]);
-              *reinterpret_cast<__half*>(base + tile_off(n, m & 63)) = __float2half_rn(sat_f16(silu_f32(gv) * uv));
+              *reinterpret_cast<__half*>(base + tile_off(n, m & 63)) =
+                  __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
             }
           }
         } else {
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
             if (n < nrows) {
               const float yv = __uint_as_float(v0[j]);
@@ -559,7 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
     }
   } else {
     // ------------------------------------------------ dequant producers
-    dequant_role<kGateUp>(a, smem, full_bar, empty_bar, abort_p, MT, KB, ntiles);
+    dequant_role<kGateUp>(a, smem, smem + size_t(C::kStages) * C::kStageBytes, full_bar, empty_bar, abort_p, MT, KB,
+                          ntiles);
   }
   __syncthreads();
   if (warp == 0) {
@@ -615,8 +702,8 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
 
   plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), plan);
   gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt);
-  const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + 1024;
-  const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + 1024;
+  const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
+  const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem_gu));
   if (e != cudaSuccess) return e;

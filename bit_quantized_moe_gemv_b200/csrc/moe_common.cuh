@@ -28,13 +28,15 @@ static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 
 // Offsets (bytes from the workspace base) of every workspace segment.
 struct WsLayout {
-  size_t counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, partial, h, shared_y, y_perm, gemm;
+  size_t counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, partial, h, shared_y, y_perm, gemm,
+      router;
   size_t total;
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared);
+size_t router_tc_ws_bytes(long long T, int H, int E);
 
 inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
   WsLayout L{};
@@ -55,6 +57,7 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   L.shared_y = take(4 * T * H);
   L.y_perm = take(4 * n * H);  // fp32 routed rows inside moe_layer
   L.gemm = take(grouped_ws_bytes(T, int(H), int(I), int(k), int(E), true));  // tcgen05 prefill scratch
+  L.router = take(router_tc_ws_bytes(T, int(H), int(E)));                   // tcgen05 router scratch
   L.total = o;
   return L;
 }

@@ -13,9 +13,16 @@ void count_launches(int n);
 
 enum TicketSlot { kTicketRoute = 0, kTicketDecodeRoute = 1, kTicketDecodeGateUp = 2 };
 
+// tc_scratch: workspace for the tensor-core router (router_tc_ws_bytes), used
+// for T > 4 when E is a multiple of 128.
 cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
-                         long long bstride, int k, int* topk_idx, float* topk_w, float* logits, WsHeader* hdr,
-                         cudaStream_t st);
+                         long long bstride, int k, int* topk_idx, float* topk_w, float* logits, void* tc_scratch,
+                         WsHeader* hdr, cudaStream_t st);
+
+bool router_tc_eligible(int T, int H, int E);
+size_t router_tc_ws_bytes(long long T, int H, int E);
+cudaError_t launch_router_tc(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
+                             long long bstride, float* logits, void* scratch, WsHeader* hdr, cudaStream_t st);
 
 // Blocks the multi-block dispatch uses for n = T*k pairs (1 = single-CTA path).
 int dispatch_blocks(long long n);

@@ -207,8 +207,8 @@ topk_rows_kernel(const float* __restrict__ logits, int T, int E, int k, int* __r
 
 // ---------------------------------------------------------------- launcher
 cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
-                         long long bstride, int k, int* topk_idx, float* topk_w, float* logits, WsHeader* hdr,
-                         cudaStream_t st) {
+                         long long bstride, int k, int* topk_idx, float* topk_w, float* logits, void* tc_scratch,
+                         WsHeader* hdr, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   if (T <= kGemvTmax) {
     const size_t smem = size_t(T) * H * sizeof(float);
@@ -223,10 +223,16 @@ cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E,
     count_launches(1);
     return cudaGetLastError();
   }
-  dim3 g((E + kRB - 1) / kRB, (T + kRB - 1) / kRB);
-  router_gemm_kernel<<<g, 256, 0, st>>>(x, T, H, W, E, bias, bstride, logits);
+  if (tc_scratch && router_tc_eligible(T, H, E)) {
+    cudaError_t e = launch_router_tc(x, T, H, W, E, bias, bstride, logits, tc_scratch, hdr, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    dim3 g((E + kRB - 1) / kRB, (T + kRB - 1) / kRB);
+    router_gemm_kernel<<<g, 256, 0, st>>>(x, T, H, W, E, bias, bstride, logits);
+    count_launches(1);
+  }
   topk_rows_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
-  count_launches(2);
+  count_launches(1);
   return cudaGetLastError();
 }
 

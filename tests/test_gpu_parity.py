@@ -56,6 +56,8 @@ SMALL = {
                              routed_qtypes=((0, 6, wlm.Q_INT4_SYM_G32), (6, 11, wlm.Q_INT2_ASYM_G16),
                                             (11, None, wlm.Q_INT8_PER_CHANNEL)),
                              shared_qtype=wlm.Q_INT8_PER_CHANNEL),
+    # E a multiple of 128 and T > 4: the tensor-core router (three-way bf16 split of W_r)
+    "tc_router": wlm.Workload("tc_router", T=300, H=512, I=256, E=128, k=4, zipf_s=0.9, seed=15),
     "tc_skew": wlm.Workload("tc_skew", T=1000, H=256, I=128, E=64, k=3, zipf_s=2.0, seed=14),
     "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
                               shared_qtype=wlm.Q_INT2_ASYM_G16),
