@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode1", choices=["decode1", "prefill8k", "prefill32k"])
+    ap.add_argument("--workload", default="decode1", choices=["decode1", "decode48", "prefill8k", "prefill32k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the CPU-baseline sample")
     return ap.parse_args()
@@ -269,6 +269,115 @@ def run_ours(args, rank, world, peaks, peak_kind):
     return line, wl, lay, bias
 
 
+def run_stack(args, rank, world, peaks, peak_kind):
+    """48-layer decode stack: one step = the step's 4 tokens (slots) through
+    all 48 layers, each layer with its own weights and fresh tokens (layers
+    are not chained, so every layer sees the specified routing). The whole
+    stack (58 GB) is resident and far larger than L2, so no flush is needed.
+    Weights are drawn on the device (workload.draw_layer_device)."""
+    import torch
+
+    from bit_quantized_moe_gemv_b200 import _lib as L
+    from bit_quantized_moe_gemv_b200.device import BlockExperts
+
+    wl = wlm.WORKLOADS[args.workload]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    NL, T, k, E, H, I = wl.layers, wl.T, wl.k, wl.E, wl.H, wl.I
+    layers, tables = [], []
+    for li in range(NL):
+        d = wlm.draw_layer_device(wl, li, device=dev)
+        layers.append(d)
+        tables.append((BlockExperts(d["qtype"], d["gu"], d["dn"], I, H, device=dev),
+                       BlockExperts(d["shared_qtype"], d["sgu"], d["sdn"], I, H, device=dev)))
+    bias, stride = wlm.gen_bias(wl)
+    b = torch.from_numpy(np.ascontiguousarray(bias)).to(dev)
+    n_steps = args.warmup + args.steps
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000003 * (rank + 1))
+    xs = torch.randn((n_steps, NL, T, H), dtype=torch.float32, device=dev, generator=g).to(torch.bfloat16)
+    idx = torch.empty((n_steps, NL, T, k), dtype=torch.int32, device=dev)
+    gw = torch.empty((n_steps, NL, T, k), dtype=torch.float32, device=dev)
+    out = torch.empty((n_steps, NL, T, H), dtype=torch.bfloat16, device=dev)
+    ws = L.new_workspace(T, H, I, E, k, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        for li in range(NL):
+            ex, sh = tables[li]
+            L.layer(xs[s, li], I, E, k, layers[li]["w_router"], b, stride, ex.table, sh.table, idx[s, li],
+                    gw[s, li], out[s, li], ws, stream=stream)
+
+    def timed_loop(first, count, host_io=None):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(count)]
+        for i in range(count):
+            s = first + i
+            evs[i][0].record(stream)
+            if host_io is not None:
+                xs[s].copy_(host_io[0][s], non_blocking=True)
+            step(s)
+            if host_io is not None:
+                host_io[1][s].copy_(out[s], non_blocking=True)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(z) for a, z in evs]
+
+    timed_loop(0, args.warmup)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    launches0 = L.launch_count()
+    times = timed_loop(args.warmup, args.steps)
+    launches = L.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
+    total_ms = float(np.sum(times))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    tokens_all = world * T * args.steps
+    value = tokens_all / (total_ms / 1e3)
+
+    xin = xs.cpu().pin_memory()
+    xout = torch.empty((n_steps, NL, T, H), dtype=torch.bfloat16).pin_memory()
+    e2e_ms = float(np.sum(timed_loop(args.warmup, args.steps, host_io=(xin, xout))))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    idx_h = idx[args.warmup:].cpu().numpy().reshape(args.steps, NL, T * k)
+    uniq = np.array([[len(np.unique(r)) for r in s] for s in idx_h])  # [steps, layers]
+    bytes_per_step = np.array([sum(wlm.per_token_layer_bytes(wl, u) for u in row) for row in uniq])
+    achieved_gbs = float(np.sum(bytes_per_step) / (np.sum(times) / 1e3) / 1e9)
+    peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; random weights of the stated architecture, drawn on the device)",
+        "config": dict(workload_config(wl, world), layers=NL,
+                       l2="inputs larger than L2 (58 GB stack streamed every step)"),
+        "roofline": {
+            "bound": "hbm", "kernel": "moe_layer x 48 layers (one launch per layer)",
+            "achieved": achieved_gbs, "peak": peak, "unit": "GB/s", "frac": achieved_gbs / peak,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_step": float(np.mean(bytes_per_step)),
+            "bytes_per_generated_token": float(np.mean(bytes_per_step)) / T,
+            "distinct_experts_per_layer_step": float(np.mean(uniq)),
+            "traffic": None,
+        },
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(NL * T * H * 2), "d2h_bytes_per_step": int(NL * T * H * 2)},
+        "gpu_launches": int(launches), "clocks": clk,
+    }
+    return line, wl, None, bias
+
+
 def run_prefill(args, rank, world, peaks, peak_kind):
     """Prefill workload: one step = moe_layer over all T tokens of one layer.
 
@@ -382,7 +491,7 @@ def main():
         budget = 150.0
         _, s_warm, _ = time_oracle(wl, lay, bias, args.warmup, budget / 4)
         tokens, secs, steps = time_oracle(wl, lay, bias, args.steps, budget, step_offset=args.warmup)
-        value = tokens / secs
+        value = tokens / secs / wl.layers  # a layer stack: layer 0 timed, every layer costs the same
         line = {
             "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True,
@@ -391,8 +500,9 @@ def main():
                            l2="flushed between steps (2 x L2 write, outside the timed events)"
                            if wl.T <= 4 else "inputs larger than L2 (1.36 GB of expert weights)"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                             "sample": f"{steps} of {args.steps} requested steps (1 token each), bounded to "
-                                       f"{budget:.0f} s"},
+                             "sample": f"{steps} of {args.steps} requested steps ({wl.T} token(s) each), bounded to "
+                                       f"{budget:.0f} s" + (f", layer 0 of {wl.layers} timed and scaled by "
+                                                             f"1/{wl.layers}" if wl.layers > 1 else "")},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
         print(json.dumps(line), flush=True)
@@ -407,13 +517,20 @@ def main():
         torch.cuda.set_device(0)
     if args.workload.startswith("prefill"):
         line, wl, lay, bias = run_prefill(args, rank, world, peaks, peak_kind)
+    elif wlm.WORKLOADS[args.workload].layers > 1:
+        line, wl, lay, bias = run_stack(args, rank, world, peaks, peak_kind)
     else:
         line, wl, lay, bias = run_ours(args, rank, world, peaks, peak_kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.workload.startswith("prefill"):
+        if lay is None:  # layer stack: time the oracle on layer 0 and scale to all layers
+            lay = wlm.gen_layer(wl, layer=0)
         tokens, secs, steps = time_oracle(wl, lay, bias, 10 ** 6, args.cpu_seconds, step_offset=10 ** 5)
-        line["cpu_baseline"] = {"value": tokens / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                                "sample": f"{steps} decode steps of 1 token through the fp64 oracle "
-                                          f"({secs:.1f} s)"}
+        per_layer = tokens / secs
+        line["cpu_baseline"] = {"value": per_layer / wl.layers, "unit": "tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{steps} layer-steps of {wl.T} token(s) through the fp64 oracle "
+                                          f"({secs:.1f} s)" + (f" on layer 0, scaled by 1/{wl.layers} layers"
+                                                               if wl.layers > 1 else "")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

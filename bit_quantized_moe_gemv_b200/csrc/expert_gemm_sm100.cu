@@ -49,8 +49,7 @@ namespace gemm {
 constexpr int BM = 128, BN = 128, BK = 64;
 constexpr int kTileBytes = BN * BK * 2;  // 16 KiB: one A or B tile
 constexpr int kThreads = 14 * 32;
-constexpr int kDqWarps = 8, kDqThreads = kDqWarps * 32;
-constexpr int kPD = 3;  // dequant global-load prefetch depth (k-blocks)
+constexpr int kDqWarps = 8;
 
 // ---------------------------------------------------------------- plan
 // Row tiles: every group (routed expert e < E, or the shared expert = E) is
@@ -65,7 +64,6 @@ struct Plan {
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
                                                     int E, int shared_rows, int max_tiles, Plan plan) {
-  __shared__ int base[kMaxE + 2];
   __shared__ int wsum[32];
   const int ngroups = E + (shared_rows > 0 ? 1 : 0);
   const int g = threadIdx.x;
@@ -90,8 +88,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     total += wsum[i];
   }
   const int excl = wb + incl - nt;
-  if (g < ngroups) base[g] = excl;
-  __syncthreads();
   if (g < ngroups) {
     const int n = g < E ? counts[g] : shared_rows;
     const int r0 = g < E ? offsets[g] : 0;
@@ -290,7 +286,7 @@ __device__ __forceinline__ const moe_qmatrix& pick(const moe_expert& e, int whic
 // One job = one k-block of one tile: 128 weight rows x 64 K of each A matrix.
 // Thread (row, half) of the 256 dequant threads handles 32 K elements of one
 // row. The tile's matrix pointers are resolved once per tile into registers;
-// global loads of the codes run kPD jobs ahead of the dequant.
+// the codes are staged in shared memory several k-blocks ahead.
 struct DqMat {
   const uint8_t* codes;   // start of this thread's row
   const uint16_t* scales; // start of this thread's row of scales (int8: &scale[row])

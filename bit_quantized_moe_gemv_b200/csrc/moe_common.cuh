@@ -53,7 +53,10 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   L.topk_w = take(4 * n);
   L.logits = take(4 * T * E);
   L.partial = take(16 * T * E);  // router partial sums of the fused decode path
-  L.h = take(4 * (n + T) * I);
+  // fp32 intermediate rows of the multi-launch path, or the decode step's fp16
+  // activations in fragment order: (T k + 1) buffers of I/16 k-steps x T x 32 B
+  const int64_t h32 = 4 * (n + T) * I, hfrag = T <= 4 ? (n + 1) * (I / 16) * T * 32 : 0;
+  L.h = take(size_t(h32 > hfrag ? h32 : hfrag));
   L.shared_y = take(4 * T * H);
   L.y_perm = take(4 * n * H);  // fp32 routed rows inside moe_layer
   L.gemm = take(grouped_ws_bytes(T, int(H), int(I), int(k), int(E), true));  // tcgen05 prefill scratch

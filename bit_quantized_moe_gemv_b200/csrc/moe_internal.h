@@ -38,12 +38,15 @@ cudaError_t launch_expert_ffn(const uint16_t* x, int T, int H, int I, int k, int
                               float* h_ws, int* active_ws, uint16_t* y_bf16, float* y_f32, WsHeader* hdr,
                               cudaStream_t st);
 
-// Fused single-launch decode step (T <= 4); see decode_fused.cu.
-bool decode_fused_eligible(int T, int H, int I, int E, int k);
-cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
-                                const float* bias, long long bstride, const moe_expert* experts,
-                                const moe_expert* shared, int* topk_idx, float* topk_w, uint16_t* out,
-                                float* partial, float* h, WsHeader* hdr, cudaStream_t st);
+// Decode step (T <= 4) as one persistent cooperative launch; see
+// decode_stream.cu. hfrag: decode_stream_hfrag_bytes of scratch for the
+// intermediate activations (fp16, in the order the down tiles read them).
+bool decode_stream_eligible(int T, int H, int I, int E, int k);
+size_t decode_stream_hfrag_bytes(int T, int I, int k);
+cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
+                                 const float* bias, long long bstride, const moe_expert* experts,
+                                 const moe_expert* shared, int* topk_idx, float* topk_w, uint16_t* out,
+                                 float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st);
 
 // Prefill experts on tcgen05 (expert_gemm_sm100.cu): plan, gather, gate/up
 // GEMM with SwiGLU epilogue, down GEMM. Routed rows go to y_f32 or y_bf16

@@ -21,9 +21,10 @@
 
 namespace {
 
-// Header (256 B) + router partials (4 T E floats) + intermediate rows
-// ((T k + T) I floats) at the limits T <= 4, E <= 1024, k <= 16, I <= 2048.
-constexpr size_t kNoAllocBytes = 640u * 1024u;
+// Header (256 B) + router partials (4 T E floats) + the intermediate
+// activations ((T k + 1) buffers of 2 T I bytes) at the limits T <= 4,
+// E <= 1024, k <= 16, I <= 2048.
+constexpr size_t kNoAllocBytes = 1280u * 1024u;
 constexpr int kNoAllocMaxT = 4, kNoAllocMaxE = 1024, kNoAllocMaxK = 16, kNoAllocMaxHI = 2048;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
@@ -61,7 +62,7 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
   if (T < 1 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (T > kNoAllocMaxT || E > kNoAllocMaxE || k > kNoAllocMaxK || H > kNoAllocMaxHI || I > kNoAllocMaxHI)
     return MOE_ERR_UNSUPPORTED;
-  if (!moe::decode_fused_eligible(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (!moe::decode_stream_eligible(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
   if (!x || !w_router || !experts_dev || !topk_idx || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   const uintptr_t misalign = (reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router) |
@@ -70,7 +71,7 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
 
   const size_t off_partial = 256;
   const size_t off_h = moe::align256(off_partial + 16u * size_t(T) * E);
-  const size_t total = off_h + 4u * size_t(T * k + T) * I;
+  const size_t total = off_h + moe::decode_stream_hfrag_bytes(T, I, k);
   if (total > kNoAllocBytes) return MOE_ERR_UNSUPPORTED;
 
   void* base = nullptr;
@@ -78,8 +79,8 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // The previous call's status and barrier words stay in the array: clear them.
   if (cudaMemsetAsync(base, 0, sizeof(moe::WsHeader), st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t e = moe::launch_decode_fused(
+  cudaError_t e = moe::launch_decode_stream(
       x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, out,
-      moe::ws_at<float>(base, off_partial), moe::ws_at<float>(base, off_h), moe::ws_at<moe::WsHeader>(base, 0), st);
+      moe::ws_at<float>(base, off_partial), moe::ws_at<void>(base, off_h), moe::ws_at<moe::WsHeader>(base, 0), st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

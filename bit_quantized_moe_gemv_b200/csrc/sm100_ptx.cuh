@@ -52,16 +52,30 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
       : "memory");
   return done != 0;
 }
-// Bounded wait; also gives up early when *abort becomes non-zero (checked
-// between suspended tries).
+// Non-blocking test of a phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Bounded wait; also gives up early when *abort becomes non-zero. Spins on
+// test_wait: a suspended try_wait resumed the warp too late to keep a
+// pipeline fed.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait_sleep(bar, parity)) {
-    if (abort && *abort) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (abort && *abort) return false;
+      if (clock64() - t0 > kWaitCycles) return false;
+    }
   }
-  return true;
 }
 
 // ---------------------------------------------------------------- bulk copies

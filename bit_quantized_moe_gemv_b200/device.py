@@ -85,3 +85,28 @@ def bf16_bits(t) -> np.ndarray:
 
 
 __all__ = ["DeviceExperts", "bf16_tensor", "bf16_bits", "Q_INT4_SYM_G32", "Q_INT2_ASYM_G16"]
+
+
+class BlockExperts:
+    """Descriptor table over experts whose matrices are slices of stacked
+    device tensors (as drawn by workload.draw_layer_device): gu = (codes,
+    scales, mins) shaped [n, 2, rows, ...] for gate/up, dn = [n, rows, ...]."""
+
+    def __init__(self, qtype, gu, dn, I, H, device="cuda"):
+        import torch
+        n = gu[0].shape[0]
+        arr = (_lib.ExpertC * n)()
+        g = qtype_group(qtype)
+        for i in range(n):
+            for name, j in (("gate", 0), ("up", 1), ("down", None)):
+                d = getattr(arr[i], name)
+                src = [t if t is None else (t[i, j] if j is not None else t[i]) for t in (gu if j is not None else dn)]
+                d.qtype, d.group = qtype, g
+                d.rows, d.cols = (I, H) if j is not None else (H, I)
+                d.codes = src[0].data_ptr()
+                d.scales = src[1].data_ptr()
+                d.mins = src[2].data_ptr() if src[2] is not None else None
+        self.n = n
+        self.keep = (gu, dn)
+        raw = np.frombuffer(bytes(arr), dtype=np.uint8).copy()
+        self.table = torch.from_numpy(raw).to(device)

@@ -244,3 +244,59 @@ def per_token_layer_bytes(wl: Workload, unique_experts: float | None = None) -> 
     routed = qmatrix_nbytes(wl.expert_qtype(0), wl.I, wl.H) * 2 + qmatrix_nbytes(wl.expert_qtype(0), wl.H, wl.I)
     shared = qmatrix_nbytes(wl.shared_qtype, wl.I, wl.H) * 2 + qmatrix_nbytes(wl.shared_qtype, wl.H, wl.I)
     return u * routed + shared + 4 * wl.E * wl.H
+
+
+# ------------------------------------------------------------------ device draws
+def _torch_seed(*parts) -> int:
+    h = hashlib.sha256(repr(parts).encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+def _draw_block(g, qtype: int, n: int, rows: int, cols: int, device):
+    """n packed [rows, cols] matrices of one qtype: (codes, scales, mins) with
+    the distributions of gen_qmatrix, drawn with torch generator g."""
+    import torch
+    bits = qtype_bits(qtype)
+    if qtype == Q_INT8_PER_CHANNEL:
+        q = torch.randint(-127, 128, (n, rows, cols), dtype=torch.int16, device=device, generator=g)
+        codes = q.to(torch.int8).view(torch.uint8)
+        scales = (torch.empty((n, rows), dtype=torch.float32, device=device).uniform_(0.005, 0.02, generator=g)
+                  / 16.0).to(torch.float16)
+        return codes, scales, None
+    codes = torch.randint(0, 256, (n, rows, cols * bits // 8), dtype=torch.int16, device=device,
+                          generator=g).to(torch.uint8)
+    ng = cols // qtype_group(qtype)
+    if qtype == Q_INT4_SYM_G32:
+        s = torch.empty((n, rows, ng), dtype=torch.float32, device=device).uniform_(0.005, 0.02, generator=g)
+        return codes, s.to(torch.float16), None
+    s = torch.empty((n, rows, ng), dtype=torch.float32, device=device).uniform_(0.01, 0.04, generator=g)
+    m = -s * torch.empty((n, rows, ng), dtype=torch.float32, device=device).uniform_(1.0, 2.0, generator=g)
+    return codes, s.to(torch.float16), m.to(torch.float16)
+
+
+def draw_layer_device(wl: Workload, layer: int, device="cuda") -> dict:
+    """One layer of `wl` drawn directly in device memory with a seeded torch
+    generator: the distributions of gen_layer, different numbers. For stacks
+    too large to draw on the host (48 layers of 512 experts are 58 GB).
+
+    All routed experts must share one qtype. Returns torch tensors:
+      w_router [E, H] fp32;
+      routed: gu = (codes [E, 2, I, .], scales, mins) for gate (index 0) and
+              up (index 1), dn = (codes [E, H, .], scales, mins);
+      shared: sgu, sdn (the same with a leading 1).
+    """
+    import torch
+    qs = {q for _, _, q in wl.routed_qtypes}
+    assert len(qs) == 1, "one routed qtype per drawn layer"
+    q = qs.pop()
+    g = torch.Generator(device=device)
+    g.manual_seed(_torch_seed(wl.seed, wl.name, "device_layer", layer))
+    out = {"qtype": q, "shared_qtype": wl.shared_qtype}
+    out["w_router"] = torch.randn((wl.E, wl.H), dtype=torch.float32, device=device, generator=g) * 0.02
+    c, s, m = _draw_block(g, q, 2 * wl.E, wl.I, wl.H, device)
+    out["gu"] = tuple(None if t is None else t.view(wl.E, 2, *t.shape[1:]) for t in (c, s, m))
+    out["dn"] = _draw_block(g, q, wl.E, wl.H, wl.I, device)
+    c, s, m = _draw_block(g, wl.shared_qtype, 2, wl.I, wl.H, device)
+    out["sgu"] = tuple(None if t is None else t.view(1, 2, *t.shape[1:]) for t in (c, s, m))
+    out["sdn"] = _draw_block(g, wl.shared_qtype, 1, wl.H, wl.I, device)
+    return out
