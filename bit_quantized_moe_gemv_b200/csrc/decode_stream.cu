@@ -371,47 +371,39 @@ __device__ __forceinline__ float key2f(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-__device__ __forceinline__ bool key_before(uint32_t k1, int i1, uint32_t k2, int i2) {
-  return k1 > k2 || (k1 == k2 && i1 < i2);
+// Best k (k <= 16) of up to 128 candidates held 4 per lane, each packed as
+// key << 32 | ~id so that a larger value is a better candidate (key desc, id
+// asc); 0 = no candidate. Each lane sorts its four (five compare-exchanges);
+// each of the k rounds takes the best lane head (a reduction on the key, one
+// on the low word among equal keys) and the winning lane pops it. A missing
+// pick reads key 0, id INT_MAX. One small instantiation: code that runs once
+// per launch pays an instruction-cache miss per line.
+__device__ __forceinline__ void cx(uint64_t& a, uint64_t& b) {
+  const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+  a = hi;
+  b = lo;
 }
-
-// Best `k` of the candidates held NPL per lane (key desc, id asc; missing
-// candidates have key 0 and id INT_MAX). Each lane sorts its own candidates;
-// each of the k rounds takes the best lane head (one reduction on the key, one
-// on the id among equal keys) and the winning lane pops its head. Writes k
-// (key, id) pairs; a missing pick reads key 0, id INT_MAX.
-template <int NPL>
-__device__ __forceinline__ void warp_topk(uint32_t (&kk)[NPL], int (&id)[NPL], int k, uint32_t* okey, int* oid) {
+__device__ __forceinline__ void warp_topk4(uint64_t (&c)[4], int k, uint32_t* okey, int* oid) {
   const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int r = 0; r < NPL; ++r)
-#pragma unroll
-    for (int i = r & 1; i + 1 < NPL; i += 2)
-      if (key_before(kk[i + 1], id[i + 1], kk[i], id[i])) {
-        const uint32_t tk = kk[i];
-        kk[i] = kk[i + 1];
-        kk[i + 1] = tk;
-        const int ti = id[i];
-        id[i] = id[i + 1];
-        id[i + 1] = ti;
-      }
+  cx(c[0], c[1]);
+  cx(c[2], c[3]);
+  cx(c[0], c[2]);
+  cx(c[1], c[3]);
+  cx(c[1], c[2]);
+#pragma unroll 1
   for (int j = 0; j < k; ++j) {
-    const uint32_t hk = kk[0];
-    const int hi = id[0];
-    const uint32_t wk = __reduce_max_sync(0xffffffffu, hk);
-    const uint32_t wi = __reduce_min_sync(0xffffffffu, hk == wk ? uint32_t(hi) : 0xffffffffu);
-    if (hk == wk && uint32_t(hi) == wi) {
-#pragma unroll
-      for (int i = 0; i + 1 < NPL; ++i) {
-        kk[i] = kk[i + 1];
-        id[i] = id[i + 1];
-      }
-      kk[NPL - 1] = 0u;
-      id[NPL - 1] = 0x7fffffff;
-    }
+    const uint32_t bk = uint32_t(c[0] >> 32), bl = uint32_t(c[0]);
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t wl = __reduce_max_sync(0xffffffffu, bk == wk ? bl : 0u);
     if (lane == 0) {
       okey[j] = wk;
-      oid[j] = int(wi);
+      oid[j] = wk ? int(~wl) : 0x7fffffff;
+    }
+    if (wk != 0u && bk == wk && bl == wl) {
+      c[0] = c[1];
+      c[1] = c[2];
+      c[2] = c[3];
+      c[3] = 0ull;
     }
   }
 }
@@ -969,71 +961,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
           }
         }
         consumer_sync();
-        const int TP = T == 1 ? 1 : T == 2 ? 2 : 4;
-        const int WPT = kCW / TP;  // warps per token
-        if (live) {
-          const int t = warp / WPT, wi = warp % WPT;
-          if (t < T) {
-            const int chunk = (E + WPT - 1) / WPT;
-            const int e0 = min(E, wi * chunk), e1 = min(E, e0 + chunk);
-            uint32_t* ok_ = s_ck + t * kCW * kMaxK + wi * k;
-            int* oi = s_ci + t * kCW * kMaxK + wi * k;
-            if (chunk <= 64) {
-              uint32_t kk[2];
-              int id[2];
+        // two rounds of warp top-k: first one job per (token, 128 logits), the
+        // jobs dealt over the warps, each keeping its chunk's best k; then one
+        // warp per token over those picks (at most 8 chunks x 16 = 128)
+        const int nch = (E + 127) >> 7;
+#pragma unroll 1
+        for (int stage = 0; stage < 2; ++stage) {
+          const int njobs = live ? (stage == 0 ? T * nch : T) : 0;
+#pragma unroll 1
+          for (int job = warp; job < njobs; job += kCW) {
+            const int t = stage == 0 ? job / nch : job, ch = stage == 0 ? job - t * nch : 0;
+            const int nc = stage == 0 ? min(128, E - (ch << 7)) : nch * k;
+            const uint32_t* ck = s_ck + t * kCW * kMaxK;
+            const int* ci = s_ci + t * kCW * kMaxK;
+            uint64_t cand[4];
 #pragma unroll
-              for (int i = 0; i < 2; ++i) {
-                const int e = e0 + lane + 32 * i;
-                kk[i] = e < e1 ? f2key(lg[t * E + e]) : 0u;
-                id[i] = e < e1 ? e : 0x7fffffff;
-              }
-              warp_topk<2>(kk, id, k, ok_, oi);
-            } else if (chunk <= 128) {
-              uint32_t kk[4];
-              int id[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int e = e0 + lane + 32 * i;
-                kk[i] = e < e1 ? f2key(lg[t * E + e]) : 0u;
-                id[i] = e < e1 ? e : 0x7fffffff;
-              }
-              warp_topk<4>(kk, id, k, ok_, oi);
-            } else if (chunk <= 256) {
-              uint32_t kk[8];
-              int id[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int e = e0 + lane + 32 * i;
-                kk[i] = e < e1 ? f2key(lg[t * E + e]) : 0u;
-                id[i] = e < e1 ? e : 0x7fffffff;
-              }
-              warp_topk<8>(kk, id, k, ok_, oi);
-            } else {
-              uint32_t kk[16];
-              int id[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int e = e0 + lane + 32 * i;
-                kk[i] = e < e1 ? f2key(lg[t * E + e]) : 0u;
-                id[i] = e < e1 ? e : 0x7fffffff;
-              }
-              warp_topk<16>(kk, id, k, ok_, oi);
+            for (int i = 0; i < 4; ++i) {
+              const int c = lane + 32 * i;
+              const uint32_t key = c >= nc ? 0u : stage == 0 ? f2key(lg[t * E + (ch << 7) + c]) : ck[c];
+              const int id = stage == 0 ? (ch << 7) + c : ci[c < nc ? c : 0];
+              cand[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(id)) : 0ull;
             }
+            uint32_t* okey = stage == 0 ? s_ck + t * kCW * kMaxK + ch * k : s_key + t * k;
+            int* oid = stage == 0 ? s_ci + t * kCW * kMaxK + ch * k : s_idx + t * k;
+            warp_topk4(cand, k, okey, oid);
           }
+          consumer_sync();
         }
-        consumer_sync();
         if (live && warp < T) {
           const int t = warp;
-          uint32_t kk[4];
-          int id[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = lane + 32 * i;
-            const bool v = c < WPT * k;
-            kk[i] = v ? s_ck[t * kCW * kMaxK + c] : 0u;
-            id[i] = v ? s_ci[t * kCW * kMaxK + c] : 0x7fffffff;
-          }
-          warp_topk<4>(kk, id, k, s_key + t * k, s_idx + t * k);
           __syncwarp();
           // renormalised softmax over the picks
           const float v0 = key2f(s_key[t * k]);
@@ -1190,19 +1146,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
         const Geo g = C.geo[dn * 4 + u.fmt];
         const int nch = g.cb / 16;
         const int c0 = warp * nch / kCW, c1 = (warp + 1) * nch / kCW;
-        if (dn) {
-          const uint8_t* frag = slot + g.bofs;
-          if (u.fmt == MOE_Q_INT4_SYM_G32) tile_mma<MOE_Q_INT4_SYM_G32, false>(slot, g, c0, c1, frag, 0, nullptr, T, acc);
-          else if (u.fmt == MOE_Q_INT2_ASYM_G16) tile_mma<MOE_Q_INT2_ASYM_G16, false>(slot, g, c0, c1, frag, 0, nullptr, T, acc);
-          else tile_mma<MOE_Q_INT8_PER_CHANNEL, false>(slot, g, c0, c1, frag, 0, nullptr, T, acc);
-        } else {
-          const int fb = s_fmap[u.fmt];
-          const uint8_t* frag = fb == 0 ? f0 : smem + L.o_x32 + (fb - 1) * 2 * T * H;
-          const int ks0 = u.k0 / 16;
-          if (u.fmt == MOE_Q_INT4_SYM_G32)
-            tile_mma<MOE_Q_INT4_SYM_G32, true>(slot, g, c0, c1, frag, ks0, corr + fb * (H / 32) * 4, T, acc);
-          else if (u.fmt == MOE_Q_INT2_ASYM_G16) tile_mma<MOE_Q_INT2_ASYM_G16, false>(slot, g, c0, c1, frag, ks0, nullptr, T, acc);
-          else tile_mma<MOE_Q_INT8_PER_CHANNEL, false>(slot, g, c0, c1, frag, ks0, nullptr, T, acc);
+        {  // one call site per instantiation (down tiles: activations in the slot)
+          const int fb = dn ? 0 : s_fmap[u.fmt];
+          const uint8_t* frag = dn ? slot + g.bofs : fb == 0 ? f0 : smem + L.o_x32 + (fb - 1) * 2 * T * H;
+          const int ks0 = dn ? 0 : u.k0 / 16;
+          if (u.fmt == MOE_Q_INT4_SYM_G32) {
+            if (dn) tile_mma<MOE_Q_INT4_SYM_G32, false>(slot, g, c0, c1, frag, 0, nullptr, T, acc);
+            else tile_mma<MOE_Q_INT4_SYM_G32, true>(slot, g, c0, c1, frag, ks0, corr + fb * (H / 32) * 4, T, acc);
+          } else if (u.fmt == MOE_Q_INT2_ASYM_G16) {
+            tile_mma<MOE_Q_INT2_ASYM_G16, false>(slot, g, c0, c1, frag, ks0, nullptr, T, acc);
+          } else {
+            tile_mma<MOE_Q_INT8_PER_CHANNEL, false>(slot, g, c0, c1, frag, ks0, nullptr, T, acc);
+          }
         }
         if (u.last) {
           // partials of this warp -> red; the last warp to arrive finishes the tile

@@ -25,15 +25,19 @@
 // image, so one 1-D bulk copy loads a B tile. Inside every 8-element group
 // the K order is (0,4,1,5,2,6,3,7): the order in which a byte-free lop3
 // unpacks eight int4 codes of one 32-bit word. Weights (A) are produced by
-// 8 dequant warps straight into the swizzled image in the same K order, so
-// the MMA's sum over K is unchanged. The gate/up epilogue writes H in the
-// same tiled form, which is the down GEMM's B operand.
+// 8 dequant warps in the same K order straight into TENSOR memory (one weight
+// row per TMEM lane, two fp16 per column; tcgen05.st), and the MMA reads A
+// from there: shared memory then carries only B (read by the MMA, written by
+// the bulk copies) and the staged raw codes, instead of also the dequantised
+// A tiles written once and read once per MMA. The gate/up epilogue writes H
+// in the tiled form the down GEMM reads as B.
 //
 // Warp roles (448 threads, one CTA per SM, persistent over the tile list):
 //   warp 0      bulk-copy producer of B tiles, TMEM allocation
 //   warp 1      MMA issuer (one thread)
 //   warps 2-5   epilogue (TMEM -> registers -> global)
-//   warps 6-13  dequant producers of A tiles
+//   warps 6-13  dequant producers of A (warp w writes TMEM lanes 32 (w % 4) ..
+//               + 31, i.e. weight rows, for half of each 64-wide k-block)
 // Every wait is bounded; an expired wait flags MOE_ERR_TIMEOUT, stops the
 // CTA's loops, drains what it issued and frees TMEM.
 #include <cuda_bf16.h>
@@ -268,13 +272,20 @@ constexpr int kRawCodeBytes = 2 * 2 * 256 * 16;  // [matrix][16-B unit][thread] 
 constexpr int kRawAuxBytes = 2 * 256 * 8;        // [matrix][thread] 8 B (scale / scales + mins)
 constexpr int kRawSlotBytes = kRawCodeBytes + kRawAuxBytes;
 
+// TMEM columns: accumulator buffers first (gate/up: gate 128 + up 128, one
+// buffer; down: 128, two buffers), then the A stages (64 K of one matrix =
+// 32 columns). gate/up: 256 + 3 x 64 = 448; down: 256 + 4 x 32 = 384.
 template <bool kGateUp>
 struct Cfg {
   static constexpr int kStages = kGateUp ? 3 : 4;
   static constexpr int kATiles = kGateUp ? 2 : 1;
-  static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
+  static constexpr int kStageBytes = kTileBytes;  // shared memory holds B only
+  static constexpr int kAccBufs = kGateUp ? 1 : 2;
   static constexpr int kAccCols = kGateUp ? 256 : 128;  // one accumulator buffer
-  static constexpr int kTmemCols = 2 * kAccCols;
+  static constexpr int kACol0 = kAccBufs * kAccCols;
+  static constexpr int kACols = 32 * kATiles;  // A columns per stage
+  static constexpr int kTmemCols = 512;
+  static_assert(kACol0 + kStages * kACols <= kTmemCols, "TMEM budget");
 };
 
 template <bool kGateUp>
@@ -377,20 +388,25 @@ __device__ __forceinline__ void raw_read(const uint8_t* slot, int w, int dt, int
 }
 
 template <bool kGateUp>
-__device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, uint64_t* full_bar,
+__device__ void dequant_role(const Args& a, uint32_t tmem, uint8_t* raw_smem, uint64_t* full_bar,
                              uint64_t* empty_bar, volatile int* abort_p, int MT, int KB, long long ntiles) {
   using C = Cfg<kGateUp>;
   constexpr int NW = kGateUp ? 2 : 1;
-  const int dt = threadIdx.x - 6 * 32;  // 0 .. 255
-  const int row = dt >> 1, half = dt & 1;
-  const long long per_cta = ntiles > blockIdx.x ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-  const long long njobs = per_cta * KB;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int dw = warp - 6;                  // 0 .. 7
+  const int q = warp & 3;                   // the TMEM lane quarter this warp may write
+  const int row = 32 * q + lane;            // weight row within the tile = TMEM lane
+  const int half = dw >> 2;                 // which 32 of the 64 K of a k-block
+  const int dt = dw * 32 + lane;            // raw-staging index, 0 .. 255
+  // 32-bit job counters and cursors: no division per job
+  const int per_cta = ntiles > blockIdx.x ? int((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  const int njobs = per_cta * KB;
   DqMat ld[NW];
-  long long ld_tile = -1;
+  int i_tile = -1, i_kb = KB - 1;  // issue cursor (local tile, k-block), one step before the first job
   int ld_wrow = 0;
-  auto resolve = [&](long long j) {
-    const long long t = blockIdx.x + (j / KB) * gridDim.x;
-    const int rt = int(t / MT), mt = int(t % MT);
+  auto resolve = [&](int lt) {
+    const int t = int(blockIdx.x) + lt * int(gridDim.x);
+    const int rt = t / MT, mt = t - rt * MT;
     const int g = a.plan.group[rt];
     const moe_expert* ex = g < a.E ? a.experts + g : a.shared;
     ld_wrow = mt * BM + row;
@@ -399,16 +415,16 @@ __device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, ui
   };
   int qts[kRawDepth][NW];
   int odd[kRawDepth];
-  auto issue = [&](long long j, int p) {
+  auto issue = [&](int j, int p) {
     if (j < njobs) {
-      if (j / KB != ld_tile) {
-        resolve(j);
-        ld_tile = j / KB;
+      if (++i_kb == KB) {
+        i_kb = 0;
+        resolve(++i_tile);
       }
       uint8_t* slot = raw_smem + size_t(p) * kRawSlotBytes;
 #pragma unroll
       for (int w = 0; w < NW; ++w) {
-        raw_issue(ld[w], int(j % KB) * BK + half * 32, slot, w, dt);
+        raw_issue(ld[w], i_kb * BK + half * 32, slot, w, dt);
         qts[p][w] = ld[w].qtype;
       }
       odd[p] = ld_wrow & 1;
@@ -419,15 +435,17 @@ __device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, ui
   for (int p = 0; p < kRawDepth; ++p) issue(p, p);
   int s = 0;
   uint32_t ph = 0;
-  for (long long j0 = 0; j0 < njobs; j0 += kRawDepth) {
+  int c_kb = 0;  // consume cursor: k-block of job j
+  for (int j0 = 0; j0 < njobs; j0 += kRawDepth) {
 #pragma unroll
     for (int p = 0; p < kRawDepth; ++p) {
-      const long long j = j0 + p;
+      const int j = j0 + p;
       if (j < njobs && !*abort_p) {
         asm volatile("cp.async.wait_group %0;" ::"n"(kRawDepth - 1) : "memory");
         RawK raw[NW];
         const uint8_t* slot = raw_smem + size_t(p) * kRawSlotBytes;
-        const int k0 = int(j % KB) * BK + half * 32;
+        const int k0 = c_kb * BK + half * 32;
+        if (++c_kb == KB) c_kb = 0;
 #pragma unroll
         for (int w = 0; w < NW; ++w) raw_read(slot, w, dt, qts[p][w], k0, odd[p] != 0, raw[w]);
         if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
@@ -438,14 +456,13 @@ __device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, ui
           for (int w = 0; w < NW; ++w) {
             uint4 o[4];
             dequant32(qts[p][w], raw[w], o);
-            uint8_t* tile = smem + size_t(s) * C::kStageBytes + size_t(w) * kTileBytes;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int chunk = 4 * half + c;
-              *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = o[c];
-            }
+            const uint32_t v[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
+                                    o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
+            ptx::tmem_st16(tmem + (uint32_t(32 * q) << 16) + uint32_t(C::kACol0 + s * C::kACols + 32 * w + 16 * half),
+                           v);
           }
-          ptx::fence_proxy_async_smem();
+          ptx::tmem_st_wait();
+          ptx::tc_fence_before();
           __syncwarp();
           if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(ptx::smem_addr(&full_bar[s]));
         }
@@ -502,8 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
     flag_error(a.hdr, MOE_ERR_TIMEOUT, where);
     *abort_p = 1;
   };
-  auto stage_a = [&](int s, int which) { return smem + size_t(s) * C::kStageBytes + size_t(which) * kTileBytes; };
-  auto stage_b = [&](int s) { return smem + size_t(s) * C::kStageBytes + size_t(C::kATiles) * kTileBytes; };
+  auto stage_b = [&](int s) { return smem + size_t(s) * C::kStageBytes; };
 
   if (warp == 0) {
     // ------------------------------------------------ B producer
@@ -540,8 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
         const int nrows = a.plan.nrows[rt];
         const int N = (nrows + 15) & ~15;
         const uint32_t idesc = ptx::idesc_f16(BM, N);
-        const int buf = it & 1;
-        const uint32_t use = uint32_t(it >> 1) & 1u;
+        const int buf = it % C::kAccBufs;
+        const uint32_t use = uint32_t(it / C::kAccBufs) & 1u;
         if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar[buf]), use ^ 1u, abort_p)) {
           fail(6000002);
           break;
@@ -556,17 +572,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t sa0 = ptx::smem_addr(stage_a(s, 0));
+          const uint32_t a0 = tmem + uint32_t(C::kACol0 + s * C::kACols);
           const uint32_t sb = ptx::smem_addr(stage_b(s));
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t bdesc = ptx::smem_desc_k128(sb + 32 * ks);
             const uint32_t acc = (kb | ks) != 0;
-            ptx::mma_f16(d0, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
-            if (kGateUp) {
-              const uint32_t sa1 = ptx::smem_addr(stage_a(s, 1));
-              ptx::mma_f16(d0 + 128, ptx::smem_desc_k128(sa1 + 32 * ks), bdesc, idesc, acc);
-            }
+            ptx::mma_f16_ts(d0, a0 + 8 * ks, bdesc, idesc, acc);
+            if (kGateUp) ptx::mma_f16_ts(d0 + 128, a0 + 32 + 8 * ks, bdesc, idesc, acc);
           }
           ptx::mma_commit(ptx::smem_addr(&empty_bar[s]));
           if (++s == C::kStages) {
@@ -590,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       const int nrows = a.plan.nrows[rt];
       const int g = a.plan.group[rt];
       const int row0 = a.plan.row0[rt];
-      const int buf = it & 1;
-      const uint32_t use = uint32_t(it >> 1) & 1u;
+      const int buf = it % C::kAccBufs;
+      const uint32_t use = uint32_t(it / C::kAccBufs) & 1u;
       if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar[buf]), use, abort_p)) {
         fail(6000004);
         break;
@@ -641,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
     }
   } else {
     // ------------------------------------------------ dequant producers
-    dequant_role<kGateUp>(a, smem, smem + size_t(C::kStages) * C::kStageBytes, full_bar, empty_bar, abort_p, MT, KB,
+    dequant_role<kGateUp>(a, tmem, smem + size_t(C::kStages) * C::kStageBytes, full_bar, empty_bar, abort_p, MT, KB,
                           ntiles);
   }
   __syncthreads();

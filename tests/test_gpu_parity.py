@@ -48,6 +48,9 @@ SMALL = {
     "fused_int4_T1": wlm.Workload("fused_int4_T1", T=1, H=1024, I=512, E=64, k=6, zipf_s=1.1, seed=8),
     "fused_int2_T4": wlm.Workload("fused_int2_T4", T=4, H=1536, I=512, E=24, k=5, seed=9,
                                   routed_qtypes=((0, None, wlm.Q_INT2_ASYM_G16),), shared_qtype=wlm.Q_INT4_SYM_G32),
+    # several router quarter-rows per CTA (E * H / 512 well above the SM count)
+    "fused_router_rows_T2": wlm.Workload("fused_router_rows_T2", T=2, H=1024, I=512, E=384, k=8, zipf_s=0.9,
+                                         seed=16),
     "small_mixed": _small_mixed(),
     "k_equals_E": wlm.Workload("k_equals_E", T=5, H=128, I=64, E=16, k=16, seed=4),
     # batches > 4 tokens with H, I multiples of 128 take the tcgen05 grouped GEMM
