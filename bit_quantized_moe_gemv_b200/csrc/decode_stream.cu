@@ -244,6 +244,11 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory"); }
 __device__ __forceinline__ bool test_wait(uint32_t bar, uint32_t parity) {
@@ -703,12 +708,22 @@ struct Producer {
     if (lane == 0) good = wait_empty(q);
     good = __shfl_sync(0xffffffffu, good, 0);
     if (!good) return false;
+    // The second barrier's count, loaded before the copies are issued and
+    // looked at after them, so its latency hides behind them: activations
+    // are due as soon as the barrier passes, not when a slot next runs out.
+    uint32_t seen = 0;
+    if (lane == 0 && !b2) seen = ld_relaxed_u32(&hdr->bar_count);
     const Unit u = C.units[q];
     issue_weights(C, u, C.slot(q));
     cp_arrive(C.full_bar(q));
     __syncwarp();
     if (lane == 0) {
       if (u.kind != kDown) ptx::mbar_arrive(C.full_bar(q));
+      if (!b2 && seen >= uint32_t(2 * G)) {
+        b2 = true;
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");  // the relaxed read above, made an acquire
+        fence_proxy_async_global();
+      }
       pump(q + 1);
     }
     return true;

@@ -25,19 +25,15 @@
 // image, so one 1-D bulk copy loads a B tile. Inside every 8-element group
 // the K order is (0,4,1,5,2,6,3,7): the order in which a byte-free lop3
 // unpacks eight int4 codes of one 32-bit word. Weights (A) are produced by
-// 8 dequant warps in the same K order straight into TENSOR memory (one weight
-// row per TMEM lane, two fp16 per column; tcgen05.st), and the MMA reads A
-// from there: shared memory then carries only B (read by the MMA, written by
-// the bulk copies) and the staged raw codes, instead of also the dequantised
-// A tiles written once and read once per MMA. The gate/up epilogue writes H
-// in the tiled form the down GEMM reads as B.
+// 8 dequant warps straight into the swizzled image in the same K order, so
+// the MMA's sum over K is unchanged. The gate/up epilogue writes H in the
+// same tiled form, which is the down GEMM's B operand.
 //
 // Warp roles (448 threads, one CTA per SM, persistent over the tile list):
 //   warp 0      bulk-copy producer of B tiles, TMEM allocation
 //   warp 1      MMA issuer (one thread)
 //   warps 2-5   epilogue (TMEM -> registers -> global)
-//   warps 6-13  dequant producers of A (warp w writes TMEM lanes 32 (w % 4) ..
-//               + 31, i.e. weight rows, for half of each 64-wide k-block)
+//   warps 6-13  dequant producers of A tiles
 // Every wait is bounded; an expired wait flags MOE_ERR_TIMEOUT, stops the
 // CTA's loops, drains what it issued and frees TMEM.
 #include <cuda_bf16.h>
@@ -54,21 +50,31 @@ constexpr int BM = 128, BN = 128, BK = 64;
 constexpr int kTileBytes = BN * BK * 2;  // 16 KiB: one A or B tile
 constexpr int kThreads = 14 * 32;
 constexpr int kDqWarps = 8;
+// A group with at least kHeavyRows rows (two or more row tiles) has its
+// weights dequantised once, into A tiles in global memory, which its GEMM
+// tiles then load like B instead of dequantising per row tile. At most
+// kMaxHeavy groups (the first ones in group order) take this path.
+constexpr int kHeavyRows = 2 * BN;
+constexpr int kMaxHeavy = 64;
 
 // ---------------------------------------------------------------- plan
 // Row tiles: every group (routed expert e < E, or the shared expert = E) is
 // cut into tiles of at most BN rows. For each tile: group, first row (a
-// dispatched row, or a token for the shared group) and row count.
+// dispatched row, or a token for the shared group) and row count. Heavy
+// groups get a slot of pre-dequantised weights (hslot[g], -1 for none).
 struct Plan {
-  int* count;   // [1] number of row tiles
+  int* count;   // [1] number of row tiles; [1] number of heavy slots used
   int* group;   // [max]
   int* row0;    // [max]
   int* nrows;   // [max]
+  int* hslot;   // [groups] heavy slot or -1
+  int* hlist;   // [heavy slots] group of each slot
 };
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
-                                                    int E, int shared_rows, int max_tiles, Plan plan) {
+                                                    int E, int shared_rows, int max_tiles, int max_heavy, Plan plan) {
   __shared__ int wsum[32];
+  __shared__ int hsum[32];
   const int ngroups = E + (shared_rows > 0 ? 1 : 0);
   const int g = threadIdx.x;
   int nt = 0;
@@ -92,6 +98,28 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     total += wsum[i];
   }
   const int excl = wb + incl - nt;
+  // heavy groups: slots in group order (a second block-wide scan)
+  const int hv = (g < ngroups && nt >= kHeavyRows / BN) ? 1 : 0;
+  int hincl = hv;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, hincl, o);
+    if (lane >= o) hincl += v;
+  }
+  if (lane == 31) hsum[w] = hincl;
+  __syncthreads();
+  int hb = 0, htotal = 0;
+  for (int i = 0; i < 32; ++i) {
+    if (i < w) hb += hsum[i];
+    htotal += hsum[i];
+  }
+  const int hslot = hb + hincl - hv;
+  if (g < ngroups) {
+    const bool heavy = hv && hslot < max_heavy;
+    plan.hslot[g] = heavy ? hslot : -1;
+    if (heavy) plan.hlist[hslot] = g;
+  }
+  if (g == 0) plan.count[1] = min(htotal, max_heavy);
   if (g < ngroups) {
     const int n = g < E ? counts[g] : shared_rows;
     const int r0 = g < E ? offsets[g] : 0;
@@ -248,6 +276,62 @@ __device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4
   }
 }
 
+// ---------------------------------------------------------------- heavy groups
+// Pre-dequantised weights of heavy slot h: the gate/up A tiles [I/128][H/64]
+// [gate, up], then the down A tiles [H/128][I/64]; each a 16 KiB tile laid
+// out exactly as the dequant warps write one into shared memory, so a GEMM
+// stage takes it with one bulk copy.
+__host__ __device__ inline size_t heavy_gu_bytes(int H, int I) { return size_t(2) * I * H * 2; }
+__host__ __device__ inline size_t heavy_slot_bytes(int H, int I) { return size_t(3) * I * H * 2; }
+
+__global__ void __launch_bounds__(256) predequant_kernel(const moe_expert* __restrict__ experts,
+                                                         const moe_expert* __restrict__ shared, int E, int H, int I,
+                                                         Plan plan, uint8_t* __restrict__ img, WsHeader* hdr) {
+  const int nslots = plan.count[1];
+  const int kbg = H / BK, kbd = I / BK;
+  const int gu_tiles = (I / BM) * kbg * 2, per_slot = gu_tiles + (H / BM) * kbd;
+  const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
+  for (int it = blockIdx.x; it < nslots * per_slot; it += gridDim.x) {
+    const int hs = it / per_slot, r = it - hs * per_slot;
+    const int g = plan.hlist[hs];
+    const moe_expert& ex = g < E ? experts[g] : *shared;
+    const moe_qmatrix* W;
+    int K, M, mt, kb;
+    size_t off;
+    if (r < gu_tiles) {  // r = (mt * kbg + kb) * 2 + (0 gate | 1 up)
+      const int q = r >> 1;
+      mt = q / kbg;
+      kb = q - mt * kbg;
+      W = (r & 1) ? &ex.up : &ex.gate;
+      K = H;
+      M = I;
+      off = size_t(r) * kTileBytes;
+    } else {  // down: q = mt * kbd + kb
+      const int q = r - gu_tiles;
+      mt = q / kbd;
+      kb = q - mt * kbd;
+      W = &ex.down;
+      K = I;
+      M = H;
+      off = heavy_gu_bytes(H, I) + size_t(q) * kTileBytes;
+    }
+    if (!qmatrix_ok(*W, M, K)) {
+      if (threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 7000001);
+      continue;
+    }
+    RawK raw;
+    load_raw(*W, mt * BM + row, kb * BK + half * 32, raw);
+    uint4 o[4];
+    dequant32(W->qtype, raw, o);
+    uint8_t* tile = img + size_t(hs) * heavy_slot_bytes(H, I) + off;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int chunk = 4 * half + c;
+      *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = o[c];
+    }
+  }
+}
+
 // ---------------------------------------------------------------- GEMM kernel
 struct Args {
   Plan plan;
@@ -262,6 +346,9 @@ struct Args {
   float* y_f32;       // down: fp32 rows out (routed rows), or nullptr
   uint16_t* y_bf16;   // down: bf16 rows out, or nullptr
   float* ys_f32;      // down: shared expert rows out (fp32 [T][H])
+  const uint8_t* aimg;  // pre-dequantised weights of the heavy slots
+  size_t aslot;         // bytes per heavy slot
+  size_t aoff;          // this GEMM's A tiles within a slot
   WsHeader* hdr;
 };
 
@@ -272,20 +359,13 @@ constexpr int kRawCodeBytes = 2 * 2 * 256 * 16;  // [matrix][16-B unit][thread] 
 constexpr int kRawAuxBytes = 2 * 256 * 8;        // [matrix][thread] 8 B (scale / scales + mins)
 constexpr int kRawSlotBytes = kRawCodeBytes + kRawAuxBytes;
 
-// TMEM columns: accumulator buffers first (gate/up: gate 128 + up 128, one
-// buffer; down: 128, two buffers), then the A stages (64 K of one matrix =
-// 32 columns). gate/up: 256 + 3 x 64 = 448; down: 256 + 4 x 32 = 384.
 template <bool kGateUp>
 struct Cfg {
   static constexpr int kStages = kGateUp ? 3 : 4;
   static constexpr int kATiles = kGateUp ? 2 : 1;
-  static constexpr int kStageBytes = kTileBytes;  // shared memory holds B only
-  static constexpr int kAccBufs = kGateUp ? 1 : 2;
+  static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
   static constexpr int kAccCols = kGateUp ? 256 : 128;  // one accumulator buffer
-  static constexpr int kACol0 = kAccBufs * kAccCols;
-  static constexpr int kACols = 32 * kATiles;  // A columns per stage
-  static constexpr int kTmemCols = 512;
-  static_assert(kACol0 + kStages * kACols <= kTmemCols, "TMEM budget");
+  static constexpr int kTmemCols = 2 * kAccCols;
 };
 
 template <bool kGateUp>
@@ -388,16 +468,12 @@ __device__ __forceinline__ void raw_read(const uint8_t* slot, int w, int dt, int
 }
 
 template <bool kGateUp>
-__device__ void dequant_role(const Args& a, uint32_t tmem, uint8_t* raw_smem, uint64_t* full_bar,
+__device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, uint64_t* full_bar,
                              uint64_t* empty_bar, volatile int* abort_p, int MT, int KB, long long ntiles) {
   using C = Cfg<kGateUp>;
   constexpr int NW = kGateUp ? 2 : 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dw = warp - 6;                  // 0 .. 7
-  const int q = warp & 3;                   // the TMEM lane quarter this warp may write
-  const int row = 32 * q + lane;            // weight row within the tile = TMEM lane
-  const int half = dw >> 2;                 // which 32 of the 64 K of a k-block
-  const int dt = dw * 32 + lane;            // raw-staging index, 0 .. 255
+  const int dt = threadIdx.x - 6 * 32;  // 0 .. 255
+  const int row = dt >> 1, half = dt & 1;
   // 32-bit job counters and cursors: no division per job
   const int per_cta = ntiles > blockIdx.x ? int((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
   const int njobs = per_cta * KB;
@@ -408,6 +484,12 @@ __device__ void dequant_role(const Args& a, uint32_t tmem, uint8_t* raw_smem, ui
     const int t = int(blockIdx.x) + lt * int(gridDim.x);
     const int rt = t / MT, mt = t - rt * MT;
     const int g = a.plan.group[rt];
+    if (a.plan.hslot[g] >= 0) {  // heavy: the producer copies this tile's A
+#pragma unroll
+      for (int w = 0; w < NW; ++w) ld[w] = DqMat{nullptr, nullptr, nullptr, 0};
+      ld_wrow = 0;
+      return;
+    }
     const moe_expert* ex = g < a.E ? a.experts + g : a.shared;
     ld_wrow = mt * BM + row;
     ld[0] = dq_mat(kGateUp ? ex->gate : ex->down, ld_wrow, a.M, a.K, a.hdr);
@@ -452,17 +534,20 @@ __device__ void dequant_role(const Args& a, uint32_t tmem, uint8_t* raw_smem, ui
           flag_error(a.hdr, MOE_ERR_TIMEOUT, 6000005);
           *abort_p = 1;
         } else {
+          if (qts[p][0] != 0) {  // qtype 0: a heavy tile (A copied in) or a flagged descriptor
 #pragma unroll
-          for (int w = 0; w < NW; ++w) {
-            uint4 o[4];
-            dequant32(qts[p][w], raw[w], o);
-            const uint32_t v[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
-                                    o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
-            ptx::tmem_st16(tmem + (uint32_t(32 * q) << 16) + uint32_t(C::kACol0 + s * C::kACols + 32 * w + 16 * half),
-                           v);
+            for (int w = 0; w < NW; ++w) {
+              uint4 o[4];
+              dequant32(qts[p][w], raw[w], o);
+              uint8_t* tile = smem + size_t(s) * C::kStageBytes + size_t(w) * kTileBytes;
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int chunk = 4 * half + c;
+                *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = o[c];
+              }
+            }
+            ptx::fence_proxy_async_smem();
           }
-          ptx::tmem_st_wait();
-          ptx::tc_fence_before();
           __syncwarp();
           if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(ptx::smem_addr(&full_bar[s]));
         }
@@ -519,7 +604,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
     flag_error(a.hdr, MOE_ERR_TIMEOUT, where);
     *abort_p = 1;
   };
-  auto stage_b = [&](int s) { return smem + size_t(s) * C::kStageBytes; };
+  auto stage_a = [&](int s, int which) { return smem + size_t(s) * C::kStageBytes + size_t(which) * kTileBytes; };
+  auto stage_b = [&](int s) { return smem + size_t(s) * C::kStageBytes + size_t(C::kATiles) * kTileBytes; };
 
   if (warp == 0) {
     // ------------------------------------------------ B producer
@@ -527,17 +613,23 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       int s = 0;
       uint32_t ph = 0;
       for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
-        const int rt = int(t / MT);
+        const int rt = int(t / MT), mt = int(t - (long long)rt * MT);
         const int nrows = a.plan.nrows[rt];
         const uint32_t bytes = uint32_t((nrows + 15) & ~15) * 128u;
+        const int hs = a.plan.hslot[a.plan.group[rt]];
+        const uint32_t abytes = hs >= 0 ? uint32_t(C::kATiles * kTileBytes) : 0u;
+        const uint8_t* asrc = hs >= 0 ? a.aimg + size_t(hs) * a.aslot + a.aoff + size_t(mt) * KB * abytes : nullptr;
         for (int kb = 0; kb < KB; ++kb) {
           if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
             fail(6000001);
             break;
           }
-          ptx::mbar_arrive_expect_tx(ptx::smem_addr(&full_bar[s]), bytes);
+          ptx::mbar_arrive_expect_tx(ptx::smem_addr(&full_bar[s]), bytes + abytes);
           ptx::bulk_g2s(ptx::smem_addr(stage_b(s)), a.bt + (size_t(rt) * KB + kb) * kTileBytes, bytes,
                         ptx::smem_addr(&full_bar[s]));
+          if (hs >= 0)
+            ptx::bulk_g2s(ptx::smem_addr(stage_a(s, 0)), asrc + size_t(kb) * abytes, abytes,
+                          ptx::smem_addr(&full_bar[s]));
           if (++s == C::kStages) {
             s = 0;
             ph ^= 1u;
@@ -556,8 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
         const int nrows = a.plan.nrows[rt];
         const int N = (nrows + 15) & ~15;
         const uint32_t idesc = ptx::idesc_f16(BM, N);
-        const int buf = it % C::kAccBufs;
-        const uint32_t use = uint32_t(it / C::kAccBufs) & 1u;
+        const int buf = it & 1;
+        const uint32_t use = uint32_t(it >> 1) & 1u;
         if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar[buf]), use ^ 1u, abort_p)) {
           fail(6000002);
           break;
@@ -572,14 +664,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a0 = tmem + uint32_t(C::kACol0 + s * C::kACols);
+          const uint32_t sa0 = ptx::smem_addr(stage_a(s, 0));
           const uint32_t sb = ptx::smem_addr(stage_b(s));
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t bdesc = ptx::smem_desc_k128(sb + 32 * ks);
             const uint32_t acc = (kb | ks) != 0;
-            ptx::mma_f16_ts(d0, a0 + 8 * ks, bdesc, idesc, acc);
-            if (kGateUp) ptx::mma_f16_ts(d0 + 128, a0 + 32 + 8 * ks, bdesc, idesc, acc);
+            ptx::mma_f16(d0, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
+            if (kGateUp) {
+              const uint32_t sa1 = ptx::smem_addr(stage_a(s, 1));
+              ptx::mma_f16(d0 + 128, ptx::smem_desc_k128(sa1 + 32 * ks), bdesc, idesc, acc);
+            }
           }
           ptx::mma_commit(ptx::smem_addr(&empty_bar[s]));
           if (++s == C::kStages) {
@@ -603,8 +698,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       const int nrows = a.plan.nrows[rt];
       const int g = a.plan.group[rt];
       const int row0 = a.plan.row0[rt];
-      const int buf = it % C::kAccBufs;
-      const uint32_t use = uint32_t(it / C::kAccBufs) & 1u;
+      const int buf = it & 1;
+      const uint32_t use = uint32_t(it >> 1) & 1u;
       if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar[buf]), use, abort_p)) {
         fail(6000004);
         break;
@@ -654,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
     }
   } else {
     // ------------------------------------------------ dequant producers
-    dequant_role<kGateUp>(a, tmem, smem + size_t(C::kStages) * C::kStageBytes, full_bar, empty_bar, abort_p, MT, KB,
+    dequant_role<kGateUp>(a, smem, smem + size_t(C::kStages) * C::kStageBytes, full_bar, empty_bar, abort_p, MT, KB,
                           ntiles);
   }
   __syncthreads();
@@ -680,10 +775,20 @@ bool grouped_eligible(int H, int I, int E, bool with_shared) {
   return (H % 128) == 0 && (I % 128) == 0 && H <= 16384 && I <= 16384 && E + (with_shared ? 1 : 0) <= 1024;
 }
 
+// Heavy slots a launch may use: routed groups with at least kHeavyRows rows
+// (at most T k / kHeavyRows of them) plus the shared group when T is that
+// large, capped at kMaxHeavy.
+int grouped_heavy_slots(long long T, int k, bool with_shared) {
+  const long long n = T * k / gemm::kHeavyRows + ((with_shared && T >= gemm::kHeavyRows) ? 1 : 0);
+  return int(n < gemm::kMaxHeavy ? n : gemm::kMaxHeavy);
+}
+
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
   const long long mt = grouped_max_tiles(T, k, E, with_shared);
-  return align256(16 * size_t(mt) + 16) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
-         align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes);
+  return align256(16 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
+         align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
+         align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes) +
+         align256(size_t(grouped_heavy_slots(T, k, with_shared)) * gemm::heavy_slot_bytes(H, I));
 }
 
 cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, int E, const int* perm_src,
@@ -701,16 +806,23 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   plan.row0 = plan.group + mt;
   plan.nrows = plan.row0 + mt;
   p += align256(16 * size_t(mt) + 16);
+  plan.hslot = reinterpret_cast<int*>(p);
+  plan.hlist = plan.hslot + (E + 1);
+  p += align256(4 * size_t(E + 1) + 4 * size_t(kMaxHeavy));
   uint8_t* xt = p;
   p += align256(size_t(mt) * (H / BK) * kTileBytes);
   uint8_t* ht = p;
+  p += align256(size_t(mt) * (I / BK) * kTileBytes);
+  uint8_t* aimg = p;
+  const int max_heavy = grouped_heavy_slots(T, k, with_shared);
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
-  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), plan);
+  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), max_heavy, plan);
   gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt);
+  if (max_heavy > 0) predequant_kernel<<<sms * 4, 256, 0, st>>>(experts, shared, E, H, I, plan, aimg, hdr);
   const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
   const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -726,22 +838,26 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.I = I;
   a.H = H;
   a.hdr = hdr;
+  a.aimg = aimg;
+  a.aslot = heavy_slot_bytes(H, I);
   // gate/up: K = H, M = I; B = gathered X tiles; out = H tiles
   a.K = H;
   a.M = I;
   a.bt = xt;
   a.ht = ht;
+  a.aoff = 0;
   grouped_gemm_kernel<true><<<sms, kThreads, smem_gu, st>>>(a);
   // down: K = I, M = H; B = H tiles; out = rows
   a.K = I;
   a.M = H;
   a.bt = ht;
   a.ht = nullptr;
+  a.aoff = heavy_gu_bytes(H, I);
   a.y_f32 = y_f32;
   a.y_bf16 = y_bf16;
   a.ys_f32 = ys_f32;
   grouped_gemm_kernel<false><<<sms, kThreads, smem_dn, st>>>(a);
-  count_launches(4);
+  count_launches(max_heavy > 0 ? 5 : 4);
   return cudaGetLastError();
 }
 
