@@ -39,6 +39,21 @@ from bit_quantized_moe_gemv_b200 import workload as wlm  # noqa: E402
 METRIC = "MoE-layer tokens/s (decode b=1..4, 8K prefill); % of HBM / tensor roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per launch of the dominant kernel(s), from the ncu
+# captures summarised in profiles/ (set to None when the kernel changes).
+NCU_TRAFFIC = {
+    # decode_stream_kernel, mean of two captured launches
+    "decode1": (33618944, "profiles/decode_stream_decode1.md"),
+    # predequant_kernel + grouped_gemm_kernel<gate/up> + <down> of one step
+    # (the gather of the activations is not included)
+    "prefill8k": (3016913736, "profiles/grouped_gemm_prefill8k.md"),
+}
+
+
+def ncu_traffic(workload):
+    t = NCU_TRAFFIC.get(workload)
+    return (t[0], t[1]) if t else (None, None)
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -257,7 +272,8 @@ def run_ours(args, rank, world, peaks, peak_kind):
             "frac": achieved_gbs / peak,
             "peak_source": f"{peak_kind} hbm_gbs",
             "algorithmic_bytes_per_step": float(np.mean(bytes_per_step)),
-            "traffic": None,
+            "traffic": ncu_traffic(args.workload)[0],
+            "traffic_source": ncu_traffic(args.workload)[1],
         },
         "warm_l2": {"ms_per_step": float(np.mean(warm)), "note": "context only, weights partly L2-resident"},
         "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -467,7 +483,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
         "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (gather + tcgen05 gate/up + down)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops, "ms_per_launch": ffn_ms,
-                     "traffic": None},
+                     "traffic": ncu_traffic(args.workload)[0], "traffic_source": ncu_traffic(args.workload)[1]},
         "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(T * H * 2), "d2h_bytes_per_step": int(T * H * 2)},
         "gpu_launches": int(launches), "clocks": clk,
