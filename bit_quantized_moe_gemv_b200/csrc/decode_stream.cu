@@ -49,7 +49,8 @@ namespace moe {
 namespace dks {
 
 constexpr int kCW = 8;                    // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;  // plus the producer warp
+constexpr int kProducers = 2;             // producer warps: unit q is issued by warp kCW + q % kProducers
+constexpr int kThreads = (kCW + kProducers) * 32;
 constexpr int kProducer = kCW;
 constexpr int kMaxT = 4;
 constexpr int kMaxK = 16;
@@ -661,6 +662,7 @@ struct Producer {
   const Ctx& C;
   WsHeader* hdr;
   int G;
+  int p;  // this producer's units are those with q % kProducers == p
   int bq = 0;       // next unit whose activations may still be due
   bool b1 = false;  // barrier 1 passed (shared down activations exist)
   bool b2 = false;  // barrier 2 passed (routed down activations exist)
@@ -669,7 +671,7 @@ struct Producer {
   __device__ __forceinline__ void pump(int issued) {
     while (bq < issued) {
       const Unit& u = C.units[bq];
-      if (u.kind == kDown) {
+      if (bq % kProducers == p && u.kind == kDown) {
         const bool ready = u.e == C.kShared ? b1 : b2;
         if (!ready) break;
         issue_acts(C, u, C.slot(bq), C.full_bar(bq));
@@ -815,7 +817,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
   if (threadIdx.x < kMaxSlots) s_cnt[threadIdx.x] = 0;
 
   // ---------------------------------------------------------- start
-  if (warp == kProducer) {
+  if (warp > kProducer) {
+    // the second producer warp has nothing to do before S1
+  } else if (warp == kProducer) {
     // mbarriers, then the router loads before anything else (the consumers
     // list the same units in the same order).
     if (lane == 0) {
@@ -874,15 +878,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
   __syncthreads();  // S1: phase-A list ready
   const int nA = s_nA, nSD = s_nSD;
 
-  if (warp == kProducer) {
-    // ------------------------------------------------ producer: one pass over all units
-    Producer PR{C, hdr, G};
-    int q = nR < C.S ? nR : C.S;
+  if (warp >= kProducer) {
+    // ------------------------------------------------ producers: unit q is issued by warp kCW + q % kProducers
+    // (the slot count is a multiple of kProducers, so each slot is only ever
+    // filled by one producer warp, in order: a slot's phases never run more
+    // than one ahead of its producer's waits)
+    const int pw = warp - kProducer;
+    Producer PR{C, hdr, G, pw};
+    const int q0 = nR < C.S ? nR : C.S;
+    int q = q0 + (pw - q0 % kProducers + kProducers) % kProducers;  // the first own unit from q0 on
     int total = nA + nSD;
-    bool ok = true;
-    for (;; ++q) {
-      if (q == nA + nSD) {
+    bool ok = true, s2 = false;
+    for (;; q += kProducers) {
+      if (!s2 && q >= nA + nSD) {
         __syncthreads();  // S2: routed lists ready, barrier 1 passed
+        s2 = true;
         total = nA + nSD + s_nB + s_nC;
         if (lane == 0) {
           fence_proxy_async_global();
@@ -1271,7 +1281,8 @@ int units_bound(int T, int H, int I, int E, int k, int G, int nper, int RQ) {
 }
 
 int pick_slots(int T, int H, int E, int k) {
-  for (int s = kMaxSlots; s >= 4; --s)
+  // a multiple of kProducers: each slot has one producer warp
+  for (int s = kMaxSlots - kMaxSlots % kProducers; s >= 4 && s >= kProducers; s -= kProducers)
     if (make_plan(T, H, E, k, s).total + kStaticSmem <= kSmemLimit) return s;
   return 0;
 }
