@@ -284,50 +284,69 @@ __device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4
 __host__ __device__ inline size_t heavy_gu_bytes(int H, int I) { return size_t(2) * I * H * 2; }
 __host__ __device__ inline size_t heavy_slot_bytes(int H, int I) { return size_t(3) * I * H * 2; }
 
+// One CTA of 256 threads per group of kPD tiles; thread (row, half) takes 32
+// K of one row of each tile. All kPD loads of a thread are issued before any
+// dequantisation, so they are in flight together.
+constexpr int kPD = 4;
 __global__ void __launch_bounds__(256) predequant_kernel(const moe_expert* __restrict__ experts,
                                                          const moe_expert* __restrict__ shared, int E, int H, int I,
                                                          Plan plan, uint8_t* __restrict__ img, WsHeader* hdr) {
   const int nslots = plan.count[1];
   const int kbg = H / BK, kbd = I / BK;
   const int gu_tiles = (I / BM) * kbg * 2, per_slot = gu_tiles + (H / BM) * kbd;
+  const int n = nslots * per_slot;
   const int row = threadIdx.x >> 1, half = threadIdx.x & 1;
-  for (int it = blockIdx.x; it < nslots * per_slot; it += gridDim.x) {
-    const int hs = it / per_slot, r = it - hs * per_slot;
-    const int g = plan.hlist[hs];
-    const moe_expert& ex = g < E ? experts[g] : *shared;
-    const moe_qmatrix* W;
-    int K, M, mt, kb;
-    size_t off;
-    if (r < gu_tiles) {  // r = (mt * kbg + kb) * 2 + (0 gate | 1 up)
-      const int q = r >> 1;
-      mt = q / kbg;
-      kb = q - mt * kbg;
-      W = (r & 1) ? &ex.up : &ex.gate;
-      K = H;
-      M = I;
-      off = size_t(r) * kTileBytes;
-    } else {  // down: q = mt * kbd + kb
-      const int q = r - gu_tiles;
-      mt = q / kbd;
-      kb = q - mt * kbd;
-      W = &ex.down;
-      K = I;
-      M = H;
-      off = heavy_gu_bytes(H, I) + size_t(q) * kTileBytes;
-    }
-    if (!qmatrix_ok(*W, M, K)) {
-      if (threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 7000001);
-      continue;
-    }
-    RawK raw;
-    load_raw(*W, mt * BM + row, kb * BK + half * 32, raw);
-    uint4 o[4];
-    dequant32(W->qtype, raw, o);
-    uint8_t* tile = img + size_t(hs) * heavy_slot_bytes(H, I) + off;
+  for (int it0 = blockIdx.x * kPD; it0 < n; it0 += gridDim.x * kPD) {
+    RawK raw[kPD];
+    int qt[kPD];
+    uint8_t* tile[kPD];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int chunk = 4 * half + c;
-      *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = o[c];
+    for (int j = 0; j < kPD; ++j) {
+      qt[j] = 0;
+      tile[j] = nullptr;
+      const int it = it0 + j;
+      if (it >= n) continue;
+      const int hs = it / per_slot, r = it - hs * per_slot;
+      const int g = plan.hlist[hs];
+      const moe_expert& ex = g < E ? experts[g] : *shared;
+      const moe_qmatrix* W;
+      int K, M, mt, kb;
+      size_t off;
+      if (r < gu_tiles) {  // r = (mt * kbg + kb) * 2 + (0 gate | 1 up)
+        const int q = r >> 1;
+        mt = q / kbg;
+        kb = q - mt * kbg;
+        W = (r & 1) ? &ex.up : &ex.gate;
+        K = H;
+        M = I;
+        off = size_t(r) * kTileBytes;
+      } else {  // down: q = mt * kbd + kb
+        const int q = r - gu_tiles;
+        mt = q / kbd;
+        kb = q - mt * kbd;
+        W = &ex.down;
+        K = I;
+        M = H;
+        off = heavy_gu_bytes(H, I) + size_t(q) * kTileBytes;
+      }
+      if (!qmatrix_ok(*W, M, K)) {
+        if (threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 7000001);
+        continue;
+      }
+      load_raw(*W, mt * BM + row, kb * BK + half * 32, raw[j]);
+      qt[j] = W->qtype;
+      tile[j] = img + size_t(hs) * heavy_slot_bytes(H, I) + off;
+    }
+#pragma unroll
+    for (int j = 0; j < kPD; ++j) {
+      if (tile[j] == nullptr) continue;
+      uint4 o[4];
+      dequant32(qt[j], raw[j], o);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int chunk = 4 * half + c;
+        *reinterpret_cast<uint4*>(tile[j] + row * 128 + ((chunk ^ (row & 7)) << 4)) = o[c];
+      }
     }
   }
 }
