@@ -485,12 +485,17 @@ __device__ __forceinline__ void copy_rows(uint32_t dst, int stride, int rows, in
 }
 
 // Producer warp: the weight copies of unit u into its slot.
-__device__ __forceinline__ void issue_weights(const Ctx& C, const Unit& u, uint8_t* slot) {
+__device__ __forceinline__ void issue_weights(const Ctx& C, const Unit& u, uint8_t* slot, uint32_t bar) {
   const Params& P = *C.P;
   const uint32_t base = ptx::smem_addr(slot);
   if (u.kind == kRouter) {
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(P.w_router + size_t(u.row0) * C.KP);
-    copy_rows(base, C.KP * 4, u.nrows, C.KP * 4, src, src, 16, size_t(C.KP) * 4);
+    // consecutive quarter-rows are one contiguous run: one bulk copy, and
+    // lane 0's arrival on the slot carries its byte count
+    if ((threadIdx.x & 31) == 0) {
+      const uint32_t bytes = uint32_t(u.nrows * C.KP * 4);
+      ptx::mbar_arrive_expect_tx(bar, bytes);
+      ptx::bulk_g2s(base, P.w_router + size_t(u.row0) * C.KP, bytes, bar);
+    }
     return;
   }
   const bool gu = u.kind == kGateUp;
@@ -716,11 +721,11 @@ struct Producer {
     uint32_t seen = 0;
     if (lane == 0 && !b2) seen = ld_relaxed_u32(&hdr->bar_count);
     const Unit u = C.units[q];
-    issue_weights(C, u, C.slot(q));
+    issue_weights(C, u, C.slot(q), C.full_bar(q));
     cp_arrive(C.full_bar(q));
     __syncwarp();
     if (lane == 0) {
-      if (u.kind != kDown) ptx::mbar_arrive(C.full_bar(q));
+      if (u.kind == kGateUp) ptx::mbar_arrive(C.full_bar(q));  // router: arrived with its copy
       if (!b2 && seen >= uint32_t(2 * G)) {
         b2 = true;
         asm volatile("fence.acq_rel.gpu;" ::: "memory");  // the relaxed read above, made an acquire
@@ -832,10 +837,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
     __syncwarp();
     for (int i = 0; i < nR && i < C.S; ++i) {
       const Unit u = router_unit(C, u0, u1, i);
-      issue_weights(C, u, C.slot(i));
+      issue_weights(C, u, C.slot(i), C.full_bar(i));
       cp_arrive(C.full_bar(i));
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(C.full_bar(i));
+      // (router units: lane 0 arrived with the copy's byte count)
     }
   } else {
     if (threadIdx.x == 32) {  // the routed descriptors into L2 for after the top-k
