@@ -733,32 +733,35 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           uint32_t v1[16];
           ptx::tmem_ld16(taddr + 128u + uint32_t(c0), v1);
           ptx::tmem_ld_wait();
-          // h = silu(g) * u -> fp16 into the H tiles (K index m of the down GEMM)
-          uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes;
+          // h = silu(g) * u -> fp16 into the H tiles (K index m of the down GEMM),
+          // at tile_off(c0 + j, m & 63): c0 is a multiple of 16, so the row's
+          // swizzle term (row & 7) is j & 7 and the offsets are c0 * 128 plus
+          // constants of j
+          const int kc = (m & 63) >> 3, e = m & 7;
+          uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes + size_t(c0) * 128 +
+                          (e < 4 ? 4 * e : 4 * (e - 4) + 2);
+          const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < nrows) {
+            if (j < nv) {
               const float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]);
-              *reinterpret_cast<__half*>(base + tile_off(n, m & 63)) =
+              *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) =
                   __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
             }
           }
         } else {
           ptx::tmem_ld_wait();
+          const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+          if (g < a.E && a.y_f32 == nullptr) {
+            uint16_t* yp = a.y_bf16 + size_t(row0 + c0) * a.H + m;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < nrows) {
-              const float yv = __uint_as_float(v0[j]);
-              if (g < a.E) {
-                const size_t o = size_t(row0 + n) * a.H + m;
-                if (a.y_f32) a.y_f32[o] = yv;
-                else a.y_bf16[o] = f32_to_bf16_rn(yv);
-              } else {
-                a.ys_f32[size_t(row0 + n) * a.H + m] = yv;
-              }
-            }
+            for (int j = 0; j < 16; ++j)
+              if (j < nv) yp[size_t(j) * a.H] = f32_to_bf16_rn(__uint_as_float(v0[j]));
+          } else {  // fp32 rows: column m of rows row0 + c0 .. (one pointer step of H per row)
+            float* yp = (g < a.E ? a.y_f32 : a.ys_f32) + size_t(row0 + c0) * a.H + m;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < nv) yp[size_t(j) * a.H] = __uint_as_float(v0[j]);
           }
         }
       }
