@@ -50,6 +50,17 @@ NCU_TRAFFIC = {
 }
 
 
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks: a job's time is its slowest
+    rank's (collective on the ranks' process group; a no-op at N = 1)."""
+    if world <= 1:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def ncu_traffic(workload):
     t = NCU_TRAFFIC.get(workload)
     return (t[0], t[1]) if t else (None, None)
@@ -221,10 +232,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
 
     total_ms = float(np.sum(times))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     tokens_all = world * wl.T * args.steps
     value = tokens_all / (total_ms / 1e3)
 
@@ -237,10 +245,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
     xout_t = torch.empty((n_steps, wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
     e2e_times = timed_loop(args.warmup, args.steps, host_io=(xin_t, xout_t))
     e2e_ms = float(np.sum(e2e_times))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     # algorithmic bytes per step: distinct routed experts + shared + router
     idx_h = idx[args.warmup:].cpu().numpy()
@@ -351,20 +356,14 @@ def run_stack(args, rank, world, peaks, peak_kind):
     clk = clocks.stop() if clocks else None
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
     total_ms = float(np.sum(times))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     tokens_all = world * T * args.steps
     value = tokens_all / (total_ms / 1e3)
 
     xin = xs.cpu().pin_memory()
     xout = torch.empty((n_steps, NL, T, H), dtype=torch.bfloat16).pin_memory()
     e2e_ms = float(np.sum(timed_loop(args.warmup, args.steps, host_io=(xin, xout))))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     idx_h = idx[args.warmup:].cpu().numpy().reshape(args.steps, NL, T * k)
     uniq = np.array([[len(np.unique(r)) for r in s] for s in idx_h])  # [steps, layers]
@@ -444,10 +443,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
     clk = clocks.stop() if clocks else None
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
     total_ms = float(np.sum(times))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     value = world * T * args.steps / (total_ms / 1e3)
 
     # expert FFN alone (routed experts), on the routing of the last step
@@ -473,7 +469,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
         step()
         xout.copy_(out, non_blocking=True)
 
-    e2e_ms = float(np.sum(timed(e2e_step, args.steps)))
+    e2e_ms = max_over_ranks(float(np.sum(timed(e2e_step, args.steps))), world, dev)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
