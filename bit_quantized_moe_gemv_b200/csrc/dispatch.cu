@@ -89,7 +89,18 @@ dispatch_scan_kernel(int nblocks, int E, int* __restrict__ hist, int* __restrict
   __shared__ int tmp[kDW];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
-    for (int b = 0; b < nblocks; ++b) {
+    int b = 0;
+    for (; b + 8 <= nblocks; b += 8) {  // eight loads in flight, then the running sum
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = hist[size_t(b + i) * E + e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        hist[size_t(b + i) * E + e] = run;
+        run += v[i];
+      }
+    }
+    for (; b < nblocks; ++b) {
       const int v = hist[size_t(b) * E + e];
       hist[size_t(b) * E + e] = run;
       run += v;

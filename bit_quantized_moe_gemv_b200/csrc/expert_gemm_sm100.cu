@@ -373,14 +373,14 @@ struct Args {
 
 // Raw-code staging: each dequant thread copies (cp.async) its own codes and
 // scales kRawDepth k-blocks ahead into a private area of shared memory.
-constexpr int kRawDepth = 4;
+constexpr int kRawDepth = 3;
 constexpr int kRawCodeBytes = 2 * 2 * 256 * 16;  // [matrix][16-B unit][thread] (int8 needs two units)
 constexpr int kRawAuxBytes = 2 * 256 * 8;        // [matrix][thread] 8 B (scale / scales + mins)
 constexpr int kRawSlotBytes = kRawCodeBytes + kRawAuxBytes;
 
 template <bool kGateUp>
 struct Cfg {
-  static constexpr int kStages = kGateUp ? 3 : 4;
+  static constexpr int kStages = kGateUp ? 3 : 5;
   static constexpr int kATiles = kGateUp ? 2 : 1;
   static constexpr int kStageBytes = (kATiles + 1) * kTileBytes;
   static constexpr int kAccCols = kGateUp ? 256 : 128;  // one accumulator buffer
