@@ -1,5 +1,5 @@
-// Decode step (T <= 4 tokens) as ONE persistent cooperative launch fed by a
-// producer warp through a ring of shared-memory slots.
+// Decode step (T <= 4 tokens) as ONE persistent cooperative launch fed by two
+// producer warps through a ring of shared-memory slots.
 //
 // Decode reads every picked expert's weights once per step, so it is bound by
 // memory bandwidth (the lcz.me forum thread "Halogen Flash Server配置與實測",
@@ -8,11 +8,15 @@
 // 如何在个人电脑上运行 180B 级模型", section "稀疏架构创造了机会", gives the step:
 // 10 of 512 routed experts plus one shared expert per token.
 //
-// One CTA per SM: 8 consumer warps and 1 producer warp. The producer copies
-// each unit of work (a tile of weight rows, its scales, and for down tiles the
-// activations) into a slot with 1-D bulk copies, one row per lane, and arms
-// the slot's mbarrier with the byte count; consumers wait on it, compute, and
-// release the slot. Work per CTA, in order:
+// One CTA per SM: 8 consumer warps and 2 producer warps (unit q is issued by
+// producer q mod 2; the slot count is even, so each slot keeps one producer).
+// A producer copies each unit of work (a 16-row tile piece of weight codes and
+// its scales, with cp.async 16 bytes per lane into rows padded for ldmatrix;
+// router rows, and for down tiles their activations, with 1-D bulk copies)
+// and the slot's mbarrier completes when every copy has landed; all consumer
+// warps wait on it, each computes its share of the tile's K, the last to
+// finish writes the tile's result, and all release the slot. Work per CTA,
+// in order:
 //   A  router quarter-rows (partial logits to global) and the shared expert's
 //      gate/up tiles dealt round-robin over the CTAs;
 //      -- grid barrier; every CTA rebuilds the logits, takes the top-k and

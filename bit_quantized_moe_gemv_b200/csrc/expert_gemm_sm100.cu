@@ -29,11 +29,16 @@
 // the MMA's sum over K is unchanged. The gate/up epilogue writes H in the
 // same tiled form, which is the down GEMM's B operand.
 //
+// Heavy groups (at least two row tiles) are dequantised once, before the
+// GEMMs, by `predequant_kernel` into A tiles of that same image; their tiles
+// then take A with a bulk copy next to B instead of from the dequant warps.
+//
 // Warp roles (448 threads, one CTA per SM, persistent over the tile list):
-//   warp 0      bulk-copy producer of B tiles, TMEM allocation
+//   warp 0      bulk-copy producer of B tiles (and of A for heavy groups),
+//               TMEM allocation
 //   warp 1      MMA issuer (one thread)
 //   warps 2-5   epilogue (TMEM -> registers -> global)
-//   warps 6-13  dequant producers of A tiles
+//   warps 6-13  dequant producers of A tiles (light groups)
 // Every wait is bounded; an expired wait flags MOE_ERR_TIMEOUT, stops the
 // CTA's loops, drains what it issued and frees TMEM.
 #include <cuda_bf16.h>
