@@ -191,6 +191,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 }
 
 // ---------------------------------------------------------------- dequant
+// (a & mask) | magic in one instruction
+__device__ __forceinline__ uint32_t lop_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
+  return d;
+}
 __device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
   __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
@@ -242,10 +248,14 @@ __device__ __forceinline__ void dequant32(int qtype, const RawK& r, uint4 (&o)[4
     const uint32_t k1032 = 0x64086408u;  // fp16x2 (1032, 1032): 1024 + 8
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      uint32_t v[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v[j] = h2_mul(h2_sub(((w[c] >> (4 * j)) & 0x000F000Fu) | 0x64006400u, k1032), s2);
-      o[c] = make_uint4(v[0], v[1], v[2], v[3]);
+      // nibbles (0,4) and (2,6) as 1024 + c, (1,5) and (3,7) as 64 + c: one
+      // lop3 each (no shift for the odd nibbles), then c - 8 exactly
+      const uint32_t x = w[c], x8 = x >> 8;
+      const uint32_t v0 = h2_sub(lop_or(x, 0x000F000Fu, 0x64006400u), k1032);
+      const uint32_t v1 = h2_sub(lop_or(x, 0x00F000F0u, 0x54005400u), 0x54805480u);  // 64 + 8
+      const uint32_t v2 = h2_sub(lop_or(x8, 0x000F000Fu, 0x64006400u), k1032);
+      const uint32_t v3 = h2_sub(lop_or(x8, 0x00F000F0u, 0x54005400u), 0x54805480u);
+      o[c] = make_uint4(h2_mul(v0, s2), h2_mul(v1, s2), h2_mul(v2, s2), h2_mul(v3, s2));
     }
   } else if (qtype == MOE_Q_INT2_ASYM_G16) {
     const uint32_t sA = h2_splat(uint16_t(r.s & 0xffffu)), sB = h2_splat(uint16_t(r.s >> 16));
