@@ -59,7 +59,7 @@ constexpr int kDqWarps = 8;
 // weights dequantised once, into A tiles in global memory, which its GEMM
 // tiles then load like B instead of dequantising per row tile. At most
 // kMaxHeavy groups (the first ones in group order) take this path.
-constexpr int kHeavyRows = 2 * BN;
+constexpr int kHeavyRows = BN + 1;
 constexpr int kMaxHeavy = 64;
 
 // ---------------------------------------------------------------- plan
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   }
   const int excl = wb + incl - nt;
   // heavy groups: slots in group order (a second block-wide scan)
-  const int hv = (g < ngroups && nt >= kHeavyRows / BN) ? 1 : 0;
+  const int hv = (g < ngroups && nt >= 2) ? 1 : 0;  // n >= kHeavyRows
   int hincl = hv;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
