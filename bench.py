@@ -46,7 +46,7 @@ NCU_TRAFFIC = {
     "decode1": (33591680, "profiles/decode_stream_decode1.md"),
     # predequant_kernel + grouped_gemm_kernel<gate/up> + <down> of one step
     # (the gather of the activations is not included)
-    "prefill8k": (2840343576, "profiles/grouped_gemm_prefill8k.md"),
+    "prefill8k": (2863281328, "profiles/grouped_gemm_prefill8k.md"),
 }
 
 
