@@ -56,6 +56,8 @@ constexpr int kCW = 8;                    // consumer warps
 constexpr int kProducers = 2;             // producer warps: unit q is issued by warp kCW + q % kProducers
 constexpr int kThreads = (kCW + kProducers) * 32;
 constexpr int kProducer = kCW;
+constexpr int kGroups = 2;               // consumer groups: tile i goes to group i % 2
+constexpr int kGW = kCW / kGroups;       // warps per group
 constexpr int kMaxT = 4;
 constexpr int kMaxK = 16;
 constexpr int kMaxSlots = 14;
@@ -249,6 +251,10 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+// Arrival counted n times.
+__device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(n) : "memory");
+}
 __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -438,6 +444,7 @@ struct Ctx {
   int RQ, KP, nper;
   int kShared;   // descriptor index of the shared expert
   const Geo* geo;  // [2][4]: slot layout of a gate/up (0) or down (1) piece per format
+  volatile int* issued;  // [kProducers]: one past the last unit each producer has taken a slot for
   __device__ uint8_t* slot(int q) const { return slots + (q % S) * kSlotBytes; }
   __device__ uint32_t full_bar(int q) const { return ptx::smem_addr(&full[q % S]); }
   __device__ uint32_t empty_bar(int q) const { return ptx::smem_addr(&empty[q % S]); }
@@ -625,17 +632,32 @@ __device__ __forceinline__ void build_frag(const Params& P, int fmt, uint8_t* fr
 
 // Bounded wait of all lanes of a consumer warp on a slot's full barrier.
 __device__ __forceinline__ bool wait_full(const Ctx& C, int q, WsHeader* hdr) {
+  // A group that skips the other group's tiles can run a ring ahead, where
+  // the slot's phase parity would match an older, completed phase: first
+  // wait until the producer of unit q has taken its slot.
+  volatile int* iss = C.issued + q % kProducers;
+  if (*iss <= q) {
+    const long long t0 = clock64();
+    while (*iss <= q) {
+      __nanosleep(32);
+      if (*reinterpret_cast<volatile int*>(&hdr->abort) || clock64() - t0 > kSpin) {
+        if (!hdr->abort) flag_error(hdr, MOE_ERR_TIMEOUT, 3500000 + q);
+        atomicExch(&hdr->abort, 1);
+        return false;
+      }
+    }
+  }
   if (ptx::mbar_wait(C.full_bar(q), uint32_t((q / C.S) & 1), &hdr->abort)) return true;
   if (!hdr->abort) flag_error(hdr, MOE_ERR_TIMEOUT, 3000000 + q);
   atomicExch(&hdr->abort, 1);
   return false;
 }
 
-// Sum of the 8 consumer warps' partials of one tile, in warp order.
+// Sum of a group's partials of one tile, in warp order.
 __device__ __forceinline__ float red_sum(const float* rs, int r, int t) {
   float v = 0.f;
 #pragma unroll
-  for (int w = 0; w < kCW; ++w) v += rs[w * 64 + r * 4 + t];
+  for (int w = 0; w < kGW; ++w) v += rs[w * 64 + r * 4 + t];
   return v;
 }
 
@@ -716,7 +738,10 @@ struct Producer {
   __device__ __forceinline__ bool issue(int q) {
     const int lane = threadIdx.x & 31;
     int good = 1;
-    if (lane == 0) good = wait_empty(q);
+    if (lane == 0) {
+      good = wait_empty(q);
+      if (good) C.issued[p] = q + 1;  // unit q's full phase is now its slot's current one
+    }
     good = __shfl_sync(0xffffffffu, good, 0);
     if (!good) return false;
     // The second barrier's count, loaded before the copies are issued and
@@ -764,6 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
   __shared__ int s_cnt[kMaxSlots];
   __shared__ Geo s_geo[8];
   __shared__ int s_nA, s_nSD, s_nB, s_nC, s_U, s_bad, s_fail;
+  __shared__ volatile int s_issued[kProducers];
   __shared__ int s_fmap[4];  // weight format -> fragment buffer
   __shared__ int s_uniq[kMaxT * kMaxK];
   __shared__ int s_slotmap[kMaxT * kMaxK];
@@ -800,6 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
   C.nper = min(kCW, kSlotBytes / (C.KP * 4));
   C.kShared = T * k;
   C.geo = s_geo;
+  C.issued = s_issued;
   if (threadIdx.x < 8) {
     const int dn = threadIdx.x >> 2, f = threadIdx.x & 3;
     const int np = f == 0 ? 1 : (dn ? P.np_dn[f] : P.np_gu[f]);
@@ -846,6 +873,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
       __syncwarp();
       // (router units: lane 0 arrived with the copy's byte count)
     }
+    if (lane == 0)
+      for (int p = 0; p < kProducers; ++p) s_issued[p] = nR < C.S ? nR : C.S;
   } else {
     if (threadIdx.x == 32) {  // the routed descriptors into L2 for after the top-k
       const uintptr_t a = reinterpret_cast<uintptr_t>(P.experts) & ~uintptr_t(15);
@@ -922,6 +951,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
     int total = nA + nSD;
     bool dead = false;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int grp = warp / kGW, gw = warp % kGW;  // consumer group, warp within it
+    int ti = -1;  // index of the current tile (the same count on every warp)
     for (int q = 0;; ++q) {
       if (q == nR) {
         // the shared expert's activations in fragment order (buffer 0), once
@@ -1164,22 +1195,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
       }
       if (q >= total) break;
       // ---------------------------------------------------- unit q
-      if (dead) continue;
+      // Router units are shared by all 8 warps (one quarter-row each); tile i
+      // (all pieces of one 16-row tile) belongs to warp group i % 2, whose 4
+      // warps split its K. Each of them releases the slot for two warps.
+      const Unit u = C.units[q];
+      const bool tile = u.kind != kRouter;
+      if (tile && u.k0 == 0) ++ti;
+      if (dead || (tile && (ti % kGroups) != grp)) continue;
       if (!wait_full(C, q, hdr)) {
         s_fail = 1;
         dead = true;
         continue;
       }
-      const Unit u = C.units[q];
       const uint8_t* slot = C.slot(q);
-      if (u.kind == kRouter) {
+      if (!tile) {
         router_unit_dot(C, u, slot, x32);
       } else {
         const bool dn = u.kind == kDown;
         if (u.k0 == 0) acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
         const Geo g = C.geo[dn * 4 + u.fmt];
         const int nch = g.cb / 16;
-        const int c0 = warp * nch / kCW, c1 = (warp + 1) * nch / kCW;
+        const int c0 = gw * nch / kGW, c1 = (gw + 1) * nch / kGW;
         {  // one call site per instantiation (down tiles: activations in the slot)
           const int fb = dn ? 0 : s_fmap[u.fmt];
           const uint8_t* frag = dn ? slot + g.bofs : fb == 0 ? f0 : smem + L.o_x32 + (fb - 1) * 2 * T * H;
@@ -1198,8 +1234,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
           const int gq = lane >> 2, tq = lane & 3, s = q % C.S;
           float* rs = red + size_t(s) * kCW * 64;
           if (tq < 2) {
-            *reinterpret_cast<float2*>(rs + warp * 64 + gq * 4 + 2 * tq) = make_float2(acc[0], acc[1]);
-            *reinterpret_cast<float2*>(rs + warp * 64 + (gq + 8) * 4 + 2 * tq) = make_float2(acc[2], acc[3]);
+            *reinterpret_cast<float2*>(rs + gw * 64 + gq * 4 + 2 * tq) = make_float2(acc[0], acc[1]);
+            *reinterpret_cast<float2*>(rs + gw * 64 + (gq + 8) * 4 + 2 * tq) = make_float2(acc[2], acc[3]);
           }
           __syncwarp();
           int prev = 0;
@@ -1208,7 +1244,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
             prev = atomicAdd(&s_cnt[s], 1);
           }
           prev = __shfl_sync(0xffffffffu, prev, 0);
-          if (prev == kCW - 1) {
+          if (prev == kGW - 1) {
             __threadfence_block();
             __syncwarp();
             if (lane == 0) s_cnt[s] = 0;
@@ -1243,7 +1279,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
         }
       }
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(C.empty_bar(q));
+      if (lane == 0) {
+        if (tile) mbar_arrive_n(C.empty_bar(q), kCW / kGW);  // the other group's share too
+        else ptx::mbar_arrive(C.empty_bar(q));
+      }
     }
     consumer_sync();
     // ------------------------------------------------ combine of the owned rows
