@@ -43,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captures summarised in profiles/ (set to None when the kernel changes).
 NCU_TRAFFIC = {
     # decode_stream_kernel, mean of two captured launches
-    "decode1": (33591680, "profiles/decode_stream_decode1.md"),
+    "decode1": (33579392, "profiles/decode_stream_decode1.md"),
     # predequant_kernel + grouped_gemm_kernel<gate/up> + <down> of one step
     # (the gather of the activations is not included)
     "prefill8k": (2863281328, "profiles/grouped_gemm_prefill8k.md"),

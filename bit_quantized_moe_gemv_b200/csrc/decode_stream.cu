@@ -13,9 +13,10 @@
 // A producer copies each unit of work (a 16-row tile piece of weight codes and
 // its scales, with cp.async 16 bytes per lane into rows padded for ldmatrix;
 // router rows, and for down tiles their activations, with 1-D bulk copies)
-// and the slot's mbarrier completes when every copy has landed; all consumer
-// warps wait on it, each computes its share of the tile's K, the last to
-// finish writes the tile's result, and all release the slot. Work per CTA,
+// and the slot's mbarrier completes when every copy has landed. Router units
+// are shared by all consumer warps; a tile goes to one of four groups of two
+// warps, which split its K; the last of the two to finish writes the tile's
+// result, and the group releases the slot. Work per CTA,
 // in order:
 //   A  router quarter-rows (partial logits to global) and the shared expert's
 //      gate/up tiles dealt round-robin over the CTAs;
@@ -56,7 +57,7 @@ constexpr int kCW = 8;                    // consumer warps
 constexpr int kProducers = 2;             // producer warps: unit q is issued by warp kCW + q % kProducers
 constexpr int kThreads = (kCW + kProducers) * 32;
 constexpr int kProducer = kCW;
-constexpr int kGroups = 2;               // consumer groups: tile i goes to group i % 2
+constexpr int kGroups = 4;               // consumer groups: tile i goes to group i % kGroups
 constexpr int kGW = kCW / kGroups;       // warps per group
 constexpr int kMaxT = 4;
 constexpr int kMaxK = 16;
@@ -1196,8 +1197,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
       if (q >= total) break;
       // ---------------------------------------------------- unit q
       // Router units are shared by all 8 warps (one quarter-row each); tile i
-      // (all pieces of one 16-row tile) belongs to warp group i % 2, whose 4
-      // warps split its K. Each of them releases the slot for two warps.
+      // (all pieces of one 16-row tile) belongs to warp group i % kGroups,
+      // whose kGW warps split its K; each of them releases the slot for
+      // kCW / kGW warps.
       const Unit u = C.units[q];
       const bool tile = u.kind != kRouter;
       if (tile && u.k0 == 0) ++ti;
