@@ -655,10 +655,10 @@ __device__ __forceinline__ bool wait_full(const Ctx& C, int q, WsHeader* hdr) {
 }
 
 // Sum of a group's partials of one tile, in warp order.
-__device__ __forceinline__ float red_sum(const float* rs, int r, int t) {
+__device__ __forceinline__ float red_sum(const float* rs, int r, int t, int nw) {
   float v = 0.f;
-#pragma unroll
-  for (int w = 0; w < kGW; ++w) v += rs[w * 64 + r * 4 + t];
+#pragma unroll 1
+  for (int w = 0; w < nw; ++w) v += rs[w * 64 + r * 4 + t];
   return v;
 }
 
@@ -1203,7 +1203,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
       const Unit u = C.units[q];
       const bool tile = u.kind != kRouter;
       if (tile && u.k0 == 0) ++ti;
-      if (dead || (tile && (ti % kGroups) != grp)) continue;
+      // phase-A tiles (before the first barrier, on every CTA's critical
+      // path) are shared by all eight warps like router units
+      const bool all8 = q < nA;
+      const int nw = all8 ? kCW : kGW, wi = all8 ? warp : gw;  // warps on this unit, this warp's share
+      if (dead || (tile && !all8 && (ti % kGroups) != grp)) continue;
       if (!wait_full(C, q, hdr)) {
         s_fail = 1;
         dead = true;
@@ -1217,7 +1221,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
         if (u.k0 == 0) acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
         const Geo g = C.geo[dn * 4 + u.fmt];
         const int nch = g.cb / 16;
-        const int c0 = gw * nch / kGW, c1 = (gw + 1) * nch / kGW;
+        const int c0 = wi * nch / nw, c1 = (wi + 1) * nch / nw;
         {  // one call site per instantiation (down tiles: activations in the slot)
           const int fb = dn ? 0 : s_fmap[u.fmt];
           const uint8_t* frag = dn ? slot + g.bofs : fb == 0 ? f0 : smem + L.o_x32 + (fb - 1) * 2 * T * H;
@@ -1236,8 +1240,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
           const int gq = lane >> 2, tq = lane & 3, s = q % C.S;
           float* rs = red + size_t(s) * kCW * 64;
           if (tq < 2) {
-            *reinterpret_cast<float2*>(rs + gw * 64 + gq * 4 + 2 * tq) = make_float2(acc[0], acc[1]);
-            *reinterpret_cast<float2*>(rs + gw * 64 + (gq + 8) * 4 + 2 * tq) = make_float2(acc[2], acc[3]);
+            *reinterpret_cast<float2*>(rs + wi * 64 + gq * 4 + 2 * tq) = make_float2(acc[0], acc[1]);
+            *reinterpret_cast<float2*>(rs + wi * 64 + (gq + 8) * 4 + 2 * tq) = make_float2(acc[2], acc[3]);
           }
           __syncwarp();
           int prev = 0;
@@ -1246,14 +1250,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
             prev = atomicAdd(&s_cnt[s], 1);
           }
           prev = __shfl_sync(0xffffffffu, prev, 0);
-          if (prev == kGW - 1) {
+          if (prev == nw - 1) {
             __threadfence_block();
             __syncwarp();
             if (lane == 0) s_cnt[s] = 0;
             if (!dn) {
               const int r = lane >> 2, t = lane & 3;
               if (t < T) {
-                float gs = red_sum(rs, r, t), us = red_sum(rs, 8 + r, t);
+                float gs = red_sum(rs, r, t, nw), us = red_sum(rs, 8 + r, t, nw);
                 if (u.fmt == MOE_Q_INT8_PER_CHANNEL) {
                   const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + g.aux0);
                   gs *= f16_to_f32(sc[r]);
@@ -1269,7 +1273,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
               for (int hh = 0; hh < 2; ++hh) {
                 const int idx = lane + 32 * hh, r = idx >> 2, t = idx & 3;
                 if (r < u.nrows && t < T) {
-                  float y = red_sum(rs, r, t);
+                  float y = red_sum(rs, r, t, nw);
                   if (u.fmt == MOE_Q_INT8_PER_CHANNEL)
                     y *= f16_to_f32(reinterpret_cast<const uint16_t*>(slot + g.aux0)[(u.row0 & 7) + r]);
                   if (u.e == C.kShared) Sy[r * 4 + t] = y;
@@ -1282,7 +1286,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
       }
       __syncwarp();
       if (lane == 0) {
-        if (tile) mbar_arrive_n(C.empty_bar(q), kCW / kGW);  // the other group's share too
+        if (tile && !all8) mbar_arrive_n(C.empty_bar(q), kCW / kGW);  // the other groups' share too
         else ptx::mbar_arrive(C.empty_bar(q));
       }
     }
