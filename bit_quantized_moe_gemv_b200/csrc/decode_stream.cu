@@ -14,10 +14,10 @@
 // its scales, with cp.async 16 bytes per lane into rows padded for ldmatrix;
 // router rows, and for down tiles their activations, with 1-D bulk copies)
 // and the slot's mbarrier completes when every copy has landed. Router units
-// are shared by all consumer warps; a tile goes to one of four groups of two
-// warps, which split its K; the last of the two to finish writes the tile's
-// result, and the group releases the slot. Work per CTA,
-// in order:
+// and the tiles of phase A are shared by all eight consumer warps; every
+// later tile goes to one of four groups of two warps, which split its K; the
+// last warp to finish writes the tile's result, and the warps that worked on
+// the unit release the slot. Work per CTA, in order:
 //   A  router quarter-rows (partial logits to global) and the shared expert's
 //      gate/up tiles dealt round-robin over the CTAs;
 //      -- grid barrier; every CTA rebuilds the logits, takes the top-k and
@@ -430,7 +430,8 @@ __device__ __forceinline__ void warp_topk4(uint64_t (&c)[4], int k, uint32_t* ok
 // arrival per producer lane (its weight copies landed) plus one more, made
 // right away for units without activations and, for down units, by the bulk
 // copy of their activations once the barrier they need has passed. empty[s]
-// completes when all 8 consumer warps are done with the slot.
+// completes after 8 arrivals: one per consumer warp for shared units, or kCW /
+// kGW from each warp of the group that owns a tile.
 constexpr int kFullCount = 33;
 
 struct Ctx {
@@ -1197,9 +1198,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
       if (q >= total) break;
       // ---------------------------------------------------- unit q
       // Router units are shared by all 8 warps (one quarter-row each); tile i
-      // (all pieces of one 16-row tile) belongs to warp group i % kGroups,
-      // whose kGW warps split its K; each of them releases the slot for
-      // kCW / kGW warps.
+      // (all pieces of one 16-row tile) after phase A belongs to warp group
+      // i % kGroups, whose kGW warps split its K; each of them releases the
+      // slot for kCW / kGW warps.
       const Unit u = C.units[q];
       const bool tile = u.kind != kRouter;
       if (tile && u.k0 == 0) ++ti;
