@@ -265,7 +265,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "f16",  # tensor-core operands (fp16 weights and activations), fp32 accumulation
         "data": "synthetic (seeded; random weights of the stated architecture)",
         "config": dict(workload_config(wl, world),
                        l2="flushed between steps (2 x L2 write, outside the timed events)"),
@@ -374,7 +374,7 @@ def run_stack(args, rank, world, peaks, peak_kind):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32",
+        "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded; random weights of the stated architecture, drawn on the device)",
         "config": dict(workload_config(wl, world), layers=NL,
                        l2="inputs larger than L2 (58 GB stack streamed every step)"),
@@ -474,7 +474,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16",
+        "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded; random weights of the stated architecture)",
         "config": dict(workload_config(wl, world), l2="inputs larger than L2 (1.36 GB of expert weights)"),
         "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (gather + tcgen05 gate/up + down)",
