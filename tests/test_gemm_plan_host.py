@@ -1,0 +1,112 @@
+"""Host-side sizing of the prefill grouped GEMM, checked on the CPU.
+
+A host program (nvcc, no GPU) includes expert_gemm_sm100.cu and checks what
+the kernels rely on: both GEMMs' dynamic shared memory (stage ring plus the
+dequant warps' raw-code staging) fits the per-CTA limit, the row-tile bound
+covers every routing, and the heavy-slot bound covers every routing's groups
+of more than one row tile (up to the slot cap), on seeded random routings
+with a skewed expert popularity.
+"""
+import json
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "bit_quantized_moe_gemv_b200", "csrc")
+
+PROGRAM = r"""
+#include "expert_gemm_sm100.cu"
+#include <cstdio>
+#include <random>
+#include <vector>
+void moe::count_launches(int) {}
+using namespace moe;
+using namespace moe::gemm;
+int main() {
+  const size_t limit = 227 * 1024;
+  const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
+  const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
+  int bad_tiles = 0, bad_heavy = 0, cases = 0;
+  std::mt19937 rng(12345);
+  const int Ts[] = {5, 37, 300, 1000, 8192};
+  const int Es[] = {8, 64, 512};
+  const int ks[] = {1, 2, 10};
+  for (int T : Ts)
+    for (int E : Es)
+      for (int k : ks) {
+        if (k > E) continue;
+        for (int rep = 0; rep < 4; ++rep) {
+          // k distinct experts per token, drawn with a Zipf-like skew (rep 0: uniform)
+          std::vector<long long> cnt(E, 0);
+          std::vector<double> wgt(E);
+          for (int e = 0; e < E; ++e) wgt[e] = rep == 0 ? 1.0 : 1.0 / std::pow(double(e + 1), 0.5 * rep);
+          for (int t = 0; t < T; ++t) {
+            std::vector<double> w = wgt;
+            for (int j = 0; j < k; ++j) {
+              std::discrete_distribution<int> d(w.begin(), w.end());
+              const int e = d(rng);
+              ++cnt[e];
+              w[e] = 0.0;
+            }
+          }
+          for (int sh = 0; sh < 2; ++sh) {
+            ++cases;
+            long long tiles = 0, heavy = 0;
+            for (int e = 0; e < E; ++e) {
+              tiles += (cnt[e] + BN - 1) / BN;
+              heavy += cnt[e] >= kHeavyRows;
+            }
+            if (sh) {
+              tiles += (T + BN - 1) / BN;
+              heavy += T >= kHeavyRows;
+            }
+            if (tiles > grouped_max_tiles(T, k, E, sh != 0)) ++bad_tiles;
+            const long long cap = heavy < kMaxHeavy ? heavy : kMaxHeavy;
+            if (cap > grouped_heavy_slots(T, k, sh != 0)) ++bad_heavy;
+          }
+        }
+      }
+  printf("{\"smem_gu\": %zu, \"smem_dn\": %zu, \"limit\": %zu, \"bad_tiles\": %d, \"bad_heavy\": %d, \"cases\": %d, "
+         "\"ws_8k\": %zu, \"ws_32k\": %zu}\n",
+         smem_gu, smem_dn, limit, bad_tiles, bad_heavy, cases, grouped_ws_bytes(8192, 2048, 768, 10, 512, true),
+         grouped_ws_bytes(32768, 2048, 768, 10, 512, true));
+  return 0;
+}
+"""
+
+
+@pytest.fixture(scope="module")
+def report(tmp_path_factory):
+    if shutil.which("nvcc") is None:
+        pytest.skip("nvcc not available")
+    d = tmp_path_factory.mktemp("gemm_plan")
+    src = d / "plan.cu"
+    src.write_text(PROGRAM)
+    exe = d / "plan"
+    subprocess.run(["nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I", CSRC, "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True, capture_output=True,
+                   timeout=600)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+def test_both_gemms_fit_shared_memory(report):
+    assert report["smem_gu"] <= report["limit"] and report["smem_dn"] <= report["limit"]
+
+
+def test_row_tile_bound_covers_every_routing(report):
+    assert report["cases"] > 0 and report["bad_tiles"] == 0
+
+
+def test_heavy_slot_bound_covers_every_routing(report):
+    assert report["bad_heavy"] == 0
+
+
+def test_prefill_workspaces_are_bounded(report):
+    # 8K and 32K tokens with H = 2048, I = 768, 512 experts, top-10 and a shared expert
+    assert 0 < report["ws_8k"] < 4 << 30
+    assert report["ws_8k"] < report["ws_32k"] < 12 << 30
