@@ -814,10 +814,12 @@ bool grouped_eligible(int H, int I, int E, bool with_shared) {
 
 // Heavy slots a launch may use: routed groups with at least kHeavyRows rows
 // (at most T k / kHeavyRows of them) plus the shared group when T is that
-// large, capped at kMaxHeavy.
-int grouped_heavy_slots(long long T, int k, bool with_shared) {
-  const long long n = T * k / gemm::kHeavyRows + ((with_shared && T >= gemm::kHeavyRows) ? 1 : 0);
-  return int(n < gemm::kMaxHeavy ? n : gemm::kMaxHeavy);
+// large, capped at kMaxHeavy and at 1 GiB of pre-dequantised weights.
+int grouped_heavy_slots(long long T, int k, bool with_shared, int H, int I) {
+  long long n = T * k / gemm::kHeavyRows + ((with_shared && T >= gemm::kHeavyRows) ? 1 : 0);
+  n = n < gemm::kMaxHeavy ? n : gemm::kMaxHeavy;
+  const long long by_bytes = (1ll << 30) / (long long)gemm::heavy_slot_bytes(H, I);
+  return int(n < by_bytes ? n : by_bytes);
 }
 
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
@@ -825,7 +827,7 @@ size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_share
   return align256(16 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
          align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes) +
-         align256(size_t(grouped_heavy_slots(T, k, with_shared)) * gemm::heavy_slot_bytes(H, I));
+         align256(size_t(grouped_heavy_slots(T, k, with_shared, H, I)) * gemm::heavy_slot_bytes(H, I));
 }
 
 cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, int E, const int* perm_src,
@@ -851,7 +853,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   uint8_t* ht = p;
   p += align256(size_t(mt) * (I / BK) * kTileBytes);
   uint8_t* aimg = p;
-  const int max_heavy = grouped_heavy_slots(T, k, with_shared);
+  const int max_heavy = grouped_heavy_slots(T, k, with_shared, H, I);
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -65,7 +65,7 @@ int main() {
             }
             if (tiles > grouped_max_tiles(T, k, E, sh != 0)) ++bad_tiles;
             const long long cap = heavy < kMaxHeavy ? heavy : kMaxHeavy;
-            if (cap > grouped_heavy_slots(T, k, sh != 0)) ++bad_heavy;
+            if (cap > grouped_heavy_slots(T, k, sh != 0, 2048, 768)) ++bad_heavy;
           }
         }
       }
