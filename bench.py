@@ -9,7 +9,10 @@ the step (route -> dispatch -> experts -> combine) over that step's token.
 Timing: W untimed warm-up steps, then K timed steps. Every step is bracketed
 by its own pair of CUDA events on the launching stream; between steps a
 2 x L2-sized buffer is overwritten (outside the event pairs) so every step
-streams its expert weights from HBM rather than L2. Multi-GPU (torchrun):
+streams its expert weights from HBM rather than L2. SM clocks and throttle
+reasons are sampled during the timed region; a region that saw a slowdown
+reason (or clocks held low with none) is run once more and the second run is
+reported. Multi-GPU (torchrun):
 every rank runs an independent replica on its own token stream (weak
 scaling, no collective in the data path); the reported time is the max over
 ranks.
@@ -140,6 +143,57 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+REJECT_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def clock_rejections(clk):
+    """Why a timed region's clock record rejects its number (empty: kept).
+
+    A hardware or thermal slowdown reason, or an SM clock held well below its
+    maximum with no reason active (a leftover clock lock). sw_power_cap alone
+    is kept (and shows in the record's reasons)."""
+    if not clk:
+        return []
+    why = [r for r in clk.get("reasons", []) if r in REJECT_REASONS]
+    sm, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    if not clk.get("reasons") and sm and mx and sm < 0.8 * mx:
+        why.append(f"sm clock {sm:.0f} of {mx:.0f} MHz with no reason active")
+    return why
+
+
+def timed_region(run, rank, world, device, sampler=None, sync=None):
+    """Run `run()` (the K timed steps) as the timed region: a barrier and a
+    device synchronize on both sides, clocks sampled on rank 0 meanwhile.
+
+    If rank 0's clock record rejects the run, every rank runs it once more and
+    the second run is kept; its record lists the first run's reasons under
+    `first_run_rejected`. Returns (run's result, clock record or None)."""
+    import torch
+    sampler = ClockSampler if sampler is None else sampler
+    if sync is None:
+        sync = torch.cuda.synchronize if device is not None and device.type == "cuda" else (lambda: None)
+    first = None
+    for attempt in (0, 1):
+        if world > 1:
+            torch.distributed.barrier()
+        sync()
+        clocks = sampler(device.index if device is not None else 0) if rank == 0 else None
+        res = run()
+        if world > 1:
+            torch.distributed.barrier()
+        sync()
+        clk = clocks.stop() if clocks else None
+        why = clock_rejections(clk)
+        if attempt == 0 and max_over_ranks(1.0 if why else 0.0, world, device) > 0:
+            first = why or ["rejected on rank 0"]
+            continue
+        break
+    if clk is not None:
+        clk["first_run_rejected"] = first
+        clk["rejections"] = clock_rejections(clk)
+    return res, clk
+
+
 # ------------------------------------------------------------------ CPU side
 def cpu_threads():
     try:
@@ -217,19 +271,14 @@ def run_ours(args, rank, world, peaks, peak_kind):
 
     # warm-up (untimed), same protocol
     timed_loop(0, args.warmup)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index) if rank == 0 else None
-    launches0 = L.launch_count()
-    t_wall = time.perf_counter()
-    times = timed_loop(args.warmup, args.steps)
-    t_wall = time.perf_counter() - t_wall
-    launches = L.launch_count() - launches0
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clk = clocks.stop() if clocks else None
+
+    def measured():
+        launches0 = L.launch_count()
+        t0 = time.perf_counter()
+        t = timed_loop(args.warmup, args.steps)
+        return t, L.launch_count() - launches0, time.perf_counter() - t0
+
+    (times, launches, t_wall), clk = timed_region(measured, rank, world, dev)
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
 
     total_ms = float(np.sum(times))
@@ -344,17 +393,13 @@ def run_stack(args, rank, world, peaks, peak_kind):
         return [a.elapsed_time(z) for a, z in evs]
 
     timed_loop(0, args.warmup)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index) if rank == 0 else None
-    launches0 = L.launch_count()
-    times = timed_loop(args.warmup, args.steps)
-    launches = L.launch_count() - launches0
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clk = clocks.stop() if clocks else None
+
+    def measured():
+        launches0 = L.launch_count()
+        t = timed_loop(args.warmup, args.steps)
+        return t, L.launch_count() - launches0
+
+    (times, launches), clk = timed_region(measured, rank, world, dev)
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
     total_ms = float(np.sum(times))
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -436,12 +481,13 @@ def run_prefill(args, rank, world, peaks, peak_kind):
 
     for _ in range(args.warmup):
         step()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index) if rank == 0 else None
-    launches0 = L.launch_count()
-    times = timed(step, args.steps)
-    launches = L.launch_count() - launches0
-    clk = clocks.stop() if clocks else None
+
+    def measured():
+        launches0 = L.launch_count()
+        t = timed(step, args.steps)
+        return t, L.launch_count() - launches0
+
+    (times, launches), clk = timed_region(measured, rank, world, dev)
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
     total_ms = float(np.sum(times))
     total_ms = max_over_ranks(total_ms, world, dev)
