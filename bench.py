@@ -94,6 +94,25 @@ def workload_config(wl, world=1):
     return {"workload": desc, "global_batch": wl.T * world, "parallelism": f"replicas x{world}"}
 
 
+def load_balance(counts, row_tile=128):
+    """How the routed rows of one prefill step spread over the routed experts
+    (the shared expert's T rows are not included): the row-count histogram,
+    the 128-row tiles the grouped GEMM runs and how full they are, and the
+    groups of more than one tile (those the pre-dequantised path may take)."""
+    c = np.asarray(counts, dtype=np.int64)
+    nz = c[c > 0]
+    tiles = (c + row_tile - 1) // row_tile
+    bins = {"0": (0, 0), "1-127": (1, 127), "128-1023": (128, 1023), "1024-8191": (1024, 8191),
+            ">=8192": (8192, np.iinfo(np.int64).max)}
+    return {"rows": int(c.sum()), "experts_empty": int(np.sum(c == 0)),
+            "experts_below_one_tile": int(np.sum((c > 0) & (c < row_tile))),
+            "rows_max": int(c.max()) if c.size else 0,
+            "rows_median_nonempty": float(np.median(nz)) if nz.size else 0.0,
+            "row_tiles": int(tiles.sum()), "tile_fill": float(c.sum() / max(1, tiles.sum() * row_tile)),
+            "groups_over_one_tile": int(np.sum(c > row_tile)),
+            "rows_histogram": {name: int(np.sum((c >= lo) & (c <= hi))) for name, (lo, hi) in bins.items()}}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -499,6 +518,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
     perm = torch.empty(T * k, dtype=torch.int32, device=dev)
     inv = torch.empty(T * k, dtype=torch.int32, device=dev)
     L.dispatch(idx, E, counts, offsets, perm, inv, ws, stream=stream)
+    balance = load_balance(counts.cpu().numpy())
     y = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
     ffn = lambda: L.expert_ffn(x, I, k, E, perm, offsets, counts, experts.table, y, ws, stream=stream)  # noqa: E731
     ffn()
@@ -527,6 +547,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops, "ms_per_launch": ffn_ms,
                      "traffic": ncu_traffic(args.workload)[0], "traffic_source": ncu_traffic(args.workload)[1]},
+        "load_balance": balance,
         "e2e": {"value": world * T * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(T * H * 2), "d2h_bytes_per_step": int(T * H * 2)},
         "gpu_launches": int(launches), "clocks": clk,
