@@ -1,8 +1,10 @@
 """ctypes binding of libmoe_b200.so (include/moe.h).
 
 Argument marshalling only: every function takes torch tensors (device
-memory) or plain integers, passes their addresses and sizes to the C ABI and
-turns a non-zero status into a MoeError. No step of the MoE computation runs
+memory) or plain integers, checks what the C ABI cannot see (each tensor is
+on a CUDA device, contiguous, of the element type the header names and large
+enough for the call), passes addresses and sizes to the C ABI and turns a
+non-zero status into a MoeError. No step of the MoE computation runs
 here. If the library is missing this module raises at import: there is no
 fallback implementation.
 """
@@ -85,9 +87,57 @@ def _check(fn, st):
         raise MoeError(fn, st)
 
 
-def _p(t):
-    """Address of a tensor (None -> NULL)."""
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+# Device-tensor arguments must live on a CUDA device (a CPU test of these
+# checks turns this off; no call reaches the library that way).
+REQUIRE_CUDA = True
+
+_KINDS = {  # element kind in include/moe.h -> accepted torch dtype names
+    "bf16": ("bfloat16", "int16", "uint16"),  # bf16 bit patterns
+    "f32": ("float32",),
+    "i32": ("int32",),
+    "u8": ("uint8",),
+}
+
+
+def _dev(t, name, kind, numel=0, optional=False):
+    """Address of a device-tensor argument after the checks the C ABI cannot
+    make: a CUDA tensor, contiguous, of the element type the header names and
+    holding at least the `numel` elements the call touches. None is passed as
+    NULL only where the header allows it."""
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name}: required (the call takes no NULL here)")
+    if REQUIRE_CUDA and not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor, got one on {t.device}")
+    if str(t.dtype).replace("torch.", "") not in _KINDS[kind]:
+        raise TypeError(f"{name}: dtype {t.dtype} where the call takes {kind}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs {numel}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _table(t, name, n, optional=False):
+    """A device array of n moe_expert descriptors (uint8 bytes)."""
+    return _dev(t, name, "u8", n * ctypes.sizeof(ExpertC), optional)
+
+
+def _ws(ws):
+    return _dev(ws, "ws", "u8")
+
+
+def _bias(bias, T, E, stride):
+    if stride < 0 or (stride > 0 and stride < E):
+        raise ValueError(f"bias_row_stride {stride}: 0 (one row for all tokens) or at least E = {E}")
+    return _dev(bias, "bias", "f32", E if stride == 0 or T == 0 else (T - 1) * stride + E, optional=True)
+
+
+def _shape2(t, name, cols=None):
+    if t.dim() != 2 or (cols is not None and t.shape[1] != cols):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected [rows, {cols if cols is not None else 'cols'}]")
+    return t.shape
 
 
 def _stream(stream):
@@ -115,54 +165,76 @@ def new_workspace(T, H, I, E, k, device="cuda"):
 
 
 def route(x, w_router, bias, bias_row_stride, k, topk_idx, topk_w, ws, logits=None, stream=None):
-    T, H = x.shape
-    E = w_router.shape[0]
-    _check("moe_route", LIB.moe_route(_p(x), T, H, _p(w_router), E, _p(bias), bias_row_stride, k, _p(topk_idx),
-                                      _p(topk_w), _p(logits), _p(ws), ws.numel(), _stream(stream)))
+    T, H = _shape2(x, "x")
+    E = _shape2(w_router, "w_router", H)[0]
+    _check("moe_route", LIB.moe_route(_dev(x, "x", "bf16"), T, H, _dev(w_router, "w_router", "f32"), E,
+                                      _bias(bias, T, E, bias_row_stride), bias_row_stride, k,
+                                      _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
+                                      _dev(logits, "logits", "f32", T * E, optional=True), _ws(ws), ws.numel(),
+                                      _stream(stream)))
 
 
 def dispatch(topk_idx, E, counts, offsets, perm_src, inv_perm, ws, stream=None):
-    T, k = topk_idx.shape
-    _check("moe_dispatch", LIB.moe_dispatch(_p(topk_idx), T, k, E, _p(counts), _p(offsets), _p(perm_src),
-                                            _p(inv_perm), _p(ws), ws.numel(), _stream(stream)))
+    T, k = _shape2(topk_idx, "topk_idx")
+    _check("moe_dispatch", LIB.moe_dispatch(_dev(topk_idx, "topk_idx", "i32"), T, k, E,
+                                            _dev(counts, "counts", "i32", E), _dev(offsets, "offsets", "i32", E + 1),
+                                            _dev(perm_src, "perm_src", "i32", T * k),
+                                            _dev(inv_perm, "inv_perm", "i32", T * k), _ws(ws), ws.numel(),
+                                            _stream(stream)))
 
 
 def expert_ffn(x, I, k, E, perm_src, offsets, counts, experts_table, y_perm, ws, stream=None):
-    T, H = x.shape
-    _check("moe_expert_ffn", LIB.moe_expert_ffn(_p(x), T, H, I, k, E, _p(perm_src), _p(offsets), _p(counts),
-                                                _p(experts_table), _p(y_perm), _p(ws), ws.numel(), _stream(stream)))
+    T, H = _shape2(x, "x")
+    _check("moe_expert_ffn", LIB.moe_expert_ffn(_dev(x, "x", "bf16"), T, H, I, k, E,
+                                                _dev(perm_src, "perm_src", "i32", T * k),
+                                                _dev(offsets, "offsets", "i32", E + 1), _dev(counts, "counts", "i32", E),
+                                                _table(experts_table, "experts_table", E),
+                                                _dev(y_perm, "y_perm", "bf16", T * k * H), _ws(ws), ws.numel(),
+                                                _stream(stream)))
 
 
 def combine(y_perm, inv_perm, topk_w, I, x, shared_table, out, ws, stream=None):
-    T, k = topk_w.shape
-    H = out.shape[1]
-    _check("moe_combine", LIB.moe_combine(_p(y_perm), _p(inv_perm), _p(topk_w), T, H, I, k, _p(x), _p(shared_table),
-                                          _p(out), _p(ws), ws.numel(), _stream(stream)))
+    T, k = _shape2(topk_w, "topk_w")
+    H = _shape2(out, "out")[1]
+    _check("moe_combine", LIB.moe_combine(_dev(y_perm, "y_perm", "bf16", T * k * H),
+                                          _dev(inv_perm, "inv_perm", "i32", T * k), _dev(topk_w, "topk_w", "f32"),
+                                          T, H, I, k, _dev(x, "x", "bf16", T * H, optional=shared_table is None),
+                                          _table(shared_table, "shared_table", 1, optional=True),
+                                          _dev(out, "out", "bf16", T * H), _ws(ws), ws.numel(), _stream(stream)))
 
 
 def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx, topk_w, out, ws,
           stream=None):
-    T, H = x.shape
-    _check("moe_layer", LIB.moe_layer(_p(x), T, H, I, E, k, _p(w_router), _p(bias), bias_row_stride,
-                                      _p(experts_table), _p(shared_table), _p(topk_idx), _p(topk_w), _p(out), _p(ws),
-                                      ws.numel(), _stream(stream)))
+    T, H = _shape2(x, "x")
+    _shape2(w_router, "w_router", H)
+    _check("moe_layer", LIB.moe_layer(_dev(x, "x", "bf16"), T, H, I, E, k, _dev(w_router, "w_router", "f32", E * H),
+                                      _bias(bias, T, E, bias_row_stride), bias_row_stride,
+                                      _table(experts_table, "experts_table", E),
+                                      _table(shared_table, "shared_table", 1, optional=True),
+                                      _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
+                                      _dev(out, "out", "bf16", T * H), _ws(ws), ws.numel(), _stream(stream)))
 
 
 def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx,
                          topk_w, out, stream=None):
     """moe_layer_decode_noalloc: the fused decode step without a workspace."""
-    T, H = x.shape
+    T, H = _shape2(x, "x")
+    _shape2(w_router, "w_router", H)
     _check("moe_layer_decode_noalloc",
-           LIB.moe_layer_decode_noalloc(_p(x), T, H, I, E, k, _p(w_router), _p(bias), bias_row_stride,
-                                        _p(experts_table), _p(shared_table), _p(topk_idx), _p(topk_w), _p(out),
+           LIB.moe_layer_decode_noalloc(_dev(x, "x", "bf16"), T, H, I, E, k, _dev(w_router, "w_router", "f32", E * H),
+                                        _bias(bias, T, E, bias_row_stride), bias_row_stride,
+                                        _table(experts_table, "experts_table", E),
+                                        _table(shared_table, "shared_table", 1, optional=True),
+                                        _dev(topk_idx, "topk_idx", "i32", T * k),
+                                        _dev(topk_w, "topk_w", "f32", T * k), _dev(out, "out", "bf16", T * H),
                                         _stream(stream)))
 
 
 def reset_status(ws, stream=None):
-    _check("moe_reset_status", LIB.moe_reset_status(_p(ws), _stream(stream)))
+    _check("moe_reset_status", LIB.moe_reset_status(_ws(ws), _stream(stream)))
 
 
 def get_status(ws, stream=None) -> int:
     v = c_i32(0)
-    _check("moe_get_status", LIB.moe_get_status(_p(ws), _stream(stream), ctypes.byref(v)))
+    _check("moe_get_status", LIB.moe_get_status(_ws(ws), _stream(stream), ctypes.byref(v)))
     return int(v.value)

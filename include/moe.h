@@ -194,10 +194,12 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
  * cannot provide the workspace moe_layer needs. This call takes the same
  * arguments as moe_layer without `ws`/`ws_bytes`, allocates nothing (no
  * cudaMalloc, no allocating library routine) and keeps its scratch in a
- * 640 KiB device array inside the library, which every GPU that loads the
+ * 1.25 MiB device array inside the library, which every GPU that loads the
  * library holds until the process exits.
- *   Limits: 1 <= T <= 4, E <= 1024, k <= 16, H <= 2048 (a multiple of 512),
- *   I <= 1024 (a multiple of 256); anything else returns MOE_ERR_UNSUPPORTED.
+ *   Limits: 1 <= T <= 4, E <= 1024, k <= 16, 256 <= H, I <= 2048 (multiples
+ *   of 256), within the fused decode kernel's own shape limits (the shapes
+ *   moe_layer runs as one launch); anything else returns
+ *   MOE_ERR_UNSUPPORTED.
  *   The first call on a device looks up the array's device address (once per
  *   device, with that device current); make that first call before any
  *   stream capture.
