@@ -116,8 +116,8 @@ def load_balance(counts, row_tile=128):
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        d = json.load(open(p))
-        return d, "measured"
+        with open(p) as f:
+            return json.load(f), "measured"
     return FALLBACK_PEAKS, "fallback"
 
 
@@ -132,17 +132,21 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.proc = None
         self.path = None
+        self.out = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
+            self.out = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(gpu_index)], stdout=open(self.path, "w"),
+                                          "-lms", "200", "-i", str(gpu_index)], stdout=self.out,
                                          stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
 
     def stop(self):
         if self.proc is None:
+            if self.out is not None:
+                self.out.close()
+                os.unlink(self.path)
             return None
         time.sleep(0.25)
         self.proc.terminate()
@@ -150,7 +154,10 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = [r for r in csv.reader(io.StringIO(open(self.path).read())) if len(r) >= 9]
+            self.proc.wait()
+        self.out.close()
+        with open(self.path) as f:
+            rows = [r for r in csv.reader(io.StringIO(f.read())) if len(r) >= 9]
         os.unlink(self.path)
         if not rows:
             return None

@@ -49,3 +49,22 @@ def test_peaks_and_traffic_sources():
         assert wl in wlm.WORKLOADS
         assert os.path.exists(os.path.join(ROOT, src)), src
         assert traffic is None or traffic > 0
+
+
+def test_clock_sampler_parses_nvidia_smi_rows(tmp_path, monkeypatch):
+    # a stand-in nvidia-smi printing two samples in the queried column order
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\n"
+                    "echo '0, 1965, 1965, 700.5, 0x0, Not Active, Not Active, Not Active, Not Active'\n"
+                    "echo '0, 1950, 1965, 710.5, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "sleep 5\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", f"{tmp_path}:{os.environ['PATH']}")
+    rec = bench.ClockSampler(0).stop()
+    assert rec == {"sm_mhz": 1957.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2}
+    assert bench.clock_rejections(rec) == []
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))
+    assert bench.ClockSampler(0).stop() is None
