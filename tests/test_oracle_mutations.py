@@ -60,6 +60,88 @@ def _ties_to_higher_index(logits, k):
     return out
 
 
+ORIG_DISPATCH = mo.dispatch
+ORIG_COMBINE = mo.combine
+ORIG_ROUTE = mo.route
+
+
+def _int8_unsigned(qtype, rows, cols, codes, scales, mins=None):
+    if qtype == mo.INT8_PER_CHANNEL:
+        q = np.asarray(codes, dtype=np.uint8).astype(np.float64).reshape(rows, cols)
+        return q * np.asarray(scales, np.float64).reshape(rows, 1)
+    return ORIG_DEQUANT(qtype, rows, cols, codes, scales, mins)
+
+
+def _int4_group16(qtype, rows, cols, codes, scales, mins=None):
+    w = ORIG_DEQUANT(qtype, rows, cols, codes, scales, mins)
+    if qtype == mo.INT4_SYM_G32:
+        s = np.asarray(scales, np.float64).reshape(rows, -1)
+        k = np.arange(cols)
+        w = w / s[:, k // 32] * s[:, np.minimum(k // 16, s.shape[1] - 1)]
+    return w
+
+
+def _sigmoid_for_silu(wg, wu, wd, x):
+    g, u = x @ wg.T, x @ wu.T
+    h = (1.0 / (1.0 + np.exp(-g))) * u
+    return h, h @ wd.T
+
+
+def _gates_not_renormalised(x_bits, w_router, bias, k):
+    logits, idx, _ = ORIG_ROUTE(x_bits, w_router, bias, k)
+    p = mo.softmax(logits)
+    return logits, idx, np.take_along_axis(p, idx.astype(np.int64), axis=1)
+
+
+def _bias_only_selects(x_bits, w_router, bias, k):
+    logits, idx, _ = ORIG_ROUTE(x_bits, w_router, bias, k)
+    p = mo.softmax(logits - np.asarray(bias, np.float64))
+    sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    return logits, idx, sel / sel.sum(axis=1, keepdims=True)
+
+
+def _dispatch_descending(idx, E):
+    counts, offsets, perm, inv = ORIG_DISPATCH(idx, E)
+    perm = perm.copy()
+    for e in range(E):
+        perm[offsets[e]:offsets[e + 1]] = perm[offsets[e]:offsets[e + 1]][::-1]
+    inv = np.empty_like(inv)
+    inv[perm] = np.arange(perm.size, dtype=inv.dtype)
+    return counts, offsets, perm, inv
+
+
+def _dispatch_inclusive_offsets(idx, E):
+    counts, offsets, perm, inv = ORIG_DISPATCH(idx, E)
+    return counts, np.concatenate([np.cumsum(counts), [offsets[-1]]]).astype(offsets.dtype), perm, inv
+
+
+def _combine_without_shared(y_perm, inv_perm, w, k, shared_y=None):
+    return ORIG_COMBINE(y_perm, inv_perm, w, k, None)
+
+
+def _combine_unweighted(y_perm, inv_perm, w, k, shared_y=None):
+    return ORIG_COMBINE(y_perm, inv_perm, np.ones_like(np.asarray(w, np.float64)), k, shared_y)
+
+
+def _combine_slots_transposed(y_perm, inv_perm, w, k, shared_y=None):
+    T = np.asarray(w).shape[0]
+    inv = np.asarray(inv_perm).reshape(k, T).T.reshape(-1)
+    return ORIG_COMBINE(y_perm, inv, w, k, shared_y)
+
+
+def _expert_rows_token_mod_k(x_bits, perm_src, offsets, k, experts, rows=None, cache=None):
+    x = mo.bf16_bits_to_f64(x_bits)
+    n = int(np.asarray(offsets)[-1])
+    rows = np.arange(n) if rows is None else np.asarray(rows)
+    owner = np.searchsorted(np.asarray(offsets), rows, side="right") - 1
+    y = np.zeros((rows.size, x.shape[1]))
+    for i, r in enumerate(rows):
+        ex = experts[int(owner[i])]
+        wg, wu, wd = (mo.dequant_qm(m) for m in (ex.gate, ex.up, ex.down))
+        _, y[i] = mo.expert_forward(wg, wu, wd, x[int(perm_src[r]) % k][None])
+    return y
+
+
 def _pins_pass():
     """Run every pin; True only if all of them pass."""
     try:
@@ -71,7 +153,11 @@ def _pins_pass():
         pins.test_layer_closed_form_through_routing()
         for k in (1, 2, 3):
             pins.test_topk_equals_brute_force_subsets(k)
-    except (AssertionError, ValueError):
+        pins.test_dispatch_matches_stable_sort()
+        pins.test_dispatch_empty_and_degenerate()
+        pins.test_sparse_oracle_equals_dense_masked(pins.wlm.WORKLOADS["tiny"])
+        pins.test_sparse_oracle_equals_dense_masked(pins._mixed_small())
+    except AssertionError:  # a value comparison failed (a crash would propagate and fail the test)
         return False
     return True
 
@@ -84,6 +170,17 @@ def _pins_pass():
     ("expert_forward", _down_transposed),
     ("route", _softmax_free_gates),
     ("topk_order", _ties_to_higher_index),
+    ("dequant", _int8_unsigned),
+    ("dequant", _int4_group16),
+    ("expert_forward", _sigmoid_for_silu),
+    ("route", _gates_not_renormalised),
+    ("route", _bias_only_selects),
+    ("dispatch", _dispatch_descending),
+    ("dispatch", _dispatch_inclusive_offsets),
+    ("combine", _combine_without_shared),
+    ("combine", _combine_unweighted),
+    ("combine", _combine_slots_transposed),
+    ("expert_rows", _expert_rows_token_mod_k),
 ])
 def test_planted_mistake_is_caught(monkeypatch, target, mutant):
     assert _pins_pass()
