@@ -4,6 +4,7 @@
 
 #include <atomic>
 
+#include "call_range.h"
 #include "moe.h"
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -48,6 +49,7 @@ size_t moe_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k)
 moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_router, int32_t E, const float* bias,
                      int64_t bias_row_stride, int32_t k, int32_t* topk_idx, float* topk_w, float* logits_out, void* ws,
                      size_t ws_bytes, void* stream) {
+  const CallRange range("moe_route");
   if (!shape_ok(T, H, 64, E, k)) return MOE_ERR_INVALID_ARG;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
@@ -64,6 +66,7 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_rou
 
 moe_status moe_dispatch(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E, int32_t* counts, int32_t* offsets,
                         int32_t* perm_src, int32_t* inv_perm, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange range("moe_dispatch");
   if (!shape_ok(T, 64, 64, E, k)) return MOE_ERR_INVALID_ARG;
   if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!topk_idx || !perm_src || !inv_perm)) return MOE_ERR_INVALID_ARG;
@@ -77,6 +80,7 @@ moe_status moe_dispatch(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E
 moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t k, int32_t E,
                           const int32_t* perm_src, const int32_t* offsets, const int32_t* counts,
                           const moe_expert* experts_dev, uint16_t* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  const CallRange range("moe_expert_ffn");
   if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !perm_src || !offsets || !counts || !experts_dev || !y_perm) return MOE_ERR_INVALID_ARG;
@@ -96,6 +100,7 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, in
 moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int32_t T, int32_t H,
                        int32_t I, int32_t k, const uint16_t* x, const moe_expert* shared_dev, uint16_t* out, void* ws,
                        size_t ws_bytes, void* stream) {
+  const CallRange range("moe_combine");
   if (!shape_ok(T, H, I, k, k)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!y_perm || !inv_perm || !topk_w || !out || (shared_dev && !x)) return MOE_ERR_INVALID_ARG;
@@ -123,6 +128,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
                      const float* bias, int64_t bias_row_stride, const moe_expert* experts_dev,
                      const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w, uint16_t* out, void* ws,
                      size_t ws_bytes, void* stream) {
+  const CallRange range("moe_layer");
   if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;

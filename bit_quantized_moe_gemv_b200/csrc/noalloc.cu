@@ -15,6 +15,7 @@
 
 #include <mutex>
 
+#include "call_range.h"
 #include "moe.h"
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -59,6 +60,7 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
                                                int64_t bias_row_stride, const moe_expert* experts_dev,
                                                const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w,
                                                uint16_t* out, void* stream) {
+  const moe::CallRange range("moe_layer_decode_noalloc");
   if (T < 1 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (T > kNoAllocMaxT || E > kNoAllocMaxE || k > kNoAllocMaxK || H > kNoAllocMaxHI || I > kNoAllocMaxHI)
     return MOE_ERR_UNSUPPORTED;
