@@ -6,8 +6,9 @@ A small host program (compiled with nvcc, run without a GPU) evaluates them
 over every shape the kernel accepts and checks the invariants the kernel
 relies on: every fp16 activation has exactly one place in the fragment
 order, tile pieces fit a slot, slot offsets are 16-byte aligned, the ring
-has an even number of slots (one producer warp per slot) and the whole plan
-fits the per-CTA shared-memory limit.
+has an even number of slots (one producer warp per slot), the whole plan
+fits the per-CTA shared-memory limit, and the workspace regions it writes
+(router partials, the activations of the picked experts) are large enough.
 """
 import json
 import os
@@ -24,10 +25,13 @@ PROGRAM = r"""
 #include <cstdio>
 #include <vector>
 void moe::count_launches(int) {}
+// the prefill scratch regions are not used by the decode kernel
+size_t moe::grouped_ws_bytes(long long, int, int, int, int, bool) { return 0; }
+size_t moe::router_tc_ws_bytes(long long, int, int) { return 0; }
 using namespace moe;
 using namespace moe::dks;
 int main() {
-  int bad_frag = 0, bad_geo = 0, bad_plan = 0, eligible = 0, checked = 0;
+  int bad_frag = 0, bad_geo = 0, bad_plan = 0, bad_ws = 0, eligible = 0, checked = 0;
   // fragment order: a bijection of (k, t) onto the fp16 slots of the buffer
   for (int fmt = 1; fmt <= 3; ++fmt)
     for (int T = 1; T <= 4; ++T)
@@ -68,10 +72,16 @@ int main() {
             if (S < 4 || S > kMaxSlots || S % kProducers || p.total + kStaticSmem > kSmemLimit ||
                 p.o_slots % 1024 || kSlotBytes % 1024)
               ++bad_plan;
+            // workspace regions the kernel writes: router partials [T, E, RQ] fp32 and the
+            // fp16 activations of every picked expert plus the shared one
+            const WsLayout L = ws_layout(T, H, I, E, k);
+            if (L.h - L.partial < size_t(4) * T * E * router_rq(H) ||
+                L.shared_y - L.h < decode_stream_hfrag_bytes(T, I, k) || L.partial % 256 || L.h % 256)
+              ++bad_ws;
           }
-  printf("{\"bad_frag\": %d, \"bad_geo\": %d, \"bad_plan\": %d, \"eligible\": %d, \"checked\": %d, "
+  printf("{\"bad_frag\": %d, \"bad_geo\": %d, \"bad_plan\": %d, \"bad_ws\": %d, \"eligible\": %d, \"checked\": %d, "
          "\"slots_decode1\": %d, \"slots_decode48\": %d, \"decode1\": %d, \"decode48\": %d}\n",
-         bad_frag, bad_geo, bad_plan, eligible, checked, pick_slots(1, 2048, 512, 10), pick_slots(4, 2048, 512, 10),
+         bad_frag, bad_geo, bad_plan, bad_ws, eligible, checked, pick_slots(1, 2048, 512, 10), pick_slots(4, 2048, 512, 10),
          int(decode_stream_eligible(1, 2048, 768, 512, 10)), int(decode_stream_eligible(4, 2048, 768, 512, 10)));
   return 0;
 }
@@ -105,6 +115,10 @@ def test_tile_pieces_fit_and_are_aligned(plan_report):
 def test_plans_fit_shared_memory_with_an_even_ring(plan_report):
     assert plan_report["bad_plan"] == 0
     assert plan_report["eligible"] > 0
+
+
+def test_workspace_holds_what_the_kernel_writes(plan_report):
+    assert plan_report["bad_ws"] == 0
 
 
 def test_the_bench_decode_shapes_take_the_fused_kernel(plan_report):
