@@ -437,26 +437,6 @@ __device__ __forceinline__ DqMat dq_mat(const moe_qmatrix& W, int row, int M, in
   return d;
 }
 
-__device__ __forceinline__ void dq_load(const DqMat& d, int k0, RawK& r) {
-  if (d.qtype == MOE_Q_INT4_SYM_G32) {
-    r.c0 = __ldg(reinterpret_cast<const uint4*>(d.codes + k0 / 2));
-    r.s = __ldg(d.scales + k0 / 32);
-  } else if (d.qtype == MOE_Q_INT2_ASYM_G16) {
-    const uint2 c = __ldg(reinterpret_cast<const uint2*>(d.codes + k0 / 4));
-    r.c0 = make_uint4(c.x, c.y, 0, 0);
-    r.s = __ldg(reinterpret_cast<const unsigned int*>(d.scales + k0 / 16));
-    r.m = __ldg(reinterpret_cast<const unsigned int*>(d.mins + k0 / 16));
-  } else if (d.qtype == MOE_Q_INT8_PER_CHANNEL) {
-    const uint4* p = reinterpret_cast<const uint4*>(d.codes + k0);
-    r.c0 = __ldg(p);
-    r.c1 = __ldg(p + 1);
-    r.s = __ldg(d.scales);
-  } else {
-    r.c0 = r.c1 = make_uint4(0, 0, 0, 0);
-    r.s = r.m = 0;
-  }
-}
-
 __device__ __forceinline__ void cp16(uint8_t* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_addr(dst)), "l"(src) : "memory");
 }
