@@ -25,12 +25,6 @@ def L():
     return _lib
 
 
-def _t(a, dtype=None):
-    import torch
-    t = torch.from_numpy(np.ascontiguousarray(a))
-    return t.cuda() if dtype is None else t.to(dtype).cuda()
-
-
 def _small_mixed():
     return wlm.Workload("small_mixed", T=19, H=128, I=64, E=12, k=3, zipf_s=0.5, uniform_frac=0.3,
                         routed_qtypes=((0, 4, wlm.Q_INT4_SYM_G32), (4, 8, wlm.Q_INT2_ASYM_G16),
