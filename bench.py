@@ -346,7 +346,8 @@ def run_ours(args, rank, world, peaks, peak_kind):
                        l2="flushed between steps (2 x L2 write, outside the timed events)"),
         "roofline": {
             "bound": "hbm",
-            "kernel": "moe_layer step (all launches of one step)",
+            "kernel": "moe_layer step: decode_stream_kernel, one launch per step (events bracket the launch)"
+                      if wl.T <= 4 else "moe_layer step (all launches of one step)",
             "achieved": achieved_gbs,
             "peak": peak,
             "unit": "GB/s",
