@@ -43,10 +43,9 @@ METRIC = "MoE-layer tokens/s (decode b=1..4, 8K prefill); % of HBM / tensor roof
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per launch of the dominant kernel(s), from the ncu
-# captures summarised in profiles/ (set to None when the kernel changes).
+# captures summarised in profiles/ (None while no capture of the current
+# kernel exists).
 NCU_TRAFFIC = {
-    # decode_stream_kernel: the last capture (profiles/decode_stream_decode1.md) predates a
-    # change in how phase-A tiles are split among the consumer warps, so it is not reported
     "decode1": (None, "profiles/decode_stream_decode1.md"),
     # predequant_kernel + grouped_gemm_kernel<gate/up> + <down> of one step
     # (the gather of the activations is not included)
@@ -78,7 +77,11 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode1", choices=["decode1", "decode48", "prefill8k", "prefill32k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bound on the CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound on each CPU-baseline sample")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="decode1 only (by default the decode1 line also carries prefill8k and decode48 results)")
+    ap.add_argument("--clock-window", type=float, default=1.2,
+                    help="seconds of back-to-back steps around the timed region while clocks are sampled")
     return ap.parse_args()
 
 
@@ -187,9 +190,30 @@ def clock_rejections(clk):
     return why
 
 
-def timed_region(run, rank, world, device, sampler=None, sync=None):
+def keep_busy(step, seconds, sync):
+    """Untimed steps back to back for about `seconds` (at least one): the
+    load around the timed region while clocks are sampled."""
+    if seconds <= 0:
+        return 0
+    t0, n = time.perf_counter(), 0
+    while True:
+        for _ in range(8):
+            step()
+            n += 1
+        sync()
+        if time.perf_counter() - t0 >= seconds:
+            return n
+
+
+def timed_region(run, rank, world, device, sampler=None, sync=None, filler=None, window=0.0):
     """Run `run()` (the K timed steps) as the timed region: a barrier and a
     device synchronize on both sides, clocks sampled on rank 0 meanwhile.
+
+    A K-step region can be far shorter than the sampler's 200 ms period, so
+    with `filler` (one untimed step of the same workload) the sampler runs
+    over a window of about `window` seconds of back-to-back steps: half before
+    the region, half after it, each side synchronised, so the timed steps
+    themselves run alone. The record states the window and its sample count.
 
     If rank 0's clock record rejects the run, every rank runs it once more and
     the second run is kept; its record lists the first run's reasons under
@@ -204,11 +228,22 @@ def timed_region(run, rank, world, device, sampler=None, sync=None):
             torch.distributed.barrier()
         sync()
         clocks = sampler(device.index if device is not None else 0) if rank == 0 else None
+        t_win = time.perf_counter()
+        n_fill = keep_busy(filler, window / 2, sync) if filler is not None else 0
+        if world > 1:
+            torch.distributed.barrier()
+        sync()
         res = run()
         if world > 1:
             torch.distributed.barrier()
         sync()
+        n_fill += keep_busy(filler, window / 2, sync) if filler is not None else 0
+        t_win = time.perf_counter() - t_win
         clk = clocks.stop() if clocks else None
+        if clk is not None:
+            clk["window_s"] = t_win
+            clk["window"] = ("the timed region inside back-to-back untimed steps of the same workload "
+                             f"({n_fill} of them)" if filler is not None else "the timed region alone")
         why = clock_rejections(clk)
         if attempt == 0 and max_over_ranks(1.0 if why else 0.0, world, device) > 0:
             first = why or ["rejected on rank 0"]
@@ -245,6 +280,39 @@ def time_oracle(wl, lay, bias, n_steps_max, seconds, step_offset=0):
         if time.perf_counter() - t0 >= seconds and steps >= 2:
             break
     return tokens, time.perf_counter() - t0, steps
+
+
+def time_oracle_tokens(wl, lay, bias, seconds, chunk=16):
+    """The fp64 oracle layer over the first tokens of the workload's input,
+    `chunk` tokens per call, until `seconds`. Returns (tokens, elapsed s)."""
+    import oracle
+    xb = wlm.gen_x(wl)
+    tokens, t0 = 0, time.perf_counter()
+    while tokens < wl.T:
+        n = min(chunk, wl.T - tokens)
+        b = bias[tokens:tokens + n] if np.ndim(bias) == 2 else bias
+        oracle.moe_layer(xb[tokens:tokens + n], lay.w_router, b, wl.k, lay.experts, lay.shared)
+        tokens += n
+        if time.perf_counter() - t0 >= seconds:
+            break
+    return tokens, time.perf_counter() - t0
+
+
+def cpu_baseline(wl, lay, bias, seconds):
+    """The fp64 oracle on the host cores, timed on a bounded sample of the
+    workload, as tokens/s of one layer (a layer stack: layer 0's rate divided
+    by the layer count, every layer costing the same)."""
+    if wl.T > 4:
+        tokens, secs = time_oracle_tokens(wl, lay, bias, seconds)
+        sample = (f"{tokens} of the {wl.T} tokens of the step through the fp64 oracle in 16-token calls "
+                  f"({secs:.1f} s; each call dequantises the experts it touches, so the rate is below what a "
+                  f"whole step would reach)")
+    else:
+        tokens, secs, steps = time_oracle(wl, lay, bias, 10 ** 6, seconds, step_offset=10 ** 5)
+        sample = (f"{steps} layer-steps of {wl.T} token(s) through the fp64 oracle ({secs:.1f} s)"
+                  + (f" on layer 0, scaled by 1/{wl.layers} layers" if wl.layers > 1 else ""))
+    return {"value": tokens / secs / wl.layers, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": sample}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -304,7 +372,12 @@ def run_ours(args, rank, world, peaks, peak_kind):
         t = timed_loop(args.warmup, args.steps)
         return t, L.launch_count() - launches0, time.perf_counter() - t0
 
-    (times, launches, t_wall), clk = timed_region(measured, rank, world, dev)
+    def filler():
+        step(args.warmup)
+        flush.fill_(1)
+
+    (times, launches, t_wall), clk = timed_region(measured, rank, world, dev, filler=filler,
+                                                  window=args.clock_window)
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
 
     total_ms = float(np.sum(times))
@@ -426,7 +499,8 @@ def run_stack(args, rank, world, peaks, peak_kind):
         t = timed_loop(args.warmup, args.steps)
         return t, L.launch_count() - launches0
 
-    (times, launches), clk = timed_region(measured, rank, world, dev)
+    (times, launches), clk = timed_region(measured, rank, world, dev, filler=lambda: step(args.warmup),
+                                          window=args.clock_window)
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
     total_ms = float(np.sum(times))
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -514,7 +588,7 @@ def run_prefill(args, rank, world, peaks, peak_kind):
         t = timed(step, args.steps)
         return t, L.launch_count() - launches0
 
-    (times, launches), clk = timed_region(measured, rank, world, dev)
+    (times, launches), clk = timed_region(measured, rank, world, dev, filler=step, window=args.clock_window)
     assert L.get_status(ws, stream) == 0, "device-side status set during the bench"
     total_ms = float(np.sum(times))
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -603,22 +677,35 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     else:
         torch.cuda.set_device(0)
-    if args.workload.startswith("prefill"):
-        line, wl, lay, bias = run_prefill(args, rank, world, peaks, peak_kind)
-    elif wlm.WORKLOADS[args.workload].layers > 1:
-        line, wl, lay, bias = run_stack(args, rank, world, peaks, peak_kind)
-    else:
-        line, wl, lay, bias = run_ours(args, rank, world, peaks, peak_kind)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.workload.startswith("prefill"):
-        if lay is None:  # layer stack: time the oracle on layer 0 and scale to all layers
-            lay = wlm.gen_layer(wl, layer=0)
-        tokens, secs, steps = time_oracle(wl, lay, bias, 10 ** 6, args.cpu_seconds, step_offset=10 ** 5)
-        per_layer = tokens / secs
-        line["cpu_baseline"] = {"value": per_layer / wl.layers, "unit": "tokens/s", "cores": cpu_threads(),
-                                "kind": "oracle",
-                                "sample": f"{steps} layer-steps of {wl.T} token(s) through the fp64 oracle "
-                                          f"({secs:.1f} s)" + (f" on layer 0, scaled by 1/{wl.layers} layers"
-                                                               if wl.layers > 1 else "")}
+    def run_one(name):
+        a = argparse.Namespace(**vars(args))
+        a.workload = name
+        if name.startswith("prefill"):
+            res = run_prefill(a, rank, world, peaks, peak_kind)
+        elif wlm.WORKLOADS[name].layers > 1:
+            res = run_stack(a, rank, world, peaks, peak_kind)
+        else:
+            res = run_ours(a, rank, world, peaks, peak_kind)
+        ln, wl, lay, bias = res
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            if lay is None:  # layer stack: time the oracle on layer 0 and scale to all layers
+                lay = wlm.gen_layer(wl, layer=0)
+            ln["cpu_baseline"] = cpu_baseline(wl, lay, bias, args.cpu_seconds)
+        import torch
+        torch.cuda.empty_cache()
+        return ln
+
+    line = run_one(args.workload)
+    if args.workload == "decode1" and not args.headline_only:
+        # the metric's other halves, measured in the same process: the 8K
+        # prefill and the 48-layer decode stack, each with its own roofline,
+        # clocks, e2e and CPU baseline
+        keep = ("value", "unit", "ms_per_step", "steps", "warmup", "config", "roofline", "e2e", "gpu_launches",
+                "clocks", "cpu_baseline", "load_balance", "dtype")
+        line["workloads"] = {}
+        for name in ("prefill8k", "decode48"):
+            sub = run_one(name)
+            line["workloads"][name] = {key: sub[key] for key in keep if key in sub}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

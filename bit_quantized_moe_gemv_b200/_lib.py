@@ -56,9 +56,9 @@ def _load():
                                    c_vp]),
         "moe_combine": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
         "moe_layer": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
-                              c_vp, c_vp, c_sz, c_vp]),
+                              c_vp, c_vp, c_vp, c_sz, c_vp]),
         "moe_layer_decode_noalloc": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp,
-                                             c_vp, c_vp, c_vp, c_vp, c_vp]),
+                                             c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
         "moe_reset_status": (c_i32, [c_vp, c_vp]),
         "moe_get_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32)]),
         "moe_launch_count": (ctypes.c_uint64, []),
@@ -204,7 +204,7 @@ def combine(y_perm, inv_perm, topk_w, I, x, shared_table, out, ws, stream=None):
 
 
 def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx, topk_w, out, ws,
-          stream=None):
+          stream=None, logits=None):
     T, H = _shape2(x, "x")
     _shape2(w_router, "w_router", H)
     _check("moe_layer", LIB.moe_layer(_dev(x, "x", "bf16"), T, H, I, E, k, _dev(w_router, "w_router", "f32", E * H),
@@ -212,11 +212,12 @@ def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_tab
                                       _table(experts_table, "experts_table", E),
                                       _table(shared_table, "shared_table", 1, optional=True),
                                       _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
+                                      _dev(logits, "logits", "f32", T * E, optional=True),
                                       _dev(out, "out", "bf16", T * H), _ws(ws), ws.numel(), _stream(stream)))
 
 
 def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx,
-                         topk_w, out, stream=None):
+                         topk_w, out, stream=None, logits=None):
     """moe_layer_decode_noalloc: the fused decode step without a workspace."""
     T, H = _shape2(x, "x")
     _shape2(w_router, "w_router", H)
@@ -226,8 +227,9 @@ def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_ta
                                         _table(experts_table, "experts_table", E),
                                         _table(shared_table, "shared_table", 1, optional=True),
                                         _dev(topk_idx, "topk_idx", "i32", T * k),
-                                        _dev(topk_w, "topk_w", "f32", T * k), _dev(out, "out", "bf16", T * H),
-                                        _stream(stream)))
+                                        _dev(topk_w, "topk_w", "f32", T * k),
+                                        _dev(logits, "logits", "f32", T * E, optional=True),
+                                        _dev(out, "out", "bf16", T * H), _stream(stream)))
 
 
 def reset_status(ws, stream=None):

@@ -126,8 +126,8 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
 
 moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k, const float* w_router,
                      const float* bias, int64_t bias_row_stride, const moe_expert* experts_dev,
-                     const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w, uint16_t* out, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w, float* logits_out,
+                     uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
   const CallRange range("moe_layer");
   if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
@@ -142,7 +142,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   WsHeader* hdr = ws_at<WsHeader>(ws, 0);
   if (decode_stream_eligible(T, H, I, E, k))
     return cuda_status(launch_decode_stream(x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev,
-                                            shared_dev, topk_idx, topk_w, out, ws_at<float>(ws, L.partial),
+                                            shared_dev, topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.partial),
                                             ws_at<void>(ws, L.h), hdr, st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
@@ -150,7 +150,8 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   int* inv = ws_at<int>(ws, L.inv);
   float* y_perm = ws_at<float>(ws, L.y_perm);  // fp32: out is rounded only once
   cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w,
-                               ws_at<float>(ws, L.logits), ws_at<void>(ws, L.router), hdr, st);
+                               logits_out ? logits_out : ws_at<float>(ws, L.logits), ws_at<void>(ws, L.router),
+                               hdr, st);
   if (e == cudaSuccess) e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, inv, ws_at<int>(ws, L.hist), hdr, st);
   float* shared_y = nullptr;
   if (T > kDecodeMaxT && grouped_eligible(H, I, E, shared_dev != nullptr)) {

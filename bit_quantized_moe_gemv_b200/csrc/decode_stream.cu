@@ -201,6 +201,7 @@ struct Params {
   const moe_expert* shared;
   int* topk_idx;
   float* topk_w;
+  float* logits_out;  // [T][E] or null
   uint16_t* out;
   float* partial;   // [T][E][RQ]
   uint8_t* hfrag;   // (T*k + 1) fragment buffers of the down activations
@@ -1105,11 +1106,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(const __grid
             const int id = s_uniq[i / W];
             dst[i] = (id >= 0 && id < E) ? src[size_t(id) * W + (i % W)] : 0u;
           }
-          if (b == 0)
+          if (b == 0) {
             for (int i = threadIdx.x; i < nk; i += kCW * 32) {
               P.topk_idx[i] = s_idx[i];
               P.topk_w[i] = s_w[i];
             }
+            if (P.logits_out)
+              for (int i = threadIdx.x; i < T * E; i += kCW * 32) P.logits_out[i] = lg[i];
+          }
         }
         consumer_sync();
         // validate the picked experts' descriptors (one thread per expert)
@@ -1373,15 +1377,15 @@ size_t decode_stream_hfrag_bytes(int T, int I, int k) {
 
 cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
                                  const float* bias, long long bstride, const moe_expert* experts,
-                                 const moe_expert* shared, int* topk_idx, float* topk_w, uint16_t* out,
-                                 float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st) {
+                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
+                                 uint16_t* out, float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st) {
   using namespace dks;
   const int grid = grid_size();
   const int S = pick_slots(T, H, E, k);
   const size_t smem = size_t(make_plan(T, H, E, k, S).total);
   cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  Params P{x, T, H, I, E, k, w_router, bias, bstride, experts, shared, topk_idx, topk_w, out, partial,
+  Params P{x, T, H, I, E, k, w_router, bias, bstride, experts, shared, topk_idx, topk_w, logits_out, out, partial,
            static_cast<uint8_t*>(hfrag), hdr, S, {0, 0, 0, 0}, {0, 0, 0, 0}};
   for (int f = 1; f <= 3; ++f) {
     P.np_gu[f] = npieces(f, H, T, false);

@@ -45,8 +45,8 @@ bool decode_stream_eligible(int T, int H, int I, int E, int k);
 size_t decode_stream_hfrag_bytes(int T, int I, int k);
 cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
                                  const float* bias, long long bstride, const moe_expert* experts,
-                                 const moe_expert* shared, int* topk_idx, float* topk_w, uint16_t* out,
-                                 float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st);
+                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
+                                 uint16_t* out, float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st);
 
 // Prefill experts on tcgen05 (expert_gemm_sm100.cu): plan, gather, gate/up
 // GEMM with SwiGLU epilogue, down GEMM. Routed rows go to y_f32 or y_bf16

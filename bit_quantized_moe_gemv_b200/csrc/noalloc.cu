@@ -11,6 +11,7 @@
 // this library until the process exits. Every call shares it, so calls that
 // may overlap on the GPU (different streams, different host threads) race
 // and must be serialised by the caller.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -32,24 +33,63 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+// Driver calls reached through the runtime's entry-point table, so the
+// library needs no link against libcuda (it loads on machines without a GPU).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device. Host code may
-// not use the symbol itself as a device pointer: cudaGetSymbolAddress gives
-// the address, once per device, with that device current.
+// Process-unique id of the current context (0 if there is none or the
+// driver cannot tell).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa{}, qb{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || a == nullptr)
+      return 0;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess || b == nullptr)
+      return 0;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+struct ScratchEntry {
+  unsigned long long ctx_id;  // CUDA context the address belongs to (0 = none yet)
+  void* ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
+
+// Device address of the scratch array in the current device's current
+// context. Host code may not use the symbol itself as a device pointer:
+// cudaGetSymbolAddress gives the address, once per device, with that device
+// current. The cached address is tied to the context it was taken in (its
+// process-unique id): after cudaDeviceReset, or with another context
+// current, the module is loaded anew and the address is looked up again.
 cudaError_t scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  unsigned long long id = current_context_id();
+  if (id == 0 || g_scratch[dev].ctx_id != id || g_scratch[dev].ptr == nullptr) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // also makes the primary context current if none was
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+    if (id == 0) id = current_context_id();
+    if (id == 0) return cudaErrorDeviceUninitialized;
+    g_scratch[dev] = ScratchEntry{id, p};
   }
-  *out = g_scratch_ptr[dev];
+  *out = g_scratch[dev].ptr;
   return cudaSuccess;
 }
 
@@ -59,7 +99,7 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
                                                int32_t k, const float* w_router, const float* bias,
                                                int64_t bias_row_stride, const moe_expert* experts_dev,
                                                const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w,
-                                               uint16_t* out, void* stream) {
+                                               float* logits_out, uint16_t* out, void* stream) {
   const moe::CallRange range("moe_layer_decode_noalloc");
   if (T < 1 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (T > kNoAllocMaxT || E > kNoAllocMaxE || k > kNoAllocMaxK || H > kNoAllocMaxHI || I > kNoAllocMaxHI)
@@ -82,7 +122,7 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
   // The previous call's status and barrier words stay in the array: clear them.
   if (cudaMemsetAsync(base, 0, sizeof(moe::WsHeader), st) != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t e = moe::launch_decode_stream(
-      x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, out,
+      x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, logits_out, out,
       moe::ws_at<float>(base, off_partial), moe::ws_at<void>(base, off_h), moe::ws_at<moe::WsHeader>(base, 0), st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -174,7 +174,8 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
  * moe_layer - the whole step (route, dispatch, experts, combine) in one call.
  * Same arguments and layouts as the four calls above; dispatch arrays and
  * intermediate rows live in the workspace and stay fp32, so `out` is rounded
- * once. Decode batches (1 <= T <= 4, H and I <= 2048) run as ONE cooperative
+ * once. `logits_out` (fp32 [T, E], NULL = not exported) receives the biased
+ * fp32 logits the selection was made on, as in moe_route. Decode batches (1 <= T <= 4, H and I <= 2048) run as ONE cooperative
  * persistent kernel whose grid barriers are bounded: if one expires the call
  * leaves MOE_ERR_TIMEOUT in the status word, and the workspace must be reset
  * with moe_reset_status before it is used again.
@@ -182,7 +183,7 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
 moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k,
                      const float* w_router, const float* bias, int64_t bias_row_stride,
                      const moe_expert* experts_dev, const moe_expert* shared_dev, int32_t* topk_idx,
-                     float* topk_w, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+                     float* topk_w, float* logits_out, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_layer_decode_noalloc - moe_layer's fused decode step for callers that
@@ -201,8 +202,8 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
  *   moe_layer runs as one launch); anything else returns
  *   MOE_ERR_UNSUPPORTED.
  *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.
+ *   device and CUDA context, with that device current); make that first call
+ *   before any stream capture.
  *   All calls share the array: calls that may overlap on the GPU (other
  *   streams, other host threads) race and must be serialised by the caller.
  *   Device-side checks still skip bad experts, but their status word lives
@@ -212,7 +213,8 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
 moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k,
                                     const float* w_router, const float* bias, int64_t bias_row_stride,
                                     const moe_expert* experts_dev, const moe_expert* shared_dev,
-                                    int32_t* topk_idx, float* topk_w, uint16_t* out, void* stream);
+                                    int32_t* topk_idx, float* topk_w, float* logits_out, uint16_t* out,
+                                    void* stream);
 
 /* Clear the device status word of a workspace (asynchronous on `stream`).
  * Call once on a fresh workspace before its first use. */

@@ -102,3 +102,67 @@ def upload_layer(lay, device="cuda"):
 def bias_tensor(bias, device="cuda"):
     import torch
     return torch.from_numpy(np.ascontiguousarray(bias, dtype=np.float32)).to(device)
+
+
+class ErrorAccumulator:
+    """assert_close over data seen in pieces: accumulates the squared error,
+    the squared reference and the largest error, then applies the same two
+    bounds (rel L2 and max abs against the rms of the whole reference)."""
+
+    def __init__(self, what):
+        self.what, self.se, self.sr, self.mx, self.n = what, 0.0, 0.0, 0.0, 0
+
+    def add(self, got, ref):
+        got = np.asarray(got, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        assert got.shape == ref.shape, (got.shape, ref.shape)
+        assert np.all(np.isfinite(got)), f"{self.what}: non-finite values"
+        err = got - ref
+        self.se += float(np.sum(err * err))
+        self.sr += float(np.sum(ref * ref))
+        self.mx = max(self.mx, float(np.abs(err).max()) if err.size else 0.0)
+        self.n += ref.size
+
+    def check(self):
+        rms = np.sqrt(self.sr / max(self.n, 1))
+        rel = np.sqrt(self.se) / max(np.sqrt(self.sr), 1e-300)
+        assert rel <= REL_L2, f"{self.what}: rel L2 {rel:.3e} > {REL_L2}"
+        assert self.mx <= MAX_ABS_RMS * rms, f"{self.what}: max abs {self.mx:.3e} > {MAX_ABS_RMS} x rms {rms:.3e}"
+        return rel, self.mx / max(rms, 1e-300)
+
+
+def check_every_row(xb, w_router, bias, k, experts, shared, idx, perm, offsets, y_perm_bits, out_bits,
+                    shared_chunk=2048):
+    """Every dispatched row and every output token of a step against the
+    oracle, one expert at a time (a whole prefill step's fp64 rows would not
+    fit in host memory at once).
+
+    y_perm_bits: the device's bf16 rows in dispatch order (moe_expert_ffn);
+    out_bits: the device's bf16 layer output (moe_layer). The routing must
+    have been checked already (check_routing); the oracle evaluates the
+    device's picks with gates from the fp64 logits.
+    Returns ((rel, max/rms) of y_perm, (rel, max/rms) of out)."""
+    x = bf16_to_f64(xb)
+    T, H = x.shape
+    gates = oracle_gates_for(oracle.router_logits(xb, w_router, bias), idx)
+    perm = np.asarray(perm, dtype=np.int64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    out_ref = np.zeros((T, H), dtype=np.float64)
+    acc_y = ErrorAccumulator("y_perm (every row)")
+    for e in range(len(experts)):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r0 == r1:
+            continue
+        wg, wu, wd = (oracle.dequant_qm(m) for m in (experts[e].gate, experts[e].up, experts[e].down))
+        src = perm[r0:r1]
+        toks, slots = src // k, src % k
+        _, y = oracle.expert_forward(wg, wu, wd, x[toks])
+        acc_y.add(bf16_to_f64(y_perm_bits[r0:r1]), y)
+        out_ref[toks] += gates[toks, slots][:, None] * y  # a token picks an expert at most once
+    if shared is not None:
+        sg, su, sd = (oracle.dequant_qm(m) for m in (shared.gate, shared.up, shared.down))
+        for c0 in range(0, T, shared_chunk):
+            out_ref[c0:c0 + shared_chunk] += oracle.expert_forward(sg, su, sd, x[c0:c0 + shared_chunk])[1]
+    acc_o = ErrorAccumulator("out (every token)")
+    acc_o.add(bf16_to_f64(out_bits), out_ref)
+    return acc_y.check(), acc_o.check()

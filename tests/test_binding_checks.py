@@ -68,14 +68,16 @@ def test_four_calls_and_layer_accept_the_test_patterns(rec, tiny):
         _lib.route(x, w_r, bias, stride, k, _i32(T, k), _f32(T, k), _ws(), logits=_f32(T, E), stream=0)
         _lib.layer(x, I, E, k, w_r, bias, stride, ex.table, sh.table, _i32(T, k), _f32(T, k), _bf16(T, H), _ws(),
                    stream=0)
+        _lib.layer(x, I, E, k, w_r, bias, stride, ex.table, sh.table, _i32(T, k), _f32(T, k), _bf16(T, H), _ws(),
+                   stream=0, logits=_f32(T, E))
         _lib.layer_decode_noalloc(x, I, E, k, w_r, bias, stride, ex.table, None, _i32(T, k), _f32(T, k),
-                                  _bf16(T, H), stream=0)
+                                  _bf16(T, H), stream=0, logits=_f32(T, E))
     _lib.dispatch(_i32(T, k), E, _i32(E), _i32(E + 1), _i32(T * k), _i32(T * k), _ws(), stream=0)
     _lib.expert_ffn(x, I, k, E, _i32(T * k), _i32(E + 1), _i32(E), ex.table, _bf16(T * k, H), _ws(), stream=0)
     _lib.combine(_bf16(T * k, H), _i32(T * k), _f32(T, k), I, x, sh.table, _bf16(T, H), _ws(), stream=0)
     _lib.combine(_bf16(T * k, H), _i32(T * k), _f32(T, k), I, None, None, _bf16(T, H), _ws(), stream=0)
     _lib.reset_status(_ws(), stream=0)
-    assert rec.calls.count("moe_route") == 3 and rec.calls.count("moe_layer") == 3
+    assert rec.calls.count("moe_route") == 3 and rec.calls.count("moe_layer") == 6
     assert rec.calls.count("moe_combine") == 2 and "moe_reset_status" in rec.calls
 
 
@@ -96,12 +98,13 @@ def test_zero_tokens_pass(rec):
 
 
 @pytest.mark.parametrize("case", ["transposed_x", "f32_x", "short_out", "short_counts", "stride_below_E",
-                                  "short_bias", "no_table", "short_table", "router_width", "i64_idx", "no_ws"])
+                                  "short_bias", "no_table", "short_table", "router_width", "i64_idx", "no_ws",
+                                  "short_logits"])
 def test_malformed_arguments_raise_before_the_call(rec, tiny, case):
     wl, lay, ex, sh = tiny
     T, k, E, H, I = wl.T, wl.k, wl.E, wl.H, wl.I
     a = dict(x=bf16_tensor(wlm.gen_x(wl), "cpu"), w_router=torch.from_numpy(lay.w_router), bias=torch.zeros(E),
-             stride=0, table=ex.table, idx=_i32(T, k), w=_f32(T, k), out=_bf16(T, H), ws=_ws())
+             stride=0, table=ex.table, idx=_i32(T, k), w=_f32(T, k), out=_bf16(T, H), ws=_ws(), logits=None)
     if case == "transposed_x":
         a["x"] = _bf16(H, T).t()
     elif case == "f32_x":
@@ -122,13 +125,15 @@ def test_malformed_arguments_raise_before_the_call(rec, tiny, case):
         a["idx"] = torch.empty((T, k), dtype=torch.int64)
     elif case == "no_ws":
         a["ws"] = None
+    elif case == "short_logits":
+        a["logits"] = _f32(T, E - 1)
     if case == "short_counts":
         with pytest.raises((ValueError, TypeError)):
             _lib.dispatch(_i32(T, k), E, _i32(E - 1), _i32(E + 1), _i32(T * k), _i32(T * k), _ws(), stream=0)
     else:
         with pytest.raises((ValueError, TypeError, AttributeError)):
             _lib.layer(a["x"], I, E, k, a["w_router"], a["bias"], a["stride"], a["table"], sh.table, a["idx"], a["w"],
-                       a["out"], a["ws"], stream=0)
+                       a["out"], a["ws"], stream=0, logits=a["logits"])
     assert rec.calls == []
 
 

@@ -121,7 +121,7 @@ def oracle_gates(xb, lay, bias, idx):
     return pu.oracle_gates_for(oracle.router_logits(xb, lay.w_router, bias), idx)
 
 
-def _layer_call(L, wl, dev, xb, bias, stride, ws):
+def _layer_call(L, wl, dev, xb, bias, stride, ws, with_logits=False):
     import torch
 
     from bit_quantized_moe_gemv_b200.device import bf16_bits, bf16_tensor
@@ -129,10 +129,13 @@ def _layer_call(L, wl, dev, xb, bias, stride, ws):
     idx = torch.empty((x.shape[0], wl.k), dtype=torch.int32, device="cuda")
     w = torch.empty((x.shape[0], wl.k), dtype=torch.float32, device="cuda")
     out = torch.empty((x.shape[0], wl.H), dtype=torch.bfloat16, device="cuda")
+    lg = torch.full((x.shape[0], wl.E), float("nan"), dtype=torch.float32, device="cuda") if with_logits else None
     L.layer(x, wl.I, wl.E, wl.k, dev["w_router"], pu.bias_tensor(bias), stride, dev["experts"].table,
-            dev["shared"].table if dev["shared"] else None, idx, w, out, ws)
+            dev["shared"].table if dev["shared"] else None, idx, w, out, ws, logits=lg)
     torch.cuda.synchronize()
     assert L.get_status(ws) == 0
+    if with_logits:
+        return idx.cpu().numpy(), w.cpu().numpy(), bf16_bits(out), lg.cpu().numpy()
     return idx.cpu().numpy(), w.cpu().numpy(), bf16_bits(out)
 
 
@@ -144,8 +147,10 @@ def test_layer_small(L, name):
     xb = wlm.gen_x(wl)
     bias, stride = wlm.gen_bias(wl)
     ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
-    idx, w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+    idx, w, out, lg = _layer_call(L, wl, dev, xb, bias, stride, ws, with_logits=True)
     ref = oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared)
+    ntied, _ = pu.check_routing(idx, w, lg, xb, lay.w_router, bias, wl.k)
+    assert ntied == 0
     np.testing.assert_array_equal(idx, ref["idx"])
     np.testing.assert_allclose(w, ref["w"], rtol=1e-5, atol=1e-6)
     pu.assert_close(pu.bf16_to_f64(out), ref["out"])
@@ -156,6 +161,10 @@ def test_layer_small(L, name):
 
 
 def _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, tokens):
+    """Outputs of the given tokens against the oracle. The routing must have
+    been checked first (pu.check_routing): the oracle evaluates the device's
+    picks, which equal its own except on flagged near-ties, where they are a
+    valid top-k within the fp32 rounding bound."""
     cache = oracle.DequantCache(lay.experts, capacity=256)
     sh = tuple(oracle.dequant_qm(m) for m in (lay.shared.gate, lay.shared.up, lay.shared.down))
     logits64 = oracle.router_logits(xb[tokens], lay.w_router, bias[tokens] if stride else bias)
@@ -176,18 +185,15 @@ def test_layer_decode1_steps(L):
     ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
     for step in range(6):
         xb = wlm.gen_x(wl, step=step)
-        idx, w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
-        logits64 = oracle.router_logits(xb, lay.w_router, bias)
-        ref_idx = oracle.topk_order(logits64, wl.k)
-        tau = pu.near_tie_tau(xb, lay.w_router, bias)
-        srt = -np.sort(-logits64, axis=1)[:, :wl.k + 1]
-        if not (np.diff(-srt, axis=1) < tau[:, None]).any():
-            np.testing.assert_array_equal(idx, ref_idx)
+        idx, w, out, lg = _layer_call(L, wl, dev, xb, bias, stride, ws, with_logits=True)
+        # selection exactly on the device's fp32 logits; against the fp64
+        # oracle bit for bit unless flagged, else a valid top-k within tau
+        pu.check_routing(idx, w, lg, xb, lay.w_router, bias, wl.k)
         _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, [0])
 
 
 @pytest.mark.parametrize("name", ["prefill8k", "prefill32k"])
-def test_prefill_full_routing_dispatch_sampled_outputs(L, name):
+def test_prefill_full_routing_dispatch_every_output(L, name):
     import torch
 
     from bit_quantized_moe_gemv_b200.device import bf16_tensor
@@ -218,11 +224,20 @@ def test_prefill_full_routing_dispatch_sampled_outputs(L, name):
     np.testing.assert_array_equal(offsets.cpu().numpy(), o)
     np.testing.assert_array_equal(perm.cpu().numpy(), p)
     np.testing.assert_array_equal(inv.cpu().numpy(), v)
-    # whole layer through moe_layer, sampled tokens against the oracle
-    out_idx, out_w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+    # the expert FFN alone: every dispatched row (bf16 y_perm)
+    from bit_quantized_moe_gemv_b200.device import bf16_bits
+    y_perm = torch.empty((T * k, wl.H), dtype=torch.bfloat16, device="cuda")
+    L.expert_ffn(x, wl.I, k, E, perm, offsets, counts, dev["experts"].table, y_perm, ws)
+    # whole layer through moe_layer: every output token
+    out_idx, out_w, out, out_lg = _layer_call(L, wl, dev, xb, bias, stride, ws, with_logits=True)
     np.testing.assert_array_equal(out_idx, gi)
+    np.testing.assert_array_equal(out_lg.view(np.uint32), logits.cpu().numpy().view(np.uint32))
+    (ry, my), (ro, mo) = pu.check_every_row(xb, lay.w_router, bias, k, lay.experts, lay.shared, gi,
+                                            perm.cpu().numpy(), offsets.cpu().numpy(), bf16_bits(y_perm), out)
+    print(f"{name}: y_perm rel {ry:.2e} max/rms {my:.2e}; out rel {ro:.2e} max/rms {mo:.2e}")
+    # and a few tokens through the per-token oracle path (moe_token)
     rng = np.random.default_rng(0)
-    tokens = sorted(set([0, T - 1] + rng.choice(T, 14, replace=False).tolist()))
+    tokens = sorted(set([0, T - 1] + rng.choice(T, 6, replace=False).tolist()))
     _check_sampled_tokens(wl, lay, xb, bias, stride, out_idx, out_w, out, tokens)
 
 
@@ -235,7 +250,8 @@ def test_decode48_two_layers(L):
         ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
         for step in (0, 199):
             xb = wlm.gen_x(wl, step=step, layer=layer)
-            idx, w, out = _layer_call(L, wl, dev, xb, bias, stride, ws)
+            idx, w, out, lg = _layer_call(L, wl, dev, xb, bias, stride, ws, with_logits=True)
+            pu.check_routing(idx, w, lg, xb, lay.w_router, bias, wl.k)
             _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, list(range(wl.T)))
 
 

@@ -100,6 +100,15 @@ def _bias_only_selects(x_bits, w_router, bias, k):
     return logits, idx, sel / sel.sum(axis=1, keepdims=True)
 
 
+def _bias_only_gates(x_bits, w_router, bias, k):
+    """Selection on the unbiased logits, gates from the biased softmax."""
+    logits = mo.router_logits(x_bits, w_router, bias)
+    idx = mo.topk_order(logits - np.asarray(bias, np.float64), k)
+    p = mo.softmax(logits)
+    sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
+    return logits, idx, sel / sel.sum(axis=1, keepdims=True)
+
+
 def _dispatch_descending(idx, E):
     counts, offsets, perm, inv = ORIG_DISPATCH(idx, E)
     perm = perm.copy()
@@ -149,6 +158,8 @@ def _pins_pass():
             pins.test_dequant_golden(case)
         for case in pins._routing_cases():
             pins.test_routing_closed_form(case)
+        for case in pins._routing_bias_cases():
+            pins.test_routing_bias_closed_form(case)
         pins.test_swiglu_expert_closed_form()
         pins.test_layer_closed_form_through_routing()
         for k in (1, 2, 3):
@@ -175,6 +186,7 @@ def _pins_pass():
     ("expert_forward", _sigmoid_for_silu),
     ("route", _gates_not_renormalised),
     ("route", _bias_only_selects),
+    ("route", _bias_only_gates),
     ("dispatch", _dispatch_descending),
     ("dispatch", _dispatch_inclusive_offsets),
     ("combine", _combine_without_shared),
@@ -187,3 +199,18 @@ def test_planted_mistake_is_caught(monkeypatch, target, mutant):
     monkeypatch.setattr(mo, target, mutant)
     monkeypatch.setattr(oracle, target, mutant)
     assert not _pins_pass(), f"a planted mistake in {target} went unnoticed"
+
+
+@pytest.mark.parametrize("mutant", [_bias_only_selects, _bias_only_gates])
+def test_bias_golden_alone_catches_bias_mistakes(monkeypatch, mutant):
+    """The hand-worked bias fixture pins the bias term by itself, without the
+    dense evaluation (which restates the same logit formula)."""
+    monkeypatch.setattr(mo, "route", mutant)
+    monkeypatch.setattr(oracle, "route", mutant)
+    failed = False
+    for case in pins._routing_bias_cases():
+        try:
+            pins.test_routing_bias_closed_form(case)
+        except AssertionError:
+            failed = True
+    assert failed

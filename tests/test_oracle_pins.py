@@ -66,6 +66,8 @@ def test_dequant_golden(case):
 
 
 def _parse_logits(tok):
+    if tok.startswith("-ln"):
+        return -math.log(float(tok[3:]))
     if tok.startswith("ln"):
         return math.log(float(tok[2:]))
     return float(tok)
@@ -93,6 +95,34 @@ def test_routing_closed_form(case):
     _, idx, w = oracle.route(wlm.f32_to_bf16_bits(x), w_r, np.zeros(E), k)
     assert idx[0].tolist() == idx_exp
     np.testing.assert_allclose(w[0], w_exp, rtol=0, atol=1e-15)
+
+
+def _routing_bias_cases():
+    cases = []
+    for line in open(os.path.join(GOLDEN, "routing_bias_closed_form.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        k, r, b, idx, w = [p.strip() for p in line.split("|")]
+        rows = lambda f, conv: [[conv(v) for v in part.split()] for part in f.split(";")]  # noqa: E731
+        cases.append((int(k), [_parse_logits(t) for t in r.split()], rows(b, _parse_logits), rows(idx, int),
+                      rows(w, float)))
+    return cases
+
+
+@pytest.mark.parametrize("case", _routing_bias_cases())
+def test_routing_bias_closed_form(case):
+    """The bias enters the logit: it moves the selection and the gates
+    (hand-worked values in tests/golden/routing_bias_closed_form.txt)."""
+    k, r, bias_rows, idx_exp, w_exp = case
+    E, H, T = len(r), 8, len(idx_exp)
+    x = np.zeros((T, H), dtype=np.float32)
+    x[:, 0] = 1.0
+    w_r = np.zeros((E, H), dtype=np.float64)
+    w_r[:, 0] = r
+    bias = np.asarray(bias_rows[0] if len(bias_rows) == 1 else bias_rows, dtype=np.float64)
+    _, idx, w = oracle.route(wlm.f32_to_bf16_bits(x), w_r, bias, k)
+    assert idx.tolist() == idx_exp
+    np.testing.assert_allclose(w, np.asarray(w_exp), rtol=0, atol=1e-15)
 
 
 def test_routing_k1_gate_is_exactly_one():

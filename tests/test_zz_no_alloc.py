@@ -1,15 +1,19 @@
-"""moe_layer_decode_noalloc against moe_layer, through the C ABI.
+"""moe_layer_decode_noalloc against moe_layer and the oracle, through the C ABI.
 
-The no-allocation entry point serves callers whose host code cannot allocate
-device memory (a host that owns every allocation and passes only inputs and
-outputs): it runs the fused decode step with scratch kept in a device array
-inside the library. Its output must match moe_layer's on the same inputs, on
-two calls in a row (the second call reuses the array the first one left
-behind). This file is collected last on purpose.
+The no-allocation entry point serves callers that cannot allocate device
+memory themselves: a host that owns every allocation and hands a kernel
+library only inputs and outputs (a plugin slot in another runtime, a process
+held to a fixed device-memory budget). It runs the same fused decode kernel
+as moe_layer with its scratch in a device array inside the library, so on
+the same inputs its outputs must be bit-identical to moe_layer's, on two
+calls in a row (the second call reuses the array the first one left behind).
+One call is also checked against the fp64 oracle. This file is collected
+last on purpose.
 """
 import numpy as np
 import pytest
 
+import oracle
 from bit_quantized_moe_gemv_b200 import workload as wlm
 from tests import parity_util as pu
 
@@ -30,32 +34,45 @@ def test_noalloc_matches_moe_layer_two_calls():
     bias, stride = wlm.gen_bias(wl)
     b = pu.bias_tensor(bias)
     ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+
+    def buffers():
+        return (torch.full((wl.T, wl.k), -1, dtype=torch.int32, device="cuda"),
+                torch.full((wl.T, wl.k), -1.0, dtype=torch.float32, device="cuda"),
+                torch.full((wl.T, wl.E), -1.0, dtype=torch.float32, device="cuda"),
+                torch.zeros((wl.T, wl.H), dtype=torch.bfloat16, device="cuda"))
+
     for step in range(2):
-        x = bf16_tensor(wlm.gen_x(wl, step=step))
-        ref_idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
-        ref_w = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
-        ref_out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+        xb = wlm.gen_x(wl, step=step)
+        x = bf16_tensor(xb)
+        r_idx, r_w, r_lg, r_out = buffers()
         L.layer(x, wl.I, wl.E, wl.k, dev["w_router"], b, stride, dev["experts"].table, dev["shared"].table,
-                ref_idx, ref_w, ref_out, ws)
-        idx = torch.full((wl.T, wl.k), -1, dtype=torch.int32, device="cuda")
-        w = torch.zeros((wl.T, wl.k), dtype=torch.float32, device="cuda")
-        out = torch.zeros((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+                r_idx, r_w, r_out, ws, logits=r_lg)
+        idx, w, lg, out = buffers()
         L.layer_decode_noalloc(x, wl.I, wl.E, wl.k, dev["w_router"], b, stride, dev["experts"].table,
-                               dev["shared"].table, idx, w, out)
+                               dev["shared"].table, idx, w, out, logits=lg)
         torch.cuda.synchronize()
-        assert L.get_status(ws) == 0
-        np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx.cpu().numpy())
-        np.testing.assert_allclose(w.cpu().numpy(), ref_w.cpu().numpy(), rtol=1e-6, atol=1e-7)
-        pu.assert_close(pu.bf16_to_f64(bf16_bits(out)), pu.bf16_to_f64(bf16_bits(ref_out)), f"call {step}")
+        assert L.get_status(ws) == 0  # moe_layer's own status word (the no-alloc one lives in the library)
+        # the same kernel on the same inputs: every output bit for bit
+        np.testing.assert_array_equal(idx.cpu().numpy(), r_idx.cpu().numpy())
+        np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), r_w.cpu().numpy().view(np.uint32))
+        np.testing.assert_array_equal(lg.cpu().numpy().view(np.uint32), r_lg.cpu().numpy().view(np.uint32))
+        np.testing.assert_array_equal(bf16_bits(out), bf16_bits(r_out))
+        if step == 1:
+            # and against the oracle: routing exactly (on the device's fp32
+            # logits; against the fp64 logits outside near-ties), outputs
+            # within the float tolerance
+            gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+            pu.check_routing(gi, gw, lg.cpu().numpy(), xb, lay.w_router, bias, wl.k)
+            ref = oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared,
+                                   routing=(gi, pu.oracle_gates_for(oracle.router_logits(xb, lay.w_router, bias), gi)))
+            pu.assert_close(pu.bf16_to_f64(bf16_bits(out)), ref["out"], "no-alloc out vs oracle")
 
 
 def test_noalloc_rejects_sizes_beyond_its_limits():
     from bit_quantized_moe_gemv_b200 import _lib as L
     lib = L.LIB
     # T = 5 exceeds the 4-token limit; E = 2048 and k = 17 exceed theirs.
-    assert lib.moe_layer_decode_noalloc(None, 5, 1024, 512, 64, 8, None, None, 0, None, None, None, None, None,
-                                        None) == 2
-    assert lib.moe_layer_decode_noalloc(None, 1, 1024, 512, 2048, 8, None, None, 0, None, None, None, None, None,
-                                        None) == 2
-    assert lib.moe_layer_decode_noalloc(None, 1, 1024, 512, 64, 17, None, None, 0, None, None, None, None, None,
-                                        None) == 2
+    args = (None, None, 0, None, None, None, None, None, None, None)
+    assert lib.moe_layer_decode_noalloc(None, 5, 1024, 512, 64, 8, *args) == 2
+    assert lib.moe_layer_decode_noalloc(None, 1, 1024, 512, 2048, 8, *args) == 2
+    assert lib.moe_layer_decode_noalloc(None, 1, 1024, 512, 64, 17, *args) == 2
