@@ -114,3 +114,56 @@ def test_tolerance_accepts_rounding_and_rejects_errors():
         assert_close(nan, ref)
     with pytest.raises(AssertionError):
         assert_close(ref[:, :-1], ref)
+
+
+def test_correctly_rounded_bf16_passes_even_with_outliers():
+    # heavy-tailed reference: a few elements far beyond 10 x rms, where the
+    # bf16 rounding alone exceeds 2e-2 x rms; the exact values rounded to
+    # bf16 must still pass, and an error of one more bf16 ulp must not
+    from tests.parity_util import bf16_half_ulp, round_bf16
+    rng = np.random.default_rng(7)
+    ref = rng.standard_normal((64, 256))
+    ref[3, 5], ref[9, 100] = 60.0 + 0.3, -45.0 - 0.17
+    assert_close(round_bf16(ref), ref)
+    bad = round_bf16(ref)
+    bad[3, 5] += 2 * bf16_half_ulp(ref[3, 5]) + MAX_ABS_RMS * np.sqrt(np.mean(ref ** 2))
+    with pytest.raises(AssertionError):
+        assert_close(bad, ref)
+
+
+def test_error_accumulator_matches_whole_array_check():
+    from tests.parity_util import ErrorAccumulator, round_bf16
+    rng = np.random.default_rng(8)
+    ref = rng.standard_normal((40, 64)) * 3
+    got = round_bf16(ref + 1e-3 * rng.standard_normal(ref.shape))
+    acc = ErrorAccumulator("pieces")
+    for i in range(0, 40, 7):
+        acc.add(got[i:i + 7], ref[i:i + 7])
+    rel, mx = acc.check()
+    rel2, mx2 = assert_close(got, ref)
+    assert abs(rel - rel2) < 1e-12 and abs(mx - mx2) < 1e-12
+    got[17, 3] += 0.5  # one planted wrong element
+    acc = ErrorAccumulator("pieces")
+    for i in range(0, 40, 7):
+        acc.add(got[i:i + 7], ref[i:i + 7])
+    with pytest.raises(AssertionError):
+        acc.check()
+
+
+def test_every_row_check_catches_one_wrong_row():
+    import oracle
+    from bit_quantized_moe_gemv_b200 import workload as wlm
+    from tests.parity_util import check_every_row
+    wl = wlm.WORKLOADS["tiny"]
+    lay, xb = wlm.gen_layer(wl), wlm.gen_x(wl)
+    bias, _ = wlm.gen_bias(wl)
+    r = oracle.moe_layer(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared)
+    f2b = lambda a: wlm.f32_to_bf16_bits(np.asarray(a, np.float32))  # noqa: E731
+    y, out = f2b(r["y_perm"]), f2b(r["out"])
+    check_every_row(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared, r["idx"], r["perm_src"], r["offsets"],
+                    y, out)
+    y_bad = y.copy()
+    y_bad[5] = f2b(r["y_perm"][5] * 1.05)  # one row 5 % off
+    with pytest.raises(AssertionError):
+        check_every_row(xb, lay.w_router, bias, wl.k, lay.experts, lay.shared, r["idx"], r["perm_src"],
+                        r["offsets"], y_bad, out)
