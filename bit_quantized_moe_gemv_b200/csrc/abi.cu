@@ -140,10 +140,11 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   const WsLayout L = ws_layout(T, H, I, E, k);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   WsHeader* hdr = ws_at<WsHeader>(ws, 0);
-  if (decode_stream_eligible(T, H, I, E, k))
-    return cuda_status(launch_decode_stream(x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev,
-                                            shared_dev, topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.partial),
-                                            ws_at<void>(ws, L.h), hdr, st));
+  if (decode_fused_eligible(T, H, I, E, k))
+    return cuda_status(launch_decode_fused(x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev,
+                                           topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.logits),
+                                           ws_at<float>(ws, L.dh), ws_at<uint32_t>(ws, L.dcnt), hdr,
+                                           kDefaultWaitCycles, st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
   int* perm = ws_at<int>(ws, L.perm);
@@ -176,7 +177,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
 
 moe_status moe_reset_status(void* ws, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+  return cuda_status(cudaMemsetAsync(ws, 0, kWsResetBytes, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_get_status(void* ws, void* stream, int32_t* device_status) {

@@ -1,0 +1,1059 @@
+// Decode step (1 <= T <= 4 tokens) as ONE persistent cooperative launch in
+// which every warp streams its own weights straight into registers.
+//
+// Decode reads each picked expert's weights once per step, so its floor is
+// memory bandwidth (the lcz.me forum thread "Halogen Flash Server配置與實測",
+// comment section: decode re-reads a fixed set of weights every step and its
+// ceiling follows bandwidth). The step itself is the one the telli.sh page
+// "Strata 与 Qwen3.8-Flash-Next：如何在个人电脑上运行 180B 级模型", section
+// "稀疏架构创造了机会", describes: 10 of 512 routed experts plus one shared
+// expert per token.
+//
+// Structure (one CTA of 16 warps per SM, all CTAs co-resident):
+//   A  router rows of this CTA (whole logits, one publication per CTA) and
+//      the shared expert's gate/up tiles of this CTA; the CTA then arrives on
+//      a grid counter and waits for every CTA's logits;
+//   -  every CTA reads all logits, takes the top-k itself (identical inputs,
+//      identical code, identical picks), lists the distinct picked experts
+//      and prefetches its down rows of each into L2;
+//   B  the routed gate/up tiles of this CTA (tile g of the step's list goes
+//      to CTA g mod G, so each expert's tiles finish early and together);
+//      finishing a tile publishes its 8 intermediate values h per token and
+//      bumps that expert's tile counter;
+//   C  this CTA's slice of output rows of every picked expert's down
+//      projection, each waiting only for ITS expert's counter (no second
+//      grid barrier); then the gate-weighted combine of those rows.
+// Every warp walks its own list of jobs (B jobs before C jobs, so a warp
+// waiting in C never holds back a tile that another waits for). A job is
+// 16 weight rows over a K range: each lane loads 16 bytes of codes of its
+// two rows per iteration, several iterations ahead, dequantises them in
+// registers and feeds mma.sync m16n8k16 (fp16 operands, fp32 accumulation)
+// with the T <= 4 tokens as the MMA's columns, read from shared memory in the
+// order the dequantisation produces pairs.
+//
+// Numerics: int4 and int2 weights become fp16 with one rounding (code times
+// the group scale, plus the min for int2), int8 codes are exact and their
+// row scale multiplies the fp32 result. Activations enter the MMA as fp16
+// after an exact power-of-two scaling that keeps them inside the fp16 range
+// (x per token; h per expert and token, from the largest |h| of that expert),
+// undone on the fp32 results: any finite bf16 input stays finite.
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include <algorithm>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace dfx {
+
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxT = 4;
+constexpr int kMaxK = 16;
+constexpr int kMaxSlots = kMaxT * kMaxK + 1;  // routed slots + the shared expert
+constexpr int kMaxJobs = 640;
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kTopChunk = 128;  // logits per first-round top-k job (4 per lane)
+
+enum : uint8_t { kRouter = 0, kGateUp = 1, kDown = 2 };
+
+// One warp's job. 8 bytes.
+struct Job {
+  uint8_t kind;
+  uint8_t slot;   // expert slot (shared = kSharedSlot); router: local row
+  uint8_t nrows;  // down: output rows (<= 16)
+  uint8_t part;   // gate/up: K part of nsplit; router: segment
+  uint16_t row0;  // gate/up: first intermediate row; down: first output row
+  uint16_t tile;  // gate/up: local tile index (reduction slot)
+};
+static_assert(sizeof(Job) == 8, "job record");
+constexpr int kSharedSlot = kMaxSlots - 1;
+
+// ---------------------------------------------------------------- formats
+// A 16-byte column of codes holds kc(F) weights of one row; its activations
+// for one token take wb(F) bytes per 32-bit word of codes, 4 words per column.
+__host__ __device__ constexpr int kc(int F) { return F == MOE_Q_INT4_SYM_G32 ? 32 : F == MOE_Q_INT2_ASYM_G16 ? 64 : 16; }
+__host__ __device__ constexpr int wbytes(int F) { return F == MOE_Q_INT4_SYM_G32 ? 16 : F == MOE_Q_INT2_ASYM_G16 ? 32 : 8; }
+__host__ __device__ constexpr int colbytes(int F) { return 4 * wbytes(F); }  // = 2 * kc(F)
+
+// Byte offset of activation (k, token t) in a buffer laid out for format F:
+// [column][token][word][pairs]. The dequantisation of a 32-bit code word
+// yields fp16 pairs, and MMA k-columns (2tq, 2tq+1) / (2tq+8, 2tq+9) take
+// them in this order:
+//   int4 word (8 nibbles i = 0..7):  (0,4) (1,5) | (2,6) (3,7)   two MMAs
+//   int2 word (16 codes i = 0..15):  (0,8) (1,9) | (2,10) (3,11) | ...  four MMAs
+//   int8 word (4 bytes i = 0..3):    (0,2) (1,3)                  one MMA
+__host__ __device__ inline int frag_pos(int F, int k, int t, int T) {
+  const int c = k / kc(F), p = k % kc(F);
+  int j, pos;
+  if (F == MOE_Q_INT4_SYM_G32) {
+    j = p >> 3;
+    const int i = p & 7;
+    pos = (i & 3) * 2 + (i >> 2);
+  } else if (F == MOE_Q_INT2_ASYM_G16) {
+    j = p >> 4;
+    const int i = p & 15;
+    pos = (i & 7) * 2 + (i >> 3);
+  } else {
+    j = p >> 2;
+    const int i = p & 3;
+    pos = (i & 1) * 2 + (i >> 1);
+  }
+  return (c * T + t) * colbytes(F) + j * wbytes(F) + pos * 2;
+}
+
+// K splits of a gate/up tile: two halves when each half is a whole number of
+// iterations (4 columns), else one.
+__host__ __device__ inline int gu_split(int F, int H) { return (H / 2) % (4 * kc(F)) == 0 ? 2 : 1; }
+
+// ---------------------------------------------------------------- plan
+// Dynamic shared memory, offsets from the base.
+struct Plan {
+  int o_x32;   // fp32 x [T][H] (router input, phase A only)
+  int o_hf;    // per-warp activations of a down job, 2 T I bytes each (phase C; over x32)
+  int o_xf;    // 3 activation buffers in fragment order, 2 T H bytes each
+  int o_lg;    // logits [T][E]
+  int o_rp;    // router partials [rows][segs][T]
+  int o_red;   // gate/up K-split sums [tiles][16][T]
+  int o_td;    // gate/up K-split arrivals [tiles]
+  int o_y;     // down results [kMaxSlots][16][T]
+  int o_jobs;  // job list
+  int o_desc;  // expert descriptors of the picked slots and the shared one
+  int total;
+};
+__host__ __device__ inline int router_rows(int E, int G) { return (E + G - 1) / G; }
+__host__ __device__ inline int router_seg(int H) { return H % 512 == 0 ? 512 : 256; }
+__host__ __device__ inline int max_tiles(int T, int I, int E, int k, int G) {
+  const int U = T * k < E ? T * k : E;
+  return (U * (I / 8) + G - 1) / G + (I / 8 + G - 1) / G;  // routed + shared
+}
+__host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int G) {
+  Plan p{};
+  int o = 0;
+  auto take = [&](int bytes, int al) {
+    o = (o + al - 1) / al * al;
+    const int r = o;
+    o += bytes;
+    return r;
+  };
+  const int x32 = 4 * T * H, hf = kWarps * 2 * T * I;
+  p.o_x32 = take(x32 > hf ? x32 : hf, 16);
+  p.o_hf = p.o_x32;
+  p.o_xf = take(3 * 2 * T * H, 16);
+  p.o_lg = take(4 * T * E, 16);
+  p.o_rp = take(4 * router_rows(E, G) * (H / router_seg(H)) * T, 16);
+  p.o_red = take(4 * max_tiles(T, I, E, k, G) * 16 * T, 16);
+  p.o_td = take(4 * max_tiles(T, I, E, k, G), 16);
+  p.o_y = take(4 * kMaxSlots * 16 * T, 16);
+  p.o_jobs = take(int(sizeof(Job)) * kMaxJobs, 16);
+  p.o_desc = take(int(sizeof(moe_expert)) * kMaxSlots, 16);
+  p.total = o;
+  return p;
+}
+
+// Output rows [n0, n0 + nr) of CTA b: H split as evenly as possible.
+__host__ __device__ inline void out_rows(int H, int G, int b, int& n0, int& nr) {
+  const int q = H / G, r = H % G;
+  n0 = b * q + (b < r ? b : r);
+  nr = q + (b < r ? 1 : 0);
+}
+// Router rows [e0, e0 + n) of CTA b.
+__host__ __device__ inline void router_range(int E, int G, int b, int& e0, int& n) {
+  const int rr = router_rows(E, G);
+  e0 = b * rr < E ? b * rr : E;
+  n = (e0 + rr < E ? e0 + rr : E) - e0;
+}
+// Local tiles of the shared expert on CTA b (tiles i = b, b + G, ... < I / 8).
+__host__ __device__ inline int shared_tiles(int I, int G, int b) { return I / 8 > b ? (I / 8 - 1 - b) / G + 1 : 0; }
+
+// Phase-A jobs of CTA b: router (row, segment), then the shared expert's
+// gate/up tiles in K parts (shared_fmt 0 = no shared expert). Returns the count.
+__host__ __device__ inline int phase_a_jobs(int H, int I, int E, int G, int b, int shared_fmt, Job* jobs) {
+  int e0, nrr;
+  router_range(E, G, b, e0, nrr);
+  const int nseg = H / router_seg(H);
+  int n = 0;
+  for (int r = 0; r < nrr; ++r)
+    for (int s = 0; s < nseg; ++s) jobs[n++] = Job{kRouter, uint8_t(r), 0, uint8_t(s), 0, 0};
+  if (shared_fmt) {
+    const int ns = gu_split(shared_fmt, H);
+    int lt = 0;
+    for (int i = b; i < I / 8; i += G, ++lt)
+      for (int p = 0; p < ns; ++p)
+        jobs[n++] = Job{kGateUp, uint8_t(kSharedSlot), 16, uint8_t(p), uint16_t(8 * i), uint16_t(lt)};
+  }
+  return n;
+}
+// Phase-B/C jobs of CTA b: gate/up tiles g = b, b + G, ... of the step's
+// expert-major list of U experts (fmt[u] their formats) in K parts; then one
+// down job per expert for this CTA's output rows, the shared one first.
+// Local tile indices continue after the shared expert's.
+__host__ __device__ inline int phase_bc_jobs(int H, int I, int G, int b, int U, const int* fmt, bool with_shared,
+                                             Job* jobs) {
+  int n = 0, lt = shared_tiles(I, G, b);
+  const int J = U * (I / 8);
+  for (int g = b; g < J; g += G, ++lt) {
+    const int u = g / (I / 8), i = g - u * (I / 8);
+    const int ns = gu_split(fmt[u], H);
+    for (int p = 0; p < ns; ++p) jobs[n++] = Job{kGateUp, uint8_t(u), 16, uint8_t(p), uint16_t(8 * i), uint16_t(lt)};
+  }
+  int n0, nr;
+  out_rows(H, G, b, n0, nr);
+  if (nr > 0) {
+    if (with_shared) jobs[n++] = Job{kDown, uint8_t(kSharedSlot), uint8_t(nr), 0, uint16_t(n0), 0};
+    for (int u = 0; u < U; ++u) jobs[n++] = Job{kDown, uint8_t(u), uint8_t(nr), 0, uint16_t(n0), 0};
+  }
+  return n;
+}
+
+struct Params {
+  const uint16_t* x;
+  int T, H, I, E, k;
+  const float* w_router;
+  const float* bias;
+  long long bstride;
+  const moe_expert* experts;
+  const moe_expert* shared;
+  int* topk_idx;
+  float* topk_w;
+  float* logits_out;
+  uint16_t* out;
+  WsHeader* hdr;
+  float* logits;   // [T][E] workspace
+  float* h;        // [kMaxSlots][T][I] workspace
+  uint32_t* cnt;   // [kMaxSlots] finished gate/up tiles per slot
+  uint32_t* amax;  // [kMaxSlots][kMaxT] bits of max |h| per slot and token
+  long long wait_cycles;
+};
+
+// ---------------------------------------------------------------- PTX bits
+__device__ __forceinline__ uint32_t lop_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));  // (a & mask) | magic
+  return d;
+}
+// ((a ^ 0x80) & 0xFF) | 0x6400 in each 16-bit half: byte q -> fp16 1024 + (q + 128).
+__device__ __forceinline__ uint32_t lop_i8(uint32_t a) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(0x00FF00FFu), "r"(0x64806480u));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2sub(uint32_t a, uint32_t b) {
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2mul(uint32_t a, uint32_t b) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2fma(uint32_t a, uint32_t b, uint32_t c) {
+  const __half2 r = __hfma2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b),
+                            *reinterpret_cast<const __half2*>(&c));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t dup16(uint32_t h) { return (h & 0xffffu) | (h << 16); }
+__device__ __forceinline__ void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                    uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint2 ldg8(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ldg2(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return uint32_t(v);
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void named_sync() { __syncthreads(); }
+
+// Power-of-two exponent that brings a magnitude below 2^15 (fp16 max 65504):
+// 0 for anything already below.
+__device__ __forceinline__ int range_exp(uint32_t abs_bits) {
+  const int e = int((abs_bits >> 23) & 0xff) - 127;  // floor(log2) of a finite positive float
+  return e >= 15 ? min(e - 14, 250) : 0;
+}
+
+// ---------------------------------------------------------------- tiles
+// Pointers of one lane's two rows in a matrix (A rows gq and gq + 8).
+struct Rows {
+  const uint8_t* c_lo;
+  const uint8_t* c_hi;
+  const uint16_t* s_lo;
+  const uint16_t* s_hi;
+  const uint16_t* m_lo;
+  const uint16_t* m_hi;
+  bool lo, hi;  // rows present
+};
+
+// Loads of one iteration (this lane's 16-byte column of both rows).
+struct Ld {
+  uint4 a, b;
+  uint2 sa, sb, ma, mb;  // int4: sa.x / sb.x = scale; int2: 4 scales / 4 mins each
+};
+
+template <int F>
+__device__ __forceinline__ void load_it(const Rows& R, int c, Ld& L) {
+  L.a = R.lo ? ldg16(R.c_lo + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.b = R.hi ? ldg16(R.c_hi + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  if (F == MOE_Q_INT4_SYM_G32) {
+    L.sa.x = R.lo ? ldg2(R.s_lo + c) : 0u;
+    L.sb.x = R.hi ? ldg2(R.s_hi + c) : 0u;
+  } else if (F == MOE_Q_INT2_ASYM_G16) {
+    L.sa = R.lo ? ldg8(R.s_lo + 4 * c) : make_uint2(0u, 0u);
+    L.sb = R.hi ? ldg8(R.s_hi + 4 * c) : make_uint2(0u, 0u);
+    L.ma = R.lo ? ldg8(R.m_lo + 4 * c) : make_uint2(0u, 0u);
+    L.mb = R.hi ? ldg8(R.m_hi + 4 * c) : make_uint2(0u, 0u);
+  }
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ uint32_t half_of(const uint2& v, int g) {  // g-th fp16 of four
+  const uint32_t w = g < 2 ? v.x : v.y;
+  return (g & 1) ? (w >> 16) : (w & 0xffffu);
+}
+
+// int4 word -> four fp16 pairs (c - 8) * s in the order of frag_pos.
+__device__ __forceinline__ void deq4(uint32_t w, uint32_t s2, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = h2mul(h2sub(lop_or(w, 0x000F000Fu, 0x64006400u), 0x64086408u), s2);   // (n0, n4): 1024 + n - 1032
+  p[1] = h2mul(h2sub(lop_or(w, 0x00F000F0u, 0x54005400u), 0x54805480u), s2);   // (n1, n5): 64 + n - 72
+  p[2] = h2mul(h2sub(lop_or(w8, 0x000F000Fu, 0x64006400u), 0x64086408u), s2);  // (n2, n6)
+  p[3] = h2mul(h2sub(lop_or(w8, 0x00F000F0u, 0x54005400u), 0x54805480u), s2);  // (n3, n7)
+}
+// int2 word (one group) -> eight fp16 pairs c * s + m, pair i = codes (i, i + 8).
+__device__ __forceinline__ void deq2(uint32_t w, uint32_t s2, uint32_t m2, uint32_t (&p)[8]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = h2fma(h2sub(lop_or(w, 0x00030003u, 0x64006400u), 0x64006400u), s2, m2);   // bits 0-1: 1024 + c
+  p[1] = h2fma(h2sub(lop_or(w, 0x000C000Cu, 0x5C005C00u), 0x5C005C00u), s2, m2);   // bits 2-3: 256 + c
+  p[2] = h2fma(h2sub(lop_or(w, 0x00300030u, 0x54005400u), 0x54005400u), s2, m2);   // bits 4-5: 64 + c
+  p[3] = h2fma(h2sub(lop_or(w, 0x00C000C0u, 0x4C004C00u), 0x4C004C00u), s2, m2);   // bits 6-7: 16 + c
+  p[4] = h2fma(h2sub(lop_or(w, 0x03000300u, 0x44004400u), 0x44004400u), s2, m2);   // bits 8-9: 4 + c
+  p[5] = h2fma(h2sub(lop_or(w8, 0x000C000Cu, 0x5C005C00u), 0x5C005C00u), s2, m2);  // bits 10-11
+  p[6] = h2fma(h2sub(lop_or(w8, 0x00300030u, 0x54005400u), 0x54005400u), s2, m2);  // bits 12-13
+  p[7] = h2fma(h2sub(lop_or(w8, 0x00C000C0u, 0x4C004C00u), 0x4C004C00u), s2, m2);  // bits 14-15
+}
+// int8 word -> two exact fp16 pairs (q0, q2), (q1, q3).
+__device__ __forceinline__ void deq8(uint32_t w, uint32_t (&p)[2]) {
+  p[0] = h2sub(lop_i8(w), 0x64806480u);
+  p[1] = h2sub(lop_i8(w >> 8), 0x64806480u);
+}
+
+// MMAs of one iteration: this lane's column c of both rows against the
+// activations of column c in `bf` (fragment order); only lanes gq < T read B.
+template <int F>
+__device__ __forceinline__ void mma_it(const Ld& L, const uint8_t* bf, int c, int T, float (&acc)[2][4]) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2;
+  const bool bv = gq < T;
+  const uint8_t* bp = bf + (size_t(c) * T + gq) * colbytes(F);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t wa = word(L.a, j), wb = word(L.b, j);
+    if (F == MOE_Q_INT4_SYM_G32) {
+      uint32_t pa[4], pb[4];
+      deq4(wa, dup16(L.sa.x), pa);
+      deq4(wb, dup16(L.sb.x), pb);
+      const uint4 b = bv ? *reinterpret_cast<const uint4*>(bp + j * 16) : make_uint4(0u, 0u, 0u, 0u);
+      mma(acc[0], pa[0], pb[0], pa[1], pb[1], b.x, b.y);
+      mma(acc[1], pa[2], pb[2], pa[3], pb[3], b.z, b.w);
+    } else if (F == MOE_Q_INT2_ASYM_G16) {
+      uint32_t pa[8], pb[8];
+      deq2(wa, dup16(half_of(L.sa, j)), dup16(half_of(L.ma, j)), pa);
+      deq2(wb, dup16(half_of(L.sb, j)), dup16(half_of(L.mb, j)), pb);
+      const uint4 b0 = bv ? *reinterpret_cast<const uint4*>(bp + j * 32) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 b1 = bv ? *reinterpret_cast<const uint4*>(bp + j * 32 + 16) : make_uint4(0u, 0u, 0u, 0u);
+      mma(acc[0], pa[0], pb[0], pa[1], pb[1], b0.x, b0.y);
+      mma(acc[1], pa[2], pb[2], pa[3], pb[3], b0.z, b0.w);
+      mma(acc[0], pa[4], pb[4], pa[5], pb[5], b1.x, b1.y);
+      mma(acc[1], pa[6], pb[6], pa[7], pb[7], b1.z, b1.w);
+    } else {
+      uint32_t pa[2], pb[2];
+      deq8(wa, pa);
+      deq8(wb, pb);
+      const uint2 b = bv ? *reinterpret_cast<const uint2*>(bp + j * 8) : make_uint2(0u, 0u);
+      mma(acc[j & 1], pa[0], pb[0], pa[1], pb[1], b.x, b.y);
+    }
+  }
+}
+
+// Iterations of loads in flight per lane (int2 carries 4 scales and 4 mins
+// per row and iteration, so it keeps fewer in registers).
+__host__ __device__ constexpr int depth(int F) { return F == MOE_Q_INT2_ASYM_G16 ? 2 : 4; }
+
+// One warp's share of a tile: iterations it = 0..nit-1, lane column
+// c = col0 + 4 it + tq; the loads of depth(F) iterations are in flight while
+// one is computed. Returns this lane's four accumulators (D rows gq, gq + 8;
+// token columns 2 tq, 2 tq + 1). One function per format, so each gets its
+// own register allocation.
+template <int F>
+__device__ __noinline__ float4 run_tile(const Rows R, int col0, int nit, const uint8_t* bf, int T) {
+  const int tq = threadIdx.x & 3;
+  constexpr int kDepth = depth(F);
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  Ld L[kDepth];
+#pragma unroll
+  for (int s = 0; s < kDepth; ++s)
+    if (s < nit) load_it<F>(R, col0 + 4 * s + tq, L[s]);
+#pragma unroll 1
+  for (int it0 = 0; it0 < nit; it0 += kDepth) {
+#pragma unroll
+    for (int s = 0; s < kDepth; ++s) {
+      const int it = it0 + s;
+      if (it < nit) {
+        mma_it<F>(L[s], bf, col0 + 4 * it + tq, T, acc);
+        if (it + kDepth < nit) load_it<F>(R, col0 + 4 * (it + kDepth) + tq, L[s]);
+      }
+    }
+  }
+  return make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+}
+__device__ __forceinline__ void run_any(int f, const Rows& R, int col0, int nit, const uint8_t* bf, int T,
+                                        float (&acc)[4]) {
+  const float4 v = f == MOE_Q_INT4_SYM_G32   ? run_tile<MOE_Q_INT4_SYM_G32>(R, col0, nit, bf, T)
+                   : f == MOE_Q_INT2_ASYM_G16 ? run_tile<MOE_Q_INT2_ASYM_G16>(R, col0, nit, bf, T)
+                                              : run_tile<MOE_Q_INT8_PER_CHANNEL>(R, col0, nit, bf, T);
+  acc[0] = v.x;
+  acc[1] = v.y;
+  acc[2] = v.z;
+  acc[3] = v.w;
+}
+
+// ---------------------------------------------------------------- top-k keys
+__device__ __forceinline__ uint32_t f2key(float f) {
+  if (f != f) f = -CUDART_INF_F;  // NaN loses to every number
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key2f(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+__device__ __forceinline__ void cswap(uint64_t& a, uint64_t& b) {
+  const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+  a = hi;
+  b = lo;
+}
+// Best k (k <= 16) of up to 128 candidates held 4 per lane as key << 32 |
+// ~id (a larger value is better: key descending, then id ascending; 0 = no
+// candidate). Each lane sorts its four; every round takes the best lane head
+// by a reduction on the key and one on the low word among equal keys, and the
+// winning lane pops it.
+__device__ __forceinline__ void warp_topk(uint64_t (&c)[4], int k, uint32_t* okey, int* oid) {
+  const int lane = threadIdx.x & 31;
+  cswap(c[0], c[1]);
+  cswap(c[2], c[3]);
+  cswap(c[0], c[2]);
+  cswap(c[1], c[3]);
+  cswap(c[1], c[2]);
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    const uint32_t hk = uint32_t(c[0] >> 32), lk = uint32_t(c[0]);
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, hk);
+    const uint32_t wl = __reduce_max_sync(0xffffffffu, hk == wk ? lk : 0u);
+    if (lane == 0) {
+      okey[j] = wk;
+      oid[j] = wk ? int(~wl) : 0x7fffffff;
+    }
+    if (wk != 0u && hk == wk && lk == wl) {
+      c[0] = c[1];
+      c[1] = c[2];
+      c[2] = c[3];
+      c[3] = 0ull;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- bounded waits
+// Spin (one thread) until *p >= target, the abort flag is raised or the
+// cycle budget runs out. Returns true when the target was reached.
+__device__ bool wait_counter(const uint32_t* p, uint32_t target, WsHeader* hdr, long long budget, int detail) {
+  if (ld_acquire(p) >= target) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire(p) >= target) return true;
+    if ((it & 15) == 0) {
+      if (*reinterpret_cast<volatile int*>(&hdr->abort)) return false;
+      if (clock64() - t0 > budget) {
+        flag_error(hdr, MOE_ERR_TIMEOUT, detail);
+        atomicExch(&hdr->abort, 1);
+        return false;
+      }
+    }
+    __nanosleep(32);
+  }
+}
+
+// ---------------------------------------------------------------- job context
+// What every job reads: set up once per launch in shared memory.
+struct Ctx {
+  const Params* P;
+  uint8_t* smem;
+  Plan L;
+  int T, H, I, E, k, G, b;
+  int e0, nrr, seg, nseg;   // router rows [e0, e0 + nrr), segments per row
+  int n0, nr;               // output rows of this CTA
+  int fmap[4];              // weight format -> activation buffer (or -1)
+  int xexp[kMaxT];          // power-of-two scaling of x per token
+  int fail;                 // a wait of this CTA gave up
+  int rdone;                // router jobs finished
+  moe_expert* desc;         // descriptors: slots 0..U-1, kSharedSlot
+};
+
+// gate/up tile part: 8 intermediate rows of gate (A rows 0-7) and of up
+// (A rows 8-15) over part p of K. The last part to finish sums the parts
+// (two fp32 values: the same sum in either order), applies SwiGLU and
+// publishes h, its largest |h| per token and one more finished tile of its
+// expert.
+__device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
+  const Params& P = *C.P;
+  const int T = C.T, H = C.H, I = C.I;
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const int slot = jb.slot;
+  const moe_expert& d = C.desc[slot];
+  const int f = d.gate.qtype, ns = gu_split(f, H);
+  const int ncol = H / kc(f) / ns, col0 = jb.part * ncol, nit = ncol / 4;
+  const int rb = row_code_bytes(f, H);
+  const int row = jb.row0 + gq;
+  const int sper = f == MOE_Q_INT8_PER_CHANNEL ? 1 : H / (f == MOE_Q_INT4_SYM_G32 ? 32 : 16);
+  Rows R;
+  R.lo = R.hi = true;
+  R.c_lo = d.gate.codes + size_t(row) * rb;
+  R.c_hi = d.up.codes + size_t(row) * rb;
+  R.s_lo = d.gate.scales + size_t(row) * sper;
+  R.s_hi = d.up.scales + size_t(row) * sper;
+  R.m_lo = f == MOE_Q_INT2_ASYM_G16 ? d.gate.mins + size_t(row) * sper : nullptr;
+  R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.up.mins + size_t(row) * sper : nullptr;
+  const uint8_t* bf = C.smem + C.L.o_xf + C.fmap[f] * 2 * T * H;
+  float acc[4];
+  run_any(f, R, col0, nit, bf, T, acc);
+  // D rows gq (gate) / gq + 8 (up), tokens 2 tq, 2 tq + 1
+  if (ns > 1) {
+    float* rs = reinterpret_cast<float*>(C.smem + C.L.o_red) + size_t(jb.tile) * 16 * T;
+    int* td = reinterpret_cast<int*>(C.smem + C.L.o_td) + jb.tile;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = gq + 8 * (i >> 1), t = 2 * tq + (i & 1);
+      if (t < T) atomicAdd(rs + r * T + t, acc[i]);
+    }
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) {
+      __threadfence_block();
+      prev = atomicAdd(td, 1);
+    }
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != ns - 1) return;
+    __threadfence_block();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = gq + 8 * (i >> 1), t = 2 * tq + (i & 1);
+      acc[i] = t < T ? *reinterpret_cast<volatile float*>(rs + r * T + t) : 0.f;
+    }
+  }
+  float* hs = P.h + size_t(slot) * T * I;
+  uint32_t* am = P.amax + slot * kMaxT;
+  float gsc = 1.f, usc = 1.f;
+  if (f == MOE_Q_INT8_PER_CHANNEL) {
+    gsc = f16_to_f32(d.gate.scales[row]);
+    usc = f16_to_f32(d.up.scales[row]);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int t = 2 * tq + i;
+    float h = 0.f;
+    if (t < T) {
+      const float sc = ldexpf(1.f, C.xexp[t]);
+      const float g = acc[i] * gsc * sc, u = acc[2 + i] * usc * sc;
+      h = silu_f32(g) * u;
+      __stcg(hs + size_t(t) * I + row, h);
+    }
+    // largest |h| of the tile per token: lanes of equal tq hold the same token
+    uint32_t a = t < T ? __float_as_uint(fabsf(h)) : 0u;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if (gq == 0 && t < T) atomicMax(am + t, a);
+  }
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) red_release(P.cnt + slot, 1u);
+}
+
+// down job: this CTA's output rows [n0, n0 + nr) of one expert (already on
+// their way into L2 since the top-k). The warp waits for the expert's
+// gate/up tiles, converts h (scaled into the fp16 range) into its own
+// activation buffer and runs the MMAs. Results go to Y[slot].
+__device__ __noinline__ void job_down(Ctx& C, const Job jb) {
+  const Params& P = *C.P;
+  const int T = C.T, I = C.I;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const int slot = jb.slot;
+  const moe_expert& d = C.desc[slot];
+  const int f = d.down.qtype;
+  const int nit = I / kc(f) / 4;
+  const int rb = row_code_bytes(f, I);
+  const int sper = f == MOE_Q_INT8_PER_CHANNEL ? 1 : I / (f == MOE_Q_INT4_SYM_G32 ? 32 : 16);
+  const int rlo = jb.row0 + gq, rhi = jb.row0 + gq + 8;
+  Rows R;
+  R.lo = gq < jb.nrows;
+  R.hi = gq + 8 < jb.nrows;
+  R.c_lo = d.down.codes + size_t(R.lo ? rlo : 0) * rb;
+  R.c_hi = d.down.codes + size_t(R.hi ? rhi : 0) * rb;
+  R.s_lo = d.down.scales + size_t(R.lo ? rlo : 0) * sper;
+  R.s_hi = d.down.scales + size_t(R.hi ? rhi : 0) * sper;
+  R.m_lo = f == MOE_Q_INT2_ASYM_G16 ? d.down.mins + size_t(R.lo ? rlo : 0) * sper : nullptr;
+  R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.down.mins + size_t(R.hi ? rhi : 0) * sper : nullptr;
+  uint8_t* hf = C.smem + C.L.o_hf + warp * 2 * T * I;
+  __shared__ int s_eh[kWarps][kMaxT];
+  int ok = 1;
+  if (lane == 0) ok = wait_counter(P.cnt + slot, uint32_t(I / 8), P.hdr, P.wait_cycles, 7100000 + slot) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (!ok) {
+    if (lane == 0) C.fail = 1;
+    return;
+  }
+  (void)ld_acquire(P.cnt + slot);  // every lane orders its reads of h after the counter
+  if (lane < T) s_eh[warp][lane] = range_exp(__ldcg(P.amax + slot * kMaxT + lane));
+  __syncwarp();
+  const float* hs = P.h + size_t(slot) * T * I;
+  for (int i = 4 * lane; i < T * I; i += 128) {  // I % 4 == 0: four values of one token
+    const int t = i / I, kk = i - t * I;
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(hs + i));
+    const int e = s_eh[warp][t];
+    *reinterpret_cast<__half*>(hf + frag_pos(f, kk, t, T)) = __float2half_rn(ldexpf(v.x, -e));
+    *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 1, t, T)) = __float2half_rn(ldexpf(v.y, -e));
+    *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 2, t, T)) = __float2half_rn(ldexpf(v.z, -e));
+    *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 3, t, T)) = __float2half_rn(ldexpf(v.w, -e));
+  }
+  __syncwarp();
+  float acc[4];
+  run_any(f, R, 0, nit, hf, T, acc);
+  float* y = reinterpret_cast<float*>(C.smem + C.L.o_y) + size_t(slot) * 16 * T;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = gq + 8 * (i >> 1), t = 2 * tq + (i & 1);
+    if (r < jb.nrows && t < T) {
+      float v = ldexpf(acc[i], s_eh[warp][t]);
+      if (f == MOE_Q_INT8_PER_CHANNEL) v *= f16_to_f32(d.down.scales[jb.row0 + r]);
+      y[r * T + t] = v;
+    }
+  }
+  __syncwarp();
+}
+
+// router part: row e0 + r, floats [s seg, (s + 1) seg) of it; the last part
+// of the CTA to finish sums each row's parts in order, adds the bias,
+// publishes the logits and arrives on the grid counter.
+__device__ __noinline__ void job_router(Ctx& C, const Job jb) {
+  const Params& P = *C.P;
+  const int T = C.T, H = C.H, E = C.E, seg = C.seg, nseg = C.nseg;
+  const int lane = threadIdx.x & 31;
+  const float* x32 = reinterpret_cast<const float*>(C.smem + C.L.o_x32);
+  float* rp = reinterpret_cast<float*>(C.smem + C.L.o_rp);
+  const int e = C.e0 + jb.slot;
+  const float* wr = P.w_router + size_t(e) * H + jb.part * seg;
+  const int nv = seg / 128;  // 16-byte loads per lane (4 or 2)
+  uint4 w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (i < nv) w[i] = ldg16(wr + 4 * lane + 128 * i);
+#pragma unroll
+  for (int t = 0; t < kMaxT; ++t) {
+    if (t >= T) break;
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i < nv) {
+        const float4 xv = *reinterpret_cast<const float4*>(x32 + t * H + jb.part * seg + 4 * lane + 128 * i);
+        a = fmaf(__uint_as_float(w[i].x), xv.x,
+                 fmaf(__uint_as_float(w[i].y), xv.y, fmaf(__uint_as_float(w[i].z), xv.z, fmaf(__uint_as_float(w[i].w), xv.w, a))));
+      }
+    a = warp_sum(a);
+    if (lane == 0) rp[(jb.slot * nseg + jb.part) * T + t] = a;
+  }
+  __syncwarp();
+  int prev = 0;
+  if (lane == 0) {
+    __threadfence_block();
+    prev = atomicAdd(&C.rdone, 1);
+  }
+  prev = __shfl_sync(0xffffffffu, prev, 0);
+  if (prev != C.nrr * nseg - 1) return;
+  __threadfence_block();
+  for (int i = lane; i < C.nrr * T; i += 32) {
+    const int r = i / T, t = i - r * T;
+    float a = 0.f;
+    for (int s = 0; s < nseg; ++s) a += *reinterpret_cast<volatile float*>(rp + (r * nseg + s) * T + t);
+    const float bv = P.bias ? P.bias[t * P.bstride + C.e0 + r] : 0.f;
+    __stcg(P.logits + size_t(t) * E + C.e0 + r, a + bv);
+  }
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) red_release(&P.hdr->bar_count, 1u);
+}
+
+// ---------------------------------------------------------------- the kernel
+__global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ Params P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ Ctx C;
+  __shared__ uint32_t s_xamax[kMaxT];
+  __shared__ int s_nA, s_nJ, s_U, s_bad;
+  __shared__ int s_idx[kMaxT * kMaxK];
+  __shared__ float s_w[kMaxT * kMaxK];
+  __shared__ uint32_t s_key[kMaxT * kMaxK];
+  __shared__ int s_slot[kMaxT * kMaxK];         // (t, j) -> slot
+  __shared__ int s_uniq[kMaxT * kMaxK];         // slot -> expert id
+  __shared__ int s_fmt[kMaxT * kMaxK];          // slot -> weight format
+  __shared__ uint32_t s_ck[kMaxT * 8 * kMaxK];  // first-round winners
+  __shared__ int s_ci[kMaxT * 8 * kMaxK];
+  __shared__ uint32_t s_bits[kMaxE / 32];
+  __shared__ uint32_t s_bpre[kMaxE / 32];
+
+  const int T = P.T, H = P.H, I = P.I, E = P.E, k = P.k;
+  const int G = gridDim.x, b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WsHeader* hdr = P.hdr;
+  const bool has_shared = P.shared != nullptr;
+  moe_expert* desc = reinterpret_cast<moe_expert*>(smem + make_plan(T, H, I, E, k, G).o_desc);
+
+  // ---------------------------------------------------------- prologue
+  if (threadIdx.x == 0) {
+    C.P = &P;
+    C.smem = smem;
+    C.L = make_plan(T, H, I, E, k, G);
+    C.T = T, C.H = H, C.I = I, C.E = E, C.k = k, C.G = G, C.b = b;
+    router_range(E, G, b, C.e0, C.nrr);
+    C.seg = router_seg(H);
+    C.nseg = H / C.seg;
+    out_rows(H, G, b, C.n0, C.nr);
+    for (int i = 0; i < 4; ++i) C.fmap[i] = -1;
+    C.fail = 0;
+    C.rdone = 0;
+    C.desc = desc;
+    s_bad = 0;
+    s_U = 0;
+  }
+  if (threadIdx.x < kMaxT) s_xamax[threadIdx.x] = 0u;
+  if (has_shared && threadIdx.x < int(sizeof(moe_expert) / 4))
+    reinterpret_cast<uint32_t*>(desc + kSharedSlot)[threadIdx.x] =
+        reinterpret_cast<const uint32_t*>(P.shared)[threadIdx.x];
+  __syncthreads();
+  const Plan& L = C.L;
+  const int ntl = max_tiles(T, I, E, k, G);
+  {
+    float* Y = reinterpret_cast<float*>(smem + L.o_y);
+    float* red = reinterpret_cast<float*>(smem + L.o_red);
+    int* tdone = reinterpret_cast<int*>(smem + L.o_td);
+    for (int i = threadIdx.x; i < kMaxSlots * 16 * T; i += kThreads) Y[i] = 0.f;
+    for (int i = threadIdx.x; i < ntl * 16 * T; i += kThreads) red[i] = 0.f;
+    for (int i = threadIdx.x; i < ntl; i += kThreads) tdone[i] = 0;
+  }
+  // x in fp32 (router) and the largest |x| per token
+  {
+    float* x32 = reinterpret_cast<float*>(smem + L.o_x32);
+    for (int i = threadIdx.x; i < T * H; i += kThreads) {
+      const float v = bf16_to_f32(P.x[i]);
+      x32[i] = v;
+      // a warp's 32 consecutive elements belong to one token (H % 32 == 0)
+      // and are all in range together (T H % 32 == 0)
+      const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v)));
+      if (lane == 0) atomicMax(&s_xamax[i / H], m);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < T) C.xexp[threadIdx.x] = range_exp(s_xamax[threadIdx.x]);
+  if (threadIdx.x == 0) {
+    bool good = true;
+    if (has_shared) {
+      good = expert_ok(desc[kSharedSlot], H, I);
+      if (!good) {
+        s_bad = 1;
+        flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
+      } else if (C.nr > 0) {
+        // the shared expert's down rows of this CTA into L2: needed whatever the routing
+        const moe_qmatrix& d = desc[kSharedSlot].down;
+        const int rb = row_code_bytes(d.qtype, I);
+        prefetch_l2(d.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
+      }
+    }
+    s_nA = phase_a_jobs(H, I, E, G, b, has_shared && good ? desc[kSharedSlot].gate.qtype : 0,
+                        reinterpret_cast<Job*>(smem + C.L.o_jobs));
+  }
+  __syncthreads();
+  const int nA = s_nA;
+  // activations of format f in fragment order (from global x: x32 is reused
+  // after phase A)
+  auto build_xf = [&](int f, int buf) {
+    uint8_t* xf = smem + L.o_xf + buf * 2 * T * H;
+    for (int i = threadIdx.x; i < T * H; i += kThreads) {
+      const int t = i / H, kk = i - t * H;
+      const float v = ldexpf(bf16_to_f32(P.x[i]), -C.xexp[t]);
+      *reinterpret_cast<__half*>(xf + frag_pos(f, kk, t, T)) = __float2half_rn(v);
+    }
+  };
+  if (has_shared && !s_bad) {
+    build_xf(desc[kSharedSlot].gate.qtype, 0);
+    if (threadIdx.x == 0) C.fmap[desc[kSharedSlot].gate.qtype] = 0;
+  }
+  if (C.nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
+  __syncthreads();
+
+  // ---------------------------------------------------------- phase A
+  {
+    const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs);
+    for (int j = warp; j < nA; j += kWarps) {
+      const Job jb = jobs[j];
+      if (jb.kind == kRouter) job_router(C, jb);
+      else job_gate_up(C, jb);
+    }
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------- routing
+  if (threadIdx.x == 0)
+    if (!wait_counter(&hdr->bar_count, uint32_t(G), hdr, P.wait_cycles, 7000000 + b)) C.fail = 1;
+  __syncthreads();
+  const bool live = !C.fail;
+  float* lg = reinterpret_cast<float*>(smem + L.o_lg);
+  if (live)
+    for (int i = threadIdx.x; i < T * E; i += kThreads) lg[i] = __ldcg(P.logits + i);
+  __syncthreads();
+  // two rounds of warp top-k: one job per (token, 128 logits), each keeping
+  // its chunk's best k; then one warp per token over those (<= 8 x 16 = 128)
+  const int nch = (E + kTopChunk - 1) / kTopChunk;
+  for (int stage = 0; stage < 2; ++stage) {
+    const int njobs = live ? (stage == 0 ? T * nch : T) : 0;
+    for (int jbi = warp; jbi < njobs; jbi += kWarps) {
+      const int t = stage == 0 ? jbi / nch : jbi, ch = stage == 0 ? jbi - t * nch : 0;
+      const int nc = stage == 0 ? min(kTopChunk, E - ch * kTopChunk) : nch * k;
+      const uint32_t* ck = s_ck + t * 8 * kMaxK;
+      const int* ci = s_ci + t * 8 * kMaxK;
+      uint64_t cand[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        const uint32_t key = c >= nc ? 0u : stage == 0 ? f2key(lg[t * E + ch * kTopChunk + c]) : ck[c];
+        const int id = stage == 0 ? ch * kTopChunk + c : ci[c < nc ? c : 0];
+        cand[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(id)) : 0ull;
+      }
+      uint32_t* okey = stage == 0 ? s_ck + t * 8 * kMaxK + ch * k : s_key + t * k;
+      int* oid = stage == 0 ? s_ci + t * 8 * kMaxK + ch * k : s_idx + t * k;
+      warp_topk(cand, k, okey, oid);
+    }
+    __syncthreads();
+  }
+  // gates: the softmax over all logits restricted to the picks and
+  // renormalised = a softmax over the picked logits
+  if (live && warp < T) {
+    const int t = warp;
+    const float v0 = key2f(s_key[t * k]);
+    float part = 0.f;
+    for (int j = lane; j < k; j += 32) part += expf(key2f(s_key[t * k + j]) - v0);
+    const float den = warp_sum(part);
+    for (int j = lane; j < k; j += 32) s_w[t * k + j] = expf(key2f(s_key[t * k + j]) - v0) / den;
+  }
+  // distinct picked experts in ascending id order through a bitmap: the
+  // slot of an id is the number of set bits below it
+  const int nk = T * k;
+  for (int i = threadIdx.x; i < kMaxE / 32; i += kThreads) s_bits[i] = 0u;
+  __syncthreads();
+  if (live && threadIdx.x < nk) {
+    const int id = s_idx[threadIdx.x];
+    if (id >= 0 && id < E) atomicOr(&s_bits[id >> 5], 1u << (id & 31));
+    else s_bad = 1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t pre = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32 / 32; ++i) {
+      const uint32_t c = __popc(s_bits[i * 32 + lane]);
+      uint32_t inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      s_bpre[i * 32 + lane] = pre + inc - c;
+      pre += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) s_U = int(pre);
+  }
+  __syncthreads();
+  const int U = s_U;
+  if (live && !s_bad && threadIdx.x < nk) {
+    const int id = s_idx[threadIdx.x], w = id >> 5;
+    const int rank = int(s_bpre[w] + __popc(s_bits[w] & ((1u << (id & 31)) - 1u)));
+    s_slot[threadIdx.x] = rank;
+    s_uniq[rank] = id;
+  }
+  __syncthreads();
+  if (live && !s_bad) {
+    constexpr int W = int(sizeof(moe_expert) / 4);
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
+    for (int i = threadIdx.x; i < U * W; i += kThreads) dst[i] = src[size_t(s_uniq[i / W]) * W + (i % W)];
+    if (b == 0) {
+      for (int i = threadIdx.x; i < nk; i += kThreads) {
+        P.topk_idx[i] = s_idx[i];
+        P.topk_w[i] = s_w[i];
+      }
+      if (P.logits_out)
+        for (int i = threadIdx.x; i < T * E; i += kThreads) P.logits_out[i] = lg[i];
+    }
+  }
+  __syncthreads();
+  if (live && !s_bad && threadIdx.x < U)
+    if (!expert_ok(desc[threadIdx.x], H, I)) s_bad = 1;
+  __syncthreads();
+  const bool work = live && !s_bad;
+  if (live && s_bad && threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 1000000);
+  if (work) {
+    // activations of the routed formats not built yet
+    for (int f = 1; f <= 3; ++f) {
+      bool used = false;
+      for (int u = 0; u < U; ++u) used |= desc[u].gate.qtype == f;
+      if (used && C.fmap[f] < 0) {
+        int nb = 0;
+        for (int g = 1; g <= 3; ++g) nb += C.fmap[g] >= 0;
+        __syncthreads();
+        if (threadIdx.x == 0) C.fmap[f] = nb;
+        build_xf(f, nb);
+        __syncthreads();
+      }
+    }
+    // this CTA's down rows of every picked expert into L2
+    if (C.nr > 0 && threadIdx.x >= 32 && threadIdx.x < 32 + U) {
+      const moe_qmatrix& dm = desc[threadIdx.x - 32].down;
+      const int rb = row_code_bytes(dm.qtype, I);
+      prefetch_l2(dm.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
+    }
+    if (threadIdx.x < U) s_fmt[threadIdx.x] = desc[threadIdx.x].gate.qtype;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      s_nJ = phase_bc_jobs(H, I, G, b, U, s_fmt, has_shared, reinterpret_cast<Job*>(smem + L.o_jobs));
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------- phases B, C
+  if (work) {
+    const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs);
+    const int nJ = s_nJ;
+    for (int j = warp; j < nJ; j += kWarps) {
+      const Job jb = jobs[j];
+      if (jb.kind == kGateUp) job_gate_up(C, jb);
+      else job_down(C, jb);
+    }
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------- combine
+  if (work && !C.fail) {
+    const float* Y = reinterpret_cast<const float*>(smem + L.o_y);
+    const int nr = C.nr, n0 = C.n0;
+    for (int i = threadIdx.x; i < T * nr; i += kThreads) {
+      const int t = i / nr, r = i - t * nr;
+      float a = 0.f;
+      for (int j = 0; j < k; ++j) a = fmaf(s_w[t * k + j], Y[(s_slot[t * k + j] * 16 + r) * T + t], a);
+      if (has_shared) a += Y[(kSharedSlot * 16 + r) * T + t];
+      P.out[size_t(t) * H + n0 + r] = f32_to_bf16_rn(a);
+    }
+  }
+
+  // ---------------------------------------------------------- exit
+  // The last CTA out clears the launch's counters for the next launch.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(&hdr->exit_count, 1u);
+    if (prev == uint32_t(G) - 1) {
+      __threadfence();
+      for (int i = 0; i < kMaxSlots; ++i) P.cnt[i] = 0u;
+      for (int i = 0; i < kMaxSlots * kMaxT; ++i) P.amax[i] = 0u;
+      hdr->bar_count = 0;
+      hdr->abort = 0;
+      hdr->exit_count = 0;
+      __threadfence();
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+constexpr int kStaticSmem = 12 * 1024;  // bound on the kernel's static shared memory
+
+int grid_size() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+// Whether the shape runs as one fused launch on a grid of G CTAs.
+bool eligible_on(int T, int H, int I, int E, int k, int G) {
+  if (T < 1 || T > kMaxT || k < 1 || k > kMaxK || E < k || E > kMaxE) return false;
+  if (H < 256 || I < 256 || H > 2048 || I > 2048 || (H % 256) || (I % 256)) return false;
+  if ((H + G - 1) / G > 16) return false;             // output rows per CTA fit one 16-row tile
+  // job lists: phase A <= router rows x segments + 2 x shared tiles, phase
+  // B/C <= 2 x routed tiles + one down job per slot
+  const int U = T * k < E ? T * k : E;
+  if (router_rows(E, G) * (H / router_seg(H)) + 2 * shared_tiles(I, G, 0) > kMaxJobs) return false;
+  if (2 * ((U * (I / 8) + G - 1) / G) + U + 1 > kMaxJobs) return false;
+  return make_plan(T, H, I, E, k, G).total + kStaticSmem <= kSmemLimit;
+}
+
+}  // namespace dfx
+
+bool decode_fused_eligible(int T, int H, int I, int E, int k) {
+  return dfx::eligible_on(T, H, I, E, k, dfx::grid_size());
+}
+
+size_t decode_fused_ws_bytes(int T, int I) {
+  return size_t(dfx::kMaxSlots) * size_t(T) * size_t(I) * sizeof(float);
+}
+
+cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
+                                const float* bias, long long bstride, const moe_expert* experts,
+                                const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
+                                uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
+                                long long wait_cycles, cudaStream_t st) {
+  using namespace dfx;
+  const int grid = grid_size();
+  const size_t smem = size_t(make_plan(T, H, I, E, k, grid).total);
+  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  Params P{x,      T,       H,        I,      E,   k,        w_router,           bias,
+           bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
+           logits_ws, h_ws, counters, counters + kMaxSlots, wait_cycles};
+  void* args[] = {&P};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(decode_fused_kernel), dim3(grid), dim3(kThreads), args,
+                                  smem, st);
+  count_launches(1);
+  return e;
+}
+
+}  // namespace moe

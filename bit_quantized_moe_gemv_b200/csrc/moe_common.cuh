@@ -26,12 +26,20 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 
+// Counters of the fused decode launch (finished gate/up tiles and the
+// largest |h| per expert slot and token), right after the header. They must
+// be zero when a launch starts; the launch leaves them zero again, and
+// moe_reset_status clears them with the header.
+constexpr size_t kDecodeCounterBytes = 2048;
+constexpr size_t kWsResetBytes = 256 + kDecodeCounterBytes;
+
 // Offsets (bytes from the workspace base) of every workspace segment.
 struct WsLayout {
-  size_t counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, partial, h, shared_y, y_perm, gemm,
-      router;
+  size_t dcnt, counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, partial, h, dh, shared_y, y_perm,
+      gemm, router;
   size_t total;
 };
+size_t decode_fused_ws_bytes(int T, int I);
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -43,6 +51,7 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   size_t o = 256;
   auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
   const int64_t n = T * k;
+  L.dcnt = take(kDecodeCounterBytes);
   L.counts = take(4 * E);
   L.offsets = take(4 * (E + 1));
   L.perm = take(4 * n);
@@ -57,6 +66,7 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   // activations in fragment order: (T k + 1) buffers of I/16 k-steps x T x 32 B
   const int64_t h32 = 4 * (n + T) * I, hfrag = T <= 4 ? (n + 1) * (I / 16) * T * 32 : 0;
   L.h = take(size_t(h32 > hfrag ? h32 : hfrag));
+  L.dh = take(T >= 1 && T <= 4 ? decode_fused_ws_bytes(int(T), int(I)) : 0);  // fused decode: h per expert slot
   L.shared_y = take(4 * T * H);
   L.y_perm = take(4 * n * H);  // fp32 routed rows inside moe_layer
   L.gemm = take(grouped_ws_bytes(T, int(H), int(I), int(k), int(E), true));  // tcgen05 prefill scratch

@@ -48,6 +48,18 @@ cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, 
                                  const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                  uint16_t* out, float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st);
 
+// Decode step (T <= 4) as one cooperative launch whose warps stream weights
+// into registers; see decode_fused.cu. logits_ws: fp32 [T][E]; h_ws:
+// decode_fused_ws_bytes; counters: kDecodeCounterBytes, zero at launch.
+// wait_cycles bounds every wait of the launch.
+bool decode_fused_eligible(int T, int H, int I, int E, int k);
+cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
+                                const float* bias, long long bstride, const moe_expert* experts,
+                                const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
+                                uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
+                                long long wait_cycles, cudaStream_t st);
+constexpr long long kDefaultWaitCycles = 2000000000LL;  // about 1 s at the B200's clock
+
 // Prefill experts on tcgen05 (expert_gemm_sm100.cu): plan, gather, gate/up
 // GEMM with SwiGLU epilogue, down GEMM. Routed rows go to y_f32 or y_bf16
 // (dispatched order), the shared expert's rows (if any) to ys_f32 [T][H].

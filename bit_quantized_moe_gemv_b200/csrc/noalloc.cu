@@ -23,9 +23,10 @@
 
 namespace {
 
-// Header (256 B) + router partials (4 T E floats) + the intermediate
-// activations ((T k + 1) buffers of 2 T I bytes) at the limits T <= 4,
-// E <= 1024, k <= 16, I <= 2048.
+// Header (256 B) + the launch's counters (2 KiB) + logits (4 T E bytes) + the
+// intermediate activations (65 expert slots x T x I floats) for every shape
+// the fused decode kernel runs with T <= 4, E <= 1024, k <= 16, I <= 2048
+// (its shared-memory plan keeps T x I <= 3072).
 constexpr size_t kNoAllocBytes = 1280u * 1024u;
 constexpr int kNoAllocMaxT = 4, kNoAllocMaxE = 1024, kNoAllocMaxK = 16, kNoAllocMaxHI = 2048;
 
@@ -104,25 +105,27 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
   if (T < 1 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (T > kNoAllocMaxT || E > kNoAllocMaxE || k > kNoAllocMaxK || H > kNoAllocMaxHI || I > kNoAllocMaxHI)
     return MOE_ERR_UNSUPPORTED;
-  if (!moe::decode_stream_eligible(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (!moe::decode_fused_eligible(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
   if (!x || !w_router || !experts_dev || !topk_idx || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   const uintptr_t misalign = (reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router) |
                               reinterpret_cast<uintptr_t>(out)) & 15u;
   if (misalign || (reinterpret_cast<uintptr_t>(experts_dev) & 7u)) return MOE_ERR_INVALID_ARG;
 
-  const size_t off_partial = 256;
-  const size_t off_h = moe::align256(off_partial + 16u * size_t(T) * E);
-  const size_t total = off_h + moe::decode_stream_hfrag_bytes(T, I, k);
+  const size_t off_counters = 256;
+  const size_t off_logits = moe::align256(off_counters + moe::kDecodeCounterBytes);
+  const size_t off_h = moe::align256(off_logits + 4u * size_t(T) * E);
+  const size_t total = off_h + moe::decode_fused_ws_bytes(T, I);
   if (total > kNoAllocBytes) return MOE_ERR_UNSUPPORTED;
 
   void* base = nullptr;
   if (scratch_for_current_device(&base) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The previous call's status and barrier words stay in the array: clear them.
-  if (cudaMemsetAsync(base, 0, sizeof(moe::WsHeader), st) != cudaSuccess) return MOE_ERR_CUDA;
-  cudaError_t e = moe::launch_decode_stream(
+  // The previous call's status word and counters stay in the array: clear them.
+  if (cudaMemsetAsync(base, 0, moe::kWsResetBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = moe::launch_decode_fused(
       x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, logits_out, out,
-      moe::ws_at<float>(base, off_partial), moe::ws_at<void>(base, off_h), moe::ws_at<moe::WsHeader>(base, 0), st);
+      moe::ws_at<float>(base, off_logits), moe::ws_at<float>(base, off_h), moe::ws_at<uint32_t>(base, off_counters),
+      moe::ws_at<moe::WsHeader>(base, 0), moe::kDefaultWaitCycles, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -1,14 +1,16 @@
 """Host-side planning of the fused decode kernel, checked on the CPU.
 
-The decode kernel's shared-memory layout, slot geometry, K-piece split and
-fragment order are computed by host/device functions in decode_stream.cu.
+The fused decode kernel (decode_fused.cu) computes its shared-memory plan,
+activation fragment order and per-CTA job lists with host/device functions.
 A small host program (compiled with nvcc, run without a GPU) evaluates them
 over every shape the kernel accepts and checks the invariants the kernel
 relies on: every fp16 activation has exactly one place in the fragment
-order, tile pieces fit a slot, slot offsets are 16-byte aligned, the ring
-has an even number of slots (one producer warp per slot), the whole plan
-fits the per-CTA shared-memory limit, and the workspace regions it writes
-(router partials, the activations of the picked experts) are large enough.
+order; the plan fits the per-CTA shared-memory limit with 16-byte aligned
+regions; over all CTAs of the grid every router row, every gate/up tile
+(both K parts) and every output row of every expert is covered exactly once;
+job fields fit their widths; local tile indices stay inside the reduction
+slots; and the workspace holds the counters, logits and intermediate
+activations the kernel writes.
 """
 import json
 import os
@@ -21,7 +23,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CSRC = os.path.join(ROOT, "bit_quantized_moe_gemv_b200", "csrc")
 
 PROGRAM = r"""
-#include "decode_stream.cu"
+#include "decode_fused.cu"
 #include <cstdio>
 #include <vector>
 void moe::count_launches(int) {}
@@ -29,60 +31,99 @@ void moe::count_launches(int) {}
 size_t moe::grouped_ws_bytes(long long, int, int, int, int, bool) { return 0; }
 size_t moe::router_tc_ws_bytes(long long, int, int) { return 0; }
 using namespace moe;
-using namespace moe::dks;
+using namespace moe::dfx;
 int main() {
-  int bad_frag = 0, bad_geo = 0, bad_plan = 0, bad_ws = 0, eligible = 0, checked = 0;
-  // fragment order: a bijection of (k, t) onto the fp16 slots of the buffer
-  for (int fmt = 1; fmt <= 3; ++fmt)
+  int bad_frag = 0, bad_plan = 0, bad_cover = 0, bad_fields = 0, bad_ws = 0, eligible = 0, checked = 0;
+  // fragment order: a bijection of (k, t) onto the fp16 places of the buffer
+  for (int f = 1; f <= 3; ++f)
     for (int T = 1; T <= 4; ++T)
       for (int K = 256; K <= 2048; K += 256) {
-        std::vector<int> seen(frag_bytes(K, T) / 2, 0);
+        std::vector<int> seen(K * T, 0);
         for (int t = 0; t < T; ++t)
           for (int k = 0; k < K; ++k) {
-            const int o = frag_off(fmt, k, t, T);
-            if (o < 0 || o % 2 || o / 2 >= int(seen.size()) || seen[o / 2]++) ++bad_frag;
+            const int o = frag_pos(f, k, t, T);
+            if (o < 0 || o % 2 || o / 2 >= K * T || seen[o / 2]++) ++bad_frag;
           }
       }
-  // tile pieces: fit a slot, 16-byte aligned parts, odd 16-byte row strides
-  for (int fmt = 1; fmt <= 3; ++fmt)
-    for (int T = 1; T <= 4; ++T)
-      for (int K = 256; K <= 2048; K += 256)
-        for (int wb = 0; wb < 2; ++wb) {
-          const int np = npieces(fmt, K, T, wb != 0);
-          if (np == 0) { ++bad_geo; continue; }
-          const Geo g = geo(fmt, K / np, T, wb != 0);
-          if (g.bytes > kSlotBytes || g.cs % 16 || ((g.cs / 16) & 1) == 0 || g.aux0 % 16 || g.aux1 % 16 ||
-              g.bofs % 16 || (g.as && (g.as % 16 || ((g.as / 16) & 1) == 0)))
-            ++bad_geo;
-        }
-  // plans of every accepted shape
+  const int Gs[] = {148, 132};
   const int Es[] = {16, 24, 32, 64, 128, 256, 384, 512, 1024};
   const int Ks[] = {1, 2, 4, 6, 8, 10, 16};
-  for (int T = 1; T <= 4; ++T)
-    for (int H = 256; H <= 2048; H += 256)
-      for (int I = 256; I <= 2048; I += 256)
-        for (int E : Es)
-          for (int k : Ks) {
-            if (k > E) continue;
-            ++checked;
-            if (!decode_stream_eligible(T, H, I, E, k)) continue;
-            ++eligible;
-            const int S = pick_slots(T, H, E, k);
-            const Plan p = make_plan(T, H, E, k, S);
-            if (S < 4 || S > kMaxSlots || S % kProducers || p.total + kStaticSmem > kSmemLimit ||
-                p.o_slots % 1024 || kSlotBytes % 1024)
-              ++bad_plan;
-            // workspace regions the kernel writes: router partials [T, E, RQ] fp32 and the
-            // fp16 activations of every picked expert plus the shared one
-            const WsLayout L = ws_layout(T, H, I, E, k);
-            if (L.h - L.partial < size_t(4) * T * E * router_rq(H) ||
-                L.shared_y - L.h < decode_stream_hfrag_bytes(T, I, k) || L.partial % 256 || L.h % 256)
-              ++bad_ws;
-          }
-  printf("{\"bad_frag\": %d, \"bad_geo\": %d, \"bad_plan\": %d, \"bad_ws\": %d, \"eligible\": %d, \"checked\": %d, "
-         "\"slots_decode1\": %d, \"slots_decode48\": %d, \"decode1\": %d, \"decode48\": %d}\n",
-         bad_frag, bad_geo, bad_plan, bad_ws, eligible, checked, pick_slots(1, 2048, 512, 10), pick_slots(4, 2048, 512, 10),
-         int(decode_stream_eligible(1, 2048, 768, 512, 10)), int(decode_stream_eligible(4, 2048, 768, 512, 10)));
+  std::vector<Job> jobs(kMaxJobs + 64);
+  for (int G : Gs)
+    for (int T = 1; T <= 4; ++T)
+      for (int H = 256; H <= 2048; H += 256)
+        for (int I = 256; I <= 2048; I += 256)
+          for (int E : Es)
+            for (int k : Ks) {
+              if (k > E) continue;
+              ++checked;
+              if (!eligible_on(T, H, I, E, k, G)) continue;
+              ++eligible;
+              const Plan p = make_plan(T, H, I, E, k, G);
+              const int offs[] = {p.o_x32, p.o_hf, p.o_xf, p.o_lg, p.o_rp, p.o_red, p.o_td, p.o_y, p.o_jobs, p.o_desc};
+              for (int o : offs)
+                if (o % 16) ++bad_plan;
+              if (p.total + kStaticSmem > kSmemLimit) ++bad_plan;
+              // every format mix of the routed experts gives the same job counts
+              // up to the K split; use the one with the most jobs (int4 splits
+              // when int2 may not)
+              const int U = T * k < E ? T * k : E;
+              for (int fm = 1; fm <= 3; ++fm) {
+                std::vector<int> fmt(U, fm);
+                std::vector<int> rows(E, 0), tparts(size_t(U + 1) * (I / 8), 0), outc(size_t(U + 1) * H, 0);
+                for (int b = 0; b < G; ++b) {
+                  int e0, nrr;
+                  router_range(E, G, b, e0, nrr);
+                  const int na = phase_a_jobs(H, I, E, G, b, fm, jobs.data());
+                  if (na > kMaxJobs) { ++bad_fields; continue; }
+                  for (int j = 0; j < na; ++j) {
+                    const Job& jb = jobs[j];
+                    if (jb.kind == kRouter) {
+                      if (jb.part == 0) rows[e0 + jb.slot]++;
+                    } else {
+                      tparts[size_t(U) * (I / 8) + jb.row0 / 8]++;
+                      if (jb.tile >= max_tiles(T, I, E, k, G)) ++bad_fields;
+                    }
+                  }
+                  const int nb = phase_bc_jobs(H, I, G, b, U, fmt.data(), true, jobs.data());
+                  if (nb > kMaxJobs) { ++bad_fields; continue; }
+                  int n0, nr;
+                  out_rows(H, G, b, n0, nr);
+                  if (nr > 16) ++bad_fields;
+                  for (int j = 0; j < nb; ++j) {
+                    const Job& jb = jobs[j];
+                    if (jb.kind == kGateUp) {
+                      tparts[size_t(jb.slot) * (I / 8) + jb.row0 / 8]++;
+                      if (jb.tile >= max_tiles(T, I, E, k, G) || jb.row0 % 8) ++bad_fields;
+                    } else {
+                      const int u = jb.slot == kSharedSlot ? U : jb.slot;
+                      if (jb.nrows != nr || jb.row0 != n0) ++bad_fields;
+                      for (int r = 0; r < jb.nrows; ++r) outc[size_t(u) * H + jb.row0 + r]++;
+                    }
+                  }
+                }
+                for (int e = 0; e < E; ++e)
+                  if (rows[e] != 1) ++bad_cover;
+                const int ns = gu_split(fm, H);
+                for (size_t i = 0; i < tparts.size(); ++i)
+                  if (tparts[i] != ns) ++bad_cover;
+                for (size_t i = 0; i < outc.size(); ++i)
+                  if (outc[i] != 1) ++bad_cover;
+              }
+              // the workspace the kernel writes: counters after the header,
+              // logits [T, E] and h of every slot
+              const WsLayout L = ws_layout(T, H, I, E, k);
+              if (L.dcnt != 256 || size_t(kMaxSlots) * (1 + kMaxT) * 4 > kDecodeCounterBytes ||
+                  L.counts < L.dcnt + kDecodeCounterBytes || L.partial - L.logits < size_t(4) * T * E ||
+                  L.shared_y - L.dh < decode_fused_ws_bytes(T, I) || L.dh % 256 || L.logits % 256)
+                ++bad_ws;
+            }
+  printf("{\"bad_frag\": %d, \"bad_plan\": %d, \"bad_cover\": %d, \"bad_fields\": %d, \"bad_ws\": %d, "
+         "\"eligible\": %d, \"checked\": %d, \"decode1\": %d, \"decode48\": %d, \"smem_decode1\": %d, "
+         "\"smem_decode48\": %d}\n",
+         bad_frag, bad_plan, bad_cover, bad_fields, bad_ws, eligible, checked,
+         int(eligible_on(1, 2048, 768, 512, 10, 148)), int(eligible_on(4, 2048, 768, 512, 10, 148)),
+         make_plan(1, 2048, 768, 512, 10, 148).total, make_plan(4, 2048, 768, 512, 10, 148).total);
   return 0;
 }
 """
@@ -96,10 +137,11 @@ def plan_report(tmp_path_factory):
     src = d / "plan.cu"
     src.write_text(PROGRAM)
     exe = d / "plan"
-    subprocess.run(["nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I", CSRC, "-I",
-                    os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True, capture_output=True,
-                   timeout=600)
-    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    r = subprocess.run(["nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I", CSRC, "-I",
+                        os.path.join(ROOT, "include"), str(src), "-o", str(exe)], capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr
     return json.loads(out.stdout.strip().splitlines()[-1])
 
@@ -108,13 +150,17 @@ def test_fragment_order_is_a_bijection(plan_report):
     assert plan_report["bad_frag"] == 0
 
 
-def test_tile_pieces_fit_and_are_aligned(plan_report):
-    assert plan_report["bad_geo"] == 0
-
-
-def test_plans_fit_shared_memory_with_an_even_ring(plan_report):
+def test_plans_fit_shared_memory_aligned(plan_report):
     assert plan_report["bad_plan"] == 0
     assert plan_report["eligible"] > 0
+
+
+def test_jobs_cover_every_row_tile_and_output_once(plan_report):
+    assert plan_report["bad_cover"] == 0
+
+
+def test_job_fields_and_tile_slots_in_range(plan_report):
+    assert plan_report["bad_fields"] == 0
 
 
 def test_workspace_holds_what_the_kernel_writes(plan_report):
@@ -123,5 +169,3 @@ def test_workspace_holds_what_the_kernel_writes(plan_report):
 
 def test_the_bench_decode_shapes_take_the_fused_kernel(plan_report):
     assert plan_report["decode1"] == 1 and plan_report["decode48"] == 1
-    assert plan_report["slots_decode1"] >= 4 and plan_report["slots_decode1"] % 2 == 0
-    assert plan_report["slots_decode48"] >= 4 and plan_report["slots_decode48"] % 2 == 0
