@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 # Every symbol include/moe.h declares (checked by the CPU test suite).
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer",
            "moe_layer_decode_noalloc", "moe_reset_status", "moe_get_status", "moe_launch_count",
-           "moe_status_string")
+           "moe_set_wait_cycles", "moe_status_string")
 
 
 class QMatrixC(ctypes.Structure):
@@ -62,6 +62,7 @@ def _load():
         "moe_reset_status": (c_i32, [c_vp, c_vp]),
         "moe_get_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32)]),
         "moe_launch_count": (ctypes.c_uint64, []),
+        "moe_set_wait_cycles": (c_i64, [c_i64]),
         "moe_status_string": (ctypes.c_char_p, [c_i32]),
     }
     for name, (res, args) in sig.items():
@@ -76,6 +77,12 @@ LIB = _load()
 def launch_count() -> int:
     """Kernels this library has launched in this process (host-side count)."""
     return int(LIB.moe_launch_count())
+
+
+def set_wait_cycles(cycles: int) -> int:
+    """Budget of every bounded wait of later fused decode launches (testing
+    the failure path); negative restores the default. Returns the previous."""
+    return int(LIB.moe_set_wait_cycles(int(cycles)))
 
 
 def status_string(st: int) -> str:

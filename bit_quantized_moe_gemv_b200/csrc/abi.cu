@@ -13,7 +13,9 @@ using namespace moe;
 
 namespace moe {
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
 void count_launches(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+long long wait_cycles() { return g_wait_cycles.load(std::memory_order_relaxed); }
 }  // namespace moe
 
 namespace {
@@ -144,7 +146,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
     return cuda_status(launch_decode_fused(x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev,
                                            topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.logits),
                                            ws_at<float>(ws, L.dh), ws_at<uint32_t>(ws, L.dcnt), hdr,
-                                           kDefaultWaitCycles, st));
+                                           wait_cycles(), st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
   int* perm = ws_at<int>(ws, L.perm);
@@ -192,6 +194,11 @@ moe_status moe_get_status(void* ws, void* stream, int32_t* device_status) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int64_t moe_set_wait_cycles(int64_t cycles) {
+  const long long v = cycles < 0 ? kDefaultWaitCycles : cycles;
+  return g_wait_cycles.exchange(v, std::memory_order_relaxed);
+}
 
 const char* moe_status_string(moe_status st) {
   switch (st) {

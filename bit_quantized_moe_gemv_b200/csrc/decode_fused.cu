@@ -491,20 +491,22 @@ __device__ __forceinline__ void warp_topk(uint64_t (&c)[4], int k, uint32_t* oke
 
 // ---------------------------------------------------------------- bounded waits
 // Spin (one thread) until *p >= target, the abort flag is raised or the
-// cycle budget runs out. Returns true when the target was reached.
+// cycle budget runs out (checked before every new poll: with a budget of 0 a
+// wait not met at its first poll gives up). Returns true when the target
+// was reached; an expired budget leaves MOE_ERR_TIMEOUT with `detail` in the
+// status word and raises the abort flag, which ends every other wait of the
+// launch.
 __device__ bool wait_counter(const uint32_t* p, uint32_t target, WsHeader* hdr, long long budget, int detail) {
   if (ld_acquire(p) >= target) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (ld_acquire(p) >= target) return true;
-    if ((it & 15) == 0) {
-      if (*reinterpret_cast<volatile int*>(&hdr->abort)) return false;
-      if (clock64() - t0 > budget) {
-        flag_error(hdr, MOE_ERR_TIMEOUT, detail);
-        atomicExch(&hdr->abort, 1);
-        return false;
-      }
+    if (clock64() - t0 >= budget) {
+      flag_error(hdr, MOE_ERR_TIMEOUT, detail);
+      atomicExch(&hdr->abort, 1);
+      return false;
     }
+    if (ld_acquire(p) >= target) return true;
+    if ((it & 15) == 0 && *reinterpret_cast<volatile int*>(&hdr->abort)) return false;
     __nanosleep(32);
   }
 }
@@ -1044,8 +1046,18 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
   using namespace dfx;
   const int grid = grid_size();
   const size_t smem = size_t(make_plan(T, H, I, E, k, grid).total);
-  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  // the kernel's dynamic shared-memory cap: raised once per device to the
+  // most any plan may take
+  static int s_cap_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !s_cap_set[dev]) {
+    e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemLimit - kStaticSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) s_cap_set[dev] = 1;
+  }
   Params P{x,      T,       H,        I,      E,   k,        w_router,           bias,
            bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
            logits_ws, h_ws, counters, counters + kMaxSlots, wait_cycles};

@@ -59,6 +59,9 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
                                 long long wait_cycles, cudaStream_t st);
 constexpr long long kDefaultWaitCycles = 2000000000LL;  // about 1 s at the B200's clock
+// The budget (SM clock cycles) every bounded wait of the fused decode launch
+// gets: kDefaultWaitCycles unless moe_set_wait_cycles changed it.
+long long wait_cycles();
 
 // Prefill experts on tcgen05 (expert_gemm_sm100.cu): plan, gather, gate/up
 // GEMM with SwiGLU epilogue, down GEMM. Routed rows go to y_f32 or y_bf16

@@ -126,6 +126,6 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
   cudaError_t e = moe::launch_decode_fused(
       x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, logits_out, out,
       moe::ws_at<float>(base, off_logits), moe::ws_at<float>(base, off_h), moe::ws_at<uint32_t>(base, off_counters),
-      moe::ws_at<moe::WsHeader>(base, 0), moe::kDefaultWaitCycles, st);
+      moe::ws_at<moe::WsHeader>(base, 0), moe::wait_cycles(), st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -229,6 +229,17 @@ moe_status moe_get_status(void* ws, void* stream, int32_t* device_status);
  * (host-side count of launch calls; thread-safe). */
 uint64_t moe_launch_count(void);
 
+/* Diagnostic for testing the failure path: the budget, in SM clock cycles,
+ * of every bounded device-side wait (grid counter, expert readiness) of the
+ * fused decode launches made after this call (moe_layer with T <= 4 and
+ * moe_layer_decode_noalloc). A wait that is not met when its budget runs out
+ * gives up: the launch ends early, its outputs are undefined and the status
+ * word reads MOE_ERR_TIMEOUT (reset the workspace before reusing it). With
+ * 0, a wait not met at its first check gives up at once. A negative value
+ * restores the default (2e9 cycles, about one second). Process-wide and
+ * thread-safe; returns the previous budget. Not meant for production use. */
+int64_t moe_set_wait_cycles(int64_t cycles);
+
 /* Static, NUL-terminated description of a status code. */
 const char* moe_status_string(moe_status st);
 

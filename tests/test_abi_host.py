@@ -84,3 +84,10 @@ def test_host_argument_checks_without_gpu(lib):
     # T = 0 is a no-op that succeeds without touching the device.
     assert L.moe_route(None, 0, 256, None, 16, None, 0, 2, None, None, None, None, 0, None) == 0
     assert L.moe_layer(None, 0, 256, 128, 16, 2, None, None, 0, None, None, None, None, None, None, None, 0, None) == 0
+
+
+def test_wait_budget_setter_round_trip(lib):
+    default = lib.set_wait_cycles(12345)
+    assert default == 2000000000
+    assert lib.set_wait_cycles(-1) == 12345
+    assert lib.set_wait_cycles(-1) == default
