@@ -36,6 +36,13 @@ class ExpertC(ctypes.Structure):
     _fields_ = [("gate", QMatrixC), ("up", QMatrixC), ("down", QMatrixC)]
 
 
+class OptionsC(ctypes.Structure):
+    _fields_ = [("flags", ctypes.c_uint32), ("shared_gate", c_vp)]
+
+
+MOE_BIAS_SELECTION_ONLY = 1
+
+
 class MoeError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
@@ -50,15 +57,17 @@ def _load():
     lib = ctypes.CDLL(path)
     sig = {
         "moe_workspace_size": (c_sz, [c_i32] * 5),
-        "moe_route": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_i32, c_vp, c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+        "moe_route": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_i32, c_vp, c_i64, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz,
+                              c_vp]),
         "moe_dispatch": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
         "moe_expert_ffn": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz,
                                    c_vp]),
-        "moe_combine": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+        "moe_combine": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz,
+                                c_vp]),
         "moe_layer": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp,
-                              c_vp, c_vp, c_vp, c_sz, c_vp]),
+                              c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
         "moe_layer_decode_noalloc": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp,
-                                             c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+                                             c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
         "moe_reset_status": (c_i32, [c_vp, c_vp]),
         "moe_get_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32)]),
         "moe_launch_count": (ctypes.c_uint64, []),
@@ -147,6 +156,15 @@ def _shape2(t, name, cols=None):
     return t.shape
 
 
+def _opts(H, bias_selection_only=False, shared_gate=None):
+    """The moe_options of a call (None = the defaults: NULL). shared_gate is a
+    device fp32 [H] tensor; the struct is read on the host during the call."""
+    if not bias_selection_only and shared_gate is None:
+        return None
+    g = _dev(shared_gate, "shared_gate", "f32", H, optional=True)
+    return ctypes.byref(OptionsC(MOE_BIAS_SELECTION_ONLY if bias_selection_only else 0, g))
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -171,14 +189,15 @@ def new_workspace(T, H, I, E, k, device="cuda"):
     return ws
 
 
-def route(x, w_router, bias, bias_row_stride, k, topk_idx, topk_w, ws, logits=None, stream=None):
+def route(x, w_router, bias, bias_row_stride, k, topk_idx, topk_w, ws, logits=None, stream=None,
+          bias_selection_only=False):
     T, H = _shape2(x, "x")
     E = _shape2(w_router, "w_router", H)[0]
     _check("moe_route", LIB.moe_route(_dev(x, "x", "bf16"), T, H, _dev(w_router, "w_router", "f32"), E,
                                       _bias(bias, T, E, bias_row_stride), bias_row_stride, k,
                                       _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
-                                      _dev(logits, "logits", "f32", T * E, optional=True), _ws(ws), ws.numel(),
-                                      _stream(stream)))
+                                      _dev(logits, "logits", "f32", T * E, optional=True),
+                                      _opts(H, bias_selection_only), _ws(ws), ws.numel(), _stream(stream)))
 
 
 def dispatch(topk_idx, E, counts, offsets, perm_src, inv_perm, ws, stream=None):
@@ -200,18 +219,19 @@ def expert_ffn(x, I, k, E, perm_src, offsets, counts, experts_table, y_perm, ws,
                                                 _stream(stream)))
 
 
-def combine(y_perm, inv_perm, topk_w, I, x, shared_table, out, ws, stream=None):
+def combine(y_perm, inv_perm, topk_w, I, x, shared_table, out, ws, stream=None, shared_gate=None):
     T, k = _shape2(topk_w, "topk_w")
     H = _shape2(out, "out")[1]
     _check("moe_combine", LIB.moe_combine(_dev(y_perm, "y_perm", "bf16", T * k * H),
                                           _dev(inv_perm, "inv_perm", "i32", T * k), _dev(topk_w, "topk_w", "f32"),
                                           T, H, I, k, _dev(x, "x", "bf16", T * H, optional=shared_table is None),
                                           _table(shared_table, "shared_table", 1, optional=True),
-                                          _dev(out, "out", "bf16", T * H), _ws(ws), ws.numel(), _stream(stream)))
+                                          _dev(out, "out", "bf16", T * H), _opts(H, shared_gate=shared_gate), _ws(ws),
+                                          ws.numel(), _stream(stream)))
 
 
 def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx, topk_w, out, ws,
-          stream=None, logits=None):
+          stream=None, logits=None, bias_selection_only=False, shared_gate=None):
     T, H = _shape2(x, "x")
     _shape2(w_router, "w_router", H)
     _check("moe_layer", LIB.moe_layer(_dev(x, "x", "bf16"), T, H, I, E, k, _dev(w_router, "w_router", "f32", E * H),
@@ -220,11 +240,12 @@ def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_tab
                                       _table(shared_table, "shared_table", 1, optional=True),
                                       _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
                                       _dev(logits, "logits", "f32", T * E, optional=True),
-                                      _dev(out, "out", "bf16", T * H), _ws(ws), ws.numel(), _stream(stream)))
+                                      _dev(out, "out", "bf16", T * H), _opts(H, bias_selection_only, shared_gate),
+                                      _ws(ws), ws.numel(), _stream(stream)))
 
 
 def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx,
-                         topk_w, out, stream=None, logits=None):
+                         topk_w, out, stream=None, logits=None, bias_selection_only=False, shared_gate=None):
     """moe_layer_decode_noalloc: the fused decode step without a workspace."""
     T, H = _shape2(x, "x")
     _shape2(w_router, "w_router", H)
@@ -236,7 +257,8 @@ def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_ta
                                         _dev(topk_idx, "topk_idx", "i32", T * k),
                                         _dev(topk_w, "topk_w", "f32", T * k),
                                         _dev(logits, "logits", "f32", T * E, optional=True),
-                                        _dev(out, "out", "bf16", T * H), _stream(stream)))
+                                        _dev(out, "out", "bf16", T * H), _opts(H, bias_selection_only, shared_gate),
+                                        _stream(stream)))
 
 
 def reset_status(ws, stream=None):

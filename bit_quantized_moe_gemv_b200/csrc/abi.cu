@@ -39,6 +39,14 @@ moe_status ws_check(void* ws, size_t ws_bytes, int64_t T, int64_t H, int64_t I, 
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Router variants asked for by `opts` (NULL = none); unknown flags are refused.
+bool read_opts(const moe_options* opts, uint32_t* flags, const float** gate) {
+  *flags = opts ? opts->flags : 0u;
+  *gate = opts ? opts->shared_gate : nullptr;
+  if (*flags & ~uint32_t(MOE_BIAS_SELECTION_ONLY)) return false;
+  return *gate == nullptr || aligned(*gate, 16);
+}
+
 }  // namespace
 
 extern "C" {
@@ -49,9 +57,12 @@ size_t moe_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k)
 }
 
 moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_router, int32_t E, const float* bias,
-                     int64_t bias_row_stride, int32_t k, int32_t* topk_idx, float* topk_w, float* logits_out, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     int64_t bias_row_stride, int32_t k, int32_t* topk_idx, float* topk_w, float* logits_out,
+                     const moe_options* opts, void* ws, size_t ws_bytes, void* stream) {
   const CallRange range("moe_route");
+  uint32_t flags = 0;
+  const float* gate = nullptr;
+  if (!read_opts(opts, &flags, &gate)) return MOE_ERR_INVALID_ARG;
   if (!shape_ok(T, H, 64, E, k)) return MOE_ERR_INVALID_ARG;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
@@ -63,7 +74,7 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_rou
   float* logits = logits_out ? logits_out : ws_at<float>(ws, L.logits);
   return cuda_status(launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w, logits,
                                   ws_at<void>(ws, L.router), ws_at<WsHeader>(ws, 0),
-                                  static_cast<cudaStream_t>(stream)));
+                                  static_cast<cudaStream_t>(stream), (flags & MOE_BIAS_SELECTION_ONLY) != 0));
 }
 
 moe_status moe_dispatch(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E, int32_t* counts, int32_t* offsets,
@@ -100,9 +111,12 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, in
 }
 
 moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int32_t T, int32_t H,
-                       int32_t I, int32_t k, const uint16_t* x, const moe_expert* shared_dev, uint16_t* out, void* ws,
-                       size_t ws_bytes, void* stream) {
+                       int32_t I, int32_t k, const uint16_t* x, const moe_expert* shared_dev, uint16_t* out,
+                       const moe_options* opts, void* ws, size_t ws_bytes, void* stream) {
   const CallRange range("moe_combine");
+  uint32_t flags = 0;
+  const float* gate = nullptr;
+  if (!read_opts(opts, &flags, &gate)) return MOE_ERR_INVALID_ARG;
   if (!shape_ok(T, H, I, k, k)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!y_perm || !inv_perm || !topk_w || !out || (shared_dev && !x)) return MOE_ERR_INVALID_ARG;
@@ -112,9 +126,15 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
   const WsLayout L = ws_layout(T, H, I, k, k);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* shared_y = nullptr;
+  float* shared_scale = nullptr;
   if (shared_dev) {
     shared_y = ws_at<float>(ws, L.shared_y);
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
+    if (gate) {
+      shared_scale = ws_at<float>(ws, L.sgate);
+      e = launch_shared_gate(x, T, H, gate, shared_scale, st);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
     if (T > kDecodeMaxT && grouped_eligible(H, I, 0, true))
       e = launch_grouped_ffn(x, T, H, I, k, 0, nullptr, nullptr, nullptr, nullptr, shared_dev, nullptr, nullptr,
                              shared_y, ws_at<void>(ws, L.gemm), ws_at<WsHeader>(ws, 0), st);
@@ -123,14 +143,17 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
                             nullptr, nullptr, shared_y, ws_at<WsHeader>(ws, 0), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
-  return cuda_status(launch_combine(y_perm, nullptr, inv_perm, topk_w, T, H, k, shared_y, out, st));
+  return cuda_status(launch_combine(y_perm, nullptr, inv_perm, topk_w, T, H, k, shared_y, shared_scale, out, st));
 }
 
 moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k, const float* w_router,
                      const float* bias, int64_t bias_row_stride, const moe_expert* experts_dev,
                      const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w, float* logits_out,
-                     uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+                     uint16_t* out, const moe_options* opts, void* ws, size_t ws_bytes, void* stream) {
   const CallRange range("moe_layer");
+  uint32_t flags = 0;
+  const float* gate = nullptr;
+  if (!read_opts(opts, &flags, &gate)) return MOE_ERR_INVALID_ARG;
   if (!shape_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
   if (bias_row_stride < 0 || (bias_row_stride > 0 && bias_row_stride < E)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
@@ -146,7 +169,8 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
     return cuda_status(launch_decode_fused(x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev,
                                            topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.logits),
                                            ws_at<float>(ws, L.dh), ws_at<uint32_t>(ws, L.dcnt), hdr,
-                                           wait_cycles(), st));
+                                           wait_cycles(), flags, gate, ws_at<float>(ws, L.logits_u),
+                                           ws_at<float>(ws, L.sgate), st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
   int* perm = ws_at<int>(ws, L.perm);
@@ -154,7 +178,12 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   float* y_perm = ws_at<float>(ws, L.y_perm);  // fp32: out is rounded only once
   cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w,
                                logits_out ? logits_out : ws_at<float>(ws, L.logits), ws_at<void>(ws, L.router),
-                               hdr, st);
+                               hdr, st, (flags & MOE_BIAS_SELECTION_ONLY) != 0);
+  float* shared_scale = nullptr;
+  if (e == cudaSuccess && shared_dev && gate) {
+    shared_scale = ws_at<float>(ws, L.sgate);
+    e = launch_shared_gate(x, T, H, gate, shared_scale, st);
+  }
   if (e == cudaSuccess) e = launch_dispatch(topk_idx, T, k, E, counts, offsets, perm, inv, ws_at<int>(ws, L.hist), hdr, st);
   float* shared_y = nullptr;
   if (T > kDecodeMaxT && grouped_eligible(H, I, E, shared_dev != nullptr)) {
@@ -162,7 +191,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
     if (e == cudaSuccess)
       e = launch_grouped_ffn(x, T, H, I, k, E, perm, offsets, counts, experts_dev, shared_dev, y_perm, nullptr,
                              shared_y, ws_at<void>(ws, L.gemm), hdr, st);
-    if (e == cudaSuccess) e = launch_combine(nullptr, y_perm, inv, topk_w, T, H, k, shared_y, out, st);
+    if (e == cudaSuccess) e = launch_combine(nullptr, y_perm, inv, topk_w, T, H, k, shared_y, shared_scale, out, st);
     return cuda_status(e);
   }
   if (e == cudaSuccess)
@@ -173,7 +202,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
     e = launch_expert_ffn(x, T, H, I, k, 1, nullptr, nullptr, nullptr, shared_dev, true,
                           ws_at<float>(ws, L.h) + size_t(T) * k * I, nullptr, nullptr, shared_y, hdr, st);
   }
-  if (e == cudaSuccess) e = launch_combine(nullptr, y_perm, inv, topk_w, T, H, k, shared_y, out, st);
+  if (e == cudaSuccess) e = launch_combine(nullptr, y_perm, inv, topk_w, T, H, k, shared_y, shared_scale, out, st);
   return cuda_status(e);
 }
 

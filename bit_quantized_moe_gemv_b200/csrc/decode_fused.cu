@@ -143,7 +143,7 @@ __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int
   p.o_hf = p.o_x32;
   p.o_xf = take(3 * 2 * T * H, 16);
   p.o_lg = take(4 * T * E, 16);
-  p.o_rp = take(4 * router_rows(E, G) * (H / router_seg(H)) * T, 16);
+  p.o_rp = take(4 * (router_rows(E, G) + 1) * (H / router_seg(H)) * T, 16);
   p.o_red = take(4 * max_tiles(T, I, E, k, G) * 16 * T, 16);
   p.o_td = take(4 * max_tiles(T, I, E, k, G), 16);
   p.o_y = take(4 * kMaxSlots * 16 * T, 16);
@@ -168,11 +168,19 @@ __host__ __device__ inline void router_range(int E, int G, int b, int& e0, int& 
 // Local tiles of the shared expert on CTA b (tiles i = b, b + G, ... < I / 8).
 __host__ __device__ inline int shared_tiles(int I, int G, int b) { return I / 8 > b ? (I / 8 - 1 - b) / G + 1 : 0; }
 
+// Router rows of CTA b, plus one for the shared expert's gate vector on the
+// last CTA when the gated variant is on (its local row index is the last).
+__host__ __device__ inline int router_rows_of(int E, int G, int b, bool gate_row) {
+  int e0, n;
+  router_range(E, G, b, e0, n);
+  return n + (gate_row && b == G - 1 ? 1 : 0);
+}
+
 // Phase-A jobs of CTA b: router (row, segment), then the shared expert's
 // gate/up tiles in K parts (shared_fmt 0 = no shared expert). Returns the count.
-__host__ __device__ inline int phase_a_jobs(int H, int I, int E, int G, int b, int shared_fmt, Job* jobs) {
-  int e0, nrr;
-  router_range(E, G, b, e0, nrr);
+__host__ __device__ inline int phase_a_jobs(int H, int I, int E, int G, int b, int shared_fmt, bool gate_row,
+                                            Job* jobs) {
+  const int nrr = router_rows_of(E, G, b, gate_row);
   const int nseg = H / router_seg(H);
   int n = 0;
   for (int r = 0; r < nrr; ++r)
@@ -226,6 +234,10 @@ struct Params {
   uint32_t* cnt;   // [kMaxSlots] finished gate/up tiles per slot
   uint32_t* amax;  // [kMaxSlots][kMaxT] bits of max |h| per slot and token
   long long wait_cycles;
+  uint32_t flags;            // MOE_BIAS_SELECTION_ONLY
+  const float* shared_gate;  // fp32 [H] or null: sigmoid-gated shared expert
+  float* logits_u;           // [T][E] unbiased logits (selection-only bias)
+  float* sgate;              // [T] shared_gate . x
 };
 
 // ---------------------------------------------------------------- PTX bits
@@ -518,7 +530,8 @@ struct Ctx {
   uint8_t* smem;
   Plan L;
   int T, H, I, E, k, G, b;
-  int e0, nrr, seg, nseg;   // router rows [e0, e0 + nrr), segments per row
+  int e0, nrr, seg, nseg;   // router rows [e0, e0 + nrr) (+ the gate row last), segments per row
+  int nreal;                // rows of W_r among them
   int n0, nr;               // output rows of this CTA
   int fmap[4];              // weight format -> activation buffer (or -1)
   int xexp[kMaxT];          // power-of-two scaling of x per token
@@ -677,8 +690,9 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb) {
   const int lane = threadIdx.x & 31;
   const float* x32 = reinterpret_cast<const float*>(C.smem + C.L.o_x32);
   float* rp = reinterpret_cast<float*>(C.smem + C.L.o_rp);
+  const bool gate_row = jb.slot >= C.nreal;  // the shared expert's gate vector
   const int e = C.e0 + jb.slot;
-  const float* wr = P.w_router + size_t(e) * H + jb.part * seg;
+  const float* wr = (gate_row ? P.shared_gate : P.w_router + size_t(e) * H) + jb.part * seg;
   const int nv = seg / 128;  // 16-byte loads per lane (4 or 2)
   uint4 w[4];
 #pragma unroll
@@ -711,8 +725,13 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb) {
     const int r = i / T, t = i - r * T;
     float a = 0.f;
     for (int s = 0; s < nseg; ++s) a += *reinterpret_cast<volatile float*>(rp + (r * nseg + s) * T + t);
+    if (r >= C.nreal) {
+      __stcg(P.sgate + t, a);
+      continue;
+    }
     const float bv = P.bias ? P.bias[t * P.bstride + C.e0 + r] : 0.f;
     __stcg(P.logits + size_t(t) * E + C.e0 + r, a + bv);
+    if (P.flags & MOE_BIAS_SELECTION_ONLY) __stcg(P.logits_u + size_t(t) * E + C.e0 + r, a);
   }
   __threadfence();
   __syncwarp();
@@ -749,7 +768,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     C.smem = smem;
     C.L = make_plan(T, H, I, E, k, G);
     C.T = T, C.H = H, C.I = I, C.E = E, C.k = k, C.G = G, C.b = b;
-    router_range(E, G, b, C.e0, C.nrr);
+    router_range(E, G, b, C.e0, C.nreal);
+    C.nrr = router_rows_of(E, G, b, P.shared_gate != nullptr && has_shared);
     C.seg = router_seg(H);
     C.nseg = H / C.seg;
     out_rows(H, G, b, C.n0, C.nr);
@@ -804,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       }
     }
     s_nA = phase_a_jobs(H, I, E, G, b, has_shared && good ? desc[kSharedSlot].gate.qtype : 0,
-                        reinterpret_cast<Job*>(smem + C.L.o_jobs));
+                        P.shared_gate != nullptr && has_shared, reinterpret_cast<Job*>(smem + C.L.o_jobs));
   }
   __syncthreads();
   const int nA = s_nA;
@@ -871,13 +891,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   }
   // gates: the softmax over all logits restricted to the picks and
   // renormalised = a softmax over the picked logits
+  // (with the selection-only bias: of the unbiased logits of the picks)
   if (live && warp < T) {
     const int t = warp;
-    const float v0 = key2f(s_key[t * k]);
-    float part = 0.f;
-    for (int j = lane; j < k; j += 32) part += expf(key2f(s_key[t * k + j]) - v0);
-    const float den = warp_sum(part);
-    for (int j = lane; j < k; j += 32) s_w[t * k + j] = expf(key2f(s_key[t * k + j]) - v0) / den;
+    const bool sel_only = (P.flags & MOE_BIAS_SELECTION_ONLY) != 0;
+    float v = -CUDART_INF_F;
+    if (lane < k) v = sel_only ? __ldcg(P.logits_u + size_t(t) * E + s_idx[t * k + lane]) : key2f(s_key[t * k + lane]);
+    float v0 = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, o));
+    const float ev = lane < k ? expf(v - v0) : 0.f;
+    const float den = warp_sum(ev);
+    if (lane < k) s_w[t * k + lane] = ev / den;
   }
   // distinct picked experts in ascending id order through a bitmap: the
   // slot of an id is the number of set bits below it
@@ -982,7 +1007,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       const int t = i / nr, r = i - t * nr;
       float a = 0.f;
       for (int j = 0; j < k; ++j) a = fmaf(s_w[t * k + j], Y[(s_slot[t * k + j] * 16 + r) * T + t], a);
-      if (has_shared) a += Y[(kSharedSlot * 16 + r) * T + t];
+      if (has_shared) {
+        const float ys = Y[(kSharedSlot * 16 + r) * T + t];
+        a = P.shared_gate ? fmaf(1.f / (1.f + expf(-__ldcg(P.sgate + t))), ys, a) : a + ys;
+      }
       P.out[size_t(t) * H + n0 + r] = f32_to_bf16_rn(a);
     }
   }
@@ -1023,7 +1051,7 @@ bool eligible_on(int T, int H, int I, int E, int k, int G) {
   // job lists: phase A <= router rows x segments + 2 x shared tiles, phase
   // B/C <= 2 x routed tiles + one down job per slot
   const int U = T * k < E ? T * k : E;
-  if (router_rows(E, G) * (H / router_seg(H)) + 2 * shared_tiles(I, G, 0) > kMaxJobs) return false;
+  if ((router_rows(E, G) + 1) * (H / router_seg(H)) + 2 * shared_tiles(I, G, 0) > kMaxJobs) return false;
   if (2 * ((U * (I / 8) + G - 1) / G) + U + 1 > kMaxJobs) return false;
   return make_plan(T, H, I, E, k, G).total + kStaticSmem <= kSmemLimit;
 }
@@ -1042,7 +1070,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
                                 const float* bias, long long bstride, const moe_expert* experts,
                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
-                                long long wait_cycles, cudaStream_t st) {
+                                long long wait_cycles, uint32_t flags, const float* shared_gate, float* logits_u_ws,
+                                float* sgate_ws, cudaStream_t st) {
   using namespace dfx;
   const int grid = grid_size();
   const size_t smem = size_t(make_plan(T, H, I, E, k, grid).total);
@@ -1060,7 +1089,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
   }
   Params P{x,      T,       H,        I,      E,   k,        w_router,           bias,
            bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
-           logits_ws, h_ws, counters, counters + kMaxSlots, wait_cycles};
+           logits_ws, h_ws, counters, counters + kMaxSlots, wait_cycles, flags, shared_gate, logits_u_ws,
+           sgate_ws};
   void* args[] = {&P};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(decode_fused_kernel), dim3(grid), dim3(kThreads), args,
                                   smem, st);

@@ -35,8 +35,8 @@ constexpr size_t kWsResetBytes = 256 + kDecodeCounterBytes;
 
 // Offsets (bytes from the workspace base) of every workspace segment.
 struct WsLayout {
-  size_t dcnt, counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, partial, h, dh, shared_y, y_perm,
-      gemm, router;
+  size_t dcnt, counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, logits_u, sgate, partial, h, dh,
+      shared_y, y_perm, gemm, router;
   size_t total;
 };
 size_t decode_fused_ws_bytes(int T, int I);
@@ -61,6 +61,8 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   L.topk_idx = take(4 * n);
   L.topk_w = take(4 * n);
   L.logits = take(4 * T * E);
+  L.logits_u = take(4 * T * E);  // unbiased logits (bias used for the selection only)
+  L.sgate = take(4 * T);         // the shared expert's per-token sigmoid gate
   L.partial = take(16 * T * E);  // router partial sums of the fused decode path
   // fp32 intermediate rows of the multi-launch path, or the decode step's fp16
   // activations in fragment order: (T k + 1) buffers of I/16 k-steps x T x 32 B

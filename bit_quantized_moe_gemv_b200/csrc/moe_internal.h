@@ -15,9 +15,11 @@ enum TicketSlot { kTicketRoute = 0, kTicketDecodeRoute = 1, kTicketDecodeGateUp 
 
 // tc_scratch: workspace for the tensor-core router (router_tc_ws_bytes), used
 // for T > 4 when E is a multiple of 128.
+// bias_selection_only: the bias picks the experts, the gates come from the
+// unbiased logits.
 cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
                          long long bstride, int k, int* topk_idx, float* topk_w, float* logits, void* tc_scratch,
-                         WsHeader* hdr, cudaStream_t st);
+                         WsHeader* hdr, cudaStream_t st, bool bias_selection_only);
 
 bool router_tc_eligible(int T, int H, int E);
 size_t router_tc_ws_bytes(long long T, int H, int E);
@@ -53,11 +55,14 @@ cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, 
 // decode_fused_ws_bytes; counters: kDecodeCounterBytes, zero at launch.
 // wait_cycles bounds every wait of the launch.
 bool decode_fused_eligible(int T, int H, int I, int E, int k);
+// flags: MOE_BIAS_SELECTION_ONLY (then logits_u_ws [T][E] holds the unbiased
+// logits); shared_gate: fp32 [H] or NULL (then sgate_ws [T] holds g . x).
 cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
                                 const float* bias, long long bstride, const moe_expert* experts,
                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
-                                long long wait_cycles, cudaStream_t st);
+                                long long wait_cycles, uint32_t flags, const float* shared_gate, float* logits_u_ws,
+                                float* sgate_ws, cudaStream_t st);
 constexpr long long kDefaultWaitCycles = 2000000000LL;  // about 1 s at the B200's clock
 // The budget (SM clock cycles) every bounded wait of the fused decode launch
 // gets: kDefaultWaitCycles unless moe_set_wait_cycles changed it.
@@ -73,8 +78,13 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
                                const moe_expert* shared, float* y_f32, uint16_t* y_bf16, float* ys_f32,
                                void* scratch, WsHeader* hdr, cudaStream_t st);
 
-// Combine routed rows given as bf16 (y_bf16) or fp32 (y_f32; the other NULL).
+// Combine routed rows given as bf16 (y_bf16) or fp32 (y_f32; the other NULL);
+// shared_scale (nullable, [T]) weighs the shared expert's rows per token.
 cudaError_t launch_combine(const uint16_t* y_bf16, const float* y_f32, const int* inv_perm, const float* topk_w,
-                           int T, int H, int k, const float* shared_y, uint16_t* out, cudaStream_t st);
+                           int T, int H, int k, const float* shared_y, const float* shared_scale, uint16_t* out,
+                           cudaStream_t st);
+
+// scale[t] = sigmoid(gate_w . x_t): the sigmoid-gated shared expert's weight.
+cudaError_t launch_shared_gate(const uint16_t* x, int T, int H, const float* gate_w, float* scale, cudaStream_t st);
 
 }  // namespace moe

@@ -23,7 +23,8 @@
 
 namespace {
 
-// Header (256 B) + the launch's counters (2 KiB) + logits (4 T E bytes) + the
+// Header (256 B) + the launch's counters (2 KiB) + logits, biased and
+// unbiased (8 T E bytes) + the shared expert's gates (4 T bytes) + the
 // intermediate activations (65 expert slots x T x I floats) for every shape
 // the fused decode kernel runs with T <= 4, E <= 1024, k <= 16, I <= 2048
 // (its shared-memory plan keeps T x I <= 3072).
@@ -100,7 +101,8 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
                                                int32_t k, const float* w_router, const float* bias,
                                                int64_t bias_row_stride, const moe_expert* experts_dev,
                                                const moe_expert* shared_dev, int32_t* topk_idx, float* topk_w,
-                                               float* logits_out, uint16_t* out, void* stream) {
+                                               float* logits_out, uint16_t* out, const moe_options* opts,
+                                               void* stream) {
   const moe::CallRange range("moe_layer_decode_noalloc");
   if (T < 1 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (T > kNoAllocMaxT || E > kNoAllocMaxE || k > kNoAllocMaxK || H > kNoAllocMaxHI || I > kNoAllocMaxHI)
@@ -112,9 +114,15 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
                               reinterpret_cast<uintptr_t>(out)) & 15u;
   if (misalign || (reinterpret_cast<uintptr_t>(experts_dev) & 7u)) return MOE_ERR_INVALID_ARG;
 
+  const uint32_t flags = opts ? opts->flags : 0u;
+  const float* gate = opts ? opts->shared_gate : nullptr;
+  if ((flags & ~uint32_t(MOE_BIAS_SELECTION_ONLY)) || (reinterpret_cast<uintptr_t>(gate) & 15u))
+    return MOE_ERR_INVALID_ARG;
   const size_t off_counters = 256;
   const size_t off_logits = moe::align256(off_counters + moe::kDecodeCounterBytes);
-  const size_t off_h = moe::align256(off_logits + 4u * size_t(T) * E);
+  const size_t off_logits_u = moe::align256(off_logits + 4u * size_t(T) * E);
+  const size_t off_sgate = moe::align256(off_logits_u + 4u * size_t(T) * E);
+  const size_t off_h = moe::align256(off_sgate + 4u * size_t(T));
   const size_t total = off_h + moe::decode_fused_ws_bytes(T, I);
   if (total > kNoAllocBytes) return MOE_ERR_UNSUPPORTED;
 
@@ -126,6 +134,7 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
   cudaError_t e = moe::launch_decode_fused(
       x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, logits_out, out,
       moe::ws_at<float>(base, off_logits), moe::ws_at<float>(base, off_h), moe::ws_at<uint32_t>(base, off_counters),
-      moe::ws_at<moe::WsHeader>(base, 0), moe::wait_cycles(), st);
+      moe::ws_at<moe::WsHeader>(base, 0), moe::wait_cycles(), flags, gate, moe::ws_at<float>(base, off_logits_u),
+      moe::ws_at<float>(base, off_sgate), st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

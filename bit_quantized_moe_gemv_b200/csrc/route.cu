@@ -20,9 +20,12 @@ namespace moe {
 
 // ---------------------------------------------------------------- top-k
 // Warp-level top-k over one row of E <= 1024 logits. Lane l holds experts
-// l, l+32, ... in registers. NaN logits are treated as -inf.
+// l, l+32, ... in registers. NaN logits are treated as -inf. gbias, when not
+// NULL, is the bias row of this token and the gates are taken on the
+// unbiased logits (logit - bias) of the picks: the bias moves the selection
+// only.
 __device__ void warp_topk_row(const float* row, int E, int k, int* idx_out, float* w_out, float* s_val,
-                              int* s_idx) {
+                              int* s_idx, const float* gbias) {
   const int lane = threadIdx.x & 31;
   float v[32];
   const int nper = (E + 31) / 32;
@@ -74,7 +77,14 @@ __device__ void warp_topk_row(const float* row, int E, int k, int* idx_out, floa
   }
   __syncwarp();
   // Renormalised softmax over the picks: the full-softmax denominator cancels.
-  const float m = s_val[0];
+  if (gbias) {
+    for (int j = lane; j < k; j += 32) s_val[j] -= gbias[s_idx[j]];
+    __syncwarp();
+  }
+  float m = -CUDART_INF_F;
+  for (int j = lane; j < k; j += 32) m = fmaxf(m, s_val[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float part = 0.f;
   for (int j = lane; j < k; j += 32) part += expf(s_val[j] - m);
   const float denom = warp_sum(part);
@@ -94,7 +104,8 @@ constexpr int kGemvTmax = 8;
 __global__ void __launch_bounds__(kGemvWarps * 32)
 router_gemv_topk_kernel(const uint16_t* __restrict__ x, int T, int H, const float* __restrict__ W, int E,
                         const float* __restrict__ bias, long long bstride, int k, float* __restrict__ logits,
-                        int* __restrict__ topk_idx, float* __restrict__ topk_w, WsHeader* hdr, int ticket_slot) {
+                        int* __restrict__ topk_idx, float* __restrict__ topk_w, WsHeader* hdr, int ticket_slot,
+                        bool bias_selection_only) {
   extern __shared__ float smem[];
   float* xs = smem;  // [T][H]
   __shared__ float s_val[kGemvWarps][kMaxK];
@@ -141,7 +152,8 @@ router_gemv_topk_kernel(const uint16_t* __restrict__ x, int T, int H, const floa
   if (!s_last) return;
   __threadfence();
   for (int t = warp; t < T; t += kGemvWarps)
-    warp_topk_row(logits + size_t(t) * E, E, k, topk_idx + t * k, topk_w + t * k, s_val[warp], s_idx[warp]);
+    warp_topk_row(logits + size_t(t) * E, E, k, topk_idx + t * k, topk_w + t * k, s_val[warp], s_idx[warp],
+                  bias_selection_only && bias ? bias + t * bstride : nullptr);
   if (threadIdx.x == 0) hdr->tickets[ticket_slot] = 0;
 }
 
@@ -195,20 +207,20 @@ router_gemm_kernel(const uint16_t* __restrict__ x, int T, int H, const float* __
 
 __global__ void __launch_bounds__(256)
 topk_rows_kernel(const float* __restrict__ logits, int T, int E, int k, int* __restrict__ topk_idx,
-                 float* __restrict__ topk_w) {
+                 float* __restrict__ topk_w, const float* __restrict__ gbias, long long gstride) {
   __shared__ float s_val[8][kMaxK];
   __shared__ int s_idx[8][kMaxK];
   const int warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
   if (t >= T) return;
   warp_topk_row(logits + size_t(t) * E, E, k, topk_idx + size_t(t) * k, topk_w + size_t(t) * k, s_val[warp],
-                s_idx[warp]);
+                s_idx[warp], gbias ? gbias + t * gstride : nullptr);
 }
 
 // ---------------------------------------------------------------- launcher
 cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
                          long long bstride, int k, int* topk_idx, float* topk_w, float* logits, void* tc_scratch,
-                         WsHeader* hdr, cudaStream_t st) {
+                         WsHeader* hdr, cudaStream_t st, bool bias_selection_only) {
   if (T == 0) return cudaSuccess;
   if (T <= kGemvTmax) {
     const size_t smem = size_t(T) * H * sizeof(float);
@@ -219,7 +231,7 @@ cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E,
     }
     const int grid = (E + kGemvWarps - 1) / kGemvWarps;
     router_gemv_topk_kernel<<<grid, kGemvWarps * 32, smem, st>>>(x, T, H, W, E, bias, bstride, k, logits, topk_idx,
-                                                                 topk_w, hdr, kTicketRoute);
+                                                                 topk_w, hdr, kTicketRoute, bias_selection_only);
     count_launches(1);
     return cudaGetLastError();
   }
@@ -231,7 +243,8 @@ cudaError_t launch_route(const uint16_t* x, int T, int H, const float* W, int E,
     router_gemm_kernel<<<g, 256, 0, st>>>(x, T, H, W, E, bias, bstride, logits);
     count_launches(1);
   }
-  topk_rows_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
+  topk_rows_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w,
+                                                bias_selection_only ? bias : nullptr, bstride);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -91,6 +91,24 @@ typedef struct moe_expert {
   moe_qmatrix down;
 } moe_expert;
 
+/*
+ * Router variants, off by default (opts = NULL in every call that takes
+ * them). The pages name a router and a shared expert without their
+ * functions (telli.sh page, section "稀疏架构创造了机会"); these two common
+ * alternatives are readings of that gap:
+ *  MOE_BIAS_SELECTION_ONLY  the bias picks the experts but the gates are the
+ *                           softmax of the unbiased logits W_r x, renormalised
+ *                           over the picks (logits_out keeps the biased ones);
+ *  shared_gate              DEVICE fp32 [H] g, or NULL: the shared expert's
+ *                           output is scaled by sigmoid(g . x) per token.
+ * The struct itself is read on the host during the call.
+ */
+#define MOE_BIAS_SELECTION_ONLY 1u
+typedef struct moe_options {
+  uint32_t flags;
+  const float* shared_gate;
+} moe_options;
+
 /* Bytes of workspace the calls below need for a problem of this size (the
  * same value serves every call). Returns 0 for shapes outside the limits.
  * Call moe_reset_status once on a new workspace before its first use. */
@@ -110,12 +128,14 @@ size_t moe_workspace_size(int32_t T, int32_t H, int32_t I, int32_t E, int32_t k)
  *             to sum to 1
  *   logits_out fp32 [T, E] out, optional (NULL = not exported): the biased
  *             fp32 logits the selection was made on
+ *   opts      NULL or router variants (flags: MOE_BIAS_SELECTION_ONLY)
  * Logits are accumulated in fp32 (fp32-exact products on the tensor-core path
  * for large T); gates use expf.
  */
 moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_router, int32_t E,
                      const float* bias, int64_t bias_row_stride, int32_t k, int32_t* topk_idx,
-                     float* topk_w, float* logits_out, void* ws, size_t ws_bytes, void* stream);
+                     float* topk_w, float* logits_out, const moe_options* opts, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /*
  * moe_dispatch - per-expert histogram, prefix sum and stable permutation.
@@ -165,17 +185,20 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, in
  *   shared_dev  DEVICE pointer to one moe_expert, or NULL for no shared expert
  *   out         bf16 [T, H] out: sum over j = 0..k-1 in order, in fp32, plus
  *               the shared expert's fp32 output, rounded once (nearest-even)
+ *   opts        NULL or router variants (shared_gate: the shared expert's
+ *               output is scaled by sigmoid(shared_gate . x) per token)
  */
 moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int32_t T,
                        int32_t H, int32_t I, int32_t k, const uint16_t* x, const moe_expert* shared_dev,
-                       uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+                       uint16_t* out, const moe_options* opts, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_layer - the whole step (route, dispatch, experts, combine) in one call.
  * Same arguments and layouts as the four calls above; dispatch arrays and
  * intermediate rows live in the workspace and stay fp32, so `out` is rounded
  * once. `logits_out` (fp32 [T, E], NULL = not exported) receives the biased
- * fp32 logits the selection was made on, as in moe_route. Decode batches (1 <= T <= 4, H and I <= 2048) run as ONE cooperative
+ * fp32 logits the selection was made on, as in moe_route; `opts` selects the
+ * router variants (both fields used). Decode batches (1 <= T <= 4, H and I <= 2048) run as ONE cooperative
  * persistent kernel whose grid barriers are bounded: if one expires the call
  * leaves MOE_ERR_TIMEOUT in the status word, and the workspace must be reset
  * with moe_reset_status before it is used again.
@@ -183,7 +206,8 @@ moe_status moe_combine(const uint16_t* y_perm, const int32_t* inv_perm, const fl
 moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t E, int32_t k,
                      const float* w_router, const float* bias, int64_t bias_row_stride,
                      const moe_expert* experts_dev, const moe_expert* shared_dev, int32_t* topk_idx,
-                     float* topk_w, float* logits_out, uint16_t* out, void* ws, size_t ws_bytes, void* stream);
+                     float* topk_w, float* logits_out, uint16_t* out, const moe_options* opts, void* ws,
+                     size_t ws_bytes, void* stream);
 
 /*
  * moe_layer_decode_noalloc - moe_layer's fused decode step for callers that
@@ -214,7 +238,7 @@ moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int32_t H, int
                                     const float* w_router, const float* bias, int64_t bias_row_stride,
                                     const moe_expert* experts_dev, const moe_expert* shared_dev,
                                     int32_t* topk_idx, float* topk_w, float* logits_out, uint16_t* out,
-                                    void* stream);
+                                    const moe_options* opts, void* stream);
 
 /* Clear the device status word of a workspace (asynchronous on `stream`).
  * Call once on a fresh workspace before its first use. */

@@ -26,6 +26,13 @@ What it computes (one MoE block of a Qwen3.8-Flash-Next-style layer):
      silu(z) = z / (1 + exp(-z)), y = W_d h            (SwiGLU FFN)
   7. out[t]   = sum_j w[t,j] y_{S_j}(x_t) + shared(x_t) (shared expert ungated)
 
+Two router variants, both readings of what the pages leave open (they name a
+router and a shared expert but not their functions), off by default:
+  * bias for selection only: S_t is chosen on the biased logits (step 3) but
+    the gates of step 4 come from the softmax of the unbiased logits W_r x;
+  * sigmoid-gated shared expert: step 7 adds sigma(g . x_t) * shared(x_t)
+    for a gate vector g [H] instead of shared(x_t).
+
 Every quantity is float64 and nothing is rounded between steps.
 Quantised weight formats (codes row-major [N, K*bits/8], groups along K):
   int4_sym_g32:      element 2i in the low nibble of byte i, 2i+1 in the high
@@ -101,14 +108,26 @@ def topk_order(logits: np.ndarray, k: int) -> np.ndarray:
     return out
 
 
-def route(x_bits, w_router, bias, k):
-    """Steps 1-4. Returns (logits [T,E], idx int32 [T,k], w float64 [T,k])."""
+def route(x_bits, w_router, bias, k, bias_selection_only=False):
+    """Steps 1-4. Returns (logits [T,E], idx int32 [T,k], w float64 [T,k]).
+
+    logits are the biased logits the selection is made on. With
+    bias_selection_only the gates are the softmax of the unbiased logits,
+    renormalised over the same picks."""
     logits = router_logits(x_bits, w_router, bias)
-    p = softmax(logits)
     idx = topk_order(logits, k)
+    gate_logits = router_logits(x_bits, w_router, np.zeros(1)) if bias_selection_only else logits
+    p = softmax(gate_logits)
     sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
     w = sel / sel.sum(axis=1, keepdims=True)
     return logits, idx, w
+
+
+def shared_gate(x_bits, gate_w):
+    """Weight of the shared expert in the sigmoid-gated variant: sigma(g . x)
+    per token, sigma(z) = 1 / (1 + exp(-z))."""
+    z = bf16_bits_to_f64(x_bits) @ np.asarray(gate_w, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(-z))
 
 
 # ---------------------------------------------------------------- dispatch
@@ -210,31 +229,36 @@ def combine(y_perm, inv_perm, w, k, shared_y=None):
     return out
 
 
-def moe_layer(x_bits, w_router, bias, k, experts, shared=None, routing=None):
+def moe_layer(x_bits, w_router, bias, k, experts, shared=None, routing=None, bias_selection_only=False,
+              shared_gate_w=None):
     """Steps 1-7 for all tokens.
 
     routing, if given, is (idx, w) to use instead of the oracle's own routing
     (used where the fp32 router of the device legitimately resolves a near-tie
-    differently). Returns dict with logits, idx, w, counts, offsets, perm_src,
-    inv_perm, y_perm, out.
+    differently). bias_selection_only and shared_gate_w select the router
+    variants (module docstring). Returns dict with logits, idx, w, counts,
+    offsets, perm_src, inv_perm, y_perm, out.
     """
     E = len(experts)
-    logits, idx, w = route(x_bits, w_router, bias, k)
+    logits, idx, w = route(x_bits, w_router, bias, k, bias_selection_only)
     if routing is not None:
         idx, w = routing
     counts, offsets, perm_src, inv_perm = dispatch(idx, E)
     y_perm = expert_rows(x_bits, perm_src, offsets, k, experts)
     sy = shared_rows(x_bits, shared) if shared is not None else None
+    if sy is not None and shared_gate_w is not None:
+        sy = sy * shared_gate(x_bits, shared_gate_w)[:, None]
     out = combine(y_perm, inv_perm, w, k, sy)
     return dict(logits=logits, idx=idx, w=w, counts=counts, offsets=offsets, perm_src=perm_src,
                 inv_perm=inv_perm, y_perm=y_perm, out=out)
 
 
-def moe_token(x_bits_row, w_router, bias_row, k, cache, shared_deq=None, routing=None):
+def moe_token(x_bits_row, w_router, bias_row, k, cache, shared_deq=None, routing=None, bias_selection_only=False,
+              shared_gate_w=None):
     """Steps 1-7 for one token, computed directly (no dispatch): used to check
     sampled tokens of large workloads. Returns (idx, w, out[H])."""
     x_bits_row = np.asarray(x_bits_row).reshape(1, -1)
-    logits, idx, w = route(x_bits_row, w_router, np.asarray(bias_row).reshape(1, -1), k)
+    logits, idx, w = route(x_bits_row, w_router, np.asarray(bias_row).reshape(1, -1), k, bias_selection_only)
     if routing is not None:
         idx, w = routing
         idx = np.asarray(idx).reshape(1, -1)
@@ -245,5 +269,6 @@ def moe_token(x_bits_row, w_router, bias_row, k, cache, shared_deq=None, routing
         wg, wu, wd = cache.get(int(idx[0, j]))
         out += w[0, j] * expert_forward(wg, wu, wd, x)[1][0]
     if shared_deq is not None:
-        out += expert_forward(*shared_deq, x)[1][0]
+        g = shared_gate(x_bits_row, shared_gate_w)[0] if shared_gate_w is not None else 1.0
+        out += g * expert_forward(*shared_deq, x)[1][0]
     return idx[0], w[0], out

@@ -72,7 +72,7 @@ def oracle_gates_for(logits64, idx):
     return sel / sel.sum(axis=1, keepdims=True)
 
 
-def check_routing(gpu_idx, gpu_w, gpu_logits, x_bits, w_router, bias, k):
+def check_routing(gpu_idx, gpu_w, gpu_logits, x_bits, w_router, bias, k, bias_selection_only=False):
     """Routing parity.
 
     1. The selection logic, exactly: the oracle's top-k and gates evaluated on
@@ -88,7 +88,12 @@ def check_routing(gpu_idx, gpu_w, gpu_logits, x_bits, w_router, bias, k):
     gl = np.asarray(gpu_logits, dtype=np.float64)
     ref_idx_on_gpu_logits = oracle.topk_order(gl, k)
     np.testing.assert_array_equal(gpu_idx, ref_idx_on_gpu_logits)
-    np.testing.assert_allclose(gpu_w, oracle_gates_for(gl, gpu_idx), rtol=2e-6, atol=1e-7)
+    # gates: on the device's logits, less the bias when it only selects
+    # (fp32 logit - bias differs from the device's own unbiased fp32 logit by
+    # at most an ulp of the biased one, hence the looser bound there)
+    gate_logits = gl - np.asarray(bias, np.float64) if bias_selection_only else gl
+    np.testing.assert_allclose(gpu_w, oracle_gates_for(gate_logits, gpu_idx),
+                               rtol=2e-5 if bias_selection_only else 2e-6, atol=1e-7)
     logits64 = oracle.router_logits(x_bits, w_router, bias)
     ref_idx = oracle.topk_order(logits64, k)
     tau = near_tie_tau(x_bits, w_router, bias)

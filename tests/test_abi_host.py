@@ -68,22 +68,22 @@ def test_status_strings(lib):
 def test_host_argument_checks_without_gpu(lib):
     L = lib.LIB
     # Null activations with T > 0: rejected before any CUDA call.
-    assert L.moe_route(None, 4, 256, None, 16, None, 0, 2, None, None, None, None, 0, None) == 1
+    assert L.moe_route(None, 4, 256, None, 16, None, 0, 2, None, None, None, None, None, 0, None) == 1
     # k > E.
-    assert L.moe_route(None, 4, 256, None, 4, None, 0, 5, None, None, None, None, 0, None) == 1
+    assert L.moe_route(None, 4, 256, None, 4, None, 0, 5, None, None, None, None, None, 0, None) == 1
     # Bad bias stride (nonzero but < E).
-    assert L.moe_layer(None, 4, 256, 128, 16, 2, None, None, 3, None, None, None, None, None, None, None, 0, None) == 1
+    assert L.moe_layer(None, 4, 256, 128, 16, 2, None, None, 3, None, None, None, None, None, None, None, None, 0, None) == 1
     assert L.moe_dispatch(None, 4, 2, 0, None, None, None, None, None, 0, None) == 1
     assert L.moe_expert_ffn(None, 4, 256, 100, 2, 16, None, None, None, None, None, None, 0, None) == 1
-    assert L.moe_combine(None, None, None, 4, 256, 128, 2, None, None, None, None, 0, None) == 1
+    assert L.moe_combine(None, None, None, 4, 256, 128, 2, None, None, None, None, None, 0, None) == 1
     assert L.moe_reset_status(None, None) == 1
     v = ctypes.c_int32(7)
     assert L.moe_get_status(None, None, ctypes.byref(v)) == 1
     # Misaligned workspace pointer.
     assert L.moe_reset_status(ctypes.c_void_p(0x1001), None) == 1
     # T = 0 is a no-op that succeeds without touching the device.
-    assert L.moe_route(None, 0, 256, None, 16, None, 0, 2, None, None, None, None, 0, None) == 0
-    assert L.moe_layer(None, 0, 256, 128, 16, 2, None, None, 0, None, None, None, None, None, None, None, 0, None) == 0
+    assert L.moe_route(None, 0, 256, None, 16, None, 0, 2, None, None, None, None, None, 0, None) == 0
+    assert L.moe_layer(None, 0, 256, 128, 16, 2, None, None, 0, None, None, None, None, None, None, None, None, 0, None) == 0
 
 
 def test_wait_budget_setter_round_trip(lib):

@@ -69,17 +69,19 @@ int main() {
               // when int2 may not)
               const int U = T * k < E ? T * k : E;
               for (int fm = 1; fm <= 3; ++fm) {
+                const bool gate = fm == 2;  // the shared-gate row on one of the format mixes
                 std::vector<int> fmt(U, fm);
-                std::vector<int> rows(E, 0), tparts(size_t(U + 1) * (I / 8), 0), outc(size_t(U + 1) * H, 0);
+                std::vector<int> rows(E + 1, 0), tparts(size_t(U + 1) * (I / 8), 0), outc(size_t(U + 1) * H, 0);
                 for (int b = 0; b < G; ++b) {
                   int e0, nrr;
                   router_range(E, G, b, e0, nrr);
-                  const int na = phase_a_jobs(H, I, E, G, b, fm, jobs.data());
+                  const int na = phase_a_jobs(H, I, E, G, b, fm, gate, jobs.data());
                   if (na > kMaxJobs) { ++bad_fields; continue; }
                   for (int j = 0; j < na; ++j) {
                     const Job& jb = jobs[j];
                     if (jb.kind == kRouter) {
-                      if (jb.part == 0) rows[e0 + jb.slot]++;
+                      if (jb.slot > nrr || (jb.slot == nrr && !(gate && b == G - 1))) ++bad_fields;
+                      if (jb.part == 0) rows[jb.slot == nrr ? E : e0 + jb.slot]++;
                     } else {
                       tparts[size_t(U) * (I / 8) + jb.row0 / 8]++;
                       if (jb.tile >= max_tiles(T, I, E, k, G)) ++bad_fields;
@@ -104,6 +106,7 @@ int main() {
                 }
                 for (int e = 0; e < E; ++e)
                   if (rows[e] != 1) ++bad_cover;
+                if (rows[E] != (gate ? 1 : 0)) ++bad_cover;
                 const int ns = gu_split(fm, H);
                 for (size_t i = 0; i < tparts.size(); ++i)
                   if (tparts[i] != ns) ++bad_cover;

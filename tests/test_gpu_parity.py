@@ -58,6 +58,13 @@ SMALL = {
     "tc_skew": wlm.Workload("tc_skew", T=1000, H=256, I=128, E=64, k=3, zipf_s=2.0, seed=14),
     "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
                               shared_qtype=wlm.Q_INT2_ASYM_G16),
+    # 256 routed experts (the pages' Coder variant keeps half of the 512) on
+    # each expert path: the fused decode kernel, the tcgen05 grouped GEMM
+    # (H, I multiples of 128) and the general kernels (H = 192)
+    "e256_fused_T2": wlm.Workload("e256_fused_T2", T=2, H=2048, I=768, E=256, k=10, zipf_s=1.1, seed=17),
+    "e256_tc": wlm.Workload("e256_tc", T=300, H=512, I=256, E=256, k=8, zipf_s=1.0, seed=18),
+    "e256_simt": wlm.Workload("e256_simt", T=37, H=192, I=128, E=256, k=8, zipf_s=0.8, seed=19,
+                              shared_qtype=wlm.Q_INT8_PER_CHANNEL),
 }
 
 

@@ -45,7 +45,7 @@ def _down_transposed(wg, wu, wd, x):
     return h, h @ wd  # uses W_d untransposed (only shape-valid when square)
 
 
-def _softmax_free_gates(x_bits, w_router, bias, k):
+def _softmax_free_gates(x_bits, w_router, bias, k, bias_selection_only=False):
     logits = mo.router_logits(x_bits, w_router, bias)
     idx = mo.topk_order(logits, k)
     sel = np.take_along_axis(logits, idx.astype(np.int64), axis=1)
@@ -87,26 +87,35 @@ def _sigmoid_for_silu(wg, wu, wd, x):
     return h, h @ wd.T
 
 
-def _gates_not_renormalised(x_bits, w_router, bias, k):
+def _gates_not_renormalised(x_bits, w_router, bias, k, bias_selection_only=False):
     logits, idx, _ = ORIG_ROUTE(x_bits, w_router, bias, k)
     p = mo.softmax(logits)
     return logits, idx, np.take_along_axis(p, idx.astype(np.int64), axis=1)
 
 
-def _bias_only_selects(x_bits, w_router, bias, k):
+def _bias_only_selects(x_bits, w_router, bias, k, bias_selection_only=False):
     logits, idx, _ = ORIG_ROUTE(x_bits, w_router, bias, k)
     p = mo.softmax(logits - np.asarray(bias, np.float64))
     sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
     return logits, idx, sel / sel.sum(axis=1, keepdims=True)
 
 
-def _bias_only_gates(x_bits, w_router, bias, k):
+def _bias_only_gates(x_bits, w_router, bias, k, bias_selection_only=False):
     """Selection on the unbiased logits, gates from the biased softmax."""
     logits = mo.router_logits(x_bits, w_router, bias)
     idx = mo.topk_order(logits - np.asarray(bias, np.float64), k)
     p = mo.softmax(logits)
     sel = np.take_along_axis(p, idx.astype(np.int64), axis=1)
     return logits, idx, sel / sel.sum(axis=1, keepdims=True)
+
+
+def _selection_only_ignored(x_bits, w_router, bias, k, bias_selection_only=False):
+    """The variant flag dropped: gates always from the biased logits."""
+    return ORIG_ROUTE(x_bits, w_router, bias, k, False)
+
+
+def _shared_gate_without_sigmoid(x_bits, gate_w):
+    return mo.bf16_bits_to_f64(x_bits) @ np.asarray(gate_w, dtype=np.float64)
 
 
 def _dispatch_descending(idx, E):
@@ -160,6 +169,11 @@ def _pins_pass():
             pins.test_routing_closed_form(case)
         for case in pins._routing_bias_cases():
             pins.test_routing_bias_closed_form(case)
+        for case in pins._variant_cases("sel"):
+            pins.test_bias_selection_only_closed_form(case)
+        for case in pins._variant_cases("gate"):
+            pins.test_shared_gate_closed_form(case)
+        pins.test_sigmoid_gated_shared_expert_through_the_layer()
         pins.test_swiglu_expert_closed_form()
         pins.test_layer_closed_form_through_routing()
         for k in (1, 2, 3):
@@ -187,6 +201,8 @@ def _pins_pass():
     ("route", _gates_not_renormalised),
     ("route", _bias_only_selects),
     ("route", _bias_only_gates),
+    ("route", _selection_only_ignored),
+    ("shared_gate", _shared_gate_without_sigmoid),
     ("dispatch", _dispatch_descending),
     ("dispatch", _dispatch_inclusive_offsets),
     ("combine", _combine_without_shared),

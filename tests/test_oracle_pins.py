@@ -125,6 +125,72 @@ def test_routing_bias_closed_form(case):
     np.testing.assert_allclose(w, np.asarray(w_exp), rtol=0, atol=1e-15)
 
 
+def _variant_cases(kind):
+    cases = []
+    for line in open(os.path.join(GOLDEN, "router_variants_closed_form.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = [p.strip() for p in line.split("|")]
+        if parts[0] != kind:
+            continue
+        if kind == "sel":
+            cases.append((int(parts[1]), [_parse_logits(t) for t in parts[2].split()],
+                          [_parse_logits(t) for t in parts[3].split()], [int(v) for v in parts[4].split()],
+                          [float(v) for v in parts[5].split()]))
+        else:
+            cases.append((_parse_logits(parts[1]), float(parts[2])))
+    return cases
+
+
+@pytest.mark.parametrize("case", _variant_cases("sel"))
+def test_bias_selection_only_closed_form(case):
+    """The bias picks the experts; the gates come from the unbiased logits
+    (hand-worked values in tests/golden/router_variants_closed_form.txt)."""
+    k, r, b, idx_exp, w_exp = case
+    E, H = len(r), 8
+    x = np.zeros((1, H), dtype=np.float32)
+    x[0, 0] = 1.0
+    w_r = np.zeros((E, H), dtype=np.float64)
+    w_r[:, 0] = r
+    logits, idx, w = oracle.route(wlm.f32_to_bf16_bits(x), w_r, np.asarray(b), k, bias_selection_only=True)
+    assert idx[0].tolist() == idx_exp
+    np.testing.assert_allclose(w[0], w_exp, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(logits[0], np.asarray(r) + np.asarray(b), rtol=0, atol=1e-15)  # biased logits
+
+
+@pytest.mark.parametrize("case", _variant_cases("gate"))
+def test_shared_gate_closed_form(case):
+    gx, expect = case
+    x = np.zeros((1, 8), dtype=np.float32)
+    x[0, 0] = 1.0
+    g = np.zeros(8)
+    g[0] = gx
+    np.testing.assert_allclose(oracle.shared_gate(wlm.f32_to_bf16_bits(x), g), [expect], rtol=0, atol=1e-15)
+
+
+def test_sigmoid_gated_shared_expert_through_the_layer():
+    """The closed-form expert as both the routed pick (gate 1, k = 1) and the
+    shared expert with sigma(g . x) = 3/4: the output is 1.75 times its y."""
+    ex, _, y_exp = _closed_form_fixture()
+    zero = _closed_form_fixture()[0]
+    zero.down = _int4_matrix_from_q(np.zeros((32, 32), dtype=np.int32), 0.125)
+    x = np.zeros((1, 32), dtype=np.float32)
+    x[0, 0] = 1.0
+    xb = wlm.f32_to_bf16_bits(x)
+    w_r = np.zeros((2, 32))
+    w_r[1, 0] = 0.5
+    g = np.zeros(32)
+    g[0] = math.log(3.0)
+    r = oracle.moe_layer(xb, w_r, np.zeros(2), 1, [zero, ex], shared=ex, shared_gate_w=g)
+    n = len(y_exp)  # the fixture's nonzero outputs; the rest are exactly 0
+    np.testing.assert_allclose(r["out"][0, :n], 1.75 * np.asarray(y_exp), rtol=0, atol=1e-12)
+    assert np.all(r["out"][0, n:] == 0.0)
+    cache = oracle.DequantCache([zero, ex])
+    sh = tuple(oracle.dequant_qm(m) for m in (ex.gate, ex.up, ex.down))
+    _, _, out_t = oracle.moe_token(xb[0], w_r, np.zeros(2), 1, cache, sh, shared_gate_w=g)
+    np.testing.assert_allclose(out_t, r["out"][0], rtol=0, atol=1e-12)
+
+
 def test_routing_k1_gate_is_exactly_one():
     rng = np.random.default_rng(3)
     x = wlm.f32_to_bf16_bits(rng.standard_normal((5, 64)).astype(np.float32))

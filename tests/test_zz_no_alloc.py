@@ -72,7 +72,7 @@ def test_noalloc_rejects_sizes_beyond_its_limits():
     from bit_quantized_moe_gemv_b200 import _lib as L
     lib = L.LIB
     # T = 5 exceeds the 4-token limit; E = 2048 and k = 17 exceed theirs.
-    args = (None, None, 0, None, None, None, None, None, None, None)
+    args = (None, None, 0, None, None, None, None, None, None, None, None)
     assert lib.moe_layer_decode_noalloc(None, 5, 1024, 512, 64, 8, *args) == 2
     assert lib.moe_layer_decode_noalloc(None, 1, 1024, 512, 2048, 8, *args) == 2
     assert lib.moe_layer_decode_noalloc(None, 1, 1024, 512, 64, 17, *args) == 2
