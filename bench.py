@@ -76,9 +76,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode1", choices=["decode1", "decode48", "prefill8k", "prefill32k"])
+    ap.add_argument("--workload", default="decode1",
+                    choices=["decode1", "verify4", "decode48", "prefill8k", "prefill32k"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="bound on each CPU-baseline sample")
+    ap.add_argument("--no-graph", action="store_true", help="decode48: plain launches instead of a CUDA graph")
     ap.add_argument("--headline-only", action="store_true",
                     help="decode1 only (by default the decode1 line also carries prefill8k and decode48 results)")
     ap.add_argument("--clock-window", type=float, default=1.2,
@@ -452,7 +454,13 @@ def run_stack(args, rank, world, peaks, peak_kind):
     all 48 layers, each layer with its own weights and fresh tokens (layers
     are not chained, so every layer sees the specified routing). The whole
     stack (58 GB) is resident and far larger than L2, so no flush is needed.
-    Weights are drawn on the device (workload.draw_layer_device)."""
+    Weights are drawn on the device (workload.draw_layer_device).
+
+    The 48 moe_layer launches of a step are captured once into a CUDA graph
+    over static input/output buffers and replayed every step (no host launch
+    overhead between layers); each step's tokens are staged into the static
+    input buffer before its start event, its routing copied out after its end
+    event. --no-graph times the plain launches instead."""
     import torch
 
     from bit_quantized_moe_gemv_b200 import _lib as L
@@ -479,25 +487,59 @@ def run_stack(args, rank, world, peaks, peak_kind):
     ws = L.new_workspace(T, H, I, E, k, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(s):
+    def layers_into(xb, ib, wb, ob):
         for li in range(NL):
             ex, sh = tables[li]
-            L.layer(xs[s, li], I, E, k, layers[li]["w_router"], b, stride, ex.table, sh.table, idx[s, li],
-                    gw[s, li], out[s, li], ws, stream=stream)
+            L.layer(xb[li], I, E, k, layers[li]["w_router"], b, stride, ex.table, sh.table, ib[li], wb[li], ob[li],
+                    ws, stream=torch.cuda.current_stream())
+
+    graph, launches_per_step = None, NL
+    if not args.no_graph:
+        x_st = torch.empty((NL, T, H), dtype=torch.bfloat16, device=dev)
+        i_st = torch.empty((NL, T, k), dtype=torch.int32, device=dev)
+        w_st = torch.empty((NL, T, k), dtype=torch.float32, device=dev)
+        o_st = torch.empty((NL, T, H), dtype=torch.bfloat16, device=dev)
+        x_st.copy_(xs[0])
+        layers_into(x_st, i_st, w_st, o_st)  # first calls outside the capture (one-time attribute set-up)
+        torch.cuda.synchronize()
+        n0 = L.launch_count()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layers_into(x_st, i_st, w_st, o_st)
+        launches_per_step = L.launch_count() - n0
+        torch.cuda.synchronize()
+
+    def step(s):
+        if graph is None:
+            layers_into(xs[s], idx[s], gw[s], out[s])
+        else:
+            graph.replay()
+
+    def stage_in(s):
+        if graph is not None:
+            x_st.copy_(xs[s])
+
+    def stage_out(s):
+        if graph is not None:
+            idx[s].copy_(i_st)
+            gw[s].copy_(w_st)
+            out[s].copy_(o_st)
 
     def timed_loop(first, count, host_io=None):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(count)]
         for i in range(count):
             s = first + i
             if host_io is None:
+                stage_in(s)
                 torch.cuda._sleep(LEAD_CYCLES)
             evs[i][0].record(stream)
             if host_io is not None:
-                xs[s].copy_(host_io[0][s], non_blocking=True)
+                (x_st if graph is not None else xs[s]).copy_(host_io[0][s], non_blocking=True)
             step(s)
             if host_io is not None:
-                host_io[1][s].copy_(out[s], non_blocking=True)
+                host_io[1][s].copy_(o_st if graph is not None else out[s], non_blocking=True)
             evs[i][1].record(stream)
+            stage_out(s)
         torch.cuda.synchronize()
         return [a.elapsed_time(z) for a, z in evs]
 
@@ -506,7 +548,9 @@ def run_stack(args, rank, world, peaks, peak_kind):
     def measured():
         launches0 = L.launch_count()
         t = timed_loop(args.warmup, args.steps)
-        return t, L.launch_count() - launches0
+        # graph replays launch the captured kernels without calling the library
+        n = L.launch_count() - launches0 if graph is None else launches_per_step * args.steps
+        return t, n
 
     (times, launches), clk = timed_region(measured, rank, world, dev, filler=lambda: step(args.warmup),
                                           window=args.clock_window)
@@ -534,7 +578,9 @@ def run_stack(args, rank, world, peaks, peak_kind):
         "config": dict(workload_config(wl, world), layers=NL,
                        l2="inputs larger than L2 (58 GB stack streamed every step)"),
         "roofline": {
-            "bound": "hbm", "kernel": "moe_layer x 48 layers (one launch per layer)",
+            "bound": "hbm",
+            "kernel": ("moe_layer x 48 layers, one CUDA graph per step (one fused decode launch per layer)"
+                       if graph is not None else "moe_layer x 48 layers (one launch per layer)"),
             "achieved": achieved_gbs, "peak": peak, "unit": "GB/s", "frac": achieved_gbs / peak,
             "peak_source": f"{peak_kind} hbm_gbs",
             "algorithmic_bytes_per_step": float(np.mean(bytes_per_step)),

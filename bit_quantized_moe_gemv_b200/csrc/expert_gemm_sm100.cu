@@ -7,7 +7,9 @@
 // used as stored, so each weight rounds once, at 2^-11; bf16 would round the
 // scale and then the product at 2^-8 each, which breaks the 2e-2 x rms
 // max-error bound on long dot products. The bf16 activations convert to fp16
-// exactly in the normal range (values beyond +-65504 saturate).
+// exactly after a per-row power-of-two scaling into fp16's range, and the
+// SwiGLU output is scaled the same way (kHShift below), both undone on the
+// fp32 results.
 //
 // Prefill pushes many tokens through each expert at once (the telli.sh page
 // "Strata 与 Qwen3.8-Flash-Next：如何在个人电脑上运行 180B 级模型", section
@@ -147,6 +149,20 @@ __device__ __forceinline__ uint32_t tile_off(int row, int k) {
 
 // ---------------------------------------------------------------- fp16 helpers
 __device__ __forceinline__ float sat_f16(float v) { return fminf(fmaxf(v, -65504.f), 65504.f); }
+
+// Range of the fp16 operands. Each gathered row of x is scaled by 2^-e
+// (e >= 0, exact) so that |x| < 2^8; the SwiGLU output h of that row is
+// stored as h 2^-(kHShift + 2e) and the down GEMM's result multiplied back.
+// For ordinary rows (|x| < 256) e = 0 and only the fixed 2^-kHShift applies,
+// which moves fp16's overflow from 65504 to 2^kHShift x 65504 and costs h
+// values below 2^(kHShift - 14) some relative precision (absolute error
+// under 2^(kHShift - 24)).
+constexpr int kHShift = 8;
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // -126 <= e <= 127
+__device__ __forceinline__ int row_exp(uint32_t amax_bf16) {  // bf16 magnitude bits
+  const int ex = int((amax_bf16 >> 7) & 0xff) - 127;          // floor(log2 |x|) of the largest element
+  return ex >= 8 ? (ex - 7 < 119 ? ex - 7 : 119) : 0;
+}
 __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -156,7 +172,7 @@ __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
 // One warp per tile row: token row -> 16 KiB swizzled tiles of X (K = H).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                           const int* __restrict__ perm_src, int E, Plan plan,
-                                                          uint8_t* __restrict__ xt) {
+                                                          uint8_t* __restrict__ xt, int* __restrict__ xexp) {
   const int ntiles = plan.count[0];
   const int KB = H / BK;
   const int lane = threadIdx.x & 31;
@@ -168,15 +184,28 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     const int r = plan.row0[rt] + row;
     const int tok = g < E ? perm_src[r] / k : r;
     const uint4* src = reinterpret_cast<const uint4*>(x + size_t(tok) * H);
+    // the row's largest |x| (bf16 magnitude bits compare as integers)
+    uint32_t am = 0;
     for (int c = lane; c < H / 8; c += 32) {
       const uint4 v = __ldg(src + c);
-      // bf16 -> fp16 (saturating at +-65504), K order (0,4,1,5,2,6,3,7)
+      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) am = max(am, max(in[i] & 0x7fffu, (in[i] >> 16) & 0x7fffu));
+    }
+    am = __reduce_max_sync(0xffffffffu, am);
+    const int e = row_exp(am);
+    const float sc = pow2f(-e);
+    if (lane == 0) xexp[size_t(rt) * BN + row] = e;
+    for (int c = lane; c < H / 8; c += 32) {
+      const uint4 v = __ldg(src + c);
+      // bf16 -> fp16 after the row's scaling (|x| < 2^8; inf saturates at
+      // +-65504), K order (0,4,1,5,2,6,3,7)
       const uint32_t in[4] = {v.x, v.y, v.z, v.w};
       float f[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        f[2 * i] = sat_f16(__uint_as_float(in[i] << 16));
-        f[2 * i + 1] = sat_f16(__uint_as_float(in[i] & 0xffff0000u));
+        f[2 * i] = sat_f16(__uint_as_float(in[i] << 16) * sc);
+        f[2 * i + 1] = sat_f16(__uint_as_float(in[i] & 0xffff0000u) * sc);
       }
       uint4 o;
       o.x = h2_bits(f[0], f[4]);
@@ -376,6 +405,7 @@ struct Args {
   int M;              // weight rows (I for gate/up, H for down)
   int I, H;
   const uint8_t* bt;  // B tiles [tiles][K/64][16 KiB]
+  const int* xexp;    // per gathered row (tile * 128 + row): the power-of-two scaling of x
   uint8_t* ht;        // gate/up: H tiles out [tiles][I/64][16 KiB]
   float* y_f32;       // down: fp32 rows out (routed rows), or nullptr
   uint16_t* y_bf16;   // down: bf16 rows out, or nullptr
@@ -736,27 +766,40 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes + size_t(c0) * 128 +
                           (e < 4 ? 4 * e : 4 * (e - 4) + 2);
           const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+          const int* xe = a.xexp + size_t(rt) * BN + c0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (j < nv) {
-              const float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]);
-              *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) =
-                  __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
+              // the row's x was scaled by 2^-e: g = g_s 2^e, u = u_s 2^e, and
+              // h 2^-(kHShift + 2e) = silu(g) 2^-e u_s 2^-kHShift
+              const int e = xe[j];
+              const float gv = __uint_as_float(v0[j]) * pow2f(e), uv = __uint_as_float(v1[j]);
+              const float hs = __fdividef(gv, 1.0f + __expf(-gv)) * pow2f(-e) * uv * (1.0f / (1 << kHShift));
+              *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) = __float2half_rn(sat_f16(hs));
             }
           }
         } else {
           ptx::tmem_ld_wait();
           const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+          // undo the scaling of h: y = y_s 2^(kHShift + 2e) for the row's e
+          const int* xe = a.xexp + size_t(rt) * BN + c0;
+          float yv[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int e = j < nv ? xe[j] : 0;
+            const float v = __uint_as_float(v0[j]);
+            yv[j] = e == 0 ? v * float(1 << kHShift) : ldexpf(v, kHShift + 2 * e);
+          }
           if (g < a.E && a.y_f32 == nullptr) {
             uint16_t* yp = a.y_bf16 + size_t(row0 + c0) * a.H + m;
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (j < nv) yp[size_t(j) * a.H] = f32_to_bf16_rn(__uint_as_float(v0[j]));
+              if (j < nv) yp[size_t(j) * a.H] = f32_to_bf16_rn(yv[j]);
           } else {  // fp32 rows: column m of rows row0 + c0 .. (one pointer step of H per row)
             float* yp = (g < a.E ? a.y_f32 : a.ys_f32) + size_t(row0 + c0) * a.H + m;
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (j < nv) yp[size_t(j) * a.H] = __uint_as_float(v0[j]);
+              if (j < nv) yp[size_t(j) * a.H] = yv[j];
           }
         }
       }
@@ -805,7 +848,7 @@ int grouped_heavy_slots(long long T, int k, bool with_shared, int H, int I) {
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
   const long long mt = grouped_max_tiles(T, k, E, with_shared);
   return align256(16 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
-         align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
+         align256(4 * size_t(mt) * gemm::BN) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(grouped_heavy_slots(T, k, with_shared, H, I)) * gemm::heavy_slot_bytes(H, I));
 }
@@ -828,6 +871,8 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   plan.hslot = reinterpret_cast<int*>(p);
   plan.hlist = plan.hslot + (E + 1);
   p += align256(4 * size_t(E + 1) + 4 * size_t(kMaxHeavy));
+  int* xexp = reinterpret_cast<int*>(p);
+  p += align256(4 * size_t(mt) * BN);
   uint8_t* xt = p;
   p += align256(size_t(mt) * (H / BK) * kTileBytes);
   uint8_t* ht = p;
@@ -840,7 +885,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), max_heavy, plan);
-  gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt);
+  gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt, xexp);
   if (max_heavy > 0) predequant_kernel<<<sms * 4, 256, 0, st>>>(experts, shared, E, H, I, plan, aimg, hdr);
   const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
   const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
@@ -859,6 +904,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.hdr = hdr;
   a.aimg = aimg;
   a.aslot = heavy_slot_bytes(H, I);
+  a.xexp = xexp;
   // gate/up: K = H, M = I; B = gathered X tiles; out = H tiles
   a.K = H;
   a.M = I;

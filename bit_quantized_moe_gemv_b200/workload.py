@@ -134,6 +134,12 @@ WORKLOADS = {
         "decode48", T=4, H=2048, I=768, E=512, k=10, layers=48, steps=200, zipf_s=1.1,
         routed_qtypes=((0, None, Q_INT2_ASYM_G16),), shared_qtype=Q_INT8_PER_CHANNEL,
     ),
+    # Verification batch of speculative decoding: one sequence's current token
+    # plus 3 drafted ones checked in one pass (4 tokens of ONE slot), the
+    # decode1 layer otherwise. The telli.sh page "Strata 与 Qwen3.8-Flash-Next：
+    # 如何在个人电脑上运行 180B 级模型", section "推测解码只有在验证通过时才节省计算",
+    # drafts up to 3 tokens that the target model verifies in one pass.
+    "verify4": Workload("verify4", T=4, H=2048, I=768, E=512, k=10, steps=200, zipf_s=1.1),
     # Prefill 8K tokens, Zipf(1.0) skew.
     "prefill8k": Workload("prefill8k", T=8192, H=2048, I=768, E=512, k=10, zipf_s=1.0),
     # Long prefill 32K, mixed per-expert precision, Zipf(1.2) + 5% uniform rows.

@@ -199,6 +199,22 @@ def test_layer_decode1_steps(L):
         _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, [0])
 
 
+def test_layer_verify4_steps(L):
+    """A speculative-decoding verification batch (4 tokens of one sequence,
+    the decode1 layer) through the fused decode kernel: routing exact against
+    the oracle (outside near-ties), every token's output within tolerance."""
+    wl = wlm.WORKLOADS["verify4"]
+    lay = wlm.gen_layer(wl)
+    dev = pu.upload_layer(lay)
+    bias, stride = wlm.gen_bias(wl)
+    ws = L.new_workspace(wl.T, wl.H, wl.I, wl.E, wl.k)
+    for step in range(3):
+        xb = wlm.gen_x(wl, step=step)
+        idx, w, out, lg = _layer_call(L, wl, dev, xb, bias, stride, ws, with_logits=True)
+        pu.check_routing(idx, w, lg, xb, lay.w_router, bias, wl.k)
+        _check_sampled_tokens(wl, lay, xb, bias, stride, idx, w, out, list(range(wl.T)))
+
+
 @pytest.mark.parametrize("name", ["prefill8k", "prefill32k"])
 def test_prefill_full_routing_dispatch_every_output(L, name):
     import torch
