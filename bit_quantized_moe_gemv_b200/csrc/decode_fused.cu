@@ -53,7 +53,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxT = 4;
 constexpr int kMaxK = 16;
 constexpr int kMaxSlots = kMaxT * kMaxK + 1;  // routed slots + the shared expert
-constexpr int kMaxJobs = 640;
+constexpr int kMaxJobs = 1280;  // two lists of kMaxJobs / 2: phase A, then phases B and C
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kTopChunk = 128;  // logits per first-round top-k job (4 per lane)
 
@@ -681,23 +681,33 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   __syncwarp();
 }
 
-// router part: row e0 + r, floats [s seg, (s + 1) seg) of it; the last part
-// of the CTA to finish sums each row's parts in order, adds the bias,
-// publishes the logits and arrives on the grid counter.
-__device__ __noinline__ void job_router(Ctx& C, const Job jb) {
+// The weights of router part (row e0 + r, floats [s seg, (s + 1) seg)) for
+// this lane: 4 (or 2) 16-byte loads. Issued before anything else of the
+// launch, so the router's bytes are on their way while the prologue runs.
+__device__ __forceinline__ void router_load(const Params& P, int e0, int nreal, int seg, const Job& jb,
+                                            uint4 (&w)[4]) {
+  const int lane = threadIdx.x & 31;
+  const bool gate_row = jb.slot >= nreal;  // the shared expert's gate vector
+  const float* wr = (gate_row ? P.shared_gate : P.w_router + size_t(e0 + jb.slot) * P.H) + jb.part * seg;
+  const int nv = seg / 128;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (i < nv) w[i] = ldg16(wr + 4 * lane + 128 * i);
+}
+
+// router part: row e0 + r, floats [s seg, (s + 1) seg) of it, with its
+// weights already loaded; the last part of the CTA to finish sums each row's
+// parts in order, adds the bias, publishes the logits and arrives on the
+// grid counter.
+__device__ __noinline__ void job_router(Ctx& C, const Job jb, const uint4 w0, const uint4 w1, const uint4 w2,
+                                        const uint4 w3) {
   const Params& P = *C.P;
   const int T = C.T, H = C.H, E = C.E, seg = C.seg, nseg = C.nseg;
   const int lane = threadIdx.x & 31;
   const float* x32 = reinterpret_cast<const float*>(C.smem + C.L.o_x32);
   float* rp = reinterpret_cast<float*>(C.smem + C.L.o_rp);
-  const bool gate_row = jb.slot >= C.nreal;  // the shared expert's gate vector
-  const int e = C.e0 + jb.slot;
-  const float* wr = (gate_row ? P.shared_gate : P.w_router + size_t(e) * H) + jb.part * seg;
   const int nv = seg / 128;  // 16-byte loads per lane (4 or 2)
-  uint4 w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (i < nv) w[i] = ldg16(wr + 4 * lane + 128 * i);
+  const uint4 w[4] = {w0, w1, w2, w3};
 #pragma unroll
   for (int t = 0; t < kMaxT; ++t) {
     if (t >= T) break;
@@ -739,46 +749,193 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb) {
 }
 
 // ---------------------------------------------------------------- the kernel
+// Routing of one CTA, run by its last T warps (one token each) while the
+// others may still work on phase A: wait for every CTA's logits, top-k per
+// token, gates, the distinct picked experts (slots), their descriptors and
+// this CTA's job list of phases B and C. Lane 0 of warp kWarps - T publishes
+// the result through `ready` (1 = go, 2 = nothing to do).
+struct RouteShared {
+  int idx[kMaxT * kMaxK];
+  float w[kMaxT * kMaxK];
+  uint32_t key[kMaxT * kMaxK];
+  int slot[kMaxT * kMaxK];      // (t, j) -> slot
+  int uniq[kMaxT * kMaxK];      // slot -> expert id
+  int fmt[kMaxT * kMaxK];       // slot -> weight format
+  uint32_t ck[kMaxT * 8 * kMaxK];  // first-round winners
+  int ci[kMaxT * 8 * kMaxK];
+  uint32_t bits[kMaxE / 32];
+  int U, nJ, bad;
+  volatile int ready;
+};
+
+__device__ __noinline__ void route_cta(Ctx& C, RouteShared& R, bool has_shared) {
+  const Params& P = *C.P;
+  const int T = C.T, E = C.E, k = C.k, H = C.H, I = C.I;
+  const int lane = threadIdx.x & 31, t = (threadIdx.x >> 5) - (kWarps - T);  // this warp's token
+  const int nthr = T * 32;
+  auto rsync = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory"); };
+  if (t == 0 && lane == 0) {
+    if (!wait_counter(&P.hdr->bar_count, uint32_t(C.G), P.hdr, P.wait_cycles, 7000000 + C.b)) C.fail = 1;
+  }
+  rsync();
+  const bool live = !C.fail;
+  float* lg = reinterpret_cast<float*>(C.smem + C.L.o_lg);
+  if (live)
+    for (int i = threadIdx.x - (kWarps - T) * 32; i < T * E; i += nthr) lg[i] = __ldcg(P.logits + i);
+  for (int i = threadIdx.x - (kWarps - T) * 32; i < kMaxE / 32; i += nthr) R.bits[i] = 0u;
+  rsync();
+  // this token's top-k in two rounds: its 128-logit chunks, then their winners
+  if (live) {
+    const int nch = (E + kTopChunk - 1) / kTopChunk;
+    for (int stage = 0; stage < 2; ++stage) {
+      for (int ch = 0; ch < (stage == 0 ? nch : 1); ++ch) {
+        const int nc = stage == 0 ? min(kTopChunk, E - ch * kTopChunk) : nch * k;
+        const uint32_t* ck = R.ck + t * 8 * kMaxK;
+        const int* ci = R.ci + t * 8 * kMaxK;
+        uint64_t cand[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int c = lane + 32 * i;
+          const uint32_t key = c >= nc ? 0u : stage == 0 ? f2key(lg[t * E + ch * kTopChunk + c]) : ck[c];
+          const int id = stage == 0 ? ch * kTopChunk + c : ci[c < nc ? c : 0];
+          cand[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(id)) : 0ull;
+        }
+        uint32_t* okey = stage == 0 ? R.ck + t * 8 * kMaxK + ch * k : R.key + t * k;
+        int* oid = stage == 0 ? R.ci + t * 8 * kMaxK + ch * k : R.idx + t * k;
+        warp_topk(cand, k, okey, oid);
+        __syncwarp();
+      }
+    }
+    // gates: the softmax over all logits restricted to the picks and
+    // renormalised = a softmax over the picked logits (of the unbiased ones
+    // when the bias only selects)
+    const bool sel_only = (P.flags & MOE_BIAS_SELECTION_ONLY) != 0;
+    float v = -CUDART_INF_F;
+    if (lane < k) v = sel_only ? __ldcg(P.logits_u + size_t(t) * E + R.idx[t * k + lane]) : key2f(R.key[t * k + lane]);
+    float v0 = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, o));
+    const float ev = lane < k ? expf(v - v0) : 0.f;
+    const float den = warp_sum(ev);
+    if (lane < k) R.w[t * k + lane] = ev / den;
+    // distinct picked experts in ascending id order through a bitmap
+    if (lane < k) {
+      const int id = R.idx[t * k + lane];
+      if (id >= 0 && id < E) atomicOr(&R.bits[id >> 5], 1u << (id & 31));
+      else R.bad = 1;
+    }
+  }
+  rsync();
+  if (t == 0) {
+    // slot of an id = set bits below it (warp scan over the bitmap words)
+    __shared__ uint32_t s_bpre[kMaxE / 32];
+    uint32_t pre = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32 / 32; ++i) {
+      const uint32_t c = __popc(R.bits[i * 32 + lane]);
+      uint32_t inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      s_bpre[i * 32 + lane] = pre + inc - c;
+      pre += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    __syncwarp();
+    const int U = int(pre);
+    if (live && !R.bad)
+      for (int i = lane; i < T * k; i += 32) {
+        const int id = R.idx[i], wd = id >> 5;
+        const int rank = int(s_bpre[wd] + __popc(R.bits[wd] & ((1u << (id & 31)) - 1u)));
+        R.slot[i] = rank;
+        R.uniq[rank] = id;
+      }
+    __syncwarp();
+    moe_expert* desc = C.desc;
+    constexpr int W = int(sizeof(moe_expert) / 4);
+    if (live && !R.bad) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
+      uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
+      for (int i = lane; i < U * W; i += 32) dst[i] = src[size_t(R.uniq[i / W]) * W + (i % W)];
+    }
+    __syncwarp();
+    bool bad = R.bad != 0;
+    if (live && !bad)
+      for (int u = lane; u < U; u += 32) {
+        if (!expert_ok(desc[u], H, I)) R.bad = 1;
+        R.fmt[u] = desc[u].gate.qtype;
+      }
+    __syncwarp();
+    bad = R.bad != 0;
+    if (live && bad && lane == 0) flag_error(P.hdr, MOE_ERR_DEVICE_FAULT, 1000000);
+    const bool work = live && !bad;
+    if (work) {
+      // this CTA's down rows of every picked expert into L2
+      if (C.nr > 0)
+        for (int u = lane; u < U; u += 32) {
+          const moe_qmatrix& dm = desc[u].down;
+          const int rb = row_code_bytes(dm.qtype, I);
+          prefetch_l2(dm.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
+        }
+      if (lane == 0)
+        R.nJ = phase_bc_jobs(H, I, C.G, C.b, U, R.fmt, has_shared, reinterpret_cast<Job*>(C.smem + C.L.o_jobs) + kMaxJobs / 2);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      R.U = U;
+      __threadfence_block();
+      R.ready = work ? 1 : 2;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Ctx C;
+  __shared__ RouteShared R;
   __shared__ uint32_t s_xamax[kMaxT];
-  __shared__ int s_nA, s_nJ, s_U, s_bad;
-  __shared__ int s_idx[kMaxT * kMaxK];
-  __shared__ float s_w[kMaxT * kMaxK];
-  __shared__ uint32_t s_key[kMaxT * kMaxK];
-  __shared__ int s_slot[kMaxT * kMaxK];         // (t, j) -> slot
-  __shared__ int s_uniq[kMaxT * kMaxK];         // slot -> expert id
-  __shared__ int s_fmt[kMaxT * kMaxK];          // slot -> weight format
-  __shared__ uint32_t s_ck[kMaxT * 8 * kMaxK];  // first-round winners
-  __shared__ int s_ci[kMaxT * 8 * kMaxK];
-  __shared__ uint32_t s_bits[kMaxE / 32];
-  __shared__ uint32_t s_bpre[kMaxE / 32];
+  __shared__ int s_nA, s_bad;
 
   const int T = P.T, H = P.H, I = P.I, E = P.E, k = P.k;
   const int G = gridDim.x, b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* hdr = P.hdr;
   const bool has_shared = P.shared != nullptr;
-  moe_expert* desc = reinterpret_cast<moe_expert*>(smem + make_plan(T, H, I, E, k, G).o_desc);
+  const bool gate_row = P.shared_gate != nullptr && has_shared;
+
+  // ---------------------------------------------------------- router loads first
+  // The phase-A job list starts with the router parts (row-major), so this
+  // warp's first job is part `warp` when there is one: load its weights now.
+  int e0, nreal;
+  router_range(E, G, b, e0, nreal);
+  const int seg = router_seg(H), nseg = H / seg;
+  const int nrr = router_rows_of(E, G, b, gate_row);
+  uint4 w0[4] = {};
+  const bool early = warp < nrr * nseg;
+  if (early) router_load(P, e0, nreal, seg, Job{kRouter, uint8_t(warp / nseg), 0, uint8_t(warp % nseg), 0, 0}, w0);
 
   // ---------------------------------------------------------- prologue
+  moe_expert* desc = reinterpret_cast<moe_expert*>(smem + make_plan(T, H, I, E, k, G).o_desc);
   if (threadIdx.x == 0) {
     C.P = &P;
     C.smem = smem;
     C.L = make_plan(T, H, I, E, k, G);
     C.T = T, C.H = H, C.I = I, C.E = E, C.k = k, C.G = G, C.b = b;
-    router_range(E, G, b, C.e0, C.nreal);
-    C.nrr = router_rows_of(E, G, b, P.shared_gate != nullptr && has_shared);
-    C.seg = router_seg(H);
-    C.nseg = H / C.seg;
+    C.e0 = e0;
+    C.nreal = nreal;
+    C.nrr = nrr;
+    C.seg = seg;
+    C.nseg = nseg;
     out_rows(H, G, b, C.n0, C.nr);
-    for (int i = 0; i < 4; ++i) C.fmap[i] = -1;
+    for (int i = 0; i < 4; ++i) C.fmap[i] = i - 1;  // formats 1..3 -> activation buffers 0..2
     C.fail = 0;
     C.rdone = 0;
     C.desc = desc;
     s_bad = 0;
-    s_U = 0;
+    R.bad = 0;
+    R.ready = 0;
+    R.U = 0;
   }
   if (threadIdx.x < kMaxT) s_xamax[threadIdx.x] = 0u;
   if (has_shared && threadIdx.x < int(sizeof(moe_expert) / 4))
@@ -823,174 +980,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         prefetch_l2(d.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
       }
     }
-    s_nA = phase_a_jobs(H, I, E, G, b, has_shared && good ? desc[kSharedSlot].gate.qtype : 0,
-                        P.shared_gate != nullptr && has_shared, reinterpret_cast<Job*>(smem + C.L.o_jobs));
+    s_nA = phase_a_jobs(H, I, E, G, b, has_shared && good ? desc[kSharedSlot].gate.qtype : 0, gate_row,
+                        reinterpret_cast<Job*>(smem + L.o_jobs));
   }
+  __syncthreads();
+  // activations in fragment order for all three formats (from global x: x32
+  // is reused after phase A), so routed experts of any format need no
+  // further barrier
+  for (int i = threadIdx.x; i < T * H; i += kThreads) {
+    const int t = i / H, kk = i - t * H;
+    const __half v = __float2half_rn(ldexpf(bf16_to_f32(P.x[i]), -C.xexp[t]));
+    for (int f = 1; f <= 3; ++f) *reinterpret_cast<__half*>(smem + L.o_xf + (f - 1) * 2 * T * H + frag_pos(f, kk, t, T)) = v;
+  }
+  if (nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
   __syncthreads();
   const int nA = s_nA;
-  // activations of format f in fragment order (from global x: x32 is reused
-  // after phase A)
-  auto build_xf = [&](int f, int buf) {
-    uint8_t* xf = smem + L.o_xf + buf * 2 * T * H;
-    for (int i = threadIdx.x; i < T * H; i += kThreads) {
-      const int t = i / H, kk = i - t * H;
-      const float v = ldexpf(bf16_to_f32(P.x[i]), -C.xexp[t]);
-      *reinterpret_cast<__half*>(xf + frag_pos(f, kk, t, T)) = __float2half_rn(v);
-    }
-  };
-  if (has_shared && !s_bad) {
-    build_xf(desc[kSharedSlot].gate.qtype, 0);
-    if (threadIdx.x == 0) C.fmap[desc[kSharedSlot].gate.qtype] = 0;
-  }
-  if (C.nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
-  __syncthreads();
 
   // ---------------------------------------------------------- phase A
   {
     const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs);
     for (int j = warp; j < nA; j += kWarps) {
       const Job jb = jobs[j];
-      if (jb.kind == kRouter) job_router(C, jb);
-      else job_gate_up(C, jb);
+      if (jb.kind == kRouter) {
+        uint4 w[4] = {};
+        if (j == warp && early) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) w[i] = w0[i];
+        } else {
+          router_load(P, e0, nreal, seg, jb, w);
+        }
+        job_router(C, jb, w[0], w[1], w[2], w[3]);
+      } else {
+        job_gate_up(C, jb);
+      }
     }
   }
-  __syncthreads();
 
   // ---------------------------------------------------------- routing
-  if (threadIdx.x == 0)
-    if (!wait_counter(&hdr->bar_count, uint32_t(G), hdr, P.wait_cycles, 7000000 + b)) C.fail = 1;
-  __syncthreads();
-  const bool live = !C.fail;
-  float* lg = reinterpret_cast<float*>(smem + L.o_lg);
-  if (live)
-    for (int i = threadIdx.x; i < T * E; i += kThreads) lg[i] = __ldcg(P.logits + i);
-  __syncthreads();
-  // two rounds of warp top-k: one job per (token, 128 logits), each keeping
-  // its chunk's best k; then one warp per token over those (<= 8 x 16 = 128)
-  const int nch = (E + kTopChunk - 1) / kTopChunk;
-  for (int stage = 0; stage < 2; ++stage) {
-    const int njobs = live ? (stage == 0 ? T * nch : T) : 0;
-    for (int jbi = warp; jbi < njobs; jbi += kWarps) {
-      const int t = stage == 0 ? jbi / nch : jbi, ch = stage == 0 ? jbi - t * nch : 0;
-      const int nc = stage == 0 ? min(kTopChunk, E - ch * kTopChunk) : nch * k;
-      const uint32_t* ck = s_ck + t * 8 * kMaxK;
-      const int* ci = s_ci + t * 8 * kMaxK;
-      uint64_t cand[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = lane + 32 * i;
-        const uint32_t key = c >= nc ? 0u : stage == 0 ? f2key(lg[t * E + ch * kTopChunk + c]) : ck[c];
-        const int id = stage == 0 ? ch * kTopChunk + c : ci[c < nc ? c : 0];
-        cand[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(id)) : 0ull;
-      }
-      uint32_t* okey = stage == 0 ? s_ck + t * 8 * kMaxK + ch * k : s_key + t * k;
-      int* oid = stage == 0 ? s_ci + t * 8 * kMaxK + ch * k : s_idx + t * k;
-      warp_topk(cand, k, okey, oid);
-    }
-    __syncthreads();
-  }
-  // gates: the softmax over all logits restricted to the picks and
-  // renormalised = a softmax over the picked logits
-  // (with the selection-only bias: of the unbiased logits of the picks)
-  if (live && warp < T) {
-    const int t = warp;
-    const bool sel_only = (P.flags & MOE_BIAS_SELECTION_ONLY) != 0;
-    float v = -CUDART_INF_F;
-    if (lane < k) v = sel_only ? __ldcg(P.logits_u + size_t(t) * E + s_idx[t * k + lane]) : key2f(s_key[t * k + lane]);
-    float v0 = v;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, o));
-    const float ev = lane < k ? expf(v - v0) : 0.f;
-    const float den = warp_sum(ev);
-    if (lane < k) s_w[t * k + lane] = ev / den;
-  }
-  // distinct picked experts in ascending id order through a bitmap: the
-  // slot of an id is the number of set bits below it
-  const int nk = T * k;
-  for (int i = threadIdx.x; i < kMaxE / 32; i += kThreads) s_bits[i] = 0u;
-  __syncthreads();
-  if (live && threadIdx.x < nk) {
-    const int id = s_idx[threadIdx.x];
-    if (id >= 0 && id < E) atomicOr(&s_bits[id >> 5], 1u << (id & 31));
-    else s_bad = 1;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t pre = 0;
-#pragma unroll
-    for (int i = 0; i < kMaxE / 32 / 32; ++i) {
-      const uint32_t c = __popc(s_bits[i * 32 + lane]);
-      uint32_t inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      s_bpre[i * 32 + lane] = pre + inc - c;
-      pre += __shfl_sync(0xffffffffu, inc, 31);
-    }
-    if (lane == 0) s_U = int(pre);
-  }
-  __syncthreads();
-  const int U = s_U;
-  if (live && !s_bad && threadIdx.x < nk) {
-    const int id = s_idx[threadIdx.x], w = id >> 5;
-    const int rank = int(s_bpre[w] + __popc(s_bits[w] & ((1u << (id & 31)) - 1u)));
-    s_slot[threadIdx.x] = rank;
-    s_uniq[rank] = id;
-  }
-  __syncthreads();
-  if (live && !s_bad) {
-    constexpr int W = int(sizeof(moe_expert) / 4);
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
-    for (int i = threadIdx.x; i < U * W; i += kThreads) dst[i] = src[size_t(s_uniq[i / W]) * W + (i % W)];
-    if (b == 0) {
-      for (int i = threadIdx.x; i < nk; i += kThreads) {
-        P.topk_idx[i] = s_idx[i];
-        P.topk_w[i] = s_w[i];
-      }
-      if (P.logits_out)
-        for (int i = threadIdx.x; i < T * E; i += kThreads) P.logits_out[i] = lg[i];
+  if (warp >= kWarps - T) route_cta(C, R, has_shared && !s_bad);
+  // every warp waits (bounded by the routing warps' own bounded waits) for
+  // the job list of phases B and C
+  if (lane == 0) {
+    const long long t0 = clock64();
+    while (R.ready == 0) {
+      __nanosleep(64);
+      if (clock64() - t0 > 4 * P.wait_cycles + 1000000) break;  // the routing warps' waits end long before
     }
   }
-  __syncthreads();
-  if (live && !s_bad && threadIdx.x < U)
-    if (!expert_ok(desc[threadIdx.x], H, I)) s_bad = 1;
-  __syncthreads();
-  const bool work = live && !s_bad;
-  if (live && s_bad && threadIdx.x == 0) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 1000000);
-  if (work) {
-    // activations of the routed formats not built yet
-    for (int f = 1; f <= 3; ++f) {
-      bool used = false;
-      for (int u = 0; u < U; ++u) used |= desc[u].gate.qtype == f;
-      if (used && C.fmap[f] < 0) {
-        int nb = 0;
-        for (int g = 1; g <= 3; ++g) nb += C.fmap[g] >= 0;
-        __syncthreads();
-        if (threadIdx.x == 0) C.fmap[f] = nb;
-        build_xf(f, nb);
-        __syncthreads();
-      }
-    }
-    // this CTA's down rows of every picked expert into L2
-    if (C.nr > 0 && threadIdx.x >= 32 && threadIdx.x < 32 + U) {
-      const moe_qmatrix& dm = desc[threadIdx.x - 32].down;
-      const int rb = row_code_bytes(dm.qtype, I);
-      prefetch_l2(dm.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
-    }
-    if (threadIdx.x < U) s_fmt[threadIdx.x] = desc[threadIdx.x].gate.qtype;
-    __syncthreads();
-    if (threadIdx.x == 0)
-      s_nJ = phase_bc_jobs(H, I, G, b, U, s_fmt, has_shared, reinterpret_cast<Job*>(smem + L.o_jobs));
-  }
-  __syncthreads();
+  __syncwarp();
+  __threadfence_block();
+  const bool work = R.ready == 1 && !s_bad;
 
   // ---------------------------------------------------------- phases B, C
   if (work) {
-    const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs);
-    const int nJ = s_nJ;
+    const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs) + kMaxJobs / 2;
+    const int nJ = R.nJ;
     for (int j = warp; j < nJ; j += kWarps) {
       const Job jb = jobs[j];
       if (jb.kind == kGateUp) job_gate_up(C, jb);
@@ -1006,12 +1050,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     for (int i = threadIdx.x; i < T * nr; i += kThreads) {
       const int t = i / nr, r = i - t * nr;
       float a = 0.f;
-      for (int j = 0; j < k; ++j) a = fmaf(s_w[t * k + j], Y[(s_slot[t * k + j] * 16 + r) * T + t], a);
+      for (int j = 0; j < k; ++j) a = fmaf(R.w[t * k + j], Y[(R.slot[t * k + j] * 16 + r) * T + t], a);
       if (has_shared) {
         const float ys = Y[(kSharedSlot * 16 + r) * T + t];
         a = P.shared_gate ? fmaf(1.f / (1.f + expf(-__ldcg(P.sgate + t))), ys, a) : a + ys;
       }
       P.out[size_t(t) * H + n0 + r] = f32_to_bf16_rn(a);
+    }
+    if (b == 0) {
+      for (int i = threadIdx.x; i < T * k; i += kThreads) {
+        P.topk_idx[i] = R.idx[i];
+        P.topk_w[i] = R.w[i];
+      }
+      if (P.logits_out) {
+        const float* lg = reinterpret_cast<const float*>(smem + L.o_lg);
+        for (int i = threadIdx.x; i < T * E; i += kThreads) P.logits_out[i] = lg[i];
+      }
     }
   }
 
@@ -1051,8 +1105,8 @@ bool eligible_on(int T, int H, int I, int E, int k, int G) {
   // job lists: phase A <= router rows x segments + 2 x shared tiles, phase
   // B/C <= 2 x routed tiles + one down job per slot
   const int U = T * k < E ? T * k : E;
-  if ((router_rows(E, G) + 1) * (H / router_seg(H)) + 2 * shared_tiles(I, G, 0) > kMaxJobs) return false;
-  if (2 * ((U * (I / 8) + G - 1) / G) + U + 1 > kMaxJobs) return false;
+  if ((router_rows(E, G) + 1) * (H / router_seg(H)) + 2 * shared_tiles(I, G, 0) > kMaxJobs / 2) return false;
+  if (2 * ((U * (I / 8) + G - 1) / G) + U + 1 > kMaxJobs / 2) return false;
   return make_plan(T, H, I, E, k, G).total + kStaticSmem <= kSmemLimit;
 }
 

@@ -76,6 +76,7 @@ struct Plan {
   int* nrows;   // [max]
   int* hslot;   // [groups] heavy slot or -1
   int* hlist;   // [heavy slots] group of each slot
+  int* tscaled; // [max] nonzero when a row of the tile has its x scaled (set by the gather)
 };
 
 __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   __shared__ int hsum[32];
   const int ngroups = E + (shared_rows > 0 ? 1 : 0);
   const int g = threadIdx.x;
+  for (int i = g; i < max_tiles; i += blockDim.x) plan.tscaled[i] = 0;
   int nt = 0;
   if (g < ngroups) {
     const int n = g < E ? counts[g] : shared_rows;
@@ -159,6 +161,22 @@ __device__ __forceinline__ float sat_f16(float v) { return fminf(fmaxf(v, -65504
 // under 2^(kHShift - 24)).
 constexpr int kHShift = 8;
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // -126 <= e <= 127
+// The exponents of 16 consecutive rows (a 64-byte aligned run); returns
+// whether any is nonzero.
+__device__ __forceinline__ bool row_exps(const int* p, int (&e)[16]) {
+  const int4* q = reinterpret_cast<const int4*>(p);
+  int any = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int4 v = q[i];
+    e[4 * i] = v.x;
+    e[4 * i + 1] = v.y;
+    e[4 * i + 2] = v.z;
+    e[4 * i + 3] = v.w;
+    any |= v.x | v.y | v.z | v.w;
+  }
+  return any != 0;
+}
 __device__ __forceinline__ int row_exp(uint32_t amax_bf16) {  // bf16 magnitude bits
   const int ex = int((amax_bf16 >> 7) & 0xff) - 127;          // floor(log2 |x|) of the largest element
   return ex >= 8 ? (ex - 7 < 119 ? ex - 7 : 119) : 0;
@@ -179,25 +197,55 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   for (long long wr = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); wr < (long long)ntiles * BN;
        wr += (long long)gridDim.x * 8) {
     const int rt = int(wr / BN), row = int(wr % BN);
-    if (row >= plan.nrows[rt]) continue;
+    if (row >= plan.nrows[rt]) {  // padding rows of a partial tile: no scaling
+      if (lane == 0) xexp[size_t(rt) * BN + row] = 0;
+      continue;
+    }
     const int g = plan.group[rt];
     const int r = plan.row0[rt] + row;
     const int tok = g < E ? perm_src[r] / k : r;
     const uint4* src = reinterpret_cast<const uint4*>(x + size_t(tok) * H);
-    // the row's largest |x| (bf16 magnitude bits compare as integers)
+    // the row's largest |x| (bf16 magnitude bits compare as integers); rows
+    // of up to 2048 elements stay in registers for the conversion below
+    constexpr int kRegChunks = 8;
+    const bool in_regs = H / 8 <= 32 * kRegChunks;
+    uint4 keep[kRegChunks];
     uint32_t am = 0;
-    for (int c = lane; c < H / 8; c += 32) {
-      const uint4 v = __ldg(src + c);
-      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) am = max(am, max(in[i] & 0x7fffu, (in[i] >> 16) & 0x7fffu));
+    for (int i = 0; i < kRegChunks; ++i) {
+      const int c = lane + 32 * i;
+      if (in_regs && c < H / 8) {
+        keep[i] = __ldg(src + c);
+        const uint32_t in[4] = {keep[i].x, keep[i].y, keep[i].z, keep[i].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) am = max(am, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
+      }
     }
+    if (!in_regs)
+      for (int c = lane; c < H / 8; c += 32) {
+        const uint4 v = __ldg(src + c);
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) am = max(am, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
+      }
     am = __reduce_max_sync(0xffffffffu, am);
     const int e = row_exp(am);
     const float sc = pow2f(-e);
-    if (lane == 0) xexp[size_t(rt) * BN + row] = e;
+    if (lane == 0) {
+      xexp[size_t(rt) * BN + row] = e;
+      if (e) atomicOr(&plan.tscaled[rt], 1);
+    }
     for (int c = lane; c < H / 8; c += 32) {
-      const uint4 v = __ldg(src + c);
+      uint4 v;
+      if (in_regs) {
+        const int i = (c - lane) / 32;
+        v = keep[0];
+#pragma unroll
+        for (int q = 1; q < kRegChunks; ++q)
+          if (q == i) v = keep[q];
+      } else {
+        v = __ldg(src + c);
+      }
       // bf16 -> fp16 after the row's scaling (|x| < 2^8; inf saturates at
       // +-65504), K order (0,4,1,5,2,6,3,7)
       const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -751,6 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * C::kAccCols);
       const int m = mt * BM + 32 * q + lane;  // weight row of this thread
+      const bool tile_scaled = a.plan.tscaled[rt] != 0;  // any row of the tile has its x scaled
       for (int c0 = 0; c0 < nrows; c0 += 16) {
         uint32_t v0[16];
         ptx::tmem_ld16(taddr + uint32_t(c0), v0);
@@ -766,29 +815,33 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes + size_t(c0) * 128 +
                           (e < 4 ? 4 * e : 4 * (e - 4) + 2);
           const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
-          const int* xe = a.xexp + size_t(rt) * BN + c0;
+          int xe[16] = {};
+          const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             if (j < nv) {
               // the row's x was scaled by 2^-e: g = g_s 2^e, u = u_s 2^e, and
               // h 2^-(kHShift + 2e) = silu(g) 2^-e u_s 2^-kHShift
-              const int e = xe[j];
-              const float gv = __uint_as_float(v0[j]) * pow2f(e), uv = __uint_as_float(v1[j]);
-              const float hs = __fdividef(gv, 1.0f + __expf(-gv)) * pow2f(-e) * uv * (1.0f / (1 << kHShift));
-              *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) = __float2half_rn(sat_f16(hs));
+              float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]) * (1.0f / (1 << kHShift));
+              if (scaled) {
+                gv *= pow2f(xe[j]);
+                uv *= pow2f(-xe[j]);
+              }
+              *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) =
+                  __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
             }
           }
         } else {
           ptx::tmem_ld_wait();
           const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
           // undo the scaling of h: y = y_s 2^(kHShift + 2e) for the row's e
-          const int* xe = a.xexp + size_t(rt) * BN + c0;
+          int xe[16] = {};
+          const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
           float yv[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const int e = j < nv ? xe[j] : 0;
-            const float v = __uint_as_float(v0[j]);
-            yv[j] = e == 0 ? v * float(1 << kHShift) : ldexpf(v, kHShift + 2 * e);
+            const float v = __uint_as_float(v0[j]) * float(1 << kHShift);
+            yv[j] = scaled ? ldexpf(v, 2 * xe[j]) : v;
           }
           if (g < a.E && a.y_f32 == nullptr) {
             uint16_t* yp = a.y_bf16 + size_t(row0 + c0) * a.H + m;
@@ -848,7 +901,7 @@ int grouped_heavy_slots(long long T, int k, bool with_shared, int H, int I) {
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
   const long long mt = grouped_max_tiles(T, k, E, with_shared);
   return align256(16 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
-         align256(4 * size_t(mt) * gemm::BN) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
+         align256(4 * size_t(mt)) + align256(4 * size_t(mt) * gemm::BN) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(grouped_heavy_slots(T, k, with_shared, H, I)) * gemm::heavy_slot_bytes(H, I));
 }
@@ -871,6 +924,8 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   plan.hslot = reinterpret_cast<int*>(p);
   plan.hlist = plan.hslot + (E + 1);
   p += align256(4 * size_t(E + 1) + 4 * size_t(kMaxHeavy));
+  plan.tscaled = reinterpret_cast<int*>(p);
+  p += align256(4 * size_t(mt));
   int* xexp = reinterpret_cast<int*>(p);
   p += align256(4 * size_t(mt) * BN);
   uint8_t* xt = p;

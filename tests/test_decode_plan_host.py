@@ -76,7 +76,7 @@ int main() {
                   int e0, nrr;
                   router_range(E, G, b, e0, nrr);
                   const int na = phase_a_jobs(H, I, E, G, b, fm, gate, jobs.data());
-                  if (na > kMaxJobs) { ++bad_fields; continue; }
+                  if (na > kMaxJobs / 2) { ++bad_fields; continue; }
                   for (int j = 0; j < na; ++j) {
                     const Job& jb = jobs[j];
                     if (jb.kind == kRouter) {
@@ -88,7 +88,7 @@ int main() {
                     }
                   }
                   const int nb = phase_bc_jobs(H, I, G, b, U, fmt.data(), true, jobs.data());
-                  if (nb > kMaxJobs) { ++bad_fields; continue; }
+                  if (nb > kMaxJobs / 2) { ++bad_fields; continue; }
                   int n0, nr;
                   out_rows(H, G, b, n0, nr);
                   if (nr > 16) ++bad_fields;
