@@ -405,6 +405,21 @@ def run_ours(args, rank, world, peaks, peak_kind):
     e2e_ms = float(np.sum(e2e_times))
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
+    # routing heat over the timed steps' tokens (untimed pass): the library's
+    # per-expert hit counters, checked against the steps' own picks
+    heat = torch.zeros(wl.E, dtype=torch.int32, device=dev)
+    for s in range(args.warmup, args.warmup + args.steps):
+        L.layer(xs[s], wl.I, wl.E, wl.k, w_r, b, stride, experts.table, shared.table, idx[s], gw[s], out[s], ws,
+                stream=stream, heat=heat)
+    torch.cuda.synchronize()
+    heat_h = heat.cpu().numpy().astype(np.int64)
+    assert np.array_equal(heat_h, np.bincount(idx[args.warmup:].cpu().numpy().ravel(), minlength=wl.E))
+    order = np.argsort(-heat_h, kind="stable")
+    routing_heat = {"steps": args.steps, "picks": int(heat_h.sum()), "experts_hit": int(np.sum(heat_h > 0)),
+                    "hottest": [[int(e), int(heat_h[e])] for e in order[:8]],
+                    "share_of_hottest_8": float(heat_h[order[:8]].sum() / max(1, heat_h.sum())),
+                    "bytes_of_hottest_8": 8 * float(wlm.per_token_layer_bytes(wl, 1) - wlm.per_token_layer_bytes(wl, 0))}
+
     # algorithmic bytes per step: distinct routed experts + shared + router
     idx_h = idx[args.warmup:].cpu().numpy()
     uniq = np.array([len(np.unique(s)) for s in idx_h.reshape(args.steps, -1)])
@@ -445,6 +460,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
         "gpu_launches": int(launches),
         "clocks": clk,
         "wall_s_timed_region": t_wall,
+        "routing_heat": routing_heat,
     }
     return line, wl, lay, bias
 

@@ -37,7 +37,7 @@ class ExpertC(ctypes.Structure):
 
 
 class OptionsC(ctypes.Structure):
-    _fields_ = [("flags", ctypes.c_uint32), ("shared_gate", c_vp)]
+    _fields_ = [("flags", ctypes.c_uint32), ("shared_gate", c_vp), ("heat", c_vp)]
 
 
 MOE_BIAS_SELECTION_ONLY = 1
@@ -156,13 +156,15 @@ def _shape2(t, name, cols=None):
     return t.shape
 
 
-def _opts(H, bias_selection_only=False, shared_gate=None):
+def _opts(H, bias_selection_only=False, shared_gate=None, heat=None, E=0):
     """The moe_options of a call (None = the defaults: NULL). shared_gate is a
-    device fp32 [H] tensor; the struct is read on the host during the call."""
-    if not bias_selection_only and shared_gate is None:
+    device fp32 [H] tensor, heat a device int32/uint32 [E] counter tensor the
+    call adds its picks to; the struct is read on the host during the call."""
+    if not bias_selection_only and shared_gate is None and heat is None:
         return None
     g = _dev(shared_gate, "shared_gate", "f32", H, optional=True)
-    return ctypes.byref(OptionsC(MOE_BIAS_SELECTION_ONLY if bias_selection_only else 0, g))
+    hp = _dev(heat, "heat", "i32", E, optional=True)
+    return ctypes.byref(OptionsC(MOE_BIAS_SELECTION_ONLY if bias_selection_only else 0, g, hp))
 
 
 def _stream(stream):
@@ -190,14 +192,15 @@ def new_workspace(T, H, I, E, k, device="cuda"):
 
 
 def route(x, w_router, bias, bias_row_stride, k, topk_idx, topk_w, ws, logits=None, stream=None,
-          bias_selection_only=False):
+          bias_selection_only=False, heat=None):
     T, H = _shape2(x, "x")
     E = _shape2(w_router, "w_router", H)[0]
     _check("moe_route", LIB.moe_route(_dev(x, "x", "bf16"), T, H, _dev(w_router, "w_router", "f32"), E,
                                       _bias(bias, T, E, bias_row_stride), bias_row_stride, k,
                                       _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
                                       _dev(logits, "logits", "f32", T * E, optional=True),
-                                      _opts(H, bias_selection_only), _ws(ws), ws.numel(), _stream(stream)))
+                                      _opts(H, bias_selection_only, heat=heat, E=E), _ws(ws), ws.numel(),
+                                      _stream(stream)))
 
 
 def dispatch(topk_idx, E, counts, offsets, perm_src, inv_perm, ws, stream=None):
@@ -231,7 +234,7 @@ def combine(y_perm, inv_perm, topk_w, I, x, shared_table, out, ws, stream=None, 
 
 
 def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx, topk_w, out, ws,
-          stream=None, logits=None, bias_selection_only=False, shared_gate=None):
+          stream=None, logits=None, bias_selection_only=False, shared_gate=None, heat=None):
     T, H = _shape2(x, "x")
     _shape2(w_router, "w_router", H)
     _check("moe_layer", LIB.moe_layer(_dev(x, "x", "bf16"), T, H, I, E, k, _dev(w_router, "w_router", "f32", E * H),
@@ -240,12 +243,14 @@ def layer(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_tab
                                       _table(shared_table, "shared_table", 1, optional=True),
                                       _dev(topk_idx, "topk_idx", "i32", T * k), _dev(topk_w, "topk_w", "f32", T * k),
                                       _dev(logits, "logits", "f32", T * E, optional=True),
-                                      _dev(out, "out", "bf16", T * H), _opts(H, bias_selection_only, shared_gate),
-                                      _ws(ws), ws.numel(), _stream(stream)))
+                                      _dev(out, "out", "bf16", T * H),
+                                      _opts(H, bias_selection_only, shared_gate, heat, E), _ws(ws), ws.numel(),
+                                      _stream(stream)))
 
 
 def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_table, shared_table, topk_idx,
-                         topk_w, out, stream=None, logits=None, bias_selection_only=False, shared_gate=None):
+                         topk_w, out, stream=None, logits=None, bias_selection_only=False, shared_gate=None,
+                         heat=None):
     """moe_layer_decode_noalloc: the fused decode step without a workspace."""
     T, H = _shape2(x, "x")
     _shape2(w_router, "w_router", H)
@@ -257,8 +262,8 @@ def layer_decode_noalloc(x, I, E, k, w_router, bias, bias_row_stride, experts_ta
                                         _dev(topk_idx, "topk_idx", "i32", T * k),
                                         _dev(topk_w, "topk_w", "f32", T * k),
                                         _dev(logits, "logits", "f32", T * E, optional=True),
-                                        _dev(out, "out", "bf16", T * H), _opts(H, bias_selection_only, shared_gate),
-                                        _stream(stream)))
+                                        _dev(out, "out", "bf16", T * H),
+                                        _opts(H, bias_selection_only, shared_gate, heat, E), _stream(stream)))
 
 
 def reset_status(ws, stream=None):

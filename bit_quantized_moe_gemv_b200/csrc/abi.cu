@@ -72,9 +72,12 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t H, const float* w_rou
   const WsLayout L = ws_layout(T, H, 64, E, k);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   float* logits = logits_out ? logits_out : ws_at<float>(ws, L.logits);
-  return cuda_status(launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w, logits,
-                                  ws_at<void>(ws, L.router), ws_at<WsHeader>(ws, 0),
-                                  static_cast<cudaStream_t>(stream), (flags & MOE_BIAS_SELECTION_ONLY) != 0));
+  cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w, logits,
+                               ws_at<void>(ws, L.router), ws_at<WsHeader>(ws, 0), static_cast<cudaStream_t>(stream),
+                               (flags & MOE_BIAS_SELECTION_ONLY) != 0);
+  if (e == cudaSuccess && opts && opts->heat)
+    e = launch_heat(topk_idx, (long long)T * k, E, opts->heat, static_cast<cudaStream_t>(stream));
+  return cuda_status(e);
 }
 
 moe_status moe_dispatch(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E, int32_t* counts, int32_t* offsets,
@@ -170,7 +173,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
                                            topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.logits),
                                            ws_at<float>(ws, L.dh), ws_at<uint32_t>(ws, L.dcnt), hdr,
                                            wait_cycles(), flags, gate, ws_at<float>(ws, L.logits_u),
-                                           ws_at<float>(ws, L.sgate), st));
+                                           ws_at<float>(ws, L.sgate), opts ? opts->heat : nullptr, st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
   int* perm = ws_at<int>(ws, L.perm);
@@ -179,6 +182,7 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
   cudaError_t e = launch_route(x, T, H, w_router, E, bias, bias_row_stride, k, topk_idx, topk_w,
                                logits_out ? logits_out : ws_at<float>(ws, L.logits), ws_at<void>(ws, L.router),
                                hdr, st, (flags & MOE_BIAS_SELECTION_ONLY) != 0);
+  if (e == cudaSuccess && opts && opts->heat) e = launch_heat(topk_idx, (long long)T * k, E, opts->heat, st);
   float* shared_scale = nullptr;
   if (e == cudaSuccess && shared_dev && gate) {
     shared_scale = ws_at<float>(ws, L.sgate);

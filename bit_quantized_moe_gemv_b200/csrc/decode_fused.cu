@@ -56,6 +56,8 @@ constexpr int kMaxSlots = kMaxT * kMaxK + 1;  // routed slots + the shared exper
 constexpr int kMaxJobs = 1280;  // two lists of kMaxJobs / 2: phase A, then phases B and C
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kTopChunk = 128;  // logits per first-round top-k job (4 per lane)
+constexpr int kMaxH = 2048;     // largest hidden size of the fused kernel
+constexpr int kMaxBias = 64;    // router bias values of one CTA's rows (rows x tokens)
 
 enum : uint8_t { kRouter = 0, kGateUp = 1, kDown = 2 };
 
@@ -70,6 +72,10 @@ struct Job {
 };
 static_assert(sizeof(Job) == 8, "job record");
 constexpr int kSharedSlot = kMaxSlots - 1;
+// Counters of an expert slot, each slot on a 128-byte line of its own (so
+// the warps polling one expert do not contend with another's): word 0 =
+// finished gate/up tiles, words 1..kMaxT = bits of the largest |h| per token.
+constexpr int kCntStride = 32;
 
 // ---------------------------------------------------------------- formats
 // A 16-byte column of codes holds kc(F) weights of one row; its activations
@@ -231,13 +237,13 @@ struct Params {
   WsHeader* hdr;
   float* logits;   // [T][E] workspace
   float* h;        // [kMaxSlots][T][I] workspace
-  uint32_t* cnt;   // [kMaxSlots] finished gate/up tiles per slot
-  uint32_t* amax;  // [kMaxSlots][kMaxT] bits of max |h| per slot and token
+  uint32_t* cnt;   // [kMaxSlots][kCntStride]: finished tiles, then max |h| bits per token
   long long wait_cycles;
   uint32_t flags;            // MOE_BIAS_SELECTION_ONLY
   const float* shared_gate;  // fp32 [H] or null: sigmoid-gated shared expert
   float* logits_u;           // [T][E] unbiased logits (selection-only bias)
   float* sgate;              // [T] shared_gate . x
+  uint32_t* heat;            // [E] routing heat, or null
 };
 
 // ---------------------------------------------------------------- PTX bits
@@ -298,6 +304,9 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 }
 __device__ __forceinline__ void red_release(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
@@ -519,7 +528,7 @@ __device__ bool wait_counter(const uint32_t* p, uint32_t target, WsHeader* hdr, 
     }
     if (ld_acquire(p) >= target) return true;
     if ((it & 15) == 0 && *reinterpret_cast<volatile int*>(&hdr->abort)) return false;
-    __nanosleep(32);
+    __nanosleep(it < 8 ? 32 : 256);  // back off: many warps may poll, and the counter's writers need its line
   }
 }
 
@@ -535,6 +544,7 @@ struct Ctx {
   int n0, nr;               // output rows of this CTA
   int fmap[4];              // weight format -> activation buffer (or -1)
   int xexp[kMaxT];          // power-of-two scaling of x per token
+  float bias[kMaxBias];     // router bias of this CTA's rows, [row][token]
   int fail;                 // a wait of this CTA gave up
   int rdone;                // router jobs finished
   moe_expert* desc;         // descriptors: slots 0..U-1, kSharedSlot
@@ -592,7 +602,7 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
     }
   }
   float* hs = P.h + size_t(slot) * T * I;
-  uint32_t* am = P.amax + slot * kMaxT;
+  uint32_t* am = P.cnt + slot * kCntStride + 1;
   float gsc = 1.f, usc = 1.f;
   if (f == MOE_Q_INT8_PER_CHANNEL) {
     gsc = f16_to_f32(d.gate.scales[row]);
@@ -614,9 +624,9 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
     for (int o = 4; o < 32; o <<= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
     if (gq == 0 && t < T) atomicMax(am + t, a);
   }
-  __threadfence();
+  // the warp barrier orders every lane's stores before lane 0's release
   __syncwarp();
-  if (lane == 0) red_release(P.cnt + slot, 1u);
+  if (lane == 0) red_release(P.cnt + slot * kCntStride, 1u);
 }
 
 // down job: this CTA's output rows [n0, n0 + nr) of one expert (already on
@@ -646,24 +656,34 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   uint8_t* hf = C.smem + C.L.o_hf + warp * 2 * T * I;
   __shared__ int s_eh[kWarps][kMaxT];
   int ok = 1;
-  if (lane == 0) ok = wait_counter(P.cnt + slot, uint32_t(I / 8), P.hdr, P.wait_cycles, 7100000 + slot) ? 1 : 0;
+  if (lane == 0)
+    ok = wait_counter(P.cnt + slot * kCntStride, uint32_t(I / 8), P.hdr, P.wait_cycles, 7100000 + slot) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok) {
     if (lane == 0) C.fail = 1;
     return;
   }
-  (void)ld_acquire(P.cnt + slot);  // every lane orders its reads of h after the counter
-  if (lane < T) s_eh[warp][lane] = range_exp(__ldcg(P.amax + slot * kMaxT + lane));
+  (void)ld_acquire(P.cnt + slot * kCntStride);  // every lane orders its reads of h after the counter
+  if (lane < T) s_eh[warp][lane] = range_exp(__ldcg(P.cnt + slot * kCntStride + 1 + lane));
   __syncwarp();
-  const float* hs = P.h + size_t(slot) * T * I;
-  for (int i = 4 * lane; i < T * I; i += 128) {  // I % 4 == 0: four values of one token
-    const int t = i / I, kk = i - t * I;
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(hs + i));
-    const int e = s_eh[warp][t];
-    *reinterpret_cast<__half*>(hf + frag_pos(f, kk, t, T)) = __float2half_rn(ldexpf(v.x, -e));
-    *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 1, t, T)) = __float2half_rn(ldexpf(v.y, -e));
-    *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 2, t, T)) = __float2half_rn(ldexpf(v.z, -e));
-    *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 3, t, T)) = __float2half_rn(ldexpf(v.w, -e));
+  const float4* hs = reinterpret_cast<const float4*>(P.h + size_t(slot) * T * I);
+  const int n4 = T * I / 4;  // I % 4 == 0: each float4 holds four values of one token
+  for (int base = lane; base < n4; base += 8 * 32) {
+    float4 v[8];  // 8 loads per lane in flight at a time
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = base + 32 * j < n4 ? __ldcg(hs + base + 32 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = 4 * (base + 32 * j);
+      if (i < T * I) {
+        const int t = i / I, kk = i - t * I;
+        const int e = s_eh[warp][t];
+        *reinterpret_cast<__half*>(hf + frag_pos(f, kk, t, T)) = __float2half_rn(ldexpf(v[j].x, -e));
+        *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 1, t, T)) = __float2half_rn(ldexpf(v[j].y, -e));
+        *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 2, t, T)) = __float2half_rn(ldexpf(v[j].z, -e));
+        *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 3, t, T)) = __float2half_rn(ldexpf(v[j].w, -e));
+      }
+    }
   }
   __syncwarp();
   float acc[4];
@@ -739,11 +759,11 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb, const uint4 w0, co
       __stcg(P.sgate + t, a);
       continue;
     }
-    const float bv = P.bias ? P.bias[t * P.bstride + C.e0 + r] : 0.f;
+    const float bv = C.bias[r * T + t];
     __stcg(P.logits + size_t(t) * E + C.e0 + r, a + bv);
     if (P.flags & MOE_BIAS_SELECTION_ONLY) __stcg(P.logits_u + size_t(t) * E + C.e0 + r, a);
   }
-  __threadfence();
+  // the warp barrier orders every lane's stores before lane 0's release
   __syncwarp();
   if (lane == 0) red_release(&P.hdr->bar_count, 1u);
 }
@@ -780,8 +800,18 @@ __device__ __noinline__ void route_cta(Ctx& C, RouteShared& R, bool has_shared) 
   rsync();
   const bool live = !C.fail;
   float* lg = reinterpret_cast<float*>(C.smem + C.L.o_lg);
-  if (live)
-    for (int i = threadIdx.x - (kWarps - T) * 32; i < T * E; i += nthr) lg[i] = __ldcg(P.logits + i);
+  if (live) {
+    // 16 loads per thread in flight at a time
+    const int r0 = threadIdx.x - (kWarps - T) * 32;
+    for (int base = r0; base < T * E; base += 16 * nthr) {
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = base + j * nthr < T * E ? __ldcg(P.logits + base + j * nthr) : 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (base + j * nthr < T * E) lg[base + j * nthr] = v[j];
+    }
+  }
   for (int i = threadIdx.x - (kWarps - T) * 32; i < kMaxE / 32; i += nthr) R.bits[i] = 0u;
   rsync();
   // this token's top-k in two rounds: its 128-logit chunks, then their winners
@@ -855,9 +885,21 @@ __device__ __noinline__ void route_cta(Ctx& C, RouteShared& R, bool has_shared) 
     moe_expert* desc = C.desc;
     constexpr int W = int(sizeof(moe_expert) / 4);
     if (live && !R.bad) {
+      // 8 loads per lane in flight at a time (the table is on its way into L2
+      // since the kernel's entry)
       const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
       uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
-      for (int i = lane; i < U * W; i += 32) dst[i] = src[size_t(R.uniq[i / W]) * W + (i % W)];
+      for (int base = lane; base < U * W; base += 8 * 32) {
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int i = base + 32 * j;
+          v[j] = i < U * W ? src[size_t(R.uniq[i / W]) * W + (i % W)] : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (base + 32 * j < U * W) dst[base + 32 * j] = v[j];
+      }
     }
     __syncwarp();
     bool bad = R.bad != 0;
@@ -914,6 +956,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   uint4 w0[4] = {};
   const bool early = warp < nrr * nseg;
   if (early) router_load(P, e0, nreal, seg, Job{kRouter, uint8_t(warp / nseg), 0, uint8_t(warp % nseg), 0, 0}, w0);
+  // then everything else the prologue reads, all in flight together: x (this
+  // thread's 8-element groups), the bias of this CTA's router rows and the
+  // shared expert's descriptor; the expert table goes into L2 for the routing
+  constexpr int kXg = kMaxT * kMaxH / 8 / kThreads;
+  const int ng = T * H / 8;
+  uint4 xg[kXg];
+#pragma unroll
+  for (int j = 0; j < kXg; ++j) {
+    const int g = threadIdx.x + j * kThreads;
+    xg[j] = g < ng ? ldg16(P.x + size_t(g) * 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float bias_v = 0.f;
+  if (P.bias && threadIdx.x < nreal * T) {
+    const int r = threadIdx.x / T, t = threadIdx.x - r * T;
+    bias_v = P.bias[t * P.bstride + e0 + r];
+  }
+  constexpr int kDescWords = int(sizeof(moe_expert) / 4);
+  uint32_t sdesc_v = 0u;
+  if (has_shared && threadIdx.x < kDescWords) sdesc_v = reinterpret_cast<const uint32_t*>(P.shared)[threadIdx.x];
+  {
+    const size_t tbytes = size_t(E) * sizeof(moe_expert);
+    const size_t l = size_t(b) * kThreads + threadIdx.x;
+    const char* tb = reinterpret_cast<const char*>(P.experts);
+    if (l * 128 < tbytes) prefetch_line_l2(tb + l * 128);
+    if (l == 0) prefetch_line_l2(tb + tbytes - 1);
+  }
 
   // ---------------------------------------------------------- prologue
   moe_expert* desc = reinterpret_cast<moe_expert*>(smem + make_plan(T, H, I, E, k, G).o_desc);
@@ -938,10 +1006,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     R.U = 0;
   }
   if (threadIdx.x < kMaxT) s_xamax[threadIdx.x] = 0u;
-  if (has_shared && threadIdx.x < int(sizeof(moe_expert) / 4))
-    reinterpret_cast<uint32_t*>(desc + kSharedSlot)[threadIdx.x] =
-        reinterpret_cast<const uint32_t*>(P.shared)[threadIdx.x];
   __syncthreads();
+  if (has_shared && threadIdx.x < kDescWords) reinterpret_cast<uint32_t*>(desc + kSharedSlot)[threadIdx.x] = sdesc_v;
+  if (threadIdx.x < kMaxBias) C.bias[threadIdx.x] = bias_v;  // zero beyond the CTA's rows
   const Plan& L = C.L;
   const int ntl = max_tiles(T, I, E, k, G);
   {
@@ -955,13 +1022,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   // x in fp32 (router) and the largest |x| per token
   {
     float* x32 = reinterpret_cast<float*>(smem + L.o_x32);
-    for (int i = threadIdx.x; i < T * H; i += kThreads) {
-      const float v = bf16_to_f32(P.x[i]);
-      x32[i] = v;
-      // a warp's 32 consecutive elements belong to one token (H % 32 == 0)
-      // and are all in range together (T H % 32 == 0)
-      const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v)));
-      if (lane == 0) atomicMax(&s_xamax[i / H], m);
+#pragma unroll
+    for (int j = 0; j < kXg; ++j) {
+      const int g = threadIdx.x + j * kThreads;
+      // a warp's 32 groups (256 elements) belong to one token (H % 256 == 0)
+      // and are all in range together (T H % 256 == 0)
+      if (g < ng) {
+        const uint32_t wv[4] = {xg[j].x, xg[j].y, xg[j].z, xg[j].w};
+        float v[8];
+        uint32_t m = 0u;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[e] = bf16_to_f32(uint16_t(e & 1 ? wv[e >> 1] >> 16 : wv[e >> 1] & 0xffffu));
+          m = max(m, __float_as_uint(fabsf(v[e])));
+        }
+        reinterpret_cast<float4*>(x32)[2 * g] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(x32)[2 * g + 1] = make_float4(v[4], v[5], v[6], v[7]);
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) atomicMax(&s_xamax[g * 8 / H], m);
+      }
     }
   }
   __syncthreads();
@@ -987,10 +1066,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   // activations in fragment order for all three formats (from global x: x32
   // is reused after phase A), so routed experts of any format need no
   // further barrier
-  for (int i = threadIdx.x; i < T * H; i += kThreads) {
-    const int t = i / H, kk = i - t * H;
-    const __half v = __float2half_rn(ldexpf(bf16_to_f32(P.x[i]), -C.xexp[t]));
-    for (int f = 1; f <= 3; ++f) *reinterpret_cast<__half*>(smem + L.o_xf + (f - 1) * 2 * T * H + frag_pos(f, kk, t, T)) = v;
+#pragma unroll
+  for (int j = 0; j < kXg; ++j) {
+    const int g = threadIdx.x + j * kThreads;
+    if (g < ng) {
+      const int t = g * 8 / H, k0 = g * 8 - t * H, ex = -C.xexp[t];
+      const uint32_t wv[4] = {xg[j].x, xg[j].y, xg[j].z, xg[j].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const __half v = __float2half_rn(ldexpf(bf16_to_f32(uint16_t(e & 1 ? wv[e >> 1] >> 16 : wv[e >> 1] & 0xffffu)), ex));
+        for (int f = 1; f <= 3; ++f)
+          *reinterpret_cast<__half*>(smem + L.o_xf + (f - 1) * 2 * T * H + frag_pos(f, k0 + e, t, T)) = v;
+      }
+    }
   }
   if (nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
   __syncthreads();
@@ -1061,6 +1149,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       for (int i = threadIdx.x; i < T * k; i += kThreads) {
         P.topk_idx[i] = R.idx[i];
         P.topk_w[i] = R.w[i];
+        if (P.heat) atomicAdd(P.heat + R.idx[i], 1u);
       }
       if (P.logits_out) {
         const float* lg = reinterpret_cast<const float*>(smem + L.o_lg);
@@ -1077,8 +1166,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     const uint32_t prev = atomicAdd(&hdr->exit_count, 1u);
     if (prev == uint32_t(G) - 1) {
       __threadfence();
-      for (int i = 0; i < kMaxSlots; ++i) P.cnt[i] = 0u;
-      for (int i = 0; i < kMaxSlots * kMaxT; ++i) P.amax[i] = 0u;
+      for (int i = 0; i < kMaxSlots; ++i)
+        for (int j = 0; j <= kMaxT; ++j) P.cnt[i * kCntStride + j] = 0u;
       hdr->bar_count = 0;
       hdr->abort = 0;
       hdr->exit_count = 0;
@@ -1100,7 +1189,8 @@ int grid_size() {
 // Whether the shape runs as one fused launch on a grid of G CTAs.
 bool eligible_on(int T, int H, int I, int E, int k, int G) {
   if (T < 1 || T > kMaxT || k < 1 || k > kMaxK || E < k || E > kMaxE) return false;
-  if (H < 256 || I < 256 || H > 2048 || I > 2048 || (H % 256) || (I % 256)) return false;
+  if (H < 256 || I < 256 || H > kMaxH || I > 2048 || (H % 256) || (I % 256)) return false;
+  if (router_rows(E, G) * T > kMaxBias) return false;
   if ((H + G - 1) / G > 16) return false;             // output rows per CTA fit one 16-row tile
   // job lists: phase A <= router rows x segments + 2 x shared tiles, phase
   // B/C <= 2 x routed tiles + one down job per slot
@@ -1125,7 +1215,7 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
                                 long long wait_cycles, uint32_t flags, const float* shared_gate, float* logits_u_ws,
-                                float* sgate_ws, cudaStream_t st) {
+                                float* sgate_ws, uint32_t* heat, cudaStream_t st) {
   using namespace dfx;
   const int grid = grid_size();
   const size_t smem = size_t(make_plan(T, H, I, E, k, grid).total);
@@ -1143,8 +1233,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
   }
   Params P{x,      T,       H,        I,      E,   k,        w_router,           bias,
            bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
-           logits_ws, h_ws, counters, counters + kMaxSlots, wait_cycles, flags, shared_gate, logits_u_ws,
-           sgate_ws};
+           logits_ws, h_ws, counters, wait_cycles, flags, shared_gate, logits_u_ws,
+           sgate_ws, heat};
   void* args[] = {&P};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(decode_fused_kernel), dim3(grid), dim3(kThreads), args,
                                   smem, st);

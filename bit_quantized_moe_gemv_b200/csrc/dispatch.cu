@@ -199,6 +199,24 @@ int dispatch_blocks(long long n) {
   return int(b > kDispatchMaxBlocks ? kDispatchMaxBlocks : b);
 }
 
+// Routing heat: heat[e] += number of picks of expert e (integer atomics, so
+// the counts are exact and independent of order).
+__global__ void __launch_bounds__(256) heat_kernel(const int* __restrict__ ids, long long n, int E,
+                                                   uint32_t* __restrict__ heat) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const int e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(heat + e, 1u);
+  }
+}
+
+cudaError_t launch_heat(const int* topk_idx, long long n, int E, uint32_t* heat, cudaStream_t st) {
+  if (n == 0 || heat == nullptr) return cudaSuccess;
+  const long long blocks = (n + 255) / 256;
+  heat_kernel<<<unsigned(blocks < 1024 ? blocks : 1024), 256, 0, st>>>(topk_idx, n, E, heat);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dispatch(const int* topk_idx, int T, int k, int E, int* counts, int* offsets, int* perm_src,
                             int* inv_perm, int* hist, WsHeader* hdr, cudaStream_t st) {
   const long long n = (long long)T * k;

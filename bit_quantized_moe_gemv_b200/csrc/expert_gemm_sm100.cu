@@ -187,6 +187,32 @@ __device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
 }
 
 // ---------------------------------------------------------------- gather
+__device__ __forceinline__ uint32_t bf16x8_absmax(const uint4& v) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) m = max(m, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
+  return m;
+}
+// Eight bf16 values (16-byte chunk c of the row) -> fp16 after scaling by
+// sc (|x sc| < 2^8; inf saturates at +-65504), K order (0,4,1,5,2,6,3,7),
+// into the row's place in its swizzled 16 KiB tile.
+__device__ __forceinline__ void store_x8(uint8_t* dst_row, int c, int row, const uint4& v, float sc) {
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  float f[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = sat_f16(__uint_as_float(in[i] << 16) * sc);
+    f[2 * i + 1] = sat_f16(__uint_as_float(in[i] & 0xffff0000u) * sc);
+  }
+  uint4 o;
+  o.x = h2_bits(f[0], f[4]);
+  o.y = h2_bits(f[1], f[5]);
+  o.z = h2_bits(f[2], f[6]);
+  o.w = h2_bits(f[3], f[7]);
+  const int kb = c >> 3, chunk = c & 7;
+  *reinterpret_cast<uint4*>(dst_row + size_t(kb) * kTileBytes + ((chunk ^ (row & 7)) << 4)) = o;
+}
 // One warp per tile row: token row -> 16 KiB swizzled tiles of X (K = H).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x, int H, int k,
                                                           const int* __restrict__ perm_src, int E, Plan plan,
@@ -205,64 +231,41 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     const int r = plan.row0[rt] + row;
     const int tok = g < E ? perm_src[r] / k : r;
     const uint4* src = reinterpret_cast<const uint4*>(x + size_t(tok) * H);
+    uint8_t* dst_row = xt + size_t(rt) * KB * kTileBytes + size_t(row) * 128;
     // the row's largest |x| (bf16 magnitude bits compare as integers); rows
-    // of up to 2048 elements stay in registers for the conversion below
+    // of up to 2048 elements stay in registers for the conversion
     constexpr int kRegChunks = 8;
-    const bool in_regs = H / 8 <= 32 * kRegChunks;
     uint4 keep[kRegChunks];
     uint32_t am = 0;
+    if (H / 8 <= 32 * kRegChunks) {
 #pragma unroll
-    for (int i = 0; i < kRegChunks; ++i) {
-      const int c = lane + 32 * i;
-      if (in_regs && c < H / 8) {
-        keep[i] = __ldg(src + c);
-        const uint32_t in[4] = {keep[i].x, keep[i].y, keep[i].z, keep[i].w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) am = max(am, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
+      for (int i = 0; i < kRegChunks; ++i) {
+        const int c = lane + 32 * i;
+        keep[i] = c < H / 8 ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        am = max(am, bf16x8_absmax(keep[i]));
       }
-    }
-    if (!in_regs)
-      for (int c = lane; c < H / 8; c += 32) {
-        const uint4 v = __ldg(src + c);
-        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) am = max(am, max(in[q] & 0x7fffu, (in[q] >> 16) & 0x7fffu));
+      am = __reduce_max_sync(0xffffffffu, am);
+      const int e = row_exp(am);
+      if (lane == 0) {
+        xexp[size_t(rt) * BN + row] = e;
+        if (e) atomicOr(&plan.tscaled[rt], 1);
       }
-    am = __reduce_max_sync(0xffffffffu, am);
-    const int e = row_exp(am);
-    const float sc = pow2f(-e);
-    if (lane == 0) {
-      xexp[size_t(rt) * BN + row] = e;
-      if (e) atomicOr(&plan.tscaled[rt], 1);
-    }
-    for (int c = lane; c < H / 8; c += 32) {
-      uint4 v;
-      if (in_regs) {
-        const int i = (c - lane) / 32;
-        v = keep[0];
+      const float sc = pow2f(-e);
 #pragma unroll
-        for (int q = 1; q < kRegChunks; ++q)
-          if (q == i) v = keep[q];
-      } else {
-        v = __ldg(src + c);
+      for (int i = 0; i < kRegChunks; ++i) {
+        const int c = lane + 32 * i;
+        if (c < H / 8) store_x8(dst_row, c, row, keep[i], sc);
       }
-      // bf16 -> fp16 after the row's scaling (|x| < 2^8; inf saturates at
-      // +-65504), K order (0,4,1,5,2,6,3,7)
-      const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-      float f[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        f[2 * i] = sat_f16(__uint_as_float(in[i] << 16) * sc);
-        f[2 * i + 1] = sat_f16(__uint_as_float(in[i] & 0xffff0000u) * sc);
+    } else {
+      for (int c = lane; c < H / 8; c += 32) am = max(am, bf16x8_absmax(__ldg(src + c)));
+      am = __reduce_max_sync(0xffffffffu, am);
+      const int e = row_exp(am);
+      if (lane == 0) {
+        xexp[size_t(rt) * BN + row] = e;
+        if (e) atomicOr(&plan.tscaled[rt], 1);
       }
-      uint4 o;
-      o.x = h2_bits(f[0], f[4]);
-      o.y = h2_bits(f[1], f[5]);
-      o.z = h2_bits(f[2], f[6]);
-      o.w = h2_bits(f[3], f[7]);
-      const int kb = c >> 3, chunk = c & 7;
-      uint8_t* dst = xt + (size_t(rt) * KB + kb) * kTileBytes + size_t(row) * 128 + ((chunk ^ (row & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = o;
+      const float sc = pow2f(-e);
+      for (int c = lane; c < H / 8; c += 32) store_x8(dst_row, c, row, __ldg(src + c), sc);
     }
   }
 }
@@ -838,10 +841,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           int xe[16] = {};
           const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
           float yv[16];
+          if (!scaled) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float v = __uint_as_float(v0[j]) * float(1 << kHShift);
-            yv[j] = scaled ? ldexpf(v, 2 * xe[j]) : v;
+            for (int j = 0; j < 16; ++j) yv[j] = __uint_as_float(v0[j]) * float(1 << kHShift);
+          } else {  // 2^(kHShift + 2e) = 2^(kHShift + e) 2^e, each a normal float for e <= 119
+#pragma unroll
+            for (int j = 0; j < 16; ++j) yv[j] = __uint_as_float(v0[j]) * pow2f(kHShift + xe[j]) * pow2f(xe[j]);
           }
           if (g < a.E && a.y_f32 == nullptr) {
             uint16_t* yp = a.y_bf16 + size_t(row0 + c0) * a.H + m;

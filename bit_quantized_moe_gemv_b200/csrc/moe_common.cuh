@@ -30,7 +30,7 @@ static_assert(sizeof(WsHeader) <= 256, "header must fit in 256 bytes");
 // largest |h| per expert slot and token), right after the header. They must
 // be zero when a launch starts; the launch leaves them zero again, and
 // moe_reset_status clears them with the header.
-constexpr size_t kDecodeCounterBytes = 2048;
+constexpr size_t kDecodeCounterBytes = 8448;  // 65 expert slots x 128 bytes, rounded to 256
 constexpr size_t kWsResetBytes = 256 + kDecodeCounterBytes;
 
 // Offsets (bytes from the workspace base) of every workspace segment.

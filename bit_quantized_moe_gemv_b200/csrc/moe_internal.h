@@ -26,6 +26,9 @@ size_t router_tc_ws_bytes(long long T, int H, int E);
 cudaError_t launch_router_tc(const uint16_t* x, int T, int H, const float* W, int E, const float* bias,
                              long long bstride, float* logits, void* scratch, WsHeader* hdr, cudaStream_t st);
 
+// heat[e] += picks of expert e among the n ids (routing heat statistics).
+cudaError_t launch_heat(const int* topk_idx, long long n, int E, uint32_t* heat, cudaStream_t st);
+
 // Blocks the multi-block dispatch uses for n = T*k pairs (1 = single-CTA path).
 int dispatch_blocks(long long n);
 
@@ -62,7 +65,7 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
                                 long long wait_cycles, uint32_t flags, const float* shared_gate, float* logits_u_ws,
-                                float* sgate_ws, cudaStream_t st);
+                                float* sgate_ws, uint32_t* heat, cudaStream_t st);
 constexpr long long kDefaultWaitCycles = 2000000000LL;  // about 1 s at the B200's clock
 // The budget (SM clock cycles) every bounded wait of the fused decode launch
 // gets: kDefaultWaitCycles unless moe_set_wait_cycles changed it.

@@ -101,12 +101,23 @@ typedef struct moe_expert {
  *                           over the picks (logits_out keeps the biased ones);
  *  shared_gate              DEVICE fp32 [H] g, or NULL: the shared expert's
  *                           output is scaled by sigmoid(g . x) per token.
+ * and one statistic:
+ *  heat                     DEVICE uint32 [E], or NULL: routing heat, the
+ *                           number of times each expert was picked; every
+ *                           call that routes (moe_route, moe_layer, the
+ *                           no-alloc call) adds its T k picks, so counts
+ *                           accumulate over calls until the caller clears
+ *                           them (the on-GPU counterpart of the heat ranking
+ *                           the cycleuser.org page, section
+ *                           "硬件形态决定了各自的走法", keeps for its expert
+ *                           cache).
  * The struct itself is read on the host during the call.
  */
 #define MOE_BIAS_SELECTION_ONLY 1u
 typedef struct moe_options {
   uint32_t flags;
   const float* shared_gate;
+  uint32_t* heat;
 } moe_options;
 
 /* Bytes of workspace the calls below need for a problem of this size (the
