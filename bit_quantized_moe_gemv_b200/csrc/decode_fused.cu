@@ -53,10 +53,10 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxT = 4;
 constexpr int kMaxK = 16;
 constexpr int kMaxSlots = kMaxT * kMaxK + 1;  // routed slots + the shared expert
-constexpr int kMaxJobs = 1280;  // two lists of kMaxJobs / 2: phase A, then phases B and C
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kTopChunk = 128;  // logits per first-round top-k job (4 per lane)
 constexpr int kMaxH = 2048;     // largest hidden size of the fused kernel
+constexpr int kMaxI = 2048;     // largest expert intermediate size
 constexpr int kMaxBias = 64;    // router bias values of one CTA's rows (rows x tokens)
 
 enum : uint8_t { kRouter = 0, kGateUp = 1, kDown = 2 };
@@ -110,9 +110,19 @@ __host__ __device__ inline int frag_pos(int F, int k, int t, int T) {
   return (c * T + t) * colbytes(F) + j * wbytes(F) + pos * 2;
 }
 
-// K splits of a gate/up tile: two halves when each half is a whole number of
-// iterations (4 columns), else one.
-__host__ __device__ inline int gu_split(int F, int H) { return (H / 2) % (4 * kc(F)) == 0 ? 2 : 1; }
+// Byte offsets of activations k0 .. k0 + 3 (k0 % 4 == 0) of one token within
+// its fragment-order word: frag_pos(F, k0, t, T) + quad_off<F>(i). int4 and
+// int2 put four consecutive k in every other fp16 slot, int8 in slots
+// 0, 2, 1, 3.
+template <int F>
+__host__ __device__ constexpr int quad_off(int i) {
+  return F == MOE_Q_INT8_PER_CHANNEL ? 2 * ((i & 1) * 2 + (i >> 1)) : 4 * i;
+}
+
+// K parts of a gate/up tile, the same for every format: two halves when each
+// half is a whole number of iterations (4 columns of 16 bytes) in every
+// format (H % 512 == 0), else one.
+__host__ __device__ inline int gu_parts(int H) { return H % 512 == 0 ? 2 : 1; }
 
 // ---------------------------------------------------------------- plan
 // Dynamic shared memory, offsets from the base.
@@ -125,7 +135,6 @@ struct Plan {
   int o_red;   // gate/up K-split sums [tiles][16][T]
   int o_td;    // gate/up K-split arrivals [tiles]
   int o_y;     // down results [kMaxSlots][16][T]
-  int o_jobs;  // job list
   int o_desc;  // expert descriptors of the picked slots and the shared one
   int total;
 };
@@ -133,7 +142,7 @@ __host__ __device__ inline int router_rows(int E, int G) { return (E + G - 1) / 
 __host__ __device__ inline int router_seg(int H) { return H % 512 == 0 ? 512 : 256; }
 __host__ __device__ inline int max_tiles(int T, int I, int E, int k, int G) {
   const int U = T * k < E ? T * k : E;
-  return (U * (I / 8) + G - 1) / G + (I / 8 + G - 1) / G;  // routed + shared
+  return ((U + 1) * (I / 8) + G - 1) / G;  // routed experts and the shared one
 }
 __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int G) {
   Plan p{};
@@ -153,7 +162,6 @@ __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int
   p.o_red = take(4 * max_tiles(T, I, E, k, G) * 16 * T, 16);
   p.o_td = take(4 * max_tiles(T, I, E, k, G), 16);
   p.o_y = take(4 * kMaxSlots * 16 * T, 16);
-  p.o_jobs = take(int(sizeof(Job)) * kMaxJobs, 16);
   p.o_desc = take(int(sizeof(moe_expert)) * kMaxSlots, 16);
   p.total = o;
   return p;
@@ -171,8 +179,12 @@ __host__ __device__ inline void router_range(int E, int G, int b, int& e0, int& 
   e0 = b * rr < E ? b * rr : E;
   n = (e0 + rr < E ? e0 + rr : E) - e0;
 }
-// Local tiles of the shared expert on CTA b (tiles i = b, b + G, ... < I / 8).
-__host__ __device__ inline int shared_tiles(int I, int G, int b) { return I / 8 > b ? (I / 8 - 1 - b) / G + 1 : 0; }
+// Gate/up tiles of CTA b in phases B and C: tiles g = b, b + G, ... of the
+// step's expert-major list of `ne` experts (I / 8 tiles each).
+__host__ __device__ inline int bc_tiles(int I, int G, int b, int ne) {
+  const int J = ne * (I / 8);
+  return J > b ? (J - 1 - b) / G + 1 : 0;
+}
 
 // Router rows of CTA b, plus one for the shared expert's gate vector on the
 // last CTA when the gated variant is on (its local row index is the last).
@@ -182,47 +194,44 @@ __host__ __device__ inline int router_rows_of(int E, int G, int b, bool gate_row
   return n + (gate_row && b == G - 1 ? 1 : 0);
 }
 
-// Phase-A jobs of CTA b: router (row, segment), then the shared expert's
-// gate/up tiles in K parts (shared_fmt 0 = no shared expert). Returns the count.
-__host__ __device__ inline int phase_a_jobs(int H, int I, int E, int G, int b, int shared_fmt, bool gate_row,
-                                            Job* jobs) {
-  const int nrr = router_rows_of(E, G, b, gate_row);
-  const int nseg = H / router_seg(H);
-  int n = 0;
-  for (int r = 0; r < nrr; ++r)
-    for (int s = 0; s < nseg; ++s) jobs[n++] = Job{kRouter, uint8_t(r), 0, uint8_t(s), 0, 0};
-  if (shared_fmt) {
-    const int ns = gu_split(shared_fmt, H);
-    int lt = 0;
-    for (int i = b; i < I / 8; i += G, ++lt)
-      for (int p = 0; p < ns; ++p)
-        jobs[n++] = Job{kGateUp, uint8_t(kSharedSlot), 16, uint8_t(p), uint16_t(8 * i), uint16_t(lt)};
-  }
-  return n;
+// Jobs are numbered per CTA and computed from their number (no lists):
+// warp w takes jobs w, w + 16, ...
+//
+// Phase A of CTA b: router parts (local row j / nseg, segment j % nseg).
+__host__ __device__ inline int phase_a_count(int H, int E, int G, int b, bool gate_row) {
+  return router_rows_of(E, G, b, gate_row) * (H / router_seg(H));
 }
-// Phase-B/C jobs of CTA b: gate/up tiles g = b, b + G, ... of the step's
-// expert-major list of U experts (fmt[u] their formats) in K parts; then one
-// down job per expert for this CTA's output rows, the shared one first.
-// Local tile indices continue after the shared expert's.
-__host__ __device__ inline int phase_bc_jobs(int H, int I, int G, int b, int U, const int* fmt, bool with_shared,
-                                             Job* jobs) {
-  int n = 0, lt = shared_tiles(I, G, b);
-  const int J = U * (I / 8);
-  for (int g = b; g < J; g += G, ++lt) {
-    const int u = g / (I / 8), i = g - u * (I / 8);
-    const int ns = gu_split(fmt[u], H);
-    for (int p = 0; p < ns; ++p) jobs[n++] = Job{kGateUp, uint8_t(u), 16, uint8_t(p), uint16_t(8 * i), uint16_t(lt)};
+__host__ __device__ inline Job phase_a_job(int H, int j) {
+  const int nseg = H / router_seg(H);
+  return Job{kRouter, uint8_t(j / nseg), 0, uint8_t(j % nseg), 0, 0};
+}
+// Phases B and C of CTA b, over the list of ne = U (+ 1) experts, the shared
+// one first (slot kSharedSlot), then the U picked ones (slots 0 .. U - 1):
+// first the gate/up parts of this CTA's tiles (tile-major, gu_parts(H) K
+// parts each; local tile index = position among this CTA's tiles), then one
+// down job per expert for this CTA's output rows.
+__host__ __device__ inline int phase_bc_count(int H, int I, int G, int b, int U, bool with_shared) {
+  int n0, nr;
+  out_rows(H, G, b, n0, nr);
+  const int ne = U + (with_shared ? 1 : 0);
+  return gu_parts(H) * bc_tiles(I, G, b, ne) + (nr > 0 ? ne : 0);
+}
+__host__ __device__ inline Job phase_bc_job(int H, int I, int G, int b, int U, bool with_shared, int j) {
+  const int ns = gu_parts(H), nt = I / 8, sh = with_shared ? 1 : 0;
+  const int ngu = ns * bc_tiles(I, G, b, U + sh);
+  if (j < ngu) {
+    const int i = j / ns, p = j - i * ns, g = b + G * i;
+    const int e = g / nt, r = g - e * nt;
+    return Job{kGateUp, uint8_t(sh && e == 0 ? kSharedSlot : e - sh), 16, uint8_t(p), uint16_t(8 * r), uint16_t(i)};
   }
   int n0, nr;
   out_rows(H, G, b, n0, nr);
-  if (nr > 0) {
-    if (with_shared) jobs[n++] = Job{kDown, uint8_t(kSharedSlot), uint8_t(nr), 0, uint16_t(n0), 0};
-    for (int u = 0; u < U; ++u) jobs[n++] = Job{kDown, uint8_t(u), uint8_t(nr), 0, uint16_t(n0), 0};
-  }
-  return n;
+  const int d = j - ngu;
+  return Job{kDown, uint8_t(sh && d == 0 ? kSharedSlot : d - sh), uint8_t(nr), 0, uint16_t(n0), 0};
 }
 
 struct Params {
+  Plan L;  // shared-memory plan of the launch
   const uint16_t* x;
   int T, H, I, E, k;
   const float* w_router;
@@ -308,8 +317,33 @@ __device__ __forceinline__ void red_release(uint32_t* p, uint32_t v) {
 __device__ __forceinline__ void prefetch_line_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
+// Bulk prefetch of [p, p + bytes) into L2 (a hint: skipped unless the range
+// is 16-byte aligned and a whole number of 16 bytes).
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+  if (bytes > 0 && ((reinterpret_cast<uintptr_t>(p) | bytes) & 15u) == 0)
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// 2^e as a float for -126 <= e <= 127 (the range scaling uses |e| <= 114):
+// multiplying by it is exact up to the one rounding of the product.
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+  return uint32_t(__half_as_ushort(lo)) | (uint32_t(__half_as_ushort(hi)) << 16);
+}
+// Activations k0 .. k0 + 3 (k0 % 4 == 0) of token t into a buffer in format
+// F's fragment order.
+template <int F>
+__device__ __forceinline__ void store4(uint8_t* buf, int k0, int t, int T, float a, float b, float c, float d) {
+  uint8_t* p = buf + frag_pos(F, k0, t, T);
+  const __half ha = __float2half_rn(a), hb = __float2half_rn(b), hc = __float2half_rn(c), hd = __float2half_rn(d);
+  if (F == MOE_Q_INT8_PER_CHANNEL) {
+    static_assert(quad_off<MOE_Q_INT8_PER_CHANNEL>(1) == 4 && quad_off<MOE_Q_INT8_PER_CHANNEL>(2) == 2, "int8 quad");
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_h2(ha, hc), pack_h2(hb, hd));
+  } else {
+    *reinterpret_cast<__half*>(p + quad_off<F>(0)) = ha;
+    *reinterpret_cast<__half*>(p + quad_off<F>(1)) = hb;
+    *reinterpret_cast<__half*>(p + quad_off<F>(2)) = hc;
+    *reinterpret_cast<__half*>(p + quad_off<F>(3)) = hd;
+  }
 }
 __device__ __forceinline__ void named_sync() { __syncthreads(); }
 
@@ -485,8 +519,10 @@ __device__ __forceinline__ void cswap(uint64_t& a, uint64_t& b) {
 // candidate). Each lane sorts its four; every round takes the best lane head
 // by a reduction on the key and one on the low word among equal keys, and the
 // winning lane pops it.
-__device__ __forceinline__ void warp_topk(uint64_t (&c)[4], int k, uint32_t* okey, int* oid) {
+__device__ __noinline__ void warp_topk(uint64_t c0, uint64_t c1, uint64_t c2, uint64_t c3, int k, uint32_t* okey,
+                                      int* oid) {
   const int lane = threadIdx.x & 31;
+  uint64_t c[4] = {c0, c1, c2, c3};
   cswap(c[0], c[1]);
   cswap(c[2], c[3]);
   cswap(c[0], c[2]);
@@ -542,7 +578,6 @@ struct Ctx {
   int e0, nrr, seg, nseg;   // router rows [e0, e0 + nrr) (+ the gate row last), segments per row
   int nreal;                // rows of W_r among them
   int n0, nr;               // output rows of this CTA
-  int fmap[4];              // weight format -> activation buffer (or -1)
   int xexp[kMaxT];          // power-of-two scaling of x per token
   float bias[kMaxBias];     // router bias of this CTA's rows, [row][token]
   int fail;                 // a wait of this CTA gave up
@@ -561,7 +596,7 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
   const int slot = jb.slot;
   const moe_expert& d = C.desc[slot];
-  const int f = d.gate.qtype, ns = gu_split(f, H);
+  const int f = d.gate.qtype, ns = gu_parts(H);
   const int ncol = H / kc(f) / ns, col0 = jb.part * ncol, nit = ncol / 4;
   const int rb = row_code_bytes(f, H);
   const int row = jb.row0 + gq;
@@ -574,7 +609,7 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   R.s_hi = d.up.scales + size_t(row) * sper;
   R.m_lo = f == MOE_Q_INT2_ASYM_G16 ? d.gate.mins + size_t(row) * sper : nullptr;
   R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.up.mins + size_t(row) * sper : nullptr;
-  const uint8_t* bf = C.smem + C.L.o_xf + C.fmap[f] * 2 * T * H;
+  const uint8_t* bf = C.smem + C.L.o_xf + (f - 1) * 2 * T * H;  // formats 1..3 -> buffers 0..2
   float acc[4];
   run_any(f, R, col0, nit, bf, T, acc);
   // D rows gq (gate) / gq + 8 (up), tokens 2 tq, 2 tq + 1
@@ -613,7 +648,7 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
     const int t = 2 * tq + i;
     float h = 0.f;
     if (t < T) {
-      const float sc = ldexpf(1.f, C.xexp[t]);
+      const float sc = exp2i(C.xexp[t]);
       const float g = acc[i] * gsc * sc, u = acc[2 + i] * usc * sc;
       h = silu_f32(g) * u;
       __stcg(hs + size_t(t) * I + row, h);
@@ -627,6 +662,28 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   // the warp barrier orders every lane's stores before lane 0's release
   __syncwarp();
   if (lane == 0) red_release(P.cnt + slot * kCntStride, 1u);
+}
+
+// h of one expert (fp32 [T][I] in the workspace) into a warp's activation
+// buffer in format F's fragment order, scaled by 2^-eh[t] per token; 8 loads
+// per lane in flight at a time.
+template <int F>
+__device__ __noinline__ void h_to_frag(const float4* hs, int T, int I, const int* eh, uint8_t* hf) {
+  const int lane = threadIdx.x & 31, n4 = T * I / 4;  // I % 4 == 0: a float4 holds four values of one token
+  for (int base = lane; base < n4; base += 8 * 32) {
+    float4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = base + 32 * j < n4 ? __ldcg(hs + base + 32 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = 4 * (base + 32 * j);
+      if (i < T * I) {
+        const int t = int(i >= I) + int(i >= 2 * I) + int(i >= 3 * I);  // T <= 4
+        const float sc = exp2i(-eh[t]);
+        store4<F>(hf, i - t * I, t, T, v[j].x * sc, v[j].y * sc, v[j].z * sc, v[j].w * sc);
+      }
+    }
+  }
 }
 
 // down job: this CTA's output rows [n0, n0 + nr) of one expert (already on
@@ -667,24 +724,9 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   if (lane < T) s_eh[warp][lane] = range_exp(__ldcg(P.cnt + slot * kCntStride + 1 + lane));
   __syncwarp();
   const float4* hs = reinterpret_cast<const float4*>(P.h + size_t(slot) * T * I);
-  const int n4 = T * I / 4;  // I % 4 == 0: each float4 holds four values of one token
-  for (int base = lane; base < n4; base += 8 * 32) {
-    float4 v[8];  // 8 loads per lane in flight at a time
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = base + 32 * j < n4 ? __ldcg(hs + base + 32 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = 4 * (base + 32 * j);
-      if (i < T * I) {
-        const int t = i / I, kk = i - t * I;
-        const int e = s_eh[warp][t];
-        *reinterpret_cast<__half*>(hf + frag_pos(f, kk, t, T)) = __float2half_rn(ldexpf(v[j].x, -e));
-        *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 1, t, T)) = __float2half_rn(ldexpf(v[j].y, -e));
-        *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 2, t, T)) = __float2half_rn(ldexpf(v[j].z, -e));
-        *reinterpret_cast<__half*>(hf + frag_pos(f, kk + 3, t, T)) = __float2half_rn(ldexpf(v[j].w, -e));
-      }
-    }
-  }
+  if (f == MOE_Q_INT4_SYM_G32) h_to_frag<MOE_Q_INT4_SYM_G32>(hs, T, I, s_eh[warp], hf);
+  else if (f == MOE_Q_INT2_ASYM_G16) h_to_frag<MOE_Q_INT2_ASYM_G16>(hs, T, I, s_eh[warp], hf);
+  else h_to_frag<MOE_Q_INT8_PER_CHANNEL>(hs, T, I, s_eh[warp], hf);
   __syncwarp();
   float acc[4];
   run_any(f, R, 0, nit, hf, T, acc);
@@ -693,7 +735,7 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   for (int i = 0; i < 4; ++i) {
     const int r = gq + 8 * (i >> 1), t = 2 * tq + (i & 1);
     if (r < jb.nrows && t < T) {
-      float v = ldexpf(acc[i], s_eh[warp][t]);
+      float v = acc[i] * exp2i(s_eh[warp][t]);
       if (f == MOE_Q_INT8_PER_CHANNEL) v *= f16_to_f32(d.down.scales[jb.row0 + r]);
       y[r * T + t] = v;
     }
@@ -728,9 +770,8 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb, const uint4 w0, co
   float* rp = reinterpret_cast<float*>(C.smem + C.L.o_rp);
   const int nv = seg / 128;  // 16-byte loads per lane (4 or 2)
   const uint4 w[4] = {w0, w1, w2, w3};
-#pragma unroll
-  for (int t = 0; t < kMaxT; ++t) {
-    if (t >= T) break;
+#pragma unroll 1
+  for (int t = 0; t < T; ++t) {
     float a = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -768,77 +809,106 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb, const uint4 w0, co
   if (lane == 0) red_release(&P.hdr->bar_count, 1u);
 }
 
-// ---------------------------------------------------------------- the kernel
-// Routing of one CTA, run by its last T warps (one token each) while the
-// others may still work on phase A: wait for every CTA's logits, top-k per
-// token, gates, the distinct picked experts (slots), their descriptors and
-// this CTA's job list of phases B and C. Lane 0 of warp kWarps - T publishes
-// the result through `ready` (1 = go, 2 = nothing to do).
+// ---------------------------------------------------------------- routing
+// Routing of one CTA, by all its warps once phase A is done: wait for every
+// CTA's logits, top-k per token (first the best k of each 128-logit chunk,
+// one warp per (token, chunk), then the best k of those, one warp per
+// token), gates, the distinct picked experts in ascending id order (slots),
+// their descriptors, and the L2 prefetch of this CTA's gate/up parts and
+// down rows of every picked expert. Returns whether phases B and C run (the
+// same answer on every CTA: identical inputs, identical code).
 struct RouteShared {
   int idx[kMaxT * kMaxK];
   float w[kMaxT * kMaxK];
   uint32_t key[kMaxT * kMaxK];
-  int slot[kMaxT * kMaxK];      // (t, j) -> slot
-  int uniq[kMaxT * kMaxK];      // slot -> expert id
-  int fmt[kMaxT * kMaxK];       // slot -> weight format
-  uint32_t ck[kMaxT * 8 * kMaxK];  // first-round winners
+  int slot[kMaxT * kMaxK];         // (t, j) -> slot
+  int uniq[kMaxT * kMaxK];         // slot -> expert id
+  uint32_t ck[kMaxT * 8 * kMaxK];  // first-round winners [t][chunk][k]
   int ci[kMaxT * 8 * kMaxK];
   uint32_t bits[kMaxE / 32];
-  int U, nJ, bad;
-  volatile int ready;
+  uint32_t bpre[kMaxE / 32];
+  int U, bad;
 };
 
-__device__ __noinline__ void route_cta(Ctx& C, RouteShared& R, bool has_shared) {
+// L2 prefetch of the rows of one gate/up job's K part: lane r < 16 takes A
+// row r (gate rows 0-7, up rows 8-15): its codes and its scales (and mins).
+__device__ __forceinline__ void prefetch_gate_up(const moe_expert& d, const Job& jb, int H, int r) {
+  const moe_qmatrix& m = r < 8 ? d.gate : d.up;
+  const int f = m.qtype, ns = gu_parts(H);
+  const int ncol = H / kc(f) / ns, col0 = jb.part * ncol, row = jb.row0 + (r & 7);
+  prefetch_l2(m.codes + size_t(row) * row_code_bytes(f, H) + size_t(col0) * 16, uint32_t(ncol * 16));
+  if (f == MOE_Q_INT4_SYM_G32) {
+    prefetch_l2(m.scales + size_t(row) * (H / 32) + col0, uint32_t(ncol * 2));
+  } else if (f == MOE_Q_INT2_ASYM_G16) {
+    prefetch_l2(m.scales + size_t(row) * (H / 16) + 4 * col0, uint32_t(ncol * 8));
+    prefetch_l2(m.mins + size_t(row) * (H / 16) + 4 * col0, uint32_t(ncol * 8));
+  }
+}
+// L2 prefetch of output rows [n0, n0 + nr) of a down matrix.
+__device__ __forceinline__ void prefetch_down(const moe_qmatrix& m, int I, int n0, int nr) {
+  const int rb = row_code_bytes(m.qtype, I);
+  prefetch_l2(m.codes + size_t(n0) * rb, uint32_t(nr * rb));
+  const int sper = m.qtype == MOE_Q_INT8_PER_CHANNEL ? 1 : I / (m.qtype == MOE_Q_INT4_SYM_G32 ? 32 : 16);
+  prefetch_l2(m.scales + size_t(n0) * sper, uint32_t(nr * sper * 2));
+  if (m.qtype == MOE_Q_INT2_ASYM_G16) prefetch_l2(m.mins + size_t(n0) * sper, uint32_t(nr * sper * 2));
+}
+
+__device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) {
   const Params& P = *C.P;
   const int T = C.T, E = C.E, k = C.k, H = C.H, I = C.I;
-  const int lane = threadIdx.x & 31, t = (threadIdx.x >> 5) - (kWarps - T);  // this warp's token
-  const int nthr = T * 32;
-  auto rsync = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory"); };
-  if (t == 0 && lane == 0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
     if (!wait_counter(&P.hdr->bar_count, uint32_t(C.G), P.hdr, P.wait_cycles, 7000000 + C.b)) C.fail = 1;
   }
-  rsync();
+  if (threadIdx.x < kMaxE / 32) R.bits[threadIdx.x] = 0u;
+  __syncthreads();
   const bool live = !C.fail;
   float* lg = reinterpret_cast<float*>(C.smem + C.L.o_lg);
   if (live) {
-    // 16 loads per thread in flight at a time
-    const int r0 = threadIdx.x - (kWarps - T) * 32;
-    for (int base = r0; base < T * E; base += 16 * nthr) {
-      float v[16];
+    // T E <= kMaxT kMaxE logits, all of a thread's loads in flight together
+    constexpr int kPer = kMaxT * kMaxE / kThreads;
+    float v[kPer];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = base + j * nthr < T * E ? __ldcg(P.logits + base + j * nthr) : 0.f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (base + j * nthr < T * E) lg[base + j * nthr] = v[j];
+    for (int j = 0; j < kPer; ++j) {
+      const int i = threadIdx.x + j * kThreads;
+      v[j] = i < T * E ? __ldcg(P.logits + i) : 0.f;
     }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j)
+      if (threadIdx.x + j * kThreads < T * E) lg[threadIdx.x + j * kThreads] = v[j];
   }
-  for (int i = threadIdx.x - (kWarps - T) * 32; i < kMaxE / 32; i += nthr) R.bits[i] = 0u;
-  rsync();
-  // this token's top-k in two rounds: its 128-logit chunks, then their winners
-  if (live) {
-    const int nch = (E + kTopChunk - 1) / kTopChunk;
-    for (int stage = 0; stage < 2; ++stage) {
-      for (int ch = 0; ch < (stage == 0 ? nch : 1); ++ch) {
-        const int nc = stage == 0 ? min(kTopChunk, E - ch * kTopChunk) : nch * k;
-        const uint32_t* ck = R.ck + t * 8 * kMaxK;
-        const int* ci = R.ci + t * 8 * kMaxK;
-        uint64_t cand[4];
+  __syncthreads();
+  // first round: the best k of each (token, chunk)
+  const int nch = (E + kTopChunk - 1) / kTopChunk;
+  if (live)
+    for (int q = warp; q < T * nch; q += kWarps) {
+      const int t = q / nch, ch = q - t * nch;
+      const int nc = min(kTopChunk, E - ch * kTopChunk);
+      uint64_t c[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = lane + 32 * i;
-          const uint32_t key = c >= nc ? 0u : stage == 0 ? f2key(lg[t * E + ch * kTopChunk + c]) : ck[c];
-          const int id = stage == 0 ? ch * kTopChunk + c : ci[c < nc ? c : 0];
-          cand[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(id)) : 0ull;
-        }
-        uint32_t* okey = stage == 0 ? R.ck + t * 8 * kMaxK + ch * k : R.key + t * k;
-        int* oid = stage == 0 ? R.ci + t * 8 * kMaxK + ch * k : R.idx + t * k;
-        warp_topk(cand, k, okey, oid);
-        __syncwarp();
+      for (int i = 0; i < 4; ++i) {
+        const int cc = lane + 32 * i;
+        const uint32_t key = cc < nc ? f2key(lg[t * E + ch * kTopChunk + cc]) : 0u;
+        c[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(ch * kTopChunk + cc)) : 0ull;
       }
+      warp_topk(c[0], c[1], c[2], c[3], k, R.ck + (t * 8 + ch) * kMaxK, R.ci + (t * 8 + ch) * kMaxK);
     }
-    // gates: the softmax over all logits restricted to the picks and
-    // renormalised = a softmax over the picked logits (of the unbiased ones
-    // when the bias only selects)
+  __syncthreads();
+  // second round (one warp per token): the best k of the chunks' winners,
+  // then the gates: the softmax over all logits restricted to the picks and
+  // renormalised = a softmax over the picked logits (of the unbiased ones when
+  // the bias only selects)
+  if (live && warp < T) {
+    const int t = warp, nc = nch * k;  // <= 128 candidates, 4 per lane
+    uint64_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int cc = lane + 32 * i, ch = cc / k, j = cc - ch * k;
+      const uint32_t key = cc < nc ? R.ck[(t * 8 + ch) * kMaxK + j] : 0u;
+      c[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(R.ci[(t * 8 + ch) * kMaxK + j])) : 0ull;
+    }
+    warp_topk(c[0], c[1], c[2], c[3], k, R.key + t * k, R.idx + t * k);
+    __syncwarp();
     const bool sel_only = (P.flags & MOE_BIAS_SELECTION_ONLY) != 0;
     float v = -CUDART_INF_F;
     if (lane < k) v = sel_only ? __ldcg(P.logits_u + size_t(t) * E + R.idx[t * k + lane]) : key2f(R.key[t * k + lane]);
@@ -847,20 +917,18 @@ __device__ __noinline__ void route_cta(Ctx& C, RouteShared& R, bool has_shared) 
     for (int o = 16; o > 0; o >>= 1) v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, o));
     const float ev = lane < k ? expf(v - v0) : 0.f;
     const float den = warp_sum(ev);
-    if (lane < k) R.w[t * k + lane] = ev / den;
-    // distinct picked experts in ascending id order through a bitmap
     if (lane < k) {
+      R.w[t * k + lane] = ev / den;
       const int id = R.idx[t * k + lane];
       if (id >= 0 && id < E) atomicOr(&R.bits[id >> 5], 1u << (id & 31));
       else R.bad = 1;
     }
   }
-  rsync();
-  if (t == 0) {
-    // slot of an id = set bits below it (warp scan over the bitmap words)
-    __shared__ uint32_t s_bpre[kMaxE / 32];
+  __syncthreads();
+  // slots: the slot of an id = set bits below it (warp scan over the bitmap)
+  if (warp == 0) {
     uint32_t pre = 0;
-#pragma unroll
+#pragma unroll 1
     for (int i = 0; i < kMaxE / 32 / 32; ++i) {
       const uint32_t c = __popc(R.bits[i * 32 + lane]);
       uint32_t inc = c;
@@ -869,75 +937,67 @@ __device__ __noinline__ void route_cta(Ctx& C, RouteShared& R, bool has_shared) 
         const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
         if (lane >= o) inc += y;
       }
-      s_bpre[i * 32 + lane] = pre + inc - c;
+      R.bpre[i * 32 + lane] = pre + inc - c;
       pre += __shfl_sync(0xffffffffu, inc, 31);
     }
     __syncwarp();
-    const int U = int(pre);
     if (live && !R.bad)
       for (int i = lane; i < T * k; i += 32) {
         const int id = R.idx[i], wd = id >> 5;
-        const int rank = int(s_bpre[wd] + __popc(R.bits[wd] & ((1u << (id & 31)) - 1u)));
+        const int rank = int(R.bpre[wd] + __popc(R.bits[wd] & ((1u << (id & 31)) - 1u)));
         R.slot[i] = rank;
         R.uniq[rank] = id;
       }
-    __syncwarp();
-    moe_expert* desc = C.desc;
-    constexpr int W = int(sizeof(moe_expert) / 4);
-    if (live && !R.bad) {
-      // 8 loads per lane in flight at a time (the table is on its way into L2
-      // since the kernel's entry)
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
-      uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
-      for (int base = lane; base < U * W; base += 8 * 32) {
-        uint32_t v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i = base + 32 * j;
-          v[j] = i < U * W ? src[size_t(R.uniq[i / W]) * W + (i % W)] : 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (base + 32 * j < U * W) dst[base + 32 * j] = v[j];
-      }
-    }
-    __syncwarp();
-    bool bad = R.bad != 0;
-    if (live && !bad)
-      for (int u = lane; u < U; u += 32) {
-        if (!expert_ok(desc[u], H, I)) R.bad = 1;
-        R.fmt[u] = desc[u].gate.qtype;
-      }
-    __syncwarp();
-    bad = R.bad != 0;
-    if (live && bad && lane == 0) flag_error(P.hdr, MOE_ERR_DEVICE_FAULT, 1000000);
-    const bool work = live && !bad;
-    if (work) {
-      // this CTA's down rows of every picked expert into L2
-      if (C.nr > 0)
-        for (int u = lane; u < U; u += 32) {
-          const moe_qmatrix& dm = desc[u].down;
-          const int rb = row_code_bytes(dm.qtype, I);
-          prefetch_l2(dm.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
-        }
-      if (lane == 0)
-        R.nJ = phase_bc_jobs(H, I, C.G, C.b, U, R.fmt, has_shared, reinterpret_cast<Job*>(C.smem + C.L.o_jobs) + kMaxJobs / 2);
-    }
-    __syncwarp();
-    if (lane == 0) {
-      R.U = U;
-      __threadfence_block();
-      R.ready = work ? 1 : 2;
-    }
+    if (lane == 0) R.U = int(pre);
   }
+  __syncthreads();
+  const int U = R.U;
+  const bool ok = live && R.bad == 0;
+  // descriptors of the picked experts (the table is in L2 since the entry),
+  // all of a thread's loads in flight together
+  moe_expert* desc = C.desc;
+  constexpr int W = int(sizeof(moe_expert) / 4);
+  if (ok) {
+    constexpr int kPer = (kMaxT * kMaxK * W + kThreads - 1) / kThreads;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
+    uint32_t v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = threadIdx.x + j * kThreads;
+      v[j] = i < U * W ? src[size_t(R.uniq[i / W]) * W + (i % W)] : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j)
+      if (threadIdx.x + j * kThreads < U * W) dst[threadIdx.x + j * kThreads] = v[j];
+  }
+  __syncthreads();
+  if (ok && warp == 0)
+    for (int u = lane; u < U; u += 32)
+      if (!expert_ok(desc[u], H, I)) R.bad = 1;
+  __syncthreads();
+  const bool work = ok && R.bad == 0;
+  if (live && !work && threadIdx.x == 0) flag_error(P.hdr, MOE_ERR_DEVICE_FAULT, 1000000);
+  if (work) {
+    // this CTA's routed gate/up parts (16 rows each) and down rows into L2
+    const int ngu = gu_parts(H) * bc_tiles(I, C.G, C.b, U + (has_shared ? 1 : 0));
+    for (int q = threadIdx.x; q < ngu * 16; q += kThreads) {
+      const Job jb = phase_bc_job(H, I, C.G, C.b, U, has_shared, q >> 4);
+      if (jb.slot != kSharedSlot) prefetch_gate_up(desc[jb.slot], jb, H, q & 15);
+    }
+    if (C.nr > 0)
+      for (int u = threadIdx.x; u < U; u += kThreads) prefetch_down(desc[u].down, I, C.n0, C.nr);
+  }
+  return work;
 }
 
+// ---------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Ctx C;
   __shared__ RouteShared R;
   __shared__ uint32_t s_xamax[kMaxT];
-  __shared__ int s_nA, s_bad;
+  __shared__ int s_bad;
 
   const int T = P.T, H = P.H, I = P.I, E = P.E, k = P.k;
   const int G = gridDim.x, b = blockIdx.x;
@@ -945,20 +1005,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   WsHeader* hdr = P.hdr;
   const bool has_shared = P.shared != nullptr;
   const bool gate_row = P.shared_gate != nullptr && has_shared;
+  const Plan& L = P.L;
 
-  // ---------------------------------------------------------- router loads first
-  // The phase-A job list starts with the router parts (row-major), so this
-  // warp's first job is part `warp` when there is one: load its weights now.
+  // ---------------------------------------------------------- loads first
+  // This warp's router part (phase-A job `warp`, when there is one), then
+  // everything else the prologue reads, all in flight together: x (this
+  // thread's 8-element groups), the bias of this CTA's router rows and the
+  // shared expert's descriptor; the expert table goes into L2 for the routing.
   int e0, nreal;
   router_range(E, G, b, e0, nreal);
   const int seg = router_seg(H), nseg = H / seg;
   const int nrr = router_rows_of(E, G, b, gate_row);
+  const int nA = nrr * nseg;
   uint4 w0[4] = {};
-  const bool early = warp < nrr * nseg;
-  if (early) router_load(P, e0, nreal, seg, Job{kRouter, uint8_t(warp / nseg), 0, uint8_t(warp % nseg), 0, 0}, w0);
-  // then everything else the prologue reads, all in flight together: x (this
-  // thread's 8-element groups), the bias of this CTA's router rows and the
-  // shared expert's descriptor; the expert table goes into L2 for the routing
+  if (warp < nA) router_load(P, e0, nreal, seg, phase_a_job(H, warp), w0);
   constexpr int kXg = kMaxT * kMaxH / 8 / kThreads;
   const int ng = T * H / 8;
   uint4 xg[kXg];
@@ -984,11 +1044,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   }
 
   // ---------------------------------------------------------- prologue
-  moe_expert* desc = reinterpret_cast<moe_expert*>(smem + make_plan(T, H, I, E, k, G).o_desc);
+  moe_expert* desc = reinterpret_cast<moe_expert*>(smem + L.o_desc);
   if (threadIdx.x == 0) {
     C.P = &P;
     C.smem = smem;
-    C.L = make_plan(T, H, I, E, k, G);
+    C.L = L;
     C.T = T, C.H = H, C.I = I, C.E = E, C.k = k, C.G = G, C.b = b;
     C.e0 = e0;
     C.nreal = nreal;
@@ -996,22 +1056,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     C.seg = seg;
     C.nseg = nseg;
     out_rows(H, G, b, C.n0, C.nr);
-    for (int i = 0; i < 4; ++i) C.fmap[i] = i - 1;  // formats 1..3 -> activation buffers 0..2
     C.fail = 0;
     C.rdone = 0;
     C.desc = desc;
     s_bad = 0;
     R.bad = 0;
-    R.ready = 0;
     R.U = 0;
   }
   if (threadIdx.x < kMaxT) s_xamax[threadIdx.x] = 0u;
   __syncthreads();
   if (has_shared && threadIdx.x < kDescWords) reinterpret_cast<uint32_t*>(desc + kSharedSlot)[threadIdx.x] = sdesc_v;
   if (threadIdx.x < kMaxBias) C.bias[threadIdx.x] = bias_v;  // zero beyond the CTA's rows
-  const Plan& L = C.L;
-  const int ntl = max_tiles(T, I, E, k, G);
   {
+    const int ntl = max_tiles(T, I, E, k, G);
     float* Y = reinterpret_cast<float*>(smem + L.o_y);
     float* red = reinterpret_cast<float*>(smem + L.o_red);
     int* tdone = reinterpret_cast<int*>(smem + L.o_td);
@@ -1045,86 +1102,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   }
   __syncthreads();
   if (threadIdx.x < T) C.xexp[threadIdx.x] = range_exp(s_xamax[threadIdx.x]);
-  if (threadIdx.x == 0) {
-    bool good = true;
-    if (has_shared) {
-      good = expert_ok(desc[kSharedSlot], H, I);
-      if (!good) {
-        s_bad = 1;
-        flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
-      } else if (C.nr > 0) {
-        // the shared expert's down rows of this CTA into L2: needed whatever the routing
-        const moe_qmatrix& d = desc[kSharedSlot].down;
-        const int rb = row_code_bytes(d.qtype, I);
-        prefetch_l2(d.codes + size_t(C.n0) * rb, uint32_t(C.nr * rb));
-      }
-    }
-    s_nA = phase_a_jobs(H, I, E, G, b, has_shared && good ? desc[kSharedSlot].gate.qtype : 0, gate_row,
-                        reinterpret_cast<Job*>(smem + L.o_jobs));
+  if (threadIdx.x == 0 && has_shared && !expert_ok(desc[kSharedSlot], H, I)) {
+    s_bad = 1;
+    flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
   }
   __syncthreads();
-  // activations in fragment order for all three formats (from global x: x32
-  // is reused after phase A), so routed experts of any format need no
-  // further barrier
+  if (has_shared && !s_bad) {
+    // the shared expert's gate/up parts of this CTA and its down rows into
+    // L2: needed whatever the routing
+    const int nsh = gu_parts(H) * bc_tiles(I, G, b, 1);  // its tiles come first in the B/C list
+    for (int q = threadIdx.x; q < nsh * 16; q += kThreads)
+      prefetch_gate_up(desc[kSharedSlot], phase_bc_job(H, I, G, b, 0, true, q >> 4), H, q & 15);
+    if (threadIdx.x == kThreads - 1 && C.nr > 0) prefetch_down(desc[kSharedSlot].down, I, C.n0, C.nr);
+  }
+  // activations in fragment order for all three formats, so routed experts
+  // of any format need no further barrier
 #pragma unroll
   for (int j = 0; j < kXg; ++j) {
     const int g = threadIdx.x + j * kThreads;
     if (g < ng) {
-      const int t = g * 8 / H, k0 = g * 8 - t * H, ex = -C.xexp[t];
+      const int t = g * 8 / H, k0 = g * 8 - t * H;
+      const float sc = exp2i(-C.xexp[t]);
       const uint32_t wv[4] = {xg[j].x, xg[j].y, xg[j].z, xg[j].w};
+      float v[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const __half v = __float2half_rn(ldexpf(bf16_to_f32(uint16_t(e & 1 ? wv[e >> 1] >> 16 : wv[e >> 1] & 0xffffu)), ex));
-        for (int f = 1; f <= 3; ++f)
-          *reinterpret_cast<__half*>(smem + L.o_xf + (f - 1) * 2 * T * H + frag_pos(f, k0 + e, t, T)) = v;
-      }
+      for (int e = 0; e < 8; ++e) v[e] = bf16_to_f32(uint16_t(e & 1 ? wv[e >> 1] >> 16 : wv[e >> 1] & 0xffffu)) * sc;
+      uint8_t* xf = smem + L.o_xf;
+      store4<MOE_Q_INT4_SYM_G32>(xf, k0, t, T, v[0], v[1], v[2], v[3]);
+      store4<MOE_Q_INT4_SYM_G32>(xf, k0 + 4, t, T, v[4], v[5], v[6], v[7]);
+      store4<MOE_Q_INT2_ASYM_G16>(xf + 2 * T * H, k0, t, T, v[0], v[1], v[2], v[3]);
+      store4<MOE_Q_INT2_ASYM_G16>(xf + 2 * T * H, k0 + 4, t, T, v[4], v[5], v[6], v[7]);
+      store4<MOE_Q_INT8_PER_CHANNEL>(xf + 4 * T * H, k0, t, T, v[0], v[1], v[2], v[3]);
+      store4<MOE_Q_INT8_PER_CHANNEL>(xf + 4 * T * H, k0 + 4, t, T, v[4], v[5], v[6], v[7]);
     }
   }
   if (nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
   __syncthreads();
-  const int nA = s_nA;
 
   // ---------------------------------------------------------- phase A
-  {
-    const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs);
-    for (int j = warp; j < nA; j += kWarps) {
-      const Job jb = jobs[j];
-      if (jb.kind == kRouter) {
-        uint4 w[4] = {};
-        if (j == warp && early) {
+  for (int j = warp; j < nA; j += kWarps) {
+    const Job jb = phase_a_job(H, j);
+    uint4 w[4] = {};
+    if (j == warp) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) w[i] = w0[i];
-        } else {
-          router_load(P, e0, nreal, seg, jb, w);
-        }
-        job_router(C, jb, w[0], w[1], w[2], w[3]);
-      } else {
-        job_gate_up(C, jb);
-      }
+      for (int i = 0; i < 4; ++i) w[i] = w0[i];
+    } else {
+      router_load(P, e0, nreal, seg, jb, w);
     }
+    job_router(C, jb, w[0], w[1], w[2], w[3]);
   }
 
   // ---------------------------------------------------------- routing
-  if (warp >= kWarps - T) route_cta(C, R, has_shared && !s_bad);
-  // every warp waits (bounded by the routing warps' own bounded waits) for
-  // the job list of phases B and C
-  if (lane == 0) {
-    const long long t0 = clock64();
-    while (R.ready == 0) {
-      __nanosleep(64);
-      if (clock64() - t0 > 4 * P.wait_cycles + 1000000) break;  // the routing warps' waits end long before
-    }
-  }
-  __syncwarp();
-  __threadfence_block();
-  const bool work = R.ready == 1 && !s_bad;
+  const bool work = route_all(C, R, has_shared) && !s_bad;
 
   // ---------------------------------------------------------- phases B, C
   if (work) {
-    const Job* jobs = reinterpret_cast<const Job*>(smem + L.o_jobs) + kMaxJobs / 2;
-    const int nJ = R.nJ;
+    const int U = R.U;
+    const int nJ = phase_bc_count(H, I, G, b, U, has_shared);
     for (int j = warp; j < nJ; j += kWarps) {
-      const Job jb = jobs[j];
+      const Job jb = phase_bc_job(H, I, G, b, U, has_shared, j);
       if (jb.kind == kGateUp) job_gate_up(C, jb);
       else job_down(C, jb);
     }
@@ -1189,14 +1225,9 @@ int grid_size() {
 // Whether the shape runs as one fused launch on a grid of G CTAs.
 bool eligible_on(int T, int H, int I, int E, int k, int G) {
   if (T < 1 || T > kMaxT || k < 1 || k > kMaxK || E < k || E > kMaxE) return false;
-  if (H < 256 || I < 256 || H > kMaxH || I > 2048 || (H % 256) || (I % 256)) return false;
+  if (H < 256 || I < 256 || H > kMaxH || I > kMaxI || (H % 256) || (I % 256)) return false;
   if (router_rows(E, G) * T > kMaxBias) return false;
   if ((H + G - 1) / G > 16) return false;             // output rows per CTA fit one 16-row tile
-  // job lists: phase A <= router rows x segments + 2 x shared tiles, phase
-  // B/C <= 2 x routed tiles + one down job per slot
-  const int U = T * k < E ? T * k : E;
-  if ((router_rows(E, G) + 1) * (H / router_seg(H)) + 2 * shared_tiles(I, G, 0) > kMaxJobs / 2) return false;
-  if (2 * ((U * (I / 8) + G - 1) / G) + U + 1 > kMaxJobs / 2) return false;
   return make_plan(T, H, I, E, k, G).total + kStaticSmem <= kSmemLimit;
 }
 
@@ -1231,7 +1262,7 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) s_cap_set[dev] = 1;
   }
-  Params P{x,      T,       H,        I,      E,   k,        w_router,           bias,
+  Params P{make_plan(T, H, I, E, k, grid), x, T, H, I, E, k, w_router, bias,
            bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
            logits_ws, h_ws, counters, wait_cycles, flags, shared_gate, logits_u_ws,
            sgate_ws, heat};

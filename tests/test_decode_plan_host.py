@@ -1,16 +1,18 @@
 """Host-side planning of the fused decode kernel, checked on the CPU.
 
 The fused decode kernel (decode_fused.cu) computes its shared-memory plan,
-activation fragment order and per-CTA job lists with host/device functions.
+activation fragment order and per-CTA jobs (computed from their number) with
+host/device functions.
 A small host program (compiled with nvcc, run without a GPU) evaluates them
 over every shape the kernel accepts and checks the invariants the kernel
 relies on: every fp16 activation has exactly one place in the fragment
-order; the plan fits the per-CTA shared-memory limit with 16-byte aligned
-regions; over all CTAs of the grid every router row, every gate/up tile
-(both K parts) and every output row of every expert is covered exactly once;
-job fields fit their widths; local tile indices stay inside the reduction
-slots; and the workspace holds the counters, logits and intermediate
-activations the kernel writes.
+order, and the four-at-a-time stores put each value there; the plan fits the
+per-CTA shared-memory limit with 16-byte aligned regions; over all CTAs of
+the grid, for every count of picked experts, every router row, every K part
+of every gate/up tile and every output row of every expert (the shared one
+included) is covered exactly once; job fields fit their widths; local tile
+indices stay inside the reduction slots; and the workspace holds the
+counters, logits and intermediate activations the kernel writes.
 """
 import json
 import os
@@ -32,9 +34,19 @@ size_t moe::grouped_ws_bytes(long long, int, int, int, int, bool) { return 0; }
 size_t moe::router_tc_ws_bytes(long long, int, int) { return 0; }
 using namespace moe;
 using namespace moe::dfx;
+template <int F>
+int check_quads(int T, int K) {
+  int bad = 0;
+  for (int t = 0; t < T; ++t)
+    for (int k0 = 0; k0 < K; k0 += 4)
+      for (int i = 0; i < 4; ++i)
+        if (frag_pos(F, k0 + i, t, T) != frag_pos(F, k0, t, T) + quad_off<F>(i)) ++bad;
+  return bad;
+}
 int main() {
   int bad_frag = 0, bad_plan = 0, bad_cover = 0, bad_fields = 0, bad_ws = 0, eligible = 0, checked = 0;
-  // fragment order: a bijection of (k, t) onto the fp16 places of the buffer
+  // fragment order: a bijection of (k, t) onto the fp16 places of the buffer,
+  // and the four-at-a-time stores land where frag_pos puts each value
   for (int f = 1; f <= 3; ++f)
     for (int T = 1; T <= 4; ++T)
       for (int K = 256; K <= 2048; K += 256) {
@@ -45,10 +57,13 @@ int main() {
             if (o < 0 || o % 2 || o / 2 >= K * T || seen[o / 2]++) ++bad_frag;
           }
       }
+  for (int T = 1; T <= 4; ++T)
+    for (int K = 256; K <= 2048; K += 256)
+      bad_frag += check_quads<MOE_Q_INT4_SYM_G32>(T, K) + check_quads<MOE_Q_INT2_ASYM_G16>(T, K) +
+                  check_quads<MOE_Q_INT8_PER_CHANNEL>(T, K);
   const int Gs[] = {148, 132};
   const int Es[] = {16, 24, 32, 64, 128, 256, 384, 512, 1024};
   const int Ks[] = {1, 2, 4, 6, 8, 10, 16};
-  std::vector<Job> jobs(kMaxJobs + 64);
   for (int G : Gs)
     for (int T = 1; T <= 4; ++T)
       for (int H = 256; H <= 2048; H += 256)
@@ -60,58 +75,64 @@ int main() {
               if (!eligible_on(T, H, I, E, k, G)) continue;
               ++eligible;
               const Plan p = make_plan(T, H, I, E, k, G);
-              const int offs[] = {p.o_x32, p.o_hf, p.o_xf, p.o_lg, p.o_rp, p.o_red, p.o_td, p.o_y, p.o_jobs, p.o_desc};
+              const int offs[] = {p.o_x32, p.o_hf, p.o_xf, p.o_lg, p.o_rp, p.o_red, p.o_td, p.o_y, p.o_desc};
               for (int o : offs)
                 if (o % 16) ++bad_plan;
               if (p.total + kStaticSmem > kSmemLimit) ++bad_plan;
-              // every format mix of the routed experts gives the same job counts
-              // up to the K split; use the one with the most jobs (int4 splits
-              // when int2 may not)
-              const int U = T * k < E ? T * k : E;
-              for (int fm = 1; fm <= 3; ++fm) {
-                const bool gate = fm == 2;  // the shared-gate row on one of the format mixes
-                std::vector<int> fmt(U, fm);
-                std::vector<int> rows(E + 1, 0), tparts(size_t(U + 1) * (I / 8), 0), outc(size_t(U + 1) * H, 0);
-                for (int b = 0; b < G; ++b) {
-                  int e0, nrr;
-                  router_range(E, G, b, e0, nrr);
-                  const int na = phase_a_jobs(H, I, E, G, b, fm, gate, jobs.data());
-                  if (na > kMaxJobs / 2) { ++bad_fields; continue; }
-                  for (int j = 0; j < na; ++j) {
-                    const Job& jb = jobs[j];
-                    if (jb.kind == kRouter) {
-                      if (jb.slot > nrr || (jb.slot == nrr && !(gate && b == G - 1))) ++bad_fields;
-                      if (jb.part == 0) rows[jb.slot == nrr ? E : e0 + jb.slot]++;
-                    } else {
-                      tparts[size_t(U) * (I / 8) + jb.row0 / 8]++;
-                      if (jb.tile >= max_tiles(T, I, E, k, G)) ++bad_fields;
+              // every picked-expert count from 1 to the most, with and
+              // without the shared expert and its gate row
+              const int Umax = T * k < E ? T * k : E;
+              const int ns = gu_parts(H);
+              for (int U = 1; U <= Umax; U += (U < 4 ? 1 : 7)) {
+                for (int v = 0; v < 2; ++v) {
+                  const bool sh = v == 1, gate = v == 1;
+                  const int ne = U + (sh ? 1 : 0);
+                  std::vector<int> rows(E + 1, 0), parts(size_t(ne) * (I / 8) * ns, 0), outc(size_t(ne) * H, 0);
+                  for (int b = 0; b < G; ++b) {
+                    int e0, nrr;
+                    router_range(E, G, b, e0, nrr);
+                    const int na = phase_a_count(H, E, G, b, gate);
+                    for (int j = 0; j < na; ++j) {
+                      const Job jb = phase_a_job(H, j);
+                      if (jb.kind != kRouter || jb.slot > nrr || (jb.slot == nrr && !(gate && b == G - 1)) ||
+                          jb.part >= H / router_seg(H))
+                        ++bad_fields;
+                      else if (jb.part == 0)
+                        rows[jb.slot == nrr ? E : e0 + jb.slot]++;
+                    }
+                    const int nb = phase_bc_count(H, I, G, b, U, sh);
+                    int n0, nr;
+                    out_rows(H, G, b, n0, nr);
+                    if (nr > 16) ++bad_fields;
+                    for (int j = 0; j < nb; ++j) {
+                      const Job jb = phase_bc_job(H, I, G, b, U, sh, j);
+                      const int e = jb.slot == kSharedSlot ? 0 : jb.slot + (sh ? 1 : 0);  // list position
+                      if ((jb.slot == kSharedSlot && !sh) || (jb.slot != kSharedSlot && jb.slot >= U)) {
+                        ++bad_fields;
+                        continue;
+                      }
+                      if (jb.kind == kGateUp) {
+                        if (jb.tile >= max_tiles(T, I, E, k, G) || jb.row0 % 8 || jb.row0 >= I || jb.part >= ns ||
+                            jb.nrows != 16)
+                          ++bad_fields;
+                        else
+                          parts[(size_t(e) * (I / 8) + jb.row0 / 8) * ns + jb.part]++;
+                      } else if (jb.kind == kDown) {
+                        if (jb.nrows != nr || jb.row0 != n0) ++bad_fields;
+                        for (int r = 0; r < jb.nrows; ++r) outc[size_t(e) * H + jb.row0 + r]++;
+                      } else {
+                        ++bad_fields;
+                      }
                     }
                   }
-                  const int nb = phase_bc_jobs(H, I, G, b, U, fmt.data(), true, jobs.data());
-                  if (nb > kMaxJobs / 2) { ++bad_fields; continue; }
-                  int n0, nr;
-                  out_rows(H, G, b, n0, nr);
-                  if (nr > 16) ++bad_fields;
-                  for (int j = 0; j < nb; ++j) {
-                    const Job& jb = jobs[j];
-                    if (jb.kind == kGateUp) {
-                      tparts[size_t(jb.slot) * (I / 8) + jb.row0 / 8]++;
-                      if (jb.tile >= max_tiles(T, I, E, k, G) || jb.row0 % 8) ++bad_fields;
-                    } else {
-                      const int u = jb.slot == kSharedSlot ? U : jb.slot;
-                      if (jb.nrows != nr || jb.row0 != n0) ++bad_fields;
-                      for (int r = 0; r < jb.nrows; ++r) outc[size_t(u) * H + jb.row0 + r]++;
-                    }
-                  }
+                  for (int e = 0; e < E; ++e)
+                    if (rows[e] != 1) ++bad_cover;
+                  if (rows[E] != (gate ? 1 : 0)) ++bad_cover;
+                  for (size_t i = 0; i < parts.size(); ++i)
+                    if (parts[i] != 1) ++bad_cover;
+                  for (size_t i = 0; i < outc.size(); ++i)
+                    if (outc[i] != 1) ++bad_cover;
                 }
-                for (int e = 0; e < E; ++e)
-                  if (rows[e] != 1) ++bad_cover;
-                if (rows[E] != (gate ? 1 : 0)) ++bad_cover;
-                const int ns = gu_split(fm, H);
-                for (size_t i = 0; i < tparts.size(); ++i)
-                  if (tparts[i] != ns) ++bad_cover;
-                for (size_t i = 0; i < outc.size(); ++i)
-                  if (outc[i] != 1) ++bad_cover;
               }
               // the workspace the kernel writes: counters after the header,
               // logits [T, E] and h of every slot
