@@ -54,7 +54,6 @@ constexpr int kMaxT = 4;
 constexpr int kMaxK = 16;
 constexpr int kMaxSlots = kMaxT * kMaxK + 1;  // routed slots + the shared expert
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kTopChunk = 128;  // logits per first-round top-k job (4 per lane)
 constexpr int kMaxH = 2048;     // largest hidden size of the fused kernel
 constexpr int kMaxI = 2048;     // largest expert intermediate size
 constexpr int kMaxBias = 64;    // router bias values of one CTA's rows (rows x tokens)
@@ -128,9 +127,9 @@ __host__ __device__ inline int gu_parts(int H) { return H % 512 == 0 ? 2 : 1; }
 // Dynamic shared memory, offsets from the base.
 struct Plan {
   int o_x32;   // fp32 x [T][H] (router input, phase A only)
+  int o_cand;  // top-k candidates of the routing [T][E / 32][k], 8 bytes each (over x32)
   int o_hf;    // per-warp activations of a down job, 2 T I bytes each (phase C; over x32)
   int o_xf;    // 3 activation buffers in fragment order, 2 T H bytes each
-  int o_lg;    // logits [T][E]
   int o_rp;    // router partials [rows][segs][T]
   int o_red;   // gate/up K-split sums [tiles][16][T]
   int o_td;    // gate/up K-split arrivals [tiles]
@@ -153,11 +152,11 @@ __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int
     o += bytes;
     return r;
   };
-  const int x32 = 4 * T * H, hf = kWarps * 2 * T * I;
-  p.o_x32 = take(x32 > hf ? x32 : hf, 16);
+  const int x32 = 4 * T * H, hf = kWarps * 2 * T * I, cand = 8 * T * ((E + 31) / 32) * k;
+  p.o_x32 = take(std::max(x32, std::max(hf, cand)), 16);
+  p.o_cand = p.o_x32;
   p.o_hf = p.o_x32;
   p.o_xf = take(3 * 2 * T * H, 16);
-  p.o_lg = take(4 * T * E, 16);
   p.o_rp = take(4 * (router_rows(E, G) + 1) * (H / router_seg(H)) * T, 16);
   p.o_red = take(4 * max_tiles(T, I, E, k, G) * 16 * T, 16);
   p.o_td = take(4 * max_tiles(T, I, E, k, G), 16);
@@ -283,8 +282,7 @@ __device__ __forceinline__ uint32_t h2fma(uint32_t a, uint32_t b, uint32_t c) {
 __device__ __forceinline__ uint32_t dup16(uint32_t h) { return (h & 0xffffu) | (h << 16); }
 __device__ __forceinline__ void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                     uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -305,6 +303,11 @@ __device__ __forceinline__ uint32_t ldg2(const void* p) {
   unsigned short v;
   asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return uint32_t(v);
+}
+__device__ __forceinline__ uint32_t ldg4(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
 }
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -428,6 +431,13 @@ __device__ __forceinline__ void mma_it(const Ld& L, const uint8_t* bf, int c, in
   const int lane = threadIdx.x & 31, gq = lane >> 2;
   const bool bv = gq < T;
   const uint8_t* bp = bf + (size_t(c) * T + gq) * colbytes(F);
+  // int4: this column's activation fragments first (64 bytes of shared
+  // memory), so their latency overlaps the dequantisation
+  // (int2 and int8 load each word's piece in its turn: fewer registers)
+  constexpr int kNb = F == MOE_Q_INT4_SYM_G32 ? 4 : 1;
+  uint4 bq[kNb];
+#pragma unroll
+  for (int i = 0; i < kNb; ++i) bq[i] = bv ? reinterpret_cast<const uint4*>(bp)[i] : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t wa = word(L.a, j), wb = word(L.b, j);
@@ -435,9 +445,8 @@ __device__ __forceinline__ void mma_it(const Ld& L, const uint8_t* bf, int c, in
       uint32_t pa[4], pb[4];
       deq4(wa, dup16(L.sa.x), pa);
       deq4(wb, dup16(L.sb.x), pb);
-      const uint4 b = bv ? *reinterpret_cast<const uint4*>(bp + j * 16) : make_uint4(0u, 0u, 0u, 0u);
-      mma(acc[0], pa[0], pb[0], pa[1], pb[1], b.x, b.y);
-      mma(acc[1], pa[2], pb[2], pa[3], pb[3], b.z, b.w);
+      mma(acc[0], pa[0], pb[0], pa[1], pb[1], bq[j].x, bq[j].y);
+      mma(acc[1], pa[2], pb[2], pa[3], pb[3], bq[j].z, bq[j].w);
     } else if (F == MOE_Q_INT2_ASYM_G16) {
       uint32_t pa[8], pb[8];
       deq2(wa, dup16(half_of(L.sa, j)), dup16(half_of(L.ma, j)), pa);
@@ -459,7 +468,9 @@ __device__ __forceinline__ void mma_it(const Ld& L, const uint8_t* bf, int c, in
 }
 
 // Iterations of loads in flight per lane (int2 carries 4 scales and 4 mins
-// per row and iteration, so it keeps fewer in registers).
+// per row and iteration, so it keeps fewer in registers). The rows of every
+// job are on their way into L2 since the routing, so these loads mostly wait
+// for L2, not DRAM.
 __host__ __device__ constexpr int depth(int F) { return F == MOE_Q_INT2_ASYM_G16 ? 2 : 4; }
 
 // One warp's share of a tile: iterations it = 0..nit-1, lane column
@@ -498,6 +509,89 @@ __device__ __forceinline__ void run_any(int f, const Rows& R, int col0, int nit,
   acc[1] = v.y;
   acc[2] = v.z;
   acc[3] = v.w;
+}
+
+// int4 tile for T <= 2 tokens with the group scales applied to fp32 sums
+// instead of to every fp16 weight: the A fragments are the exact codes
+// (c - 8), and B column n of the MMA carries only the activations that A
+// lane tq = n & 3 contributes (token n >> 2), so D column n is the sum over
+// group n & 3 of the iteration's four 16-byte columns (one int4 group each).
+// Each lane then scales its two columns by their group scales (loaded as one
+// 32-bit pair) and adds them to fp32 accumulators. Same four results per
+// lane as run_tile. Needs 4-byte aligned scale rows.
+struct Ld4 {
+  uint4 a, b;      // codes of rows gq and gq + 8, this lane's column
+  uint32_t sa, sb;  // fp16 scales of this lane's two D columns, rows gq and gq + 8
+};
+__device__ __forceinline__ void load_i4(const Rows& R, int c, int cs, Ld4& L) {
+  L.a = R.lo ? ldg16(R.c_lo + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.b = R.hi ? ldg16(R.c_hi + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.sa = R.lo ? ldg4(R.s_lo + cs) : 0u;
+  L.sb = R.hi ? ldg4(R.s_hi + cs) : 0u;
+}
+// int4 word -> four fp16 pairs (c - 8), exact, in the order of frag_pos.
+__device__ __forceinline__ void deq4_codes(uint32_t w, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = h2sub(lop_or(w, 0x000F000Fu, 0x64006400u), 0x64086408u);
+  p[1] = h2sub(lop_or(w, 0x00F000F0u, 0x54005400u), 0x54805480u);
+  p[2] = h2sub(lop_or(w8, 0x000F000Fu, 0x64006400u), 0x64086408u);
+  p[3] = h2sub(lop_or(w8, 0x00F000F0u, 0x54005400u), 0x54805480u);
+}
+__device__ __noinline__ float4 run_tile_i4(const Rows R, int col0, int nit, const uint8_t* bf, int T) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const int dt = gq - tq;
+  const bool bv = dt == 0 || (dt == 4 && T == 2);  // B column gq takes A lane tq's activations
+  const int bt = dt == 4 ? 1 : 0;                   // of this token
+  const int g0 = (2 * tq) & 3;                      // groups of this lane's D columns 2 tq, 2 tq + 1
+  constexpr int kDepth = 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  Ld4 L[kDepth];
+#pragma unroll
+  for (int s = 0; s < kDepth; ++s)
+    if (s < nit) load_i4(R, col0 + 4 * s + tq, col0 + 4 * s + g0, L[s]);
+#pragma unroll 1
+  for (int it0 = 0; it0 < nit; it0 += kDepth) {
+#pragma unroll
+    for (int s = 0; s < kDepth; ++s) {
+      const int it = it0 + s;
+      if (it < nit) {
+        const uint4* bp = reinterpret_cast<const uint4*>(bf + (size_t(col0 + 4 * it + tq) * T + bt) * 64);
+        uint4 bq[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bq[j] = bv ? bp[j] : make_uint4(0u, 0u, 0u, 0u);
+        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pa[4], pb[4];
+          deq4_codes(word(L[s].a, j), pa);
+          deq4_codes(word(L[s].b, j), pb);
+          float (&d)[4] = j < 2 ? d0 : d1;
+          mma(d, pa[0], pb[0], pa[1], pb[1], bq[j].x, bq[j].y);
+          mma(d, pa[2], pb[2], pa[3], pb[3], bq[j].z, bq[j].w);
+        }
+        const float2 sa = __half22float2(*reinterpret_cast<const __half2*>(&L[s].sa));
+        const float2 sb = __half22float2(*reinterpret_cast<const __half2*>(&L[s].sb));
+        acc[0] = fmaf(sa.x, d0[0] + d1[0], acc[0]);
+        acc[1] = fmaf(sa.y, d0[1] + d1[1], acc[1]);
+        acc[2] = fmaf(sb.x, d0[2] + d1[2], acc[2]);
+        acc[3] = fmaf(sb.y, d0[3] + d1[3], acc[3]);
+        if (it + kDepth < nit) load_i4(R, col0 + 4 * (it + kDepth) + tq, col0 + 4 * (it + kDepth) + g0, L[s]);
+      }
+    }
+  }
+  // lane (gq, tq) holds groups g0, g0 + 1 of token tq >> 1: add the other
+  // two groups (lane tq ^ 1), then give lane tq = 0 both tokens (token 1
+  // from lane tq = 2), the layout of run_tile (tokens 2 tq, 2 tq + 1)
+  float lo = acc[0] + acc[1], hi = acc[2] + acc[3];
+  lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+  hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+  const float lo1 = __shfl_xor_sync(0xffffffffu, lo, 2), hi1 = __shfl_xor_sync(0xffffffffu, hi, 2);
+  return tq == 0 ? make_float4(lo, lo1, hi, hi1) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+// The int4 path of a tile: run_tile_i4 where it applies, else run_tile.
+__device__ __forceinline__ bool i4_grouped(int f, int T, const Rows& R) {
+  return f == MOE_Q_INT4_SYM_G32 && T <= 2 &&
+         ((reinterpret_cast<uintptr_t>(R.s_lo) | reinterpret_cast<uintptr_t>(R.s_hi)) & 3u) == 0;
 }
 
 // ---------------------------------------------------------------- top-k keys
@@ -611,7 +705,12 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.up.mins + size_t(row) * sper : nullptr;
   const uint8_t* bf = C.smem + C.L.o_xf + (f - 1) * 2 * T * H;  // formats 1..3 -> buffers 0..2
   float acc[4];
-  run_any(f, R, col0, nit, bf, T, acc);
+  if (i4_grouped(f, T, R)) {
+    const float4 v = run_tile_i4(R, col0, nit, bf, T);
+    acc[0] = v.x, acc[1] = v.y, acc[2] = v.z, acc[3] = v.w;
+  } else {
+    run_any(f, R, col0, nit, bf, T, acc);
+  }
   // D rows gq (gate) / gq + 8 (up), tokens 2 tq, 2 tq + 1
   if (ns > 1) {
     float* rs = reinterpret_cast<float*>(C.smem + C.L.o_red) + size_t(jb.tile) * 16 * T;
@@ -664,6 +763,30 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   if (lane == 0) red_release(P.cnt + slot * kCntStride, 1u);
 }
 
+// L2 prefetch of piece w (0..5) of gate/up tile r (intermediate rows
+// 8r .. 8r + 7, whole K) of an expert: 0/1 the gate/up codes, 2/3 their
+// scales, 4/5 their mins (int2).
+__device__ __noinline__ void prefetch_tile_piece(const moe_expert& d, int H, int r, int w) {
+  const moe_qmatrix& m = (w & 1) ? d.up : d.gate;
+  const int f = m.qtype;
+  const int rb = H >> (f == MOE_Q_INT4_SYM_G32 ? 1 : f == MOE_Q_INT2_ASYM_G16 ? 2 : 0);
+  const int sper = f == MOE_Q_INT8_PER_CHANNEL ? 1 : H >> (f == MOE_Q_INT4_SYM_G32 ? 5 : 4);
+  const size_t row = size_t(8) * r;
+  if (w < 2) prefetch_l2(m.codes + row * rb, uint32_t(8 * rb));
+  else if (w < 4) prefetch_l2(m.scales + row * sper, uint32_t(16 * sper));
+  else if (f == MOE_Q_INT2_ASYM_G16) prefetch_l2(m.mins + row * sper, uint32_t(16 * sper));
+}
+// L2 prefetch of output rows [n0, n0 + nr) of a down matrix: piece 0 codes,
+// 1 scales, 2 mins (int2).
+__device__ __noinline__ void prefetch_down_piece(const moe_qmatrix& m, int I, int n0, int nr, int w) {
+  const int f = m.qtype;
+  const int rb = I >> (f == MOE_Q_INT4_SYM_G32 ? 1 : f == MOE_Q_INT2_ASYM_G16 ? 2 : 0);
+  const int sper = f == MOE_Q_INT8_PER_CHANNEL ? 1 : I >> (f == MOE_Q_INT4_SYM_G32 ? 5 : 4);
+  if (w == 0) prefetch_l2(m.codes + size_t(n0) * rb, uint32_t(nr * rb));
+  else if (w == 1) prefetch_l2(m.scales + size_t(n0) * sper, uint32_t(nr * sper * 2));
+  else if (m.qtype == MOE_Q_INT2_ASYM_G16) prefetch_l2(m.mins + size_t(n0) * sper, uint32_t(nr * sper * 2));
+}
+
 // h of one expert (fp32 [T][I] in the workspace) into a warp's activation
 // buffer in format F's fragment order, scaled by 2^-eh[t] per token; 8 loads
 // per lane in flight at a time.
@@ -712,6 +835,9 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.down.mins + size_t(R.hi ? rhi : 0) * sper : nullptr;
   uint8_t* hf = C.smem + C.L.o_hf + warp * 2 * T * I;
   __shared__ int s_eh[kWarps][kMaxT];
+  // this job's rows into L2 while its expert's gate/up tiles finish (the
+  // shared expert's are there since phase A)
+  if (slot != kSharedSlot && lane < 3) prefetch_down_piece(d.down, I, jb.row0, jb.nrows, lane);
   int ok = 1;
   if (lane == 0)
     ok = wait_counter(P.cnt + slot * kCntStride, uint32_t(I / 8), P.hdr, P.wait_cycles, 7100000 + slot) ? 1 : 0;
@@ -729,7 +855,12 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   else h_to_frag<MOE_Q_INT8_PER_CHANNEL>(hs, T, I, s_eh[warp], hf);
   __syncwarp();
   float acc[4];
-  run_any(f, R, 0, nit, hf, T, acc);
+  if (i4_grouped(f, T, R)) {
+    const float4 v = run_tile_i4(R, 0, nit, hf, T);
+    acc[0] = v.x, acc[1] = v.y, acc[2] = v.z, acc[3] = v.w;
+  } else {
+    run_any(f, R, 0, nit, hf, T, acc);
+  }
   float* y = reinterpret_cast<float*>(C.smem + C.L.o_y) + size_t(slot) * 16 * T;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -811,104 +942,92 @@ __device__ __noinline__ void job_router(Ctx& C, const Job jb, const uint4 w0, co
 
 // ---------------------------------------------------------------- routing
 // Routing of one CTA, by all its warps once phase A is done: wait for every
-// CTA's logits, top-k per token (first the best k of each 128-logit chunk,
-// one warp per (token, chunk), then the best k of those, one warp per
-// token), gates, the distinct picked experts in ascending id order (slots),
-// their descriptors, and the L2 prefetch of this CTA's gate/up parts and
-// down rows of every picked expert. Returns whether phases B and C run (the
-// same answer on every CTA: identical inputs, identical code).
+// CTA's logits; top-k per token in two rounds (each warp sorts 32-logit
+// chunks and keeps the best k of each; then every kept candidate's rank
+// among its token's candidates, the best k by rank); gates; the distinct
+// picked experts in ascending id order (slots) and their descriptors.
+// Returns whether phases B and C run (the same answer on every CTA:
+// identical inputs, identical code).
 struct RouteShared {
   int idx[kMaxT * kMaxK];
   float w[kMaxT * kMaxK];
   uint32_t key[kMaxT * kMaxK];
-  int slot[kMaxT * kMaxK];         // (t, j) -> slot
-  int uniq[kMaxT * kMaxK];         // slot -> expert id
-  uint32_t ck[kMaxT * 8 * kMaxK];  // first-round winners [t][chunk][k]
-  int ci[kMaxT * 8 * kMaxK];
+  int slot[kMaxT * kMaxK];  // (t, j) -> slot
+  int uniq[kMaxT * kMaxK];  // slot -> expert id
   uint32_t bits[kMaxE / 32];
-  uint32_t bpre[kMaxE / 32];
+  uint32_t bpre[kMaxE / 32];  // set bits in the words before
   int U, bad;
 };
 
-// L2 prefetch of the rows of one gate/up job's K part: lane r < 16 takes A
-// row r (gate rows 0-7, up rows 8-15): its codes and its scales (and mins).
-__device__ __forceinline__ void prefetch_gate_up(const moe_expert& d, const Job& jb, int H, int r) {
-  const moe_qmatrix& m = r < 8 ? d.gate : d.up;
-  const int f = m.qtype, ns = gu_parts(H);
-  const int ncol = H / kc(f) / ns, col0 = jb.part * ncol, row = jb.row0 + (r & 7);
-  prefetch_l2(m.codes + size_t(row) * row_code_bytes(f, H) + size_t(col0) * 16, uint32_t(ncol * 16));
-  if (f == MOE_Q_INT4_SYM_G32) {
-    prefetch_l2(m.scales + size_t(row) * (H / 32) + col0, uint32_t(ncol * 2));
-  } else if (f == MOE_Q_INT2_ASYM_G16) {
-    prefetch_l2(m.scales + size_t(row) * (H / 16) + 4 * col0, uint32_t(ncol * 8));
-    prefetch_l2(m.mins + size_t(row) * (H / 16) + 4 * col0, uint32_t(ncol * 8));
-  }
-}
-// L2 prefetch of output rows [n0, n0 + nr) of a down matrix.
-__device__ __forceinline__ void prefetch_down(const moe_qmatrix& m, int I, int n0, int nr) {
-  const int rb = row_code_bytes(m.qtype, I);
-  prefetch_l2(m.codes + size_t(n0) * rb, uint32_t(nr * rb));
-  const int sper = m.qtype == MOE_Q_INT8_PER_CHANNEL ? 1 : I / (m.qtype == MOE_Q_INT4_SYM_G32 ? 32 : 16);
-  prefetch_l2(m.scales + size_t(n0) * sper, uint32_t(nr * sper * 2));
-  if (m.qtype == MOE_Q_INT2_ASYM_G16) prefetch_l2(m.mins + size_t(n0) * sper, uint32_t(nr * sper * 2));
+// Bitonic sort of 32 keys, one per lane, into descending lane order.
+__device__ __forceinline__ uint64_t warp_sort32_desc(uint64_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+      // the lower lane of a pair keeps the larger key in a descending run
+      const bool keep_max = ((lane & size) == 0) == ((lane & stride) == 0);
+      v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  return v;
 }
 
 __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) {
   const Params& P = *C.P;
-  const int T = C.T, E = C.E, k = C.k, H = C.H, I = C.I;
+  const int T = C.T, E = C.E, k = C.k, H = C.H, I = C.I, G = C.G, b = C.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    if (!wait_counter(&P.hdr->bar_count, uint32_t(C.G), P.hdr, P.wait_cycles, 7000000 + C.b)) C.fail = 1;
+    if (!wait_counter(&P.hdr->bar_count, uint32_t(G), P.hdr, P.wait_cycles, 7000000 + b)) C.fail = 1;
   }
   if (threadIdx.x < kMaxE / 32) R.bits[threadIdx.x] = 0u;
   __syncthreads();
   const bool live = !C.fail;
-  float* lg = reinterpret_cast<float*>(C.smem + C.L.o_lg);
-  if (live) {
-    // T E <= kMaxT kMaxE logits, all of a thread's loads in flight together
-    constexpr int kPer = kMaxT * kMaxE / kThreads;
-    float v[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int i = threadIdx.x + j * kThreads;
-      v[j] = i < T * E ? __ldcg(P.logits + i) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j)
-      if (threadIdx.x + j * kThreads < T * E) lg[threadIdx.x + j * kThreads] = v[j];
-  }
-  __syncthreads();
-  // first round: the best k of each (token, chunk)
-  const int nch = (E + kTopChunk - 1) / kTopChunk;
+  // first round: chunk ch of token t = logits [32 ch, 32 ch + 32); CTA 0 also
+  // exports the logits
+  const int n32 = (E + 31) / 32, nc = n32 * k;
+  uint64_t* cand = reinterpret_cast<uint64_t*>(C.smem + C.L.o_cand);  // [T][n32][k]
   if (live)
-    for (int q = warp; q < T * nch; q += kWarps) {
-      const int t = q / nch, ch = q - t * nch;
-      const int nc = min(kTopChunk, E - ch * kTopChunk);
-      uint64_t c[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int cc = lane + 32 * i;
-        const uint32_t key = cc < nc ? f2key(lg[t * E + ch * kTopChunk + cc]) : 0u;
-        c[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(ch * kTopChunk + cc)) : 0ull;
+    for (int q = warp; q < T * n32; q += kWarps) {
+      const int t = q / n32, e = (q - t * n32) * 32 + lane;
+      uint64_t v = 0ull;
+      if (e < E) {
+        const float l = __ldcg(P.logits + size_t(t) * E + e);
+        if (b == 0 && P.logits_out) P.logits_out[size_t(t) * E + e] = l;
+        v = (uint64_t(f2key(l)) << 32) | uint64_t(~uint32_t(e));  // key descending, then id ascending
       }
-      warp_topk(c[0], c[1], c[2], c[3], k, R.ck + (t * 8 + ch) * kMaxK, R.ci + (t * 8 + ch) * kMaxK);
+      v = warp_sort32_desc(v);
+      if (lane < k) cand[size_t(q) * k + lane] = v;
     }
   __syncthreads();
-  // second round (one warp per token): the best k of the chunks' winners,
-  // then the gates: the softmax over all logits restricted to the picks and
-  // renormalised = a softmax over the picked logits (of the unbiased ones when
-  // the bias only selects)
-  if (live && warp < T) {
-    const int t = warp, nc = nch * k;  // <= 128 candidates, 4 per lane
-    uint64_t c[4];
+  // second round: a candidate's rank among its token's candidates (keys are
+  // distinct: the low word is the id); the best k go to their rank's place
+  if (live)
+    for (int q = threadIdx.x; q < T * nc; q += kThreads) {
+      const int t = q / nc;
+      const uint64_t v = cand[q];
+      if (v == 0ull) continue;  // no logit (chunk past E)
+      const uint64_t* c = cand + size_t(t) * nc;
+      int rank = 0;
+      for (int j = 0; j < nc; j += 8) {  // 8 loads in flight, then 8 compares
+        uint64_t w[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int cc = lane + 32 * i, ch = cc / k, j = cc - ch * k;
-      const uint32_t key = cc < nc ? R.ck[(t * 8 + ch) * kMaxK + j] : 0u;
-      c[i] = key ? (uint64_t(key) << 32) | uint64_t(~uint32_t(R.ci[(t * 8 + ch) * kMaxK + j])) : 0ull;
+        for (int u = 0; u < 8; ++u) w[u] = j + u < nc ? c[j + u] : 0ull;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) rank += w[u] > v ? 1 : 0;
+      }
+      if (rank < k) {
+        R.key[t * k + rank] = uint32_t(v >> 32);
+        R.idx[t * k + rank] = int(~uint32_t(v));
+      }
     }
-    warp_topk(c[0], c[1], c[2], c[3], k, R.key + t * k, R.idx + t * k);
-    __syncwarp();
+  __syncthreads();
+  // gates (one warp per token): the softmax over all logits restricted to the
+  // picks and renormalised = a softmax over the picked logits (of the
+  // unbiased ones when the bias only selects)
+  if (live && warp < T) {
+    const int t = warp;
     const bool sel_only = (P.flags & MOE_BIAS_SELECTION_ONLY) != 0;
     float v = -CUDART_INF_F;
     if (lane < k) v = sel_only ? __ldcg(P.logits_u + size_t(t) * E + R.idx[t * k + lane]) : key2f(R.key[t * k + lane]);
@@ -925,40 +1044,35 @@ __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) 
     }
   }
   __syncthreads();
-  // slots: the slot of an id = set bits below it (warp scan over the bitmap)
+  moe_expert* desc = C.desc;
   if (warp == 0) {
-    uint32_t pre = 0;
-#pragma unroll 1
-    for (int i = 0; i < kMaxE / 32 / 32; ++i) {
-      const uint32_t c = __popc(R.bits[i * 32 + lane]);
-      uint32_t inc = c;
+    // slots: the slot of an id = set bits below it (warp scan over the bitmap)
+    static_assert(kMaxE / 32 == 32, "one bitmap word per lane");
+    const uint32_t c = __popc(R.bits[lane]);
+    uint32_t inc = c;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      R.bpre[i * 32 + lane] = pre + inc - c;
-      pre += __shfl_sync(0xffffffffu, inc, 31);
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
     }
+    R.bpre[lane] = inc - c;
     __syncwarp();
-    if (live && !R.bad)
+    if (live && R.bad == 0)
       for (int i = lane; i < T * k; i += 32) {
         const int id = R.idx[i], wd = id >> 5;
         const int rank = int(R.bpre[wd] + __popc(R.bits[wd] & ((1u << (id & 31)) - 1u)));
         R.slot[i] = rank;
         R.uniq[rank] = id;
       }
-    if (lane == 0) R.U = int(pre);
+    if (lane == 31) R.U = int(inc);
   }
   __syncthreads();
   const int U = R.U;
-  const bool ok = live && R.bad == 0;
-  // descriptors of the picked experts (the table is in L2 since the entry),
-  // all of a thread's loads in flight together
-  moe_expert* desc = C.desc;
+  // descriptors of the picked experts (the table is in L2 since the entry):
+  // U W <= kMaxT kMaxK W words over all threads, loads first
   constexpr int W = int(sizeof(moe_expert) / 4);
-  if (ok) {
-    constexpr int kPer = (kMaxT * kMaxK * W + kThreads - 1) / kThreads;
+  constexpr int kPer = (kMaxT * kMaxK * W + kThreads - 1) / kThreads;
+  if (live && R.bad == 0) {
     const uint32_t* src = reinterpret_cast<const uint32_t*>(P.experts);
     uint32_t* dst = reinterpret_cast<uint32_t*>(desc);
     uint32_t v[kPer];
@@ -972,22 +1086,10 @@ __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) 
       if (threadIdx.x + j * kThreads < U * W) dst[threadIdx.x + j * kThreads] = v[j];
   }
   __syncthreads();
-  if (ok && warp == 0)
-    for (int u = lane; u < U; u += 32)
-      if (!expert_ok(desc[u], H, I)) R.bad = 1;
+  if (live && R.bad == 0 && threadIdx.x < U && !expert_ok(desc[threadIdx.x], H, I)) R.bad = 1;
   __syncthreads();
-  const bool work = ok && R.bad == 0;
+  const bool work = live && R.bad == 0;
   if (live && !work && threadIdx.x == 0) flag_error(P.hdr, MOE_ERR_DEVICE_FAULT, 1000000);
-  if (work) {
-    // this CTA's routed gate/up parts (16 rows each) and down rows into L2
-    const int ngu = gu_parts(H) * bc_tiles(I, C.G, C.b, U + (has_shared ? 1 : 0));
-    for (int q = threadIdx.x; q < ngu * 16; q += kThreads) {
-      const Job jb = phase_bc_job(H, I, C.G, C.b, U, has_shared, q >> 4);
-      if (jb.slot != kSharedSlot) prefetch_gate_up(desc[jb.slot], jb, H, q & 15);
-    }
-    if (C.nr > 0)
-      for (int u = threadIdx.x; u < U; u += kThreads) prefetch_down(desc[u].down, I, C.n0, C.nr);
-  }
   return work;
 }
 
@@ -1107,16 +1209,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
     flag_error(hdr, MOE_ERR_DEVICE_FAULT, 2000000);
   }
   __syncthreads();
-  if (has_shared && !s_bad) {
-    // the shared expert's gate/up parts of this CTA and its down rows into
-    // L2: needed whatever the routing
-    const int nsh = gu_parts(H) * bc_tiles(I, G, b, 1);  // its tiles come first in the B/C list
-    for (int q = threadIdx.x; q < nsh * 16; q += kThreads)
-      prefetch_gate_up(desc[kSharedSlot], phase_bc_job(H, I, G, b, 0, true, q >> 4), H, q & 15);
-    if (threadIdx.x == kThreads - 1 && C.nr > 0) prefetch_down(desc[kSharedSlot].down, I, C.n0, C.nr);
+  if (nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
+  __syncthreads();
+
+  // ---------------------------------------------------------- phase A
+  for (int j = warp; j < nA; j += kWarps) {
+    const Job jb = phase_a_job(H, j);
+    uint4 w[4] = {};
+    if (j == warp) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = w0[i];
+    } else {
+      router_load(P, e0, nreal, seg, jb, w);
+    }
+    job_router(C, jb, w[0], w[1], w[2], w[3]);
   }
-  // activations in fragment order for all three formats, so routed experts
-  // of any format need no further barrier
+  // While the grid gathers the logits: the shared expert's gate/up tiles of
+  // this CTA and its down rows into L2 (needed whatever the routing), and the
+  // activations in fragment order for all three formats (so routed experts
+  // of any format need no further barrier).
+  if (has_shared && !s_bad) {
+    const int nsh = bc_tiles(I, G, b, 1);  // its tiles come first in the B/C list
+    for (int q = threadIdx.x; q < nsh * 6; q += kThreads)
+      prefetch_tile_piece(desc[kSharedSlot], H, b + G * (q / 6), q % 6);
+    if (C.nr > 0 && threadIdx.x >= kThreads - 3)
+      prefetch_down_piece(desc[kSharedSlot].down, I, C.n0, C.nr, threadIdx.x - (kThreads - 3));
+  }
 #pragma unroll
   for (int j = 0; j < kXg; ++j) {
     const int g = threadIdx.x + j * kThreads;
@@ -1135,21 +1253,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
       store4<MOE_Q_INT8_PER_CHANNEL>(xf + 4 * T * H, k0, t, T, v[0], v[1], v[2], v[3]);
       store4<MOE_Q_INT8_PER_CHANNEL>(xf + 4 * T * H, k0 + 4, t, T, v[4], v[5], v[6], v[7]);
     }
-  }
-  if (nrr == 0 && threadIdx.x == 0) red_release(&hdr->bar_count, 1u);  // no router rows: arrive at once
-  __syncthreads();
-
-  // ---------------------------------------------------------- phase A
-  for (int j = warp; j < nA; j += kWarps) {
-    const Job jb = phase_a_job(H, j);
-    uint4 w[4] = {};
-    if (j == warp) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] = w0[i];
-    } else {
-      router_load(P, e0, nreal, seg, jb, w);
-    }
-    job_router(C, jb, w[0], w[1], w[2], w[3]);
   }
 
   // ---------------------------------------------------------- routing
@@ -1186,10 +1289,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
         P.topk_idx[i] = R.idx[i];
         P.topk_w[i] = R.w[i];
         if (P.heat) atomicAdd(P.heat + R.idx[i], 1u);
-      }
-      if (P.logits_out) {
-        const float* lg = reinterpret_cast<const float*>(smem + L.o_lg);
-        for (int i = threadIdx.x; i < T * E; i += kThreads) P.logits_out[i] = lg[i];
       }
     }
   }

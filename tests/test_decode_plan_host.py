@@ -75,7 +75,7 @@ int main() {
               if (!eligible_on(T, H, I, E, k, G)) continue;
               ++eligible;
               const Plan p = make_plan(T, H, I, E, k, G);
-              const int offs[] = {p.o_x32, p.o_hf, p.o_xf, p.o_lg, p.o_rp, p.o_red, p.o_td, p.o_y, p.o_desc};
+              const int offs[] = {p.o_x32, p.o_cand, p.o_hf, p.o_xf, p.o_rp, p.o_red, p.o_td, p.o_y, p.o_desc};
               for (int o : offs)
                 if (o % 16) ++bad_plan;
               if (p.total + kStaticSmem > kSmemLimit) ++bad_plan;
