@@ -108,6 +108,14 @@ moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, in
     return cuda_status(launch_grouped_ffn(x, T, H, I, k, E, perm_src, offsets, counts, experts_dev, nullptr, nullptr,
                                           y_perm, nullptr, ws_at<void>(ws, L.gemm), ws_at<WsHeader>(ws, 0),
                                           static_cast<cudaStream_t>(stream)));
+  // decode sizes: the fused decode kernel's expert phases on the given routing
+  if (decode_fused_eligible(T, H, I, E, k))
+    return cuda_status(launch_decode_fused(x, T, H, I, E, k, nullptr, nullptr, 0, experts_dev, nullptr, nullptr,
+                                           nullptr, nullptr, nullptr, ws_at<float>(ws, L.logits),
+                                           ws_at<float>(ws, L.dh), ws_at<uint32_t>(ws, L.dcnt),
+                                           ws_at<WsHeader>(ws, 0), wait_cycles(), 0u, nullptr,
+                                           ws_at<float>(ws, L.logits_u), ws_at<float>(ws, L.sgate), nullptr, perm_src,
+                                           offsets, counts, y_perm, static_cast<cudaStream_t>(stream)));
   return cuda_status(launch_expert_ffn(x, T, H, I, k, E, perm_src, offsets, counts, experts_dev, false,
                                        ws_at<float>(ws, L.h), ws_at<int>(ws, L.active), y_perm, nullptr,
                                        ws_at<WsHeader>(ws, 0), static_cast<cudaStream_t>(stream)));
@@ -173,7 +181,8 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
                                            topk_idx, topk_w, logits_out, out, ws_at<float>(ws, L.logits),
                                            ws_at<float>(ws, L.dh), ws_at<uint32_t>(ws, L.dcnt), hdr,
                                            wait_cycles(), flags, gate, ws_at<float>(ws, L.logits_u),
-                                           ws_at<float>(ws, L.sgate), opts ? opts->heat : nullptr, st));
+                                           ws_at<float>(ws, L.sgate), opts ? opts->heat : nullptr, nullptr, nullptr,
+                                           nullptr, nullptr, st));
   int* counts = ws_at<int>(ws, L.counts);
   int* offsets = ws_at<int>(ws, L.offsets);
   int* perm = ws_at<int>(ws, L.perm);

@@ -252,6 +252,13 @@ struct Params {
   float* logits_u;           // [T][E] unbiased logits (selection-only bias)
   float* sgate;              // [T] shared_gate . x
   uint32_t* heat;            // [E] routing heat, or null
+  // Experts only (the moe_expert_ffn call at decode sizes): the routing is
+  // given as dispatch arrays, nothing is routed or combined, and every
+  // dispatched row's expert output goes to y_perm. Null otherwise.
+  const int* perm_src;  // [T k] token * k + pick of each row
+  const int* offsets;   // [E + 1] first row of each expert
+  const int* counts;    // [E] rows of each expert
+  uint16_t* y_perm;     // bf16 [T k, H]
 };
 
 // ---------------------------------------------------------------- PTX bits
@@ -978,12 +985,21 @@ __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) 
   const Params& P = *C.P;
   const int T = C.T, E = C.E, k = C.k, H = C.H, I = C.I, G = C.G, b = C.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
+  const bool given = P.counts != nullptr;  // experts only: the picks are the dispatched experts
+  if (threadIdx.x == 0 && !given) {
     if (!wait_counter(&P.hdr->bar_count, uint32_t(G), P.hdr, P.wait_cycles, 7000000 + b)) C.fail = 1;
   }
   if (threadIdx.x < kMaxE / 32) R.bits[threadIdx.x] = 0u;
   __syncthreads();
   const bool live = !C.fail;
+  if (given) {
+    // the experts with rows (at most T k of them, each used by at most T rows)
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      const int c = __ldg(P.counts + e);
+      if (c < 0 || c > T) R.bad = 1;
+      else if (c > 0) atomicOr(&R.bits[e >> 5], 1u << (e & 31));
+    }
+  } else {
   // first round: chunk ch of token t = logits [32 ch, 32 ch + 32); CTA 0 also
   // exports the logits
   const int n32 = (E + 31) / 32, nc = n32 * k;
@@ -1043,6 +1059,7 @@ __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) 
       else R.bad = 1;
     }
   }
+  }
   __syncthreads();
   moe_expert* desc = C.desc;
   if (warp == 0) {
@@ -1056,18 +1073,26 @@ __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) 
       if (lane >= o) inc += y;
     }
     R.bpre[lane] = inc - c;
-    __syncwarp();
-    if (live && R.bad == 0)
-      for (int i = lane; i < T * k; i += 32) {
-        const int id = R.idx[i], wd = id >> 5;
-        const int rank = int(R.bpre[wd] + __popc(R.bits[wd] & ((1u << (id & 31)) - 1u)));
-        R.slot[i] = rank;
-        R.uniq[rank] = id;
-      }
-    if (lane == 31) R.U = int(inc);
+    if (lane == 31) {
+      R.U = int(inc);
+      if (int(inc) > T * k) R.bad = 1;  // more experts than rows (experts only: bad counts)
+    }
   }
   __syncthreads();
   const int U = R.U;
+  if (live && R.bad == 0) {
+    // slot of an expert = picked experts below it; routing: slot of each pick
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+      const uint32_t wb = R.bits[e >> 5];
+      if ((wb >> (e & 31)) & 1u) R.uniq[R.bpre[e >> 5] + __popc(wb & ((1u << (e & 31)) - 1u))] = e;
+    }
+    if (!given)
+      for (int i = threadIdx.x; i < T * k; i += kThreads) {
+        const int id = R.idx[i], wd = id >> 5;
+        R.slot[i] = int(R.bpre[wd] + __popc(R.bits[wd] & ((1u << (id & 31)) - 1u)));
+      }
+  }
+  __syncthreads();
   // descriptors of the picked experts (the table is in L2 since the entry):
   // U W <= kMaxT kMaxK W words over all threads, loads first
   constexpr int W = int(sizeof(moe_expert) / 4);
@@ -1107,6 +1132,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   WsHeader* hdr = P.hdr;
   const bool has_shared = P.shared != nullptr;
   const bool gate_row = P.shared_gate != nullptr && has_shared;
+  const bool given = P.counts != nullptr;  // experts only: no router, no combine
   const Plan& L = P.L;
 
   // ---------------------------------------------------------- loads first
@@ -1117,7 +1143,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   int e0, nreal;
   router_range(E, G, b, e0, nreal);
   const int seg = router_seg(H), nseg = H / seg;
-  const int nrr = router_rows_of(E, G, b, gate_row);
+  const int nrr = given ? 0 : router_rows_of(E, G, b, gate_row);
   const int nA = nrr * nseg;
   uint4 w0[4] = {};
   if (warp < nA) router_load(P, e0, nreal, seg, phase_a_job(H, warp), w0);
@@ -1271,7 +1297,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
   __syncthreads();
 
   // ---------------------------------------------------------- combine
-  if (work && !C.fail) {
+  if (work && !C.fail && given) {
+    // experts only: this CTA's columns [n0, n0 + nr) of every dispatched row,
+    // rounded once to bf16 (the rows of an expert are [offsets[e],
+    // offsets[e] + counts[e]); a row's token is perm_src / k)
+    const float* Y = reinterpret_cast<const float*>(smem + L.o_y);
+    const int nr = C.nr, n0 = C.n0, U = R.U;
+    for (int r = threadIdx.x; r < T * k; r += kThreads) R.slot[r] = -1;
+    __syncthreads();
+    for (int u = threadIdx.x; u < U; u += kThreads) {
+      const int e = R.uniq[u], r0 = __ldg(P.offsets + e), c = __ldg(P.counts + e);
+      for (int j = 0; j < c; ++j)
+        if (r0 + j >= 0 && r0 + j < T * k) R.slot[r0 + j] = u;
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < T * k * nr; q += kThreads) {
+      const int r = q / nr, i = q - r * nr;
+      const int u = R.slot[r], ps = __ldg(P.perm_src + r), t = ps / k;
+      if (u >= 0 && ps >= 0 && t < T) P.y_perm[size_t(r) * H + n0 + i] = f32_to_bf16_rn(Y[(u * 16 + i) * T + t]);
+    }
+  } else if (work && !C.fail) {
     const float* Y = reinterpret_cast<const float*>(smem + L.o_y);
     const int nr = C.nr, n0 = C.n0;
     for (int i = threadIdx.x; i < T * nr; i += kThreads) {
@@ -1345,7 +1390,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
                                 long long wait_cycles, uint32_t flags, const float* shared_gate, float* logits_u_ws,
-                                float* sgate_ws, uint32_t* heat, cudaStream_t st) {
+                                float* sgate_ws, uint32_t* heat, const int32_t* perm_src, const int32_t* offsets,
+                                const int32_t* counts, uint16_t* y_perm, cudaStream_t st) {
   using namespace dfx;
   const int grid = grid_size();
   const size_t smem = size_t(make_plan(T, H, I, E, k, grid).total);
@@ -1364,7 +1410,7 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
   Params P{make_plan(T, H, I, E, k, grid), x, T, H, I, E, k, w_router, bias,
            bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
            logits_ws, h_ws, counters, wait_cycles, flags, shared_gate, logits_u_ws,
-           sgate_ws, heat};
+           sgate_ws, heat, perm_src, offsets, counts, y_perm};
   void* args[] = {&P};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(decode_fused_kernel), dim3(grid), dim3(kThreads), args,
                                   smem, st);

@@ -60,12 +60,16 @@ cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, 
 bool decode_fused_eligible(int T, int H, int I, int E, int k);
 // flags: MOE_BIAS_SELECTION_ONLY (then logits_u_ws [T][E] holds the unbiased
 // logits); shared_gate: fp32 [H] or NULL (then sgate_ws [T] holds g . x).
+// perm_src/offsets/counts/y_perm non-null: experts only (moe_expert_ffn):
+// the dispatched experts run on every row and write bf16 y_perm rows;
+// w_router, shared, topk_idx, topk_w, out are then unused (may be null).
 cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
                                 const float* bias, long long bstride, const moe_expert* experts,
                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
                                 uint16_t* out, float* logits_ws, float* h_ws, uint32_t* counters, WsHeader* hdr,
                                 long long wait_cycles, uint32_t flags, const float* shared_gate, float* logits_u_ws,
-                                float* sgate_ws, uint32_t* heat, cudaStream_t st);
+                                float* sgate_ws, uint32_t* heat, const int32_t* perm_src, const int32_t* offsets,
+                                const int32_t* counts, uint16_t* y_perm, cudaStream_t st);
 constexpr long long kDefaultWaitCycles = 2000000000LL;  // about 1 s at the B200's clock
 // The budget (SM clock cycles) every bounded wait of the fused decode launch
 // gets: kDefaultWaitCycles unless moe_set_wait_cycles changed it.

@@ -135,6 +135,6 @@ extern "C" moe_status moe_layer_decode_noalloc(const uint16_t* x, int32_t T, int
       x, T, H, I, E, k, w_router, bias, bias_row_stride, experts_dev, shared_dev, topk_idx, topk_w, logits_out, out,
       moe::ws_at<float>(base, off_logits), moe::ws_at<float>(base, off_h), moe::ws_at<uint32_t>(base, off_counters),
       moe::ws_at<moe::WsHeader>(base, 0), moe::wait_cycles(), flags, gate, moe::ws_at<float>(base, off_logits_u),
-      moe::ws_at<float>(base, off_sgate), opts ? opts->heat : nullptr, st);
+      moe::ws_at<float>(base, off_sgate), opts ? opts->heat : nullptr, nullptr, nullptr, nullptr, nullptr, st);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -176,7 +176,11 @@ moe_status moe_dispatch(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E
  *   y_perm      bf16 [T*k, H] out: row r = expert(r) applied to token
  *               perm_src[r] / k, accumulated in fp32, rounded once to bf16
  * Malformed descriptors of a used expert flag MOE_ERR_DEVICE_FAULT and
- * their rows are left unwritten.
+ * their rows are left unwritten. Decode sizes (1 <= T <= 4, H and I
+ * multiples of 256 up to 2048) run as one cooperative launch of the decode
+ * kernel's expert phases: there a malformed descriptor or counts that do not
+ * fit T tokens leave every row unwritten, and an expired bounded wait leaves
+ * MOE_ERR_TIMEOUT (reset the workspace with moe_reset_status after either).
  */
 moe_status moe_expert_ffn(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t k, int32_t E,
                           const int32_t* perm_src, const int32_t* offsets, const int32_t* counts,
