@@ -35,7 +35,7 @@ constexpr size_t kWsResetBytes = 256 + kDecodeCounterBytes;
 
 // Offsets (bytes from the workspace base) of every workspace segment.
 struct WsLayout {
-  size_t dcnt, counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, logits_u, sgate, partial, h, dh,
+  size_t dcnt, counts, offsets, perm, inv, hist, active, topk_idx, topk_w, logits, logits_u, sgate, h, dh,
       shared_y, y_perm, gemm, router;
   size_t total;
 };
@@ -63,11 +63,7 @@ inline WsLayout ws_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k)
   L.logits = take(4 * T * E);
   L.logits_u = take(4 * T * E);  // unbiased logits (bias used for the selection only)
   L.sgate = take(4 * T);         // the shared expert's per-token sigmoid gate
-  L.partial = take(16 * T * E);  // router partial sums of the fused decode path
-  // fp32 intermediate rows of the multi-launch path, or the decode step's fp16
-  // activations in fragment order: (T k + 1) buffers of I/16 k-steps x T x 32 B
-  const int64_t h32 = 4 * (n + T) * I, hfrag = T <= 4 ? (n + 1) * (I / 16) * T * 32 : 0;
-  L.h = take(size_t(h32 > hfrag ? h32 : hfrag));
+  L.h = take(size_t(4 * (n + T) * I));  // fp32 intermediate rows of the multi-launch path
   L.dh = take(T >= 1 && T <= 4 ? decode_fused_ws_bytes(int(T), int(I)) : 0);  // fused decode: h per expert slot
   L.shared_y = take(4 * T * H);
   L.y_perm = take(4 * n * H);  // fp32 routed rows inside moe_layer

@@ -43,16 +43,6 @@ cudaError_t launch_expert_ffn(const uint16_t* x, int T, int H, int I, int k, int
                               float* h_ws, int* active_ws, uint16_t* y_bf16, float* y_f32, WsHeader* hdr,
                               cudaStream_t st);
 
-// Decode step (T <= 4) as one persistent cooperative launch; see
-// decode_stream.cu. hfrag: decode_stream_hfrag_bytes of scratch for the
-// intermediate activations (fp16, in the order the down tiles read them).
-bool decode_stream_eligible(int T, int H, int I, int E, int k);
-size_t decode_stream_hfrag_bytes(int T, int I, int k);
-cudaError_t launch_decode_stream(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
-                                 const float* bias, long long bstride, const moe_expert* experts,
-                                 const moe_expert* shared, int* topk_idx, float* topk_w, float* logits_out,
-                                 uint16_t* out, float* partial, void* hfrag, WsHeader* hdr, cudaStream_t st);
-
 // Decode step (T <= 4) as one cooperative launch whose warps stream weights
 // into registers; see decode_fused.cu. logits_ws: fp32 [T][E]; h_ws:
 // decode_fused_ws_bytes; counters: kDecodeCounterBytes, zero at launch.

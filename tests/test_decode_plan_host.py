@@ -138,7 +138,7 @@ int main() {
               // logits [T, E] and h of every slot
               const WsLayout L = ws_layout(T, H, I, E, k);
               if (L.dcnt != 256 || size_t(kMaxSlots) * kCntStride * 4 > kDecodeCounterBytes ||
-                  L.counts < L.dcnt + kDecodeCounterBytes || L.partial - L.logits < size_t(4) * T * E ||
+                  L.counts < L.dcnt + kDecodeCounterBytes || L.logits_u - L.logits < size_t(4) * T * E ||
                   L.shared_y - L.dh < decode_fused_ws_bytes(T, I) || L.dh % 256 || L.logits % 256)
                 ++bad_ws;
             }
