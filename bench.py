@@ -47,7 +47,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captures summarised in profiles/ (None while no capture of the current
 # kernel exists).
 NCU_TRAFFIC = {
-    "decode1": (None, "profiles/decode_stream_decode1.md"),
+    # decode_fused_kernel of one step (dram read + write of one launch)
+    "decode1": (33783296, "profiles/decode_fused_decode1.md"),
     # predequant_kernel + grouped_gemm_kernel<gate/up> + <down> of one step
     # (the gather of the activations is not included)
     "prefill8k": (2863281328, "profiles/grouped_gemm_prefill8k.md"),
