@@ -153,7 +153,8 @@ __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int
     return r;
   };
   const int x32 = 4 * T * H, hf = kWarps * 2 * T * I, cand = 8 * T * ((E + 31) / 32) * k;
-  p.o_x32 = take(std::max(x32, std::max(hf, cand)), 16);
+  const int big = hf > cand ? hf : cand;
+  p.o_x32 = take(x32 > big ? x32 : big, 16);
   p.o_cand = p.o_x32;
   p.o_hf = p.o_x32;
   p.o_xf = take(3 * 2 * T * H, 16);
@@ -405,6 +406,12 @@ __device__ __forceinline__ uint32_t half_of(const uint2& v, int g) {  // g-th fp
   return (g & 1) ? (w >> 16) : (w & 0xffffu);
 }
 
+// Code -> fp16 by the published "magic number" conversion (as in the int4
+// kernels of FasterTransformer and Marlin): OR the code bits into the
+// mantissa of an fp16 constant whose exponent makes one unit of those bits
+// worth 1, then subtract the constant. Here the low nibble of a byte sits
+// under 1024 (0x6400) and the high nibble under 64 (0x5400, where bits 4-7
+// are worth 1 each), so neither needs a shift.
 // int4 word -> four fp16 pairs (c - 8) * s in the order of frag_pos.
 __device__ __forceinline__ void deq4(uint32_t w, uint32_t s2, uint32_t (&p)[4]) {
   const uint32_t w8 = w >> 8;

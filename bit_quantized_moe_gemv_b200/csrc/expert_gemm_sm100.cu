@@ -271,7 +271,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 }
 
 // ---------------------------------------------------------------- dequant
-// (a & mask) | magic in one instruction
+// (a & mask) | magic in one instruction: the first step of the published
+// "magic number" code -> fp16 conversion (OR the code under an fp16 exponent
+// whose mantissa unit is worth 1, then subtract that constant)
 __device__ __forceinline__ uint32_t lop_or(uint32_t a, uint32_t mask, uint32_t magic) {
   uint32_t d;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(magic));
