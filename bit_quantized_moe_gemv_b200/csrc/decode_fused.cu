@@ -127,7 +127,7 @@ __host__ __device__ inline int gu_parts(int H) { return H % 512 == 0 ? 2 : 1; }
 // Dynamic shared memory, offsets from the base.
 struct Plan {
   int o_x32;   // fp32 x [T][H] (router input, phase A only)
-  int o_cand;  // top-k candidates of the routing [T][E / 32][k], 8 bytes each (over x32)
+  int o_cand;  // top-k candidates of the routing [T][E / 32][k] and their survivors [T][k k], 8 bytes each (over x32)
   int o_hf;    // per-warp activations of a down job, 2 T I bytes each (phase C; over x32)
   int o_xf;    // 3 activation buffers in fragment order, 2 T H bytes each
   int o_rp;    // router partials [rows][segs][T]
@@ -152,7 +152,8 @@ __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int
     o += bytes;
     return r;
   };
-  const int x32 = 4 * T * H, hf = kWarps * 2 * T * I, cand = 8 * T * ((E + 31) / 32) * k;
+  // routing candidates: [T][E / 32][k], then up to k^2 survivors per token
+  const int x32 = 4 * T * H, hf = kWarps * 2 * T * I, cand = 8 * T * (((E + 31) / 32) * k + k * k);
   const int big = hf > cand ? hf : cand;
   p.o_x32 = take(x32 > big ? x32 : big, 16);
   p.o_cand = p.o_x32;
@@ -970,6 +971,9 @@ struct RouteShared {
   int uniq[kMaxT * kMaxK];  // slot -> expert id
   uint32_t bits[kMaxE / 32];
   uint32_t bpre[kMaxE / 32];  // set bits in the words before
+  uint64_t best[kMaxT * kMaxE / 32];  // each chunk's best candidate
+  uint64_t cut[kMaxT];                // the k-th best chunk winner of each token
+  int nsurv[kMaxT];                   // candidates at or above it
   int U, bad;
 };
 
@@ -1022,24 +1026,43 @@ __device__ __noinline__ bool route_all(Ctx& C, RouteShared& R, bool has_shared) 
       }
       v = warp_sort32_desc(v);
       if (lane < k) cand[size_t(q) * k + lane] = v;
+      if (lane == 0) R.best[q] = v;
     }
   __syncthreads();
-  // second round: a candidate's rank among its token's candidates (keys are
-  // distinct: the low word is the id); the best k go to their rank's place
+  // cutoff of each token: its k-th best chunk winner. Those k winners are k
+  // logits at or above it, so every one of the token's top k is too; and
+  // only the k chunks they head can hold candidates at or above it, so at
+  // most k^2 candidates survive (all of them when there are fewer than k
+  // chunks: cutoff 0)
+  if (live && warp < T) {
+    const int t = warp;
+    uint64_t v = lane < n32 ? R.best[t * n32 + lane] : 0ull;
+    v = warp_sort32_desc(v);
+    const uint64_t cut = __shfl_sync(0xffffffffu, v, k - 1);
+    if (lane == 0) {
+      R.cut[t] = n32 >= k ? cut : 0ull;
+      R.nsurv[t] = 0;
+    }
+  }
+  __syncthreads();
+  uint64_t* surv = cand + size_t(T) * nc;  // [T][k k]
   if (live)
     for (int q = threadIdx.x; q < T * nc; q += kThreads) {
       const int t = q / nc;
       const uint64_t v = cand[q];
-      if (v == 0ull) continue;  // no logit (chunk past E)
-      const uint64_t* c = cand + size_t(t) * nc;
+      if (v != 0ull && v >= R.cut[t]) surv[t * k * k + atomicAdd(&R.nsurv[t], 1)] = v;  // v == 0: no logit
+    }
+  __syncthreads();
+  // second round: a survivor's rank among its token's survivors (keys are
+  // distinct: the low word is the id); the best k go to their rank's place
+  if (live)
+    for (int q = threadIdx.x; q < T * k * k; q += kThreads) {
+      const int t = q / (k * k), i = q - t * (k * k), ns = R.nsurv[t];
+      if (i >= ns) continue;
+      const uint64_t* c = surv + size_t(t) * k * k;
+      const uint64_t v = c[i];
       int rank = 0;
-      for (int j = 0; j < nc; j += 8) {  // 8 loads in flight, then 8 compares
-        uint64_t w[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) w[u] = j + u < nc ? c[j + u] : 0ull;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) rank += w[u] > v ? 1 : 0;
-      }
+      for (int j = 0; j < ns; ++j) rank += c[j] > v ? 1 : 0;
       if (rank < k) {
         R.key[t * k + rank] = uint32_t(v >> 32);
         R.idx[t * k + rank] = int(~uint32_t(v));
