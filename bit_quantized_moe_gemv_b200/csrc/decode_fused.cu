@@ -135,6 +135,8 @@ struct Plan {
   int o_td;    // gate/up K-split arrivals [tiles]
   int o_y;     // down results [kMaxSlots][16][T]
   int o_desc;  // expert descriptors of the picked slots and the shared one
+  int o_stage;      // per-warp staging buffers of int4/int2 job rows, or -1
+  int stage_bytes;  // bytes of one warp's staging buffer
   int total;
 };
 __host__ __device__ inline int router_rows(int E, int G) { return (E + G - 1) / G; }
@@ -143,6 +145,17 @@ __host__ __device__ inline int max_tiles(int T, int I, int E, int k, int G) {
   const int U = T * k < E ? T * k : E;
   return ((U + 1) * (I / 8) + G - 1) / G;  // routed experts and the shared one
 }
+// Row pitches of a staged job with ncol 16-byte code columns per row: codes
+// ncol * 16 + 16 (one spare 16-byte unit, so consecutive rows start on
+// different banks), scales (and int2 mins) of those columns rounded up to 16.
+__host__ __device__ inline void stage_pitches(int f, int ncol, int& cp, int& sp) {
+  cp = ncol * 16 + 16;
+  const int s = f == MOE_Q_INT2_ASYM_G16 ? ncol * 8 : ncol * 2;
+  sp = (s + 15) / 16 * 16;
+}
+constexpr int kStaticSmemBound = 12 * 1024;  // bound on the kernel's static shared memory
+
+
 __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int G) {
   Plan p{};
   int o = 0;
@@ -164,6 +177,20 @@ __host__ __device__ inline Plan make_plan(int T, int H, int I, int E, int k, int
   p.o_td = take(4 * max_tiles(T, I, E, k, G), 16);
   p.o_y = take(4 * kMaxSlots * 16 * T, 16);
   p.o_desc = take(int(sizeof(moe_expert)) * kMaxSlots, 16);
+  // staging: the largest int4 or int2 job (16 rows of a gate/up part or of
+  // a down slice) with the row pitches of stage_pitches, when it fits
+  int sb = 0;
+  for (int f = MOE_Q_INT4_SYM_G32; f <= MOE_Q_INT2_ASYM_G16; ++f) {
+    const int nm = f == MOE_Q_INT2_ASYM_G16 ? 2 : 1;
+    int cp, sp;
+    stage_pitches(f, H / kc(f) / gu_parts(H), cp, sp);
+    sb = sb > 16 * (cp + nm * sp) ? sb : 16 * (cp + nm * sp);
+    stage_pitches(f, I / kc(f), cp, sp);
+    sb = sb > 16 * (cp + nm * sp) ? sb : 16 * (cp + nm * sp);
+  }
+  p.stage_bytes = sb;
+  p.o_stage = -1;
+  if (o + 16 + kWarps * sb + kStaticSmemBound <= kSmemLimit) p.o_stage = take(kWarps * sb, 16);
   p.total = o;
   return p;
 }
@@ -318,6 +345,11 @@ __device__ __forceinline__ uint32_t ldg4(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
+// The warp's staging copies have landed and every lane may read them.
+__device__ __forceinline__ void stage_wait() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+}
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -384,18 +416,41 @@ struct Ld {
   uint2 sa, sb, ma, mb;  // int4: sa.x / sb.x = scale; int2: 4 scales / 4 mins each
 };
 
-template <int F>
+// Weight loads from global memory (streamed, not kept in L1) or from this
+// warp's staging buffer in shared memory (kSmem: generic loads).
+template <bool kSmem>
+__device__ __forceinline__ uint4 ldw16(const void* p) {
+  if constexpr (kSmem) return *reinterpret_cast<const uint4*>(p);
+  else return ldg16(p);
+}
+template <bool kSmem>
+__device__ __forceinline__ uint2 ldw8(const void* p) {
+  if constexpr (kSmem) return *reinterpret_cast<const uint2*>(p);
+  else return ldg8(p);
+}
+template <bool kSmem>
+__device__ __forceinline__ uint32_t ldw4(const void* p) {
+  if constexpr (kSmem) return *reinterpret_cast<const uint32_t*>(p);
+  else return ldg4(p);
+}
+template <bool kSmem>
+__device__ __forceinline__ uint32_t ldw2(const void* p) {
+  if constexpr (kSmem) return uint32_t(*reinterpret_cast<const uint16_t*>(p));
+  else return ldg2(p);
+}
+
+template <int F, bool kSmem>
 __device__ __forceinline__ void load_it(const Rows& R, int c, Ld& L) {
-  L.a = R.lo ? ldg16(R.c_lo + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
-  L.b = R.hi ? ldg16(R.c_hi + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.a = R.lo ? ldw16<kSmem>(R.c_lo + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.b = R.hi ? ldw16<kSmem>(R.c_hi + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
   if (F == MOE_Q_INT4_SYM_G32) {
-    L.sa.x = R.lo ? ldg2(R.s_lo + c) : 0u;
-    L.sb.x = R.hi ? ldg2(R.s_hi + c) : 0u;
+    L.sa.x = R.lo ? ldw2<kSmem>(R.s_lo + c) : 0u;
+    L.sb.x = R.hi ? ldw2<kSmem>(R.s_hi + c) : 0u;
   } else if (F == MOE_Q_INT2_ASYM_G16) {
-    L.sa = R.lo ? ldg8(R.s_lo + 4 * c) : make_uint2(0u, 0u);
-    L.sb = R.hi ? ldg8(R.s_hi + 4 * c) : make_uint2(0u, 0u);
-    L.ma = R.lo ? ldg8(R.m_lo + 4 * c) : make_uint2(0u, 0u);
-    L.mb = R.hi ? ldg8(R.m_hi + 4 * c) : make_uint2(0u, 0u);
+    L.sa = R.lo ? ldw8<kSmem>(R.s_lo + 4 * c) : make_uint2(0u, 0u);
+    L.sb = R.hi ? ldw8<kSmem>(R.s_hi + 4 * c) : make_uint2(0u, 0u);
+    L.ma = R.lo ? ldw8<kSmem>(R.m_lo + 4 * c) : make_uint2(0u, 0u);
+    L.mb = R.hi ? ldw8<kSmem>(R.m_hi + 4 * c) : make_uint2(0u, 0u);
   }
 }
 
@@ -489,19 +544,32 @@ __device__ __forceinline__ void mma_it(const Ld& L, const uint8_t* bf, int c, in
 __host__ __device__ constexpr int depth(int F) { return F == MOE_Q_INT2_ASYM_G16 ? 2 : 4; }
 
 // One warp's share of a tile: iterations it = 0..nit-1, lane column
-// c = col0 + 4 it + tq; the loads of depth(F) iterations are in flight while
-// one is computed. Returns this lane's four accumulators (D rows gq, gq + 8;
-// token columns 2 tq, 2 tq + 1). One function per format, so each gets its
-// own register allocation.
-template <int F>
-__device__ __noinline__ float4 run_tile(const Rows R, int col0, int nit, const uint8_t* bf, int T) {
+// wc = wcol0 + 4 it + tq of the weights (global, or the staged copy) against
+// activation column c = col0 + 4 it + tq; the loads of depth(F) iterations
+// are in flight while one is computed. Returns this lane's four accumulators
+// (D rows gq, gq + 8; token columns 2 tq, 2 tq + 1). One function per format
+// and source, so each gets its own register allocation.
+template <int F, bool kSmem>
+__device__ __noinline__ float4 run_tile(const Rows R, int wcol0, int col0, int nit, const uint8_t* bf, int T) {
   const int tq = threadIdx.x & 3;
-  constexpr int kDepth = depth(F);
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  if constexpr (kSmem) {
+    // staged rows: once they have landed, one iteration at a time
+    // (shared-memory latency) in a small loop
+    stage_wait();
+#pragma unroll 1
+    for (int it = 0; it < nit; ++it) {
+      Ld L;
+      load_it<F, true>(R, wcol0 + 4 * it + tq, L);
+      mma_it<F>(L, bf, col0 + 4 * it + tq, T, acc);
+    }
+    return make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+  }
+  constexpr int kDepth = kSmem ? 1 : depth(F);
   Ld L[kDepth];
 #pragma unroll
   for (int s = 0; s < kDepth; ++s)
-    if (s < nit) load_it<F>(R, col0 + 4 * s + tq, L[s]);
+    if (s < nit) load_it<F, kSmem>(R, wcol0 + 4 * s + tq, L[s]);
 #pragma unroll 1
   for (int it0 = 0; it0 < nit; it0 += kDepth) {
 #pragma unroll
@@ -509,17 +577,19 @@ __device__ __noinline__ float4 run_tile(const Rows R, int col0, int nit, const u
       const int it = it0 + s;
       if (it < nit) {
         mma_it<F>(L[s], bf, col0 + 4 * it + tq, T, acc);
-        if (it + kDepth < nit) load_it<F>(R, col0 + 4 * (it + kDepth) + tq, L[s]);
+        if (it + kDepth < nit) load_it<F, kSmem>(R, wcol0 + 4 * (it + kDepth) + tq, L[s]);
       }
     }
   }
   return make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1], acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
 }
-__device__ __forceinline__ void run_any(int f, const Rows& R, int col0, int nit, const uint8_t* bf, int T,
+template <bool kSmem>
+__device__ __forceinline__ void run_any(int f, const Rows& R, int wcol0, int col0, int nit, const uint8_t* bf, int T,
                                         float (&acc)[4]) {
-  const float4 v = f == MOE_Q_INT4_SYM_G32   ? run_tile<MOE_Q_INT4_SYM_G32>(R, col0, nit, bf, T)
-                   : f == MOE_Q_INT2_ASYM_G16 ? run_tile<MOE_Q_INT2_ASYM_G16>(R, col0, nit, bf, T)
-                                              : run_tile<MOE_Q_INT8_PER_CHANNEL>(R, col0, nit, bf, T);
+  const float4 v = f == MOE_Q_INT4_SYM_G32 ? run_tile<MOE_Q_INT4_SYM_G32, kSmem>(R, wcol0, col0, nit, bf, T)
+                   : f == MOE_Q_INT2_ASYM_G16
+                       ? run_tile<MOE_Q_INT2_ASYM_G16, kSmem>(R, wcol0, col0, nit, bf, T)
+                       : run_tile<MOE_Q_INT8_PER_CHANNEL, false>(R, wcol0, col0, nit, bf, T);  // int8: never staged
   acc[0] = v.x;
   acc[1] = v.y;
   acc[2] = v.z;
@@ -538,11 +608,12 @@ struct Ld4 {
   uint4 a, b;      // codes of rows gq and gq + 8, this lane's column
   uint32_t sa, sb;  // fp16 scales of this lane's two D columns, rows gq and gq + 8
 };
+template <bool kSmem>
 __device__ __forceinline__ void load_i4(const Rows& R, int c, int cs, Ld4& L) {
-  L.a = R.lo ? ldg16(R.c_lo + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
-  L.b = R.hi ? ldg16(R.c_hi + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
-  L.sa = R.lo ? ldg4(R.s_lo + cs) : 0u;
-  L.sb = R.hi ? ldg4(R.s_hi + cs) : 0u;
+  L.a = R.lo ? ldw16<kSmem>(R.c_lo + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.b = R.hi ? ldw16<kSmem>(R.c_hi + size_t(c) * 16) : make_uint4(0u, 0u, 0u, 0u);
+  L.sa = R.lo ? ldw4<kSmem>(R.s_lo + cs) : 0u;
+  L.sb = R.hi ? ldw4<kSmem>(R.s_hi + cs) : 0u;
 }
 // int4 word -> four fp16 pairs (c - 8), exact, in the order of frag_pos.
 __device__ __forceinline__ void deq4_codes(uint32_t w, uint32_t (&p)[4]) {
@@ -552,18 +623,20 @@ __device__ __forceinline__ void deq4_codes(uint32_t w, uint32_t (&p)[4]) {
   p[2] = h2sub(lop_or(w8, 0x000F000Fu, 0x64006400u), 0x64086408u);
   p[3] = h2sub(lop_or(w8, 0x00F000F0u, 0x54005400u), 0x54805480u);
 }
-__device__ __noinline__ float4 run_tile_i4(const Rows R, int col0, int nit, const uint8_t* bf, int T) {
+template <bool kSmem>
+__device__ __noinline__ float4 run_tile_i4(const Rows R, int wcol0, int col0, int nit, const uint8_t* bf, int T) {
   const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
   const int dt = gq - tq;
   const bool bv = dt == 0 || (dt == 4 && T == 2);  // B column gq takes A lane tq's activations
   const int bt = dt == 4 ? 1 : 0;                   // of this token
   const int g0 = (2 * tq) & 3;                      // groups of this lane's D columns 2 tq, 2 tq + 1
-  constexpr int kDepth = 4;
+  constexpr int kDepth = kSmem ? 1 : 4;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   Ld4 L[kDepth];
+  if constexpr (kSmem) stage_wait();  // the staged rows have landed
 #pragma unroll
   for (int s = 0; s < kDepth; ++s)
-    if (s < nit) load_i4(R, col0 + 4 * s + tq, col0 + 4 * s + g0, L[s]);
+    if (s < nit) load_i4<kSmem>(R, wcol0 + 4 * s + tq, wcol0 + 4 * s + g0, L[s]);
 #pragma unroll 1
   for (int it0 = 0; it0 < nit; it0 += kDepth) {
 #pragma unroll
@@ -590,7 +663,8 @@ __device__ __noinline__ float4 run_tile_i4(const Rows R, int col0, int nit, cons
         acc[1] = fmaf(sa.y, d0[1] + d1[1], acc[1]);
         acc[2] = fmaf(sb.x, d0[2] + d1[2], acc[2]);
         acc[3] = fmaf(sb.y, d0[3] + d1[3], acc[3]);
-        if (it + kDepth < nit) load_i4(R, col0 + 4 * (it + kDepth) + tq, col0 + 4 * (it + kDepth) + g0, L[s]);
+        if (it + kDepth < nit)
+          load_i4<kSmem>(R, wcol0 + 4 * (it + kDepth) + tq, wcol0 + 4 * (it + kDepth) + g0, L[s]);
       }
     }
   }
@@ -694,6 +768,83 @@ struct Ctx {
   moe_expert* desc;         // descriptors: slots 0..U-1, kSharedSlot
 };
 
+// ---------------------------------------------------------------- staging
+// int4 and int2 job rows come into the warp's own shared-memory buffer by
+// per-lane asynchronous copies (cp.async, 16 bytes each): all of a job's
+// bytes are in flight at once and none of them occupies registers. Job row r
+// (A rows 0-15) lies at r * cp, its scales at 16 cp + r * sp and its int2
+// mins at 16 cp + 16 sp + r * sp (stage_pitches).
+__device__ __forceinline__ bool stage_aligned(const moe_qmatrix& m) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(m.codes) | reinterpret_cast<uintptr_t>(m.scales) |
+                      (m.qtype == MOE_Q_INT2_ASYM_G16 ? reinterpret_cast<uintptr_t>(m.mins) : 0u);
+  return (a & 15u) == 0;
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+// Rows [row_lo, row_lo + n_lo) of m_lo become job rows 0.., rows [row_hi,
+// row_hi + n_hi) of m_hi job rows 8..; columns [col0, col0 + ncol) of 16
+// code bytes each, of a K-column matrix. The 16-byte pieces are dealt to the
+// lanes row-major; one commit group for the whole job.
+__device__ __noinline__ void stage_issue(const moe_qmatrix& m_lo, int row_lo, int n_lo, const moe_qmatrix& m_hi,
+                                         int row_hi, int n_hi, int K, int col0, int ncol, uint8_t* sb, int cp,
+                                         int sp) {
+  const int lane = threadIdx.x & 31;
+  const bool i2 = m_lo.qtype == MOE_Q_INT2_ASYM_G16;
+  const int rb = K >> (i2 ? 2 : 1);    // code bytes per row
+  const int sper = K >> (i2 ? 4 : 5);  // scales per row
+  // codes: piece (r, c) for c < ncol
+  {
+    int r = 0, c = lane;
+    while (c >= ncol) c -= ncol, ++r;
+    for (; r < 16;) {
+      const bool lo = r < 8;
+      const int rr = r & 7;
+      if (rr < (lo ? n_lo : n_hi)) {
+        const moe_qmatrix& m = lo ? m_lo : m_hi;
+        cp_async16(sb + r * cp + c * 16, m.codes + size_t((lo ? row_lo : row_hi) + rr) * rb + size_t(col0 + c) * 16);
+      }
+      c += 32;
+      while (c >= ncol) c -= ncol, ++r;
+    }
+  }
+  // scales, then int2 mins: su pieces per row
+  const int su = ncol * (i2 ? 8 : 2) / 16;
+  for (int mi = 0; mi < (i2 ? 2 : 1); ++mi) {
+    int r = 0, c = lane;
+    while (c >= su) c -= su, ++r;
+    for (; r < 16;) {
+      const bool lo = r < 8;
+      const int rr = r & 7;
+      if (rr < (lo ? n_lo : n_hi)) {
+        const moe_qmatrix& m = lo ? m_lo : m_hi;
+        const uint16_t* base = (mi ? m.mins : m.scales) + size_t((lo ? row_lo : row_hi) + rr) * sper +
+                               size_t(col0) * (i2 ? 4 : 1);
+        cp_async16(sb + 16 * cp + mi * 16 * sp + r * sp + c * 16, reinterpret_cast<const uint8_t*>(base) + c * 16);
+      }
+      c += 32;
+      while (c >= su) c -= su, ++r;
+    }
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Rows of a staged job for run_tile / run_tile_i4 (weight columns from 0).
+__device__ __forceinline__ Rows staged_rows(uint8_t* sb, int cp, int sp, bool lo, bool hi) {
+  const int gq = (threadIdx.x & 31) >> 2;
+  Rows R;
+  R.lo = lo;
+  R.hi = hi;
+  R.c_lo = sb + gq * cp;
+  R.c_hi = sb + (gq + 8) * cp;
+  R.s_lo = reinterpret_cast<const uint16_t*>(sb + 16 * cp + gq * sp);
+  R.s_hi = reinterpret_cast<const uint16_t*>(sb + 16 * cp + (gq + 8) * sp);
+  R.m_lo = reinterpret_cast<const uint16_t*>(sb + 16 * cp + 16 * sp + gq * sp);
+  R.m_hi = reinterpret_cast<const uint16_t*>(sb + 16 * cp + 16 * sp + (gq + 8) * sp);
+  return R;
+}
+
 // gate/up tile part: 8 intermediate rows of gate (A rows 0-7) and of up
 // (A rows 8-15) over part p of K. The last part to finish sums the parts
 // (two fp32 values: the same sum in either order), applies SwiGLU and
@@ -702,7 +853,7 @@ struct Ctx {
 __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   const Params& P = *C.P;
   const int T = C.T, H = C.H, I = C.I;
-  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3, warp = threadIdx.x >> 5;
   const int slot = jb.slot;
   const moe_expert& d = C.desc[slot];
   const int f = d.gate.qtype, ns = gu_parts(H);
@@ -720,11 +871,23 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
   R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.up.mins + size_t(row) * sper : nullptr;
   const uint8_t* bf = C.smem + C.L.o_xf + (f - 1) * 2 * T * H;  // formats 1..3 -> buffers 0..2
   float acc[4];
-  if (i4_grouped(f, T, R)) {
-    const float4 v = run_tile_i4(R, col0, nit, bf, T);
+  if (C.L.o_stage >= 0 && f != MOE_Q_INT8_PER_CHANNEL && stage_aligned(d.gate) && stage_aligned(d.up)) {
+    uint8_t* sb = C.smem + C.L.o_stage + warp * C.L.stage_bytes;
+    int cp, sp;
+    stage_pitches(f, ncol, cp, sp);
+    stage_issue(d.gate, jb.row0, 8, d.up, jb.row0, 8, H, col0, ncol, sb, cp, sp);
+    const Rows S = staged_rows(sb, cp, sp, true, true);  // the tile loop waits for the copies
+    if (i4_grouped(f, T, S)) {
+      const float4 v = run_tile_i4<true>(S, 0, col0, nit, bf, T);
+      acc[0] = v.x, acc[1] = v.y, acc[2] = v.z, acc[3] = v.w;
+    } else {
+      run_any<true>(f, S, 0, col0, nit, bf, T, acc);
+    }
+  } else if (i4_grouped(f, T, R)) {
+    const float4 v = run_tile_i4<false>(R, col0, col0, nit, bf, T);
     acc[0] = v.x, acc[1] = v.y, acc[2] = v.z, acc[3] = v.w;
   } else {
-    run_any(f, R, col0, nit, bf, T, acc);
+    run_any<false>(f, R, col0, col0, nit, bf, T, acc);
   }
   // D rows gq (gate) / gq + 8 (up), tokens 2 tq, 2 tq + 1
   if (ns > 1) {
@@ -850,15 +1013,26 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   R.m_hi = f == MOE_Q_INT2_ASYM_G16 ? d.down.mins + size_t(R.hi ? rhi : 0) * sper : nullptr;
   uint8_t* hf = C.smem + C.L.o_hf + warp * 2 * T * I;
   __shared__ int s_eh[kWarps][kMaxT];
-  // this job's rows into L2 while its expert's gate/up tiles finish (the
-  // shared expert's are there since phase A)
-  if (slot != kSharedSlot && lane < 3) prefetch_down_piece(d.down, I, jb.row0, jb.nrows, lane);
+  // this job's rows on their way while its expert's gate/up tiles finish:
+  // into the warp's staging buffer (int4, int2), else into L2 (the shared
+  // expert's are in L2 since phase A)
+  const bool staged = C.L.o_stage >= 0 && f != MOE_Q_INT8_PER_CHANNEL && stage_aligned(d.down);
+  uint8_t* sb = C.smem + C.L.o_stage + warp * C.L.stage_bytes;
+  int cp = 0, sp = 0;
+  if (staged) {
+    stage_pitches(f, I / kc(f), cp, sp);
+    stage_issue(d.down, jb.row0, min(int(jb.nrows), 8), d.down, jb.row0 + 8, max(int(jb.nrows) - 8, 0), I, 0,
+                I / kc(f), sb, cp, sp);
+  } else if (slot != kSharedSlot && lane < 3) {
+    prefetch_down_piece(d.down, I, jb.row0, jb.nrows, lane);
+  }
   int ok = 1;
   if (lane == 0)
     ok = wait_counter(P.cnt + slot * kCntStride, uint32_t(I / 8), P.hdr, P.wait_cycles, 7100000 + slot) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok) {
     if (lane == 0) C.fail = 1;
+    if (staged) stage_wait();  // the copies land before the warp moves on
     return;
   }
   (void)ld_acquire(P.cnt + slot * kCntStride);  // every lane orders its reads of h after the counter
@@ -870,11 +1044,19 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   else h_to_frag<MOE_Q_INT8_PER_CHANNEL>(hs, T, I, s_eh[warp], hf);
   __syncwarp();
   float acc[4];
-  if (i4_grouped(f, T, R)) {
-    const float4 v = run_tile_i4(R, 0, nit, hf, T);
+  if (staged) {
+    const Rows S = staged_rows(sb, cp, sp, R.lo, R.hi);  // the tile loop waits for the copies
+    if (i4_grouped(f, T, S)) {
+      const float4 v = run_tile_i4<true>(S, 0, 0, nit, hf, T);
+      acc[0] = v.x, acc[1] = v.y, acc[2] = v.z, acc[3] = v.w;
+    } else {
+      run_any<true>(f, S, 0, 0, nit, hf, T, acc);
+    }
+  } else if (i4_grouped(f, T, R)) {
+    const float4 v = run_tile_i4<false>(R, 0, 0, nit, hf, T);
     acc[0] = v.x, acc[1] = v.y, acc[2] = v.z, acc[3] = v.w;
   } else {
-    run_any(f, R, 0, nit, hf, T, acc);
+    run_any<false>(f, R, 0, 0, nit, hf, T, acc);
   }
   float* y = reinterpret_cast<float*>(C.smem + C.L.o_y) + size_t(slot) * 16 * T;
 #pragma unroll
@@ -1387,7 +1569,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------- host side
-constexpr int kStaticSmem = 12 * 1024;  // bound on the kernel's static shared memory
+constexpr int kStaticSmem = kStaticSmemBound;
 
 int grid_size() {
   int dev = 0, sms = 0;

@@ -79,6 +79,22 @@ int main() {
               for (int o : offs)
                 if (o % 16) ++bad_plan;
               if (p.total + kStaticSmem > kSmemLimit) ++bad_plan;
+              // staging buffers: aligned, and each warp's holds the largest
+              // int4 / int2 job it may stage (a gate/up part or a down slice)
+              if (p.o_stage >= 0) {
+                if (p.o_stage % 16 || p.stage_bytes % 16 || p.o_stage + kWarps * p.stage_bytes > p.total) ++bad_plan;
+                for (int f = MOE_Q_INT4_SYM_G32; f <= MOE_Q_INT2_ASYM_G16; ++f) {
+                  const int nm = f == MOE_Q_INT2_ASYM_G16 ? 2 : 1;
+                  const int ncols[2] = {H / kc(f) / gu_parts(H), I / kc(f)};
+                  for (int ncol : ncols) {
+                    int cp, sp;
+                    stage_pitches(f, ncol, cp, sp);
+                    if (16 * (cp + nm * sp) > p.stage_bytes || cp % 16 || sp % 16 ||
+                        (ncol * (f == MOE_Q_INT2_ASYM_G16 ? 8 : 2)) % 16)
+                      ++bad_plan;
+                  }
+                }
+              }
               // every picked-expert count from 1 to the most, with and
               // without the shared expert and its gate row
               const int Umax = T * k < E ? T * k : E;
@@ -144,10 +160,11 @@ int main() {
             }
   printf("{\"bad_frag\": %d, \"bad_plan\": %d, \"bad_cover\": %d, \"bad_fields\": %d, \"bad_ws\": %d, "
          "\"eligible\": %d, \"checked\": %d, \"decode1\": %d, \"decode48\": %d, \"smem_decode1\": %d, "
-         "\"smem_decode48\": %d}\n",
+         "\"smem_decode48\": %d, \"staged_decode1\": %d}\n",
          bad_frag, bad_plan, bad_cover, bad_fields, bad_ws, eligible, checked,
          int(eligible_on(1, 2048, 768, 512, 10, 148)), int(eligible_on(4, 2048, 768, 512, 10, 148)),
-         make_plan(1, 2048, 768, 512, 10, 148).total, make_plan(4, 2048, 768, 512, 10, 148).total);
+         make_plan(1, 2048, 768, 512, 10, 148).total, make_plan(4, 2048, 768, 512, 10, 148).total,
+         int(make_plan(1, 2048, 768, 512, 10, 148).o_stage >= 0));
   return 0;
 }
 """
@@ -193,3 +210,4 @@ def test_workspace_holds_what_the_kernel_writes(plan_report):
 
 def test_the_bench_decode_shapes_take_the_fused_kernel(plan_report):
     assert plan_report["decode1"] == 1 and plan_report["decode48"] == 1
+    assert plan_report["staged_decode1"] == 1  # one-token decode stages its int4 rows
