@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernel exists).
 NCU_TRAFFIC = {
     # decode_fused_kernel of one step (dram read + write of one launch)
-    "decode1": (33783296, "profiles/decode_fused_decode1.md"),
+    "decode1": (33757696, "profiles/decode_fused_decode1.md"),
     # predequant_kernel + grouped_gemm_kernel<gate/up> + <down> of one step
     # (the gather of the activations is not included)
     "prefill8k": (2863281328, "profiles/grouped_gemm_prefill8k.md"),
@@ -436,6 +436,12 @@ def run_ours(args, rank, world, peaks, peak_kind):
     # launches are queued before its start event runs (the events then time
     # the device, not the host's submission of the next call)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # one untimed pass first: the first launch of each kernel loads its code
+    L.route(xs[args.warmup], w_r, b, stride, k, idx[args.warmup], gw[args.warmup], ws, stream=stream)
+    L.dispatch(idx[args.warmup], E, counts, offsets, perm, inv, ws, stream=stream)
+    L.expert_ffn(xs[args.warmup], wl.I, k, E, perm, offsets, counts, experts.table, y_perm, ws, stream=stream)
+    L.combine(y_perm, inv, gw[args.warmup], wl.I, xs[args.warmup], shared.table, out4, ws, stream=stream)
+    torch.cuda.synchronize()
     launches0 = L.launch_count()
     for i in range(args.steps):
         s = args.warmup + i
