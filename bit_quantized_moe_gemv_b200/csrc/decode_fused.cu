@@ -1,5 +1,5 @@
 // Decode step (1 <= T <= 4 tokens) as ONE persistent cooperative launch in
-// which every warp streams its own weights straight into registers.
+// which every warp fetches and dequantises its own weight rows.
 //
 // Decode reads each picked expert's weights once per step, so its floor is
 // memory bandwidth (the lcz.me forum thread "Halogen Flash Server配置與實測",
@@ -10,24 +10,30 @@
 // expert per token.
 //
 // Structure (one CTA of 16 warps per SM, all CTAs co-resident):
-//   A  router rows of this CTA (whole logits, one publication per CTA) and
-//      the shared expert's gate/up tiles of this CTA; the CTA then arrives on
-//      a grid counter and waits for every CTA's logits;
-//   -  every CTA reads all logits, takes the top-k itself (identical inputs,
-//      identical code, identical picks), lists the distinct picked experts
-//      and prefetches its down rows of each into L2;
-//   B  the routed gate/up tiles of this CTA (tile g of the step's list goes
-//      to CTA g mod G, so each expert's tiles finish early and together);
-//      finishing a tile publishes its 8 intermediate values h per token and
-//      bumps that expert's tile counter;
-//   C  this CTA's slice of output rows of every picked expert's down
-//      projection, each waiting only for ITS expert's counter (no second
-//      grid barrier); then the gate-weighted combine of those rows.
-// Every warp walks its own list of jobs (B jobs before C jobs, so a warp
-// waiting in C never holds back a tile that another waits for). A job is
-// 16 weight rows over a K range: each lane loads 16 bytes of codes of its
-// two rows per iteration, several iterations ahead, dequantises them in
-// registers and feeds mma.sync m16n8k16 (fp16 operands, fp32 accumulation)
+//   A  router rows of this CTA (whole logits, one publication per CTA; the
+//      weights are loaded at the kernel's entry); the CTA then arrives on a
+//      grid counter, and while every CTA's logits gather it converts x for
+//      the tensor cores and prefetches its rows of the shared expert;
+//   -  every CTA, all warps, reads all logits and takes the top-k itself
+//      (identical inputs, identical code, identical picks): 32-logit chunks
+//      sorted per warp, a cutoff at each token's k-th best chunk winner, the
+//      survivors ranked; then the gates, the distinct picked experts (slots)
+//      and their descriptors;
+//   B  the gate/up tiles of this CTA in the list "shared expert, then the
+//      picked ones" (tile g goes to CTA g mod G, so each expert's tiles
+//      finish early and together); finishing a tile publishes its 8
+//      intermediate values h per token and bumps that expert's tile counter;
+//   C  this CTA's slice of output rows of every expert's down projection,
+//      each waiting only for ITS expert's counter (no second grid barrier);
+//      then the gate-weighted combine of those rows.
+// Jobs are numbered per CTA and computed from their numbers; warp w takes
+// jobs w, w + 16, ... (B jobs before C jobs, so a warp waiting in C never
+// holds back a tile that another waits for). A job is 16 weight rows over a
+// K range. int4 and int2 rows are copied into the warp's own shared-memory
+// buffer by per-lane cp.async (all of the job at once) when the buffers fit,
+// else each lane loads 16 bytes of its two rows per iteration straight into
+// registers, several iterations ahead; the codes are dequantised in
+// registers and fed to mma.sync m16n8k16 (fp16 operands, fp32 accumulation)
 // with the T <= 4 tokens as the MMA's columns, read from shared memory in the
 // order the dequantisation produces pairs.
 //
