@@ -395,7 +395,6 @@ __device__ __forceinline__ void store4(uint8_t* buf, int k0, int t, int T, float
     *reinterpret_cast<__half*>(p + quad_off<F>(3)) = hd;
   }
 }
-__device__ __forceinline__ void named_sync() { __syncthreads(); }
 
 // Power-of-two exponent that brings a magnitude below 2^15 (fp16 max 65504):
 // 0 for anything already below.
@@ -698,43 +697,6 @@ __device__ __forceinline__ uint32_t f2key(float f) {
 __device__ __forceinline__ float key2f(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
-__device__ __forceinline__ void cswap(uint64_t& a, uint64_t& b) {
-  const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
-  a = hi;
-  b = lo;
-}
-// Best k (k <= 16) of up to 128 candidates held 4 per lane as key << 32 |
-// ~id (a larger value is better: key descending, then id ascending; 0 = no
-// candidate). Each lane sorts its four; every round takes the best lane head
-// by a reduction on the key and one on the low word among equal keys, and the
-// winning lane pops it.
-__device__ __noinline__ void warp_topk(uint64_t c0, uint64_t c1, uint64_t c2, uint64_t c3, int k, uint32_t* okey,
-                                      int* oid) {
-  const int lane = threadIdx.x & 31;
-  uint64_t c[4] = {c0, c1, c2, c3};
-  cswap(c[0], c[1]);
-  cswap(c[2], c[3]);
-  cswap(c[0], c[2]);
-  cswap(c[1], c[3]);
-  cswap(c[1], c[2]);
-#pragma unroll 1
-  for (int j = 0; j < k; ++j) {
-    const uint32_t hk = uint32_t(c[0] >> 32), lk = uint32_t(c[0]);
-    const uint32_t wk = __reduce_max_sync(0xffffffffu, hk);
-    const uint32_t wl = __reduce_max_sync(0xffffffffu, hk == wk ? lk : 0u);
-    if (lane == 0) {
-      okey[j] = wk;
-      oid[j] = wk ? int(~wl) : 0x7fffffff;
-    }
-    if (wk != 0u && hk == wk && lk == wl) {
-      c[0] = c[1];
-      c[1] = c[2];
-      c[2] = c[3];
-      c[3] = 0ull;
-    }
-  }
-}
-
 // ---------------------------------------------------------------- bounded waits
 // Spin (one thread) until *p >= target, the abort flag is raised or the
 // cycle budget runs out (checked before every new poll: with a budget of 0 a

@@ -91,7 +91,7 @@ def test_duplicated_router_rows_resolve_to_lower_index(L, path):
     w_r = (rng.standard_normal((E, H)) * 0.02).astype(np.float32)
     bias = np.zeros(E, dtype=np.float32)
     # two tied groups far above the rest (random rows give |logit| < ~5):
-    # ids spread over the whole range so the decode kernel's 128-logit
+    # ids spread over the whole range so the decode kernel's 32-logit
     # chunks each hold part of a group
     top = sorted({3, E // 2 + 1, E - 2})
     mid = sorted({1, E // 4 + 3, (3 * E) // 4, E - 1} - set(top))
