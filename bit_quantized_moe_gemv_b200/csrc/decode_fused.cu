@@ -280,6 +280,7 @@ struct Params {
   WsHeader* hdr;
   float* logits;   // [T][E] workspace
   float* h;        // [kMaxSlots][T][I] workspace
+  __half* h16;     // [kMaxSlots][2 T I bytes]: h as fp16 in the down format's fragment order (workspace)
   uint32_t* cnt;   // [kMaxSlots][kCntStride]: finished tiles, then max |h| bits per token
   long long wait_cycles;
   uint32_t flags;            // MOE_BIAS_SELECTION_ONLY
@@ -897,6 +898,9 @@ __device__ __noinline__ void job_gate_up(Ctx& C, const Job jb) {
       const float g = acc[i] * gsc * sc, u = acc[2 + i] * usc * sc;
       h = silu_f32(g) * u;
       __stcg(hs + size_t(t) * I + row, h);
+      // also in fp16, unscaled, where the down job's activations go: used
+      // as they are when no token of the expert needs range scaling
+      P.h16[size_t(slot) * T * I + frag_pos(f, row, t, T) / 2] = __float2half_rn(h);
     }
     // largest |h| of the tile per token: lanes of equal tq hold the same token
     uint32_t a = t < T ? __float_as_uint(fabsf(h)) : 0u;
@@ -1006,10 +1010,28 @@ __device__ __noinline__ void job_down(Ctx& C, const Job jb) {
   (void)ld_acquire(P.cnt + slot * kCntStride);  // every lane orders its reads of h after the counter
   if (lane < T) s_eh[warp][lane] = range_exp(__ldcg(P.cnt + slot * kCntStride + 1 + lane));
   __syncwarp();
-  const float4* hs = reinterpret_cast<const float4*>(P.h + size_t(slot) * T * I);
-  if (f == MOE_Q_INT4_SYM_G32) h_to_frag<MOE_Q_INT4_SYM_G32>(hs, T, I, s_eh[warp], hf);
-  else if (f == MOE_Q_INT2_ASYM_G16) h_to_frag<MOE_Q_INT2_ASYM_G16>(hs, T, I, s_eh[warp], hf);
-  else h_to_frag<MOE_Q_INT8_PER_CHANNEL>(hs, T, I, s_eh[warp], hf);
+  bool unscaled = true;
+  for (int t = 0; t < T; ++t) unscaled &= s_eh[warp][t] == 0;
+  if (unscaled) {
+    // every |h| of the expert fits fp16: its tiles' fp16 copy is exactly what
+    // the conversion below would produce; 8 loads per lane in flight
+    const uint4* src = reinterpret_cast<const uint4*>(P.h16 + size_t(slot) * T * I);
+    uint4* dst = reinterpret_cast<uint4*>(hf);
+    const int n16 = T * I / 8;  // 16-byte pieces
+    for (int base = lane; base < n16; base += 8 * 32) {
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = base + 32 * j < n16 ? __ldcg(src + base + 32 * j) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (base + 32 * j < n16) dst[base + 32 * j] = v[j];
+    }
+  } else {
+    const float4* hs = reinterpret_cast<const float4*>(P.h + size_t(slot) * T * I);
+    if (f == MOE_Q_INT4_SYM_G32) h_to_frag<MOE_Q_INT4_SYM_G32>(hs, T, I, s_eh[warp], hf);
+    else if (f == MOE_Q_INT2_ASYM_G16) h_to_frag<MOE_Q_INT2_ASYM_G16>(hs, T, I, s_eh[warp], hf);
+    else h_to_frag<MOE_Q_INT8_PER_CHANNEL>(hs, T, I, s_eh[warp], hf);
+  }
   __syncwarp();
   float acc[4];
   if (staged) {
@@ -1562,7 +1584,8 @@ bool decode_fused_eligible(int T, int H, int I, int E, int k) {
 }
 
 size_t decode_fused_ws_bytes(int T, int I) {
-  return size_t(dfx::kMaxSlots) * size_t(T) * size_t(I) * sizeof(float);
+  // h of every expert slot in fp32, then in fp16 (fragment order)
+  return size_t(dfx::kMaxSlots) * size_t(T) * size_t(I) * (sizeof(float) + sizeof(__half));
 }
 
 cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, int k, const float* w_router,
@@ -1589,7 +1612,8 @@ cudaError_t launch_decode_fused(const uint16_t* x, int T, int H, int I, int E, i
   }
   Params P{make_plan(T, H, I, E, k, grid), x, T, H, I, E, k, w_router, bias,
            bstride, experts, shared, topk_idx, topk_w, logits_out, out, hdr,
-           logits_ws, h_ws, counters, wait_cycles, flags, shared_gate, logits_u_ws,
+           logits_ws, h_ws, reinterpret_cast<__half*>(h_ws + size_t(kMaxSlots) * T * I), counters, wait_cycles, flags,
+           shared_gate, logits_u_ws,
            sgate_ws, heat, perm_src, offsets, counts, y_perm};
   void* args[] = {&P};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(decode_fused_kernel), dim3(grid), dim3(kThreads), args,

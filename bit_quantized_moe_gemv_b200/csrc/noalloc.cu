@@ -25,11 +25,11 @@ namespace {
 
 // Header (256 B) + the launch's counters + logits, biased and unbiased
 // (8 T E bytes) + the shared expert's gates (4 T bytes) + the intermediate
-// activations (65 expert slots x T x I floats): enough for T I <= 4096 at
-// E = 512 (the decode shapes: one token at I <= 2048, up to four at
-// I <= 1024); a call whose scratch would not fit returns
+// activations (65 expert slots x T x I values, fp32 and fp16): enough for
+// T I <= 4096 at E <= 1024 (the decode shapes: one token at I <= 2048, up to
+// four at I <= 1024); a call whose scratch would not fit returns
 // MOE_ERR_UNSUPPORTED.
-constexpr size_t kNoAllocBytes = 1280u * 1024u;
+constexpr size_t kNoAllocBytes = 2048u * 1024u;
 constexpr int kNoAllocMaxT = 4, kNoAllocMaxE = 1024, kNoAllocMaxK = 16, kNoAllocMaxHI = 2048;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];

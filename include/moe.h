@@ -234,13 +234,13 @@ moe_status moe_layer(const uint16_t* x, int32_t T, int32_t H, int32_t I, int32_t
  * cannot provide the workspace moe_layer needs. This call takes the same
  * arguments as moe_layer without `ws`/`ws_bytes`, allocates nothing (no
  * cudaMalloc, no allocating library routine) and keeps its scratch in a
- * 1.25 MiB device array inside the library, which every GPU that loads the
+ * 2 MiB device array inside the library, which every GPU that loads the
  * library holds until the process exits.
  *   Limits: 1 <= T <= 4, E <= 1024, k <= 16, 256 <= H, I <= 2048 (multiples
  *   of 256), within the fused decode kernel's own shape limits (the shapes
- *   moe_layer runs as one launch), and a scratch of at most 1.25 MiB
- *   (256 B + the counters + 8 T E bytes of logits + 65 T I fp32
- *   activations: T I <= 4096 at E = 512); anything else returns
+ *   moe_layer runs as one launch), and a scratch of at most 2 MiB
+ *   (256 B + the counters + 8 T E bytes of logits + 65 T I activations in
+ *   fp32 and fp16: T I <= 4096 at E <= 1024); anything else returns
  *   MOE_ERR_UNSUPPORTED.
  *   The first call on a device looks up the array's device address (once per
  *   device and CUDA context, with that device current); make that first call
