@@ -19,60 +19,54 @@
 namespace moe {
 
 // ---------------------------------------------------------------- top-k
-// Warp-level top-k over one row of E <= 1024 logits. Lane l holds experts
-// l, l+32, ... in registers. NaN logits are treated as -inf. gbias, when not
-// NULL, is the bias row of this token and the gates are taken on the
-// unbiased logits (logit - bias) of the picks: the bias moves the selection
-// only.
-__device__ void warp_topk_row(const float* row, int E, int k, int* idx_out, float* w_out, float* s_val,
-                              int* s_idx, const float* gbias) {
+// Order-preserving 32-bit key of a float (NaN as -inf): a larger key is a
+// larger value; 0 is never the key of a value.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) f = -CUDART_INF_F;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+// Warp-level top-k over one row of E <= 32 NPER logits. Lane l holds the
+// keys of experts l, l+32, ... in registers (0 = no expert or already
+// picked). Each round takes every lane's best (a strict '>' keeps the lower
+// index among equal keys), the largest key by a warp reduction and, among
+// the lanes holding it, the lowest expert index by a second one; the
+// winning lane clears that key. gbias, when not NULL, is the bias row of
+// this token and the gates are taken on the unbiased logits (logit - bias)
+// of the picks: the bias moves the selection only.
+template <int NPER>
+__device__ void warp_topk_row_n(const float* row, int E, int k, int* idx_out, float* w_out, float* s_val,
+                                int* s_idx, const float* gbias) {
   const int lane = threadIdx.x & 31;
-  float v[32];
-  const int nper = (E + 31) / 32;
+  uint32_t key[NPER];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPER; ++i) {
     const int e = lane + 32 * i;
-    float t = -CUDART_INF_F;
-    if (i < nper && e < E) {
-      t = __ldcg(row + e);
-      if (t != t) t = -CUDART_INF_F;
-    }
-    v[i] = t;
+    key[i] = e < E ? order_key(__ldcg(row + e)) : 0u;
   }
-  uint32_t avail = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (i < nper && lane + 32 * i < E) avail |= 1u << i;
-
   for (int j = 0; j < k; ++j) {
-    // Local best among available: larger value, ties to the lower index
-    // (i ascending means index ascending, so a strict '>' keeps the first).
-    float bv = -CUDART_INF_F;
-    int be = 0x7fffffff;
+    uint32_t bk = 0u;
+    int bi = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if ((avail >> i) & 1u) {
-        const int e = lane + 32 * i;
-        if (be == 0x7fffffff || v[i] > bv) {
-          bv = v[i];
-          be = e;
-        }
+    for (int i = 0; i < NPER; ++i)
+      if (key[i] > bk) {
+        bk = key[i];
+        bi = i;
       }
-    }
+    const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t mine = bk == wk ? uint32_t(lane + 32 * bi) : 0xffffffffu;
+    const uint32_t we = __reduce_min_sync(0xffffffffu, mine);
+    if (mine == we) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      const bool better = (oe != 0x7fffffff) && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be));
-      if (better) {
-        bv = ov;
-        be = oe;
-      }
+      for (int i = 0; i < NPER; ++i)
+        if (i == bi) key[i] = 0u;
     }
-    if ((be & 31) == lane) avail &= ~(1u << (be >> 5));
     if (lane == 0) {
-      s_val[j] = bv;
-      s_idx[j] = be;
+      s_val[j] = key_value(wk);
+      s_idx[j] = int(we);
     }
   }
   __syncwarp();
@@ -93,6 +87,11 @@ __device__ void warp_topk_row(const float* row, int E, int k, int* idx_out, floa
     w_out[j] = expf(s_val[j] - m) / denom;
   }
   __syncwarp();
+}
+__device__ void warp_topk_row(const float* row, int E, int k, int* idx_out, float* w_out, float* s_val,
+                              int* s_idx, const float* gbias) {
+  if (E <= 512) warp_topk_row_n<16>(row, E, k, idx_out, w_out, s_val, s_idx, gbias);
+  else warp_topk_row_n<32>(row, E, k, idx_out, w_out, s_val, s_idx, gbias);
 }
 
 // ---------------------------------------------------------------- decode GEMV
