@@ -21,7 +21,7 @@
 // one more group holding every token).
 //
 // Layout ("swap AB"): the weight rows are the MMA's M side (128 per tile),
-// tokens its N side (up to 128 per tile), so a small expert wastes no M.
+// tokens its N side (up to 128 per row tile), so a small expert wastes no M.
 // Activations are stored once, by `gather_rows_kernel`, as 16 KiB tiles of
 // 128 rows x 64 fp16 already in the 128-byte-swizzled K-major shared-memory
 // image, so one 1-D bulk copy loads a B tile. Inside every 8-element group
@@ -32,17 +32,21 @@
 // same tiled form, which is the down GEMM's B operand.
 //
 // Heavy groups (at least two row tiles) are dequantised once, before the
-// GEMMs, by `predequant_kernel` into A tiles of that same image; their tiles
-// then take A with a bulk copy next to B instead of from the dequant warps.
-//
-// Warp roles (448 threads, one CTA per SM, persistent over the tile list):
-//   warp 0      bulk-copy producer of B tiles (and of A for heavy groups),
-//               TMEM allocation
+// GEMMs, by `predequant_kernel` into A tiles of that same image, and run in
+// `wide_gemm_kernel`: tiles of two A tiles x 256 tokens (two row tiles), A
+// and B both taken by bulk copies. An MMA of N = 256 reads each A tile of
+// shared memory once for twice the tokens, which halves the A bytes per
+// multiply-add that come from L2 and that the tensor core reads from shared
+// memory (at 128 x 128 both streams are near their limits together).
+// The other groups' row tiles run in `grouped_gemm_kernel`, whose warps
+// dequantise A per tile:
+//   warp 0      bulk-copy producer of B tiles, TMEM allocation
 //   warp 1      MMA issuer (one thread)
 //   warps 2-5   epilogue (TMEM -> registers -> global)
-//   warps 6-13  dequant producers of A tiles (light groups)
-// Every wait is bounded; an expired wait flags MOE_ERR_TIMEOUT, stops the
-// CTA's loops, drains what it issued and frees TMEM.
+//   warps 6-13  dequant producers of A tiles
+// Both kernels are persistent (one CTA per SM over their tile lists). Every
+// wait is bounded; an expired wait flags MOE_ERR_TIMEOUT, stops the CTA's
+// loops, drains what it issued and frees TMEM.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -68,21 +72,49 @@ constexpr int kMaxHeavy = 64;
 // Row tiles: every group (routed expert e < E, or the shared expert = E) is
 // cut into tiles of at most BN rows. For each tile: group, first row (a
 // dispatched row, or a token for the shared group) and row count. Heavy
-// groups get a slot of pre-dequantised weights (hslot[g], -1 for none).
+// groups get a slot of pre-dequantised weights (hslot[g], -1 for none). The
+// row tiles of a heavy group are paired into wide tiles (rows 2j and 2j + 1
+// of the group; wlist holds the first), which `wide_gemm_kernel` runs; the
+// row tiles of the other groups are listed in llist for
+// `grouped_gemm_kernel`. A row tile is also the unit of the gathered
+// activations and of the gate/up output tiles, whichever kernel made them.
 struct Plan {
-  int* count;   // [1] number of row tiles; [1] number of heavy slots used
+  int* count;   // [0] row tiles, [1] heavy slots used, [2] wide tiles, [3] light row tiles
   int* group;   // [max]
   int* row0;    // [max]
   int* nrows;   // [max]
+  int* wlist;   // [max] first row tile of each wide tile
+  int* llist;   // [max] row tiles of the groups without a heavy slot
   int* hslot;   // [groups] heavy slot or -1
   int* hlist;   // [heavy slots] group of each slot
   int* tscaled; // [max] nonzero when a row of the tile has its x scaled (set by the gather)
 };
 
+// Exclusive prefix sum over the 1024 threads of the block; *total gets the sum.
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  __syncthreads();  // wsum free (a previous scan may still read it)
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  int wb = 0, tot = 0;
+  for (int i = 0; i < 32; ++i) {
+    if (i < w) wb += wsum[i];
+    tot += wsum[i];
+  }
+  *total = tot;
+  return wb + incl - v;
+}
+
 __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
-                                                    int E, int shared_rows, int max_tiles, int max_heavy, Plan plan) {
+                                                    int E, int shared_rows, int max_tiles, int max_heavy, Plan plan,
+                                                    WsHeader* hdr) {
   __shared__ int wsum[32];
-  __shared__ int hsum[32];
   const int ngroups = E + (shared_rows > 0 ? 1 : 0);
   const int g = threadIdx.x;
   for (int i = g; i < max_tiles; i += blockDim.x) plan.tscaled[i] = 0;
@@ -91,54 +123,38 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     const int n = g < E ? counts[g] : shared_rows;
     nt = (n + BN - 1) / BN;
   }
-  // block-wide exclusive scan of nt (1024 threads)
-  int incl = nt;
-  const int lane = g & 31, w = g >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) wsum[w] = incl;
-  __syncthreads();
-  int wb = 0, total = 0;
-  for (int i = 0; i < 32; ++i) {
-    if (i < w) wb += wsum[i];
-    total += wsum[i];
-  }
-  const int excl = wb + incl - nt;
-  // heavy groups: slots in group order (a second block-wide scan)
+  int total, htotal, wtotal, ltotal;
+  const int excl = block_excl_scan(nt, wsum, &total);
+  // heavy groups: slots in group order
   const int hv = (g < ngroups && nt >= 2) ? 1 : 0;  // n >= kHeavyRows
-  int hincl = hv;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, hincl, o);
-    if (lane >= o) hincl += v;
-  }
-  if (lane == 31) hsum[w] = hincl;
-  __syncthreads();
-  int hb = 0, htotal = 0;
-  for (int i = 0; i < 32; ++i) {
-    if (i < w) hb += hsum[i];
-    htotal += hsum[i];
-  }
-  const int hslot = hb + hincl - hv;
+  const int hslot = block_excl_scan(hv, wsum, &htotal);
+  const bool heavy = hv && hslot < max_heavy;
+  const int nw = heavy ? (nt + 1) / 2 : 0, nl = heavy ? 0 : nt;
+  const int wexcl = block_excl_scan(nw, wsum, &wtotal);
+  const int lexcl = block_excl_scan(nl, wsum, &ltotal);
+  const bool fits = total <= max_tiles;  // the host's bound covers every routing
   if (g < ngroups) {
-    const bool heavy = hv && hslot < max_heavy;
     plan.hslot[g] = heavy ? hslot : -1;
     if (heavy) plan.hlist[hslot] = g;
   }
-  if (g == 0) plan.count[1] = min(htotal, max_heavy);
-  if (g < ngroups) {
+  if (g == 0) {
+    plan.count[0] = fits ? total : 0;
+    plan.count[1] = min(htotal, max_heavy);
+    plan.count[2] = fits ? wtotal : 0;
+    plan.count[3] = fits ? ltotal : 0;
+    if (!fits) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 7000002);
+  }
+  if (g < ngroups && fits) {
     const int n = g < E ? counts[g] : shared_rows;
     const int r0 = g < E ? offsets[g] : 0;
-    for (int t = 0; t < nt && excl + t < max_tiles; ++t) {
+    for (int t = 0; t < nt; ++t) {
       plan.group[excl + t] = g;
       plan.row0[excl + t] = r0 + t * BN;
       plan.nrows[excl + t] = min(BN, n - t * BN);
     }
+    for (int j = 0; j < nw; ++j) plan.wlist[wexcl + j] = excl + 2 * j;
+    for (int t = 0; t < nl; ++t) plan.llist[lexcl + t] = excl + t;
   }
-  if (g == 0) plan.count[0] = min(total, max_tiles);
 }
 
 // Byte offset of element (row, k) inside a swizzled 128-row x 64-col 16-bit tile,
@@ -469,6 +485,65 @@ struct Args {
   WsHeader* hdr;
 };
 
+// ---------------------------------------------------------------- epilogues
+// Gate/up: 16 columns (rows c0 .. c0 + 15 of row tile rt) of weight row m,
+// g in v0 and u in v1 -> h = silu(g) u in fp16 into the H tiles (the down
+// GEMM's B: row c of tile rt, K index m), at tile_off(c0 + j, m & 63): c0 is
+// a multiple of 16, so the row's swizzle term (row & 7) is j & 7 and the
+// offsets are c0 * 128 plus constants of j.
+__device__ __forceinline__ void epi_h16(const Args& a, int rt, int m, int c0, int nrows, bool tile_scaled,
+                                        const uint32_t (&v0)[16], const uint32_t (&v1)[16]) {
+  const int kc = (m & 63) >> 3, e = m & 7;
+  uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes + size_t(c0) * 128 +
+                  (e < 4 ? 4 * e : 4 * (e - 4) + 2);
+  const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+  int xe[16] = {};
+  const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < nv) {
+      // the row's x was scaled by 2^-e: g = g_s 2^e, u = u_s 2^e, and
+      // h 2^-(kHShift + 2e) = silu(g) 2^-e u_s 2^-kHShift
+      float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]) * (1.0f / (1 << kHShift));
+      if (scaled) {
+        gv *= pow2f(xe[j]);
+        uv *= pow2f(-xe[j]);
+      }
+      *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) =
+          __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
+    }
+  }
+}
+
+// Down: 16 columns (rows c0 .. c0 + 15 of row tile rt, dispatched rows
+// row0 + c0 .. of group g) of output column m -> y, undoing the scaling of h:
+// y = y_s 2^(kHShift + 2e) for the row's e.
+__device__ __forceinline__ void epi_y16(const Args& a, int rt, int g, int row0, int m, int c0, int nrows,
+                                        bool tile_scaled, const uint32_t (&v0)[16]) {
+  const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+  int xe[16] = {};
+  const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
+  float yv[16];
+  if (!scaled) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) yv[j] = __uint_as_float(v0[j]) * float(1 << kHShift);
+  } else {  // 2^(kHShift + 2e) = 2^(kHShift + e) 2^e, each a normal float for e <= 119
+#pragma unroll
+    for (int j = 0; j < 16; ++j) yv[j] = __uint_as_float(v0[j]) * pow2f(kHShift + xe[j]) * pow2f(xe[j]);
+  }
+  if (g < a.E && a.y_f32 == nullptr) {
+    uint16_t* yp = a.y_bf16 + size_t(row0 + c0) * a.H + m;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < nv) yp[size_t(j) * a.H] = f32_to_bf16_rn(yv[j]);
+  } else {  // fp32 rows: column m of rows row0 + c0 .. (one pointer step of H per row)
+    float* yp = (g < a.E ? a.y_f32 : a.ys_f32) + size_t(row0 + c0) * a.H + m;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < nv) yp[size_t(j) * a.H] = yv[j];
+  }
+}
+
 // Raw-code staging: each dequant thread copies (cp.async) its own codes and
 // scales kRawDepth k-blocks ahead into a private area of shared memory.
 constexpr int kRawDepth = 3;
@@ -579,14 +654,8 @@ __device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, ui
   int ld_wrow = 0;
   auto resolve = [&](int lt) {
     const int t = int(blockIdx.x) + lt * int(gridDim.x);
-    const int rt = t / MT, mt = t - rt * MT;
-    const int g = a.plan.group[rt];
-    if (a.plan.hslot[g] >= 0) {  // heavy: the producer copies this tile's A
-#pragma unroll
-      for (int w = 0; w < NW; ++w) ld[w] = DqMat{nullptr, nullptr, nullptr, 0};
-      ld_wrow = 0;
-      return;
-    }
+    const int li = t / MT, mt = t - li * MT;
+    const int g = a.plan.group[a.plan.llist[li]];
     const moe_expert* ex = g < a.E ? a.experts + g : a.shared;
     ld_wrow = mt * BM + row;
     ld[0] = dq_mat(kGateUp ? ex->gate : ex->down, ld_wrow, a.M, a.K, a.hdr);
@@ -631,7 +700,7 @@ __device__ void dequant_role(const Args& a, uint8_t* smem, uint8_t* raw_smem, ui
           flag_error(a.hdr, MOE_ERR_TIMEOUT, 6000005);
           *abort_p = 1;
         } else {
-          if (qts[p][0] != 0) {  // qtype 0: a heavy tile (A copied in) or a flagged descriptor
+          if (qts[p][0] != 0) {  // qtype 0: a flagged descriptor
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
               uint4 o[4];
@@ -670,9 +739,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles_rows = a.plan.count[0];
+  const int nlight = a.plan.count[3];
   const int MT = a.M / BM, KB = a.K / BK;
-  const long long ntiles = (long long)ntiles_rows * MT;
+  const long long ntiles = (long long)nlight * MT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -710,23 +779,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       int s = 0;
       uint32_t ph = 0;
       for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
-        const int rt = int(t / MT), mt = int(t - (long long)rt * MT);
+        const int rt = a.plan.llist[int(t / MT)];
         const int nrows = a.plan.nrows[rt];
         const uint32_t bytes = uint32_t((nrows + 15) & ~15) * 128u;
-        const int hs = a.plan.hslot[a.plan.group[rt]];
-        const uint32_t abytes = hs >= 0 ? uint32_t(C::kATiles * kTileBytes) : 0u;
-        const uint8_t* asrc = hs >= 0 ? a.aimg + size_t(hs) * a.aslot + a.aoff + size_t(mt) * KB * abytes : nullptr;
         for (int kb = 0; kb < KB; ++kb) {
           if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
             fail(6000001);
             break;
           }
-          ptx::mbar_arrive_expect_tx(ptx::smem_addr(&full_bar[s]), bytes + abytes);
+          ptx::mbar_arrive_expect_tx(ptx::smem_addr(&full_bar[s]), bytes);
           ptx::bulk_g2s(ptx::smem_addr(stage_b(s)), a.bt + (size_t(rt) * KB + kb) * kTileBytes, bytes,
                         ptx::smem_addr(&full_bar[s]));
-          if (hs >= 0)
-            ptx::bulk_g2s(ptx::smem_addr(stage_a(s, 0)), asrc + size_t(kb) * abytes, abytes,
-                          ptx::smem_addr(&full_bar[s]));
           if (++s == C::kStages) {
             s = 0;
             ph ^= 1u;
@@ -741,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       uint32_t ph = 0;
       int it = 0;
       for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
-        const int rt = int(t / MT);
+        const int rt = a.plan.llist[int(t / MT)];
         const int nrows = a.plan.nrows[rt];
         const int N = (nrows + 15) & ~15;
         const uint32_t idesc = ptx::idesc_f16(BM, N);
@@ -791,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
     const int q = warp & 3;  // TMEM lane quarter this warp may read
     int it = 0;
     for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
-      const int rt = int(t / MT), mt = int(t % MT);
+      const int rt = a.plan.llist[int(t / MT)], mt = int(t % MT);
       const int nrows = a.plan.nrows[rt];
       const int g = a.plan.group[rt];
       const int row0 = a.plan.row0[rt];
@@ -812,55 +875,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
           uint32_t v1[16];
           ptx::tmem_ld16(taddr + 128u + uint32_t(c0), v1);
           ptx::tmem_ld_wait();
-          // h = silu(g) * u -> fp16 into the H tiles (K index m of the down GEMM),
-          // at tile_off(c0 + j, m & 63): c0 is a multiple of 16, so the row's
-          // swizzle term (row & 7) is j & 7 and the offsets are c0 * 128 plus
-          // constants of j
-          const int kc = (m & 63) >> 3, e = m & 7;
-          uint8_t* base = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes + size_t(c0) * 128 +
-                          (e < 4 ? 4 * e : 4 * (e - 4) + 2);
-          const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
-          int xe[16] = {};
-          const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j < nv) {
-              // the row's x was scaled by 2^-e: g = g_s 2^e, u = u_s 2^e, and
-              // h 2^-(kHShift + 2e) = silu(g) 2^-e u_s 2^-kHShift
-              float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]) * (1.0f / (1 << kHShift));
-              if (scaled) {
-                gv *= pow2f(xe[j]);
-                uv *= pow2f(-xe[j]);
-              }
-              *reinterpret_cast<__half*>(base + j * 128 + ((kc ^ (j & 7)) << 4)) =
-                  __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
-            }
-          }
+          epi_h16(a, rt, m, c0, nrows, tile_scaled, v0, v1);
         } else {
           ptx::tmem_ld_wait();
-          const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
-          // undo the scaling of h: y = y_s 2^(kHShift + 2e) for the row's e
-          int xe[16] = {};
-          const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
-          float yv[16];
-          if (!scaled) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) yv[j] = __uint_as_float(v0[j]) * float(1 << kHShift);
-          } else {  // 2^(kHShift + 2e) = 2^(kHShift + e) 2^e, each a normal float for e <= 119
-#pragma unroll
-            for (int j = 0; j < 16; ++j) yv[j] = __uint_as_float(v0[j]) * pow2f(kHShift + xe[j]) * pow2f(xe[j]);
-          }
-          if (g < a.E && a.y_f32 == nullptr) {
-            uint16_t* yp = a.y_bf16 + size_t(row0 + c0) * a.H + m;
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (j < nv) yp[size_t(j) * a.H] = f32_to_bf16_rn(yv[j]);
-          } else {  // fp32 rows: column m of rows row0 + c0 .. (one pointer step of H per row)
-            float* yp = (g < a.E ? a.y_f32 : a.ys_f32) + size_t(row0 + c0) * a.H + m;
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (j < nv) yp[size_t(j) * a.H] = yv[j];
-          }
+          epi_y16(a, rt, g, row0, m, c0, nrows, tile_scaled, v0);
         }
       }
       ptx::tc_fence_before();
@@ -876,6 +894,221 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
   if (warp == 0) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+
+// ---------------------------------------------------------------- wide tiles
+// Heavy groups (weights pre-dequantised into A tiles): tiles of two A tiles x
+// up to 256 tokens (a pair of row tiles). gate/up: A0 = gate rows
+// [128 mt, +128), A1 = up rows of the same range; down: A0 and A1 = down rows
+// [256 mt, +128) and [256 mt + 128, +128). One MMA of N = 256 takes each A
+// tile once for 256 tokens, so a k-block brings 64 KiB into shared memory for
+// 2 x 128 x 256 x 64 multiply-adds, and the tensor core reads 96 KiB of
+// shared memory for them: two thirds of the bytes per multiply-add of a
+// 128 x 128 tile with two A tiles, and half of those with one.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over the wide tiles):
+//   warp 0      bulk-copy producer (A tiles and the two B halves), TMEM allocation
+//   warp 1      MMA issuer (one thread)
+//   warps 2-9   epilogue: warp 2 + 4 c + i reads TMEM lane quarter (warp % 4)
+//               of token half c (row tile wlist[w] + c)
+// The accumulators take all 512 TMEM columns (A0's at 0, A1's at 256), so
+// the MMAs of a tile start once the previous tile's epilogue has read them.
+constexpr int kWStages = 3;
+constexpr int kWStageBytes = 4 * kTileBytes;  // A0, A1, B (256 rows)
+constexpr int kWEpiWarps = 8;
+constexpr int kWThreads = (2 + kWEpiWarps) * 32;
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kWStages], empty_bar[kWStages], accf_bar, acce_bar, drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwide = a.plan.count[2], nrt = a.plan.count[0];
+  // down: the last 256-row block holds only A0 when M / 128 is odd
+  const int MT = kGateUp ? a.M / BM : (a.M / BM + 1) / 2, KB = a.K / BK;
+  const long long ntiles = (long long)nwide * MT;
+  auto has_a1 = [&](int mt) { return kGateUp || 2 * mt + 1 < a.M / BM; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWStages; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&full_bar[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&empty_bar[s]), 1);
+    }
+    ptx::mbar_init(ptx::smem_addr(&accf_bar), 1);
+    ptx::mbar_init(ptx::smem_addr(&acce_bar), kWEpiWarps);
+    ptx::mbar_init(ptx::smem_addr(&drain_bar), 1);
+    abort_sh = 0;
+    ptx::mbar_init_fence();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_addr(&tmem_base_sh), 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int* abort_p = &abort_sh;
+
+  auto fail = [&](int where) {
+    flag_error(a.hdr, MOE_ERR_TIMEOUT, where);
+    *abort_p = 1;
+  };
+  // The two row tiles of wide tile w: the first (rt0, n0 rows) and its
+  // partner rt0 + 1 when it belongs to the same group (n1 rows, else 0).
+  auto halves = [&](int w, int& rt0, int& n0, int& n1) {
+    rt0 = a.plan.wlist[w];
+    n0 = a.plan.nrows[rt0];
+    n1 = (rt0 + 1 < nrt && a.plan.group[rt0 + 1] == a.plan.group[rt0]) ? a.plan.nrows[rt0 + 1] : 0;
+  };
+  auto stage = [&](int s) { return smem + size_t(s) * kWStageBytes; };
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, armed = 0, armed_ph = 0;  // bit i: stage i armed, and its phase
+      for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
+        const int w = int(t / MT), mt = int(t - (long long)w * MT);
+        int rt0, n0, n1;
+        halves(w, rt0, n0, n1);
+        const uint32_t b0 = uint32_t((n0 + 15) & ~15) * 128u, b1 = uint32_t((n1 + 15) & ~15) * 128u;
+        const int hs = a.plan.hslot[a.plan.group[rt0]];
+        if (hs < 0) {  // a wide tile always belongs to a group with a slot
+          flag_error(a.hdr, MOE_ERR_DEVICE_FAULT, 7000003);
+          *abort_p = 1;
+          break;
+        }
+        const uint8_t* img = a.aimg + size_t(hs) * a.aslot + a.aoff;
+        const bool a1 = has_a1(mt);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
+            fail(6000011);
+            break;
+          }
+          armed |= 1u << s;
+          armed_ph = (armed_ph & ~(1u << s)) | (ph << s);
+          const uint32_t bar = ptx::smem_addr(&full_bar[s]);
+          const uint32_t dst = ptx::smem_addr(stage(s));
+          ptx::mbar_arrive_expect_tx(bar, (a1 ? 2u : 1u) * kTileBytes + b0 + b1);
+          if (kGateUp) {  // image [mt][kb][gate, up]
+            ptx::bulk_g2s(dst, img + (size_t(mt) * KB + kb) * 2 * kTileBytes, 2u * kTileBytes, bar);
+          } else {        // image [128-row block][kb]
+            ptx::bulk_g2s(dst, img + (size_t(2 * mt) * KB + kb) * kTileBytes, kTileBytes, bar);
+            if (a1)
+              ptx::bulk_g2s(dst + kTileBytes, img + (size_t(2 * mt + 1) * KB + kb) * kTileBytes, kTileBytes, bar);
+          }
+          ptx::bulk_g2s(dst + 2u * kTileBytes, a.bt + (size_t(rt0) * KB + kb) * kTileBytes, b0, bar);
+          if (b1) ptx::bulk_g2s(dst + 3u * kTileBytes, a.bt + (size_t(rt0 + 1) * KB + kb) * kTileBytes, b1, bar);
+          if (++s == kWStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // After an abort, let the copies already issued land (bounded) before the
+      // CTA exits: a stage's full barrier waits for nothing but its bytes.
+      if (*abort_p)
+        for (int i = 0; i < kWStages; ++i)
+          if (armed & (1u << i)) ptx::mbar_wait(ptx::smem_addr(&full_bar[i]), (armed_ph >> i) & 1u, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
+        const int w = int(t / MT);
+        const bool a1 = has_a1(int(t - (long long)w * MT));
+        int rt0, n0, n1;
+        halves(w, rt0, n0, n1);
+        const uint32_t idesc = ptx::idesc_f16(BM, (n0 + n1 + 15) & ~15);
+        if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar), (uint32_t(it) & 1u) ^ 1u, abort_p)) {
+          fail(6000012);
+          break;
+        }
+        ptx::tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!ptx::mbar_wait(ptx::smem_addr(&full_bar[s]), ph, abort_p)) {
+            fail(6000013);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa0 = ptx::smem_addr(stage(s));
+          const uint32_t sb = sa0 + 2u * kTileBytes;
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks) {
+            const uint64_t bdesc = ptx::smem_desc_k128(sb + 32 * ks);
+            const uint32_t acc = (kb | ks) != 0;
+            ptx::mma_f16(tmem, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
+            if (a1) ptx::mma_f16(tmem + 256u, ptx::smem_desc_k128(sa0 + kTileBytes + 32 * ks), bdesc, idesc, acc);
+          }
+          ptx::mma_commit(ptx::smem_addr(&empty_bar[s]));
+          if (++s == kWStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_addr(&accf_bar));
+      }
+      // Drain: wait (bounded) for every MMA this thread issued.
+      ptx::mma_commit(ptx::smem_addr(&drain_bar));
+      ptx::mbar_wait(ptx::smem_addr(&drain_bar), 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;              // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;    // token half: row tile wlist[w] + half
+    int it = 0;
+    for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
+      const int w = int(t / MT), mt = int(t - (long long)w * MT);
+      int rt0, n0, n1;
+      halves(w, rt0, n0, n1);
+      if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar), uint32_t(it) & 1u, abort_p)) {
+        fail(6000014);
+        break;
+      }
+      ptx::tc_fence_after();
+      const int rt = rt0 + half, nrows = half ? n1 : n0;
+      if (nrows > 0) {
+        const int g = a.plan.group[rt], row0 = a.plan.row0[rt];
+        const bool tile_scaled = a.plan.tscaled[rt] != 0;
+        const bool a1 = has_a1(mt);
+        const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t(half * BN);
+        // weight row of this thread: gate/up row m of A0 and A1; down rows m and m + 128
+        const int m = (kGateUp ? mt * BM : mt * 2 * BM) + 32 * q + lane;
+        for (int c0 = 0; c0 < nrows; c0 += 16) {
+          uint32_t v0[16], v1[16];
+          ptx::tmem_ld16(taddr + uint32_t(c0), v0);
+          ptx::tmem_ld16(taddr + 256u + uint32_t(c0), v1);
+          ptx::tmem_ld_wait();
+          if (kGateUp) {
+            epi_h16(a, rt, m, c0, nrows, tile_scaled, v0, v1);
+          } else {
+            epi_y16(a, rt, g, row0, m, c0, nrows, tile_scaled, v0);
+            if (a1) epi_y16(a, rt, g, row0, m + BM, c0, nrows, tile_scaled, v1);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&acce_bar));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -907,7 +1140,7 @@ int grouped_heavy_slots(long long T, int k, bool with_shared, int H, int I) {
 
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
   const long long mt = grouped_max_tiles(T, k, E, with_shared);
-  return align256(16 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
+  return align256(20 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
          align256(4 * size_t(mt)) + align256(4 * size_t(mt) * gemm::BN) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(grouped_heavy_slots(T, k, with_shared, H, I)) * gemm::heavy_slot_bytes(H, I));
@@ -927,7 +1160,9 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   plan.group = plan.count + 4;
   plan.row0 = plan.group + mt;
   plan.nrows = plan.row0 + mt;
-  p += align256(16 * size_t(mt) + 16);
+  plan.wlist = plan.nrows + mt;
+  plan.llist = plan.wlist + mt;
+  p += align256(20 * size_t(mt) + 16);
   plan.hslot = reinterpret_cast<int*>(p);
   plan.hlist = plan.hslot + (E + 1);
   p += align256(4 * size_t(E + 1) + 4 * size_t(kMaxHeavy));
@@ -946,7 +1181,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
-  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), max_heavy, plan);
+  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), max_heavy, plan, hdr);
   gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt, xexp);
   if (max_heavy > 0) predequant_kernel<<<sms * 4, 256, 0, st>>>(experts, shared, E, H, I, plan, aimg, hdr);
   const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
@@ -955,6 +1190,11 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
                                        int(smem_gu));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_dn));
+  if (e != cudaSuccess) return e;
+  const size_t smem_w = size_t(kWStages) * kWStageBytes + 1024;
+  e = cudaFuncSetAttribute(wide_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_w));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(wide_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_w));
   if (e != cudaSuccess) return e;
   Args a{};
   a.plan = plan;
@@ -973,6 +1213,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.bt = xt;
   a.ht = ht;
   a.aoff = 0;
+  if (max_heavy > 0) wide_gemm_kernel<true><<<sms, kWThreads, smem_w, st>>>(a);
   grouped_gemm_kernel<true><<<sms, kThreads, smem_gu, st>>>(a);
   // down: K = I, M = H; B = H tiles; out = rows
   a.K = I;
@@ -983,8 +1224,9 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.y_f32 = y_f32;
   a.y_bf16 = y_bf16;
   a.ys_f32 = ys_f32;
+  if (max_heavy > 0) wide_gemm_kernel<false><<<sms, kWThreads, smem_w, st>>>(a);
   grouped_gemm_kernel<false><<<sms, kThreads, smem_dn, st>>>(a);
-  count_launches(max_heavy > 0 ? 5 : 4);
+  count_launches(max_heavy > 0 ? 7 : 4);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,9 @@
 """Host-side sizing of the prefill grouped GEMM, checked on the CPU.
 
 A host program (nvcc, no GPU) includes expert_gemm_sm100.cu and checks what
-the kernels rely on: both GEMMs' dynamic shared memory (stage ring plus the
-dequant warps' raw-code staging) fits the per-CTA limit, the row-tile bound
+the kernels rely on: the dynamic shared memory of both dequantising GEMMs
+(stage ring plus the dequant warps' raw-code staging) and of the wide-tile
+GEMM (three 64 KiB stages) fits the per-CTA limit, the row-tile bound
 covers every routing, and the heavy-slot bound covers every routing's groups
 of more than one row tile (up to the slot cap), on seeded random routings
 with a skewed expert popularity.
@@ -29,6 +30,7 @@ int main() {
   const size_t limit = 227 * 1024;
   const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
   const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
+  const size_t smem_w = size_t(kWStages) * kWStageBytes + 1024;
   int bad_tiles = 0, bad_heavy = 0, cases = 0;
   std::mt19937 rng(12345);
   const int Ts[] = {5, 37, 300, 1000, 8192};
@@ -69,9 +71,9 @@ int main() {
           }
         }
       }
-  printf("{\"smem_gu\": %zu, \"smem_dn\": %zu, \"limit\": %zu, \"bad_tiles\": %d, \"bad_heavy\": %d, \"cases\": %d, "
+  printf("{\"smem_gu\": %zu, \"smem_dn\": %zu, \"smem_w\": %zu, \"limit\": %zu, \"bad_tiles\": %d, \"bad_heavy\": %d, \"cases\": %d, "
          "\"ws_8k\": %zu, \"ws_32k\": %zu}\n",
-         smem_gu, smem_dn, limit, bad_tiles, bad_heavy, cases, grouped_ws_bytes(8192, 2048, 768, 10, 512, true),
+         smem_gu, smem_dn, smem_w, limit, bad_tiles, bad_heavy, cases, grouped_ws_bytes(8192, 2048, 768, 10, 512, true),
          grouped_ws_bytes(32768, 2048, 768, 10, 512, true));
   return 0;
 }
@@ -94,8 +96,9 @@ def report(tmp_path_factory):
     return json.loads(out.stdout.strip().splitlines()[-1])
 
 
-def test_both_gemms_fit_shared_memory(report):
+def test_every_gemm_fits_shared_memory(report):
     assert report["smem_gu"] <= report["limit"] and report["smem_dn"] <= report["limit"]
+    assert report["smem_w"] <= report["limit"]
 
 
 def test_row_tile_bound_covers_every_routing(report):

@@ -56,6 +56,11 @@ SMALL = {
     # E a multiple of 128 and T > 4: the tensor-core router (three-way bf16 split of W_r)
     "tc_router": wlm.Workload("tc_router", T=300, H=512, I=256, E=128, k=4, zipf_s=0.9, seed=15),
     "tc_skew": wlm.Workload("tc_skew", T=1000, H=256, I=128, E=64, k=3, zipf_s=2.0, seed=14),
+    # groups of 5, 3 and 2 row tiles (and the shared expert's 5) paired into
+    # 256-token tiles, each with a partial last tile; H / 128 odd, so the down
+    # GEMM's last 256-row weight block holds one 128-row tile
+    "tc_wide_odd_h": wlm.Workload("tc_wide_odd_h", T=600, H=384, I=256, E=10, k=2, zipf_s=0.8, seed=20,
+                                  routed_qtypes=((0, 7, wlm.Q_INT4_SYM_G32), (7, None, wlm.Q_INT2_ASYM_G16))),
     "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
                               shared_qtype=wlm.Q_INT2_ASYM_G16),
     # 256 routed experts (the pages' Coder variant keeps half of the 512) on
