@@ -544,6 +544,128 @@ __device__ __forceinline__ void epi_y16(const Args& a, int rt, int g, int row0, 
   }
 }
 
+// Staged epilogues for a warp's 32 weight rows m = mbase + lane (mbase a
+// multiple of 32) and 16 tokens: the warp writes its outputs into its own
+// shared-memory scratch in the destination's byte order and then stores them
+// as 16-byte pieces, one store instruction per lane for 4 fp32 or 8 fp16/bf16
+// values instead of one per value. fp32 rows first:
+constexpr int kEpiScratch = 2048;  // bytes of scratch per epilogue warp
+
+__device__ __forceinline__ void epi_y16_f32_staged(const Args& a, int rt, int g, int row0, int mbase, int c0,
+                                                   int nrows, bool tile_scaled, const uint32_t (&v0)[16],
+                                                   uint8_t* scr) {
+  const int lane = threadIdx.x & 31;
+  const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+  int xe[16] = {};
+  const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
+  float* s32 = reinterpret_cast<float*>(scr);
+#pragma unroll
+  for (int j = 0; j < 16; ++j)  // undo the scaling of h: y = y_s 2^(kHShift + 2e) for the row's e
+    s32[j * 32 + lane] = scaled ? __uint_as_float(v0[j]) * pow2f(kHShift + xe[j]) * pow2f(xe[j])
+                                : __uint_as_float(v0[j]) * float(1 << kHShift);
+  __syncwarp();
+  float* y = g < a.E ? a.y_f32 : a.ys_f32;  // 128 contiguous bytes per token
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int p = lane + 32 * i;  // token p / 8, 4 values p % 8
+    const int j = p >> 3, part = p & 7;
+    if (j < nv)
+      *reinterpret_cast<uint4*>(y + size_t(row0 + c0 + j) * a.H + mbase + part * 4) =
+          *reinterpret_cast<const uint4*>(scr + j * 128 + part * 16);
+  }
+  __syncwarp();
+}
+
+// 16-bit outputs (fp16 h, bf16 y) in token pairs: each lane converts two
+// tokens' values of its column with one paired conversion and stores them as
+// one 32-bit word ([token pair][column] in the scratch); the read-back splits
+// the pairs with byte permutes into one 16-byte piece for each of the two
+// tokens.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void epi_h16_pairs(const Args& a, int rt, int mbase, int c0, int nrows, bool tile_scaled,
+                                              const uint32_t (&v0)[16], const uint32_t (&v1)[16], uint8_t* scr) {
+  const int lane = threadIdx.x & 31;
+  const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+  int xe[16] = {};
+  const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
+  uint32_t* s32 = reinterpret_cast<uint32_t*>(scr);
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    float h[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int j = 2 * jj + t;
+      // the row's x was scaled by 2^-e: g = g_s 2^e, u = u_s 2^e, and
+      // h 2^-(kHShift + 2e) = silu(g) 2^-e u_s 2^-kHShift
+      float gv = __uint_as_float(v0[j]), uv = __uint_as_float(v1[j]) * (1.0f / (1 << kHShift));
+      if (scaled) {
+        gv *= pow2f(xe[j]);
+        uv *= pow2f(-xe[j]);
+      }
+      h[t] = sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
+    }
+    s32[jj * 32 + lane] = h2_bits(h[0], h[1]);
+  }
+  __syncwarp();
+  // lane: token pair jj, 16-byte chunk kcl = K values 8 kcl + (0..7) of its
+  // 64-K block half, in the order (0,4,1,5,2,6,3,7)
+  const int jj = lane >> 2, kcl = lane & 3;
+  const uint4 w0 = *reinterpret_cast<const uint4*>(s32 + jj * 32 + kcl * 8);
+  const uint4 w1 = *reinterpret_cast<const uint4*>(s32 + jj * 32 + kcl * 8 + 4);
+  const uint4 ev = make_uint4(__byte_perm(w0.x, w1.x, 0x5410), __byte_perm(w0.y, w1.y, 0x5410),
+                              __byte_perm(w0.z, w1.z, 0x5410), __byte_perm(w0.w, w1.w, 0x5410));
+  const uint4 od = make_uint4(__byte_perm(w0.x, w1.x, 0x7632), __byte_perm(w0.y, w1.y, 0x7632),
+                              __byte_perm(w0.z, w1.z, 0x7632), __byte_perm(w0.w, w1.w, 0x7632));
+  const int kc = 4 * ((mbase & 63) >> 5) + kcl;
+  uint8_t* tile = a.ht + (size_t(rt) * (a.I / BK) + (mbase >> 6)) * kTileBytes;
+  const int r0 = c0 + 2 * jj;
+  if (2 * jj < nv) *reinterpret_cast<uint4*>(tile + size_t(r0) * 128 + ((kc ^ (r0 & 7)) << 4)) = ev;
+  if (2 * jj + 1 < nv) *reinterpret_cast<uint4*>(tile + size_t(r0 + 1) * 128 + ((kc ^ ((r0 + 1) & 7)) << 4)) = od;
+  __syncwarp();
+}
+
+__device__ __forceinline__ void epi_y16_pairs(const Args& a, int rt, int g, int row0, int mbase, int c0, int nrows,
+                                              bool tile_scaled, const uint32_t (&v0)[16], uint8_t* scr) {
+  if (!(g < a.E && a.y_f32 == nullptr)) {  // fp32 rows
+    epi_y16_f32_staged(a, rt, g, row0, mbase, c0, nrows, tile_scaled, v0, scr);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int nv = nrows - c0 < 16 ? nrows - c0 : 16;
+  int xe[16] = {};
+  const bool scaled = tile_scaled && row_exps(a.xexp + size_t(rt) * BN + c0, xe);
+  uint32_t* s32 = reinterpret_cast<uint32_t*>(scr);
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    float y2[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int j = 2 * jj + t;
+      // undo the scaling of h: y = y_s 2^(kHShift + 2e) for the row's e
+      y2[t] = scaled ? __uint_as_float(v0[j]) * pow2f(kHShift + xe[j]) * pow2f(xe[j])
+                     : __uint_as_float(v0[j]) * float(1 << kHShift);
+    }
+    s32[jj * 32 + lane] = pack_bf16x2(y2[0], y2[1]);
+  }
+  __syncwarp();
+  // lane: token pair jj, columns mbase + 8 cg .. + 7
+  const int jj = lane >> 2, cg = lane & 3;
+  const uint4 w0 = *reinterpret_cast<const uint4*>(s32 + jj * 32 + cg * 8);
+  const uint4 w1 = *reinterpret_cast<const uint4*>(s32 + jj * 32 + cg * 8 + 4);
+  const uint4 ev = make_uint4(__byte_perm(w0.x, w0.y, 0x5410), __byte_perm(w0.z, w0.w, 0x5410),
+                              __byte_perm(w1.x, w1.y, 0x5410), __byte_perm(w1.z, w1.w, 0x5410));
+  const uint4 od = make_uint4(__byte_perm(w0.x, w0.y, 0x7632), __byte_perm(w0.z, w0.w, 0x7632),
+                              __byte_perm(w1.x, w1.y, 0x7632), __byte_perm(w1.z, w1.w, 0x7632));
+  uint16_t* y = a.y_bf16 + size_t(row0 + c0 + 2 * jj) * a.H + mbase + cg * 8;
+  if (2 * jj < nv) *reinterpret_cast<uint4*>(y) = ev;
+  if (2 * jj + 1 < nv) *reinterpret_cast<uint4*>(y + a.H) = od;
+  __syncwarp();
+}
+
 // Raw-code staging: each dequant thread copies (cp.async) its own codes and
 // scales kRawDepth k-blocks ahead into a private area of shared memory.
 constexpr int kRawDepth = 3;
@@ -627,7 +749,7 @@ __device__ __forceinline__ void raw_issue(const DqMat& d, int k0, uint8_t* slot,
 __device__ __forceinline__ void raw_read(const uint8_t* slot, int w, int dt, int qtype, int k0, bool odd_row_scale,
                                          RawK& r) {
   r.c0 = *reinterpret_cast<const uint4*>(slot + ((w * 2 + 0) * 256 + dt) * 16);
-  r.c1 = *reinterpret_cast<const uint4*>(slot + ((w * 2 + 1) * 256 + dt) * 16);
+  if (qtype == MOE_Q_INT8_PER_CHANNEL) r.c1 = *reinterpret_cast<const uint4*>(slot + ((w * 2 + 1) * 256 + dt) * 16);
   const uint2 aux = *reinterpret_cast<const uint2*>(slot + kRawCodeBytes + (w * 256 + dt) * 8);
   if (qtype == MOE_Q_INT4_SYM_G32) {
     r.s = ((k0 / 32) & 1) ? (aux.x >> 16) : (aux.x & 0xffffu);
@@ -783,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
         const int nrows = a.plan.nrows[rt];
         const uint32_t bytes = uint32_t((nrows + 15) & ~15) * 128u;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!ptx::mbar_wait(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p)) {
+          if (!ptx::mbar_wait_sleep(ptx::smem_addr(&empty_bar[s]), ph ^ 1u, abort_p, 64)) {
             fail(6000001);
             break;
           }
@@ -860,7 +982,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
       const int row0 = a.plan.row0[rt];
       const int buf = it & 1;
       const uint32_t use = uint32_t(it >> 1) & 1u;
-      if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar[buf]), use, abort_p)) {
+      // double-buffered accumulators: the epilogue's wake-up latency is hidden
+      if (!ptx::mbar_wait_sleep(ptx::smem_addr(&accf_bar[buf]), use, abort_p, 256)) {
         fail(6000004);
         break;
       }
@@ -899,49 +1022,70 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(Args a) {
 
 
 // ---------------------------------------------------------------- wide tiles
-// Heavy groups (weights pre-dequantised into A tiles): tiles of two A tiles x
-// up to 256 tokens (a pair of row tiles). gate/up: A0 = gate rows
-// [128 mt, +128), A1 = up rows of the same range; down: A0 and A1 = down rows
-// [256 mt, +128) and [256 mt + 128, +128). One MMA of N = 256 takes each A
-// tile once for 256 tokens, so a k-block brings 64 KiB into shared memory for
-// 2 x 128 x 256 x 64 multiply-adds, and the tensor core reads 96 KiB of
-// shared memory for them: two thirds of the bytes per multiply-add of a
-// 128 x 128 tile with two A tiles, and half of those with one.
+// Heavy groups (weights pre-dequantised into A tiles) run in
+// `wide_gemm_kernel<kGateUp, NA, NB>`: tiles of NA A tiles (128 weight rows
+// each) x NB tokens (one or two row tiles of the group), both operands taken
+// by bulk copies. gate/up: NA = 2, A0 = gate rows [128 mt, +128), A1 = the up
+// rows of the same range; down: A0 (and A1) = down rows [128 NA mt, +128)
+// (and the next 128). One MMA of N = 256 takes each A tile once for 256
+// tokens, halving the A bytes per multiply-add that come from L2 and that the
+// tensor core reads from shared memory, next to N = 128. The accumulators of a
+// tile take NA x NB TMEM columns: with 512 a tile's MMAs start once the
+// previous tile's epilogue has read them, with 256 they alternate between two
+// buffers and the epilogue overlaps the next tile's main loop.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over the wide tiles):
-//   warp 0      bulk-copy producer (A tiles and the two B halves), TMEM allocation
+// Warp roles (320 threads, one CTA per SM, persistent over the tiles):
+//   warp 0      bulk-copy producer (A tiles and the B rows), TMEM allocation
 //   warp 1      MMA issuer (one thread)
-//   warps 2-9   epilogue: warp 2 + 4 c + i reads TMEM lane quarter (warp % 4)
-//               of token half c (row tile wlist[w] + c)
-// The accumulators take all 512 TMEM columns (A0's at 0, A1's at 256), so
-// the MMAs of a tile start once the previous tile's epilogue has read them.
-constexpr int kWStages = 3;
-constexpr int kWStageBytes = 4 * kTileBytes;  // A0, A1, B (256 rows)
+//   warps 2-9   epilogue: warp 2 + 4 p + i reads TMEM lane quarter (warp % 4)
+//               for token part p (of two) of the tile
+template <int NA, int NB>
+struct WCfg {
+  static constexpr int kStageBytes = (NA + NB / BN) * kTileBytes;
+  static constexpr int kAccCols = NA * NB;        // one tile's accumulators
+  static constexpr int kBufs = 512 / kAccCols;    // 1 or 2
+  static constexpr int kStages = (200 * 1024) / kStageBytes < 6 ? (200 * 1024) / kStageBytes : 6;
+};
 constexpr int kWEpiWarps = 8;
 constexpr int kWThreads = (2 + kWEpiWarps) * 32;
+// Tile shapes of the two GEMMs (A tiles x tokens).
+constexpr int kGuNA = 2, kGuNB = 256;
+constexpr int kDnNA = 1, kDnNB = 256;
+template <int NA, int NB>
+constexpr size_t wide_smem_bytes() {
+  return size_t(WCfg<NA, NB>::kStages) * WCfg<NA, NB>::kStageBytes + size_t(kWEpiWarps) * kEpiScratch + 1024;
+}
 
-template <bool kGateUp>
+template <bool kGateUp, int NA, int NB>
 __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
+  using C = WCfg<NA, NB>;
+  static_assert(!kGateUp || NA == 2, "gate/up tiles hold the gate and the up rows");
+  static_assert(C::kBufs * C::kAccCols == 512, "accumulators fill TMEM");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full_bar[kWStages], empty_bar[kWStages], accf_bar, acce_bar, drain_bar;
+  __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages], accf_bar[C::kBufs],
+      acce_bar[C::kBufs], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwide = a.plan.count[2], nrt = a.plan.count[0];
-  // down: the last 256-row block holds only A0 when M / 128 is odd
-  const int MT = kGateUp ? a.M / BM : (a.M / BM + 1) / 2, KB = a.K / BK;
-  const long long ntiles = (long long)nwide * MT;
-  auto has_a1 = [&](int mt) { return kGateUp || 2 * mt + 1 < a.M / BM; };
+  // weight-row blocks: gate/up one 128-row block per tile; down NA blocks per
+  // tile, the last holding only A0 when M / 128 is not a multiple of NA
+  const int MT = kGateUp ? a.M / BM : (a.M / BM + NA - 1) / NA, KB = a.K / BK;
+  constexpr int kParts = NB / BN;  // row tiles per tile: token slots of a wide tile
+  const long long ntiles = (long long)nwide * (2 / kParts) * MT;
+  auto has_a1 = [&](int mt) { return NA == 2 && (kGateUp || 2 * mt + 1 < a.M / BM); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kWStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       ptx::mbar_init(ptx::smem_addr(&full_bar[s]), 1);
       ptx::mbar_init(ptx::smem_addr(&empty_bar[s]), 1);
     }
-    ptx::mbar_init(ptx::smem_addr(&accf_bar), 1);
-    ptx::mbar_init(ptx::smem_addr(&acce_bar), kWEpiWarps);
+    for (int b = 0; b < C::kBufs; ++b) {
+      ptx::mbar_init(ptx::smem_addr(&accf_bar[b]), 1);
+      ptx::mbar_init(ptx::smem_addr(&acce_bar[b]), kWEpiWarps);
+    }
     ptx::mbar_init(ptx::smem_addr(&drain_bar), 1);
     abort_sh = 0;
     ptx::mbar_init_fence();
@@ -960,14 +1104,27 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
     flag_error(a.hdr, MOE_ERR_TIMEOUT, where);
     *abort_p = 1;
   };
-  // The two row tiles of wide tile w: the first (rt0, n0 rows) and its
-  // partner rt0 + 1 when it belongs to the same group (n1 rows, else 0).
-  auto halves = [&](int w, int& rt0, int& n0, int& n1) {
-    rt0 = a.plan.wlist[w];
-    n0 = a.plan.nrows[rt0];
-    n1 = (rt0 + 1 < nrt && a.plan.group[rt0 + 1] == a.plan.group[rt0]) ? a.plan.nrows[rt0 + 1] : 0;
+  // Tile t: weight block mt and its tokens: the row tiles rt0 (n0 rows) and,
+  // for NB = 256, its partner rt0 + 1 when that belongs to the same group (n1
+  // rows, else 0). For NB = 128 a wide tile's two row tiles are two tiles (the
+  // second skipped when empty).
+  auto tile_of = [&](long long t, int& mt, int& rt0, int& n0, int& n1) {
+    const long long u = t / MT;
+    mt = int(t - u * MT);
+    const int w = int(u / (2 / kParts)), second = int(u - (long long)w * (2 / kParts));
+    const int r = a.plan.wlist[w];
+    const bool pair = r + 1 < nrt && a.plan.group[r + 1] == a.plan.group[r];
+    if (kParts == 2) {
+      rt0 = r;
+      n0 = a.plan.nrows[r];
+      n1 = pair ? a.plan.nrows[r + 1] : 0;
+    } else {
+      rt0 = r + second;
+      n0 = (second == 0 || pair) ? a.plan.nrows[rt0] : 0;
+      n1 = 0;
+    }
   };
-  auto stage = [&](int s) { return smem + size_t(s) * kWStageBytes; };
+  auto stage = [&](int s) { return smem + size_t(s) * C::kStageBytes; };
 
   if (warp == 0) {
     // ------------------------------------------------ producer
@@ -975,9 +1132,9 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
       int s = 0;
       uint32_t ph = 0, armed = 0, armed_ph = 0;  // bit i: stage i armed, and its phase
       for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
-        const int w = int(t / MT), mt = int(t - (long long)w * MT);
-        int rt0, n0, n1;
-        halves(w, rt0, n0, n1);
+        int mt, rt0, n0, n1;
+        tile_of(t, mt, rt0, n0, n1);
+        if (n0 == 0) continue;  // the empty second row tile of a single one
         const uint32_t b0 = uint32_t((n0 + 15) & ~15) * 128u, b1 = uint32_t((n1 + 15) & ~15) * 128u;
         const int hs = a.plan.hslot[a.plan.group[rt0]];
         if (hs < 0) {  // a wide tile always belongs to a group with a slot
@@ -1000,13 +1157,14 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
           if (kGateUp) {  // image [mt][kb][gate, up]
             ptx::bulk_g2s(dst, img + (size_t(mt) * KB + kb) * 2 * kTileBytes, 2u * kTileBytes, bar);
           } else {        // image [128-row block][kb]
-            ptx::bulk_g2s(dst, img + (size_t(2 * mt) * KB + kb) * kTileBytes, kTileBytes, bar);
+            ptx::bulk_g2s(dst, img + (size_t(NA * mt) * KB + kb) * kTileBytes, kTileBytes, bar);
             if (a1)
-              ptx::bulk_g2s(dst + kTileBytes, img + (size_t(2 * mt + 1) * KB + kb) * kTileBytes, kTileBytes, bar);
+              ptx::bulk_g2s(dst + kTileBytes, img + (size_t(NA * mt + 1) * KB + kb) * kTileBytes, kTileBytes, bar);
           }
-          ptx::bulk_g2s(dst + 2u * kTileBytes, a.bt + (size_t(rt0) * KB + kb) * kTileBytes, b0, bar);
-          if (b1) ptx::bulk_g2s(dst + 3u * kTileBytes, a.bt + (size_t(rt0 + 1) * KB + kb) * kTileBytes, b1, bar);
-          if (++s == kWStages) {
+          const uint32_t db = dst + uint32_t(NA) * kTileBytes;
+          ptx::bulk_g2s(db, a.bt + (size_t(rt0) * KB + kb) * kTileBytes, b0, bar);
+          if (b1) ptx::bulk_g2s(db + kTileBytes, a.bt + (size_t(rt0 + 1) * KB + kb) * kTileBytes, b1, bar);
+          if (++s == C::kStages) {
             s = 0;
             ph ^= 1u;
           }
@@ -1015,7 +1173,7 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
       // After an abort, let the copies already issued land (bounded) before the
       // CTA exits: a stage's full barrier waits for nothing but its bytes.
       if (*abort_p)
-        for (int i = 0; i < kWStages; ++i)
+        for (int i = 0; i < C::kStages; ++i)
           if (armed & (1u << i)) ptx::mbar_wait(ptx::smem_addr(&full_bar[i]), (armed_ph >> i) & 1u, nullptr);
     }
   } else if (warp == 1) {
@@ -1024,17 +1182,20 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
-      for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
-        const int w = int(t / MT);
-        const bool a1 = has_a1(int(t - (long long)w * MT));
-        int rt0, n0, n1;
-        halves(w, rt0, n0, n1);
+      for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
+        int mt, rt0, n0, n1;
+        tile_of(t, mt, rt0, n0, n1);
+        if (n0 == 0) continue;
+        const bool a1 = has_a1(mt);
         const uint32_t idesc = ptx::idesc_f16(BM, (n0 + n1 + 15) & ~15);
-        if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar), (uint32_t(it) & 1u) ^ 1u, abort_p)) {
+        const int buf = it % C::kBufs;
+        const uint32_t use = uint32_t(it / C::kBufs) & 1u;
+        if (!ptx::mbar_wait(ptx::smem_addr(&acce_bar[buf]), use ^ 1u, abort_p)) {
           fail(6000012);
           break;
         }
         ptx::tc_fence_after();
+        const uint32_t d0 = tmem + uint32_t(buf * C::kAccCols);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           if (!ptx::mbar_wait(ptx::smem_addr(&full_bar[s]), ph, abort_p)) {
@@ -1044,22 +1205,23 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
           }
           ptx::tc_fence_after();
           const uint32_t sa0 = ptx::smem_addr(stage(s));
-          const uint32_t sb = sa0 + 2u * kTileBytes;
+          const uint32_t sb = sa0 + uint32_t(NA) * kTileBytes;
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t bdesc = ptx::smem_desc_k128(sb + 32 * ks);
             const uint32_t acc = (kb | ks) != 0;
-            ptx::mma_f16(tmem, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
-            if (a1) ptx::mma_f16(tmem + 256u, ptx::smem_desc_k128(sa0 + kTileBytes + 32 * ks), bdesc, idesc, acc);
+            ptx::mma_f16(d0, ptx::smem_desc_k128(sa0 + 32 * ks), bdesc, idesc, acc);
+            if (a1) ptx::mma_f16(d0 + uint32_t(NB), ptx::smem_desc_k128(sa0 + kTileBytes + 32 * ks), bdesc, idesc, acc);
           }
           ptx::mma_commit(ptx::smem_addr(&empty_bar[s]));
-          if (++s == kWStages) {
+          if (++s == C::kStages) {
             s = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        ptx::mma_commit(ptx::smem_addr(&accf_bar));
+        ptx::mma_commit(ptx::smem_addr(&accf_bar[buf]));
+        ++it;
       }
       // Drain: wait (bounded) for every MMA this thread issued.
       ptx::mma_commit(ptx::smem_addr(&drain_bar));
@@ -1067,42 +1229,59 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
     }
   } else {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;              // TMEM lane quarter this warp may read
-    const int half = (warp - 2) >> 2;    // token half: row tile wlist[w] + half
+    const int q = warp & 3;            // TMEM lane quarter this warp may read
+    const int part = (warp - 2) >> 2;  // token part of the tile: NB / 2 tokens
+    uint8_t* scr = smem + size_t(C::kStages) * C::kStageBytes + size_t(warp - 2) * kEpiScratch;
     int it = 0;
-    for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x, ++it) {
-      const int w = int(t / MT), mt = int(t - (long long)w * MT);
-      int rt0, n0, n1;
-      halves(w, rt0, n0, n1);
-      if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar), uint32_t(it) & 1u, abort_p)) {
+    for (long long t = blockIdx.x; t < ntiles && !*abort_p; t += gridDim.x) {
+      int mt, rt0, n0, n1;
+      tile_of(t, mt, rt0, n0, n1);
+      if (n0 == 0) continue;
+      const int buf = it % C::kBufs;
+      const uint32_t use = uint32_t(it / C::kBufs) & 1u;
+      if (!ptx::mbar_wait(ptx::smem_addr(&accf_bar[buf]), use, abort_p)) {
         fail(6000014);
         break;
       }
       ptx::tc_fence_after();
-      const int rt = rt0 + half, nrows = half ? n1 : n0;
-      if (nrows > 0) {
+      // this warp's tokens: row tile rt, rows [c_lo, c_hi) of it, at TMEM column col0 + (row - c_lo)
+      int rt, c_lo, c_hi, col0;
+      if (kParts == 2) {
+        rt = rt0 + part;
+        c_lo = 0;
+        c_hi = part ? n1 : n0;
+        col0 = part * BN;
+      } else {
+        rt = rt0;
+        c_lo = part * (BN / 2);
+        c_hi = n0 < c_lo + BN / 2 ? n0 : c_lo + BN / 2;
+        col0 = c_lo;
+      }
+      if (c_hi > c_lo) {
         const int g = a.plan.group[rt], row0 = a.plan.row0[rt];
         const bool tile_scaled = a.plan.tscaled[rt] != 0;
         const bool a1 = has_a1(mt);
-        const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t(half * BN);
-        // weight row of this thread: gate/up row m of A0 and A1; down rows m and m + 128
-        const int m = (kGateUp ? mt * BM : mt * 2 * BM) + 32 * q + lane;
-        for (int c0 = 0; c0 < nrows; c0 += 16) {
+        const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + uint32_t(buf * C::kAccCols + col0 - c_lo);
+        // weight rows of this warp: gate/up rows mbase + lane of A0 and A1;
+        // down rows mbase + lane (and mbase + 128 + lane)
+        const int mbase = (kGateUp ? mt * BM : mt * NA * BM) + 32 * q;
+        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
           uint32_t v0[16], v1[16];
           ptx::tmem_ld16(taddr + uint32_t(c0), v0);
-          ptx::tmem_ld16(taddr + 256u + uint32_t(c0), v1);
+          if (a1) ptx::tmem_ld16(taddr + uint32_t(NB + c0), v1);
           ptx::tmem_ld_wait();
           if (kGateUp) {
-            epi_h16(a, rt, m, c0, nrows, tile_scaled, v0, v1);
+            epi_h16_pairs(a, rt, mbase, c0, c_hi, tile_scaled, v0, v1, scr);
           } else {
-            epi_y16(a, rt, g, row0, m, c0, nrows, tile_scaled, v0);
-            if (a1) epi_y16(a, rt, g, row0, m + BM, c0, nrows, tile_scaled, v1);
+            epi_y16_pairs(a, rt, g, row0, mbase, c0, c_hi, tile_scaled, v0, scr);
+            if (a1) epi_y16_pairs(a, rt, g, row0, mbase + BM, c0, c_hi, tile_scaled, v1, scr);
           }
         }
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&acce_bar));
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_addr(&acce_bar[buf]));
+      ++it;
     }
   }
   __syncthreads();
@@ -1191,10 +1370,12 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_dn));
   if (e != cudaSuccess) return e;
-  const size_t smem_w = size_t(kWStages) * kWStageBytes + 1024;
-  e = cudaFuncSetAttribute(wide_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_w));
+  const size_t smem_wgu = wide_smem_bytes<kGuNA, kGuNB>(), smem_wdn = wide_smem_bytes<kDnNA, kDnNB>();
+  e = cudaFuncSetAttribute(wide_gemm_kernel<true, kGuNA, kGuNB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(smem_wgu));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(wide_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_w));
+  e = cudaFuncSetAttribute(wide_gemm_kernel<false, kDnNA, kDnNB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(smem_wdn));
   if (e != cudaSuccess) return e;
   Args a{};
   a.plan = plan;
@@ -1213,7 +1394,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.bt = xt;
   a.ht = ht;
   a.aoff = 0;
-  if (max_heavy > 0) wide_gemm_kernel<true><<<sms, kWThreads, smem_w, st>>>(a);
+  if (max_heavy > 0) wide_gemm_kernel<true, kGuNA, kGuNB><<<sms, kWThreads, smem_wgu, st>>>(a);
   grouped_gemm_kernel<true><<<sms, kThreads, smem_gu, st>>>(a);
   // down: K = I, M = H; B = H tiles; out = rows
   a.K = I;
@@ -1224,7 +1405,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.y_f32 = y_f32;
   a.y_bf16 = y_bf16;
   a.ys_f32 = ys_f32;
-  if (max_heavy > 0) wide_gemm_kernel<false><<<sms, kWThreads, smem_w, st>>>(a);
+  if (max_heavy > 0) wide_gemm_kernel<false, kDnNA, kDnNB><<<sms, kWThreads, smem_wdn, st>>>(a);
   grouped_gemm_kernel<false><<<sms, kThreads, smem_dn, st>>>(a);
   count_launches(max_heavy > 0 ? 7 : 4);
   return cudaGetLastError();

@@ -55,6 +55,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
   }
 }
 
+// Bounded wait that sleeps ns nanoseconds between tests: for waits whose
+// wake-up latency the pipeline hides, so that the waiting warp neither
+// takes issue slots nor shared-memory bandwidth from the warps doing work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                                uint32_t ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(ns);
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 15) == 0) {
+      if (abort && *abort) return false;
+      if (clock64() - t0 > kWaitCycles) return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- bulk copies
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),

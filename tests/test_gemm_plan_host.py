@@ -3,7 +3,7 @@
 A host program (nvcc, no GPU) includes expert_gemm_sm100.cu and checks what
 the kernels rely on: the dynamic shared memory of both dequantising GEMMs
 (stage ring plus the dequant warps' raw-code staging) and of the wide-tile
-GEMM (three 64 KiB stages) fits the per-CTA limit, the row-tile bound
+GEMMs (stage ring plus the epilogue warps' scratch) fits the per-CTA limit, the row-tile bound
 covers every routing, and the heavy-slot bound covers every routing's groups
 of more than one row tile (up to the slot cap), on seeded random routings
 with a skewed expert popularity.
@@ -30,7 +30,7 @@ int main() {
   const size_t limit = 227 * 1024;
   const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
   const size_t smem_dn = size_t(Cfg<false>::kStages) * Cfg<false>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
-  const size_t smem_w = size_t(kWStages) * kWStageBytes + 1024;
+  const size_t smem_w = wide_smem_bytes<kGuNA, kGuNB>() > wide_smem_bytes<kDnNA, kDnNB>() ? wide_smem_bytes<kGuNA, kGuNB>() : wide_smem_bytes<kDnNA, kDnNB>();
   int bad_tiles = 0, bad_heavy = 0, cases = 0;
   std::mt19937 rng(12345);
   const int Ts[] = {5, 37, 300, 1000, 8192};
