@@ -49,9 +49,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # decode_fused_kernel of one step (dram read + write of one launch)
     "decode1": (34066688, "profiles/decode_fused_decode1.md"),
-    # gather_rows + predequant + grouped_gemm_kernel<gate/up> + <down> of one
-    # moe_expert_ffn call (the launches the prefill roofline times)
-    "prefill8k": (2813476352, "profiles/grouped_gemm_prefill8k.md"),
+    # gather_rows + predequant + the wide-tile and the dequantising GEMMs
+    # (gate/up and down) of one moe_expert_ffn call (the launches the prefill
+    # roofline times)
+    "prefill8k": (2768424448, "profiles/grouped_gemm_prefill8k.md"),
 }
 
 

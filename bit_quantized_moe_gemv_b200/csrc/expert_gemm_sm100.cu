@@ -399,9 +399,11 @@ __host__ __device__ inline size_t heavy_slot_bytes(int H, int I) { return size_t
 
 // One CTA of 256 threads per group of kPD tiles; thread (row, half) takes 32
 // K of one row of each tile. All kPD loads of a thread are issued before any
-// dequantisation, so they are in flight together.
-constexpr int kPD = 4;
-__global__ void __launch_bounds__(256) predequant_kernel(const moe_expert* __restrict__ experts,
+// dequantisation, so they are in flight together; four CTAs per SM (at most
+// 64 registers per thread) keep more of them in flight than two CTAs with
+// twice the tiles each.
+constexpr int kPD = 2;
+__global__ void __launch_bounds__(256, 4) predequant_kernel(const moe_expert* __restrict__ experts,
                                                          const moe_expert* __restrict__ shared, int E, int H, int I,
                                                          Plan plan, uint8_t* __restrict__ img, WsHeader* hdr) {
   const int nslots = plan.count[1];
