@@ -67,6 +67,9 @@ constexpr int kDqWarps = 8;
 // kMaxHeavy groups (the first ones in group order) take this path.
 constexpr int kHeavyRows = BN + 1;
 constexpr int kMaxHeavy = 64;
+// Int4 groups of at most kMmaRows rows run on mma.sync (one pass of two
+// 8-token column blocks per job); larger single-tile groups on tcgen05.
+constexpr int kMmaRows = 16;
 
 // ---------------------------------------------------------------- plan
 // Row tiles: every group (routed expert e < E, or the shared expert = E) is
@@ -74,17 +77,20 @@ constexpr int kMaxHeavy = 64;
 // dispatched row, or a token for the shared group) and row count. Heavy
 // groups get a slot of pre-dequantised weights (hslot[g], -1 for none). The
 // row tiles of a heavy group are paired into wide tiles (rows 2j and 2j + 1
-// of the group; wlist holds the first), which `wide_gemm_kernel` runs; the
-// row tiles of the other groups are listed in llist for
-// `grouped_gemm_kernel`. A row tile is also the unit of the gathered
-// activations and of the gate/up output tiles, whichever kernel made them.
+// of the group; wlist holds the first), which `wide_gemm_kernel` runs. A
+// group of one row tile whose three matrices are int4 is listed in mlist for
+// `light_mma_kernel`; the row tiles of the remaining groups are listed in
+// llist for `grouped_gemm_kernel`. A row tile is also the unit of the
+// gathered activations and of the gate/up output tiles, whichever kernel
+// made them.
 struct Plan {
-  int* count;   // [0] row tiles, [1] heavy slots used, [2] wide tiles, [3] light row tiles
+  int* count;   // [0] row tiles, [1] heavy slots used, [2] wide tiles, [3] llist tiles, [4] mlist tiles
   int* group;   // [max]
   int* row0;    // [max]
   int* nrows;   // [max]
   int* wlist;   // [max] first row tile of each wide tile
-  int* llist;   // [max] row tiles of the groups without a heavy slot
+  int* llist;   // [max] row tiles for the dequantising tcgen05 GEMM
+  int* mlist;   // [max] row tiles for the mma.sync GEMV
   int* hslot;   // [groups] heavy slot or -1
   int* hlist;   // [heavy slots] group of each slot
   int* tscaled; // [max] nonzero when a row of the tile has its x scaled (set by the gather)
@@ -111,8 +117,17 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   return wb + incl - v;
 }
 
+// A group's three matrices are all well-formed int4 (the mma.sync path).
+__device__ __forceinline__ bool all_int4(const moe_expert& ex, int H, int I) {
+  return ex.gate.qtype == MOE_Q_INT4_SYM_G32 && ex.up.qtype == MOE_Q_INT4_SYM_G32 &&
+         ex.down.qtype == MOE_Q_INT4_SYM_G32 && qmatrix_ok(ex.gate, I, H) && qmatrix_ok(ex.up, I, H) &&
+         qmatrix_ok(ex.down, H, I);
+}
+
 __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ counts, const int* __restrict__ offsets,
-                                                    int E, int shared_rows, int max_tiles, int max_heavy, Plan plan,
+                                                    const moe_expert* __restrict__ experts,
+                                                    const moe_expert* __restrict__ shared, int H, int I, int E,
+                                                    int shared_rows, int max_tiles, int max_heavy, Plan plan,
                                                     WsHeader* hdr) {
   __shared__ int wsum[32];
   const int ngroups = E + (shared_rows > 0 ? 1 : 0);
@@ -123,15 +138,18 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     const int n = g < E ? counts[g] : shared_rows;
     nt = (n + BN - 1) / BN;
   }
-  int total, htotal, wtotal, ltotal;
+  int total, htotal, wtotal, ltotal, mtotal;
   const int excl = block_excl_scan(nt, wsum, &total);
   // heavy groups: slots in group order
   const int hv = (g < ngroups && nt >= 2) ? 1 : 0;  // n >= kHeavyRows
   const int hslot = block_excl_scan(hv, wsum, &htotal);
   const bool heavy = hv && hslot < max_heavy;
-  const int nw = heavy ? (nt + 1) / 2 : 0, nl = heavy ? 0 : nt;
+  const bool mma = !heavy && nt == 1 && (g < E ? counts[g] : shared_rows) <= kMmaRows &&
+                   all_int4(g < E ? experts[g] : *shared, H, I);
+  const int nw = heavy ? (nt + 1) / 2 : 0, nl = (heavy || mma) ? 0 : nt, nm = mma ? 1 : 0;
   const int wexcl = block_excl_scan(nw, wsum, &wtotal);
   const int lexcl = block_excl_scan(nl, wsum, &ltotal);
+  const int mexcl = block_excl_scan(nm, wsum, &mtotal);
   const bool fits = total <= max_tiles;  // the host's bound covers every routing
   if (g < ngroups) {
     plan.hslot[g] = heavy ? hslot : -1;
@@ -142,6 +160,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     plan.count[1] = min(htotal, max_heavy);
     plan.count[2] = fits ? wtotal : 0;
     plan.count[3] = fits ? ltotal : 0;
+    plan.count[4] = fits ? mtotal : 0;
     if (!fits) flag_error(hdr, MOE_ERR_DEVICE_FAULT, 7000002);
   }
   if (g < ngroups && fits) {
@@ -154,6 +173,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
     }
     for (int j = 0; j < nw; ++j) plan.wlist[wexcl + j] = excl + 2 * j;
     for (int t = 0; t < nl; ++t) plan.llist[lexcl + t] = excl + t;
+    if (nm) plan.mlist[mexcl] = excl;
   }
 }
 
@@ -1293,6 +1313,176 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
   }
 }
 
+
+// ---------------------------------------------------------------- int4 groups of one row tile
+// A group with at most 128 rows (one row tile) streams its weights once for
+// few tokens (median 9 at 8K prefill): a GEMV more than a GEMM. Its row tile
+// runs as warp jobs on mma.sync m16n8k16 (fp16 operands, fp32 accumulation)
+// with the A fragments dequantised in registers straight from the codes, the
+// way the decode kernel streams its experts: no shared-memory round trip of
+// the weights. A job is 16 weight rows (of gate and up, or of down) against
+// the row tile's tokens, 8 per MMA column block.
+//
+// Each lane takes one 16-byte code column (32 int4 codes along K, one group
+// scale) of rows g and g + 8 (g = lane / 4) per iteration; the four lanes of
+// a group take four consecutive columns. One 32-bit code word gives the
+// fp16 pairs (n0, n4), (n1, n5), (n2, n6), (n3, n7) of its eight codes; the
+// gathered activation tiles store each 8 K values in the order
+// (0,4,1,5,2,6,3,7), so the 16-byte chunk of a token's row that holds the
+// same 8 K values gives the matching B pairs in the same registers. The MMA
+// sums over a permutation of K, which leaves the dot products unchanged.
+constexpr int kLmWarps = 8;
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// int4 word (codes n0..n7 of K 8i..8i+7) -> fp16 pairs (n_j, n_{j+4}) * s, j = 0..3
+__device__ __forceinline__ void deq4_pairs(uint32_t w, uint32_t s2, uint32_t (&p)[4]) {
+  const uint32_t w8 = w >> 8;
+  p[0] = h2_mul(h2_sub(lop_or(w, 0x000F000Fu, 0x64006400u), 0x64086408u), s2);
+  p[1] = h2_mul(h2_sub(lop_or(w, 0x00F000F0u, 0x54005400u), 0x54805480u), s2);
+  p[2] = h2_mul(h2_sub(lop_or(w8, 0x000F000Fu, 0x64006400u), 0x64086408u), s2);
+  p[3] = h2_mul(h2_sub(lop_or(w8, 0x00F000F0u, 0x54005400u), 0x54805480u), s2);
+}
+
+struct LmRows {  // one matrix: this lane's rows g and g + 8 (codes, scales)
+  const uint8_t* lo;
+  const uint8_t* hi;
+  const uint16_t* slo;
+  const uint16_t* shi;
+};
+struct LmLd {  // one column of both rows
+  uint4 a, b;
+  uint32_t sa, sb;
+};
+__device__ __forceinline__ void lm_load(const LmRows& R, int c, LmLd& L) {
+  L.a = __ldg(reinterpret_cast<const uint4*>(R.lo) + c);
+  L.b = __ldg(reinterpret_cast<const uint4*>(R.hi) + c);
+  L.sa = __ldg(R.slo + c);
+  L.sb = __ldg(R.shi + c);
+}
+__device__ __forceinline__ uint32_t u4_word(const uint4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// One matrix's share of a job: rows g, g + 8 of R against tokens
+// n0 .. n0 + 8 NBP - 1 of the activation tile btile (K / 64 k-blocks), the
+// loads of two iterations in flight.
+template <int NBP>
+__device__ __forceinline__ void lm_kloop(const LmRows& R, const uint8_t* btile, int nit, int n0,
+                                         float (&acc)[NBP][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int b = 0; b < NBP; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
+  LmLd L[2];
+  lm_load(R, tig, L[0]);
+  if (nit > 1) lm_load(R, 4 + tig, L[1]);
+#pragma unroll 1
+  for (int it0 = 0; it0 < nit; it0 += 2) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int it = it0 + s;
+      if (it < nit) {
+        const int c = 4 * it + tig;  // this lane's code column: K [32 c, 32 c + 32)
+        const uint8_t* bk = btile + size_t(c >> 1) * kTileBytes;
+        const uint32_t sa = h2_splat(uint16_t(L[s].sa)), sb = h2_splat(uint16_t(L[s].sb));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pa[4], pb[4];
+          deq4_pairs(u4_word(L[s].a, j), sa, pa);
+          deq4_pairs(u4_word(L[s].b, j), sb, pb);
+          const int ch = ((c & 1) << 2) + j;  // 16-byte chunk of K [32 c + 8 j, +8) in the k-block
+#pragma unroll
+          for (int b = 0; b < NBP; ++b) {
+            const int r = n0 + 8 * b + g;  // token row of the tile (< 128; rows past n are unused columns)
+            const uint4 bq = *reinterpret_cast<const uint4*>(bk + r * 128 + ((ch ^ (r & 7)) << 4));
+            mma16816(acc[b], pa[0], pb[0], pa[1], pb[1], bq.x, bq.y);
+            mma16816(acc[b], pa[2], pb[2], pa[3], pb[3], bq.z, bq.w);
+          }
+        }
+        if (it + 2 < nit) lm_load(R, 4 * (it + 2) + tig, L[s]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ LmRows lm_rows(const moe_qmatrix& W, int m_lo, int K) {
+  LmRows R;
+  R.lo = W.codes + size_t(m_lo) * (K / 2);
+  R.hi = W.codes + size_t(m_lo + 8) * (K / 2);
+  R.slo = W.scales + size_t(m_lo) * (K / 32);
+  R.shi = W.scales + size_t(m_lo + 8) * (K / 32);
+  return R;
+}
+
+// One job: rows [16 rb, 16 rb + 16) of the weight matrices against the n
+// tokens of row tile rt, NBP blocks of 8 tokens per pass over K (gate, then
+// up, for gate/up).
+template <bool kGateUp, int NBP>
+__device__ void lm_job(const Args& a, int rt, int rb, int n) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+  const int K = a.K, KB = K / BK, nit = K / 128;
+  const int grp = a.plan.group[rt];
+  const moe_expert& ex = grp < a.E ? a.experts[grp] : *a.shared;
+  const int m_lo = rb * 16 + g;
+  const uint8_t* btile = a.bt + size_t(rt) * KB * kTileBytes;
+  const bool tile_scaled = a.plan.tscaled[rt] != 0;
+  for (int n0 = 0; n0 < n; n0 += 8 * NBP) {
+    float acc[NBP][4], acu[NBP][4];
+    lm_kloop<NBP>(lm_rows(kGateUp ? ex.gate : ex.down, m_lo, K), btile, nit, n0, acc);
+    if (kGateUp) lm_kloop<NBP>(lm_rows(ex.up, m_lo, K), btile, nit, n0, acu);
+    // D: (row m_lo, tokens 2 tig, 2 tig + 1), (row m_lo + 8, the same tokens)
+#pragma unroll
+    for (int b = 0; b < NBP; ++b)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int r = n0 + 8 * b + 2 * tig + (v & 1);
+        if (r >= n) continue;
+        const int m = m_lo + (v >> 1) * 8;
+        const int e = tile_scaled ? a.xexp[size_t(rt) * BN + r] : 0;
+        if (kGateUp) {
+          // the row's x was scaled by 2^-e: g = g_s 2^e, u = u_s 2^e, and
+          // h 2^-(kHShift + 2e) = silu(g) 2^-e u_s 2^-kHShift
+          float gv = acc[b][v], uv = acu[b][v] * (1.0f / (1 << kHShift));
+          if (e) {
+            gv *= pow2f(e);
+            uv *= pow2f(-e);
+          }
+          const int kc = (m & 63) >> 3, e8 = m & 7;
+          uint8_t* dst = a.ht + (size_t(rt) * (a.I / BK) + (m >> 6)) * kTileBytes + size_t(r) * 128 +
+                         ((kc ^ (r & 7)) << 4) + (e8 < 4 ? 4 * e8 : 4 * (e8 - 4) + 2);
+          *reinterpret_cast<__half*>(dst) = __float2half_rn(sat_f16(__fdividef(gv, 1.0f + __expf(-gv)) * uv));
+        } else {
+          // undo the scaling of h: y = y_s 2^(kHShift + 2e)
+          const float y = acc[b][v] * pow2f(kHShift + e) * pow2f(e);
+          const size_t at = size_t(a.plan.row0[rt] + r) * a.H + m;
+          if (grp < a.E && a.y_f32 == nullptr) a.y_bf16[at] = f32_to_bf16_rn(y);
+          else (grp < a.E ? a.y_f32 : a.ys_f32)[at] = y;
+        }
+      }
+  }
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kLmWarps * 32, 2) light_mma_kernel(Args a) {
+  const int nm = a.plan.count[4];
+  const int nrb = a.M / 16;  // 16-row weight blocks per matrix
+  const long long njobs = (long long)nm * nrb;
+  const long long nwarps = (long long)gridDim.x * kLmWarps;
+  for (long long j = (long long)blockIdx.x * kLmWarps + (threadIdx.x >> 5); j < njobs; j += nwarps) {
+    const int mi = int(j / nrb), rb = int(j - (long long)mi * nrb);
+    const int rt = a.plan.mlist[mi];
+    const int n = a.plan.nrows[rt];
+    if (n <= 8) lm_job<kGateUp, 1>(a, rt, rb, n);
+    else lm_job<kGateUp, 2>(a, rt, rb, n);  // n <= kMmaRows: one pass
+  }
+}
 }  // namespace gemm
 }  // namespace moe
 
@@ -1321,7 +1511,7 @@ int grouped_heavy_slots(long long T, int k, bool with_shared, int H, int I) {
 
 size_t grouped_ws_bytes(long long T, int H, int I, int k, int E, bool with_shared) {
   const long long mt = grouped_max_tiles(T, k, E, with_shared);
-  return align256(20 * size_t(mt) + 16) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
+  return align256(24 * size_t(mt) + 32) + align256(4 * size_t(E + 1) + 4 * size_t(gemm::kMaxHeavy)) +
          align256(4 * size_t(mt)) + align256(4 * size_t(mt) * gemm::BN) + align256(size_t(mt) * (H / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(mt) * (I / gemm::BK) * gemm::kTileBytes) +
          align256(size_t(grouped_heavy_slots(T, k, with_shared, H, I)) * gemm::heavy_slot_bytes(H, I));
@@ -1338,12 +1528,13 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   uint8_t* p = static_cast<uint8_t*>(scratch);
   Plan plan;
   plan.count = reinterpret_cast<int*>(p);
-  plan.group = plan.count + 4;
+  plan.group = plan.count + 8;
   plan.row0 = plan.group + mt;
   plan.nrows = plan.row0 + mt;
   plan.wlist = plan.nrows + mt;
   plan.llist = plan.wlist + mt;
-  p += align256(20 * size_t(mt) + 16);
+  plan.mlist = plan.llist + mt;
+  p += align256(24 * size_t(mt) + 32);
   plan.hslot = reinterpret_cast<int*>(p);
   plan.hlist = plan.hslot + (E + 1);
   p += align256(4 * size_t(E + 1) + 4 * size_t(kMaxHeavy));
@@ -1362,7 +1553,8 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
-  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, E, with_shared ? T : 0, int(mt), max_heavy, plan, hdr);
+  plan_kernel<<<1, 1024, 0, st>>>(counts, offsets, experts, shared, H, I, E, with_shared ? T : 0, int(mt), max_heavy,
+                                  plan, hdr);
   gather_rows_kernel<<<sms * 4, 256, 0, st>>>(x, H, k, perm_src, E, plan, xt, xexp);
   if (max_heavy > 0) predequant_kernel<<<sms * 4, 256, 0, st>>>(experts, shared, E, H, I, plan, aimg, hdr);
   const size_t smem_gu = size_t(Cfg<true>::kStages) * Cfg<true>::kStageBytes + size_t(kRawDepth) * kRawSlotBytes + 1024;
@@ -1398,6 +1590,7 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.aoff = 0;
   if (max_heavy > 0) wide_gemm_kernel<true, kGuNA, kGuNB><<<sms, kWThreads, smem_wgu, st>>>(a);
   grouped_gemm_kernel<true><<<sms, kThreads, smem_gu, st>>>(a);
+  light_mma_kernel<true><<<sms * 2, kLmWarps * 32, 0, st>>>(a);
   // down: K = I, M = H; B = H tiles; out = rows
   a.K = I;
   a.M = H;
@@ -1409,7 +1602,8 @@ cudaError_t launch_grouped_ffn(const uint16_t* x, int T, int H, int I, int k, in
   a.ys_f32 = ys_f32;
   if (max_heavy > 0) wide_gemm_kernel<false, kDnNA, kDnNB><<<sms, kWThreads, smem_wdn, st>>>(a);
   grouped_gemm_kernel<false><<<sms, kThreads, smem_dn, st>>>(a);
-  count_launches(max_heavy > 0 ? 7 : 4);
+  light_mma_kernel<false><<<sms * 2, kLmWarps * 32, 0, st>>>(a);
+  count_launches(max_heavy > 0 ? 9 : 6);
   return cudaGetLastError();
 }
 
