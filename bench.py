@@ -49,10 +49,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # decode_fused_kernel of one step (dram read + write of one launch)
     "decode1": (34066688, "profiles/decode_fused_decode1.md"),
-    # gather_rows + predequant + the wide-tile and the dequantising GEMMs
-    # (gate/up and down) of one moe_expert_ffn call (the launches the prefill
-    # roofline times)
-    "prefill8k": (2768424448, "profiles/grouped_gemm_prefill8k.md"),
+    # gather_rows + predequant + the wide-tile, the dequantising and the
+    # mma.sync GEMMs (gate/up and down) of one moe_expert_ffn call (the
+    # launches the prefill roofline times)
+    "prefill8k": (2759788032, "profiles/grouped_gemm_prefill8k.md"),
 }
 
 
@@ -758,7 +758,8 @@ def run_prefill(args, rank, world, peaks, peak_kind):
         "vs_baseline": None, "dtype": "f16",
         "data": "synthetic (seeded; random weights of the stated architecture)",
         "config": dict(workload_config(wl, world), l2="inputs larger than L2 (1.36 GB of expert weights)"),
-        "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (gather + tcgen05 gate/up + down)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "moe_expert_ffn (gather, pre-dequantisation, tcgen05 and mma.sync gate/up and down)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} bf16_tflops", "flops_per_launch": flops, "ms_per_launch": ffn_ms,
                      "traffic": ncu_traffic(args.workload)[0], "traffic_source": ncu_traffic(args.workload)[1]},
