@@ -61,6 +61,14 @@ SMALL = {
     # GEMM's last 256-row weight block holds one 128-row tile
     "tc_wide_odd_h": wlm.Workload("tc_wide_odd_h", T=600, H=384, I=256, E=10, k=2, zipf_s=0.8, seed=20,
                                   routed_qtypes=((0, 7, wlm.Q_INT4_SYM_G32), (7, None, wlm.Q_INT2_ASYM_G16))),
+    # a handful of tokens on the tcgen05 path: every expert (and the shared
+    # one) on the mma.sync GEMV path; then a mix where the int2/int8 experts
+    # and the int8 shared expert take the dequantising GEMM beside it
+    "tc_few_tokens": wlm.Workload("tc_few_tokens", T=12, H=256, I=256, E=16, k=4, zipf_s=0.5, seed=21),
+    "tc_few_tokens_mixed": wlm.Workload("tc_few_tokens_mixed", T=9, H=384, I=128, E=12, k=3, zipf_s=0.3, seed=22,
+                                        routed_qtypes=((0, 5, wlm.Q_INT4_SYM_G32), (5, 9, wlm.Q_INT2_ASYM_G16),
+                                                       (9, None, wlm.Q_INT8_PER_CHANNEL)),
+                                        shared_qtype=wlm.Q_INT8_PER_CHANNEL),
     "k1_ragged": wlm.Workload("k1_ragged", T=37, H=192, I=128, E=40, k=1, zipf_s=0.3, seed=6,
                               shared_qtype=wlm.Q_INT2_ASYM_G16),
     # 256 routed experts (the pages' Coder variant keeps half of the 512) on
