@@ -117,6 +117,19 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   return wb + incl - v;
 }
 
+// The GEMM that takes a group of n rows: its numbers of wide tiles (pairs of
+// row tiles, when it has a heavy slot), of row tiles for the dequantising
+// GEMM and of row tiles for the mma.sync GEMV (one tile of at most kMmaRows
+// rows whose matrices are all int4). Every row tile lands in exactly one list.
+struct GroupLists {
+  int nw, nl, nm;
+};
+__host__ __device__ inline GroupLists group_lists(int n, bool heavy_slot, bool all_int4) {
+  const int nt = (n + BN - 1) / BN;
+  const bool mma = !heavy_slot && nt == 1 && n <= kMmaRows && all_int4;
+  return GroupLists{heavy_slot ? (nt + 1) / 2 : 0, (heavy_slot || mma) ? 0 : nt, mma ? 1 : 0};
+}
+
 // A group's three matrices are all well-formed int4 (the mma.sync path).
 __device__ __forceinline__ bool all_int4(const moe_expert& ex, int H, int I) {
   return ex.gate.qtype == MOE_Q_INT4_SYM_G32 && ex.up.qtype == MOE_Q_INT4_SYM_G32 &&
@@ -144,9 +157,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ coun
   const int hv = (g < ngroups && nt >= 2) ? 1 : 0;  // n >= kHeavyRows
   const int hslot = block_excl_scan(hv, wsum, &htotal);
   const bool heavy = hv && hslot < max_heavy;
-  const bool mma = !heavy && nt == 1 && (g < E ? counts[g] : shared_rows) <= kMmaRows &&
-                   all_int4(g < E ? experts[g] : *shared, H, I);
-  const int nw = heavy ? (nt + 1) / 2 : 0, nl = (heavy || mma) ? 0 : nt, nm = mma ? 1 : 0;
+  const int n_g = g < ngroups ? (g < E ? counts[g] : shared_rows) : 0;
+  // descriptors are read only for the groups that could take the mma.sync path
+  const bool int4 = !heavy && nt == 1 && n_g <= kMmaRows && all_int4(g < E ? experts[g] : *shared, H, I);
+  const GroupLists gl = group_lists(n_g, heavy, int4);
+  const int nw = gl.nw, nl = gl.nl, nm = gl.nm;
   const int wexcl = block_excl_scan(nw, wsum, &wtotal);
   const int lexcl = block_excl_scan(nl, wsum, &ltotal);
   const int mexcl = block_excl_scan(nm, wsum, &mtotal);
