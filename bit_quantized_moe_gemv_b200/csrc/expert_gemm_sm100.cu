@@ -1329,10 +1329,11 @@ __global__ void __launch_bounds__(kWThreads, 1) wide_gemm_kernel(Args a) {
 }
 
 
-// ---------------------------------------------------------------- int4 groups of one row tile
-// A group with at most 128 rows (one row tile) streams its weights once for
-// few tokens (median 9 at 8K prefill): a GEMV more than a GEMM. Its row tile
-// runs as warp jobs on mma.sync m16n8k16 (fp16 operands, fp32 accumulation)
+// ---------------------------------------------------------------- int4 groups of a few rows
+// An int4 group of at most kMmaRows rows streams its weights once for a
+// handful of tokens (at 8K prefill 138 of the 185 single-tile groups): a
+// GEMV more than a GEMM. Its row tile runs as warp jobs on mma.sync
+// m16n8k16 (fp16 operands, fp32 accumulation)
 // with the A fragments dequantised in registers straight from the codes, the
 // way the decode kernel streams its experts: no shared-memory round trip of
 // the weights. A job is 16 weight rows (of gate and up, or of down) against
