@@ -51,6 +51,18 @@ def test_peaks_and_traffic_sources():
         assert traffic is None or traffic > 0
 
 
+def test_traffic_figures_match_their_profile_summaries():
+    # the DRAM traffic the bench reports is the figure its ncu summary states
+    # (read + write per launch or call, written with thousands separators)
+    import re
+    for wl, (traffic, src) in bench.NCU_TRAFFIC.items():
+        if traffic is None:
+            continue
+        text = open(os.path.join(ROOT, src)).read()
+        stated = {int(m.replace(",", "")) for m in re.findall(r"(\d{1,3}(?:,\d{3}){2,}) B\b", text)}
+        assert traffic in stated, (wl, traffic, sorted(stated))
+
+
 def test_clock_sampler_parses_nvidia_smi_rows(tmp_path, monkeypatch):
     # a stand-in nvidia-smi printing two samples in the queried column order
     fake = tmp_path / "nvidia-smi"
